@@ -1,0 +1,324 @@
+"""Plain CPU oracle of the score-then-select decode step.
+
+TEST INFRASTRUCTURE: only tests, the smoke check and the bench's CPU-baseline leg may
+import this. It shares no code with the CUDA path and never calls it.
+
+Everything is float64 except where the method fixes a rounding decision (the proxy
+cache's stored precision, the NVFP4 codes), which is taken in float32 exactly as the
+method states it, so that integer-valued results (codes, selected indices) can be
+compared bit for bit.
+
+Sources (page title, then the part of the page):
+  [JSSA]  "Joint Subspace Sparse Attention for Efficient Long-Context Decoding"
+          - Figure 1: for one KV head, the mean of its query heads scores a projected-key
+            cache in a shared low-dimensional subspace; the top-B positions are selected;
+            all query heads of the group share that index set; attention then reads the
+            original full-dimensional keys and values at those positions.
+          - Abstract: distinct per-KV-head selections under the standard GQA layout.
+          - Table 15: per-KV-head selection (the variant built here).
+          - Figure 10: the projected scoring cache may be stored at reduced precision
+            while the full KV cache and the final attention stay BF16.
+  [JQS]   "Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse Attention"
+          - Full text: NVFP4 cache; a dense FP4 scan scores the whole key history; 128-token
+            blocks are selected; FP16 value aggregation with FP32 accumulation; calibrated
+            key centring; at most two BF16 pages kept; cache packed from BF16 activations.
+
+Readings where the pages are silent (each listed in the design notes):
+  * block score = max over the block's valid tokens (and, on the NVFP4 path, over the
+    group's query heads); the proxy scores are unscaled (scaling does not change order);
+  * forced blocks (sink, last, kept) count against the budget; ties go to the lower index;
+  * attention is exact softmax over the selected tokens only.
+
+Parity pins live in tests/test_oracle_*.py. The aggregation of per-head NVFP4 scores into
+one score per block (max over heads) is a reading the pages do not fix: its *definition*
+is parity unpinned; its implementation is checked by brute force on tiny inputs.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import formats as F
+
+# ============================================================================================
+# Writer: projected-key cache  [JSSA, Figure 1; Figure 10]
+# ============================================================================================
+
+
+def proxy_keys_f32(k_bits: np.ndarray, P: np.ndarray) -> np.ndarray:
+    """Projected keys k~ = k . P, evaluated in float32.
+
+    k_bits: stored BF16 keys [n][d]; P: float32 [d][r].
+    Fixed evaluation: for each output j, acc = 0; for i = 0..d-1 in order,
+    acc = fp32(acc + fp32(k_i * P_ij)) (two roundings per term, no fused multiply-add).
+    """
+    k32 = F.bf16_to_f64(k_bits).astype(np.float32)
+    P32 = np.asarray(P, dtype=np.float32)
+    acc = np.zeros((k32.shape[0], P32.shape[1]), dtype=np.float32)
+    for i in range(k32.shape[1]):
+        prod = k32[:, i:i + 1] * P32[i:i + 1, :]       # float32 x float32 -> rounded float32
+        acc = acc + prod                                # rounded float32
+    return acc
+
+
+def proxy_store(k_bits: np.ndarray, P: np.ndarray, dtype: str):
+    """Stored proxy cache entries: float32 values ('f32') or BF16 bit patterns ('bf16')."""
+    acc = proxy_keys_f32(k_bits, P)
+    if dtype == "f32":
+        return acc
+    if dtype == "bf16":
+        return F.f32_to_bf16_rne(acc)
+    raise ValueError(dtype)
+
+
+def proxy_decode(stored, dtype: str) -> np.ndarray:
+    if dtype == "f32":
+        return np.asarray(stored, dtype=np.float32).astype(np.float64)
+    return F.bf16_to_f64(stored)
+
+
+# ============================================================================================
+# Score: group-mean projected query against the projected keys  [JSSA, Figure 1]
+# ============================================================================================
+
+
+def proxy_query(q_bits: np.ndarray, P: np.ndarray) -> np.ndarray:
+    """q~ = (mean of the group's query heads) . P, float64. q_bits: BF16 [G][d]."""
+    qbar = F.bf16_to_f64(q_bits).mean(axis=0)
+    return qbar @ np.asarray(P, dtype=np.float64)
+
+
+def token_scores(proxy: np.ndarray, qt: np.ndarray) -> np.ndarray:
+    """s_t = q~ . k~_t for every token (float64). proxy: decoded [L][r]."""
+    return proxy @ qt
+
+
+def block_max(s: np.ndarray, S: int) -> np.ndarray:
+    """beta_j = max of s over the valid tokens of block j (tokens j*S .. j*S+S-1, < L)."""
+    L = s.shape[-1]
+    nb = (L + S - 1) // S
+    pad = nb * S - L
+    if pad:
+        s = np.concatenate([s, np.full(s.shape[:-1] + (pad,), -np.inf)], axis=-1)
+    return s.reshape(s.shape[:-1] + (nb, S)).max(axis=-1)
+
+
+# ============================================================================================
+# Select: forced blocks, then the best-scoring rest  [JSSA, Figure 1; JQS, Full text]
+# ============================================================================================
+
+
+def forced_blocks(nb: int, force_sink: bool, force_last: bool, keep=()) -> np.ndarray:
+    f = set()
+    if force_sink:
+        f.add(0)
+    if force_last:
+        f.add(nb - 1)
+    for j in keep:
+        if 0 <= j < nb:
+            f.add(int(j))
+    return np.array(sorted(f), dtype=np.int64)
+
+
+def select_blocks(beta: np.ndarray, budget: int, forced: np.ndarray) -> np.ndarray:
+    """Indices of the selected blocks, ascending.
+
+    If the budget covers every block, every block is selected. Otherwise the forced blocks
+    are taken first and the remaining budget - |forced| slots go to the other blocks in
+    order of decreasing score, ties to the lower index.
+    """
+    nb = beta.shape[0]
+    if nb <= budget:
+        return np.arange(nb, dtype=np.int64)
+    forced = np.asarray(forced, dtype=np.int64)
+    is_forced = np.zeros(nb, dtype=bool)
+    is_forced[forced] = True
+    rest = np.nonzero(~is_forced)[0]
+    order = np.lexsort((rest, -beta[rest]))             # primary: -beta, secondary: index
+    take = rest[order[: budget - len(forced)]]
+    return np.sort(np.concatenate([forced, take]))
+
+
+def kth_threshold(beta: np.ndarray, budget: int, forced: np.ndarray):
+    """(s*, tau): the last score taken from the non-forced blocks, and its tie tolerance.
+
+    tau = 1e-4 * max(|s*|, 1e-30): the relative near-tie band within which two selections
+    are both valid top-k sets.
+    """
+    nb = beta.shape[0]
+    is_forced = np.zeros(nb, dtype=bool)
+    is_forced[np.asarray(forced, dtype=np.int64)] = True
+    rest = beta[~is_forced]
+    need = budget - int(is_forced.sum())
+    if nb <= budget or need <= 0 or rest.size == 0:
+        return None, None
+    s_star = np.sort(rest)[::-1][need - 1]
+    return s_star, 1e-4 * max(abs(s_star), 1e-30)
+
+
+def selection_valid(beta: np.ndarray, budget: int, forced: np.ndarray, got: np.ndarray,
+                    rel_tol: float = 1e-4) -> tuple[bool, str]:
+    """Is ``got`` a valid selection, up to near-ties at the k-th score?
+
+    Valid iff: it has the right size; it holds every forced block; every chosen non-forced
+    block scores at least s* - tau; every unchosen block scores at most s* + tau; and it
+    is strictly ascending.
+    """
+    nb = beta.shape[0]
+    got = np.asarray(got, dtype=np.int64)
+    want = select_blocks(beta, budget, forced)
+    if len(got) != len(want):
+        return False, f"size {len(got)} != {len(want)}"
+    if np.any(np.diff(got) <= 0):
+        return False, "not strictly ascending"
+    if np.any(got < 0) or np.any(got >= nb):
+        return False, "index out of range"
+    if nb <= budget:
+        return bool(np.array_equal(got, want)), "dense"
+    if not set(np.asarray(forced).tolist()) <= set(got.tolist()):
+        return False, "forced block missing"
+    if np.array_equal(got, want):
+        return True, "exact"
+    s_star, _ = kth_threshold(beta, budget, forced)
+    tau = rel_tol * max(abs(s_star), 1e-30)
+    extra = np.setdiff1d(got, want)
+    missing = np.setdiff1d(want, got)
+    if np.all(beta[extra] >= s_star - tau) and np.all(beta[missing] <= s_star + tau):
+        return True, f"near-tie ({len(extra)} swapped)"
+    return False, f"{len(extra)} swapped outside the tie band"
+
+
+def block_tokens(sel: np.ndarray, S: int, L: int) -> np.ndarray:
+    """Token positions covered by the selected blocks (valid tokens only), ascending."""
+    if len(sel) == 0:
+        return np.zeros(0, dtype=np.int64)
+    t = (np.asarray(sel, dtype=np.int64)[:, None] * S + np.arange(S)[None, :]).reshape(-1)
+    return t[t < L]
+
+
+# ============================================================================================
+# Sparse attention and the log-sum-exp combine  [JSSA, Figure 1; JQS, Full text]
+# ============================================================================================
+
+
+def sparse_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, tokens: np.ndarray,
+                     scale: float) -> np.ndarray:
+    """o_h = sum_t softmax_t(scale * q_h . k_t) v_t over the given tokens only (float64).
+
+    q: [G][d], K/V: [L][d] (decoded), tokens: positions. Softmax is normalised over the
+    selected tokens only.
+    """
+    Kt = K[tokens]
+    Vt = V[tokens]
+    logits = scale * (q @ Kt.T)                               # [G][T]
+    m = logits.max(axis=1, keepdims=True)
+    p = np.exp(logits - m)
+    return (p @ Vt) / p.sum(axis=1, keepdims=True)
+
+
+def attention_partial(q: np.ndarray, K: np.ndarray, V: np.ndarray, tokens: np.ndarray,
+                      scale: float):
+    """One split's partial state (m, l, o) with o unnormalised: o = sum_t e^(x_t - m) v_t."""
+    if len(tokens) == 0:
+        G, d = q.shape[0], V.shape[1]
+        return np.full(G, -np.inf), np.zeros(G), np.zeros((G, d))
+    logits = scale * (q @ K[tokens].T)
+    m = logits.max(axis=1)
+    p = np.exp(logits - m[:, None])
+    return m, p.sum(axis=1), p @ V[tokens]
+
+
+def lse_combine(ms, ls, os_) -> np.ndarray:
+    """o = sum_s e^(m_s - M) o_s / sum_s e^(m_s - M) l_s, M = max_s m_s."""
+    ms = np.asarray(ms)
+    M = ms.max(axis=0)
+    w = np.exp(ms - M[None, :])
+    w = np.where(np.isfinite(ms), w, 0.0)
+    num = np.einsum("sg,sgd->gd", w, np.asarray(os_))
+    den = np.einsum("sg,sg->g", w, np.asarray(ls))
+    return num / den[:, None]
+
+
+# ============================================================================================
+# NVFP4 path  [JQS, Full text]
+# ============================================================================================
+
+E2M1_MAX = 6.0
+UE4M3_MAX = 448.0
+
+
+def nvfp4_pack(x32: np.ndarray, g: np.float32):
+    """Pack float32 values [n][d] into NVFP4: E2M1 codes [n][d] and UE4M3 scales [n][d/16].
+
+    Per group of 16 consecutive elements:
+      a = max |x|; sf = fp32(a / fp32(6 g)); sigma = UE4M3(sf) (nearest even, satfinite);
+      if sigma decodes to 0 every code is 0; else e_i = E2M1(fp32(x_i / fp32(sigma g)))
+      (nearest even, satfinite). All divisions and products are rounded float32 ops.
+    """
+    x32 = np.asarray(x32, dtype=np.float32)
+    n, d = x32.shape
+    g = np.float32(g)
+    grp = x32.reshape(n, d // 16, 16)
+    a = np.abs(grp).max(axis=2)                                   # exact
+    den = np.float32(np.float32(E2M1_MAX) * g)
+    sf = (a / den).astype(np.float32)
+    sig = F.ue4m3_encode(sf)
+    sigv = F.ue4m3_value(sig).astype(np.float32)                  # exact in float32
+    den2 = (sigv * g).astype(np.float32)
+    safe = np.where(sigv > 0, den2, np.float32(1.0))
+    t = (grp / safe[:, :, None]).astype(np.float32)
+    codes = F.e2m1_encode(t)
+    codes = np.where((sigv > 0)[:, :, None], codes, 0).astype(np.uint8)
+    return codes.reshape(n, d), sig.astype(np.uint8)
+
+
+def nvfp4_dequant(codes: np.ndarray, scales: np.ndarray, g) -> np.ndarray:
+    """float64 values e * sigma * g for codes [n][d], scales [n][d/16]."""
+    n, d = codes.shape
+    e = F.e2m1_value(codes).reshape(n, d // 16, 16)
+    s = F.ue4m3_value(scales)[:, :, None]
+    return (e * s * np.float64(np.float32(g))).reshape(n, d)
+
+
+def centre(k_bits: np.ndarray, mu: np.ndarray) -> np.ndarray:
+    """x = fp32(k) - mu, a rounded float32 subtraction."""
+    return (F.bf16_to_f64(k_bits).astype(np.float32) - np.asarray(mu, dtype=np.float32)
+            ).astype(np.float32)
+
+
+def query_scale(q_bits_all: np.ndarray) -> np.float32:
+    """Per-step query tensor scale g_q = fp32(max |q| / fp32(6 * 448)) over the whole q."""
+    a = np.float32(np.abs(F.bf16_to_f64(q_bits_all)).max())
+    return np.float32(a / np.float32(E2M1_MAX * UE4M3_MAX))
+
+
+def nvfp4_head_scores(q_codes, q_scales, g_q, k_codes, k_scales, g_k) -> np.ndarray:
+    """s[h, t] = sum over d of dequant(q_h) * dequant(k_t), float64. -> [G][L]."""
+    qd = nvfp4_dequant(q_codes, q_scales, g_q)
+    kd = nvfp4_dequant(k_codes, k_scales, g_k)
+    return qd @ kd.T
+
+
+def nvfp4_block_scores(head_scores: np.ndarray, S: int) -> np.ndarray:
+    """beta_j = max over the group's heads and the block's valid tokens."""
+    return block_max(head_scores.max(axis=0), S)
+
+
+def block_quant_error(x32: np.ndarray, codes: np.ndarray, scales: np.ndarray, g_k, S: int,
+                      L: int) -> np.ndarray:
+    """Squared NVFP4 error of each complete block: sum over tokens and dims of (x - deq x)^2.
+
+    Only complete blocks ((j + 1) * S <= L) have an error; incomplete ones get -inf.
+    """
+    err_tok = ((x32.astype(np.float64) - nvfp4_dequant(codes, scales, g_k)) ** 2).sum(axis=1)
+    nb = (L + S - 1) // S
+    out = np.full(nb, -np.inf)
+    nfull = L // S
+    out[:nfull] = err_tok[: nfull * S].reshape(nfull, S).sum(axis=1)
+    return out
+
+
+def kept_blocks(err: np.ndarray, n_keep: int) -> np.ndarray:
+    """The n_keep complete blocks with the largest quantisation error (ties: lower index)."""
+    valid = np.nonzero(np.isfinite(err))[0]
+    order = np.lexsort((valid, -err[valid]))
+    return np.sort(valid[order[:n_keep]])

@@ -1,0 +1,91 @@
+"""One decode step of one row (sequence b, KV head g), composed from the oracle's parts.
+
+TEST INFRASTRUCTURE: only tests, the smoke check and the bench's CPU-baseline leg use this.
+
+Order of the step, following "Joint Subspace Sparse Attention for Efficient Long-Context
+Decoding" (Figure 1) and "Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse
+Attention" (Full text):
+  1. the row's scoring cache: projected keys k . P (stored f32 / bf16), or the centred
+     keys packed to NVFP4;
+  2. proxy block scores beta (max over each block's valid tokens);
+  3. forced blocks plus the best-scoring rest, ascending;
+  4. exact softmax attention of every query head of the group over the selected tokens.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import formats as F
+from . import method as M
+
+
+@dataclass
+class RowParams:
+    S: int                     # block size
+    budget: int                # k, blocks
+    scale: float               # softmax scale
+    proxy: str                 # 'f32' | 'bf16' | 'nvfp4'
+    v_dtype: str               # 'bf16' | 'f16'
+    force_sink: bool = False
+    force_last: bool = False
+    n_keep: int = 0            # NVFP4: blocks kept at full precision
+
+
+def decode_v(v_bits: np.ndarray, v_dtype: str) -> np.ndarray:
+    return F.f16_to_f64(v_bits) if v_dtype == "f16" else F.bf16_to_f64(v_bits)
+
+
+def row_scoring_cache(p: RowParams, k_bits, P=None, mu=None, g_k=None):
+    """The row's stored scoring cache: proxy entries, or (codes, scales, x32) for NVFP4."""
+    if p.proxy == "nvfp4":
+        x32 = M.centre(k_bits, mu)
+        codes, scales = M.nvfp4_pack(x32, g_k)
+        return codes, scales, x32
+    return M.proxy_store(k_bits, P, p.proxy)
+
+
+def row_block_scores(p: RowParams, cache, q_bits, L: int, P=None, g_q=None, g_k=None,
+                     q_all_bits=None):
+    """beta [nb] for one row from its scoring cache."""
+    if p.proxy == "nvfp4":
+        codes, scales, _ = cache
+        qx = F.bf16_to_f64(q_bits).astype(np.float32)
+        q_codes, q_scales = M.nvfp4_pack(qx, g_q)
+        hs = M.nvfp4_head_scores(q_codes, q_scales, g_q, codes[:L], scales[:L], g_k)
+        return M.nvfp4_block_scores(hs, p.S)
+    qt = M.proxy_query(q_bits, P)
+    s = M.token_scores(M.proxy_decode(cache, p.proxy)[:L], qt)
+    return M.block_max(s, p.S)
+
+
+def row_forced(p: RowParams, nb: int, cache=None, L: int = 0, g_k=None):
+    keep = ()
+    if p.proxy == "nvfp4" and p.n_keep > 0:
+        codes, scales, x32 = cache
+        err = M.block_quant_error(x32[:L], codes[:L], scales[:L], g_k, p.S, L)
+        keep = M.kept_blocks(err, p.n_keep)
+    return M.forced_blocks(nb, p.force_sink, p.force_last, keep), keep
+
+
+def decode_row(p: RowParams, k_bits, v_bits, q_bits, L: int, P=None, mu=None, g_k=None,
+               g_q=None, sel_override=None):
+    """Full oracle step for one row. Returns a dict of every intermediate.
+
+    ``sel_override``: attend over this selection instead of the oracle's own (used once a
+    GPU selection has been accepted as a valid top-k under the near-tie rule).
+    """
+    cache = row_scoring_cache(p, k_bits[:L], P, mu, g_k)
+    beta = row_block_scores(p, cache, q_bits, L, P=P, g_q=g_q, g_k=g_k)
+    nb = beta.shape[0]
+    forced, keep = row_forced(p, nb, cache, L, g_k)
+    sel = M.select_blocks(beta, p.budget, forced)
+    use = sel if sel_override is None else np.asarray(sel_override, dtype=np.int64)
+    tokens = M.block_tokens(use, p.S, L)
+    q = F.bf16_to_f64(q_bits)
+    K = F.bf16_to_f64(k_bits[:L])
+    V = decode_v(v_bits[:L], p.v_dtype)
+    out = M.sparse_attention(q, K, V, tokens, p.scale)
+    return dict(cache=cache, beta=beta, forced=forced, keep=keep, sel=sel, tokens=tokens,
+                out=out)

@@ -1,0 +1,211 @@
+"""Pins of the oracle's writer, scorer, selector and attention.
+
+Each check is against something other than the oracle's own formula: identities that
+reduce the method to a textbook result, brute-force enumeration, exact arithmetic, or
+error bounds of IEEE float32.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from oracle import formats as F
+from oracle import method as M
+
+
+def _bf16(x):
+    return F.f32_to_bf16_rne(np.asarray(x, dtype=np.float32))
+
+
+# ---------------------------------------------------------------- writer (projected keys)
+
+def test_proxy_identity_projection_is_exact():
+    rng = np.random.default_rng(0)
+    k = _bf16(rng.standard_normal((50, 16)) * 4)
+    P = np.eye(16, dtype=np.float32)
+    out = M.proxy_keys_f32(k, P)
+    assert np.array_equal(out, F.bf16_to_f64(k).astype(np.float32))
+
+
+def test_proxy_single_entry_projection():
+    rng = np.random.default_rng(1)
+    k = _bf16(rng.standard_normal((20, 8)))
+    P = np.zeros((8, 3), dtype=np.float32)
+    P[5, 2] = np.float32(0.3)
+    out = M.proxy_keys_f32(k, P)
+    assert np.all(out[:, :2] == 0)
+    want = (F.bf16_to_f64(k)[:, 5].astype(np.float32) * np.float32(0.3)).astype(np.float32)
+    assert np.array_equal(out[:, 2], want)
+
+
+def test_proxy_summation_order_is_ascending():
+    # 2^24 + 1 is not a float32: adding in index order loses the 1, reversed order keeps it.
+    k = _bf16(np.array([[2.0 ** 24, 1.0, -(2.0 ** 24)]]))
+    P = np.ones((3, 1), dtype=np.float32)
+    assert M.proxy_keys_f32(k, P)[0, 0] == 0.0
+
+
+def test_proxy_float32_error_bound():
+    rng = np.random.default_rng(2)
+    d, r = 128, 32
+    k = _bf16(rng.standard_normal((300, d)) * 3)
+    P = rng.standard_normal((d, r)).astype(np.float32)
+    kd = F.bf16_to_f64(k)
+    exact = kd @ P.astype(np.float64)
+    got = M.proxy_keys_f32(k, P).astype(np.float64)
+    u = 2.0 ** -24
+    gamma = d * u / (1 - d * u)
+    bound = gamma * (np.abs(kd) @ np.abs(P.astype(np.float64)))
+    assert np.all(np.abs(got - exact) <= bound)
+    # and the bf16 store is the nearest-even rounding of that float32 value
+    st = M.proxy_store(k, P, "bf16")
+    assert np.all(np.abs(F.bf16_to_f64(st) - got) <= np.abs(got) * 2.0 ** -8 + 1e-38)
+
+
+# ---------------------------------------------------------------- scoring
+
+def test_group_mean_linearity():
+    rng = np.random.default_rng(3)
+    q = _bf16(rng.standard_normal((5, 64)))
+    P = rng.standard_normal((64, 16)).astype(np.float32)
+    per_head = F.bf16_to_f64(q) @ P.astype(np.float64)
+    assert np.allclose(M.proxy_query(q, P), per_head.mean(axis=0), rtol=1e-13, atol=1e-13)
+
+
+def test_full_rank_identity_equals_exact_group_mean_score():
+    rng = np.random.default_rng(4)
+    d, L = 32, 100
+    q = _bf16(rng.standard_normal((4, d)))
+    k = _bf16(rng.standard_normal((L, d)))
+    P = np.eye(d, dtype=np.float32)
+    s = M.token_scores(M.proxy_decode(M.proxy_store(k, P, "f32"), "f32"), M.proxy_query(q, P))
+    qd, kd = F.bf16_to_f64(q), F.bf16_to_f64(k)
+    for t in range(L):
+        exact = math.fsum(sum(qd[h, i] for h in range(4)) / 4 * kd[t, i] for i in range(d))
+        assert abs(s[t] - exact) <= 1e-12 * (1 + abs(exact))
+
+
+def test_block_max_loops():
+    rng = np.random.default_rng(5)
+    for L, S in [(37, 8), (64, 16), (5, 1), (130, 64)]:
+        s = rng.standard_normal(L)
+        got = M.block_max(s, S)
+        nb = (L + S - 1) // S
+        assert got.shape == (nb,)
+        for j in range(nb):
+            assert got[j] == max(s[t] for t in range(j * S, min(L, (j + 1) * S)))
+    s = rng.standard_normal(17)
+    assert np.array_equal(M.block_max(s, 1), s)
+
+
+# ---------------------------------------------------------------- selection
+
+def _brute_select(beta, budget, forced):
+    nb = len(beta)
+    if nb <= budget:
+        return list(range(nb))
+    rest = [j for j in range(nb) if j not in set(forced)]
+    need = budget - len(forced)
+
+    def beats(a, b):  # a ranks before b
+        return beta[a] > beta[b] or (beta[a] == beta[b] and a < b)
+
+    winners = []
+    for T in itertools.combinations(rest, need):
+        out = [j for j in rest if j not in T]
+        if all(beats(a, b) for a in T for b in out):
+            winners.append(sorted(list(forced) + list(T)))
+    assert len(winners) == 1
+    return winners[0]
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_select_exhaustive(seed):
+    rng = np.random.default_rng(seed)
+    nb = int(rng.integers(1, 11))
+    budget = int(rng.integers(1, 9))
+    beta = rng.integers(-3, 4, size=nb).astype(np.float64)      # many exact ties
+    fs, fl = bool(rng.integers(0, 2)), bool(rng.integers(0, 2))
+    forced = M.forced_blocks(nb, fs, fl)
+    if nb > budget and len(forced) > budget:
+        return
+    got = M.select_blocks(beta, budget, forced)
+    assert got.tolist() == _brute_select(beta, budget, forced.tolist())
+
+
+def test_select_invariants():
+    rng = np.random.default_rng(7)
+    beta = rng.standard_normal(1000)
+    forced = M.forced_blocks(1000, True, True)
+    sel = M.select_blocks(beta, 64, forced)
+    assert len(sel) == 64 and {0, 999} <= set(sel.tolist())
+    chosen = np.setdiff1d(sel, forced)
+    rest = np.setdiff1d(np.setdiff1d(np.arange(1000), sel), forced)
+    assert beta[chosen].min() >= beta[rest].max()
+    assert np.all(np.diff(sel) > 0)
+    assert M.select_blocks(beta[:50], 64, forced[:1]).tolist() == list(range(50))
+
+
+def test_selection_validity_rule():
+    beta = np.array([5.0, 4.0, 3.0, 3.00001, 1.0, 0.0])
+    forced = np.array([], dtype=np.int64)
+    ok, why = M.selection_valid(beta, 3, forced, np.array([0, 1, 3]))
+    assert ok and why == "exact"
+    ok, why = M.selection_valid(beta, 3, forced, np.array([0, 1, 2]))   # within 1e-4 rel
+    assert ok and why.startswith("near-tie")
+    ok, _ = M.selection_valid(beta, 3, forced, np.array([0, 1, 4]))
+    assert not ok
+    ok, _ = M.selection_valid(beta, 3, forced, np.array([0, 1]))
+    assert not ok
+
+
+# ---------------------------------------------------------------- attention
+
+def _dense_attention_bruteforce(q, K, V, scale):
+    G, d = q.shape
+    out = np.zeros((G, d))
+    for h in range(G):
+        logits = [scale * math.fsum(q[h, i] * K[t, i] for i in range(d)) for t in range(len(K))]
+        m = max(logits)
+        w = [math.exp(x - m) for x in logits]
+        z = math.fsum(w)
+        for i in range(d):
+            out[h, i] = math.fsum(w[t] * V[t, i] for t in range(len(K))) / z
+    return out
+
+
+def test_budget_covering_all_blocks_is_dense_attention():
+    rng = np.random.default_rng(8)
+    G, d, L, S = 3, 16, 45, 8
+    q = rng.standard_normal((G, d))
+    K = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    nb = (L + S - 1) // S
+    sel = M.select_blocks(rng.standard_normal(nb), nb + 2, M.forced_blocks(nb, True, True))
+    toks = M.block_tokens(sel, S, L)
+    assert toks.tolist() == list(range(L))
+    got = M.sparse_attention(q, K, V, toks, 0.25)
+    assert np.allclose(got, _dense_attention_bruteforce(q, K, V, 0.25), rtol=1e-12, atol=1e-12)
+
+
+def test_one_hot_selection_returns_value_row():
+    rng = np.random.default_rng(9)
+    q, K, V = rng.standard_normal((2, 8)), rng.standard_normal((30, 8)), rng.standard_normal((30, 8))
+    got = M.sparse_attention(q, K, V, np.array([17]), 1.0)
+    assert np.array_equal(got, np.broadcast_to(V[17], (2, 8)))
+
+
+@pytest.mark.parametrize("nsplit", [1, 2, 5, 13])
+def test_lse_combine_split_invariance(nsplit):
+    rng = np.random.default_rng(10 + nsplit)
+    G, d, T = 4, 32, 200
+    q = rng.standard_normal((G, d)) * 2
+    K, V = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    toks = np.sort(rng.choice(T, 120, replace=False))
+    cuts = np.sort(rng.choice(np.arange(1, len(toks)), nsplit - 1, replace=False)) if nsplit > 1 else []
+    parts = np.split(toks, cuts)
+    parts.append(np.zeros(0, dtype=np.int64))                 # an empty split is ignored
+    st = [M.attention_partial(q, K, V, p, 0.3) for p in parts]
+    got = M.lse_combine([s[0] for s in st], [s[1] for s in st], [s[2] for s in st])
+    assert np.allclose(got, M.sparse_attention(q, K, V, toks, 0.3), rtol=1e-12, atol=1e-12)

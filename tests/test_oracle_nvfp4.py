@@ -1,0 +1,122 @@
+"""Pins of the oracle's NVFP4 path: packing, block-scaled dot products, block errors."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from oracle import formats as F
+from oracle import method as M
+
+
+def test_exactly_representable_groups_round_trip():
+    rng = np.random.default_rng(0)
+    n, d = 40, 128
+    codes = rng.integers(0, 16, size=(n, d)).astype(np.uint8)
+    codes[:, ::16] = 7                       # a 6 in every group: group scale becomes 1.0
+    x = F.e2m1_value(codes).astype(np.float32)
+    c2, s2 = M.nvfp4_pack(x, np.float32(1.0))
+    assert np.all(s2 == 0x38)
+    # -0 and +0 both decode to 0; compare values, and codes where the value is non-zero
+    assert np.array_equal(F.e2m1_value(c2), F.e2m1_value(codes))
+    nz = F.e2m1_value(codes) != 0
+    assert np.array_equal(c2[nz], codes[nz])
+
+
+def test_zero_group_has_zero_scale_and_codes():
+    x = np.zeros((2, 32), dtype=np.float32)
+    x[1, 16:] = np.linspace(-1, 1, 16)
+    c, s = M.nvfp4_pack(x, np.float32(0.01))
+    assert s[0].tolist() == [0, 0] and s[1, 0] == 0
+    assert np.all(c[0] == 0) and np.all(c[1, :16] == 0)
+
+
+def test_scale_saturates():
+    x = np.full((1, 16), 1e6, dtype=np.float32)
+    c, s = M.nvfp4_pack(x, np.float32(1.0))
+    assert s[0, 0] == 0x7E and np.all(c == 7)
+
+
+def test_per_element_error_bound():
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal((500, 128)) * rng.uniform(0.01, 5, size=(500, 1))).astype(np.float32)
+    g = np.float32(np.abs(x).max() / 2688.0)
+    codes, scales = M.nvfp4_pack(x, g)
+    deq = M.nvfp4_dequant(codes, scales, g)
+    sig = F.ue4m3_value(scales).repeat(16, axis=1) * float(g)
+    # the E2M1 grid's largest half-gap is 1.0 (between 4 and 6) in units of sigma * g
+    assert np.all(np.abs(x - deq) <= sig * 1.0 + 1e-30)
+    rel = np.linalg.norm(x - deq) / np.linalg.norm(x)
+    assert rel < 0.12
+
+
+def test_factored_block_scaled_dot_equals_dequantised_dot():
+    """g_q g_k sum_c sq_c sk_c sum_i eq_i ek_i, evaluated by loops, equals deq(q) . deq(k)."""
+    rng = np.random.default_rng(2)
+    q = (rng.standard_normal((3, 128)) * 2).astype(np.float32)
+    k = rng.standard_normal((7, 128)).astype(np.float32)
+    gq, gk = np.float32(0.0013), np.float32(0.0021)
+    qc, qs = M.nvfp4_pack(q, gq)
+    kc, ks = M.nvfp4_pack(k, gk)
+    got = M.nvfp4_head_scores(qc, qs, gq, kc, ks, gk)
+    for h in range(3):
+        for t in range(7):
+            terms = []
+            for c in range(8):
+                inner = sum(F.E2M1_MAG[qc[h, 16 * c + i] & 7] * (-1 if qc[h, 16 * c + i] & 8 else 1)
+                            * F.E2M1_MAG[kc[t, 16 * c + i] & 7] * (-1 if kc[t, 16 * c + i] & 8 else 1)
+                            for i in range(16))
+                terms.append(float(F.ue4m3_value(qs[h, c])) * float(F.ue4m3_value(ks[t, c])) * inner)
+            want = float(gq) * float(gk) * math.fsum(terms)
+            assert abs(got[h, t] - want) <= 1e-12 * (1 + abs(want))
+
+
+def test_block_scores_max_over_heads_and_tokens_loops():
+    rng = np.random.default_rng(3)
+    hs = rng.standard_normal((5, 300))
+    got = M.nvfp4_block_scores(hs, 128)
+    for j in range(3):
+        want = max(hs[h, t] for h in range(5) for t in range(j * 128, min(300, j * 128 + 128)))
+        assert got[j] == want
+
+
+def test_block_error_exact_and_single_perturbation():
+    S = 16
+    codes = np.full((64, 32), 2, dtype=np.uint8)            # value 1.0
+    codes[:, 0] = 7                                         # a 6 -> group scale 1.0
+    codes[:, 16] = 7
+    x = F.e2m1_value(codes).astype(np.float32)
+    c, s = M.nvfp4_pack(x, np.float32(1.0))
+    err = M.block_quant_error(x, c, s, np.float32(1.0), S, 64)
+    assert np.all(err == 0)
+    x2 = x.copy()
+    x2[37, 5] = np.float32(1.2)                              # rounds to 1.0 -> error 0.04
+    c2, s2 = M.nvfp4_pack(x2, np.float32(1.0))
+    err2 = M.block_quant_error(x2, c2, s2, np.float32(1.0), S, 64)
+    assert err2.tolist()[:2] == [0.0, 0.0] and err2[3] == 0.0
+    assert abs(err2[2] - (float(np.float32(1.2)) - 1.0) ** 2) < 1e-15
+    # the incomplete last block has no error
+    err3 = M.block_quant_error(x2[:60], c2[:60], s2[:60], np.float32(1.0), S, 60)
+    assert err3.shape == (4,) and err3[3] == -np.inf
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_kept_blocks_exhaustive(seed):
+    rng = np.random.default_rng(seed)
+    nb = int(rng.integers(1, 9))
+    err = rng.integers(0, 4, size=nb).astype(np.float64)
+    if rng.integers(0, 2):
+        err[-1] = -np.inf
+    valid = [j for j in range(nb) if np.isfinite(err[j])]
+    n = min(2, len(valid))
+    best = None
+    for T in itertools.combinations(valid, n):
+        key = sorted([(-err[j], j) for j in T])
+        if best is None or key < best[0]:
+            best = (key, sorted(T))
+    assert M.kept_blocks(err, 2).tolist() == best[1]
+
+
+def test_query_scale():
+    q = F.f32_to_bf16_rne(np.array([[0.5, -3.0], [2.0, 1.0]], dtype=np.float32))
+    assert M.query_scale(q) == np.float32(np.float32(3.0) / np.float32(2688.0))
