@@ -1,0 +1,203 @@
+/*
+ * qs.h - C ABI of libqs: score-then-select sparse attention for one decode step (sm_100a).
+ *
+ * The decode step, per row = (sequence b, KV head g):
+ *   1. score  - a cheap proxy score of the current query against the row's whole key
+ *               history, reduced to one score per block of S tokens (max over the block);
+ *   2. select - the top-k blocks per row (forced blocks first), ties to the lower index;
+ *   3. attend - exact softmax attention of each of the group's query heads over the
+ *               selected original keys and values only, FP32 accumulation, split over the
+ *               selection and finished by a log-sum-exp combine.
+ *
+ * Sources:
+ *   "Joint Subspace Sparse Attention for Efficient Long-Context Decoding"
+ *     Figure 1: the mean of a KV head's query heads scores a projected-key cache in a
+ *     shared low-dimensional subspace; the top-B positions are shared by the group's query
+ *     heads; gather-free indexed attention reads the original keys/values at them.
+ *     Abstract: distinct per-KV-head selections under the standard GQA cache layout.
+ *     Figure 9: the step's stages are scoring preparation, candidate scoring, top-B
+ *     selection and sparse attention.
+ *     Figure 10: the projected scoring cache may be kept at reduced precision while the
+ *     full KV cache and the final attention stay BF16.
+ *   "Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse Attention"
+ *     Full text: NVFP4 scoring keys scanned densely on FP4 tensor cores; 128-token blocks;
+ *     FP16 value aggregation with FP32 accumulation; calibrated key centring; at most two
+ *     blocks kept at BF16 per sequence; the cache is packed directly from BF16 activations.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise; the caller owns
+ *     every buffer (caches, inputs, outputs and the workspace). The library allocates no
+ *     device memory and keeps no pointer after the call returns.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and never
+ *     synchronise, except qs_device_status.
+ *   - Arguments are validated on the host before any launch. On failure the call returns
+ *     QS_ERR_INVALID_ARG (bad pointer/size) or QS_ERR_UNSUPPORTED (a shape this build does
+ *     not implement) and launches nothing. There is no fallback path.
+ *   - Values that live on the device (sequence lengths, page-table entries, n_new, the
+ *     selection) are checked by the kernels: an out-of-range value skips the access and
+ *     records QS_ERR_DEVICE_BOUNDS in the workspace status word, which qs_device_status
+ *     reads. Waits inside kernels are bounded; running out records QS_ERR_DEVICE_TIMEOUT.
+ *   - A launch error is returned as QS_ERR_CUDA (the CUDA error is left for
+ *     cudaGetLastError by the caller).
+ *   - Entry points are re-entrant and keep no global state; two calls that share a
+ *     workspace must not overlap on the GPU.
+ *
+ * Memory layouts (row-major, innermost last):
+ *   K, V pages      [num_pages][Hkv][page_size][head_dim]   BF16 (V may be FP16)
+ *   proxy (rank r)  [num_pages][Hkv][page_size][r]          F32 or BF16
+ *   proxy (NVFP4)   [num_pages][Hkv][page_size][head_dim/2] u8: E2M1 codes, element 2i in
+ *                                                           the low nibble of byte i
+ *   proxy_scale     [num_pages][Hkv][page_size][head_dim/16] u8: UE4M3 scale per 16 elems
+ *   page_table      [batch][max_pages_per_seq]              int32 physical page ids
+ *   seq_lens        [batch]                                 int32 tokens in the cache
+ *   P               [Hkv][head_dim][r]                      F32
+ *   q, out          [batch][Hq][head_dim]                   q BF16; out F32 or BF16
+ *   k_new, v_new    [batch][Hkv][max_new][head_dim]         K BF16, V as v_dtype
+ *   block scores    [batch][Hkv][nb_stride]  F32, nb_stride = ceil(max_context / page_size)
+ *                                                                 * (page_size / block_size)
+ *   sel             [batch][Hkv][budget]     int32 ascending block ids, padded with -1
+ *   n_sel           [batch][Hkv]             int32 = min(budget, ceil(seq_len / block_size))
+ * Query head h belongs to KV head h / (Hq / Hkv).
+ */
+#ifndef QS_H
+#define QS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *qs_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  QS_OK = 0,
+  QS_ERR_INVALID_ARG = 1,
+  QS_ERR_UNSUPPORTED = 2,
+  QS_ERR_CUDA = 3,
+  QS_ERR_DEVICE_BOUNDS = 4,
+  QS_ERR_DEVICE_TIMEOUT = 5
+} qs_status;
+
+typedef enum { QS_F32 = 0, QS_BF16 = 1, QS_F16 = 2, QS_NVFP4 = 3 } qs_dtype;
+
+/* Problem statement of one attention layer's decode step. */
+typedef struct {
+  int32_t n_q_heads;      /* Hq; Hq % Hkv == 0 and the group G = Hq / Hkv <= 8          */
+  int32_t n_kv_heads;     /* Hkv                                                          */
+  int32_t head_dim;       /* d: 64 or 128 (NVFP4 scoring needs 128)                       */
+  int32_t page_size;      /* tokens per cache page: 128                                   */
+  int32_t block_size;     /* S: a power of two dividing page_size (1 = token level)       */
+  int32_t budget;         /* k: blocks selected per row, >= 1                             */
+  int32_t proxy_rank;     /* r > 0: projected-key proxy; 0: NVFP4 centred keys            */
+  int32_t proxy_dtype;    /* qs_dtype: F32 or BF16 (rank r), NVFP4 (r == 0)               */
+  int32_t v_dtype;        /* qs_dtype of stored V: BF16 or F16                            */
+  int32_t v_agg_dtype;    /* precision of the P.V operands: BF16 or F16 (FP32 accumulate) */
+  int32_t out_dtype;      /* F32 or BF16                                                  */
+  int32_t force_sink;     /* 1: block 0 is always selected                                */
+  int32_t force_last;     /* 1: the block holding the newest token is always selected     */
+  int32_t n_keep_hp;      /* NVFP4: 0..2 blocks with the largest quantisation error are
+                             kept at full precision and always selected                  */
+  float softmax_scale;    /* 0 => 1/sqrt(d)                                               */
+} qs_config;
+
+/* The paged caches of one layer. All pointers are device pointers owned by the caller. */
+typedef struct {
+  void *k;                    /* K pages, BF16                                            */
+  void *v;                    /* V pages, v_dtype                                         */
+  void *proxy;                /* scoring cache (layout above)                             */
+  uint8_t *proxy_scale;       /* NVFP4 only: UE4M3 scales; NULL otherwise                 */
+  float *block_err;           /* NVFP4 only: [batch][Hkv][nb_stride] squared quantisation
+                                 error of each complete block (written by qs_append_kv)   */
+  const float *key_center;    /* NVFP4 only: [batch][Hkv][d] calibrated centring mean     */
+  const float *key_gscale;    /* NVFP4 only: 1 float, the key tensor scale g_k            */
+  const int32_t *page_table;  /* [batch][max_pages_per_seq]                               */
+  int32_t *seq_lens;          /* [batch]; advanced by qs_append_kv / qs_decode            */
+  int32_t max_pages_per_seq;  /* row stride of page_table                                 */
+  int32_t num_pages;          /* physical pages in k / v / proxy                          */
+  int32_t max_context;        /* upper bound of every seq_len; sizes nb_stride           */
+} qs_cache;
+
+/* Bytes of workspace that the calls below need for `batch` sequences (host only, no
+   device access). QS_ERR_INVALID_ARG / QS_ERR_UNSUPPORTED as for the other calls. */
+qs_status qs_workspace_size(const qs_config *cfg, int32_t batch, int32_t max_context,
+                            size_t *bytes /* host */);
+
+/* Zero the workspace status word and counters (async on stream). Call once after
+   allocating a workspace, before any other call uses it. */
+qs_status qs_workspace_init(void *ws, size_t ws_bytes, qs_stream_t stream);
+
+/* Append n_new[b] tokens to every KV head of sequence b, then advance seq_lens[b].
+   Writes K/V into page slot seq_lens[b] + i and the row's scoring cache:
+     rank r: proxy = k.P[g] in float32 (ascending index, one rounding per product and per
+             sum), stored F32 or rounded to nearest-even BF16;
+     NVFP4:  x = float(k) - key_center[b][g] (float32), packed per 16 elements to UE4M3
+             scale + E2M1 codes with the tensor scale g_k; each block of S tokens that this
+             call completes gets block_err = sum of squared (x - dequant(x)).
+   k_new/v_new: [batch][Hkv][max_new][d]; n_new: device int32 [batch], each <= max_new;
+   P: [Hkv][d][r] (NULL for NVFP4). Pages for the new tokens must be in page_table. */
+qs_status qs_append_kv(const qs_config *cfg, const qs_cache *cache, const void *k_new,
+                       const void *v_new, const int32_t *n_new, int32_t max_new,
+                       const float *P, int32_t batch, void *ws, qs_stream_t stream);
+
+/* Proxy block scores of every row (stage 1).
+   rank r: qbar = mean of the group's query heads (float32), q~ = qbar.P[g] (float32),
+           s_t = q~ . proxy_t (float32 accumulation), beta_j = max of s over the block's
+           valid tokens (t < seq_len).
+   NVFP4:  the whole q tensor is packed with g_q = max|q| / 2688; per head h,
+           s_{h,t} = g_q g_k sum_c sq_{h,c} sk_{t,c} sum_i eq_{h,16c+i} ek_{t,16c+i} on the
+           block-scaled FP4 tensor cores; beta_j = max over the group's heads and the
+           block's valid tokens.
+   Blocks past ceil(seq_len / S) that share a page with valid tokens are written -inf;
+   entries past the last page of a row are not written.
+   q: [batch][Hq][d] BF16; P as in qs_append_kv; block_scores: [batch][Hkv][nb_stride]. */
+qs_status qs_score(const qs_config *cfg, const qs_cache *cache, const void *q,
+                   const float *P, int32_t batch, float *block_scores, void *ws,
+                   qs_stream_t stream);
+
+/* Top-k block selection of every row (stage 2).
+   nb = ceil(seq_len / S). If nb <= budget every block is selected. Otherwise the forced
+   set F (block 0 if force_sink, block nb-1 if force_last, and on the NVFP4 path the
+   n_keep_hp complete blocks with the largest block_err, ties to the lower index) is taken
+   first; the remaining budget - |F| blocks are the best-scoring others, ties to the lower
+   index. NaN scores rank as the lowest finite value. Output ascending, padded with -1. */
+qs_status qs_select_topk(const qs_config *cfg, const qs_cache *cache,
+                         const float *block_scores, int32_t batch, int32_t *sel,
+                         int32_t *n_sel, void *ws, qs_stream_t stream);
+
+/* Exact softmax attention over the selected blocks' valid tokens (stage 3).
+   For every query head h of row (b, g): o_h = sum_t softmax_t(scale * q_h.k_t) v_t over
+   t in the selected blocks (t < seq_len), normalised over those tokens only. Logits are
+   float32 sums of BF16 products; P.V operands are v_agg_dtype, accumulated in float32.
+   The selection is split across CTAs; partial (max, sum, o) states are merged by a
+   log-sum-exp combine. out: [batch][Hq][d] in out_dtype. */
+qs_status qs_sparse_attn(const qs_config *cfg, const qs_cache *cache, const void *q,
+                         const int32_t *sel, const int32_t *n_sel, int32_t batch, void *out,
+                         void *ws, qs_stream_t stream);
+
+/* One decode step: append one token per sequence (k_new/v_new: [batch][Hkv][d]), then
+   score, select and attend over seq_len + 1 tokens. sel_out / n_sel_out may be NULL; the
+   selection then stays in the workspace. */
+qs_status qs_decode(const qs_config *cfg, const qs_cache *cache, const void *q,
+                    const void *k_new, const void *v_new, const float *P, int32_t batch,
+                    void *out, int32_t *sel_out, int32_t *n_sel_out, void *ws,
+                    qs_stream_t stream);
+
+/* Synchronise `stream`, return the first device-side error recorded in the workspace
+   since the last call (QS_OK if none) and clear it. `detail` (HOST pointer, may be NULL)
+   receives {kernel id, index} of that error. Returns QS_ERR_CUDA if the synchronisation
+   or the read-back fails. Kernel ids: 1 append, 2 block error, 3 scoring prep, 4 score,
+   5 select, 6 attention, 7 combine. */
+qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
+
+/* Static string naming a status code. */
+const char *qs_status_string(qs_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t qs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QS_H */

@@ -1,0 +1,14 @@
+"""Score-then-select sparse decode attention for B200 (sm_100a).
+
+The decode path runs in libqs.so (hand-written CUDA behind the C ABI in include/qs.h);
+this package is its ctypes binding plus torch helpers that allocate the caches. There is
+no CPU fallback: importing the binding's entry points requires the built library.
+"""
+from .binding import (QsError, LIB_PATH, EXPORTS, lib, make_config, make_cache, qs_version,
+                      qs_workspace_size, qs_workspace_init, qs_append_kv, qs_score,
+                      qs_select_topk, qs_sparse_attn, qs_decode, qs_device_status,
+                      status_string)
+
+__all__ = ["QsError", "LIB_PATH", "EXPORTS", "lib", "make_config", "make_cache", "qs_version",
+           "qs_workspace_size", "qs_workspace_init", "qs_append_kv", "qs_score",
+           "qs_select_topk", "qs_sparse_attn", "qs_decode", "qs_device_status", "status_string"]

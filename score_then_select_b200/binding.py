@@ -1,0 +1,186 @@
+"""ctypes binding of libqs (include/qs.h): the same entry points, argument marshalling only.
+
+Every function takes device buffers as torch tensors (or raw integer addresses) and a CUDA
+stream (a torch.cuda.Stream, a raw handle, or None for torch's current stream), calls the
+C entry point of the same name, and raises QsError when it returns a status other than
+QS_OK. No computation happens here.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqs.so")
+
+QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA, QS_ERR_DEVICE_BOUNDS, \
+    QS_ERR_DEVICE_TIMEOUT = range(6)
+QS_F32, QS_BF16, QS_F16, QS_NVFP4 = range(4)
+DTYPE_CODES = {"f32": QS_F32, "bf16": QS_BF16, "f16": QS_F16, "nvfp4": QS_NVFP4}
+
+
+class QsError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class qs_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_q_heads", "n_kv_heads", "head_dim", "page_size", "block_size", "budget",
+        "proxy_rank", "proxy_dtype", "v_dtype", "v_agg_dtype", "out_dtype", "force_sink",
+        "force_last", "n_keep_hp")] + [("softmax_scale", ctypes.c_float)]
+
+
+class qs_cache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("proxy", ctypes.c_void_p),
+                ("proxy_scale", ctypes.c_void_p), ("block_err", ctypes.c_void_p),
+                ("key_center", ctypes.c_void_p), ("key_gscale", ctypes.c_void_p),
+                ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("max_context", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqs.so from the package directory; fail loudly if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m score_then_select_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        cfgp, cachep = ctypes.POINTER(qs_config), ctypes.POINTER(qs_cache)
+        sig = {
+            "qs_version": ([], i32),
+            "qs_status_string": ([i32], ctypes.c_char_p),
+            "qs_workspace_size": ([cfgp, i32, i32, ctypes.POINTER(sz)], i32),
+            "qs_workspace_init": ([vp, sz, vp], i32),
+            "qs_append_kv": ([cfgp, cachep, vp, vp, vp, i32, vp, i32, vp, vp], i32),
+            "qs_score": ([cfgp, cachep, vp, vp, i32, vp, vp, vp], i32),
+            "qs_select_topk": ([cfgp, cachep, vp, i32, vp, vp, vp, vp], i32),
+            "qs_sparse_attn": ([cfgp, cachep, vp, vp, vp, i32, vp, vp, vp], i32),
+            "qs_decode": ([cfgp, cachep, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp], i32),
+            "qs_device_status": ([vp, vp, ctypes.POINTER(ctypes.c_uint32)], i32),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_init",
+           "qs_append_kv", "qs_score", "qs_select_topk", "qs_sparse_attn", "qs_decode",
+           "qs_device_status")
+
+
+def status_string(s: int) -> str:
+    return lib().qs_status_string(int(s)).decode()
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != QS_OK:
+        raise QsError(st, where)
+
+
+def make_config(*, n_q_heads, n_kv_heads, head_dim, block_size, budget, proxy_rank,
+                proxy_dtype, v_dtype="bf16", v_agg_dtype="bf16", out_dtype="bf16",
+                force_sink=False, force_last=False, n_keep_hp=0, softmax_scale=0.0,
+                page_size=128) -> qs_config:
+    c = qs_config()
+    c.n_q_heads, c.n_kv_heads, c.head_dim = n_q_heads, n_kv_heads, head_dim
+    c.page_size, c.block_size, c.budget = page_size, block_size, budget
+    c.proxy_rank = proxy_rank
+    c.proxy_dtype = DTYPE_CODES[proxy_dtype]
+    c.v_dtype, c.v_agg_dtype = DTYPE_CODES[v_dtype], DTYPE_CODES[v_agg_dtype]
+    c.out_dtype = DTYPE_CODES[out_dtype]
+    c.force_sink, c.force_last, c.n_keep_hp = int(force_sink), int(force_last), n_keep_hp
+    c.softmax_scale = softmax_scale
+    return c
+
+
+def make_cache(*, k, v, proxy, page_table, seq_lens, max_context, proxy_scale=None,
+               block_err=None, key_center=None, key_gscale=None) -> qs_cache:
+    c = qs_cache()
+    c.k, c.v, c.proxy = _ptr(k), _ptr(v), _ptr(proxy)
+    c.proxy_scale, c.block_err = _ptr(proxy_scale), _ptr(block_err)
+    c.key_center, c.key_gscale = _ptr(key_center), _ptr(key_gscale)
+    c.page_table, c.seq_lens = _ptr(page_table), _ptr(seq_lens)
+    c.max_pages_per_seq = int(page_table.shape[1]) if hasattr(page_table, "shape") else 0
+    c.num_pages = int(k.shape[0]) if hasattr(k, "shape") else 0
+    c.max_context = int(max_context)
+    return c
+
+
+# ------------------------------------------------------------------ entry points
+
+def qs_version() -> int:
+    return lib().qs_version()
+
+
+def qs_workspace_size(cfg: qs_config, batch: int, max_context: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().qs_workspace_size(ctypes.byref(cfg), batch, max_context, ctypes.byref(n)),
+           "qs_workspace_size")
+    return n.value
+
+
+def qs_workspace_init(ws, nbytes: int, stream=None):
+    _check(lib().qs_workspace_init(_ptr(ws), nbytes, _stream(stream)), "qs_workspace_init")
+
+
+def qs_append_kv(cfg, cache, k_new, v_new, n_new, max_new, P, batch, ws, stream=None):
+    _check(lib().qs_append_kv(ctypes.byref(cfg), ctypes.byref(cache), _ptr(k_new), _ptr(v_new),
+                              _ptr(n_new), max_new, _ptr(P), batch, _ptr(ws), _stream(stream)),
+           "qs_append_kv")
+
+
+def qs_score(cfg, cache, q, P, batch, block_scores, ws, stream=None):
+    _check(lib().qs_score(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(P), batch,
+                          _ptr(block_scores), _ptr(ws), _stream(stream)), "qs_score")
+
+
+def qs_select_topk(cfg, cache, block_scores, batch, sel, n_sel, ws, stream=None):
+    _check(lib().qs_select_topk(ctypes.byref(cfg), ctypes.byref(cache), _ptr(block_scores),
+                                batch, _ptr(sel), _ptr(n_sel), _ptr(ws), _stream(stream)),
+           "qs_select_topk")
+
+
+def qs_sparse_attn(cfg, cache, q, sel, n_sel, batch, out, ws, stream=None):
+    _check(lib().qs_sparse_attn(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(sel),
+                                _ptr(n_sel), batch, _ptr(out), _ptr(ws), _stream(stream)),
+           "qs_sparse_attn")
+
+
+def qs_decode(cfg, cache, q, k_new, v_new, P, batch, out, sel_out, n_sel_out, ws, stream=None):
+    _check(lib().qs_decode(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(k_new),
+                           _ptr(v_new), _ptr(P), batch, _ptr(out), _ptr(sel_out),
+                           _ptr(n_sel_out), _ptr(ws), _stream(stream)), "qs_decode")
+
+
+def qs_device_status(ws, stream=None) -> tuple[int, int, int]:
+    """(status, kernel id, index) of the first device-side error since the last read."""
+    detail = (ctypes.c_uint32 * 2)()
+    st = lib().qs_device_status(_ptr(ws), _stream(stream), detail)
+    return st, detail[0], detail[1]

@@ -1,0 +1,403 @@
+// api.cu - the C ABI of libqs: argument validation, launch plans, workspace layout and
+// the entry points declared in include/qs.h. No device memory is allocated here.
+#include <cmath>
+#include <cstring>
+
+#include "qs_internal.h"
+
+namespace qs {
+
+int num_sms() {
+  static thread_local int cached = 0;
+  if (cached > 0) return cached;
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+    cached = n;
+  else {
+    cudaGetLastError();
+    cached = 148;
+  }
+  return cached;
+}
+
+static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Attention split plan: choose splits per row so the grid fills whole waves of resident
+// CTAs (2 per SM) as evenly as possible; tokens per split is a multiple of the tile.
+static void plan_splits(int rows, int slots, int& splits, int& tps) {
+  const int slots_per_wave = 2 * num_sms();
+  double best = 1e30;
+  splits = 1;
+  tps = 64;
+  for (int s = 1; s <= 64; ++s) {
+    int t = (slots + s - 1) / s;
+    t = (t + 63) / 64 * 64;
+    if (t > 2048) continue;
+    if ((s - 1) * t >= slots && s > 1) break;  // later splits would be empty
+    const long long ctas = (long long)rows * s;
+    const long long waves = (ctas + slots_per_wave - 1) / slots_per_wave;
+    // time model: waves x tokens per CTA, plus a small per-CTA fixed cost
+    const double cost = double(waves) * (t + 96.0);
+    if (cost < best - 1e-9) {
+      best = cost;
+      splits = s;
+      tps = t;
+    }
+  }
+}
+
+static qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
+  if (!c) return QS_ERR_INVALID_ARG;
+  if (batch < 1 || batch > kMaxBatch || max_context < 1) return QS_ERR_INVALID_ARG;
+  if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads) return QS_ERR_INVALID_ARG;
+  if (c->budget < 1 || c->page_size < 1 || c->block_size < 1) return QS_ERR_INVALID_ARG;
+  if (!is_pow2(c->block_size) || c->page_size % c->block_size) return QS_ERR_INVALID_ARG;
+  if (c->force_sink < 0 || c->force_sink > 1 || c->force_last < 0 || c->force_last > 1)
+    return QS_ERR_INVALID_ARG;
+  if (c->n_keep_hp < 0 || c->n_keep_hp > 2) return QS_ERR_INVALID_ARG;
+  if (!(c->softmax_scale >= 0.0f) || !std::isfinite(c->softmax_scale)) return QS_ERR_INVALID_ARG;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  if (G > kMaxGroup) return QS_ERR_UNSUPPORTED;
+  if (c->page_size != kPage) return QS_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return QS_ERR_UNSUPPORTED;
+  const int r = c->proxy_rank;
+  if (r < 0) return QS_ERR_INVALID_ARG;
+  if (r > 0) {
+    const bool ok = (c->proxy_dtype == QS_F32 && (r == 16 || (r == 32 && c->head_dim == 128))) ||
+                    (c->proxy_dtype == QS_BF16 && (r == 32 || (r == 64 && c->head_dim == 128)));
+    if (!ok) return QS_ERR_UNSUPPORTED;
+    if (c->n_keep_hp != 0) return QS_ERR_INVALID_ARG;
+  } else {
+    if (c->proxy_dtype != QS_NVFP4) return QS_ERR_INVALID_ARG;
+    if (c->head_dim != 128) return QS_ERR_UNSUPPORTED;
+    if (c->block_size != kPage) return QS_ERR_UNSUPPORTED;
+  }
+  if (c->v_dtype != QS_BF16 && c->v_dtype != QS_F16) return QS_ERR_INVALID_ARG;
+  if (c->v_agg_dtype != QS_BF16 && c->v_agg_dtype != QS_F16) return QS_ERR_INVALID_ARG;
+  if (c->v_dtype == QS_F16 && c->v_agg_dtype != QS_F16) return QS_ERR_UNSUPPORTED;
+  if (c->out_dtype != QS_F32 && c->out_dtype != QS_BF16) return QS_ERR_INVALID_ARG;
+
+  p.batch = batch;
+  p.Hq = c->n_q_heads;
+  p.Hkv = c->n_kv_heads;
+  p.G = G;
+  p.d = c->head_dim;
+  p.S = c->block_size;
+  p.budget = c->budget;
+  p.r = r;
+  p.proxy_dtype = c->proxy_dtype;
+  p.v_dtype = c->v_dtype;
+  p.v_agg_dtype = c->v_agg_dtype;
+  p.out_dtype = c->out_dtype;
+  p.force_sink = c->force_sink;
+  p.force_last = c->force_last;
+  p.n_keep = c->n_keep_hp;
+  p.scale = c->softmax_scale > 0.0f ? c->softmax_scale : 1.0f / std::sqrt(float(c->head_dim));
+  const long long pages = (max_context + kPage - 1) / kPage;
+  const long long nbs = pages * (kPage / p.S);
+  if (nbs > kMaxSelectBlocks) return QS_ERR_UNSUPPORTED;
+  p.nb_stride = int(nbs);
+  const long long slots = (long long)p.budget * p.S;
+  if (slots > 64LL * 2048) return QS_ERR_UNSUPPORTED;
+
+  WsLayout& w = p.ws;
+  w.nb_stride = p.nb_stride;
+  plan_splits(batch * p.Hkv, int(slots), w.splits, w.tokens_per_split);
+  size_t off = size_t(kHdrWords) * 4;
+  const size_t rows = size_t(batch) * p.Hkv, rows_q = size_t(batch) * p.Hq;
+  w.qt = off;      off = align_up(off + rows * (r > 0 ? r : 1) * 4, 256);
+  w.qcodes = off;  off = align_up(off + (r == 0 ? rows_q * p.d / 2 : 0), 256);
+  w.qscales = off; off = align_up(off + (r == 0 ? rows_q * p.d / 16 : 0), 256);
+  w.qgscale = off; off = align_up(off + 16, 256);
+  w.scores = off;  off = align_up(off + rows * p.nb_stride * 4, 256);
+  w.sel = off;     off = align_up(off + rows * p.budget * 4, 256);
+  w.nsel = off;    off = align_up(off + rows * 4, 256);
+  w.part_ml = off; off = align_up(off + rows_q * w.splits * 2 * 4, 256);
+  w.part_o = off;  off = align_up(off + rows_q * w.splits * p.d * 4, 256);
+  w.total = off;
+  return QS_OK;
+}
+
+static qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy) {
+  if (!c || !c->k || !c->v || !c->page_table || !c->seq_lens) return QS_ERR_INVALID_ARG;
+  if (c->max_pages_per_seq < 1 || c->num_pages < 1 || c->max_context < 1) return QS_ERR_INVALID_ARG;
+  if ((long long)c->num_pages * p.Hkv * kPage >= (1LL << 31)) return QS_ERR_UNSUPPORTED;
+  if (!aligned(c->k, 16) || !aligned(c->v, 16)) return QS_ERR_INVALID_ARG;
+  if (need_proxy) {
+    if (!c->proxy || !aligned(c->proxy, 16)) return QS_ERR_INVALID_ARG;
+    if (p.r == 0 && (!c->proxy_scale || !c->key_center || !c->key_gscale)) return QS_ERR_INVALID_ARG;
+  }
+  return QS_OK;
+}
+
+static uint32_t* hdr_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
+template <typename T>
+static T* ws_at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ws) + off);
+}
+
+static qs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QS_OK : QS_ERR_CUDA; }
+
+// ------------------------------------------------------------ stage bodies (validated input)
+static qs_status do_append(const Plan& p, const qs_cache* c, const void* k_new, const void* v_new,
+                           const int32_t* n_new, int max_new, const float* P, const void* q,
+                           void* ws, cudaStream_t s) {
+  AppendParams a{};
+  a.k_new = static_cast<const uint16_t*>(k_new);
+  a.v_new = static_cast<const uint16_t*>(v_new);
+  a.n_new = n_new;
+  a.P = P;
+  a.k = static_cast<uint16_t*>(c->k);
+  a.v = static_cast<uint16_t*>(c->v);
+  a.proxy = c->proxy;
+  a.proxy_scale = c->proxy_scale;
+  a.key_center = c->key_center;
+  a.key_gscale = c->key_gscale;
+  a.page_table = c->page_table;
+  a.seq_lens = c->seq_lens;
+  a.hdr = hdr_of(ws);
+  a.q = (p.r > 0) ? static_cast<const uint16_t*>(q) : nullptr;
+  a.qt = ws_at<float>(ws, p.ws.qt);
+  a.batch = p.batch;
+  a.Hkv = p.Hkv;
+  a.G = p.G;
+  a.d = p.d;
+  a.r = p.r;
+  a.max_new = max_new;
+  a.max_pages_per_seq = c->max_pages_per_seq;
+  a.num_pages = c->num_pages;
+  a.max_context = c->max_context;
+  qs_status st = cuda_status(launch_append(p, a, s));
+  if (st != QS_OK || p.r != 0) return st;
+  BlockErrParams e{};
+  e.k = a.k;
+  e.key_center = c->key_center;
+  e.key_gscale = c->key_gscale;
+  e.page_table = c->page_table;
+  e.seq_lens = c->seq_lens;
+  e.n_new = n_new;
+  e.block_err = c->block_err;
+  e.hdr = a.hdr;
+  e.batch = p.batch;
+  e.Hkv = p.Hkv;
+  e.d = p.d;
+  e.S = p.S;
+  e.nb_stride = p.nb_stride;
+  e.max_pages_per_seq = c->max_pages_per_seq;
+  e.num_pages = c->num_pages;
+  e.max_blocks_per_call = max_new / p.S + 1;
+  return cuda_status(launch_block_err(p, e, s));
+}
+
+static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws, cudaStream_t s) {
+  if (p.r > 0) {
+    PrepParams a{static_cast<const uint16_t*>(q), P, ws_at<float>(ws, p.ws.qt),
+                 p.batch, p.Hkv, p.G, p.d, p.r};
+    return cuda_status(launch_prep(p, a, s));
+  }
+  QPackParams a{static_cast<const uint16_t*>(q), ws_at<uint8_t>(ws, p.ws.qcodes),
+                ws_at<uint8_t>(ws, p.ws.qscales), ws_at<float>(ws, p.ws.qgscale),
+                p.batch * p.Hq * p.d, p.d};
+  return cuda_status(launch_qpack(p, a, s));
+}
+
+static qs_status do_score(const Plan& p, const qs_cache* c, float* scores, void* ws, cudaStream_t s) {
+  ScoreParams a{};
+  a.proxy = c->proxy;
+  a.proxy_scale = c->proxy_scale;
+  a.qt = ws_at<float>(ws, p.ws.qt);
+  a.qcodes = ws_at<uint8_t>(ws, p.ws.qcodes);
+  a.qscales = ws_at<uint8_t>(ws, p.ws.qscales);
+  a.qgscale = ws_at<float>(ws, p.ws.qgscale);
+  a.key_gscale = c->key_gscale;
+  a.page_table = c->page_table;
+  a.seq_lens = c->seq_lens;
+  a.scores = scores;
+  a.hdr = hdr_of(ws);
+  a.batch = p.batch;
+  a.Hkv = p.Hkv;
+  a.G = p.G;
+  a.d = p.d;
+  a.S = p.S;
+  a.nb_stride = p.nb_stride;
+  a.max_pages_per_seq = c->max_pages_per_seq;
+  a.num_pages = c->num_pages;
+  a.max_context = c->max_context;
+  return cuda_status(launch_score(p, a, s));
+}
+
+static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores, int32_t* sel,
+                           int32_t* n_sel, void* ws, cudaStream_t s) {
+  SelectParams a{};
+  a.scores = scores;
+  a.block_err = (p.r == 0 && p.n_keep > 0) ? c->block_err : nullptr;
+  a.seq_lens = c->seq_lens;
+  a.sel = sel;
+  a.n_sel = n_sel;
+  a.hdr = hdr_of(ws);
+  a.rows = p.batch * p.Hkv;
+  a.Hkv = p.Hkv;
+  a.S = p.S;
+  a.nb_stride = p.nb_stride;
+  a.budget = p.budget;
+  a.force_sink = p.force_sink;
+  a.force_last = p.force_last;
+  a.n_keep = a.block_err ? p.n_keep : 0;
+  return cuda_status(launch_select(p, a, s));
+}
+
+static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, const int32_t* sel,
+                           const int32_t* n_sel, void* out, void* ws, cudaStream_t s) {
+  AttnParams a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(c->k);
+  a.v = static_cast<const uint16_t*>(c->v);
+  a.sel = sel;
+  a.n_sel = n_sel;
+  a.page_table = c->page_table;
+  a.seq_lens = c->seq_lens;
+  a.part_ml = ws_at<float>(ws, p.ws.part_ml);
+  a.part_o = ws_at<float>(ws, p.ws.part_o);
+  a.hdr = hdr_of(ws);
+  a.batch = p.batch;
+  a.Hkv = p.Hkv;
+  a.G = p.G;
+  a.S = p.S;
+  a.budget = p.budget;
+  a.splits = p.ws.splits;
+  a.tokens_per_split = p.ws.tokens_per_split;
+  a.max_pages_per_seq = c->max_pages_per_seq;
+  a.num_pages = c->num_pages;
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  qs_status st = cuda_status(launch_attn(p, a, s));
+  if (st != QS_OK) return st;
+  CombineParams cb{a.part_ml, a.part_o, out, p.batch * p.Hq, p.ws.splits, p.d,
+                   p.out_dtype == QS_BF16 ? 1 : 0};
+  return cuda_status(launch_combine(p, cb, s));
+}
+
+}  // namespace qs
+
+using namespace qs;
+
+extern "C" {
+
+int32_t qs_version(void) { return 10000; }
+
+const char* qs_status_string(qs_status s) {
+  switch (s) {
+    case QS_OK: return "ok";
+    case QS_ERR_INVALID_ARG: return "invalid argument";
+    case QS_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case QS_ERR_CUDA: return "CUDA error";
+    case QS_ERR_DEVICE_BOUNDS: return "device-side bounds check failed";
+    case QS_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+qs_status qs_workspace_size(const qs_config* cfg, int32_t batch, int32_t max_context, size_t* bytes) {
+  if (!bytes) return QS_ERR_INVALID_ARG;
+  Plan p;
+  qs_status st = make_plan(cfg, batch, max_context, p);
+  if (st != QS_OK) return st;
+  *bytes = p.ws.total;
+  return QS_OK;
+}
+
+qs_status qs_workspace_init(void* ws, size_t ws_bytes, qs_stream_t stream) {
+  if (!ws || ws_bytes < size_t(kHdrWords) * 4 || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, size_t(kHdrWords) * 4, stream));
+}
+
+qs_status qs_append_kv(const qs_config* cfg, const qs_cache* cache, const void* k_new,
+                       const void* v_new, const int32_t* n_new, int32_t max_new, const float* P,
+                       int32_t batch, void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if ((st = check_cache(p, cache, true)) != QS_OK) return st;
+  if (!k_new || !v_new || !n_new || max_new < 1 || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
+  if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
+  if (p.r == 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
+  return do_append(p, cache, k_new, v_new, n_new, max_new, P, nullptr, ws, stream);
+}
+
+qs_status qs_score(const qs_config* cfg, const qs_cache* cache, const void* q, const float* P,
+                   int32_t batch, float* block_scores, void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if ((st = check_cache(p, cache, true)) != QS_OK) return st;
+  if (!q || !aligned(q, 4) || !block_scores || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
+  if ((st = do_prep(p, q, P, ws, stream)) != QS_OK) return st;
+  return do_score(p, cache, block_scores, ws, stream);
+}
+
+qs_status qs_select_topk(const qs_config* cfg, const qs_cache* cache, const float* block_scores,
+                         int32_t batch, int32_t* sel, int32_t* n_sel, void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (!cache || !cache->seq_lens) return QS_ERR_INVALID_ARG;
+  if (!block_scores || !sel || !n_sel || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (p.r == 0 && p.n_keep > 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
+  return do_select(p, cache, block_scores, sel, n_sel, ws, stream);
+}
+
+qs_status qs_sparse_attn(const qs_config* cfg, const qs_cache* cache, const void* q,
+                         const int32_t* sel, const int32_t* n_sel, int32_t batch, void* out,
+                         void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if ((st = check_cache(p, cache, false)) != QS_OK) return st;
+  if (!q || !aligned(q, 4) || !sel || !n_sel || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  return do_attend(p, cache, q, sel, n_sel, out, ws, stream);
+}
+
+qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, const void* k_new,
+                    const void* v_new, const float* P, int32_t batch, void* out, int32_t* sel_out,
+                    int32_t* n_sel_out, void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if ((st = check_cache(p, cache, true)) != QS_OK) return st;
+  if (!q || !aligned(q, 4) || !k_new || !v_new || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
+  if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
+  if (p.r == 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
+  if ((sel_out == nullptr) != (n_sel_out == nullptr)) return QS_ERR_INVALID_ARG;
+  int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, p.ws.sel);
+  int32_t* nsel = n_sel_out ? n_sel_out : ws_at<int32_t>(ws, p.ws.nsel);
+  float* scores = ws_at<float>(ws, p.ws.scores);
+  // append (+ fused scoring prep on the rank-r path)
+  if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, P, q, ws, stream)) != QS_OK) return st;
+  if (p.r == 0 && (st = do_prep(p, q, P, ws, stream)) != QS_OK) return st;
+  if ((st = do_score(p, cache, scores, ws, stream)) != QS_OK) return st;
+  if ((st = do_select(p, cache, scores, sel, nsel, ws, stream)) != QS_OK) return st;
+  return do_attend(p, cache, q, sel, nsel, out, ws, stream);
+}
+
+qs_status qs_device_status(void* ws, qs_stream_t stream, uint32_t* detail) {
+  if (!ws) return QS_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return QS_ERR_CUDA;
+  uint32_t h[3] = {0, 0, 0};
+  if (cudaMemcpy(h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return QS_ERR_CUDA;
+  if (detail) {
+    detail[0] = h[1];
+    detail[1] = h[2];
+  }
+  if (h[0] != 0) {
+    if (cudaMemset(ws, 0, sizeof(h)) != cudaSuccess) return QS_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return QS_ERR_CUDA;
+  }
+  return static_cast<qs_status>(h[0]);
+}
+
+}  // extern "C"

@@ -1,0 +1,476 @@
+// append.cu - cache writers fused with the KV append, and the scoring-prep kernels.
+//
+// Rank-r writer ("Joint Subspace Sparse Attention for Efficient Long-Context Decoding",
+// Figure 1): the projected-key cache entry of a new token is k . P[g], evaluated in float32
+// in ascending index order with one rounding per product and per sum (no fused
+// multiply-add), then stored as float32 or rounded to nearest-even BF16 (Figure 10 allows
+// a reduced-precision scoring cache).
+//
+// NVFP4 writer ("Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse
+// Attention", Full text): the persistent scoring cache is packed straight from the BF16
+// keys after calibrated centring: x = float(k) - mu (float32), then per 16 elements
+// a = max|x|, sf = a / (6 g_k), sigma = UE4M3(sf), e_i = E2M1(x_i / (sigma g_k)), every
+// step a correctly rounded float32 operation, every conversion nearest-even and
+// saturating. Blocks completed by the append get their squared quantisation error, which
+// decides the blocks kept at full precision.
+#include "qs_device.cuh"
+
+namespace qs {
+
+// ============================================================ NVFP4 element / scale codecs
+// E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}: count the rounding thresholds passed; a
+// value exactly on a midpoint goes to the neighbour with the even code (strict '>' where
+// the lower code is even, '>=' where the upper code is even); beyond 6 saturates to 6.
+QS_DEV uint32_t e2m1_encode(float t) {
+  const uint32_t sign = (__float_as_uint(t) >> 31) << 3;
+  const float a = fabsf(t);
+  const uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+                     (a >= 3.5f) + (a > 5.0f);
+  return sign | c;
+}
+QS_DEV float e2m1_decode(uint32_t c) {
+  const uint32_t m = c & 7u;
+  // magnitudes: m < 4 -> m/2 ; m >= 4 -> {2, 3, 4, 6}
+  float v = (m < 4u) ? 0.5f * float(m) : (m == 7u ? 6.0f : float(m - 2u));
+  return (c & 8u) ? -v : v;
+}
+// UE4M3 (bias 7, 3 mantissa bits, subnormal step 2^-9, largest finite 448 = 0x7E):
+// nearest even, saturating; non-positive and NaN inputs give code 0.
+QS_DEV uint32_t ue4m3_encode(float sf) {
+  if (!(sf > 0.0f)) return 0u;
+  if (sf >= 448.0f) return 0x7Eu;
+  const uint32_t u = __float_as_uint(sf);
+  const int e = int(u >> 23) - 127;
+  if (e < -6) return __float2uint_rn(sf * 512.0f);  // subnormal range: m * 2^-9, m <= 8
+  const uint32_t mant = u & 0x7FFFFFu;
+  uint32_t code = (uint32_t(e + 7) << 3) | (mant >> 20);
+  const uint32_t rem = mant & 0xFFFFFu;
+  if (rem > 0x80000u || (rem == 0x80000u && (code & 1u))) code += 1u;
+  return code > 0x7Eu ? 0x7Eu : code;
+}
+QS_DEV float ue4m3_decode(uint32_t c) {
+  const uint32_t e = c >> 3, m = c & 7u;
+  if (e == 0u) return float(m) * 0.001953125f;
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// Pack one group of 16 float32 values; returns the scale code and writes 8 code bytes.
+QS_DEV uint32_t nvfp4_pack16(const float (&x)[16], float g, uint32_t (&packed)[2]) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
+  const float sf = __fdiv_rn(a, __fmul_rn(6.0f, g));
+  const uint32_t sc = ue4m3_encode(sf);
+  const float sv = ue4m3_decode(sc);
+  packed[0] = packed[1] = 0u;
+  if (sv > 0.0f) {
+    const float den = __fmul_rn(sv, g);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t c = e2m1_encode(__fdiv_rn(x[i], den));
+      packed[i >> 3] |= c << (4 * (i & 7));
+    }
+  }
+  return sc;
+}
+
+// ============================================================ shared helpers
+// Resolve the cache slot of token t of sequence b; false (and an error flag) if invalid.
+QS_DEV bool cache_slot(const int32_t* page_table, int b, int t, int mpps, int num_pages,
+                       int max_context, uint32_t* hdr, uint32_t kid, int& page, int& slot) {
+  const int pi = t / kPage;
+  if (t < 0 || t >= max_context || pi >= mpps) {
+    flag_error(hdr, QS_ERR_DEVICE_BOUNDS, kid, uint32_t(b));
+    return false;
+  }
+  page = page_table[size_t(b) * mpps + pi];
+  if (page < 0 || page >= num_pages) {
+    flag_error(hdr, QS_ERR_DEVICE_BOUNDS, kid, uint32_t(b));
+    return false;
+  }
+  slot = t % kPage;
+  return true;
+}
+
+// Scoring prep of one row: qbar = (sum of the group's query heads) / G, q~ = qbar . P[g].
+// Uses smem scratch of d floats; P read from global (it is small and L2-resident).
+QS_DEV void row_prep(const uint16_t* q, const float* Pg, float* qt_row, float* qbar_s, int b,
+                     int g, int Hkv, int G, int d, int r) {
+  const int Hq = Hkv * G;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float s = 0.0f;
+    for (int h = 0; h < G; ++h) s += bf16_to_f32(q[(size_t(b) * Hq + g * G + h) * d + i]);
+    qbar_s[i] = s / float(G);
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < r; j += blockDim.x) {
+    float acc = 0.0f;
+    for (int i = 0; i < d; ++i) acc = fmaf(qbar_s[i], Pg[i * r + j], acc);
+    qt_row[j] = acc;
+  }
+}
+
+// Advance seq_lens once every CTA of the append grid has read them ("last CTA" pattern).
+QS_DEV void finish_append(const AppendParams& a) {
+  __shared__ int s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned total = gridDim.x * gridDim.y;
+    const unsigned prev = atomicAdd(a.hdr + kCtrAppend, 1u);
+    s_last = (prev == total - 1u);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int b = threadIdx.x; b < a.batch; b += blockDim.x) {
+    int n = a.n_new ? a.n_new[b] : 1;
+    if (n < 0 || n > a.max_new) n = 0;
+    a.seq_lens[b] += n;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    a.hdr[kCtrAppend] = 0u;
+    __threadfence();
+  }
+}
+
+// ============================================================ rank-r writer
+// CTA = one row (b, g) x TT tokens. Thread (tg, og) computes a 4-token x 4-output
+// micro-tile, so each k_i / P_ij loaded from shared memory feeds 4 products.
+template <typename PT, int R, int D>
+__global__ void __launch_bounds__(64 * R / 16)
+append_rankr_kernel(const AppendParams a) {
+  constexpr int TT = 64;
+  constexpr int NT = TT * R / 16;
+  constexpr int OG = R / 4;          // output groups of 4
+  extern __shared__ __align__(16) float smem[];
+  float* Ps = smem;                  // [D][R]
+  float* kT = smem + D * R;          // [D][TT] keys as float, token-minor
+  __shared__ int s_page[TT], s_slot[TT];
+
+  const int row = blockIdx.y;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  int n_b = a.n_new ? a.n_new[b] : 1;
+  if (n_b < 0 || n_b > a.max_new) {
+    if (threadIdx.x == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_APPEND, uint32_t(b));
+    n_b = 0;
+  }
+  const int old = a.seq_lens[b];
+  const int t0 = blockIdx.x * TT;
+  const int cnt = min(TT, n_b - t0);
+  const bool prep = (a.q != nullptr) && blockIdx.x == 0;
+
+  if (cnt > 0 || prep) {
+    const float* Pg = a.P + size_t(g) * D * R;
+    for (int i = threadIdx.x; i < D * R / 4; i += NT)
+      reinterpret_cast<float4*>(Ps)[i] = reinterpret_cast<const float4*>(Pg)[i];
+  }
+  if (cnt > 0) {
+    if (threadIdx.x < TT) {
+      int page = -1, slot = 0;
+      if (int(threadIdx.x) < cnt)
+        cache_slot(a.page_table, b, old + t0 + threadIdx.x, a.max_pages_per_seq, a.num_pages,
+                   a.max_context, a.hdr, KID_APPEND, page, slot);
+      s_page[threadIdx.x] = page;
+      s_slot[threadIdx.x] = slot;
+    }
+    // keys -> smem (transposed, float) and K/V rows -> cache, 16 bytes per thread-step
+    constexpr int CH = D / 8;  // 16-byte chunks per row
+    for (int it = threadIdx.x; it < TT * CH; it += NT) {
+      const int n = it / CH, c = it % CH;
+      if (n < cnt) {
+        const size_t src = ((size_t(b) * a.Hkv + g) * a.max_new + t0 + n) * D + c * 8;
+        const uint4 kv = *reinterpret_cast<const uint4*>(a.k_new + src);
+        const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          kT[(c * 8 + 2 * e) * TT + n] = bf16_lo(w[e]);
+          kT[(c * 8 + 2 * e + 1) * TT + n] = bf16_hi(w[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kT[(c * 8 + e) * TT + n] = 0.0f;
+      }
+    }
+    __syncthreads();
+    for (int it = threadIdx.x; it < cnt * CH; it += NT) {
+      const int n = it / CH, c = it % CH;
+      const int page = s_page[n];
+      if (page < 0) continue;
+      const size_t src = ((size_t(b) * a.Hkv + g) * a.max_new + t0 + n) * D + c * 8;
+      const size_t dst = ((size_t(page) * a.Hkv + g) * kPage + s_slot[n]) * D + c * 8;
+      *reinterpret_cast<uint4*>(a.k + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+      *reinterpret_cast<uint4*>(a.v + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+    }
+    // projected keys: ascending i, separate float32 roundings for product and sum
+    const int tg = threadIdx.x / OG, og = threadIdx.x % OG;
+    float acc[4][4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = 0.0f;
+#pragma unroll 4
+    for (int i = 0; i < D; ++i) {
+      const float4 kk = *reinterpret_cast<const float4*>(kT + i * TT + tg * 4);
+      const float4 pp = *reinterpret_cast<const float4*>(Ps + i * R + og * 4);
+      const float kx[4] = {kk.x, kk.y, kk.z, kk.w};
+      const float px[4] = {pp.x, pp.y, pp.z, pp.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = __fadd_rn(acc[x][y], __fmul_rn(kx[x], px[y]));
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int n = tg * 4 + x;
+      if (n >= cnt) continue;
+      const int page = s_page[n];
+      if (page < 0) continue;
+      const size_t base = ((size_t(page) * a.Hkv + g) * kPage + s_slot[n]) * R + og * 4;
+      if constexpr (sizeof(PT) == 4) {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.proxy) + base) =
+            make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+      } else {
+        const uint32_t lo = uint32_t(f32_to_bf16_rn(acc[x][0])) |
+                            (uint32_t(f32_to_bf16_rn(acc[x][1])) << 16);
+        const uint32_t hi = uint32_t(f32_to_bf16_rn(acc[x][2])) |
+                            (uint32_t(f32_to_bf16_rn(acc[x][3])) << 16);
+        *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.proxy) + base) =
+            make_uint2(lo, hi);
+      }
+    }
+  }
+  if (prep) {
+    __syncthreads();
+    float* qbar = kT;  // reuse (the keys are no longer needed)
+    const int Hq = a.Hkv * a.G;
+    for (int i = threadIdx.x; i < D; i += NT) {
+      float s = 0.0f;
+      for (int h = 0; h < a.G; ++h) s += bf16_to_f32(a.q[(size_t(b) * Hq + g * a.G + h) * D + i]);
+      qbar[i] = s / float(a.G);
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < R; j += NT) {
+      float acc = 0.0f;
+      for (int i = 0; i < D; ++i) acc = fmaf(qbar[i], Ps[i * R + j], acc);
+      a.qt[size_t(row) * R + j] = acc;
+    }
+  }
+  finish_append(a);
+}
+
+// ============================================================ NVFP4 writer
+// CTA = one row x 64 tokens; thread = (token, 16-element group).
+__global__ void __launch_bounds__(128) append_nvfp4_kernel(const AppendParams a) {
+  constexpr int TT = 64, D = 128, GR = D / 16;
+  __shared__ int s_page[TT], s_slot[TT];
+  __shared__ float s_mu[D];
+  const int row = blockIdx.y;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  int n_b = a.n_new ? a.n_new[b] : 1;
+  if (n_b < 0 || n_b > a.max_new) {
+    if (threadIdx.x == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_APPEND, uint32_t(b));
+    n_b = 0;
+  }
+  const int old = a.seq_lens[b];
+  const int t0 = blockIdx.x * TT;
+  const int cnt = min(TT, n_b - t0);
+  if (cnt > 0) {
+    const float gk = *a.key_gscale;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) s_mu[i] = a.key_center[size_t(row) * D + i];
+    if (threadIdx.x < TT) {
+      int page = -1, slot = 0;
+      if (int(threadIdx.x) < cnt)
+        cache_slot(a.page_table, b, old + t0 + threadIdx.x, a.max_pages_per_seq, a.num_pages,
+                   a.max_context, a.hdr, KID_APPEND, page, slot);
+      s_page[threadIdx.x] = page;
+      s_slot[threadIdx.x] = slot;
+    }
+    __syncthreads();
+    // K/V rows to the cache
+    constexpr int CH = D / 8;
+    for (int it = threadIdx.x; it < cnt * CH; it += blockDim.x) {
+      const int n = it / CH, c = it % CH;
+      const int page = s_page[n];
+      if (page < 0) continue;
+      const size_t src = ((size_t(b) * a.Hkv + g) * a.max_new + t0 + n) * D + c * 8;
+      const size_t dst = ((size_t(page) * a.Hkv + g) * kPage + s_slot[n]) * D + c * 8;
+      *reinterpret_cast<uint4*>(a.k + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+      *reinterpret_cast<uint4*>(a.v + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+    }
+    // centre and pack
+    for (int it = threadIdx.x; it < cnt * GR; it += blockDim.x) {
+      const int n = it / GR, gr = it % GR;
+      const int page = s_page[n];
+      if (page < 0) continue;
+      const size_t src = ((size_t(b) * a.Hkv + g) * a.max_new + t0 + n) * D + gr * 16;
+      const uint4 k0 = *reinterpret_cast<const uint4*>(a.k_new + src);
+      const uint4 k1 = *reinterpret_cast<const uint4*>(a.k_new + src + 8);
+      const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+      float x[16];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        x[2 * e] = __fsub_rn(bf16_lo(w[e]), s_mu[gr * 16 + 2 * e]);
+        x[2 * e + 1] = __fsub_rn(bf16_hi(w[e]), s_mu[gr * 16 + 2 * e + 1]);
+      }
+      uint32_t packed[2];
+      const uint32_t sc = nvfp4_pack16(x, gk, packed);
+      const size_t tok = (size_t(page) * a.Hkv + g) * kPage + s_slot[n];
+      *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(a.proxy) + tok * (D / 2) + gr * 8) =
+          make_uint2(packed[0], packed[1]);
+      a.proxy_scale[tok * GR + gr] = uint8_t(sc);
+    }
+  }
+  finish_append(a);
+}
+
+// ============================================================ NVFP4 block error
+// CTA = one (row, block) pair that this append may have completed. Thread = token; the
+// squared errors are reduced in a fixed order (deterministic float32 result).
+__global__ void __launch_bounds__(128) block_err_kernel(const BlockErrParams a) {
+  constexpr int D = 128, GR = D / 16;
+  __shared__ float s_mu[D];
+  __shared__ float s_red[4];
+  const int row = blockIdx.y;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  int n_b = a.n_new ? a.n_new[b] : 1;
+  const int new_len = a.seq_lens[b];
+  const int old = new_len - n_b;
+  const int j = old / a.S + blockIdx.x;
+  if (n_b <= 0 || old < 0 || (j + 1) * a.S > new_len || j >= a.nb_stride) return;  // not completed here
+  const float gk = *a.key_gscale;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) s_mu[i] = a.key_center[size_t(row) * D + i];
+  __syncthreads();
+  float err = 0.0f;
+  for (int tt = threadIdx.x; tt < a.S; tt += blockDim.x) {
+    const int t = j * a.S + tt;
+    const int pi = t / kPage;
+    if (pi >= a.max_pages_per_seq) { flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_BLOCKERR, b); continue; }
+    const int page = a.page_table[size_t(b) * a.max_pages_per_seq + pi];
+    if (page < 0 || page >= a.num_pages) { flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_BLOCKERR, b); continue; }
+    const uint16_t* kr = a.k + ((size_t(page) * a.Hkv + g) * kPage + t % kPage) * D;
+    float e_tok = 0.0f;
+#pragma unroll 1
+    for (int gr = 0; gr < GR; ++gr) {
+      const uint4 k0 = *reinterpret_cast<const uint4*>(kr + gr * 16);
+      const uint4 k1 = *reinterpret_cast<const uint4*>(kr + gr * 16 + 8);
+      const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+      float x[16];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        x[2 * e] = __fsub_rn(bf16_lo(w[e]), s_mu[gr * 16 + 2 * e]);
+        x[2 * e + 1] = __fsub_rn(bf16_hi(w[e]), s_mu[gr * 16 + 2 * e + 1]);
+      }
+      uint32_t packed[2];
+      const float sv = ue4m3_decode(nvfp4_pack16(x, gk, packed));
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float dq = __fmul_rn(__fmul_rn(e2m1_decode((packed[i >> 3] >> (4 * (i & 7))) & 15u), sv), gk);
+        const float df = __fsub_rn(x[i], dq);
+        e_tok = __fadd_rn(e_tok, __fmul_rn(df, df));
+      }
+    }
+    err = __fadd_rn(err, e_tok);
+  }
+  // fixed-order reduction: warp butterfly then warps in index order
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) err += __shfl_xor_sync(kFull, err, m);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = err;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.0f;
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) tot += s_red[w];
+    a.block_err[size_t(row) * a.nb_stride + j] = tot;
+  }
+}
+
+// ============================================================ scoring prep
+__global__ void __launch_bounds__(128) prep_rankr_kernel(const PrepParams a) {
+  __shared__ float qbar[256];
+  const int row = blockIdx.x;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  row_prep(a.q, a.P + size_t(g) * a.d * a.r, a.qt + size_t(row) * a.r, qbar, b, g, a.Hkv, a.G,
+           a.d, a.r);
+}
+
+// NVFP4 query packing: one CTA; g_q = max|q| / 2688 over the whole q tensor, then every
+// head's query is packed like the keys (without centring).
+__global__ void __launch_bounds__(1024) qpack_kernel(const QPackParams a) {
+  __shared__ float s_red[32];
+  __shared__ float s_g;
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < a.n; i += blockDim.x) m = fmaxf(m, fabsf(bf16_to_f32(a.q[i])));
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? s_red[threadIdx.x] : 0.0f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) {
+      s_g = __fdiv_rn(v, 2688.0f);
+      *a.gscale = s_g;
+    }
+  }
+  __syncthreads();
+  const float gq = s_g;
+  for (int grp = threadIdx.x; grp < a.n / 16; grp += blockDim.x) {
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = bf16_to_f32(a.q[size_t(grp) * 16 + i]);
+    uint32_t packed[2];
+    const uint32_t sc = nvfp4_pack16(x, gq, packed);
+    *reinterpret_cast<uint2*>(a.codes + size_t(grp) * 8) = make_uint2(packed[0], packed[1]);
+    a.scales[grp] = uint8_t(sc);
+  }
+}
+
+// ============================================================ launchers
+template <typename PT, int R, int D>
+static cudaError_t launch_rankr(const Plan& p, const AppendParams& a, cudaStream_t s) {
+  constexpr int NT = 64 * R / 16;
+  const size_t smem = size_t(D) * R * 4 + size_t(D) * 64 * 4;
+  auto k = append_rankr_kernel<PT, R, D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.max_new + 63) / 64, a.batch * a.Hkv);
+  k<<<grid, NT, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) {
+  if (p.r == 0) {
+    dim3 grid((a.max_new + 63) / 64, a.batch * a.Hkv);
+    append_nvfp4_kernel<<<grid, 128, 0, s>>>(a);
+    return cudaGetLastError();
+  }
+  const bool f32 = p.proxy_dtype == QS_F32;
+  if (p.d == 64) {
+    if (f32 && p.r == 16) return launch_rankr<float, 16, 64>(p, a, s);
+    if (!f32 && p.r == 32) return launch_rankr<uint16_t, 32, 64>(p, a, s);
+  } else {
+    if (f32 && p.r == 16) return launch_rankr<float, 16, 128>(p, a, s);
+    if (f32 && p.r == 32) return launch_rankr<float, 32, 128>(p, a, s);
+    if (!f32 && p.r == 32) return launch_rankr<uint16_t, 32, 128>(p, a, s);
+    if (!f32 && p.r == 64) return launch_rankr<uint16_t, 64, 128>(p, a, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_block_err(const Plan& p, const BlockErrParams& a, cudaStream_t s) {
+  dim3 grid(a.max_blocks_per_call, a.batch * a.Hkv);
+  block_err_kernel<<<grid, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s) {
+  prep_rankr_kernel<<<a.batch * a.Hkv, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s) {
+  qpack_kernel<<<1, 1024, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace qs

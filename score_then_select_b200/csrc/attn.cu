@@ -1,0 +1,313 @@
+// attn.cu - split-K sparse attention over the selected blocks, and the LSE combine.
+//
+// "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 1 and
+// Abstract: gather-free indexed attention reads the original full-dimensional keys and
+// values of the selected positions straight from the standard GQA paged cache, with a
+// distinct selection per KV head shared by that head's query heads.
+// "Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse Attention", Full
+// text: value aggregation in FP16 with FP32 accumulation over contiguous block tiles.
+//
+// CTA = (row, split): the split's slice of the row's selected token slots is streamed in
+// 64-token tiles (K and V, 16-byte cp.async into an XOR-swizzled 3-stage ring); each of
+// the 4 warps owns 16 tokens of a tile and keeps its own online-softmax state.
+//
+// Tensor-core mapping (mma.m16n8k16, FP32 accumulate), transposed so that the group's
+// <= 8 query heads fill the N = 8 side:
+//   S^T[16 tok x 8 heads]  = K[16 tok x d] . Q^T[d x 8 heads]      (A = K via ldmatrix)
+//   O^T[d x 8 heads]      += V^T[d x 16 tok] . P^T[16 tok x 8 heads] (A = V via ldmatrix.trans,
+//                                                                    B = P via movmatrix)
+// Each warp's partial (max, sum, o) is merged across warps in shared memory and written
+// as one split partial; the combine kernel merges splits by log-sum-exp. Scores are kept
+// in base 2 (scale * log2 e folded into the logits).
+#include "qs_device.cuh"
+
+namespace qs {
+
+constexpr int kTileT = 64;
+constexpr int kAttnStages = 3;
+constexpr int kMaxTokensPerSplit = 2048;
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kTileBytes = kTileT * kRowBytes;          // one of K or V
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kRingBytes = kAttnStages * kStageBytes;
+  static constexpr int kRowsOff = kRingBytes;                    // int32 [kMaxTokensPerSplit]
+  static constexpr int kTotal = kRowsOff + kMaxTokensPerSplit * 4;
+};
+
+// byte offset of (token row r, 16-byte chunk c) inside a swizzled tile
+template <int D>
+QS_DEV uint32_t swz(int r, int c) {
+  return uint32_t(r * (D * 2) + ((c ^ (r & 7)) << 4));
+}
+
+template <int D, bool V_F16, bool AGG_F16>
+__global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
+  using SM = AttnSmem<D>;
+  constexpr int KS = D / 16;       // k-steps over the head dimension
+  constexpr int CH = D / 8;        // 16-byte chunks per row
+  extern __shared__ __align__(128) uint8_t smem[];
+  int* s_rows = reinterpret_cast<int*>(smem + SM::kRowsOff);
+
+  const int split = blockIdx.x, row = blockIdx.y;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  const int Hq = a.Hkv * a.G;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  int n = a.n_sel[row];
+  int L = a.seq_lens[b];
+  if (n < 0 || n > a.budget || L < 0) {
+    if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
+    n = 0;
+  }
+  const int slots = n * a.S;
+  const int s0 = split * a.tokens_per_split;
+  const int s1 = min(s0 + a.tokens_per_split, slots);
+  const int cnt = s1 - s0;
+
+  // ---------------- token table of this split: cache row index or -1
+  for (int i = tid; i < a.tokens_per_split; i += 128) {
+    int r = -1;
+    if (i < cnt) {
+      const int gs = s0 + i;
+      const int blk = a.sel[size_t(row) * a.budget + gs / a.S];
+      const int nbr = (L + a.S - 1) / a.S;
+      if (blk >= nbr) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
+      const int t = (blk >= 0 && blk < nbr) ? blk * a.S + gs % a.S : L;
+      if (t < L) {
+        const int pi = t / kPage;
+        const int page = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
+        if (page >= 0 && page < a.num_pages) r = (page * a.Hkv + g) * kPage + (t % kPage);
+        else flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
+      }
+    }
+    s_rows[i] = r;
+  }
+
+  // ---------------- query fragments (B operand of S^T): head = lane/4, dims 2*(lane%4)+{0,1}
+  uint32_t qb[KS][2];
+  {
+    const int h = lane >> 2;
+    const uint16_t* qr = a.q + (size_t(b) * Hq + g * a.G + (h < a.G ? h : 0)) * D;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int d0 = ks * 16 + 2 * (lane & 3);
+      qb[ks][0] = h < a.G ? *reinterpret_cast<const uint32_t*>(qr + d0) : 0u;
+      qb[ks][1] = h < a.G ? *reinterpret_cast<const uint32_t*>(qr + d0 + 8) : 0u;
+    }
+  }
+  __syncthreads();
+
+  const int tiles = (cnt + kTileT - 1) / kTileT;
+  const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k);
+  const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v);
+
+  auto issue = [&](int tile) {
+    if (tile < tiles) {
+      uint8_t* st = smem + (tile % kAttnStages) * SM::kStageBytes;
+#pragma unroll
+      for (int it = 0; it < kTileT * CH / 128; ++it) {
+        const int idx = it * 128 + tid;
+        const int r = idx / CH, c = idx % CH;
+        const int cr = s_rows[tile * kTileT + r];
+        const size_t off = size_t(cr < 0 ? 0 : cr) * (D * 2) + c * 16;
+        cp_async16_zfill(st + swz<D>(r, c), kbase + off, cr >= 0);
+        cp_async16_zfill(st + SM::kTileBytes + swz<D>(r, c), vbase + off, cr >= 0);
+      }
+    }
+    cp_async_commit();
+  };
+
+  // online-softmax state for heads h0 = 2*(lane%4), h1 = h0 + 1 (replicated across lanes
+  // with equal lane%4); l is this lane's partial sum over its own tokens
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
+  float o[KS][4];
+#pragma unroll
+  for (int m = 0; m < KS; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.0f;
+
+  issue(0);
+  issue(1);
+  for (int tile = 0; tile < tiles; ++tile) {
+    cp_async_wait<1>();
+    __syncthreads();
+    issue(tile + 2);
+    const uint8_t* st = smem + (tile % kAttnStages) * SM::kStageBytes;
+    const uint32_t kst = smem_u32(st), vst = smem_u32(st + SM::kTileBytes);
+
+    // S^T = K Q^T for this warp's 16 tokens
+    float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(a0, a1, a2, a3, kst + swz<D>(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
+      mma_bf16(c, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+    }
+    const int tl = tile * kTileT + warp * 16 + (lane >> 2);
+    const bool v0 = s_rows[tl] >= 0, v1 = s_rows[tl + 8] >= 0;
+    float x0 = v0 ? c[0] * a.scale_log2 : -INFINITY;
+    float x1 = v0 ? c[1] * a.scale_log2 : -INFINITY;
+    float x2 = v1 ? c[2] * a.scale_log2 : -INFINITY;
+    float x3 = v1 ? c[3] * a.scale_log2 : -INFINITY;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o2));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
+    const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
+    const float al0 = ex2(m0 - base0), al1 = ex2(m1 - base1);
+    m0 = mn0;
+    m1 = mn1;
+    const float p0 = ex2(x0 - base0), p1 = ex2(x1 - base1);
+    const float p2 = ex2(x2 - base0), p3 = ex2(x3 - base1);
+    l0 = l0 * al0 + p0 + p2;
+    l1 = l1 * al1 + p1 + p3;
+#pragma unroll
+    for (int m = 0; m < KS; ++m) {
+      o[m][0] *= al0;
+      o[m][1] *= al1;
+      o[m][2] *= al0;
+      o[m][3] *= al1;
+    }
+    // P^T as the B operand: transpose the two 8x8 (token x head) quadrants
+    uint32_t pb0, pb1;
+    if constexpr (AGG_F16) {
+      pb0 = movmatrix_t(pack_f16x2(p0, p1));
+      pb1 = movmatrix_t(pack_f16x2(p2, p3));
+    } else {
+      pb0 = movmatrix_t(pack_bf16x2(p0, p1));
+      pb1 = movmatrix_t(pack_bf16x2(p2, p3));
+    }
+    // O^T += V^T P^T over the head dimension
+#pragma unroll
+    for (int m = 0; m < KS; ++m) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_t(a0, a1, a2, a3,
+                vst + swz<D>(warp * 16 + (lane & 7) + ((lane >> 4) << 3), m * 2 + ((lane >> 3) & 1)));
+      if constexpr (AGG_F16) {
+        if constexpr (!V_F16) {
+          a0 = bf16x2_to_f16x2(a0);
+          a1 = bf16x2_to_f16x2(a1);
+          a2 = bf16x2_to_f16x2(a2);
+          a3 = bf16x2_to_f16x2(a3);
+        }
+        mma_f16(o[m], a0, a1, a2, a3, pb0, pb1);
+      } else {
+        mma_bf16(o[m], a0, a1, a2, a3, pb0, pb1);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // ---------------- merge the 4 warps' states, write this split's partial
+#pragma unroll
+  for (int o2 = 4; o2 < 32; o2 <<= 1) {
+    l0 += __shfl_xor_sync(kFull, l0, o2);
+    l1 += __shfl_xor_sync(kFull, l1, o2);
+  }
+  float* s_m = reinterpret_cast<float*>(smem);          // [4][8]
+  float* s_l = s_m + 32;                                // [4][8]
+  float* s_o = s_l + 32;                                // [4][8][D]
+  if (lane < 4) {
+    s_m[warp * 8 + 2 * lane] = m0;
+    s_m[warp * 8 + 2 * lane + 1] = m1;
+    s_l[warp * 8 + 2 * lane] = l0;
+    s_l[warp * 8 + 2 * lane + 1] = l1;
+  }
+  {
+    const int h0 = 2 * (lane & 3);
+#pragma unroll
+    for (int m = 0; m < KS; ++m) {
+      const int d0 = m * 16 + (lane >> 2);
+      float* ow = s_o + warp * 8 * D;
+      ow[h0 * D + d0] = o[m][0];
+      ow[(h0 + 1) * D + d0] = o[m][1];
+      ow[h0 * D + d0 + 8] = o[m][2];
+      ow[(h0 + 1) * D + d0 + 8] = o[m][3];
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < a.G * D; idx += 128) {
+    const int h = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w * 8 + h]);
+    const float base = M == -INFINITY ? 0.0f : M;
+    float lsum = 0.0f, osum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float wt = ex2(s_m[w * 8 + h] - base);
+      lsum += wt * s_l[w * 8 + h];
+      osum += wt * s_o[(w * 8 + h) * D + d];
+    }
+    const size_t rq = size_t(b) * Hq + g * a.G + h;
+    const size_t pidx = rq * a.splits + split;
+    a.part_o[pidx * D + d] = osum;
+    if (d == 0) {
+      a.part_ml[pidx * 2] = M;
+      a.part_ml[pidx * 2 + 1] = lsum;
+    }
+  }
+}
+
+// out[h][d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s; rows with no tokens -> 0
+__global__ void combine_kernel(const CombineParams a) {
+  const int rq = blockIdx.x;
+  const float* ml = a.part_ml + size_t(rq) * a.splits * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < a.splits; ++s)
+    if (ml[2 * s + 1] > 0.0f) M = fmaxf(M, ml[2 * s]);
+  for (int d = threadIdx.x; d < a.d; d += blockDim.x) {
+    float num = 0.0f, den = 0.0f;
+    for (int s = 0; s < a.splits; ++s) {
+      const float l = ml[2 * s + 1];
+      if (!(l > 0.0f)) continue;
+      const float w = ex2(ml[2 * s] - M);
+      den += w * l;
+      num += w * a.part_o[(size_t(rq) * a.splits + s) * a.d + d];
+    }
+    const float r = den > 0.0f ? num / den : 0.0f;
+    if (a.out_bf16)
+      reinterpret_cast<uint16_t*>(a.out)[size_t(rq) * a.d + d] = f32_to_bf16_rn(r);
+    else
+      reinterpret_cast<float*>(a.out)[size_t(rq) * a.d + d] = r;
+  }
+}
+
+template <int D, bool VF, bool AF>
+static cudaError_t launch_attn_t(const AttnParams& a, cudaStream_t s) {
+  auto k = attn_kernel<D, VF, AF>;
+  const int smem = AttnSmem<D>::kTotal;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.splits, a.batch * a.Hkv);
+  k<<<grid, 128, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s) {
+  const bool vf = p.v_dtype == QS_F16, af = p.v_agg_dtype == QS_F16;
+  if (p.d == 128) {
+    if (vf) return launch_attn_t<128, true, true>(a, s);
+    if (af) return launch_attn_t<128, false, true>(a, s);
+    return launch_attn_t<128, false, false>(a, s);
+  }
+  if (p.d == 64) {
+    if (vf) return launch_attn_t<64, true, true>(a, s);
+    if (af) return launch_attn_t<64, false, true>(a, s);
+    return launch_attn_t<64, false, false>(a, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_combine(const Plan& p, const CombineParams& a, cudaStream_t s) {
+  combine_kernel<<<a.rows_q, a.d, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace qs

@@ -1,0 +1,164 @@
+// qs_internal.h - parameter blocks and launchers shared by the libqs translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/qs.h"
+
+namespace qs {
+
+// kernel ids recorded with device-side errors (documented in qs.h)
+enum KernelId : uint32_t {
+  KID_APPEND = 1,
+  KID_BLOCKERR = 2,
+  KID_PREP = 3,
+  KID_SCORE = 4,
+  KID_SELECT = 5,
+  KID_ATTN = 6,
+  KID_COMBINE = 7
+};
+
+constexpr int kPage = 128;          // tokens per page (the only page size built)
+constexpr int kMaxBatch = 1024;     // sequences per call
+constexpr int kMaxGroup = 8;        // query heads per KV head
+constexpr int kMaxSelectBlocks = 32768;
+constexpr int kHdrWords = 64;       // workspace header (256 bytes)
+constexpr int kCtrAppend = 16;      // header word: append "last CTA" counter
+
+// Workspace carve-up (byte offsets); computed identically by qs_workspace_size and calls.
+struct WsLayout {
+  size_t qt = 0;        // rank r: q~ [batch][Hkv][r] f32
+  size_t qcodes = 0;    // NVFP4: packed q codes [batch][Hq][d/2] u8
+  size_t qscales = 0;   // NVFP4: q scales [batch][Hq][d/16] u8
+  size_t qgscale = 0;   // NVFP4: g_q (1 float)
+  size_t scores = 0;    // [batch][Hkv][nb_stride] f32
+  size_t sel = 0;       // [batch][Hkv][budget] i32
+  size_t nsel = 0;      // [batch][Hkv] i32
+  size_t part_ml = 0;   // [batch][Hq][splits][2] f32
+  size_t part_o = 0;    // [batch][Hq][splits][d] f32
+  size_t total = 0;
+  int nb_stride = 0;
+  int splits = 0;       // attention splits per row
+  int tokens_per_split = 0;
+};
+
+struct Plan {
+  int batch, Hq, Hkv, G, d, S, budget, r, nb_stride;
+  int proxy_dtype, v_dtype, v_agg_dtype, out_dtype;
+  int force_sink, force_last, n_keep;
+  float scale;
+  WsLayout ws;
+};
+
+// ------------------------------------------------------------ kernel parameter blocks
+struct AppendParams {
+  const uint16_t* k_new;   // [batch][Hkv][max_new][d]
+  const uint16_t* v_new;
+  const int32_t* n_new;    // [batch] or nullptr (=> 1 token each)
+  const float* P;          // [Hkv][d][r]
+  uint16_t* k;             // cache pages
+  uint16_t* v;
+  void* proxy;
+  uint8_t* proxy_scale;
+  const float* key_center;
+  const float* key_gscale;
+  const int32_t* page_table;
+  int32_t* seq_lens;
+  uint32_t* hdr;
+  // fused scoring prep (rank r): q~ of each row, or nullptr
+  const uint16_t* q;
+  float* qt;
+  int batch, Hkv, G, d, r, max_new, max_pages_per_seq, num_pages, max_context;
+};
+
+struct BlockErrParams {
+  const uint16_t* k;
+  const float* key_center;
+  const float* key_gscale;
+  const int32_t* page_table;
+  const int32_t* seq_lens;  // already advanced
+  const int32_t* n_new;     // [batch] or nullptr (=> 1)
+  float* block_err;
+  uint32_t* hdr;
+  int batch, Hkv, d, S, nb_stride, max_pages_per_seq, num_pages, max_blocks_per_call;
+};
+
+struct PrepParams {          // rank r scoring prep (standalone qs_score)
+  const uint16_t* q;
+  const float* P;
+  float* qt;
+  int batch, Hkv, G, d, r;
+};
+
+struct QPackParams {         // NVFP4 query packing
+  const uint16_t* q;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* gscale;
+  int n;                     // batch * Hq * d
+  int d;
+};
+
+struct ScoreParams {
+  const void* proxy;
+  const uint8_t* proxy_scale;
+  const float* qt;           // rank r: [batch][Hkv][r]
+  const uint8_t* qcodes;     // NVFP4
+  const uint8_t* qscales;
+  const float* qgscale;
+  const float* key_gscale;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  float* scores;
+  uint32_t* hdr;
+  int batch, Hkv, G, d, S, nb_stride, max_pages_per_seq, num_pages, max_context;
+};
+
+struct SelectParams {
+  const float* scores;
+  const float* block_err;    // NVFP4 kept blocks, or nullptr
+  const int32_t* seq_lens;
+  int32_t* sel;
+  int32_t* n_sel;
+  uint32_t* hdr;
+  int rows, Hkv, S, nb_stride, budget, force_sink, force_last, n_keep;
+};
+
+struct AttnParams {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* sel;
+  const int32_t* n_sel;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  float* part_ml;
+  float* part_o;
+  uint32_t* hdr;
+  int batch, Hkv, G, S, budget, splits, tokens_per_split, max_pages_per_seq, num_pages;
+  float scale_log2;          // softmax scale * log2(e)
+};
+
+struct CombineParams {
+  const float* part_ml;
+  const float* part_o;
+  void* out;
+  int rows_q;                // batch * Hq
+  int splits, d, out_bf16;
+};
+
+// ------------------------------------------------------------ launchers (return launch error)
+cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s);
+cudaError_t launch_block_err(const Plan& p, const BlockErrParams& a, cudaStream_t s);
+cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s);
+cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s);
+cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s);
+cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s);
+cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s);
+cudaError_t launch_combine(const Plan& p, const CombineParams& a, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace qs

@@ -1,0 +1,321 @@
+// select.cu - per-row top-k block selection.
+//
+// "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 1 and
+// Table 15: each KV head selects its own top-B positions, shared by its query heads.
+// "Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse Attention", Full text:
+// blocks kept at full precision are always attended.
+//
+// Result (deterministic): if nb <= k every block; otherwise the forced set F (sink, last,
+// kept) plus the k - |F| best other blocks by score, equal scores ordered by lower index;
+// ascending.
+//
+// Algorithm, one CTA per row, each thread owning ITEMS consecutive blocks in registers:
+//   1. forced blocks are marked (the kept blocks are the n_keep complete blocks with the
+//      largest block error, found by two block-wide arg-max reductions);
+//   2. one pass of a 2048-bin histogram that is linear in the score between the active
+//      minimum and maximum (a monotone map, so every block in a higher bin scores higher)
+//      selects every bin above the threshold bin and leaves only the threshold bin active;
+//   3. an exact MSB-first radix select (4 x 8-bit digits) over order-preserving uint32
+//      keys of the remaining active blocks narrows them to one key value;
+//   4. the remaining slots go to the lowest-indexed blocks holding that key;
+//   5. a block-wide scan over the per-thread counts writes the ascending indices.
+#include <cfloat>
+
+#include "qs_device.cuh"
+
+namespace qs {
+
+constexpr int kLinBins = 2048;
+
+// float -> uint32 whose unsigned order is the float order (NaN ranks as -FLT_MAX, -0 == +0)
+QS_DEV uint32_t order_key(float v) {
+  if (v != v) v = -FLT_MAX;
+  if (v == 0.0f) v = 0.0f;
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int NT>
+struct BlockOps {
+  static constexpr int NW = NT / 32;
+  int* s_i;      // [NW + 1]
+  float* s_f;    // [2 * NW]
+
+  // exclusive prefix sum over threads; total via *total
+  QS_DEV int exclusive_sum(int v, int* total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_i[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int t = lane < NW ? s_i[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, t, o);
+        if (lane >= o) t += y;
+      }
+      if (lane < NW) s_i[lane] = t;              // inclusive warp totals
+      if (lane == NW - 1) s_i[NW] = t;
+    }
+    __syncthreads();
+    const int before = (w == 0 ? 0 : s_i[w - 1]) + x - v;
+    *total = s_i[NW];
+    __syncthreads();
+    return before;
+  }
+  QS_DEV int sum(int v) {
+    int t;
+    exclusive_sum(v, &t);
+    return t;
+  }
+  QS_DEV void minmax(float& lo, float& hi) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    lo = warp_min(lo);
+    hi = warp_max(hi);
+    if (lane == 0) { s_f[w] = lo; s_f[NW + w] = hi; }
+    __syncthreads();
+    lo = s_f[0];
+    hi = s_f[NW];
+    for (int i = 1; i < NW; ++i) { lo = fminf(lo, s_f[i]); hi = fmaxf(hi, s_f[NW + i]); }
+    __syncthreads();
+  }
+  // arg-max of (value, -index) over the CTA; returns the index (or -1 if none valid)
+  QS_DEV int argmax(float v, int idx) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    unsigned long long key = idx < 0 ? 0ull
+                                     : ((unsigned long long)order_key(v) << 32) |
+                                           (0xffffffffu - uint32_t(idx));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(kFull, key, o);
+      key = y > key ? y : key;
+    }
+    __shared__ unsigned long long s_k[NW];
+    if (lane == 0) s_k[w] = key;
+    __syncthreads();
+    unsigned long long best = 0ull;
+    for (int i = 0; i < NW; ++i) best = s_k[i] > best ? s_k[i] : best;
+    __syncthreads();
+    return best == 0ull ? -1 : int(0xffffffffu - uint32_t(best & 0xffffffffull));
+  }
+};
+
+// Threshold bin search over a histogram: the largest bin b with (#active in bins >= b)
+// >= need. Writes the count strictly above b.
+template <int NT>
+QS_DEV void find_threshold_bin(const int* hist, int nbins, int need, int* s_bin, int* s_above,
+                               BlockOps<NT>& ops) {
+  // suffix sums: process bins from the top; thread t owns a contiguous range of bins
+  constexpr int MAXPER = (kLinBins + NT - 1) / NT;
+  const int per = (nbins + NT - 1) / NT;
+  // thread t owns bins [nbins - (t+1)*per, nbins - t*per) (top bins for low t)
+  const int hi_b = nbins - int(threadIdx.x) * per;
+  const int lo_b = max(hi_b - per, 0);
+  int local = 0;
+  for (int bn = lo_b; bn < hi_b; ++bn) local += hist[bn];
+  int total;
+  const int above_me = ops.exclusive_sum(local, &total);  // count in bins above my range
+  if (above_me < need && above_me + local >= need) {
+    int acc = above_me;
+    for (int bn = hi_b - 1; bn >= lo_b; --bn) {
+      if (acc + hist[bn] >= need) {
+        *s_bin = bn;
+        *s_above = acc;
+        break;
+      }
+      acc += hist[bn];
+    }
+  }
+  (void)MAXPER;
+  __syncthreads();
+}
+
+template <int NT, int ITEMS>
+__global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
+  constexpr int NW = NT / 32;
+  __shared__ int s_i[NW + 1];
+  __shared__ float s_f[2 * NW];
+  __shared__ int hist[kLinBins];
+  __shared__ int s_bin, s_above, s_forced[4], s_nforced;
+  BlockOps<NT> ops{s_i, s_f};
+
+  const int row = blockIdx.x;
+  const int b = row / a.Hkv;
+  const int tid = threadIdx.x;
+  int L = a.seq_lens[b];
+  const int nb_cap = a.nb_stride < NT * ITEMS ? a.nb_stride : NT * ITEMS;
+  int nb = (L + a.S - 1) / a.S;
+  if (L < 0 || nb > nb_cap) {
+    if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
+    nb = L < 0 ? 0 : nb_cap;
+    if (L < 0) L = 0;
+  }
+  int32_t* sel = a.sel + size_t(row) * a.budget;
+  const int k = a.budget;
+  const int n_out = nb < k ? nb : k;
+  if (tid == 0) a.n_sel[row] = n_out;
+
+  if (nb <= k) {  // the budget covers every block
+    for (int i = tid; i < k; i += NT) sel[i] = i < nb ? i : -1;
+    return;
+  }
+
+  // ---------------- forced blocks
+  const int j0 = tid * ITEMS;
+  if (a.n_keep > 0 && a.block_err != nullptr) {
+    const float* err = a.block_err + size_t(row) * a.nb_stride;
+    const int ncomplete = min(L / a.S, nb);
+    int kept0 = -1;
+    for (int r = 0; r < a.n_keep; ++r) {
+      float bv = -INFINITY;
+      int bi = -1;
+      for (int i = 0; i < ITEMS; ++i) {
+        const int j = j0 + i;
+        if (j < ncomplete && j != kept0) {
+          const float e = err[j];
+          if (bi < 0 || order_key(e) > order_key(bv)) { bv = e; bi = j; }
+        }
+      }
+      const int best = ops.argmax(bv, bi);
+      if (tid == 0) s_forced[2 + r] = best;
+      kept0 = best;
+      __syncthreads();
+    }
+  }
+  if (tid == 0) {
+    s_forced[0] = a.force_sink ? 0 : -1;
+    s_forced[1] = a.force_last ? nb - 1 : -1;
+    if (!(a.n_keep > 0 && a.block_err != nullptr)) { s_forced[2] = -1; s_forced[3] = -1; }
+    if (a.n_keep < 2) s_forced[3] = -1;
+    if (a.n_keep < 1) s_forced[2] = -1;
+    // dedupe
+    int n = 0;
+    for (int i = 0; i < 4; ++i) {
+      const int f = s_forced[i];
+      bool dup = f < 0;
+      for (int q = 0; q < i && !dup; ++q) dup = (s_forced[q] == f);
+      if (dup) s_forced[i] = -1; else ++n;
+    }
+    s_nforced = n;
+  }
+  __syncthreads();
+  int need = k - s_nforced;
+  if (need < 0) need = 0;
+
+  // ---------------- load scores into registers
+  const float* sc = a.scores + size_t(row) * a.nb_stride;
+  float v[ITEMS];
+  uint32_t active = 0u, chosen = 0u;
+#pragma unroll
+  for (int i = 0; i < ITEMS; ++i) {
+    const int j = j0 + i;
+    v[i] = -FLT_MAX;
+    if (j < nb) {
+      float x = sc[j];
+      if (x != x) x = -FLT_MAX;
+      x = fminf(fmaxf(x, -FLT_MAX), FLT_MAX);
+      v[i] = x;
+      bool f = false;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) f |= (s_forced[q] == j);
+      if (f) chosen |= 1u << i; else active |= 1u << i;
+    }
+  }
+
+  // ---------------- linear-bin pass
+  if (need > 0) {
+    float lo = FLT_MAX, hi = -FLT_MAX;
+#pragma unroll
+    for (int i = 0; i < ITEMS; ++i)
+      if (active >> i & 1u) { lo = fminf(lo, v[i]); hi = fmaxf(hi, v[i]); }
+    ops.minmax(lo, hi);
+    if (hi > lo) {
+      for (int i = tid; i < kLinBins; i += NT) hist[i] = 0;
+      __syncthreads();
+      const double scale = double(kLinBins) / (double(hi) - double(lo));
+      int bins[ITEMS];
+#pragma unroll
+      for (int i = 0; i < ITEMS; ++i) {
+        int bn = int((double(v[i]) - double(lo)) * scale);
+        bn = bn < 0 ? 0 : (bn >= kLinBins ? kLinBins - 1 : bn);
+        bins[i] = bn;
+        if (active >> i & 1u) atomicAdd(&hist[bn], 1);
+      }
+      __syncthreads();
+      find_threshold_bin<NT>(hist, kLinBins, need, &s_bin, &s_above, ops);
+      const int bstar = s_bin;
+#pragma unroll
+      for (int i = 0; i < ITEMS; ++i) {
+        if (!(active >> i & 1u)) continue;
+        if (bins[i] > bstar) { chosen |= 1u << i; active &= ~(1u << i); }
+        else if (bins[i] < bstar) active &= ~(1u << i);
+      }
+      need -= s_above;
+      __syncthreads();
+    }
+  }
+
+  // ---------------- exact radix select on order keys over what is left
+  for (int shift = 24; shift >= 0 && need > 0; shift -= 8) {
+    const int na = ops.sum(__popc(active));
+    if (na == need) break;
+    for (int i = tid; i < 256; i += NT) hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < ITEMS; ++i)
+      if (active >> i & 1u) atomicAdd(&hist[(order_key(v[i]) >> shift) & 255u], 1);
+    __syncthreads();
+    find_threshold_bin<NT>(hist, 256, need, &s_bin, &s_above, ops);
+    const uint32_t dstar = uint32_t(s_bin);
+#pragma unroll
+    for (int i = 0; i < ITEMS; ++i) {
+      if (!(active >> i & 1u)) continue;
+      const uint32_t dg = (order_key(v[i]) >> shift) & 255u;
+      if (dg > dstar) { chosen |= 1u << i; active &= ~(1u << i); }
+      else if (dg < dstar) active &= ~(1u << i);
+    }
+    need -= s_above;
+    __syncthreads();
+  }
+  // remaining actives share one key (or exactly fill the need): lowest indices first
+  if (need > 0) {
+    int tot;
+    const int before = ops.exclusive_sum(__popc(active), &tot);
+    int rank = before;
+#pragma unroll
+    for (int i = 0; i < ITEMS; ++i) {
+      if (active >> i & 1u) {
+        if (rank < need) chosen |= 1u << i;
+        ++rank;
+      }
+    }
+  }
+
+  // ---------------- ascending output
+  int tot;
+  int pos = ops.exclusive_sum(__popc(chosen), &tot);
+#pragma unroll
+  for (int i = 0; i < ITEMS; ++i)
+    if (chosen >> i & 1u) {
+      if (pos < k) sel[pos] = j0 + i;
+      ++pos;
+    }
+  if (tot != n_out && tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
+  for (int i = tot + tid; i < k; i += NT) sel[i] = -1;
+}
+
+cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s) {
+  const int nbs = a.nb_stride;
+  if (nbs <= 256 * 4) select_kernel<256, 4><<<a.rows, 256, 0, s>>>(a);
+  else if (nbs <= 256 * 16) select_kernel<256, 16><<<a.rows, 256, 0, s>>>(a);
+  else if (nbs <= 1024 * 32) select_kernel<1024, 32><<<a.rows, 1024, 0, s>>>(a);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace qs

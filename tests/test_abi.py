@@ -1,0 +1,81 @@
+"""The C-ABI library loads and exports every entry point declared in include/qs.h; host
+validation and workspace sizing work without a GPU (no compute call is made)."""
+import os
+import re
+
+import pytest
+
+import score_then_select_b200 as qs
+from score_then_select_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names += re.findall(r"\b(qs_[a-z0-9_]+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    L = qs.lib()
+    declared = _declared()
+    assert "qs_decode" in declared and "qs_sparse_attn" in declared
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings():
+    assert qs.qs_version() >= 10000
+    assert qs.status_string(B.QS_ERR_DEVICE_TIMEOUT).startswith("device-side")
+
+
+def _cfg(**kw):
+    base = dict(n_q_heads=40, n_kv_heads=8, head_dim=128, block_size=128, budget=64,
+                proxy_rank=32, proxy_dtype="bf16", force_sink=True, force_last=True)
+    base.update(kw)
+    return qs.make_config(**base)
+
+
+def test_workspace_size_is_positive_and_monotone():
+    a = qs.qs_workspace_size(_cfg(), 16, 131072)
+    b = qs.qs_workspace_size(_cfg(), 16, 262144)
+    assert 0 < a < b
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=96), B.QS_ERR_UNSUPPORTED),
+    (dict(n_q_heads=41), B.QS_ERR_INVALID_ARG),
+    (dict(n_q_heads=80), B.QS_ERR_UNSUPPORTED),          # group of 10 > 8
+    (dict(block_size=48), B.QS_ERR_INVALID_ARG),
+    (dict(budget=0), B.QS_ERR_INVALID_ARG),
+    (dict(proxy_rank=48), B.QS_ERR_UNSUPPORTED),
+    (dict(proxy_rank=0), B.QS_ERR_INVALID_ARG),          # rank 0 needs the NVFP4 proxy
+    (dict(v_dtype="f16", v_agg_dtype="bf16"), B.QS_ERR_UNSUPPORTED),
+    (dict(block_size=1, budget=2048), None),
+])
+def test_host_validation(kw, status):
+    if status is None:
+        assert qs.qs_workspace_size(_cfg(**kw), 16, 32768) > 0
+        return
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_workspace_size(_cfg(**kw), 16, 131072)
+    assert e.value.status == status
+
+
+def test_token_level_context_limit():
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_workspace_size(_cfg(block_size=1, budget=2048), 16, 65536)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+
+
+def test_null_pointers_rejected_without_launch():
+    cfg = _cfg()
+    cache = B.qs_cache()
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_decode(cfg, cache, 0, 0, 0, 0, 16, 0, None, None, 0, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG

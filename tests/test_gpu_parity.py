@@ -1,0 +1,148 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the same seeded inputs.
+
+Sizes: the small copies of every workload (several tiles, several pages, ragged tails).
+The bar:
+  * writer: projected-key cache bit-exact (F32 / BF16 bits); NVFP4 codes and scales
+    bit-exact;
+  * block scores: float32 against float64, |diff| <= 2e-5 * max(|beta|);
+  * selection: identical sets, except blocks within 1e-4 relative of the k-th score, where
+    the oracle confirms the GPU's set is a valid top-k;
+  * attention: max-abs <= 2e-2 (BF16 outputs), relative L2 <= 1e-3 (FP32 outputs),
+    against the oracle evaluated on the GPU's (validated) selection.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import method as M
+from tests.util import oracle_row, query_scale_all, row_params
+
+pytestmark = pytest.mark.gpu
+
+RANKR = [synth.TINY, synth.TINY_NEEDLE] + [synth.small(w) for w in
+                                          (synth.TOKEN32K, synth.BLOCK128K, synth.RAGGED)]
+NVFP4 = [synth.small(synth.NVFP4_128K)]
+
+
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tests.gpu_util import Filled  # noqa: F401  (imports the library)
+
+
+def _check_out(w, got, want, where):
+    if w.out_dtype == "f32":
+        rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+        assert rel <= 1e-3, f"{where}: rel-L2 {rel:.3e}"
+    else:
+        err = np.abs(got - want).max()
+        assert err <= 2e-2, f"{where}: max-abs {err:.3e}"
+
+
+def _run_workload(w):
+    from tests.gpu_util import Filled, out_to_f64
+    import score_then_select_b200 as qs
+    inp = synth.Inputs(w)
+    f = Filled(inp)
+    out, sel, nsel = f.decode()
+    st = f.status()
+    assert st[0] == 0, f"device status {st}"
+    # standalone stages on the same (now complete) caches
+    lay = f.layer
+    scores = torch.full((w.batch, w.n_kv_heads, lay.nb_stride), np.nan, dtype=torch.float32,
+                        device="cuda")
+    qs.qs_score(f.cfg, f.cache, f.q, f.P, w.batch, scores, lay.ws)
+    sel2 = torch.full_like(sel, -7)
+    nsel2 = torch.zeros_like(nsel)
+    qs.qs_select_topk(f.cfg, f.cache, scores, w.batch, sel2, nsel2, lay.ws)
+    out2 = torch.zeros_like(out)
+    qs.qs_sparse_attn(f.cfg, f.cache, f.q, sel2, nsel2, w.batch, out2, lay.ws)
+    st = f.status()
+    assert st[0] == 0, f"device status {st}"
+    assert torch.equal(sel, sel2) and torch.equal(nsel, nsel2)
+    assert torch.equal(out, out2)
+    return inp, f, out_to_f64(out), sel.cpu().numpy(), nsel.cpu().numpy(), scores.cpu().numpy()
+
+
+@pytest.mark.parametrize("w", RANKR, ids=lambda w: w.name)
+def test_rankr_parity(w):
+    _gpu()
+    inp, f, out, sel, nsel, scores = _run_workload(w)
+    G = w.group
+    for b in range(w.batch):
+        L = int(inp.lens[b])
+        nb = -(-L // w.block_size)
+        for g in range(w.n_kv_heads):
+            row = inp.row(b, g)
+            r = oracle_row(inp, b, g, row=row)
+            where = f"{w.name} row ({b},{g})"
+            # writer: bit-exact
+            got_proxy = f.row_proxy(b, g)
+            assert np.array_equal(got_proxy, r["cache"]), f"{where}: proxy cache differs"
+            # scores
+            beta = scores[b, g, :nb]
+            tol = 2e-5 * max(np.abs(r["beta"]).max(), 1e-30)
+            assert np.all(np.abs(beta - r["beta"]) <= tol), f"{where}: block scores"
+            # selection
+            n = int(nsel[b, g])
+            got = sel[b, g, :n]
+            assert np.all(sel[b, g, n:] == -1)
+            ok, why = M.selection_valid(r["beta"], w.budget, r["forced"], got)
+            assert ok, f"{where}: selection {why}"
+            # attention over the GPU's selection
+            rr = r if np.array_equal(got, r["sel"]) else oracle_row(inp, b, g, row=row,
+                                                                     sel_override=got)
+            _check_out(w, out[b, g * G:(g + 1) * G], rr["out"], where)
+
+
+def test_needle_selected_on_gpu():
+    _gpu()
+    inp, f, out, sel, nsel, scores = _run_workload(synth.TINY_NEEDLE)
+    assert 37 in sel[0, 0].tolist()
+
+
+def test_dense_rows_reduce_to_dense_attention():
+    """Ragged rows whose budget covers every block: the output is dense attention."""
+    _gpu()
+    w = synth.small(synth.RAGGED)
+    inp, f, out, sel, nsel, scores = _run_workload(w)
+    from oracle import formats as F
+    for b in range(w.batch):
+        L = int(inp.lens[b])
+        if -(-L // w.block_size) > w.budget:
+            continue
+        for g in range(w.n_kv_heads):
+            k, v, q = inp.row(b, g)
+            dense = M.sparse_attention(F.bf16_to_f64(q), F.bf16_to_f64(k[:L]),
+                                       F.bf16_to_f64(v[:L]), np.arange(L), w.scale)
+            assert sel[b, g, :nsel[b, g]].tolist() == list(range(-(-L // w.block_size)))
+            _check_out(w, out[b, g * w.group:(g + 1) * w.group], dense, f"dense row {b},{g}")
+
+
+def test_bad_page_table_entry_is_reported_not_faulted():
+    """A page id outside the cache is skipped by every kernel and reported as a bounds
+    error through the workspace status word."""
+    _gpu()
+    import score_then_select_b200 as qs
+    from tests.gpu_util import Filled
+    w = synth.small(synth.BLOCK128K)
+    inp = synth.Inputs(w)
+    f = Filled(inp)
+    assert f.status()[0] == 0
+    f.layer.page_table[0, 3] = inp.num_pages + 5        # host-side corruption
+    f.decode()
+    st, kid, info = f.status()
+    assert st == qs.binding.QS_ERR_DEVICE_BOUNDS
+    assert f.status()[0] == 0                            # the status was cleared
+
+
+def test_host_validation_rejects_before_launch():
+    _gpu()
+    import score_then_select_b200 as qs
+    from tests.gpu_util import Filled, cfg_kwargs
+    w = synth.TINY
+    bad = dict(cfg_kwargs(w), head_dim=96)
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_workspace_size(qs.make_config(**bad), 1, 2048)
+    assert e.value.status == qs.binding.QS_ERR_UNSUPPORTED
