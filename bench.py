@@ -1,0 +1,489 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of score-then-select sparse attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one qs_decode call over one batch: append the new token of every sequence,
+score the whole key history through the proxy cache, select the top-k blocks per
+(sequence, KV head), and attend over the selected keys and values. The default workload
+is the 128K-context, batch-16 block-level step (40 query / 8 KV heads, d = 128, rank-32
+BF16 proxy, 128-token blocks, budget 64 with the sink and last blocks forced); its
+seeded synthetic caches (about 9 GiB) exceed the L2, so no flush is needed.
+
+One JSON line is printed by rank 0. With N > 1 (torchrun), every rank runs its own batch
+of the same shape on its own GPU (weak scaling: the rows are independent, no collective
+is on the data path); the process group only provides the barrier and the max-over-ranks
+time.
+
+--impl reference times the CPU oracle (tests-only float64 implementation) on a bounded
+sample of the same workload, on the host cores, and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "sparse decode attn steps/s at 128K ctx, batch 16; achieved HBM GB/s vs peak"
+WORKLOADS = {"block128k": synth.BLOCK128K, "token32k": synth.TOKEN32K, "ragged": synth.RAGGED,
+             "nvfp4": synth.NVFP4_128K, "tiny": synth.TINY}
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="block128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=16, help="rows timed for the CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (small cases for profiling only)")
+    return ap.parse_args(argv)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (measured copy bandwidth)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6650 GB/s (earlier measurement on this pool)"
+
+
+# ------------------------------------------------------------------ clocks (NVML sampling)
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class Clocks:
+    """Samples SM clock and clock-event reasons of one GPU from a thread (read-only)."""
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.ok = False
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _read(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for bit, name in _REASONS.items():
+            if r & bit and bit != 0x1:
+                self.reasons.add(name)
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self._read()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if not self.ok:
+            return
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._loop, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self._stop.set()
+        self._t.join()
+        try:
+            self._read()
+        except Exception:
+            pass
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ byte accounting
+
+def step_bytes(w, lens, sel, nsel):
+    """Algorithmic bytes of one decode step: proxy-cache bytes streamed + selected K/V bytes
+    (valid tokens only) + q + out."""
+    d, S = w.head_dim, w.block_size
+    if w.proxy_dtype == "nvfp4":
+        per_tok = d // 2 + d // 16
+    else:
+        per_tok = w.proxy_rank * (4 if w.proxy_dtype == "f32" else 2)
+    proxy = int(np.sum(lens.astype(np.int64))) * w.n_kv_heads * per_tok
+    tokens = 0
+    for b in range(w.batch):
+        L = int(lens[b])
+        for g in range(w.n_kv_heads):
+            blk = sel[b, g, :int(nsel[b, g])].astype(np.int64)
+            tokens += int(np.minimum(S, L - blk * S).sum())
+    kv = tokens * d * 2 * 2
+    q = w.batch * w.n_q_heads * d * 2
+    out = w.batch * w.n_q_heads * d * (4 if w.out_dtype == "f32" else 2)
+    return {"proxy": proxy, "kv": kv, "q": q, "out": out, "total": proxy + kv + q + out,
+            "selected_tokens": tokens}
+
+
+def src_hash(*names):
+    h = hashlib.sha1()
+    for n in names:
+        with open(os.path.join(ROOT, "score_then_select_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch recorded by a committed ncu summary, if its source hash still
+    matches the kernel's current source; else None."""
+    p = os.path.join(ROOT, "profiles", f"{kernel_file}.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("workload") != workload:
+            return None
+        if d.get("src_hash") != src_hash(*d["sources"]):
+            return None
+        return d.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_prepare(w, inp, rows, threads):
+    """The rows' stored inputs and scoring caches, built by the oracle (untimed)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import method as M
+    from oracle import step as OS
+    from tests.util import row_params
+
+    p = row_params(w)
+
+    def prep(bg):
+        b, g = bg
+        k, v, q = inp.row(b, g)
+        L = int(inp.lens[b])
+        P = inp.P[g] if inp.P is not None else None
+        mu = inp.mu[b, g] if inp.mu is not None else None
+        cache = OS.row_scoring_cache(p, k[:L], P, mu, inp.g_k)
+        return (b, g, k, v, q, L, P, cache)
+
+    with threadpool_limits(limits=1):
+        with cf.ThreadPoolExecutor(threads) as ex:
+            prepared = list(ex.map(prep, rows))
+    g_q = None
+    if w.proxy_dtype == "nvfp4":
+        g_q = M.query_scale(np.stack([x[4] for x in prepared]))
+    return p, prepared, g_q
+
+
+def oracle_time(w, inp, prep, threads):
+    """Seconds for the oracle's decode step (score + select + attend) over prepared rows,
+    one row per thread, BLAS pinned to one thread."""
+    from threadpoolctl import threadpool_limits
+    from oracle import formats as F
+    from oracle import method as M
+    from oracle import step as OS
+
+    p, prepared, g_q = prep
+
+    def one(x):
+        b, g, k, v, q, L, P, cache = x
+        beta = OS.row_block_scores(p, cache, q, L, P=P, g_q=g_q, g_k=inp.g_k)
+        forced, _ = OS.row_forced(p, beta.shape[0], cache, L, inp.g_k)
+        sel = M.select_blocks(beta, p.budget, forced)
+        tok = M.block_tokens(sel, p.S, L)
+        return M.sparse_attention(F.bf16_to_f64(q), F.bf16_to_f64(k[tok]),
+                                  OS.decode_v(v[tok], p.v_dtype), np.arange(len(tok)), p.scale)
+
+    with threadpool_limits(limits=1):
+        with cf.ThreadPoolExecutor(threads) as ex:
+            t0 = time.perf_counter()
+            list(ex.map(one, prepared))
+            return time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, inp, nrows, cpu_work_s=10.0, max_wall_s=20.0):
+    """The oracle on a bounded sample: `nrows` rows of one step, one row per host thread,
+    repeated until about `cpu_work_s` seconds of CPU work (wall time x threads) are done."""
+    rows = [(b, g) for b in range(w.batch) for g in range(w.n_kv_heads)][:nrows]
+    threads = min(host_cores(), len(rows))
+    prep = oracle_prepare(w, inp, rows, threads)
+    total, passes = 0.0, 0
+    while passes < 1 or (total * threads < cpu_work_s and total < max_wall_s):
+        total += oracle_time(w, inp, prep, threads)
+        passes += 1
+    t = total / passes
+    total_rows = w.batch * w.n_kv_heads
+    return {"value": (len(rows) / total_rows) / t, "unit": "steps/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{len(rows)} of {total_rows} (sequence, KV head) rows of one step, "
+                      f"{passes} passes ({total:.1f} s wall); score+select+attend from "
+                      f"prepared scoring caches, float64 numpy, one row per thread"}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def config_of(w, lens):
+    return {"workload": w.name, "global_batch": w.batch, "context": int(lens.max()),
+            "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+            "block_size": w.block_size, "budget_blocks": w.budget, "proxy": w.proxy_dtype,
+            "proxy_rank": w.proxy_rank, "parallelism": "independent rows per GPU",
+            "l2": "no flush: per-step inputs (proxy cache + selected K/V) exceed the 126 MB L2"}
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    world, rank, local = dist_setup()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    inp = synth.Inputs(w)
+    cores = host_cores()
+    rows_all = [(b, g) for b in range(w.batch) for g in range(w.n_kv_heads)]
+    per_step = min(cores, len(rows_all), 8)
+    total_rows = len(rows_all)
+    prep = oracle_prepare(w, inp, rows_all[:per_step], per_step)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = oracle_time(w, inp, prep, per_step)
+        if i >= args.warmup:
+            times.append(t)
+    t_step = sum(times) / len(times)
+    value = (per_step / total_rows) / t_step
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, inp.lens),
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": per_step,
+                             "kind": "oracle",
+                             "sample": f"{per_step} of {total_rows} rows per step, "
+                                       "score+select+attend from prepared scoring caches"},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_setup()
+    if world != args.gpus:
+        print(f"--gpus {args.gpus} but WORLD_SIZE {world}: launch N > 1 with torchrun",
+              file=sys.stderr)
+        return 2
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    import score_then_select_b200 as qs
+    from tests.gpu_util import Filled
+
+    w0 = WORKLOADS[args.workload]
+    if args.batch:
+        w0 = w0.replace(batch=args.batch)
+    w = w0 if rank == 0 else w0.replace(seed=w0.seed + 1000 * rank)
+    inp = synth.Inputs(w)
+    f = Filled(inp)
+    lay, cfg, cache = f.layer, f.cfg, f.cache
+    B = w.batch
+    lens = inp.lens
+    start_lens = torch.from_numpy((lens - 1).astype(np.int32)).cuda()
+    out = torch.zeros((B, w.n_q_heads, w.head_dim),
+                      dtype=torch.float32 if w.out_dtype == "f32" else torch.bfloat16, device="cuda")
+    sel = torch.zeros((B, w.n_kv_heads, w.budget), dtype=torch.int32, device="cuda")
+    nsel = torch.zeros((B, w.n_kv_heads), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lay.seq_lens.copy_(start_lens, non_blocking=True)
+        qs.qs_decode(cfg, cache, f.q, f.k_last, f.v_last, f.P, B, out, sel, nsel, lay.ws, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    st = qs.qs_device_status(lay.ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st}")
+    nsel_h = nsel.cpu().numpy()
+    sel_h = sel.cpu().numpy()
+    launches_per_step = 4 if w.proxy_rank > 0 else 6
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---------------- timed region: K fused decode steps
+    clocks = Clocks(local)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    t_ms = e0.elapsed_time(e1) / args.steps
+    t_max = torch.tensor([t_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    t_ms = float(t_max.item())
+    st = qs.qs_device_status(lay.ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device status after timing {st}")
+
+    # ---------------- per-stage breakdown through the standalone entry points
+    n_stage = min(args.steps, 50)
+    ones = torch.ones((B,), dtype=torch.int32, device="cuda")
+    scores = torch.empty((B, w.n_kv_heads, lay.nb_stride), dtype=torch.float32, device="cuda")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_stage + 3)]
+    for i in range(n_stage + 3):          # no host sync inside: the host stays ahead
+        ev = evs[i]
+        lay.seq_lens.copy_(start_lens, non_blocking=True)
+        ev[0].record(stream)
+        qs.qs_append_kv(cfg, cache, f.k_last, f.v_last, ones, 1, f.P, B, lay.ws, stream)
+        ev[1].record(stream)
+        qs.qs_score(cfg, cache, f.q, f.P, B, scores, lay.ws, stream)
+        ev[2].record(stream)
+        qs.qs_select_topk(cfg, cache, scores, B, sel, nsel, lay.ws, stream)
+        ev[3].record(stream)
+        qs.qs_sparse_attn(cfg, cache, f.q, sel, nsel, B, out, lay.ws, stream)
+        ev[4].record(stream)
+    torch.cuda.synchronize()
+    acc = np.zeros(4)
+    for ev in evs[3:]:
+        acc += [ev[j].elapsed_time(ev[j + 1]) for j in range(4)]
+    stage_us = dict(zip(["append", "score", "select", "attend"], (acc / n_stage * 1e3).tolist()))
+
+    # ---------------- end to end: host buffers, copies inside the timed region
+    q_h = f.q.cpu().pin_memory()
+    k_h = f.k_last.cpu().pin_memory()
+    v_h = f.v_last.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_d, k_d, v_d = torch.empty_like(f.q), torch.empty_like(f.k_last), torch.empty_like(f.v_last)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        lay.seq_lens.copy_(start_lens, non_blocking=True)
+        qs.qs_decode(cfg, cache, q_d, k_d, v_d, f.P, B, out, sel, nsel, lay.ws, stream)
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    n_e2e = max(args.steps, 10)
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(n_e2e):
+        e2e_step()
+    e2e_ms = (time.perf_counter() - t0) * 1e3 / n_e2e
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_t.item())
+    h2d = q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2
+    d2h = out_h.numel() * out_h.element_size()
+
+    # ---------------- roofline
+    peak, peak_src = peaks()
+    by = step_bytes(w, lens, sel_h, nsel_h)
+    score_us = stage_us["score"]
+    score_kernel_file = "score.cu" if w.proxy_rank > 0 else "score_nvfp4.cu"
+    traffic = profiled_traffic(score_kernel_file.replace(".cu", ""), w.name)
+    roof = {"bound": "hbm", "kernel": "score (scoring prep + proxy scan, one qs_score call)",
+            "achieved": by["proxy"] / (score_us * 1e-6) / 1e9, "peak": peak, "unit": "GB/s",
+            "frac": by["proxy"] / (score_us * 1e-6) / 1e9 / peak, "peak_source": peak_src,
+            "algorithmic_bytes_per_launch": by["proxy"], "launch_us": score_us,
+            "traffic": traffic}
+    step_gbs = by["total"] / (t_ms * 1e-3) / 1e9
+    value = world * 1e3 / t_ms
+    line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; shapes of the pages' 128K batch-16 decode)",
+            "config": config_of(w, lens),
+            "tokens_per_s": value * B, "us_per_layer_step": t_ms * 1e3,
+            "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": step_gbs / peak, "bytes_per_step": by},
+            "stage_us": stage_us, "roofline": roof, "clocks": clk,
+            "e2e": {"value": world * 1e3 / e2e_ms, "unit": "steps/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps * launches_per_step}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

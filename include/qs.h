@@ -124,7 +124,7 @@ typedef struct {
 qs_status qs_workspace_size(const qs_config *cfg, int32_t batch, int32_t max_context,
                             size_t *bytes /* host */);
 
-/* Zero the workspace status word and counters (async on stream). Call once after
+/* Zero the whole workspace (status word and counters; async on stream). Call once after
    allocating a workspace, before any other call uses it. */
 qs_status qs_workspace_init(void *ws, size_t ws_bytes, qs_stream_t stream);
 
@@ -188,7 +188,7 @@ qs_status qs_decode(const qs_config *cfg, const qs_cache *cache, const void *q,
    since the last call (QS_OK if none) and clear it. `detail` (HOST pointer, may be NULL)
    receives {kernel id, index} of that error. Returns QS_ERR_CUDA if the synchronisation
    or the read-back fails. Kernel ids: 1 append, 2 block error, 3 scoring prep, 4 score,
-   5 select, 6 attention, 7 combine. */
+   5 select, 6 attention (with its log-sum-exp combine). */
 qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
 
 /* Static string naming a status code. */

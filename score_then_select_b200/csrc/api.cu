@@ -117,6 +117,7 @@ static qs_status make_plan(const qs_config* c, int batch, int max_context, Plan&
   w.nsel = off;    off = align_up(off + rows * 4, 256);
   w.part_ml = off; off = align_up(off + rows_q * w.splits * 2 * 4, 256);
   w.part_o = off;  off = align_up(off + rows_q * w.splits * p.d * 4, 256);
+  w.row_ctr = off; off = align_up(off + rows * 4, 256);
   w.total = off;
   return QS_OK;
 }
@@ -204,7 +205,8 @@ static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws,
   return cuda_status(launch_qpack(p, a, s));
 }
 
-static qs_status do_score(const Plan& p, const qs_cache* c, float* scores, void* ws, cudaStream_t s) {
+static qs_status do_score(const Plan& p, const qs_cache* c, float* scores, void* ws, cudaStream_t s,
+                          bool pdl) {
   ScoreParams a{};
   a.proxy = c->proxy;
   a.proxy_scale = c->proxy_scale;
@@ -226,11 +228,11 @@ static qs_status do_score(const Plan& p, const qs_cache* c, float* scores, void*
   a.max_pages_per_seq = c->max_pages_per_seq;
   a.num_pages = c->num_pages;
   a.max_context = c->max_context;
-  return cuda_status(launch_score(p, a, s));
+  return cuda_status(launch_score(p, a, s, pdl));
 }
 
 static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores, int32_t* sel,
-                           int32_t* n_sel, void* ws, cudaStream_t s) {
+                           int32_t* n_sel, void* ws, cudaStream_t s, bool pdl) {
   SelectParams a{};
   a.scores = scores;
   a.block_err = (p.r == 0 && p.n_keep > 0) ? c->block_err : nullptr;
@@ -246,11 +248,11 @@ static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores
   a.force_sink = p.force_sink;
   a.force_last = p.force_last;
   a.n_keep = a.block_err ? p.n_keep : 0;
-  return cuda_status(launch_select(p, a, s));
+  return cuda_status(launch_select(p, a, s, pdl));
 }
 
 static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, const int32_t* sel,
-                           const int32_t* n_sel, void* out, void* ws, cudaStream_t s) {
+                           const int32_t* n_sel, void* out, void* ws, cudaStream_t s, bool pdl) {
   AttnParams a{};
   a.q = static_cast<const uint16_t*>(q);
   a.k = static_cast<const uint16_t*>(c->k);
@@ -261,6 +263,9 @@ static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, cons
   a.seq_lens = c->seq_lens;
   a.part_ml = ws_at<float>(ws, p.ws.part_ml);
   a.part_o = ws_at<float>(ws, p.ws.part_o);
+  a.row_ctr = ws_at<uint32_t>(ws, p.ws.row_ctr);
+  a.out = out;
+  a.out_bf16 = p.out_dtype == QS_BF16 ? 1 : 0;
   a.hdr = hdr_of(ws);
   a.batch = p.batch;
   a.Hkv = p.Hkv;
@@ -272,11 +277,7 @@ static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, cons
   a.max_pages_per_seq = c->max_pages_per_seq;
   a.num_pages = c->num_pages;
   a.scale_log2 = p.scale * 1.4426950408889634f;
-  qs_status st = cuda_status(launch_attn(p, a, s));
-  if (st != QS_OK) return st;
-  CombineParams cb{a.part_ml, a.part_o, out, p.batch * p.Hq, p.ws.splits, p.d,
-                   p.out_dtype == QS_BF16 ? 1 : 0};
-  return cuda_status(launch_combine(p, cb, s));
+  return cuda_status(launch_attn(p, a, s, pdl));
 }
 
 }  // namespace qs
@@ -310,7 +311,7 @@ qs_status qs_workspace_size(const qs_config* cfg, int32_t batch, int32_t max_con
 
 qs_status qs_workspace_init(void* ws, size_t ws_bytes, qs_stream_t stream) {
   if (!ws || ws_bytes < size_t(kHdrWords) * 4 || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
-  return cuda_status(cudaMemsetAsync(ws, 0, size_t(kHdrWords) * 4, stream));
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, stream));
 }
 
 qs_status qs_append_kv(const qs_config* cfg, const qs_cache* cache, const void* k_new,
@@ -336,7 +337,7 @@ qs_status qs_score(const qs_config* cfg, const qs_cache* cache, const void* q, c
   if (!q || !aligned(q, 4) || !block_scores || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
   if ((st = do_prep(p, q, P, ws, stream)) != QS_OK) return st;
-  return do_score(p, cache, block_scores, ws, stream);
+  return do_score(p, cache, block_scores, ws, stream, true);
 }
 
 qs_status qs_select_topk(const qs_config* cfg, const qs_cache* cache, const float* block_scores,
@@ -347,7 +348,7 @@ qs_status qs_select_topk(const qs_config* cfg, const qs_cache* cache, const floa
   if (!cache || !cache->seq_lens) return QS_ERR_INVALID_ARG;
   if (!block_scores || !sel || !n_sel || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (p.r == 0 && p.n_keep > 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
-  return do_select(p, cache, block_scores, sel, n_sel, ws, stream);
+  return do_select(p, cache, block_scores, sel, n_sel, ws, stream, false);
 }
 
 qs_status qs_sparse_attn(const qs_config* cfg, const qs_cache* cache, const void* q,
@@ -358,7 +359,7 @@ qs_status qs_sparse_attn(const qs_config* cfg, const qs_cache* cache, const void
   if (st != QS_OK) return st;
   if ((st = check_cache(p, cache, false)) != QS_OK) return st;
   if (!q || !aligned(q, 4) || !sel || !n_sel || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
-  return do_attend(p, cache, q, sel, n_sel, out, ws, stream);
+  return do_attend(p, cache, q, sel, n_sel, out, ws, stream, false);
 }
 
 qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, const void* k_new,
@@ -379,9 +380,9 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   // append (+ fused scoring prep on the rank-r path)
   if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, P, q, ws, stream)) != QS_OK) return st;
   if (p.r == 0 && (st = do_prep(p, q, P, ws, stream)) != QS_OK) return st;
-  if ((st = do_score(p, cache, scores, ws, stream)) != QS_OK) return st;
-  if ((st = do_select(p, cache, scores, sel, nsel, ws, stream)) != QS_OK) return st;
-  return do_attend(p, cache, q, sel, nsel, out, ws, stream);
+  if ((st = do_score(p, cache, scores, ws, stream, true)) != QS_OK) return st;
+  if ((st = do_select(p, cache, scores, sel, nsel, ws, stream, true)) != QS_OK) return st;
+  return do_attend(p, cache, q, sel, nsel, out, ws, stream, true);
 }
 
 qs_status qs_device_status(void* ws, qs_stream_t stream, uint32_t* detail) {

@@ -260,6 +260,91 @@ append_rankr_kernel(const AppendParams a) {
   finish_append(a);
 }
 
+// ============================================================ rank-r writer, one new token
+// The decode step appends one token per row: CTA = one row. Thread j < R computes
+// projected entry j with the same ascending, separately rounded float32 evaluation as the
+// bulk writer (so both writers produce identical bits); with a query given, threads
+// R..2R-1 compute the row's q~ (the fused scoring prep).
+template <typename PT, int R, int D>
+__global__ void __launch_bounds__(128) append_one_rankr_kernel(const AppendParams a) {
+  __shared__ __align__(16) float Ps[D * R];
+  __shared__ float kf[D], qbar[D];
+  __shared__ int s_page, s_slot;
+  pdl_trigger();
+  const int row = blockIdx.x;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  const int tid = threadIdx.x;
+  int n_b = a.n_new ? a.n_new[b] : 1;
+  if (n_b < 0 || n_b > 1) {
+    if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_APPEND, uint32_t(b));
+    n_b = 0;
+  }
+  // every global load of the prologue is issued before any is consumed
+  const float* Pg = a.P + size_t(g) * D * R;
+  constexpr int NP4 = D * R / 4 / 128;               // float4 loads of P per thread
+  float4 pv[NP4];
+#pragma unroll
+  for (int j = 0; j < NP4; ++j) pv[j] = reinterpret_cast<const float4*>(Pg)[j * 128 + tid];
+  const size_t src = size_t(row) * a.max_new * D;  // token 0 of this row in k_new / v_new
+  const bool has_k = n_b == 1 && tid < D;
+  const uint16_t kraw = has_k ? a.k_new[src + tid] : uint16_t(0);
+  const bool prep = a.q != nullptr && tid < D;
+  uint16_t qraw[kMaxGroup];
+  {
+    const int Hq = a.Hkv * a.G;
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+      qraw[h] = (prep && h < a.G) ? a.q[(size_t(b) * Hq + g * a.G + h) * D + tid] : uint16_t(0);
+  }
+  if (tid == 0) {
+    int page = -1, slot = 0;
+    if (n_b == 1)
+      cache_slot(a.page_table, b, a.seq_lens[b], a.max_pages_per_seq, a.num_pages,
+                 a.max_context, a.hdr, KID_APPEND, page, slot);
+    s_page = page;
+    s_slot = slot;
+  }
+#pragma unroll
+  for (int j = 0; j < NP4; ++j) reinterpret_cast<float4*>(Ps)[j * 128 + tid] = pv[j];
+  if (has_k) kf[tid] = bf16_to_f32(kraw);
+  if (prep) {
+    float s = 0.0f;
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+      if (h < a.G) s += bf16_to_f32(qraw[h]);
+    qbar[tid] = s / float(a.G);
+  }
+  __syncthreads();
+  const int page = s_page;
+  if (n_b == 1 && page >= 0) {
+    const size_t dst = ((size_t(page) * a.Hkv + g) * kPage + s_slot) * D;
+    constexpr int CH = D / 8;
+    if (tid < CH)
+      reinterpret_cast<uint4*>(a.k + dst)[tid] = reinterpret_cast<const uint4*>(a.k_new + src)[tid];
+    else if (tid < 2 * CH)
+      reinterpret_cast<uint4*>(a.v + dst)[tid - CH] =
+          reinterpret_cast<const uint4*>(a.v_new + src)[tid - CH];
+    if (tid < R) {
+      float acc = 0.0f;
+#pragma unroll 8
+      for (int i = 0; i < D; ++i) acc = __fadd_rn(acc, __fmul_rn(kf[i], Ps[i * R + tid]));
+      const size_t pdst = ((size_t(page) * a.Hkv + g) * kPage + s_slot) * R + tid;
+      if constexpr (sizeof(PT) == 4)
+        reinterpret_cast<float*>(a.proxy)[pdst] = acc;
+      else
+        reinterpret_cast<uint16_t*>(a.proxy)[pdst] = f32_to_bf16_rn(acc);
+    }
+  }
+  if (a.q != nullptr && tid >= 64 && tid < 64 + R) {
+    const int j = tid - 64;
+    float acc = 0.0f;
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) acc = fmaf(qbar[i], Ps[i * R + j], acc);
+    a.qt[size_t(row) * R + j] = acc;
+  }
+  finish_append(a);
+}
+
 // ============================================================ NVFP4 writer
 // CTA = one row x 64 tokens; thread = (token, 16-element group).
 __global__ void __launch_bounds__(128) append_nvfp4_kernel(const AppendParams a) {
@@ -431,8 +516,9 @@ static cudaError_t launch_rankr(const Plan& p, const AppendParams& a, cudaStream
   constexpr int NT = 64 * R / 16;
   const size_t smem = size_t(D) * R * 4 + size_t(D) * 64 * 4;
   auto k = append_rankr_kernel<PT, R, D>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (attr != cudaSuccess) return attr;
   dim3 grid((a.max_new + 63) / 64, a.batch * a.Hkv);
   k<<<grid, NT, smem, s>>>(a);
   return cudaGetLastError();
@@ -445,6 +531,21 @@ cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) 
     return cudaGetLastError();
   }
   const bool f32 = p.proxy_dtype == QS_F32;
+  if (a.max_new == 1) {
+#define QS_ONE(PT, R, D) \
+  { append_one_rankr_kernel<PT, R, D><<<a.batch * a.Hkv, 128, 0, s>>>(a); return cudaGetLastError(); }
+    if (p.d == 64) {
+      if (f32 && p.r == 16) QS_ONE(float, 16, 64)
+      if (!f32 && p.r == 32) QS_ONE(uint16_t, 32, 64)
+    } else {
+      if (f32 && p.r == 16) QS_ONE(float, 16, 128)
+      if (f32 && p.r == 32) QS_ONE(float, 32, 128)
+      if (!f32 && p.r == 32) QS_ONE(uint16_t, 32, 128)
+      if (!f32 && p.r == 64) QS_ONE(uint16_t, 64, 128)
+    }
+#undef QS_ONE
+    return cudaErrorInvalidValue;
+  }
   if (p.d == 64) {
     if (f32 && p.r == 16) return launch_rankr<float, 16, 64>(p, a, s);
     if (!f32 && p.r == 32) return launch_rankr<uint16_t, 32, 64>(p, a, s);

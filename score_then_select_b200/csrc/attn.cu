@@ -1,4 +1,4 @@
-// attn.cu - split-K sparse attention over the selected blocks, and the LSE combine.
+// attn.cu - split-K sparse attention over the selected blocks with its LSE combine.
 //
 // "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 1 and
 // Abstract: gather-free indexed attention reads the original full-dimensional keys and
@@ -17,8 +17,9 @@
 //   O^T[d x 8 heads]      += V^T[d x 16 tok] . P^T[16 tok x 8 heads] (A = V via ldmatrix.trans,
 //                                                                    B = P via movmatrix)
 // Each warp's partial (max, sum, o) is merged across warps in shared memory and written
-// as one split partial; the combine kernel merges splits by log-sum-exp. Scores are kept
-// in base 2 (scale * log2 e folded into the logits).
+// as one split partial; the last CTA of a row to finish (a workspace counter) merges the
+// row's splits by log-sum-exp and writes the output. Scores are kept in base 2
+// (scale * log2 e folded into the logits).
 #include "qs_device.cuh"
 
 namespace qs {
@@ -51,6 +52,7 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
   extern __shared__ __align__(128) uint8_t smem[];
   int* s_rows = reinterpret_cast<int*>(smem + SM::kRowsOff);
 
+  pdl_wait();      // the selection comes from the kernel before
   const int split = blockIdx.x, row = blockIdx.y;
   const int b = row / a.Hkv, g = row % a.Hkv;
   const int Hq = a.Hkv * a.G;
@@ -67,23 +69,63 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
   const int s1 = min(s0 + a.tokens_per_split, slots);
   const int cnt = s1 - s0;
 
-  // ---------------- token table of this split: cache row index or -1
-  for (int i = tid; i < a.tokens_per_split; i += 128) {
-    int r = -1;
-    if (i < cnt) {
-      const int gs = s0 + i;
-      const int blk = a.sel[size_t(row) * a.budget + gs / a.S];
-      const int nbr = (L + a.S - 1) / a.S;
-      if (blk >= nbr) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
-      const int t = (blk >= 0 && blk < nbr) ? blk * a.S + gs % a.S : L;
-      if (t < L) {
-        const int pi = t / kPage;
-        const int page = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
-        if (page >= 0 && page < a.num_pages) r = (page * a.Hkv + g) * kPage + (t % kPage);
-        else flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
+  // ---------------- token table of this split: cache row index or -1.
+  // Selection entries [i0, i1) cover the split's slots; each entry (a block of S tokens
+  // inside one page) is resolved once, 8 entries per thread in flight at a time; the
+  // per-entry base rows are staged in the (still unused) tile ring.
+  {
+    int* e_base = reinterpret_cast<int*>(smem);                 // [entries] row of token 0
+    int* e_len = e_base + (kMaxTokensPerSplit + 1);             // [entries] valid tokens
+    const int i0 = s0 / a.S;
+    const int i1 = cnt > 0 ? (s1 + a.S - 1) / a.S : i0;
+    const int ne = i1 - i0;
+    const int nbr = (L + a.S - 1) / a.S;
+    const int32_t* selr = a.sel + size_t(row) * a.budget;
+    for (int u0 = 0; u0 < ne; u0 += 128 * 8) {
+      int blk[8], pg[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int u = u0 + j * 128 + tid;
+        blk[j] = u < ne ? selr[i0 + u] : -1;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        pg[j] = -1;
+        const int u = u0 + j * 128 + tid;
+        if (u < ne) {
+          if (blk[j] < 0 || blk[j] >= nbr) {
+            flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
+            blk[j] = -1;
+          } else {
+            const int pi = blk[j] * a.S / kPage;
+            pg[j] = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
+            if (pg[j] < 0 || pg[j] >= a.num_pages) {
+              flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
+              pg[j] = -1;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int u = u0 + j * 128 + tid;
+        if (u < ne) {
+          const int t0 = blk[j] * a.S;
+          e_base[u] = pg[j] >= 0 ? (pg[j] * a.Hkv + g) * kPage + (t0 % kPage) : -1;
+          e_len[u] = pg[j] >= 0 ? min(a.S, L - t0) : 0;
+        }
       }
     }
-    s_rows[i] = r;
+    __syncthreads();
+    for (int i = tid; i < a.tokens_per_split; i += 128) {
+      int r = -1;
+      if (i < cnt) {
+        const int gs = s0 + i;
+        const int u = gs / a.S - i0, off = gs % a.S;
+        if (off < e_len[u]) r = e_base[u] + off;
+      }
+      s_rows[i] = r;
+    }
   }
 
   // ---------------- query fragments (B operand of S^T): head = lane/4, dims 2*(lane%4)+{0,1}
@@ -253,61 +295,83 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
       a.part_ml[pidx * 2 + 1] = lsum;
     }
   }
-}
 
-// out[h][d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s; rows with no tokens -> 0
-__global__ void combine_kernel(const CombineParams a) {
-  const int rq = blockIdx.x;
-  const float* ml = a.part_ml + size_t(rq) * a.splits * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < a.splits; ++s)
-    if (ml[2 * s + 1] > 0.0f) M = fmaxf(M, ml[2 * s]);
-  for (int d = threadIdx.x; d < a.d; d += blockDim.x) {
-    float num = 0.0f, den = 0.0f;
-    for (int s = 0; s < a.splits; ++s) {
-      const float l = ml[2 * s + 1];
-      if (!(l > 0.0f)) continue;
-      const float w = ex2(ml[2 * s] - M);
-      den += w * l;
-      num += w * a.part_o[(size_t(rq) * a.splits + s) * a.d + d];
-    }
-    const float r = den > 0.0f ? num / den : 0.0f;
-    if (a.out_bf16)
-      reinterpret_cast<uint16_t*>(a.out)[size_t(rq) * a.d + d] = f32_to_bf16_rn(r);
-    else
-      reinterpret_cast<float*>(a.out)[size_t(rq) * a.d + d] = r;
+  // ---------------- the last split of the row to finish merges all splits (LSE combine):
+  // out[h][d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s; a row with no tokens -> 0
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned prev = atomicAdd(a.row_ctr + row, 1u);
+    s_last = prev == unsigned(a.splits - 1);
   }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float* s_w = reinterpret_cast<float*>(smem);          // [G][splits] weights, then [G] 1/den
+  const int ns = a.splits;
+  for (int i = tid; i < a.G * ns; i += 128) {
+    const int h = i / ns, sp = i % ns;
+    const size_t pidx = (size_t(b) * Hq + g * a.G + h) * ns + sp;
+    s_w[i] = __ldcg(a.part_ml + pidx * 2);
+    s_w[a.G * ns + i] = __ldcg(a.part_ml + pidx * 2 + 1);
+  }
+  __syncthreads();
+  if (tid < a.G) {
+    const int h = tid;
+    float M = -INFINITY;
+    for (int sp = 0; sp < ns; ++sp)
+      if (s_w[a.G * ns + h * ns + sp] > 0.0f) M = fmaxf(M, s_w[h * ns + sp]);
+    float den = 0.0f;
+    for (int sp = 0; sp < ns; ++sp) {
+      const float l = s_w[a.G * ns + h * ns + sp];
+      const float wt = l > 0.0f ? ex2(s_w[h * ns + sp] - M) : 0.0f;
+      s_w[h * ns + sp] = wt;
+      den += wt * l;
+    }
+    s_w[2 * a.G * ns + h] = den > 0.0f ? 1.0f / den : 0.0f;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < a.G * D; idx += 128) {
+    const int h = idx / D, d = idx % D;
+    const size_t rq = size_t(b) * Hq + g * a.G + h;
+    float num = 0.0f;
+    for (int sp = 0; sp < ns; ++sp) {
+      const float wt = s_w[h * ns + sp];
+      if (wt != 0.0f) num += wt * __ldcg(a.part_o + (rq * ns + sp) * D + d);
+    }
+    const float r = num * s_w[2 * a.G * ns + h];
+    if (a.out_bf16)
+      reinterpret_cast<uint16_t*>(a.out)[rq * D + d] = f32_to_bf16_rn(r);
+    else
+      reinterpret_cast<float*>(a.out)[rq * D + d] = r;
+  }
+  if (tid == 0) a.row_ctr[row] = 0u;
 }
 
 template <int D, bool VF, bool AF>
-static cudaError_t launch_attn_t(const AttnParams& a, cudaStream_t s) {
+static cudaError_t launch_attn_t(const AttnParams& a, cudaStream_t s, bool pdl) {
   auto k = attn_kernel<D, VF, AF>;
   const int smem = AttnSmem<D>::kTotal;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(a.splits, a.batch * a.Hkv);
-  k<<<grid, 128, smem, s>>>(a);
-  return cudaGetLastError();
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (attr != cudaSuccess) return attr;
+  return launch_k(k, dim3(a.splits, a.batch * a.Hkv), dim3(128), smem, s, pdl, a);
 }
 
-cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s) {
+cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl) {
   const bool vf = p.v_dtype == QS_F16, af = p.v_agg_dtype == QS_F16;
   if (p.d == 128) {
-    if (vf) return launch_attn_t<128, true, true>(a, s);
-    if (af) return launch_attn_t<128, false, true>(a, s);
-    return launch_attn_t<128, false, false>(a, s);
+    if (vf) return launch_attn_t<128, true, true>(a, s, pdl);
+    if (af) return launch_attn_t<128, false, true>(a, s, pdl);
+    return launch_attn_t<128, false, false>(a, s, pdl);
   }
   if (p.d == 64) {
-    if (vf) return launch_attn_t<64, true, true>(a, s);
-    if (af) return launch_attn_t<64, false, true>(a, s);
-    return launch_attn_t<64, false, false>(a, s);
+    if (vf) return launch_attn_t<64, true, true>(a, s, pdl);
+    if (af) return launch_attn_t<64, false, true>(a, s, pdl);
+    return launch_attn_t<64, false, false>(a, s, pdl);
   }
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_combine(const Plan& p, const CombineParams& a, cudaStream_t s) {
-  combine_kernel<<<a.rows_q, a.d, 0, s>>>(a);
-  return cudaGetLastError();
 }
 
 }  // namespace qs

@@ -17,6 +17,14 @@ namespace qs {
 
 constexpr unsigned kFull = 0xffffffffu;
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before the kernel
+// ahead of it in the stream has finished; pdl_wait() blocks until that kernel has
+// completed and its memory is visible (a no-op for a normal launch). pdl_trigger() lets
+// the next kernel in the stream begin launching early.
+QS_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+QS_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- status word
 // ws header (uint32 words): [0] first error code, [1] kernel id, [2] index, [16..] counters.
 QS_DEV void flag_error(uint32_t* hdr, uint32_t code, uint32_t kernel, uint32_t info) {

@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <utility>
 
 #include "../../include/qs.h"
 
@@ -16,8 +17,7 @@ enum KernelId : uint32_t {
   KID_PREP = 3,
   KID_SCORE = 4,
   KID_SELECT = 5,
-  KID_ATTN = 6,
-  KID_COMBINE = 7
+  KID_ATTN = 6
 };
 
 constexpr int kPage = 128;          // tokens per page (the only page size built)
@@ -38,6 +38,7 @@ struct WsLayout {
   size_t nsel = 0;      // [batch][Hkv] i32
   size_t part_ml = 0;   // [batch][Hq][splits][2] f32
   size_t part_o = 0;    // [batch][Hq][splits][d] f32
+  size_t row_ctr = 0;   // [batch][Hkv] u32 attention split counters
   size_t total = 0;
   int nb_stride = 0;
   int splits = 0;       // attention splits per row
@@ -136,28 +137,40 @@ struct AttnParams {
   const int32_t* seq_lens;
   float* part_ml;
   float* part_o;
+  uint32_t* row_ctr;         // [batch * Hkv] splits finished (self-resetting)
+  void* out;
   uint32_t* hdr;
   int batch, Hkv, G, S, budget, splits, tokens_per_split, max_pages_per_seq, num_pages;
+  int out_bf16;
   float scale_log2;          // softmax scale * log2(e)
 };
 
-struct CombineParams {
-  const float* part_ml;
-  const float* part_o;
-  void* out;
-  int rows_q;                // batch * Hq
-  int splits, d, out_bf16;
-};
+// Launch `kern` on `s`; with `pdl` the launch may overlap the tail of the previous kernel
+// in the stream (the kernel must call pdl_wait() before reading that kernel's results).
+template <typename... P, typename... A>
+inline cudaError_t launch_k(void (*kern)(P...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t s, bool pdl, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
 
 // ------------------------------------------------------------ launchers (return launch error)
 cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s);
 cudaError_t launch_block_err(const Plan& p, const BlockErrParams& a, cudaStream_t s);
 cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s);
 cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s);
-cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s);
-cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s);
-cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s);
-cudaError_t launch_combine(const Plan& p, const CombineParams& a, cudaStream_t s);
+cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl);
+cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s, bool pdl);
+cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl);
 
 int num_sms();
 

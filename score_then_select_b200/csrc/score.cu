@@ -13,9 +13,9 @@
 //   - one elected producer lane per CTA streams each unit's contiguous page chunk
 //     (128 tokens x r entries, 8 or 16 KiB) with a bulk TMA copy into a shared-memory
 //     ring, completion tracked by mbarrier transaction counts;
-//   - consumer warps read 16-byte vectors from shared memory (LPT lanes per token),
-//     dot them with their slice of q~ in FP32, sum across the token's lanes and reduce the
-//     block max with warp shuffles.
+//   - each consumer lane owns whole tokens: it reads the token's 16-byte chunks from shared
+//     memory in a lane-rotated order (conflict-free 128-bit loads), dots them with q~ in
+//     FP32 with one accumulator per chunk, and the block max is a warp-shuffle reduction.
 #include "qs_device.cuh"
 
 namespace qs {
@@ -88,16 +88,19 @@ QS_DEV Unit decode_unit(const ScoreParams& a, const int* prefix, int u, int& b) 
 }
 
 template <typename PT, int R>
-__global__ void __launch_bounds__(kScoreThreads) score_rankr_kernel(const ScoreParams a) {
+__global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const ScoreParams a) {
   using SH = ProxyShape<PT, R>;
   constexpr int NST = SH::kStages;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* slots = smem;                                          // [NST][page bytes]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + NST * SH::kPageBytes);
   uint64_t* empty = full + NST;
-  int* prefix = reinterpret_cast<int*>(empty + NST);              // [batch + 1]
+  int4* info = reinterpret_cast<int4*>(empty + NST);              // [NST] {row, page idx, nv, ok}
+  int* prefix = reinterpret_cast<int*>(info + NST);               // [batch + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();      // q~ and seq_lens come from the kernel before
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
@@ -114,91 +117,128 @@ __global__ void __launch_bounds__(kScoreThreads) score_rankr_kernel(const ScoreP
   const int n_units = u1 - u0;
 
   if (warp == 0) {
-    // ---------------- producer: one lane issues the bulk copies
-    if (lane == 0) {
-      int b = 0;
-      for (int k = 0; k < n_units; ++k) {
-        const int s = k % NST;
-        const uint32_t ph = uint32_t(k / NST) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u)) {
-          flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_SCORE, uint32_t(k));
-          break;
+    // ---------------- producer warp: the 32 lanes resolve 32 units' pages in parallel,
+    // then lane 0 issues their bulk copies in order
+    int b = 0;
+    bool dead = false;
+    for (int k0 = 0; k0 < n_units && !dead; k0 += 32) {
+      Unit x{};
+      x.ok = false;
+      x.nv = 0;
+      if (k0 + lane < n_units) x = decode_unit(a, prefix, u0 + k0 + lane, b);
+      const int row = x.b * a.Hkv + x.g;
+      const int m = min(32, n_units - k0);
+      for (int j = 0; j < m; ++j) {
+        const int jrow = __shfl_sync(kFull, row, j);
+        const int jp = __shfl_sync(kFull, x.p, j);
+        const int jnv = __shfl_sync(kFull, x.nv, j);
+        const int jok = __shfl_sync(kFull, int(x.ok), j);
+        const int jpage = __shfl_sync(kFull, x.page, j);
+        const int jg = __shfl_sync(kFull, x.g, j);
+        if (lane == 0) {
+          const int k = k0 + j;
+          const int s = k % NST;
+          const uint32_t ph = uint32_t(k / NST) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u)) {
+            flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_SCORE, uint32_t(k));
+            dead = true;
+          } else {
+            info[s] = make_int4(jrow, jp, jnv, jok);
+            if (jok) {
+              const uint32_t bytes = uint32_t(jnv) * SH::kTokenBytes;
+              const uint8_t* src = reinterpret_cast<const uint8_t*>(a.proxy) +
+                                   (size_t(jpage) * a.Hkv + jg) * size_t(SH::kPageBytes);
+              mbar_arrive_expect_tx(&full[s], bytes);
+              bulk_g2s(slots + s * SH::kPageBytes, src, bytes, &full[s]);
+            } else {
+              flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SCORE, uint32_t(jrow));
+              mbar_arrive(&full[s]);
+            }
+          }
         }
-        const Unit x = decode_unit(a, prefix, u0 + k, b);
-        if (x.ok) {
-          const uint32_t bytes = uint32_t(x.nv) * SH::kTokenBytes;
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(a.proxy) +
-                               (size_t(x.page) * a.Hkv + x.g) * size_t(SH::kPageBytes);
-          mbar_arrive_expect_tx(&full[s], bytes);
-          bulk_g2s(slots + s * SH::kPageBytes, src, bytes, &full[s]);
-        } else {
-          flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SCORE, uint32_t(x.b));
-          mbar_arrive(&full[s]);
-        }
+        dead = __shfl_sync(kFull, int(dead), 0) != 0;
+        if (dead) break;
       }
     }
     return;
   }
 
-  // ---------------- consumers
+  // ---------------- consumers: each lane owns whole tokens (token m*32 + lane, m < 4) and
+  // reads its 16-byte chunks in a lane-rotated order so that every quarter-warp's
+  // 128-bit shared loads hit distinct banks; one accumulator per chunk position.
+  constexpr int CPT = SH::kTokenBytes / 16;           // 16-byte chunks per token: 4 or 8
+  constexpr int EPC = SH::kEPL;                       // elements per chunk: 8 (bf16) / 4 (f32)
   const int c = warp - 1;
-  const int part = lane % SH::kLPT;
-  const int tok_in_step = lane / SH::kLPT;
-  float qv[SH::kEPL];
+  const int rot = (SH::kTokenBytes == 64) ? (lane >> 1) : lane;
+  float qr[CPT][EPC];                                 // q~ permuted by this lane's rotation
   int cur_row = -1;
-  int b = 0;
   const int bpp = kPage / a.S;  // blocks per page
   for (int k = c; k < n_units; k += kScoreConsumers) {
     const int s = k % NST;
     const uint32_t ph = uint32_t(k / NST) & 1u;
-    const Unit x = decode_unit(a, prefix, u0 + k, b);
     if (!mbar_wait(&full[s], ph)) {
       if (lane == 0) flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_SCORE, uint32_t(k));
       break;
     }
-    const int row = x.b * a.Hkv + x.g;
-    if (x.ok) {
+    const int4 x = info[s];                  // {row, page index in row, valid tokens, ok}
+    const int row = x.x;
+    if (x.w) {
       if (row != cur_row) {
         cur_row = row;
 #pragma unroll
-        for (int e = 0; e < SH::kEPL; ++e) qv[e] = a.qt[size_t(row) * R + part * SH::kEPL + e];
+        for (int kk = 0; kk < CPT; ++kk) {
+          const int ch = (kk + rot) & (CPT - 1);
+#pragma unroll
+          for (int e = 0; e < EPC; ++e) qr[kk][e] = a.qt[size_t(row) * R + ch * EPC + e];
+        }
       }
       const uint8_t* slot = slots + s * SH::kPageBytes;
-      float* out = a.scores + size_t(row) * a.nb_stride + size_t(x.p) * bpp;
-      float m_run = -INFINITY;
+      float* out = a.scores + size_t(row) * a.nb_stride + size_t(x.y) * bpp;
+      const int nv = x.z;
+      float sc[kPage / 32];
 #pragma unroll
-      for (int i = 0; i < SH::kIter; ++i) {
-        const uint4 v = *reinterpret_cast<const uint4*>(slot + (i * 32 + lane) * 16);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float acc = 0.0f;
-        if constexpr (sizeof(PT) == 2) {
+      for (int m = 0; m < kPage / 32; ++m) {
+        const int tok = m * 32 + lane;
+        const uint8_t* tp = slot + tok * SH::kTokenBytes;
+        float acc[CPT];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            acc = fmaf(bf16_lo(w[e]), qv[2 * e], acc);
-            acc = fmaf(bf16_hi(w[e]), qv[2 * e + 1], acc);
+        for (int kk = 0; kk < CPT; ++kk) {
+          const uint4 v = *reinterpret_cast<const uint4*>(tp + (((kk + rot) & (CPT - 1)) << 4));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          float t = 0.0f;
+          if constexpr (sizeof(PT) == 2) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              t = fmaf(bf16_lo(w[e]), qr[kk][2 * e], t);
+              t = fmaf(bf16_hi(w[e]), qr[kk][2 * e + 1], t);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) t = fmaf(__uint_as_float(w[e]), qr[kk][e], t);
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc = fmaf(__uint_as_float(w[e]), qv[e], acc);
+          acc[kk] = t;
         }
+        float dot = 0.0f;
 #pragma unroll
-        for (int o = 1; o < SH::kLPT; o <<= 1) acc += __shfl_xor_sync(kFull, acc, o);
-        const int tok = i * SH::kTPW + tok_in_step;
-        const float sc = tok < x.nv ? acc : -INFINITY;
-        if (a.S >= SH::kTPW) {
-          m_run = fmaxf(m_run, sc);
-          if ((((i + 1) * SH::kTPW) & (a.S - 1)) == 0) {
+        for (int kk = 0; kk < CPT; ++kk) dot += acc[kk];
+        sc[m] = tok < nv ? dot : -INFINITY;
+      }
+      if (a.S >= 32) {
+        const int per = a.S / 32;                      // m-steps per block
+        for (int blk = 0; blk < kPage / a.S; ++blk) {
+          float mx = -INFINITY;
 #pragma unroll
-            for (int o = SH::kLPT; o < 32; o <<= 1)
-              m_run = fmaxf(m_run, __shfl_xor_sync(kFull, m_run, o));
-            if (lane == 0) out[(i * SH::kTPW) / a.S] = m_run;
-            m_run = -INFINITY;
-          }
-        } else {
-          float v2 = sc;
-          for (int o = SH::kLPT; o < SH::kLPT * a.S; o <<= 1)
-            v2 = fmaxf(v2, __shfl_xor_sync(kFull, v2, o));
-          if ((lane & (SH::kLPT * a.S - 1)) == 0) out[tok / a.S] = v2;
+          for (int m = 0; m < kPage / 32; ++m)
+            if (m / per == blk) mx = fmaxf(mx, sc[m]);
+          mx = warp_max(mx);
+          if (lane == 0) out[blk] = mx;
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < kPage / 32; ++m) {
+          float v2 = sc[m];
+          for (int o = 1; o < a.S; o <<= 1) v2 = fmaxf(v2, __shfl_xor_sync(kFull, v2, o));
+          if ((lane & (a.S - 1)) == 0) out[(m * 32 + lane) / a.S] = v2;
         }
       }
     }
@@ -208,34 +248,40 @@ __global__ void __launch_bounds__(kScoreThreads) score_rankr_kernel(const ScoreP
 }
 
 template <typename PT, int R>
-static cudaError_t launch_rankr_score(const ScoreParams& a, cudaStream_t st) {
+static cudaError_t launch_rankr_score(const ScoreParams& a, cudaStream_t st, bool pdl) {
   using SH = ProxyShape<PT, R>;
-  const size_t smem = size_t(SH::kStages) * SH::kPageBytes + 2 * SH::kStages * sizeof(uint64_t) +
-                      size_t(a.batch + 1) * sizeof(int);
+  const size_t smem_max = size_t(SH::kStages) * SH::kPageBytes +
+                          2 * SH::kStages * sizeof(uint64_t) + SH::kStages * sizeof(int4) +
+                          size_t(kMaxBatch + 1) * sizeof(int);
+  const size_t smem = smem_max - size_t(kMaxBatch - a.batch) * sizeof(int);
   auto k = score_rankr_kernel<PT, R>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kScoreThreads, smem);
-  if (e != cudaSuccess) return e;
+  // one-time per-process kernel attributes (sized for the largest batch)
+  static int per_sm = [&] {
+    int n = 0;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max)) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kScoreThreads, smem_max) != cudaSuccess)
+      n = 0;
+    return n;
+  }();
+  if (per_sm <= 0) return cudaErrorInvalidConfiguration;
   const long long units = (long long)a.batch * a.Hkv *
                           ((a.max_context + kPage - 1) / kPage);
   long long grid = (long long)num_sms() * (per_sm > 0 ? per_sm : 1);
   if (grid > units) grid = units;
   if (grid < 1) grid = 1;
-  k<<<int(grid), kScoreThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_k(k, dim3(unsigned(grid)), dim3(kScoreThreads), smem, st, pdl, a);
 }
 
-cudaError_t launch_score_nvfp4(const Plan& p, const ScoreParams& a, cudaStream_t s);
+cudaError_t launch_score_nvfp4(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl);
 
-cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s) {
-  if (p.r == 0) return launch_score_nvfp4(p, a, s);
+cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl) {
+  if (p.r == 0) return launch_score_nvfp4(p, a, s, pdl);
   const bool f32 = p.proxy_dtype == QS_F32;
-  if (f32 && p.r == 16) return launch_rankr_score<float, 16>(a, s);
-  if (f32 && p.r == 32) return launch_rankr_score<float, 32>(a, s);
-  if (!f32 && p.r == 32) return launch_rankr_score<uint16_t, 32>(a, s);
-  if (!f32 && p.r == 64) return launch_rankr_score<uint16_t, 64>(a, s);
+  if (f32 && p.r == 16) return launch_rankr_score<float, 16>(a, s, pdl);
+  if (f32 && p.r == 32) return launch_rankr_score<float, 32>(a, s, pdl);
+  if (!f32 && p.r == 32) return launch_rankr_score<uint16_t, 32>(a, s, pdl);
+  if (!f32 && p.r == 64) return launch_rankr_score<uint16_t, 64>(a, s, pdl);
   return cudaErrorInvalidValue;
 }
 

@@ -3,7 +3,7 @@
 
 namespace qs {
 
-cudaError_t launch_score_nvfp4(const Plan& p, const ScoreParams& a, cudaStream_t s) {
+cudaError_t launch_score_nvfp4(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl) {
   return cudaErrorNotSupported;
 }
 

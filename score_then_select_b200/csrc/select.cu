@@ -144,6 +144,8 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   __shared__ int s_bin, s_above, s_forced[4], s_nforced;
   BlockOps<NT> ops{s_i, s_f};
 
+  pdl_wait();      // the scores come from the kernel before
+  pdl_trigger();
   const int row = blockIdx.x;
   const int b = row / a.Hkv;
   const int tid = threadIdx.x;
@@ -309,13 +311,12 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   for (int i = tot + tid; i < k; i += NT) sel[i] = -1;
 }
 
-cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s) {
+cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s, bool pdl) {
   const int nbs = a.nb_stride;
-  if (nbs <= 256 * 4) select_kernel<256, 4><<<a.rows, 256, 0, s>>>(a);
-  else if (nbs <= 256 * 16) select_kernel<256, 16><<<a.rows, 256, 0, s>>>(a);
-  else if (nbs <= 1024 * 32) select_kernel<1024, 32><<<a.rows, 1024, 0, s>>>(a);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (nbs <= 256 * 4) return launch_k(select_kernel<256, 4>, dim3(a.rows), dim3(256), 0, s, pdl, a);
+  if (nbs <= 256 * 16) return launch_k(select_kernel<256, 16>, dim3(a.rows), dim3(256), 0, s, pdl, a);
+  if (nbs <= 1024 * 32) return launch_k(select_kernel<1024, 32>, dim3(a.rows), dim3(1024), 0, s, pdl, a);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace qs

@@ -38,7 +38,7 @@ class Filled:
         if w.proxy_dtype == "nvfp4":
             lay.key_center.copy_(torch.from_numpy(inp.mu))
             lay.key_gscale.fill_(float(inp.g_k))
-        self.P = torch.from_numpy(inp.P).to(device) if inp.P is not None else None
+        self.P = torch.from_numpy(np.array(inp.P)).to(device) if inp.P is not None else None
         self.q = u16(Q).to(device)
         self.cfg = lay.cfg
         self.cache = lay.cache()
