@@ -191,6 +191,30 @@ qs_status qs_decode(const qs_config *cfg, const qs_cache *cache, const void *q,
    5 select, 6 attention (with its log-sum-exp combine). */
 qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
 
+/* Sparse attention without a workspace, for callers that cannot allocate device memory:
+   for example a plugin of a host framework that owns all device memory and hands its
+   kernels only their inputs and outputs, or a decode loop that may not call cudaMalloc
+   because the allocation would synchronise the device. The pages describe no such call;
+   it exists for these callers only.
+   Computes exactly what qs_sparse_attn computes, with the same kernel; its split partials
+   and per-row counters live in one static device array of QS_ATTN_STATIC_SCRATCH_BYTES
+   inside the library (each GPU that loads the library holds it until the process exits),
+   so the call allocates nothing and takes no workspace. The first call on a device looks
+   up that array's device address (once per device, with the device current); make that
+   first call before any stream capture. Every call clears the array's counters before
+   its kernel runs, and all calls on a device share the array: calls whose work overlaps
+   on the GPU (different streams, or different threads without ordering) race and must
+   not be issued. Device-side bounds checks still skip invalid accesses, but their status
+   word is not reported by this call.
+   Returns QS_ERR_UNSUPPORTED if batch * Hq * splits * (head_dim + 2) * 4 bytes of partials
+   plus batch * Hkv * 4 bytes of counters exceed QS_ATTN_STATIC_SCRATCH_BYTES (the split
+   count is the one qs_sparse_attn plans for the shape), and QS_ERR_CUDA if the address
+   lookup or a launch fails; other arguments as for qs_sparse_attn. */
+#define QS_ATTN_STATIC_SCRATCH_BYTES (4u << 20)
+qs_status qs_sparse_attn_noalloc(const qs_config *cfg, const qs_cache *cache, const void *q,
+                                 const int32_t *sel, const int32_t *n_sel, int32_t batch,
+                                 void *out, qs_stream_t stream);
+
 /* Static string naming a status code. */
 const char *qs_status_string(qs_status s);
 

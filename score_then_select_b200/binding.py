@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
             "qs_sparse_attn": ([cfgp, cachep, vp, vp, vp, i32, vp, vp, vp], i32),
             "qs_decode": ([cfgp, cachep, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp], i32),
             "qs_device_status": ([vp, vp, ctypes.POINTER(ctypes.c_uint32)], i32),
+            "qs_sparse_attn_noalloc": ([cfgp, cachep, vp, vp, vp, i32, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -75,7 +76,7 @@ def lib() -> ctypes.CDLL:
 
 EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_init",
            "qs_append_kv", "qs_score", "qs_select_topk", "qs_sparse_attn", "qs_decode",
-           "qs_device_status")
+           "qs_device_status", "qs_sparse_attn_noalloc")
 
 
 def status_string(s: int) -> str:
@@ -177,6 +178,18 @@ def qs_decode(cfg, cache, q, k_new, v_new, P, batch, out, sel_out, n_sel_out, ws
     _check(lib().qs_decode(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(k_new),
                            _ptr(v_new), _ptr(P), batch, _ptr(out), _ptr(sel_out),
                            _ptr(n_sel_out), _ptr(ws), _stream(stream)), "qs_decode")
+
+
+def qs_sparse_attn_noalloc(cfg, cache, q, sel, n_sel, batch, out, stream=None):
+    """qs_sparse_attn without a workspace: the library's static device scratch is used.
+
+    For callers that cannot allocate device memory (a framework that owns all of it, or a
+    loop where an allocation would synchronise the device). Calls that overlap on the GPU
+    share that scratch and race.
+    """
+    _check(lib().qs_sparse_attn_noalloc(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q),
+                                        _ptr(sel), _ptr(n_sel), batch, _ptr(out),
+                                        _stream(stream)), "qs_sparse_attn_noalloc")
 
 
 def qs_device_status(ws, stream=None) -> tuple[int, int, int]:

@@ -49,7 +49,7 @@ static void plan_splits(int rows, int slots, int& splits, int& tps) {
   }
 }
 
-static qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
+qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   if (!c) return QS_ERR_INVALID_ARG;
   if (batch < 1 || batch > kMaxBatch || max_context < 1) return QS_ERR_INVALID_ARG;
   if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads) return QS_ERR_INVALID_ARG;
@@ -122,7 +122,7 @@ static qs_status make_plan(const qs_config* c, int batch, int max_context, Plan&
   return QS_OK;
 }
 
-static qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy) {
+qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy) {
   if (!c || !c->k || !c->v || !c->page_table || !c->seq_lens) return QS_ERR_INVALID_ARG;
   if (c->max_pages_per_seq < 1 || c->num_pages < 1 || c->max_context < 1) return QS_ERR_INVALID_ARG;
   if ((long long)c->num_pages * p.Hkv * kPage >= (1LL << 31)) return QS_ERR_UNSUPPORTED;

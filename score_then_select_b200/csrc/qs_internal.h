@@ -174,4 +174,8 @@ cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s, bool
 
 int num_sms();
 
+// host-side validation and launch planning (api.cu)
+qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p);
+qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy);
+
 }  // namespace qs
