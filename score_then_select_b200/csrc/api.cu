@@ -109,8 +109,7 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   size_t off = size_t(kHdrWords) * 4;
   const size_t rows = size_t(batch) * p.Hkv, rows_q = size_t(batch) * p.Hq;
   w.qt = off;      off = align_up(off + rows * (r > 0 ? r : 1) * 4, 256);
-  w.qcodes = off;  off = align_up(off + (r == 0 ? rows_q * p.d / 2 : 0), 256);
-  w.qscales = off; off = align_up(off + (r == 0 ? rows_q * p.d / 16 : 0), 256);
+  w.qtile = off;   off = align_up(off + (r == 0 ? rows * kQTileBytes : 0), 256);
   w.qgscale = off; off = align_up(off + 16, 256);
   w.scores = off;  off = align_up(off + rows * p.nb_stride * 4, 256);
   w.sel = off;     off = align_up(off + rows * p.budget * 4, 256);
@@ -199,9 +198,9 @@ static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws,
                  p.batch, p.Hkv, p.G, p.d, p.r};
     return cuda_status(launch_prep(p, a, s));
   }
-  QPackParams a{static_cast<const uint16_t*>(q), ws_at<uint8_t>(ws, p.ws.qcodes),
-                ws_at<uint8_t>(ws, p.ws.qscales), ws_at<float>(ws, p.ws.qgscale),
-                p.batch * p.Hq * p.d, p.d};
+  QPackParams a{static_cast<const uint16_t*>(q), ws_at<uint8_t>(ws, p.ws.qtile),
+                ws_at<float>(ws, p.ws.qgscale), p.batch * p.Hq * p.d, p.batch * p.Hkv, p.Hkv,
+                p.G};
   return cuda_status(launch_qpack(p, a, s));
 }
 
@@ -211,8 +210,7 @@ static qs_status do_score(const Plan& p, const qs_cache* c, float* scores, void*
   a.proxy = c->proxy;
   a.proxy_scale = c->proxy_scale;
   a.qt = ws_at<float>(ws, p.ws.qt);
-  a.qcodes = ws_at<uint8_t>(ws, p.ws.qcodes);
-  a.qscales = ws_at<uint8_t>(ws, p.ws.qscales);
+  a.qtile = ws_at<uint8_t>(ws, p.ws.qtile);
   a.qgscale = ws_at<float>(ws, p.ws.qgscale);
   a.key_gscale = c->key_gscale;
   a.page_table = c->page_table;

@@ -401,10 +401,12 @@ __global__ void __launch_bounds__(128) append_nvfp4_kernel(const AppendParams a)
       }
       uint32_t packed[2];
       const uint32_t sc = nvfp4_pack16(x, gk, packed);
-      const size_t tok = (size_t(page) * a.Hkv + g) * kPage + s_slot[n];
-      *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(a.proxy) + tok * (D / 2) + gr * 8) =
-          make_uint2(packed[0], packed[1]);
-      a.proxy_scale[tok * GR + gr] = uint8_t(sc);
+      // page-head layouts read directly by the FP4 tensor-core scan (see include/qs.h)
+      const size_t ph = size_t(page) * a.Hkv + g;
+      const int slot = s_slot[n];
+      *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(a.proxy) + ph * kNvfp4PageCodeBytes +
+                                nvfp4_code_off(slot, gr)) = make_uint2(packed[0], packed[1]);
+      a.proxy_scale[ph * kNvfp4PageScaleBytes + nvfp4_scale_off(slot, gr)] = uint8_t(sc);
     }
   }
   finish_append(a);
@@ -480,7 +482,9 @@ __global__ void __launch_bounds__(128) prep_rankr_kernel(const PrepParams a) {
 }
 
 // NVFP4 query packing: one CTA; g_q = max|q| / 2688 over the whole q tensor, then every
-// head's query is packed like the keys (without centring).
+// head's query is packed like the keys (without centring) into its row's query tile: the
+// group's heads as the B operand of the FP4 scan ([4 chunks][8 heads][16 B], heads past
+// the group zero) followed by their scales in the tensor-core scale-factor order.
 __global__ void __launch_bounds__(1024) qpack_kernel(const QPackParams a) {
   __shared__ float s_red[32];
   __shared__ float s_g;
@@ -497,16 +501,24 @@ __global__ void __launch_bounds__(1024) qpack_kernel(const QPackParams a) {
       *a.gscale = s_g;
     }
   }
+  // zero the tiles (padding heads and unused scale bytes), then fill them
+  for (size_t i = threadIdx.x; i < size_t(a.rows) * kQTileBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(a.tiles)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
   const float gq = s_g;
-  for (int grp = threadIdx.x; grp < a.n / 16; grp += blockDim.x) {
+  constexpr int GR = 8;  // 16-element groups per head (d = 128)
+  for (int it = threadIdx.x; it < a.rows * a.G * GR; it += blockDim.x) {
+    const int gr = it % GR, n = (it / GR) % a.G, row = it / (GR * a.G);
+    const int b = row / a.Hkv, g = row % a.Hkv;
+    const uint16_t* qh = a.q + (size_t(b) * a.Hkv * a.G + g * a.G + n) * 128 + gr * 16;
     float x[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = bf16_to_f32(a.q[size_t(grp) * 16 + i]);
+    for (int i = 0; i < 16; ++i) x[i] = bf16_to_f32(qh[i]);
     uint32_t packed[2];
     const uint32_t sc = nvfp4_pack16(x, gq, packed);
-    *reinterpret_cast<uint2*>(a.codes + size_t(grp) * 8) = make_uint2(packed[0], packed[1]);
-    a.scales[grp] = uint8_t(sc);
+    uint8_t* tile = a.tiles + size_t(row) * kQTileBytes;
+    *reinterpret_cast<uint2*>(tile + qtile_code_off(n, gr)) = make_uint2(packed[0], packed[1]);
+    tile[qtile_scale_off(n, gr)] = uint8_t(sc);
   }
 }
 

@@ -165,6 +165,69 @@ QS_DEV float ex2(float x) {
   return y;
 }
 
+// ---------------------------------------------------------------- tcgen05 (5th-gen tensor cores)
+// Tensor memory (TMEM) is allocated in columns by one full warp; addresses are
+// (lane << 16) | column. A warp may read only lanes 32*(warp%4) .. +31.
+QS_DEV void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_u32(smem_dst)), "r"(ncols) : "memory");
+}
+QS_DEV void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+QS_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+QS_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+QS_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, K-major, no swizzle: 8-row x 16-byte core matrices,
+// `lbo` bytes between the core matrices along K, `sbo` bytes between 8-row groups.
+QS_DEV uint64_t smem_desc_kmajor(const void* p, uint32_t lbo, uint32_t sbo) {
+  const uint64_t start = (smem_u32(p) >> 4) & 0x3FFFu;
+  return start | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) | (uint64_t((sbo >> 4) & 0x3FFFu) << 32) |
+         (uint64_t(1) << 46);  // descriptor version 1; base offset 0; layout: no swizzle
+}
+
+// Copy one 32-row x 16-byte block from shared memory to TMEM columns [taddr, taddr+4),
+// replicated to each of the four 32-lane groups.
+QS_DEV void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// D[tmem] (+)= A(smem, FP4 E2M1) x B(smem, FP4 E2M1)^T with per-16-element UE4M3 scales of A
+// and B read from TMEM; M = 128, K = 64 per instruction.
+QS_DEV void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                        uint32_t sfa_tmem, uint32_t sfb_tmem, bool accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n}\n"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(uint32_t(accumulate)),
+        "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Arrive on `bar` once every tcgen05 operation issued so far by this thread has completed.
+QS_DEV void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar)) : "memory");
+}
+
+// This warp's 32 lanes x 8 consecutive 32-bit columns.
+QS_DEV void tc_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  // the load and its completion wait sit in one asm block, so no use of r can be moved
+  // between them
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- warp reductions
 QS_DEV float warp_max(float v) {
 #pragma unroll

@@ -30,8 +30,7 @@ constexpr int kCtrAppend = 16;      // header word: append "last CTA" counter
 // Workspace carve-up (byte offsets); computed identically by qs_workspace_size and calls.
 struct WsLayout {
   size_t qt = 0;        // rank r: q~ [batch][Hkv][r] f32
-  size_t qcodes = 0;    // NVFP4: packed q codes [batch][Hq][d/2] u8
-  size_t qscales = 0;   // NVFP4: q scales [batch][Hq][d/16] u8
+  size_t qtile = 0;     // NVFP4: query tiles [batch][Hkv][kQTileBytes]
   size_t qgscale = 0;   // NVFP4: g_q (1 float)
   size_t scores = 0;    // [batch][Hkv][nb_stride] f32
   size_t sel = 0;       // [batch][Hkv][budget] i32
@@ -95,19 +94,44 @@ struct PrepParams {          // rank r scoring prep (standalone qs_score)
 
 struct QPackParams {         // NVFP4 query packing
   const uint16_t* q;
-  uint8_t* codes;
-  uint8_t* scales;
+  uint8_t* tiles;            // [batch * Hkv][kQTileBytes]
   float* gscale;
   int n;                     // batch * Hq * d
-  int d;
+  int rows, Hkv, G;
 };
+
+// ---- NVFP4 layouts (d = 128; documented in include/qs.h) -----------------------------
+// Codes of one (page, KV head): [4 chunks][128 tokens][16 bytes]; chunk c of a token holds
+// its elements 32c .. 32c+31 (two per byte, even element in the low nibble). A plain
+// contiguous copy of the 8 KiB lands in shared memory as the K-major, no-swizzle operand
+// of the FP4 tensor-core MMA (8-token x 16-byte core matrices).
+constexpr int kNvfp4PageCodeBytes = 128 * 64;
+// Scales of one (page, KV head): two 512-byte blocks (elements 0..63 and 64..127); in a
+// block, token m's 4 scales sit at 16 * (m % 32) + 4 * (m / 32): the order the tensor
+// cores' scale-factor copy expects.
+constexpr int kNvfp4PageScaleBytes = 1024;
+// Query tile of one row: 512 bytes of B-operand codes [4 chunks][8 heads][16 B] and two
+// 512-byte scale blocks (head n's 4 scales at 16 * n).
+constexpr int kQTileBytes = 512 + 1024;
+
+__host__ __device__ inline int nvfp4_code_off(int token, int group) {
+  return (group >> 1) * 2048 + token * 16 + (group & 1) * 8;
+}
+__host__ __device__ inline int nvfp4_scale_off(int token, int group) {
+  return (group >> 2) * 512 + 16 * (token & 31) + 4 * (token >> 5) + (group & 3);
+}
+__host__ __device__ inline int qtile_code_off(int head, int group) {
+  return (group >> 1) * 128 + head * 16 + (group & 1) * 8;
+}
+__host__ __device__ inline int qtile_scale_off(int head, int group) {
+  return 512 + (group >> 2) * 512 + 16 * head + (group & 3);
+}
 
 struct ScoreParams {
   const void* proxy;
   const uint8_t* proxy_scale;
   const float* qt;           // rank r: [batch][Hkv][r]
-  const uint8_t* qcodes;     // NVFP4
-  const uint8_t* qscales;
+  const uint8_t* qtile;      // NVFP4: [batch][Hkv][kQTileBytes]
   const float* qgscale;
   const float* key_gscale;
   const int32_t* page_table;

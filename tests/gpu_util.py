@@ -72,9 +72,17 @@ class Filled:
         npg = -(-L // 128)
         pages = torch.from_numpy(self.inp.page_table[b, :npg].astype(np.int64)).cuda()
         if self.w.proxy_dtype == "nvfp4":
-            c = self.layer.proxy[pages, g].reshape(npg * 128, -1)[:L].cpu().numpy()
-            s = self.layer.proxy_scale[pages, g].reshape(npg * 128, -1)[:L].cpu().numpy()
-            codes = np.empty((L, c.shape[1] * 2), dtype=np.uint8)
+            # page codes: [4 chunks][128 tokens][16 bytes], chunk c = bytes 16c..16c+15 of
+            # the token's 64-byte row; page scales: token m, group j at
+            # (j // 4) * 512 + 16 * (m % 32) + 4 * (m // 32) + j % 4 (layouts of include/qs.h)
+            raw = self.layer.proxy[pages, g].reshape(npg, 4, 128, 16).cpu().numpy()
+            c = raw.transpose(0, 2, 1, 3).reshape(npg * 128, 64)[:L]
+            rs = self.layer.proxy_scale[pages, g].reshape(npg, 1024).cpu().numpy()
+            m = np.arange(128)[:, None]
+            j = np.arange(8)[None, :]
+            idx = (j // 4) * 512 + 16 * (m % 32) + 4 * (m // 32) + j % 4
+            s = rs[:, idx].reshape(npg * 128, 8)[:L]
+            codes = np.empty((L, 128), dtype=np.uint8)
             codes[:, 0::2] = c & 15
             codes[:, 1::2] = c >> 4
             return codes, s

@@ -96,6 +96,49 @@ def test_rankr_parity(w):
             _check_out(w, out[b, g * G:(g + 1) * G], rr["out"], where)
 
 
+@pytest.mark.parametrize("w", NVFP4, ids=lambda w: w.name)
+def test_nvfp4_parity(w):
+    """NVFP4 path: codes and scales bit-exact, FP4 tensor-core block scores within 1e-4 of
+    the largest score, block errors within 1e-5 relative, kept blocks and selection valid
+    up to near-ties, attention within the BF16 bound."""
+    _gpu()
+    inp, f, out, sel, nsel, scores = _run_workload(w)
+    gq = query_scale_all(inp)
+    berr = f.layer.block_err.cpu().numpy()
+    G = w.group
+    for b in range(w.batch):
+        L = int(inp.lens[b])
+        nb = -(-L // w.block_size)
+        for g in range(w.n_kv_heads):
+            row = inp.row(b, g)
+            r = oracle_row(inp, b, g, row=row, g_q=gq)
+            where = f"{w.name} row ({b},{g})"
+            codes, scl = f.row_proxy(b, g)
+            ocodes, oscl, x32 = r["cache"]
+            assert np.array_equal(scl, oscl), f"{where}: scales differ"
+            assert np.array_equal(codes, ocodes), f"{where}: codes differ"
+            beta = scores[b, g, :nb]
+            tol = 1e-4 * max(np.abs(r["beta"]).max(), 1e-30)
+            bad = np.abs(beta - r["beta"]) > tol
+            assert not bad.any(), f"{where}: block scores {np.nonzero(bad)[0][:5]}"
+            # block errors (float32 sums vs float64) and the kept pair they imply
+            err_or = M.block_quant_error(x32, ocodes, oscl, inp.g_k, w.block_size, L)
+            nfull = L // w.block_size
+            eg = berr[b, g, :nfull]
+            assert np.allclose(eg, err_or[:nfull], rtol=1e-5, atol=0), f"{where}: block errors"
+            kept = M.kept_blocks(np.concatenate([eg.astype(np.float64), err_or[nfull:]]),
+                                 w.n_keep_hp)
+            okk, why = M.selection_valid(err_or[:nfull], w.n_keep_hp, np.zeros(0, np.int64), kept)
+            assert okk, f"{where}: kept blocks {why}"
+            forced = M.forced_blocks(nb, w.force_sink, w.force_last, kept)
+            n = int(nsel[b, g])
+            got = sel[b, g, :n]
+            ok, why = M.selection_valid(r["beta"], w.budget, forced, got)
+            assert ok, f"{where}: selection {why}"
+            rr = oracle_row(inp, b, g, row=row, g_q=gq, sel_override=got)
+            _check_out(w, out[b, g * G:(g + 1) * G], rr["out"], where)
+
+
 def test_needle_selected_on_gpu():
     _gpu()
     inp, f, out, sel, nsel, scores = _run_workload(synth.TINY_NEEDLE)
