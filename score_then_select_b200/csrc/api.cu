@@ -334,6 +334,7 @@ qs_status qs_score(const qs_config* cfg, const qs_cache* cache, const void* q, c
   if ((st = check_cache(p, cache, true)) != QS_OK) return st;
   if (!q || !aligned(q, 4) || !block_scores || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
+  if (p.r == 0 && !aligned(q, 16)) return QS_ERR_INVALID_ARG;
   if ((st = do_prep(p, q, P, ws, stream)) != QS_OK) return st;
   return do_score(p, cache, block_scores, ws, stream, true);
 }
@@ -370,7 +371,7 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   if (!q || !aligned(q, 4) || !k_new || !v_new || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
-  if (p.r == 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
+  if (p.r == 0 && (!cache->block_err || !aligned(q, 16))) return QS_ERR_INVALID_ARG;
   if ((sel_out == nullptr) != (n_sel_out == nullptr)) return QS_ERR_INVALID_ARG;
   int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, p.ws.sel);
   int32_t* nsel = n_sel_out ? n_sel_out : ws_at<int32_t>(ws, p.ws.nsel);

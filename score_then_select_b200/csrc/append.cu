@@ -481,34 +481,48 @@ __global__ void __launch_bounds__(128) prep_rankr_kernel(const PrepParams a) {
            a.d, a.r);
 }
 
-// NVFP4 query packing: one CTA; g_q = max|q| / 2688 over the whole q tensor, then every
-// head's query is packed like the keys (without centring) into its row's query tile: the
-// group's heads as the B operand of the FP4 scan ([4 chunks][8 heads][16 B], heads past
-// the group zero) followed by their scales in the tensor-core scale-factor order.
-__global__ void __launch_bounds__(1024) qpack_kernel(const QPackParams a) {
-  __shared__ float s_red[32];
+// NVFP4 query packing: CTA = one row (sequence, KV head). g_q = max|q| / 2688 over the
+// whole q tensor (every CTA computes the same maximum from L2-resident q; CTA 0 stores
+// it), then the group's heads are packed like the keys (without centring) into the row's
+// query tile: [4 chunks][8 heads][16 B] B-operand codes (heads past the group zero)
+// followed by their scales in the tensor-core scale-factor order.
+__global__ void __launch_bounds__(256) qpack_kernel(const QPackParams a) {
+  __shared__ float s_red[8];
   __shared__ float s_g;
+  const int tid = threadIdx.x, row = blockIdx.x;
   float m = 0.0f;
-  for (int i = threadIdx.x; i < a.n; i += blockDim.x) m = fmaxf(m, fabsf(bf16_to_f32(a.q[i])));
-  m = warp_max(m);
-  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < (blockDim.x >> 5) ? s_red[threadIdx.x] : 0.0f;
-    v = warp_max(v);
-    if (threadIdx.x == 0) {
-      s_g = __fdiv_rn(v, 2688.0f);
-      *a.gscale = s_g;
+  const uint4* q4 = reinterpret_cast<const uint4*>(a.q);
+  const int n4 = a.n / 8;
+  for (int i0 = 0; i0 < n4; i0 += 256 * 4) {
+    uint4 w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = i0 + j * 256 + tid;
+      w[j] = i < n4 ? q4[i] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t x[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16_lo(x[e])), fabsf(bf16_hi(x[e]))));
     }
   }
-  // zero the tiles (padding heads and unused scale bytes), then fill them
-  for (size_t i = threadIdx.x; i < size_t(a.rows) * kQTileBytes / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(a.tiles)[i] = make_uint4(0u, 0u, 0u, 0u);
+  m = warp_max(m);
+  if ((tid & 31) == 0) s_red[tid >> 5] = m;
+  uint4* tile4 = reinterpret_cast<uint4*>(a.tiles + size_t(row) * kQTileBytes);
+  for (int i = tid; i < kQTileBytes / 16; i += 256) tile4[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  if (tid == 0) {
+    float v = s_red[0];
+    for (int w = 1; w < 8; ++w) v = fmaxf(v, s_red[w]);
+    s_g = __fdiv_rn(v, 2688.0f);
+    if (row == 0) *a.gscale = s_g;
+  }
   __syncthreads();
   const float gq = s_g;
   constexpr int GR = 8;  // 16-element groups per head (d = 128)
-  for (int it = threadIdx.x; it < a.rows * a.G * GR; it += blockDim.x) {
-    const int gr = it % GR, n = (it / GR) % a.G, row = it / (GR * a.G);
+  if (tid < a.G * GR) {
+    const int gr = tid % GR, n = tid / GR;
     const int b = row / a.Hkv, g = row % a.Hkv;
     const uint16_t* qh = a.q + (size_t(b) * a.Hkv * a.G + g * a.G + n) * 128 + gr * 16;
     float x[16];
@@ -582,7 +596,7 @@ cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s) {
 }
 
 cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s) {
-  qpack_kernel<<<1, 1024, 0, s>>>(a);
+  qpack_kernel<<<a.rows, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

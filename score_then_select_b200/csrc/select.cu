@@ -9,7 +9,8 @@
 // kept) plus the k - |F| best other blocks by score, equal scores ordered by lower index;
 // ascending.
 //
-// Algorithm, one CTA per row, each thread owning ITEMS consecutive blocks in registers:
+// Algorithm, one CTA per row; thread t owns blocks t, t + NT, t + 2 NT, ... in registers
+// (coalesced loads); shared-memory bitmaps restore index order at the end:
 //   1. forced blocks are marked (the kept blocks are the n_keep complete blocks with the
 //      largest block error, found by two block-wide arg-max reductions);
 //   2. one pass of a 2048-bin histogram that is linear in the score between the active
@@ -17,8 +18,11 @@
 //      selects every bin above the threshold bin and leaves only the threshold bin active;
 //   3. an exact MSB-first radix select (4 x 8-bit digits) over order-preserving uint32
 //      keys of the remaining active blocks narrows them to one key value;
-//   4. the remaining slots go to the lowest-indexed blocks holding that key;
-//   5. a block-wide scan over the per-thread counts writes the ascending indices.
+//   4. the remaining slots go to the lowest-indexed blocks holding that key (a scan over
+//      the bitmap of remaining candidates);
+//   5. a scan over the bitmap of chosen blocks writes the ascending indices.
+// The count left in the threshold bin is read from the histogram, so no extra block-wide
+// reduction is needed between passes.
 #include <cfloat>
 
 #include "qs_device.cuh"
@@ -138,10 +142,14 @@ QS_DEV void find_threshold_bin(const int* hist, int nbins, int need, int* s_bin,
 template <int NT, int ITEMS>
 __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   constexpr int NW = NT / 32;
+  constexpr int CAP = NT * ITEMS;                 // blocks one CTA can hold
+  constexpr int NWORDS = CAP / 32;                // bitmap words
+  constexpr int WPT = (NWORDS + NT - 1) / NT;     // bitmap words per thread (contiguous)
   __shared__ int s_i[NW + 1];
   __shared__ float s_f[2 * NW];
   __shared__ int hist[kLinBins];
-  __shared__ int s_bin, s_above, s_forced[4], s_nforced;
+  __shared__ uint32_t chosen_bits[NWORDS], active_bits[NWORDS];
+  __shared__ int s_bin, s_above, s_cnt, s_forced[4], s_nforced;
   BlockOps<NT> ops{s_i, s_f};
 
   pdl_wait();      // the scores come from the kernel before
@@ -150,7 +158,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   const int b = row / a.Hkv;
   const int tid = threadIdx.x;
   int L = a.seq_lens[b];
-  const int nb_cap = a.nb_stride < NT * ITEMS ? a.nb_stride : NT * ITEMS;
+  const int nb_cap = a.nb_stride < CAP ? a.nb_stride : CAP;
   int nb = (L + a.S - 1) / a.S;
   if (L < 0 || nb > nb_cap) {
     if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
@@ -167,8 +175,17 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     return;
   }
 
-  // ---------------- forced blocks
-  const int j0 = tid * ITEMS;
+  // item i of this thread is block j = i * NT + tid (coalesced loads)
+  const float* sc = a.scores + size_t(row) * a.nb_stride;
+  float v[ITEMS];
+#pragma unroll
+  for (int i = 0; i < ITEMS; ++i) {
+    const int j = i * NT + tid;
+    v[i] = j < nb ? sc[j] : -FLT_MAX;
+  }
+  for (int w = tid; w < NWORDS; w += NT) chosen_bits[w] = active_bits[w] = 0u;
+
+  // ---------------- forced blocks: sink, last, and the kept (largest-error) blocks
   if (a.n_keep > 0 && a.block_err != nullptr) {
     const float* err = a.block_err + size_t(row) * a.nb_stride;
     const int ncomplete = min(L / a.S, nb);
@@ -176,11 +193,11 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     for (int r = 0; r < a.n_keep; ++r) {
       float bv = -INFINITY;
       int bi = -1;
-      for (int i = 0; i < ITEMS; ++i) {
-        const int j = j0 + i;
-        if (j < ncomplete && j != kept0) {
-          const float e = err[j];
-          if (bi < 0 || order_key(e) > order_key(bv)) { bv = e; bi = j; }
+      for (int j = tid; j < ncomplete; j += NT) {
+        const float e = err[j];
+        if (j != kept0 && (bi < 0 || order_key(e) > order_key(bv))) {
+          bv = e;
+          bi = j;
         }
       }
       const int best = ops.argmax(bv, bi);
@@ -192,10 +209,8 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   if (tid == 0) {
     s_forced[0] = a.force_sink ? 0 : -1;
     s_forced[1] = a.force_last ? nb - 1 : -1;
-    if (!(a.n_keep > 0 && a.block_err != nullptr)) { s_forced[2] = -1; s_forced[3] = -1; }
-    if (a.n_keep < 2) s_forced[3] = -1;
-    if (a.n_keep < 1) s_forced[2] = -1;
-    // dedupe
+    if (!(a.n_keep > 0 && a.block_err != nullptr) || a.n_keep < 1) s_forced[2] = -1;
+    if (!(a.n_keep > 0 && a.block_err != nullptr) || a.n_keep < 2) s_forced[3] = -1;
     int n = 0;
     for (int i = 0; i < 4; ++i) {
       const int f = s_forced[i];
@@ -207,30 +222,24 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   }
   __syncthreads();
   int need = k - s_nforced;
-  if (need < 0) need = 0;
-
-  // ---------------- load scores into registers
-  const float* sc = a.scores + size_t(row) * a.nb_stride;
-  float v[ITEMS];
   uint32_t active = 0u, chosen = 0u;
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) {
-    const int j = j0 + i;
-    v[i] = -FLT_MAX;
+    const int j = i * NT + tid;
     if (j < nb) {
-      float x = sc[j];
-      if (x != x) x = -FLT_MAX;
-      x = fminf(fmaxf(x, -FLT_MAX), FLT_MAX);
-      v[i] = x;
       bool f = false;
 #pragma unroll
       for (int q = 0; q < 4; ++q) f |= (s_forced[q] == j);
       if (f) chosen |= 1u << i; else active |= 1u << i;
+      float x = v[i];
+      if (x != x) x = -FLT_MAX;                      // NaN ranks lowest
+      v[i] = fminf(fmaxf(x, -FLT_MAX), FLT_MAX);
     }
   }
+  int n_active = nb - s_nforced;                     // known exactly: no reduction needed
 
-  // ---------------- linear-bin pass
-  if (need > 0) {
+  // ---------------- linear-bin pass: everything above the threshold bin is chosen
+  if (need > 0 && n_active > need) {
     float lo = FLT_MAX, hi = -FLT_MAX;
 #pragma unroll
     for (int i = 0; i < ITEMS; ++i)
@@ -240,32 +249,35 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
       for (int i = tid; i < kLinBins; i += NT) hist[i] = 0;
       __syncthreads();
       const double scale = double(kLinBins) / (double(hi) - double(lo));
-      int bins[ITEMS];
+      // monotone in the score, so a higher bin always holds higher scores (recomputed
+      // below rather than kept, to stay within the 64 registers of a 1024-thread CTA)
+      auto bin_of = [&](float x) {
+        int bn = int((double(x) - double(lo)) * scale);
+        return bn < 0 ? 0 : (bn >= kLinBins ? kLinBins - 1 : bn);
+      };
 #pragma unroll
-      for (int i = 0; i < ITEMS; ++i) {
-        int bn = int((double(v[i]) - double(lo)) * scale);
-        bn = bn < 0 ? 0 : (bn >= kLinBins ? kLinBins - 1 : bn);
-        bins[i] = bn;
-        if (active >> i & 1u) atomicAdd(&hist[bn], 1);
-      }
+      for (int i = 0; i < ITEMS; ++i)
+        if (active >> i & 1u) atomicAdd(&hist[bin_of(v[i])], 1);
       __syncthreads();
       find_threshold_bin<NT>(hist, kLinBins, need, &s_bin, &s_above, ops);
       const int bstar = s_bin;
+      const int above = s_above;
+      const int cnt = hist[bstar];
 #pragma unroll
       for (int i = 0; i < ITEMS; ++i) {
         if (!(active >> i & 1u)) continue;
-        if (bins[i] > bstar) { chosen |= 1u << i; active &= ~(1u << i); }
-        else if (bins[i] < bstar) active &= ~(1u << i);
+        const int bn = bin_of(v[i]);
+        if (bn > bstar) { chosen |= 1u << i; active &= ~(1u << i); }
+        else if (bn < bstar) active &= ~(1u << i);
       }
-      need -= s_above;
+      need -= above;
+      n_active = cnt;
       __syncthreads();
     }
   }
 
   // ---------------- exact radix select on order keys over what is left
-  for (int shift = 24; shift >= 0 && need > 0; shift -= 8) {
-    const int na = ops.sum(__popc(active));
-    if (na == need) break;
+  for (int shift = 24; shift >= 0 && need > 0 && n_active > need; shift -= 8) {
     for (int i = tid; i < 256; i += NT) hist[i] = 0;
     __syncthreads();
 #pragma unroll
@@ -274,6 +286,8 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     __syncthreads();
     find_threshold_bin<NT>(hist, 256, need, &s_bin, &s_above, ops);
     const uint32_t dstar = uint32_t(s_bin);
+    const int above = s_above;
+    const int cnt = hist[dstar];
 #pragma unroll
     for (int i = 0; i < ITEMS; ++i) {
       if (!(active >> i & 1u)) continue;
@@ -281,32 +295,58 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
       if (dg > dstar) { chosen |= 1u << i; active &= ~(1u << i); }
       else if (dg < dstar) active &= ~(1u << i);
     }
-    need -= s_above;
+    need -= above;
+    n_active = cnt;
     __syncthreads();
   }
-  // remaining actives share one key (or exactly fill the need): lowest indices first
-  if (need > 0) {
-    int tot;
-    const int before = ops.exclusive_sum(__popc(active), &tot);
-    int rank = before;
+
+  // ---------------- index order: chosen blocks, plus the `need` lowest-indexed actives
 #pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      if (active >> i & 1u) {
-        if (rank < need) chosen |= 1u << i;
-        ++rank;
+  for (int i = 0; i < ITEMS; ++i) {
+    const int j = i * NT + tid;
+    if (chosen >> i & 1u) atomicOr(&chosen_bits[j >> 5], 1u << (j & 31));
+    if (need > 0 && (active >> i & 1u)) atomicOr(&active_bits[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  const int w0 = tid * WPT;
+  if (need > 0) {
+    // remaining actives share one key (or exactly fill the need): lowest indices first
+    int cnt = 0;
+#pragma unroll
+    for (int w = 0; w < WPT; ++w)
+      if (w0 + w < NWORDS) cnt += __popc(active_bits[w0 + w]);
+    int tot;
+    int before = ops.exclusive_sum(cnt, &tot);
+#pragma unroll
+    for (int w = 0; w < WPT; ++w) {
+      if (w0 + w >= NWORDS) break;
+      uint32_t bits = active_bits[w0 + w];
+      while (bits != 0u && before < need) {
+        const uint32_t low = bits & (~bits + 1u);
+        chosen_bits[w0 + w] |= low;
+        bits ^= low;
+        ++before;
       }
     }
+    __syncthreads();
   }
-
-  // ---------------- ascending output
-  int tot;
-  int pos = ops.exclusive_sum(__popc(chosen), &tot);
+  int cnt = 0;
 #pragma unroll
-  for (int i = 0; i < ITEMS; ++i)
-    if (chosen >> i & 1u) {
-      if (pos < k) sel[pos] = j0 + i;
+  for (int w = 0; w < WPT; ++w)
+    if (w0 + w < NWORDS) cnt += __popc(chosen_bits[w0 + w]);
+  int tot;
+  int pos = ops.exclusive_sum(cnt, &tot);
+#pragma unroll
+  for (int w = 0; w < WPT; ++w) {
+    if (w0 + w >= NWORDS) break;
+    uint32_t bits = chosen_bits[w0 + w];
+    while (bits != 0u) {
+      const int bit = __ffs(bits) - 1;
+      if (pos < k) sel[pos] = (w0 + w) * 32 + bit;
       ++pos;
+      bits &= bits - 1u;
     }
+  }
   if (tot != n_out && tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
   for (int i = tot + tid; i < k; i += NT) sel[i] = -1;
 }
