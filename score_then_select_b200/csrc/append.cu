@@ -413,61 +413,61 @@ __global__ void __launch_bounds__(128) append_nvfp4_kernel(const AppendParams a)
 }
 
 // ============================================================ NVFP4 block error
-// CTA = one (row, block) pair that this append may have completed. Thread = token; the
-// squared errors are reduced in a fixed order (deterministic float32 result).
-__global__ void __launch_bounds__(128) block_err_kernel(const BlockErrParams a) {
+// CTA = one (row, block) pair that this append may have completed; 256 threads, each
+// owning (token, 16-element group) items i = tid + 256 m. An item's error is summed over
+// its 16 elements in order, a thread's items in order, then warps by butterfly and the
+// 8 warp sums in order: a fixed, deterministic float32 reduction.
+__global__ void __launch_bounds__(256) block_err_kernel(const BlockErrParams a) {
   constexpr int D = 128, GR = D / 16;
   __shared__ float s_mu[D];
-  __shared__ float s_red[4];
+  __shared__ float s_red[8];
+  pdl_wait();      // the cache and seq_lens come from the append kernel before
   const int row = blockIdx.y;
   const int b = row / a.Hkv, g = row % a.Hkv;
-  int n_b = a.n_new ? a.n_new[b] : 1;
+  const int n_b = a.n_new ? a.n_new[b] : 1;
   const int new_len = a.seq_lens[b];
   const int old = new_len - n_b;
   const int j = old / a.S + blockIdx.x;
   if (n_b <= 0 || old < 0 || (j + 1) * a.S > new_len || j >= a.nb_stride) return;  // not completed here
   const float gk = *a.key_gscale;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) s_mu[i] = a.key_center[size_t(row) * D + i];
+  if (threadIdx.x < D) s_mu[threadIdx.x] = a.key_center[size_t(row) * D + threadIdx.x];
   __syncthreads();
   float err = 0.0f;
-  for (int tt = threadIdx.x; tt < a.S; tt += blockDim.x) {
+  for (int i = threadIdx.x; i < a.S * GR; i += 256) {
+    const int tt = i / GR, gr = i % GR;
     const int t = j * a.S + tt;
     const int pi = t / kPage;
     if (pi >= a.max_pages_per_seq) { flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_BLOCKERR, b); continue; }
     const int page = a.page_table[size_t(b) * a.max_pages_per_seq + pi];
     if (page < 0 || page >= a.num_pages) { flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_BLOCKERR, b); continue; }
-    const uint16_t* kr = a.k + ((size_t(page) * a.Hkv + g) * kPage + t % kPage) * D;
-    float e_tok = 0.0f;
-#pragma unroll 1
-    for (int gr = 0; gr < GR; ++gr) {
-      const uint4 k0 = *reinterpret_cast<const uint4*>(kr + gr * 16);
-      const uint4 k1 = *reinterpret_cast<const uint4*>(kr + gr * 16 + 8);
-      const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-      float x[16];
+    const uint16_t* kr = a.k + ((size_t(page) * a.Hkv + g) * kPage + t % kPage) * D + gr * 16;
+    const uint4 k0 = *reinterpret_cast<const uint4*>(kr);
+    const uint4 k1 = *reinterpret_cast<const uint4*>(kr + 8);
+    const uint32_t w[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+    float x[16];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        x[2 * e] = __fsub_rn(bf16_lo(w[e]), s_mu[gr * 16 + 2 * e]);
-        x[2 * e + 1] = __fsub_rn(bf16_hi(w[e]), s_mu[gr * 16 + 2 * e + 1]);
-      }
-      uint32_t packed[2];
-      const float sv = ue4m3_decode(nvfp4_pack16(x, gk, packed));
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float dq = __fmul_rn(__fmul_rn(e2m1_decode((packed[i >> 3] >> (4 * (i & 7))) & 15u), sv), gk);
-        const float df = __fsub_rn(x[i], dq);
-        e_tok = __fadd_rn(e_tok, __fmul_rn(df, df));
-      }
+    for (int e = 0; e < 8; ++e) {
+      x[2 * e] = __fsub_rn(bf16_lo(w[e]), s_mu[gr * 16 + 2 * e]);
+      x[2 * e + 1] = __fsub_rn(bf16_hi(w[e]), s_mu[gr * 16 + 2 * e + 1]);
     }
-    err = __fadd_rn(err, e_tok);
-  }
-  // fixed-order reduction: warp butterfly then warps in index order
+    uint32_t packed[2];
+    const float sv = ue4m3_decode(nvfp4_pack16(x, gk, packed));
+    float e_it = 0.0f;
 #pragma unroll
-  for (int m = 16; m > 0; m >>= 1) err += __shfl_xor_sync(kFull, err, m);
+    for (int e = 0; e < 16; ++e) {
+      const float dq = __fmul_rn(__fmul_rn(e2m1_decode((packed[e >> 3] >> (4 * (e & 7))) & 15u), sv), gk);
+      const float df = __fsub_rn(x[e], dq);
+      e_it = __fadd_rn(e_it, __fmul_rn(df, df));
+    }
+    err = __fadd_rn(err, e_it);
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) err = __fadd_rn(err, __shfl_xor_sync(kFull, err, m));
   if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = err;
   __syncthreads();
   if (threadIdx.x == 0) {
     float tot = 0.0f;
-    for (int w = 0; w < int(blockDim.x >> 5); ++w) tot += s_red[w];
+    for (int w = 0; w < 8; ++w) tot = __fadd_rn(tot, s_red[w]);
     a.block_err[size_t(row) * a.nb_stride + j] = tot;
   }
 }
@@ -585,9 +585,8 @@ cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) 
 }
 
 cudaError_t launch_block_err(const Plan& p, const BlockErrParams& a, cudaStream_t s) {
-  dim3 grid(a.max_blocks_per_call, a.batch * a.Hkv);
-  block_err_kernel<<<grid, 128, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(block_err_kernel, dim3(a.max_blocks_per_call, a.batch * a.Hkv), dim3(256), 0, s,
+                  true, a);
 }
 
 cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s) {

@@ -16,8 +16,10 @@
 //   2. one pass of a 2048-bin histogram that is linear in the score between the active
 //      minimum and maximum (a monotone map, so every block in a higher bin scores higher)
 //      selects every bin above the threshold bin and leaves only the threshold bin active;
-//   3. an exact MSB-first radix select (4 x 8-bit digits) over order-preserving uint32
-//      keys of the remaining active blocks narrows them to one key value;
+//   3. the few blocks left in the threshold bin are ranked pairwise (score descending,
+//      index ascending) and the first ones taken; only if many are left (many equal or
+//      nearly equal scores) does an exact MSB-first radix select (4 x 8-bit digits) over
+//      order-preserving uint32 keys narrow them to one key value;
 //   4. the remaining slots go to the lowest-indexed blocks holding that key (a scan over
 //      the bitmap of remaining candidates);
 //   5. a scan over the bitmap of chosen blocks writes the ascending indices.
@@ -30,6 +32,7 @@
 namespace qs {
 
 constexpr int kLinBins = 2048;
+constexpr int kRankCap = 1024;     // candidates ranked pairwise after the histogram pass
 
 // float -> uint32 whose unsigned order is the float order (NaN ranks as -FLT_MAX, -0 == +0)
 QS_DEV uint32_t order_key(float v) {
@@ -149,6 +152,8 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   __shared__ float s_f[2 * NW];
   __shared__ int hist[kLinBins];
   __shared__ uint32_t chosen_bits[NWORDS], active_bits[NWORDS];
+  __shared__ float list_v[kRankCap];
+  __shared__ int list_j[kRankCap];
   __shared__ int s_bin, s_above, s_cnt, s_forced[4], s_nforced;
   BlockOps<NT> ops{s_i, s_f};
 
@@ -276,7 +281,37 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     }
   }
 
-  // ---------------- exact radix select on order keys over what is left
+  // ---------------- few candidates left (the usual case): rank them all pairwise under the
+  // order (higher score, then lower index) and keep the first `need`
+  if (need > 0 && n_active > need && n_active <= kRankCap) {
+    if (tid == 0) s_cnt = 0;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < ITEMS; ++i) {
+      if (active >> i & 1u) {
+        const int slot = atomicAdd(&s_cnt, 1);
+        list_v[slot] = v[i];
+        list_j[slot] = i * NT + tid;
+      }
+    }
+    __syncthreads();
+    const int n = s_cnt;
+    for (int c = tid; c < n; c += NT) {
+      const float vc = list_v[c];
+      const int jc = list_j[c];
+      int rank = 0;
+      for (int o = 0; o < n; ++o) {
+        const float vo = list_v[o];
+        rank += (vo > vc) || (vo == vc && list_j[o] < jc);
+      }
+      if (rank < need) atomicOr(&chosen_bits[jc >> 5], 1u << (jc & 31));
+    }
+    need = 0;
+    active = 0u;
+  }
+
+  // ---------------- exact radix select on order keys over what is left (many equal or
+  // nearly equal scores)
   for (int shift = 24; shift >= 0 && need > 0 && n_active > need; shift -= 8) {
     for (int i = tid; i < 256; i += NT) hist[i] = 0;
     __syncthreads();
