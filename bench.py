@@ -272,6 +272,29 @@ def dist_setup():
     return world, rank, local
 
 
+def rank_workload(w, rank: int):
+    """Each rank decodes its own batch of the same shape (weak scaling): rank r > 0 draws
+    its inputs from seed + 1000 r, so no two ranks process the same rows."""
+    return w if rank == 0 else w.replace(seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (all ranks call this in the same order)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_steps_per_s(ms_per_step_max: float, world: int) -> float:
+    """Whole-job throughput: every rank ran the same number of steps; the job took as long
+    as its slowest rank."""
+    return world * 1e3 / ms_per_step_max
+
+
 def config_of(w, lens):
     return {"workload": w.name, "global_batch": w.batch, "context": int(lens.max()),
             "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
@@ -336,7 +359,7 @@ def run_ours(args):
     w0 = WORKLOADS[args.workload]
     if args.batch:
         w0 = w0.replace(batch=args.batch)
-    w = w0 if rank == 0 else w0.replace(seed=w0.seed + 1000 * rank)
+    w = rank_workload(w0, rank)
     inp = synth.Inputs(w)
     f = Filled(inp)
     lay, cfg, cache = f.layer, f.cfg, f.cache
@@ -379,11 +402,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier()
-    t_ms = e0.elapsed_time(e1) / args.steps
-    t_max = torch.tensor([t_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    t_ms = float(t_max.item())
+    t_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, "cuda")
     st = qs.qs_device_status(lay.ws)
     if st[0] != 0:
         raise RuntimeError(f"device status after timing {st}")
@@ -434,11 +453,7 @@ def run_ours(args):
     t0 = time.perf_counter()
     for _ in range(n_e2e):
         e2e_step()
-    e2e_ms = (time.perf_counter() - t0) * 1e3 / n_e2e
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_t.item())
+    e2e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3 / n_e2e, world, "cuda")
     h2d = q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2
     d2h = out_h.numel() * out_h.element_size()
 
@@ -454,7 +469,7 @@ def run_ours(args):
             "algorithmic_bytes_per_launch": by["proxy"], "launch_us": score_us,
             "traffic": traffic}
     step_gbs = by["total"] / (t_ms * 1e-3) / 1e9
-    value = world * 1e3 / t_ms
+    value = aggregate_steps_per_s(t_ms, world)
     line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -464,7 +479,7 @@ def run_ours(args):
             "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s",
                          "frac": step_gbs / peak, "bytes_per_step": by},
             "stage_us": stage_us, "roofline": roof, "clocks": clk,
-            "e2e": {"value": world * 1e3 / e2e_ms, "unit": "steps/s",
+            "e2e": {"value": aggregate_steps_per_s(e2e_ms, world), "unit": "steps/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * launches_per_step}
