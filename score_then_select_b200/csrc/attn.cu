@@ -9,7 +9,9 @@
 //
 // CTA = (row, split): the split's slice of the row's selected token slots is streamed in
 // 64-token tiles (K and V, 16-byte cp.async into an XOR-swizzled 3-stage ring); each of
-// the 4 warps owns 16 tokens of a tile and keeps its own online-softmax state.
+// the 4 warps owns 16 tokens of a tile and keeps its own online-softmax state. The first
+// two tiles' pages are resolved and their loads started before the rest of the split's
+// pages are resolved.
 //
 // Tensor-core mapping (mma.m16n8k16, FP32 accumulate), transposed so that the group's
 // <= 8 query heads fill the N = 8 side:
@@ -27,6 +29,7 @@ namespace qs {
 constexpr int kTileT = 64;
 constexpr int kAttnStages = 3;
 constexpr int kMaxTokensPerSplit = 2048;
+constexpr int kEntCap = kMaxTokensPerSplit / 16 + 8;   // staged entries (blocks >= 16 tokens)
 
 template <int D>
 struct AttnSmem {
@@ -69,64 +72,82 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
   const int s1 = min(s0 + a.tokens_per_split, slots);
   const int cnt = s1 - s0;
 
-  // ---------------- token table of this split: cache row index or -1.
-  // Selection entries [i0, i1) cover the split's slots; each entry (a block of S tokens
-  // inside one page) is resolved once, 8 entries per thread in flight at a time; the
-  // per-entry base rows are staged in the (still unused) tile ring.
-  {
-    int* e_base = reinterpret_cast<int*>(smem);                 // [entries] row of token 0
-    int* e_len = e_base + (kMaxTokensPerSplit + 1);             // [entries] valid tokens
-    const int i0 = s0 / a.S;
-    const int i1 = cnt > 0 ? (s1 + a.S - 1) / a.S : i0;
-    const int ne = i1 - i0;
-    const int nbr = (L + a.S - 1) / a.S;
-    const int32_t* selr = a.sel + size_t(row) * a.budget;
-    for (int u0 = 0; u0 < ne; u0 += 128 * 8) {
-      int blk[8], pg[8];
+  // ---------------- token table of this split: cache row index of each slot, or -1.
+  // Slots [lo, hi) are resolved on demand: for blocks of >= 16 tokens each selection entry
+  // (a block inside one page) is looked up once into a small staging table; for smaller
+  // blocks each slot looks up its own block. Lookups are issued 8 per thread at a time.
+  // The first two tiles are resolved first so that their loads start before the rest of
+  // the table is built.
+  __shared__ int e_base[kEntCap], e_len[kEntCap];
+  const int32_t* selr = a.sel + size_t(row) * a.budget;
+  const int nbr = (L + a.S - 1) / a.S;
+  auto lookup = [&](int blk, int& pg) {      // physical page of a selected block, or -1
+    pg = -1;
+    if (blk < 0 || blk >= nbr) {
+      flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
+      return;
+    }
+    const int pi = blk * a.S / kPage;
+    pg = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
+    if (pg < 0 || pg >= a.num_pages) {
+      flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
+      pg = -1;
+    }
+  };
+  auto resolve = [&](int lo, int hi) {       // slots [lo, hi) of this split, hi <= cnt
+    if (hi <= lo) return;
+    if (a.S >= 16) {
+      const int e0 = (s0 + lo) / a.S, ne = (s0 + hi - 1) / a.S + 1 - e0;
+      for (int u0 = 0; u0 < ne; u0 += 128 * 8) {
+        int blk[8], pg[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int u = u0 + j * 128 + tid;
-        blk[j] = u < ne ? selr[i0 + u] : -1;
-      }
+        for (int j = 0; j < 8; ++j) {
+          const int u = u0 + j * 128 + tid;
+          blk[j] = u < ne ? selr[e0 + u] : -1;
+        }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        pg[j] = -1;
-        const int u = u0 + j * 128 + tid;
-        if (u < ne) {
-          if (blk[j] < 0 || blk[j] >= nbr) {
-            flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
-            blk[j] = -1;
-          } else {
-            const int pi = blk[j] * a.S / kPage;
-            pg[j] = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
-            if (pg[j] < 0 || pg[j] >= a.num_pages) {
-              flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
-              pg[j] = -1;
-            }
+        for (int j = 0; j < 8; ++j) {
+          const int u = u0 + j * 128 + tid;
+          pg[j] = -1;
+          if (u < ne) lookup(blk[j], pg[j]);
+          if (u < ne) {
+            const int t0 = blk[j] * a.S;
+            e_base[u] = pg[j] >= 0 ? (pg[j] * a.Hkv + g) * kPage + (t0 % kPage) : -1;
+            e_len[u] = pg[j] >= 0 ? min(a.S, L - t0) : 0;
           }
         }
       }
+      __syncthreads();
+      for (int i = lo + tid; i < hi; i += 128) {
+        const int gs = s0 + i;
+        const int u = gs / a.S - e0, off = gs % a.S;
+        s_rows[i] = off < e_len[u] ? e_base[u] + off : -1;
+      }
+      __syncthreads();
+    } else {
+      for (int i0 = lo; i0 < hi; i0 += 128 * 8) {
+        int blk[8], pg[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int u = u0 + j * 128 + tid;
-        if (u < ne) {
-          const int t0 = blk[j] * a.S;
-          e_base[u] = pg[j] >= 0 ? (pg[j] * a.Hkv + g) * kPage + (t0 % kPage) : -1;
-          e_len[u] = pg[j] >= 0 ? min(a.S, L - t0) : 0;
+        for (int j = 0; j < 8; ++j) {
+          const int i = i0 + j * 128 + tid;
+          blk[j] = i < hi ? selr[(s0 + i) / a.S] : -1;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = i0 + j * 128 + tid;
+          if (i < hi) {
+            lookup(blk[j], pg[j]);
+            const int t = blk[j] * a.S + (s0 + i) % a.S;
+            s_rows[i] = (pg[j] >= 0 && t < L) ? (pg[j] * a.Hkv + g) * kPage + (t % kPage) : -1;
+          }
         }
       }
     }
-    __syncthreads();
-    for (int i = tid; i < a.tokens_per_split; i += 128) {
-      int r = -1;
-      if (i < cnt) {
-        const int gs = s0 + i;
-        const int u = gs / a.S - i0, off = gs % a.S;
-        if (off < e_len[u]) r = e_base[u] + off;
-      }
-      s_rows[i] = r;
-    }
-  }
+  };
+  const int tiles = (cnt + kTileT - 1) / kTileT;
+  for (int i = cnt + tid; i < tiles * kTileT; i += 128) s_rows[i] = -1;
+  const int head = min(cnt, 2 * kTileT);
+  resolve(0, head);
 
   // ---------------- query fragments (B operand of S^T): head = lane/4, dims 2*(lane%4)+{0,1}
   uint32_t qb[KS][2];
@@ -142,7 +163,6 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
   }
   __syncthreads();
 
-  const int tiles = (cnt + kTileT - 1) / kTileT;
   const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k);
   const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v);
 
@@ -171,6 +191,7 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
 
   issue(0);
   issue(1);
+  resolve(head, cnt);        // the rest of the table, while the first two tiles load
   for (int tile = 0; tile < tiles; ++tile) {
     cp_async_wait<1>();
     __syncthreads();

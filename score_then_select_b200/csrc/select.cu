@@ -253,11 +253,13 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     if (hi > lo) {
       for (int i = tid; i < kLinBins; i += NT) hist[i] = 0;
       __syncthreads();
-      const double scale = double(kLinBins) / (double(hi) - double(lo));
-      // monotone in the score, so a higher bin always holds higher scores (recomputed
-      // below rather than kept, to stay within the 64 registers of a 1024-thread CTA)
+      // bin = trunc((x - lo) * scale): a rounded subtraction, a rounded product by a
+      // positive constant and a truncation are each monotone, so a higher bin always holds
+      // higher scores (recomputed below rather than kept, to stay within the 64 registers
+      // of a 1024-thread CTA); an overflowing range saturates and only coarsens the bins
+      const float scale = float(kLinBins) / (hi - lo);
       auto bin_of = [&](float x) {
-        int bn = int((double(x) - double(lo)) * scale);
+        const int bn = __float2int_rz((x - lo) * scale);
         return bn < 0 ? 0 : (bn >= kLinBins ? kLinBins - 1 : bn);
       };
 #pragma unroll
