@@ -383,7 +383,9 @@ def run_ours(args):
         raise RuntimeError(f"device status {st}")
     nsel_h = nsel.cpu().numpy()
     sel_h = sel.cpu().numpy()
-    launches_per_step = 4 if w.proxy_rank > 0 else 6
+    # append [+ block errors + query tiles] + score + select + attention [+ row merge when
+    # the selected runs are >= 8 slots; shorter runs merge inside the attention kernel]
+    launches_per_step = (4 if w.proxy_rank > 0 else 6) + (1 if w.block_size >= 8 else 0)
 
     def barrier():
         if world > 1:

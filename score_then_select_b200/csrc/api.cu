@@ -1,6 +1,7 @@
 // api.cu - the C ABI of libqs: argument validation, launch plans, workspace layout and
 // the entry points declared in include/qs.h. No device memory is allocated here.
 #include <cmath>
+#include <algorithm>
 #include <cstring>
 
 #include "qs_internal.h"
@@ -25,9 +26,10 @@ static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Attention split plan: choose splits per row so the grid fills whole waves of resident
-// CTAs (2 per SM) as evenly as possible; tokens per split is a multiple of the tile.
-static void plan_splits(int rows, int slots, int& splits, int& tps) {
+// Split plan of the gather kernel (selections of runs shorter than 8 slots): splits per row
+// so the (row, split) grid fills whole waves of resident CTAs (2 per SM) as evenly as
+// possible; tokens per split is a multiple of the 64-token tile.
+static void plan_gather_splits(int rows, int slots, int& splits, int& tps) {
   const int slots_per_wave = 2 * num_sms();
   double best = 1e30;
   splits = 1;
@@ -47,6 +49,24 @@ static void plan_splits(int rows, int slots, int& splits, int& tps) {
       tps = t;
     }
   }
+}
+
+// Attention work plan (runs of >= 8 slots): each row's selected slots form
+// ceil(budget * S / 64) tiles, cut into chunks of up to kChunkTilesMax tiles (one partial
+// each; a chunk's runs of min(S, 64) slots must fit one warp's lanes);
+// a persistent grid of kAttnCtasPerSm CTAs per SM (no more CTAs than chunks) claims them.
+static void plan_attention(int rows, long long slots, int S, WsLayout& w) {
+  const long long tpr = (slots + 63) / 64;
+  const int runs_per_tile = S >= 64 ? 1 : 64 / S;         // a chunk's runs fit one warp
+  const int kt = std::max(1, std::min(kChunkTilesMax, 32 / runs_per_tile));
+  const long long cpr = (tpr + kt - 1) / kt;
+  const long long chunks = rows * cpr;                   // < 2^31: checked by the caller
+  long long C = (long long)kAttnCtasPerSm * num_sms();
+  if (C > chunks) C = chunks;
+  w.tiles_per_row = int(tpr);
+  w.chunk_tiles = kt;
+  w.chunks_per_row = int(cpr);
+  w.attn_ctas = int(C);
 }
 
 qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
@@ -105,7 +125,14 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
 
   WsLayout& w = p.ws;
   w.nb_stride = p.nb_stride;
-  plan_splits(batch * p.Hkv, int(slots), w.splits, w.tokens_per_split);
+  if ((long long)batch * p.Hkv * ((slots + 63) / 64) >= (1LL << 31)) return QS_ERR_UNSUPPORTED;
+  plan_attention(batch * p.Hkv, slots, p.S, w);
+  if (p.S < kAttnTmaMinRun) {
+    plan_gather_splits(batch * p.Hkv, int(slots), w.gsplits, w.g_tokens_per_split);
+    w.parts_per_head = w.gsplits;
+  } else {
+    w.parts_per_head = w.chunks_per_row;
+  }
   size_t off = size_t(kHdrWords) * 4;
   const size_t rows = size_t(batch) * p.Hkv, rows_q = size_t(batch) * p.Hq;
   w.qt = off;      off = align_up(off + rows * (r > 0 ? r : 1) * 4, 256);
@@ -114,8 +141,8 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   w.scores = off;  off = align_up(off + rows * p.nb_stride * 4, 256);
   w.sel = off;     off = align_up(off + rows * p.budget * 4, 256);
   w.nsel = off;    off = align_up(off + rows * 4, 256);
-  w.part_ml = off; off = align_up(off + rows_q * w.splits * 2 * 4, 256);
-  w.part_o = off;  off = align_up(off + rows_q * w.splits * p.d * 4, 256);
+  w.part_ml = off; off = align_up(off + rows_q * w.parts_per_head * 2 * 4, 256);
+  w.part_o = off;  off = align_up(off + rows_q * w.parts_per_head * p.d * 4, 256);
   w.row_ctr = off; off = align_up(off + rows * 4, 256);
   w.total = off;
   return QS_OK;
@@ -265,13 +292,16 @@ static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, cons
   a.out = out;
   a.out_bf16 = p.out_dtype == QS_BF16 ? 1 : 0;
   a.hdr = hdr_of(ws);
-  a.batch = p.batch;
+  a.rows = p.batch * p.Hkv;
   a.Hkv = p.Hkv;
   a.G = p.G;
   a.S = p.S;
   a.budget = p.budget;
-  a.splits = p.ws.splits;
-  a.tokens_per_split = p.ws.tokens_per_split;
+  a.tiles_per_row = p.ws.tiles_per_row;
+  a.chunk_tiles = p.ws.chunk_tiles;
+  a.chunks_per_row = p.ws.chunks_per_row;
+  a.gsplits = p.ws.gsplits;
+  a.g_tokens_per_split = p.ws.g_tokens_per_split;
   a.max_pages_per_seq = c->max_pages_per_seq;
   a.num_pages = c->num_pages;
   a.scale_log2 = p.scale * 1.4426950408889634f;

@@ -1,4 +1,5 @@
-// attn.cu - split-K sparse attention over the selected blocks with its LSE combine.
+// attn.cu - sparse attention over the selected blocks with its LSE combine (selected runs
+// of >= 8 slots; shorter runs use attn_gather.cu).
 //
 // "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 1 and
 // Abstract: gather-free indexed attention reads the original full-dimensional keys and
@@ -7,196 +8,345 @@
 // "Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse Attention", Full
 // text: value aggregation in FP16 with FP32 accumulation over contiguous block tiles.
 //
-// CTA = (row, split): the split's slice of the row's selected token slots is streamed in
-// 64-token tiles (K and V, 16-byte cp.async into an XOR-swizzled 3-stage ring); each of
-// the 4 warps owns 16 tokens of a tile and keeps its own online-softmax state. The first
-// two tiles' pages are resolved and their loads started before the rest of the split's
-// pages are resolved.
+// Work decomposition (persistent grid, dynamic): a row (sequence, KV head) holds
+// `tiles_per_row` 64-token tiles of selected slots, cut into chunks of `chunk_tiles` tiles;
+// CTAs claim chunks in order from a workspace counter, so CTAs that the memory system
+// serves faster simply take more chunks, and a row is finished (and merged) as soon as its
+// last chunk is, instead of at the end of the kernel.
+//
+// Warp roles (warp-specialised; no block-wide barrier in the loop):
+//   * producer warp (warp 4): claims chunks two ahead and resolves the chunk's runs
+//     (a run is min(S, 64) slots of one selected block: lane = run) through selection
+//     entry -> page table in a pipeline one chunk apart per stage; then fills one stage of
+//     the shared-memory ring per tile: full and empty runs move as 64-element x run-height
+//     boxes by the TMA unit (tensor maps over the K and V caches, 128-byte swizzle; empty
+//     runs read zeros from outside the tensor), a ragged last block by 16-byte cp.async
+//     with zero fill, and the first tile of a chunk also brings the row's queries. Both
+//     kinds of copy are counted on the stage's `full` barrier; per-stage metadata carries
+//     the valid-slot mask and the chunk's identity. After the last chunk it posts an end
+//     marker.
+//   * consumer warps (warps 0-3): each owns 16 tokens of every tile and keeps its own
+//     online-softmax state (base 2, scale * log2 e folded into the logits). At the end of
+//     a chunk the four states are merged in a fixed order into the chunk's partial
+//     (max, sum, o); the chunk that completes its row's count merges the row's partials by
+//     log-sum-exp into the output.
 //
 // Tensor-core mapping (mma.m16n8k16, FP32 accumulate), transposed so that the group's
 // <= 8 query heads fill the N = 8 side:
 //   S^T[16 tok x 8 heads]  = K[16 tok x d] . Q^T[d x 8 heads]      (A = K via ldmatrix)
 //   O^T[d x 8 heads]      += V^T[d x 16 tok] . P^T[16 tok x 8 heads] (A = V via ldmatrix.trans,
 //                                                                    B = P via movmatrix)
-// Each warp's partial (max, sum, o) is merged across warps in shared memory and written
-// as one split partial; the last CTA of a row to finish (a workspace counter) merges the
-// row's splits by log-sum-exp and writes the output. Scores are kept in base 2
-// (scale * log2 e folded into the logits).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
 #include "qs_device.cuh"
 
 namespace qs {
 
 constexpr int kTileT = 64;
 constexpr int kAttnStages = 3;
-constexpr int kMaxTokensPerSplit = 2048;
-constexpr int kEntCap = kMaxTokensPerSplit / 16 + 8;   // staged entries (blocks >= 16 tokens)
+constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = 32 * kConsumerWarps;
+constexpr int kAttnThreads = kConsumerThreads + 32;
+constexpr int kHalfBytes = kTileT * 128;         // 64 rows x 64 elements (one swizzled box column)
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kRowBytes = D * 2;
-  static constexpr int kTileBytes = kTileT * kRowBytes;          // one of K or V
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kRingBytes = kAttnStages * kStageBytes;
-  static constexpr int kRowsOff = kRingBytes;                    // int32 [kMaxTokensPerSplit]
-  static constexpr int kTotal = kRowsOff + kMaxTokensPerSplit * 4;
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kHalves * kHalfBytes;           // one of K or V
+  static constexpr int kQBytes = (kMaxGroup * D * 2 + 1023) / 1024 * 1024;
+  static constexpr int kStageBytes = 2 * kTileBytes + kQBytes;      // multiple of 1024
+  static constexpr int kMetaOff = kAttnStages * kStageBytes;        // u32 [stages][4]
+  static constexpr int kBarOff = kMetaOff + kAttnStages * 16;       // u64 full[], empty[]
+  static constexpr int kMlOff = kBarOff + 2 * kAttnStages * 8;      // f32 [2][m [4][8], l [4][8]]
+  static constexpr int kMiscOff = kMlOff + 2 * 64 * 4;              // i32 abort, u64 barrier
+  static constexpr int kScrOff = kMiscOff + 16;                     // merge buffer
+  static constexpr int kBufStride = D + 4;                          // floats per head (merge)
+  static constexpr int kUsed = kScrOff + 2 * 8 * kBufStride * 4;
+  static constexpr int kTotal = kUsed + 1024;                       // + alignment slack
 };
+static_assert(AttnSmem<128>::kTotal + 1024 <= 228 * 1024 / kAttnCtasPerSm,
+              "kAttnCtasPerSm CTAs must fit one SM");
 
-// byte offset of (token row r, 16-byte chunk c) inside a swizzled tile
-template <int D>
+// Byte offset of (token row r, 16-byte chunk c) inside a K or V tile: the 128-byte
+// swizzle of the TMA unit, column halves of 64 elements 8 KiB apart.
 QS_DEV uint32_t swz(int r, int c) {
-  return uint32_t(r * (D * 2) + ((c ^ (r & 7)) << 4));
+  return uint32_t((c >> 3) * kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Bounded mbarrier wait that also gives up once another warp of the CTA has given up
+// (`abort` set): no wait in this kernel can outlast the others.
+QS_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  for (uint32_t i = 0; i < (1u << 22); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 63 && *abort) return false;
+  }
+  *abort = 1;
+  return false;
+}
+
+// Per-stage metadata word 3: chunk-in-row | first-tile flag | last-tile flag.
+constexpr uint32_t kMetaFirst = 1u << 16, kMetaLast = 1u << 17;
+
+// Barrier of the four consumer warps on an mbarrier (count 4), bounded like every wait
+// here: a warp that gives up cannot leave the others waiting on a hardware barrier.
+QS_DEV void consumer_sync(uint64_t* bar, uint32_t& phase, int lane, volatile int* abort) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  wait_or_abort(bar, phase, abort);
+  phase ^= 1u;
+  __syncwarp();
 }
 
 template <int D, bool V_F16, bool AGG_F16>
-__global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
+__global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
+    attn_kernel(const __grid_constant__ AttnParams a, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v) {
   using SM = AttnSmem<D>;
   constexpr int KS = D / 16;       // k-steps over the head dimension
   constexpr int CH = D / 8;        // 16-byte chunks per row
-  extern __shared__ __align__(128) uint8_t smem[];
-  int* s_rows = reinterpret_cast<int*>(smem + SM::kRowsOff);
+  constexpr int NS = kAttnStages;
+  extern __shared__ uint8_t smem_raw[];
+  // the swizzled boxes need 1024-byte aligned stages
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint32_t* meta = reinterpret_cast<uint32_t*>(smem + SM::kMetaOff);   // [stage][mask lo, hi, row, info]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
+  uint64_t* empty = full + NS;
+  float* s_ml = reinterpret_cast<float*>(smem + SM::kMlOff);         // [2][m [4][8], l [4][8]]
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::kMiscOff);
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + SM::kMiscOff + 8);
+  float* s_buf = reinterpret_cast<float*>(smem + SM::kScrOff);
 
-  pdl_wait();      // the selection comes from the kernel before
-  const int split = blockIdx.x, row = blockIdx.y;
-  const int b = row / a.Hkv, g = row % a.Hkv;
-  const int Hq = a.Hkv * a.G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  int n = a.n_sel[row];
-  int L = a.seq_lens[b];
-  if (n < 0 || n > a.budget || L < 0) {
-    if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
-    n = 0;
-  }
-  const int slots = n * a.S;
-  const int s0 = split * a.tokens_per_split;
-  const int s1 = min(s0 + a.tokens_per_split, slots);
-  const int cnt = s1 - s0;
-
-  // ---------------- token table of this split: cache row index of each slot, or -1.
-  // Slots [lo, hi) are resolved on demand: for blocks of >= 16 tokens each selection entry
-  // (a block inside one page) is looked up once into a small staging table; for smaller
-  // blocks each slot looks up its own block. Lookups are issued 8 per thread at a time.
-  // The first two tiles are resolved first so that their loads start before the rest of
-  // the table is built.
-  __shared__ int e_base[kEntCap], e_len[kEntCap];
-  const int32_t* selr = a.sel + size_t(row) * a.budget;
-  const int nbr = (L + a.S - 1) / a.S;
-  auto lookup = [&](int blk, int& pg) {      // physical page of a selected block, or -1
-    pg = -1;
-    if (blk < 0 || blk >= nbr) {
-      flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
-      return;
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1 + 32);            // producer lane 0 + one cp.async arrival per lane
+      mbar_init(&empty[s], kConsumerWarps);
+      meta[4 * s + 2] = 0xffffffffu;          // an unfilled stage reads as the end marker
     }
-    const int pi = blk * a.S / kPage;
-    pg = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
-    if (pg < 0 || pg >= a.num_pages) {
-      flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
-      pg = -1;
-    }
-  };
-  auto resolve = [&](int lo, int hi) {       // slots [lo, hi) of this split, hi <= cnt
-    if (hi <= lo) return;
-    if (a.S >= 16) {
-      const int e0 = (s0 + lo) / a.S, ne = (s0 + hi - 1) / a.S + 1 - e0;
-      for (int u0 = 0; u0 < ne; u0 += 128 * 8) {
-        int blk[8], pg[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int u = u0 + j * 128 + tid;
-          blk[j] = u < ne ? selr[e0 + u] : -1;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int u = u0 + j * 128 + tid;
-          pg[j] = -1;
-          if (u < ne) lookup(blk[j], pg[j]);
-          if (u < ne) {
-            const int t0 = blk[j] * a.S;
-            e_base[u] = pg[j] >= 0 ? (pg[j] * a.Hkv + g) * kPage + (t0 % kPage) : -1;
-            e_len[u] = pg[j] >= 0 ? min(a.S, L - t0) : 0;
-          }
-        }
-      }
-      __syncthreads();
-      for (int i = lo + tid; i < hi; i += 128) {
-        const int gs = s0 + i;
-        const int u = gs / a.S - e0, off = gs % a.S;
-        s_rows[i] = off < e_len[u] ? e_base[u] + off : -1;
-      }
-      __syncthreads();
-    } else {
-      for (int i0 = lo; i0 < hi; i0 += 128 * 8) {
-        int blk[8], pg[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = i0 + j * 128 + tid;
-          blk[j] = i < hi ? selr[(s0 + i) / a.S] : -1;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = i0 + j * 128 + tid;
-          if (i < hi) {
-            lookup(blk[j], pg[j]);
-            const int t = blk[j] * a.S + (s0 + i) % a.S;
-            s_rows[i] = (pg[j] >= 0 && t < L) ? (pg[j] * a.Hkv + g) * kPage + (t % kPage) : -1;
-          }
-        }
-      }
-    }
-  };
-  const int tiles = (cnt + kTileT - 1) / kTileT;
-  for (int i = cnt + tid; i < tiles * kTileT; i += 128) s_rows[i] = -1;
-  const int head = min(cnt, 2 * kTileT);
-  resolve(0, head);
-
-  // ---------------- query fragments (B operand of S^T): head = lane/4, dims 2*(lane%4)+{0,1}
-  uint32_t qb[KS][2];
-  {
-    const int h = lane >> 2;
-    const uint16_t* qr = a.q + (size_t(b) * Hq + g * a.G + (h < a.G ? h : 0)) * D;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int d0 = ks * 16 + 2 * (lane & 3);
-      qb[ks][0] = h < a.G ? *reinterpret_cast<const uint32_t*>(qr + d0) : 0u;
-      qb[ks][1] = h < a.G ? *reinterpret_cast<const uint32_t*>(qr + d0 + 8) : 0u;
-    }
+    mbar_init(cbar, kConsumerWarps);
+    *s_abort = 0;
+    fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();      // the selection comes from the kernel before
+  pdl_trigger();   // the row merge may be scheduled now; it waits for this grid to finish
 
-  const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k);
-  const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v);
+  const int Hq = a.Hkv * a.G;
+  const int tpr = a.tiles_per_row, cpr = a.chunks_per_row, ktiles = a.chunk_tiles;
+  const int nchunks = a.rows * cpr;
 
-  auto issue = [&](int tile) {
-    if (tile < tiles) {
-      uint8_t* st = smem + (tile % kAttnStages) * SM::kStageBytes;
+  if (warp == kConsumerWarps) {
+    // ======================= producer: chunk claims, run table, copies ================
+    // A run is hb = min(S, 64) consecutive slots of a tile: one selected block, or one half
+    // of a 128-slot block; lane u of a chunk's table holds run u (tile u / rpt, run u % rpt).
+    // Three stages a chunk apart: A loads the selection entry and the row's n_sel / length;
+    // B validates and loads the page-table entry; C yields the cache row of the run's first
+    // slot and its valid count (0: empty; hb: full; else a ragged last block).
+    const int hb = a.run_h, lg_hb = a.log2_run, rpt = kTileT >> lg_hb, lgS = a.log2_S;
+    uint32_t* next_ctr = a.hdr + kCtrAttnNext;
+    struct RunA { int row, sl, blk, n, L; };
+    struct RunB { int pg, t0, g, cnt, row; };
+    auto stage_a = [&](int c) {
+      RunA r{0, 0, -1, 0, 0};
+      if (c < nchunks) {
+        r.row = c / cpr;
+        const int tin0 = (c - r.row * cpr) * ktiles, j = lane >> (6 - lg_hb);
+        if (j < min(ktiles, tpr - tin0)) {
+          r.sl = (tin0 + j) * kTileT + ((lane & (rpt - 1)) << lg_hb);
+          r.n = a.n_sel[r.row];
+          r.L = a.seq_lens[r.row / a.Hkv];
+          const int e = r.sl >> lgS;
+          if (e < a.budget) r.blk = a.sel[size_t(r.row) * a.budget + e];
+        } else {
+          r.n = -2;                                        // no such run in this chunk
+        }
+      }
+      return r;
+    };
+    auto stage_b = [&](int c, const RunA& x) {
+      RunB r{-1, 0, 0, 0, x.row};
+      if (c >= nchunks || x.n == -2) return r;
+      const int b = x.row / a.Hkv;
+      r.g = x.row - b * a.Hkv;
+      if (x.n < 0 || x.n > a.budget || x.L < 0) {
+        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
+        return r;
+      }
+      if (x.sl >= (x.n << lgS)) return r;                  // beyond the row's selection
+      const int nbr = (x.L + (1 << lgS) - 1) >> lgS;
+      if (x.blk < 0 || x.blk >= nbr) {
+        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
+        return r;
+      }
+      r.t0 = (x.blk << lgS) + (x.sl & ((1 << lgS) - 1));
+      if (r.t0 >= x.L) return r;                           // ragged tail of the last block
+      r.cnt = min(hb, x.L - r.t0);
+      const int pi = r.t0 >> 7;                            // kPage = 128
+      r.pg = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
+      return r;                                            // pg is checked once it has landed
+    };
+    auto stage_c = [&](const RunB& x, int& y, int& cnt) {
+      cnt = x.cnt;
+      y = -1;
+      if (cnt == 0) return;
+      if (x.pg < 0 || x.pg >= a.num_pages) {
+        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
+        cnt = 0;
+        return;
+      }
+      y = (x.pg * a.Hkv + x.g) * kPage + (x.t0 & (kPage - 1));
+    };
+
+    // chunk claims: three in flight from the start, then one per chunk, two chunks ahead
+    unsigned claim0 = 0, claim1 = 0, pend = 0;
+    if (lane == 0) {
+      claim0 = atomicAdd(next_ctr, 1u);
+      claim1 = atomicAdd(next_ctr, 1u);
+      pend = atomicAdd(next_ctr, 1u);
+    }
+    int c_cur = int(min(__shfl_sync(kFull, claim0, 0), unsigned(nchunks)));
+    int c_n1 = int(min(__shfl_sync(kFull, claim1, 0), unsigned(nchunks)));
+    RunA pa = stage_a(c_n1);
+    RunB pb = stage_b(c_cur, stage_a(c_cur));
+
+    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k);
+    const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v);
+    int t = 0;                                             // stages filled so far
+    bool ok = true;
+    while (ok && c_cur < nchunks) {
+      int run_y, run_cnt;
+      stage_c(pb, run_y, run_cnt);
+      pb = stage_b(c_n1, pa);
+      const int c_n2 = int(min(__shfl_sync(kFull, pend, 0), unsigned(nchunks)));
+      pa = stage_a(c_n2);
+      if (lane == 0) pend = c_n2 < nchunks ? atomicAdd(next_ctr, 1u) : unsigned(nchunks);
+
+      const int row = c_cur / cpr, ci = c_cur - row * cpr;
+      const int nt = min(ktiles, tpr - ci * ktiles);
+      const int b = row / a.Hkv, g = row - b * a.Hkv;
+      for (int j = 0; j < nt; ++j, ++t) {
+        // the tile's runs: lane r < rpt takes run r
+        const int src = (j << (6 - lg_hb)) + (lane & (rpt - 1));
+        const int ry = __shfl_sync(kFull, run_y, src), rc = __shfl_sync(kFull, run_cnt, src);
+        unsigned long long mask = 0;
+        uint32_t tma_bytes = 0;
+        for (int r = 0; r < rpt; ++r) {
+          const int cr = __shfl_sync(kFull, rc, r);
+          if (cr > 0) mask |= (cr >= 64 ? ~0ull : ((1ull << cr) - 1)) << (r << lg_hb);
+          if (cr == 0 || cr == hb) tma_bytes += uint32_t(2 * SM::kHalves * hb * 128);
+        }
+        const int s = t % NS;
+        bool got = true;
+        if (lane == 0 && t >= NS) got = wait_or_abort(&empty[s], ((t / NS) - 1) & 1, s_abort);
+        ok = __shfl_sync(kFull, got, 0);
+        __syncwarp();
+        if (!ok) break;
+
+        uint8_t* st = smem + s * SM::kStageBytes;
+        if (j == 0) {                                      // a chunk starts: the row's queries
+          const uint16_t* qr = a.q + (size_t(b) * Hq + g * a.G) * D;
+          for (int w = lane; w < a.G * D / 2; w += 32)
+            cp_async4(st + 2 * SM::kTileBytes + 4 * w, qr + 2 * w);
+        }
+        if (lane == 0) {
+          meta[4 * s] = uint32_t(mask);
+          meta[4 * s + 1] = uint32_t(mask >> 32);
+          meta[4 * s + 2] = uint32_t(row);
+          meta[4 * s + 3] = uint32_t(ci) | (j == 0 ? kMetaFirst : 0u) | (j + 1 == nt ? kMetaLast : 0u);
+          mbar_arrive_expect_tx(&full[s], tma_bytes);
+        }
+        __syncwarp();                                      // the byte count is posted first
+        // full and empty runs: box copies (an empty run reads zeros from outside the tensor)
+        if (lane < rpt && (rc == 0 || rc == hb)) {
+          const int y = rc ? ry : -hb;
 #pragma unroll
-      for (int it = 0; it < kTileT * CH / 128; ++it) {
-        const int idx = it * 128 + tid;
-        const int r = idx / CH, c = idx % CH;
-        const int cr = s_rows[tile * kTileT + r];
-        const size_t off = size_t(cr < 0 ? 0 : cr) * (D * 2) + c * 16;
-        cp_async16_zfill(st + swz<D>(r, c), kbase + off, cr >= 0);
-        cp_async16_zfill(st + SM::kTileBytes + swz<D>(r, c), vbase + off, cr >= 0);
+          for (int h = 0; h < SM::kHalves; ++h) {
+            const uint32_t off = h * kHalfBytes + ((lane << lg_hb) << 7);
+            tma_load_2d(st + off, &tm_k, 64 * h, y, &full[s]);
+            tma_load_2d(st + SM::kTileBytes + off, &tm_v, 64 * h, y, &full[s]);
+          }
+        }
+        // a ragged run: 16-byte copies of its valid rows, zeros for the rest
+        for (int r = 0; r < rpt; ++r) {
+          const int cr = __shfl_sync(kFull, rc, r), y0 = __shfl_sync(kFull, ry, r);
+          if (cr == 0 || cr == hb) continue;
+          for (int i = lane; i < hb; i += 32) {
+            const int rt = (r << lg_hb) + i;
+            const bool v = i < cr;
+            const size_t off = size_t(v ? y0 + i : 0) * (D * 2);
+#pragma unroll
+            for (int ch = 0; ch < CH; ++ch) {
+              cp_async16_zfill(st + swz(rt, ch), kbase + off + ch * 16, v);
+              cp_async16_zfill(st + SM::kTileBytes + swz(rt, ch), vbase + off + ch * 16, v);
+            }
+          }
+        }
+        cp_async_mbar_arrive_noinc(&full[s]);
+      }
+      c_cur = c_n1;
+      c_n1 = c_n2;
+    }
+    // end marker: one more stage whose row is -1
+    if (ok) {
+      const int s = t % NS;
+      bool got = true;
+      if (lane == 0 && t >= NS) got = wait_or_abort(&empty[s], ((t / NS) - 1) & 1, s_abort);
+      ok = __shfl_sync(kFull, got, 0);
+      __syncwarp();
+      if (ok) {
+        if (lane == 0) {
+          meta[4 * s + 2] = 0xffffffffu;
+          mbar_arrive_expect_tx(&full[s], 0u);
+        }
+        cp_async_mbar_arrive_noinc(&full[s]);
+        ++t;
       }
     }
-    cp_async_commit();
-  };
+    // every copy issued must land before the CTA exits
+    if (lane == 0) {
+      for (int j = t > NS ? t - NS : 0; j < t; ++j)
+        if (!mbar_wait(&full[j % NS], (j / NS) & 1)) *s_abort = 1;
+    }
+    if (lane == 0 && pend > 0x7fffffffu) *s_abort = 1;     // the last claim has returned
+    __syncwarp();
+    return;
+  }
 
-  // online-softmax state for heads h0 = 2*(lane%4), h1 = h0 + 1 (replicated across lanes
-  // with equal lane%4); l is this lane's partial sum over its own tokens
+  // ======================= consumers: online softmax, chunk partials, row merge ==========
+  uint32_t cphase = 0, mpar = 0;
+  const int h0 = 2 * (lane & 3);                           // this lane's heads h0, h0 + 1
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
   float o[KS][4];
 #pragma unroll
   for (int m = 0; m < KS; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.0f;
-
-  issue(0);
-  issue(1);
-  resolve(head, cnt);        // the rest of the table, while the first two tiles load
-  for (int tile = 0; tile < tiles; ++tile) {
-    cp_async_wait<1>();
-    __syncthreads();
-    issue(tile + 2);
-    const uint8_t* st = smem + (tile % kAttnStages) * SM::kStageBytes;
+  uint32_t qb[KS][2];
+  for (int t = 0;; ++t) {
+    const int s = t % NS;
+    if (!wait_or_abort(&full[s], (t / NS) & 1, s_abort)) break;
+    const uint32_t lo = meta[4 * s], hi = meta[4 * s + 1];
+    const int row = int(meta[4 * s + 2]);
+    const uint32_t info = meta[4 * s + 3];
+    if (row < 0 || row >= a.rows || int(info & 0xffffu) >= cpr) break;   // end marker
+    const uint8_t* st = smem + s * SM::kStageBytes;
+    if (info & kMetaFirst) {
+      // query fragments (B operand of S^T): head = lane/4, dims 2*(lane%4)+{0,1}
+      const int h = lane >> 2;
+      const uint16_t* qs = reinterpret_cast<const uint16_t*>(st + 2 * SM::kTileBytes) + h * D;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int d0 = ks * 16 + 2 * (lane & 3);
+        qb[ks][0] = h < a.G ? *reinterpret_cast<const uint32_t*>(qs + d0) : 0u;
+        qb[ks][1] = h < a.G ? *reinterpret_cast<const uint32_t*>(qs + d0 + 8) : 0u;
+      }
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.0f;
+#pragma unroll
+      for (int m = 0; m < KS; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.0f;
+    }
     const uint32_t kst = smem_u32(st), vst = smem_u32(st + SM::kTileBytes);
 
     // S^T = K Q^T for this warp's 16 tokens
@@ -204,11 +354,12 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(a0, a1, a2, a3, kst + swz<D>(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
+      ldsm_x4(a0, a1, a2, a3, kst + swz(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
       mma_bf16(c, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
     }
-    const int tl = tile * kTileT + warp * 16 + (lane >> 2);
-    const bool v0 = s_rows[tl] >= 0, v1 = s_rows[tl + 8] >= 0;
+    const int tl = warp * 16 + (lane >> 2);       // tokens tl and tl + 8 (same 32-slot word)
+    const uint32_t vm = warp < 2 ? lo : hi;
+    const bool v0 = (vm >> (tl & 31)) & 1u, v1 = (vm >> ((tl + 8) & 31)) & 1u;
     float x0 = v0 ? c[0] * a.scale_log2 : -INFINITY;
     float x1 = v0 ? c[1] * a.scale_log2 : -INFINITY;
     float x2 = v1 ? c[2] * a.scale_log2 : -INFINITY;
@@ -250,7 +401,7 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
     for (int m = 0; m < KS; ++m) {
       uint32_t a0, a1, a2, a3;
       ldsm_x4_t(a0, a1, a2, a3,
-                vst + swz<D>(warp * 16 + (lane & 7) + ((lane >> 4) << 3), m * 2 + ((lane >> 3) & 1)));
+                vst + swz(warp * 16 + (lane & 7) + ((lane >> 4) << 3), m * 2 + ((lane >> 3) & 1)));
       if constexpr (AGG_F16) {
         if constexpr (!V_F16) {
           a0 = bf16x2_to_f16x2(a0);
@@ -263,134 +414,251 @@ __global__ void __launch_bounds__(128, 2) attn_kernel(const AttnParams a) {
         mma_bf16(o[m], a0, a1, a2, a3, pb0, pb1);
       }
     }
-  }
-  cp_async_wait<0>();
-  __syncthreads();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);        // this warp is done with the stage
+    if (!(info & kMetaLast)) continue;
 
-  // ---------------- merge the 4 warps' states, write this split's partial
+    // ---------------- end of a chunk: merge the four warps (fixed order) into its partial.
+    // The (max, sum) exchange alternates between two buffers so that a warp already at the
+    // next chunk's end cannot overwrite what warp 0 still reads.
+    float* s_m = s_ml + 64 * mpar;
+    float* s_l = s_m + 32;
+    mpar ^= 1;
 #pragma unroll
-  for (int o2 = 4; o2 < 32; o2 <<= 1) {
-    l0 += __shfl_xor_sync(kFull, l0, o2);
-    l1 += __shfl_xor_sync(kFull, l1, o2);
-  }
-  float* s_m = reinterpret_cast<float*>(smem);          // [4][8]
-  float* s_l = s_m + 32;                                // [4][8]
-  float* s_o = s_l + 32;                                // [4][8][D]
-  if (lane < 4) {
-    s_m[warp * 8 + 2 * lane] = m0;
-    s_m[warp * 8 + 2 * lane + 1] = m1;
-    s_l[warp * 8 + 2 * lane] = l0;
-    s_l[warp * 8 + 2 * lane + 1] = l1;
-  }
-  {
-    const int h0 = 2 * (lane & 3);
-#pragma unroll
-    for (int m = 0; m < KS; ++m) {
-      const int d0 = m * 16 + (lane >> 2);
-      float* ow = s_o + warp * 8 * D;
-      ow[h0 * D + d0] = o[m][0];
-      ow[(h0 + 1) * D + d0] = o[m][1];
-      ow[h0 * D + d0 + 8] = o[m][2];
-      ow[(h0 + 1) * D + d0 + 8] = o[m][3];
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+      l0 += __shfl_xor_sync(kFull, l0, o2);
+      l1 += __shfl_xor_sync(kFull, l1, o2);
     }
-  }
-  __syncthreads();
-  for (int idx = tid; idx < a.G * D; idx += 128) {
-    const int h = idx / D, d = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w * 8 + h]);
-    const float base = M == -INFINITY ? 0.0f : M;
-    float lsum = 0.0f, osum = 0.0f;
+    if (lane < 4) {
+      s_m[warp * 8 + h0] = m0;
+      s_m[warp * 8 + h0 + 1] = m1;
+    }
+    consumer_sync(cbar, cphase, lane, s_abort);
+    float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      const float wt = ex2(s_m[w * 8 + h] - base);
-      lsum += wt * s_l[w * 8 + h];
-      osum += wt * s_o[(w * 8 + h) * D + d];
+      M0 = fmaxf(M0, s_m[w * 8 + h0]);
+      M1 = fmaxf(M1, s_m[w * 8 + h0 + 1]);
     }
-    const size_t rq = size_t(b) * Hq + g * a.G + h;
-    const size_t pidx = rq * a.splits + split;
-    a.part_o[pidx * D + d] = osum;
-    if (d == 0) {
-      a.part_ml[pidx * 2] = M;
-      a.part_ml[pidx * 2 + 1] = lsum;
+    {
+      const float f0 = ex2(m0 - (M0 == -INFINITY ? 0.0f : M0));
+      const float f1 = ex2(m1 - (M1 == -INFINITY ? 0.0f : M1));
+#pragma unroll
+      for (int m = 0; m < KS; ++m) {
+        o[m][0] *= f0;
+        o[m][1] *= f1;
+        o[m][2] *= f0;
+        o[m][3] *= f1;
+      }
+      if (lane < 4) {
+        s_l[warp * 8 + h0] = l0 * f0;
+        s_l[warp * 8 + h0 + 1] = l1 * f1;
+      }
+    }
+    auto park = [&](float* dst) {
+#pragma unroll
+      for (int m = 0; m < KS; ++m) {
+        const int d0 = m * 16 + (lane >> 2);
+        dst[h0 * SM::kBufStride + d0] = o[m][0];
+        dst[(h0 + 1) * SM::kBufStride + d0] = o[m][1];
+        dst[h0 * SM::kBufStride + d0 + 8] = o[m][2];
+        dst[(h0 + 1) * SM::kBufStride + d0 + 8] = o[m][3];
+      }
+    };
+    auto add = [&](const float* src) {
+#pragma unroll
+      for (int m = 0; m < KS; ++m) {
+        const int d0 = m * 16 + (lane >> 2);
+        o[m][0] += src[h0 * SM::kBufStride + d0];
+        o[m][1] += src[(h0 + 1) * SM::kBufStride + d0];
+        o[m][2] += src[h0 * SM::kBufStride + d0 + 8];
+        o[m][3] += src[(h0 + 1) * SM::kBufStride + d0 + 8];
+      }
+    };
+    float* slot0 = s_buf;
+    float* slot1 = s_buf + 8 * SM::kBufStride;
+    if (warp >= 2) park(warp == 2 ? slot0 : slot1);        // o2 -> slot 0, o3 -> slot 1
+    consumer_sync(cbar, cphase, lane, s_abort);
+    if (warp < 2) add(warp == 0 ? slot0 : slot1);          // o0 + o2, o1 + o3
+    consumer_sync(cbar, cphase, lane, s_abort);
+    if (warp == 1) park(slot0);
+    consumer_sync(cbar, cphase, lane, s_abort);
+    if (warp == 0) {
+      add(slot0);                                          // (o0 + o2) + (o1 + o3)
+      const int ci = int(info & 0xffffu);
+      const size_t rq0 = size_t(row / a.Hkv) * Hq + (row % a.Hkv) * a.G;
+      const size_t p0i = (rq0 + h0) * cpr + ci, p1i = (rq0 + h0 + 1) * cpr + ci;
+#pragma unroll
+      for (int m = 0; m < KS; ++m) {
+        const int d0 = m * 16 + (lane >> 2);
+        if (h0 < a.G) {
+          __stcg(a.part_o + p0i * D + d0, o[m][0]);
+          __stcg(a.part_o + p0i * D + d0 + 8, o[m][2]);
+        }
+        if (h0 + 1 < a.G) {
+          __stcg(a.part_o + p1i * D + d0, o[m][1]);
+          __stcg(a.part_o + p1i * D + d0 + 8, o[m][3]);
+        }
+      }
+      if (lane < 4) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int h = h0 + k;
+          if (h < a.G) {
+            const size_t pi = (rq0 + h) * cpr + ci;
+            const float M = fmaxf(fmaxf(s_m[h], s_m[8 + h]), fmaxf(s_m[16 + h], s_m[24 + h]));
+            const float L = (s_l[h] + s_l[16 + h]) + (s_l[8 + h] + s_l[24 + h]);
+            __stcg(a.part_ml + pi * 2, M);
+            __stcg(a.part_ml + pi * 2 + 1, L);
+          }
+        }
+      }
     }
   }
+  if (tid == 0 && *s_abort) flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_ATTN, blockIdx.x);
+}
 
-  // ---------------- the last split of the row to finish merges all splits (LSE combine):
-  // out[h][d] = sum_s 2^(m_s - M) o_s[d] / sum_s 2^(m_s - M) l_s; a row with no tokens -> 0
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const unsigned prev = atomicAdd(a.row_ctr + row, 1u);
-    s_last = prev == unsigned(a.splits - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  float* s_w = reinterpret_cast<float*>(smem);          // [G][splits] weights, then [G] 1/den
-  const int ns = a.splits;
-  for (int i = tid; i < a.G * ns; i += 128) {
-    const int h = i / ns, sp = i % ns;
-    const size_t pidx = (size_t(b) * Hq + g * a.G + h) * ns + sp;
-    s_w[i] = __ldcg(a.part_ml + pidx * 2);
-    s_w[a.G * ns + i] = __ldcg(a.part_ml + pidx * 2 + 1);
-  }
-  __syncthreads();
-  if (tid < a.G) {
-    const int h = tid;
+// ---------------------------------------------------------------- combine
+// One CTA per (row, query head): the head's chunk partials -> output by log-sum-exp,
+//   out[d] = sum_p 2^(m_p - M) o_p[d] / sum_p 2^(m_p - M) l_p  (a row with no tokens -> 0).
+// Thread d owns output element d; all of its partial loads are in flight together.
+// Waits for the attention grid (programmatic dependent launch), then resets the chunk
+// claim counter for the next attention launch.
+template <int D>
+__global__ void __launch_bounds__(D) attn_combine_kernel(const AttnParams a) {
+  extern __shared__ float s_w[];                           // [cpr] weights, then 1/den
+  pdl_wait();
+  const int row = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int cpr = a.chunks_per_row;
+  if (row == 0 && h == 0 && tid == 0) a.hdr[kCtrAttnNext] = 0u;
+  const size_t rq = size_t(row / a.Hkv) * (a.Hkv * a.G) + (row % a.Hkv) * a.G + h;
+  const float* ml = a.part_ml + rq * cpr * 2;
+  if (tid < 32) {
     float M = -INFINITY;
-    for (int sp = 0; sp < ns; ++sp)
-      if (s_w[a.G * ns + h * ns + sp] > 0.0f) M = fmaxf(M, s_w[h * ns + sp]);
-    float den = 0.0f;
-    for (int sp = 0; sp < ns; ++sp) {
-      const float l = s_w[a.G * ns + h * ns + sp];
-      const float wt = l > 0.0f ? ex2(s_w[h * ns + sp] - M) : 0.0f;
-      s_w[h * ns + sp] = wt;
-      den += wt * l;
+    for (int p = lane; p < cpr; p += 32) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(ml) + p);
+      if (v.y > 0.0f) M = fmaxf(M, v.x);
     }
-    s_w[2 * a.G * ns + h] = den > 0.0f ? 1.0f / den : 0.0f;
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
+    float den = 0.0f;
+    for (int p = lane; p < cpr; p += 32) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(ml) + p);
+      const float w = v.y > 0.0f ? ex2(v.x - M) : 0.0f;
+      s_w[p] = w;
+      den += w * v.y;
+    }
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(kFull, den, o2);
+    if (lane == 0) s_w[cpr] = den > 0.0f ? 1.0f / den : 0.0f;
   }
   __syncthreads();
-  for (int idx = tid; idx < a.G * D; idx += 128) {
-    const int h = idx / D, d = idx % D;
-    const size_t rq = size_t(b) * Hq + g * a.G + h;
-    float num = 0.0f;
-    for (int sp = 0; sp < ns; ++sp) {
-      const float wt = s_w[h * ns + sp];
-      if (wt != 0.0f) num += wt * __ldcg(a.part_o + (rq * ns + sp) * D + d);
-    }
-    const float r = num * s_w[2 * a.G * ns + h];
-    if (a.out_bf16)
-      reinterpret_cast<uint16_t*>(a.out)[rq * D + d] = f32_to_bf16_rn(r);
-    else
-      reinterpret_cast<float*>(a.out)[rq * D + d] = r;
+  const float* po = a.part_o + rq * cpr * D + tid;
+  float acc = 0.0f;
+  int p = 0;
+  for (; p + 8 <= cpr; p += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldcg(po + size_t(p + u) * D);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += s_w[p + u] * v[u];
   }
-  if (tid == 0) a.row_ctr[row] = 0u;
+  for (; p < cpr; ++p) acc += s_w[p] * __ldcg(po + size_t(p) * D);
+  const float r = acc * s_w[cpr];
+  const size_t oi = rq * D + tid;
+  if (a.out_bf16)
+    reinterpret_cast<uint16_t*>(a.out)[oi] = f32_to_bf16_rn(r);
+  else
+    reinterpret_cast<float*>(a.out)[oi] = r;
+}
+
+// ------------------------------------------------------------------ tensor maps (host)
+// A 2-D map over one cache tensor viewed as [num_pages * Hkv * 128 rows][d] 16-bit
+// elements; boxes of 64 elements x `box_rows` rows, 128-byte swizzle. Maps are cached by
+// (address, rows, d, box_rows): encoding is a host-only call but not free.
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+static bool cache_map(const void* base, uint64_t rows, int d, int box_rows, CUtensorMap* out) {
+  struct Entry { const void* base; uint64_t rows; int d, box_rows; CUtensorMap map; };
+  static std::mutex mu;
+  static Entry entries[16];
+  static int n_entries = 0, next = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_entries; ++i) {
+    const Entry& e = entries[i];
+    if (e.base == base && e.rows == rows && e.d == d && e.box_rows == box_rows) {
+      *out = e.map;
+      return true;
+    }
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn || rows == 0 || rows >= (1ull << 31)) return false;
+  CUtensorMap m;
+  const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+  const cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  Entry& e = entries[next];
+  e = Entry{base, rows, d, box_rows, m};
+  next = (next + 1) % 16;
+  if (n_entries < 16) ++n_entries;
+  *out = m;
+  return true;
 }
 
 template <int D, bool VF, bool AF>
-static cudaError_t launch_attn_t(const AttnParams& a, cudaStream_t s, bool pdl) {
+static cudaError_t launch_attn_t(const AttnParams& a, const CUtensorMap& mk, const CUtensorMap& mv,
+                                 int grid, cudaStream_t s, bool pdl) {
   auto k = attn_kernel<D, VF, AF>;
   const int smem = AttnSmem<D>::kTotal;
   static const cudaError_t attr =
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (attr != cudaSuccess) return attr;
-  return launch_k(k, dim3(a.splits, a.batch * a.Hkv), dim3(128), smem, s, pdl, a);
+  cudaError_t e = launch_k(k, dim3(grid), dim3(kAttnThreads), smem, s, pdl, a, mk, mv);
+  if (e != cudaSuccess) return e;
+  // the row merge, launched behind the attention grid (it waits for it before reading)
+  const size_t csmem = size_t(a.chunks_per_row + 1) * sizeof(float);
+  return launch_k(attn_combine_kernel<D>, dim3(a.rows, a.G), dim3(D), csmem, s, true, a);
 }
 
-cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl) {
+cudaError_t launch_attn(const Plan& p, const AttnParams& a_in, cudaStream_t s, bool pdl) {
+  if (p.S < kAttnTmaMinRun) return launch_attn_gather(p, a_in, s, pdl);
+  AttnParams a = a_in;
+  a.run_h = p.S < kTileT ? p.S : kTileT;
+  a.log2_S = 0;
+  while ((1 << a.log2_S) < p.S) ++a.log2_S;
+  a.log2_run = a.log2_S < 6 ? a.log2_S : 6;
+  CUtensorMap mk, mv;
+  std::memset(&mk, 0, sizeof(mk));
+  std::memset(&mv, 0, sizeof(mv));
+  const uint64_t rows = uint64_t(a.num_pages) * a.Hkv * kPage;
+  if (!cache_map(a.k, rows, p.d, a.run_h, &mk) || !cache_map(a.v, rows, p.d, a.run_h, &mv))
+    return cudaErrorNotSupported;
   const bool vf = p.v_dtype == QS_F16, af = p.v_agg_dtype == QS_F16;
+  const int grid = p.ws.attn_ctas;
   if (p.d == 128) {
-    if (vf) return launch_attn_t<128, true, true>(a, s, pdl);
-    if (af) return launch_attn_t<128, false, true>(a, s, pdl);
-    return launch_attn_t<128, false, false>(a, s, pdl);
+    if (vf) return launch_attn_t<128, true, true>(a, mk, mv, grid, s, pdl);
+    if (af) return launch_attn_t<128, false, true>(a, mk, mv, grid, s, pdl);
+    return launch_attn_t<128, false, false>(a, mk, mv, grid, s, pdl);
   }
   if (p.d == 64) {
-    if (vf) return launch_attn_t<64, true, true>(a, s, pdl);
-    if (af) return launch_attn_t<64, false, true>(a, s, pdl);
-    return launch_attn_t<64, false, false>(a, s, pdl);
+    if (vf) return launch_attn_t<64, true, true>(a, mk, mv, grid, s, pdl);
+    if (af) return launch_attn_t<64, false, true>(a, mk, mv, grid, s, pdl);
+    return launch_attn_t<64, false, false>(a, mk, mv, grid, s, pdl);
   }
   return cudaErrorInvalidValue;
 }

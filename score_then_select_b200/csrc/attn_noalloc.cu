@@ -57,8 +57,8 @@ extern "C" qs_status qs_sparse_attn_noalloc(const qs_config* cfg, const qs_cache
   const size_t hdr_bytes = size_t(kHdrWords) * 4;
   const size_t ctr_off = hdr_bytes;
   const size_t ml_off = up256(ctr_off + rows * 4);
-  const size_t o_off = up256(ml_off + rows_q * p.ws.splits * 2 * 4);
-  const size_t need = o_off + rows_q * p.ws.splits * p.d * 4;
+  const size_t o_off = up256(ml_off + rows_q * p.ws.parts_per_head * 2 * 4);
+  const size_t need = o_off + rows_q * p.ws.parts_per_head * p.d * 4;
   if (need > kStaticScratch) return QS_ERR_UNSUPPORTED;
   void* base = nullptr;
   if ((st = scratch_address(&base)) != QS_OK) return st;
@@ -80,13 +80,16 @@ extern "C" qs_status qs_sparse_attn_noalloc(const qs_config* cfg, const qs_cache
   a.out = out;
   a.out_bf16 = p.out_dtype == QS_BF16 ? 1 : 0;
   a.hdr = reinterpret_cast<uint32_t*>(s8);
-  a.batch = p.batch;
+  a.rows = p.batch * p.Hkv;
   a.Hkv = p.Hkv;
   a.G = p.G;
   a.S = p.S;
   a.budget = p.budget;
-  a.splits = p.ws.splits;
-  a.tokens_per_split = p.ws.tokens_per_split;
+  a.tiles_per_row = p.ws.tiles_per_row;
+  a.chunk_tiles = p.ws.chunk_tiles;
+  a.chunks_per_row = p.ws.chunks_per_row;
+  a.gsplits = p.ws.gsplits;
+  a.g_tokens_per_split = p.ws.g_tokens_per_split;
   a.max_pages_per_seq = cache->max_pages_per_seq;
   a.num_pages = cache->num_pages;
   a.scale_log2 = p.scale * 1.4426950408889634f;

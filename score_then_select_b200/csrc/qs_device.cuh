@@ -90,6 +90,29 @@ QS_DEV void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint6
       : "memory");
 }
 
+// 2-D tiled tensor copy (TMA unit) of one box at element coordinates (x, y) of the tensor
+// map, signalling completion on `bar` through its transaction count. x * element size
+// must be a multiple of 16 bytes; y may lie outside the tensor (out-of-range rows are
+// filled with zeros). No cluster multicast.
+QS_DEV void tma_load_2d(void* dst_smem, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst_smem)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y),
+        "r"(smem_u32(bar))
+      : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued before has landed; the arrival
+// is not added to the pending count (the barrier's expected count includes it).
+QS_DEV void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// Barrier among `nthreads` threads (whole warps) of the CTA on hardware barrier `id`.
+QS_DEV void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async (16 bytes)
 QS_DEV void cp_async16(void* dst_smem, const void* src_gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)),
@@ -100,6 +123,11 @@ QS_DEV void cp_async16_zfill(void* dst_smem, const void* src_gmem, bool valid) {
   // src-size 0 writes 16 zero bytes without reading global memory
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)),
                "l"(src_gmem), "r"(valid ? 16 : 0)
+               : "memory");
+}
+QS_DEV void cp_async4(void* dst_smem, const void* src_gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)),
+               "l"(src_gmem)
                : "memory");
 }
 QS_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }

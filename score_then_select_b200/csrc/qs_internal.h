@@ -26,6 +26,10 @@ constexpr int kMaxGroup = 8;        // query heads per KV head
 constexpr int kMaxSelectBlocks = 32768;
 constexpr int kHdrWords = 64;       // workspace header (256 bytes)
 constexpr int kCtrAppend = 16;      // header word: append "last CTA" counter
+constexpr int kAttnCtasPerSm = 2;   // resident attention CTAs per SM (shared-memory bound)
+constexpr int kAttnTmaMinRun = 8;   // shorter selected runs (block size) use the gather kernel
+constexpr int kChunkTilesMax = 8;   // attention work unit: up to 8 tiles (512 slots) of one row
+constexpr int kCtrAttnNext = 17;    // header word: next attention chunk to claim
 
 // Workspace carve-up (byte offsets); computed identically by qs_workspace_size and calls.
 struct WsLayout {
@@ -35,13 +39,18 @@ struct WsLayout {
   size_t scores = 0;    // [batch][Hkv][nb_stride] f32
   size_t sel = 0;       // [batch][Hkv][budget] i32
   size_t nsel = 0;      // [batch][Hkv] i32
-  size_t part_ml = 0;   // [batch][Hq][splits][2] f32
-  size_t part_o = 0;    // [batch][Hq][splits][d] f32
-  size_t row_ctr = 0;   // [batch][Hkv] u32 attention split counters
+  size_t part_ml = 0;   // [batch][Hq][parts_per_head][2] f32 attention partials (m, l)
+  size_t part_o = 0;    // [batch][Hq][parts_per_head][d] f32 attention partials o
+  size_t row_ctr = 0;   // [batch][Hkv] u32 attention segments finished per row
   size_t total = 0;
   int nb_stride = 0;
-  int splits = 0;       // attention splits per row
-  int tokens_per_split = 0;
+  int attn_ctas = 0;     // attention grid (persistent; chunks claimed dynamically)
+  int tiles_per_row = 0; // 64-token tiles of selected slots per row
+  int chunk_tiles = 0;   // tiles per attention chunk: min(8, 32 / runs per tile)
+  int chunks_per_row = 0;  // chunks per row (one partial each)
+  int gsplits = 0;      // gather kernel (runs < kAttnTmaMinRun): splits per row
+  int g_tokens_per_split = 0;
+  int parts_per_head = 0;  // attention partials per query head in the workspace
 };
 
 struct Plan {
@@ -161,10 +170,14 @@ struct AttnParams {
   const int32_t* seq_lens;
   float* part_ml;
   float* part_o;
-  uint32_t* row_ctr;         // [batch * Hkv] splits finished (self-resetting)
+  uint32_t* row_ctr;         // [batch * Hkv] segments finished (self-resetting)
   void* out;
   uint32_t* hdr;
-  int batch, Hkv, G, S, budget, splits, tokens_per_split, max_pages_per_seq, num_pages;
+  int rows, Hkv, G, S, budget, tiles_per_row, chunk_tiles, chunks_per_row, max_pages_per_seq,
+      num_pages;
+  int run_h;                 // min(S, 64): rows of one box copy
+  int log2_S, log2_run;
+  int gsplits, g_tokens_per_split;   // gather kernel split plan
   int out_bf16;
   float scale_log2;          // softmax scale * log2(e)
 };
@@ -194,6 +207,7 @@ cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s);
 cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s);
 cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s, bool pdl);
+cudaError_t launch_attn_gather(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl);
 
 int num_sms();
