@@ -383,9 +383,9 @@ def run_ours(args):
         raise RuntimeError(f"device status {st}")
     nsel_h = nsel.cpu().numpy()
     sel_h = sel.cpu().numpy()
-    # append [+ block errors + query tiles] + score + select + attention [+ row merge when
-    # the selected runs are >= 8 slots; shorter runs merge inside the attention kernel]
-    launches_per_step = (4 if w.proxy_rank > 0 else 6) + (1 if w.block_size >= 8 else 0)
+    # append [+ block errors + query tiles] + score + select + attention (1 or 2 launches)
+    launches_per_step = (3 if w.proxy_rank > 0 else 5) + qs.qs_attention_launches(
+        lay.cfg, w.batch, lay.max_context)
 
     def barrier():
         if world > 1:

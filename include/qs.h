@@ -33,6 +33,8 @@
  *   - Arguments are validated on the host before any launch. On failure the call returns
  *     QS_ERR_INVALID_ARG (bad pointer/size) or QS_ERR_UNSUPPORTED (a shape this build does
  *     not implement) and launches nothing. There is no fallback path.
+ *   - Cache tensors (K, V, proxy) and q must be 16-byte aligned (q may be 4-byte aligned
+ *     for qs_score on the rank-r path).
  *   - Values that live on the device (sequence lengths, page-table entries, n_new, the
  *     selection) are checked by the kernels: an out-of-range value skips the access and
  *     records QS_ERR_DEVICE_BOUNDS in the workspace status word, which qs_device_status
@@ -100,6 +102,11 @@ typedef struct {
   int32_t n_keep_hp;      /* NVFP4: 0..2 blocks with the largest quantisation error are
                              kept at full precision and always selected                  */
   float softmax_scale;    /* 0 => 1/sqrt(d)                                               */
+  int32_t attn_path;      /* attention kernel: 0 chosen per shape (the tile pipeline when
+                             block_size >= 8 and there are >= 40 tiles of 64 selected slots
+                             per resident CTA, else the gather kernel); 1 tile pipeline
+                             (needs block_size >= 8); 2 gather kernel. Same results up to
+                             float32 summation order.                                    */
 } qs_config;
 
 /* The paged caches of one layer. All pointers are device pointers owned by the caller. */
@@ -123,6 +130,11 @@ typedef struct {
    device access). QS_ERR_INVALID_ARG / QS_ERR_UNSUPPORTED as for the other calls. */
 qs_status qs_workspace_size(const qs_config *cfg, int32_t batch, int32_t max_context,
                             size_t *bytes /* host */);
+
+/* Number of kernel launches qs_sparse_attn makes for this shape (1: gather kernel with an
+   in-kernel merge; 2: tile pipeline, then the row merge). Host only. */
+qs_status qs_attention_launches(const qs_config *cfg, int32_t batch, int32_t max_context,
+                                int32_t *launches /* host */);
 
 /* Zero the whole workspace (status word and counters; async on stream). Call once after
    allocating a workspace, before any other call uses it. */
@@ -171,7 +183,7 @@ qs_status qs_select_topk(const qs_config *cfg, const qs_cache *cache,
    t in the selected blocks (t < seq_len), normalised over those tokens only. Logits are
    float32 sums of BF16 products; P.V operands are v_agg_dtype, accumulated in float32.
    The selection is split across CTAs; partial (max, sum, o) states are merged by a
-   log-sum-exp combine. out: [batch][Hq][d] in out_dtype. */
+   log-sum-exp combine. out: [batch][Hq][d] in out_dtype. q is 16-byte aligned. */
 qs_status qs_sparse_attn(const qs_config *cfg, const qs_cache *cache, const void *q,
                          const int32_t *sel, const int32_t *n_sel, int32_t batch, void *out,
                          void *ws, qs_stream_t stream);

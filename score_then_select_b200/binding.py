@@ -28,7 +28,8 @@ class qs_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "n_q_heads", "n_kv_heads", "head_dim", "page_size", "block_size", "budget",
         "proxy_rank", "proxy_dtype", "v_dtype", "v_agg_dtype", "out_dtype", "force_sink",
-        "force_last", "n_keep_hp")] + [("softmax_scale", ctypes.c_float)]
+        "force_last", "n_keep_hp")] + [("softmax_scale", ctypes.c_float),
+                                         ("attn_path", ctypes.c_int32)]
 
 
 class qs_cache(ctypes.Structure):
@@ -58,6 +59,7 @@ def lib() -> ctypes.CDLL:
             "qs_status_string": ([i32], ctypes.c_char_p),
             "qs_workspace_size": ([cfgp, i32, i32, ctypes.POINTER(sz)], i32),
             "qs_workspace_init": ([vp, sz, vp], i32),
+            "qs_attention_launches": ([cfgp, i32, i32, ctypes.POINTER(i32)], i32),
             "qs_append_kv": ([cfgp, cachep, vp, vp, vp, i32, vp, i32, vp, vp], i32),
             "qs_score": ([cfgp, cachep, vp, vp, i32, vp, vp, vp], i32),
             "qs_select_topk": ([cfgp, cachep, vp, i32, vp, vp, vp, vp], i32),
@@ -76,7 +78,7 @@ def lib() -> ctypes.CDLL:
 
 EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_init",
            "qs_append_kv", "qs_score", "qs_select_topk", "qs_sparse_attn", "qs_decode",
-           "qs_device_status", "qs_sparse_attn_noalloc")
+           "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches")
 
 
 def status_string(s: int) -> str:
@@ -108,7 +110,7 @@ def _check(st: int, where: str):
 def make_config(*, n_q_heads, n_kv_heads, head_dim, block_size, budget, proxy_rank,
                 proxy_dtype, v_dtype="bf16", v_agg_dtype="bf16", out_dtype="bf16",
                 force_sink=False, force_last=False, n_keep_hp=0, softmax_scale=0.0,
-                page_size=128) -> qs_config:
+                page_size=128, attn_path=0) -> qs_config:
     c = qs_config()
     c.n_q_heads, c.n_kv_heads, c.head_dim = n_q_heads, n_kv_heads, head_dim
     c.page_size, c.block_size, c.budget = page_size, block_size, budget
@@ -118,6 +120,7 @@ def make_config(*, n_q_heads, n_kv_heads, head_dim, block_size, budget, proxy_ra
     c.out_dtype = DTYPE_CODES[out_dtype]
     c.force_sink, c.force_last, c.n_keep_hp = int(force_sink), int(force_last), n_keep_hp
     c.softmax_scale = softmax_scale
+    c.attn_path = attn_path
     return c
 
 
@@ -144,6 +147,13 @@ def qs_workspace_size(cfg: qs_config, batch: int, max_context: int) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().qs_workspace_size(ctypes.byref(cfg), batch, max_context, ctypes.byref(n)),
            "qs_workspace_size")
+    return n.value
+
+
+def qs_attention_launches(cfg: qs_config, batch: int, max_context: int) -> int:
+    n = ctypes.c_int32(0)
+    _check(lib().qs_attention_launches(ctypes.byref(cfg), batch, max_context, ctypes.byref(n)),
+           "qs_attention_launches")
     return n.value
 
 

@@ -58,10 +58,14 @@ static void plan_gather_splits(int rows, int slots, int& splits, int& tps) {
 static void plan_attention(int rows, long long slots, int S, WsLayout& w) {
   const long long tpr = (slots + 63) / 64;
   const int runs_per_tile = S >= 64 ? 1 : 64 / S;         // a chunk's runs fit one warp
-  const int kt = std::max(1, std::min(kChunkTilesMax, 32 / runs_per_tile));
+  const int kt_max = std::max(1, std::min(kChunkTilesMax, 32 / runs_per_tile));
+  // about kChunksPerCta chunks per CTA, so the dynamic claims can even out the CTAs' speeds
+  const long long ctas = (long long)kAttnCtasPerSm * num_sms();
+  const long long want = rows * tpr / (ctas * kChunksPerCta);
+  const int kt = int(std::max(1LL, std::min<long long>(kt_max, want)));
   const long long cpr = (tpr + kt - 1) / kt;
   const long long chunks = rows * cpr;                   // < 2^31: checked by the caller
-  long long C = (long long)kAttnCtasPerSm * num_sms();
+  long long C = ctas;
   if (C > chunks) C = chunks;
   w.tiles_per_row = int(tpr);
   w.chunk_tiles = kt;
@@ -126,12 +130,20 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   WsLayout& w = p.ws;
   w.nb_stride = p.nb_stride;
   if ((long long)batch * p.Hkv * ((slots + 63) / 64) >= (1LL << 31)) return QS_ERR_UNSUPPORTED;
-  plan_attention(batch * p.Hkv, slots, p.S, w);
-  if (p.S < kAttnTmaMinRun) {
+  if (c->attn_path < 0 || c->attn_path > 2) return QS_ERR_INVALID_ARG;
+  if (c->attn_path == 1 && p.S < kAttnTmaMinRun) return QS_ERR_UNSUPPORTED;
+  {
+    const long long tiles = (long long)batch * p.Hkv * ((slots + 63) / 64);
+    const long long ctas = (long long)kAttnCtasPerSm * num_sms();
+    p.attn_tma = c->attn_path == 1 ||
+                 (c->attn_path == 0 && p.S >= kAttnTmaMinRun && tiles >= kTmaMinTilesPerCta * ctas);
+  }
+  if (p.attn_tma) {
+    plan_attention(batch * p.Hkv, slots, p.S, w);
+    w.parts_per_head = w.chunks_per_row;
+  } else {
     plan_gather_splits(batch * p.Hkv, int(slots), w.gsplits, w.g_tokens_per_split);
     w.parts_per_head = w.gsplits;
-  } else {
-    w.parts_per_head = w.chunks_per_row;
   }
   size_t off = size_t(kHdrWords) * 4;
   const size_t rows = size_t(batch) * p.Hkv, rows_q = size_t(batch) * p.Hq;
@@ -337,6 +349,16 @@ qs_status qs_workspace_size(const qs_config* cfg, int32_t batch, int32_t max_con
   return QS_OK;
 }
 
+qs_status qs_attention_launches(const qs_config* cfg, int32_t batch, int32_t max_context,
+                                int32_t* launches) {
+  Plan p;
+  const qs_status st = make_plan(cfg, batch, max_context, p);
+  if (st != QS_OK) return st;
+  if (!launches) return QS_ERR_INVALID_ARG;
+  *launches = p.attn_tma ? 2 : 1;
+  return QS_OK;
+}
+
 qs_status qs_workspace_init(void* ws, size_t ws_bytes, qs_stream_t stream) {
   if (!ws || ws_bytes < size_t(kHdrWords) * 4 || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, stream));
@@ -387,7 +409,7 @@ qs_status qs_sparse_attn(const qs_config* cfg, const qs_cache* cache, const void
   qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
   if (st != QS_OK) return st;
   if ((st = check_cache(p, cache, false)) != QS_OK) return st;
-  if (!q || !aligned(q, 4) || !sel || !n_sel || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (!q || !aligned(q, 16) || !sel || !n_sel || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   return do_attend(p, cache, q, sel, n_sel, out, ws, stream, false);
 }
 
@@ -398,7 +420,7 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
   if (st != QS_OK) return st;
   if ((st = check_cache(p, cache, true)) != QS_OK) return st;
-  if (!q || !aligned(q, 4) || !k_new || !v_new || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (!q || !aligned(q, 16) || !k_new || !v_new || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
   if (p.r == 0 && (!cache->block_err || !aligned(q, 16))) return QS_ERR_INVALID_ARG;

@@ -1,5 +1,6 @@
-// attn.cu - sparse attention over the selected blocks with its LSE combine (selected runs
-// of >= 8 slots; shorter runs use attn_gather.cu).
+// attn.cu - sparse attention over the selected blocks with its LSE combine: the tile
+// pipeline for selected runs of >= 8 slots and enough work per CTA (otherwise
+// attn_gather.cu).
 //
 // "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 1 and
 // Abstract: gather-free indexed attention reads the original full-dimensional keys and
@@ -10,19 +11,19 @@
 //
 // Work decomposition (persistent grid, dynamic): a row (sequence, KV head) holds
 // `tiles_per_row` 64-token tiles of selected slots, cut into chunks of `chunk_tiles` tiles;
-// CTAs claim chunks in order from a workspace counter, so CTAs that the memory system
-// serves faster simply take more chunks, and a row is finished (and merged) as soon as its
-// last chunk is, instead of at the end of the kernel.
+// CTA c starts with chunks c and c + C, then claims the rest in order from a workspace
+// counter, so CTAs that the memory system serves faster simply take more chunks.
 //
 // Warp roles (warp-specialised; no block-wide barrier in the loop):
-//   * producer warp (warp 4): claims chunks two ahead and resolves the chunk's runs
+//   * producer warp (warp 4): claims chunks ahead and resolves the chunk's runs
 //     (a run is min(S, 64) slots of one selected block: lane = run) through selection
 //     entry -> page table in a pipeline one chunk apart per stage; then fills one stage of
 //     the shared-memory ring per tile: full and empty runs move as 64-element x run-height
 //     boxes by the TMA unit (tensor maps over the K and V caches, 128-byte swizzle; empty
 //     runs read zeros from outside the tensor), a ragged last block by 16-byte cp.async
-//     with zero fill, and the first tile of a chunk also brings the row's queries. Both
-//     kinds of copy are counted on the stage's `full` barrier; per-stage metadata carries
+//     with zero fill (counted on the stage's ragged-copy barrier), and the first tile of a
+//     chunk also brings the row's queries (a bulk copy). The box and bulk copies are counted
+//     on the stage's `full` barrier by their bytes; per-stage metadata carries
 //     the valid-slot mask and the chunk's identity. After the last chunk it posts an end
 //     marker.
 //   * consumer warps (warps 0-3): each owns 16 tokens of every tile and keeps its own
@@ -60,8 +61,8 @@ struct AttnSmem {
   static constexpr int kQBytes = (kMaxGroup * D * 2 + 1023) / 1024 * 1024;
   static constexpr int kStageBytes = 2 * kTileBytes + kQBytes;      // multiple of 1024
   static constexpr int kMetaOff = kAttnStages * kStageBytes;        // u32 [stages][4]
-  static constexpr int kBarOff = kMetaOff + kAttnStages * 16;       // u64 full[], empty[]
-  static constexpr int kMlOff = kBarOff + 2 * kAttnStages * 8;      // f32 [2][m [4][8], l [4][8]]
+  static constexpr int kBarOff = kMetaOff + kAttnStages * 16;       // u64 full[], empty[], rag[]
+  static constexpr int kMlOff = kBarOff + 3 * kAttnStages * 8;      // f32 [2][m [4][8], l [4][8]]
   static constexpr int kMiscOff = kMlOff + 2 * 64 * 4;              // i32 abort, u64 barrier
   static constexpr int kScrOff = kMiscOff + 16;                     // merge buffer
   static constexpr int kBufStride = D + 4;                          // floats per head (merge)
@@ -88,8 +89,10 @@ QS_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
   return false;
 }
 
-// Per-stage metadata word 3: chunk-in-row | first-tile flag | last-tile flag.
+// Per-stage metadata word 3: chunk-in-row | first-tile flag | last-tile flag | ragged-copy
+// flag | phase parity of the stage's ragged-copy barrier.
 constexpr uint32_t kMetaFirst = 1u << 16, kMetaLast = 1u << 17;
+constexpr uint32_t kMetaRag = 1u << 18, kMetaRagPhase = 1u << 19;
 
 // Barrier of the four consumer warps on an mbarrier (count 4), bounded like every wait
 // here: a warp that gives up cannot leave the others waiting on a hardware barrier.
@@ -115,6 +118,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
   uint32_t* meta = reinterpret_cast<uint32_t*>(smem + SM::kMetaOff);   // [stage][mask lo, hi, row, info]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
   uint64_t* empty = full + NS;
+  uint64_t* rag = empty + NS;       // ragged-run copies of a stage (one cp.async arrival per lane)
   float* s_ml = reinterpret_cast<float*>(smem + SM::kMlOff);         // [2][m [4][8], l [4][8]]
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::kMiscOff);
   uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + SM::kMiscOff + 8);
@@ -123,8 +127,9 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1 + 32);            // producer lane 0 + one cp.async arrival per lane
+      mbar_init(&full[s], 1);                 // producer lane 0 (with the stage's byte count)
       mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&rag[s], 32);
       meta[4 * s + 2] = 0xffffffffu;          // an unfilled stage reads as the end marker
     }
     mbar_init(cbar, kConsumerWarps);
@@ -201,44 +206,65 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
       y = (x.pg * a.Hkv + x.g) * kPage + (x.t0 & (kPage - 1));
     };
 
-    // chunk claims: three in flight from the start, then one per chunk, two chunks ahead
-    unsigned claim0 = 0, claim1 = 0, pend = 0;
+    // chunks: the first two of each CTA are fixed (blockIdx, blockIdx + C), the rest are
+    // claimed from the counter (value + 2C), two claims in flight, each used two chunks
+    // after it is issued (an atomic on the shared counter is slow under full HBM load)
+    const unsigned C2 = 2u * gridDim.x;
+    unsigned pend_a = 0, pend_b = 0;
     if (lane == 0) {
-      claim0 = atomicAdd(next_ctr, 1u);
-      claim1 = atomicAdd(next_ctr, 1u);
-      pend = atomicAdd(next_ctr, 1u);
+      pend_a = atomicAdd(next_ctr, 1u) + C2;
+      pend_b = atomicAdd(next_ctr, 1u) + C2;
     }
-    int c_cur = int(min(__shfl_sync(kFull, claim0, 0), unsigned(nchunks)));
-    int c_n1 = int(min(__shfl_sync(kFull, claim1, 0), unsigned(nchunks)));
+    int c_cur = int(min(blockIdx.x, unsigned(nchunks)));
+    int c_n1 = int(min(blockIdx.x + gridDim.x, unsigned(nchunks)));
     RunA pa = stage_a(c_n1);
     RunB pb = stage_b(c_cur, stage_a(c_cur));
 
     const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k);
     const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v);
     int t = 0;                                             // stages filled so far
+    int kseq = 0;                                          // chunks started by this CTA
+    uint32_t rag_uses = 0;                                 // bit s: parity of stage s's ragged uses
     bool ok = true;
     while (ok && c_cur < nchunks) {
       int run_y, run_cnt;
       stage_c(pb, run_y, run_cnt);
       pb = stage_b(c_n1, pa);
-      const int c_n2 = int(min(__shfl_sync(kFull, pend, 0), unsigned(nchunks)));
+      // the two pending claims alternate by chunk parity: neither register is touched
+      // until two chunks after its atomic was issued
+      int c_n2;
+      if ((kseq & 1) == 0) {
+        c_n2 = int(min(__shfl_sync(kFull, pend_a, 0), unsigned(nchunks)));
+        if (lane == 0) pend_a = c_n2 < nchunks ? atomicAdd(next_ctr, 1u) + C2 : unsigned(nchunks);
+      } else {
+        c_n2 = int(min(__shfl_sync(kFull, pend_b, 0), unsigned(nchunks)));
+        if (lane == 0) pend_b = c_n2 < nchunks ? atomicAdd(next_ctr, 1u) + C2 : unsigned(nchunks);
+      }
+      ++kseq;
       pa = stage_a(c_n2);
-      if (lane == 0) pend = c_n2 < nchunks ? atomicAdd(next_ctr, 1u) : unsigned(nchunks);
 
       const int row = c_cur / cpr, ci = c_cur - row * cpr;
       const int nt = min(ktiles, tpr - ci * ktiles);
       const int b = row / a.Hkv, g = row - b * a.Hkv;
-      for (int j = 0; j < nt; ++j, ++t) {
-        // the tile's runs: lane r < rpt takes run r
-        const int src = (j << (6 - lg_hb)) + (lane & (rpt - 1));
-        const int ry = __shfl_sync(kFull, run_y, src), rc = __shfl_sync(kFull, run_cnt, src);
-        unsigned long long mask = 0;
-        uint32_t tma_bytes = 0;
-        for (int r = 0; r < rpt; ++r) {
-          const int cr = __shfl_sync(kFull, rc, r);
-          if (cr > 0) mask |= (cr >= 64 ? ~0ull : ((1ull << cr) - 1)) << (r << lg_hb);
-          if (cr == 0 || cr == hb) tma_bytes += uint32_t(2 * SM::kHalves * hb * 128);
+      // per-tile summary, lane j for tile j of the chunk: valid-slot mask, box bytes,
+      // whether a ragged run needs the 16-byte copy path
+      uint32_t t_lo = 0, t_hi = 0, t_bytes = 0, t_rag = 0;
+      for (int r = 0; r < rpt; ++r) {
+        const int cr = __shfl_sync(kFull, run_cnt, ((lane << (6 - lg_hb)) + r) & 31);
+        if (cr > 0) {
+          const unsigned long long m = (cr >= 64 ? ~0ull : ((1ull << cr) - 1)) << (r << lg_hb);
+          t_lo |= uint32_t(m);
+          t_hi |= uint32_t(m >> 32);
         }
+        if (cr == 0 || cr == hb) t_bytes += uint32_t(2 * SM::kHalves * hb * 128);
+        else t_rag = 1;
+      }
+      const uint32_t q_bytes = uint32_t(a.G * D * 2);
+      const uint16_t* qrow = a.q + (size_t(b) * Hq + g * a.G) * D;
+      // box copy owned by this lane: run lane / (2 halves), column half, K or V
+      const int box_r = lane / (2 * SM::kHalves), box_h = (lane >> 1) % SM::kHalves, box_v = lane & 1;
+      const bool box_lane = lane < rpt * SM::kHalves * 2;
+      for (int j = 0; j < nt; ++j, ++t) {
         const int s = t % NS;
         bool got = true;
         if (lane == 0 && t >= NS) got = wait_or_abort(&empty[s], ((t / NS) - 1) & 1, s_abort);
@@ -247,45 +273,53 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
         if (!ok) break;
 
         uint8_t* st = smem + s * SM::kStageBytes;
-        if (j == 0) {                                      // a chunk starts: the row's queries
-          const uint16_t* qr = a.q + (size_t(b) * Hq + g * a.G) * D;
-          for (int w = lane; w < a.G * D / 2; w += 32)
-            cp_async4(st + 2 * SM::kTileBytes + 4 * w, qr + 2 * w);
-        }
-        if (lane == 0) {
-          meta[4 * s] = uint32_t(mask);
-          meta[4 * s + 1] = uint32_t(mask >> 32);
-          meta[4 * s + 2] = uint32_t(row);
-          meta[4 * s + 3] = uint32_t(ci) | (j == 0 ? kMetaFirst : 0u) | (j + 1 == nt ? kMetaLast : 0u);
-          mbar_arrive_expect_tx(&full[s], tma_bytes);
-        }
-        __syncwarp();                                      // the byte count is posted first
-        // full and empty runs: box copies (an empty run reads zeros from outside the tensor)
-        if (lane < rpt && (rc == 0 || rc == hb)) {
-          const int y = rc ? ry : -hb;
+        const uint32_t lo = __shfl_sync(kFull, t_lo, j), hi = __shfl_sync(kFull, t_hi, j);
+        const uint32_t bytes = __shfl_sync(kFull, t_bytes, j) + (j == 0 ? q_bytes : 0u);
+        const bool ragged = __shfl_sync(kFull, t_rag, j) != 0;
+        uint32_t rag_bits = 0;
+        if (ragged) {
+          // a ragged run: 16-byte copies of its valid rows, zeros for the rest, counted on
+          // the stage's ragged-copy barrier (its phase parity travels in the metadata)
+          rag_bits = kMetaRag | ((rag_uses >> s) & 1u ? kMetaRagPhase : 0u);
+          rag_uses ^= 1u << s;
+          for (int r = 0; r < rpt; ++r) {
+            const int src = (j << (6 - lg_hb)) + r;
+            const int cr = __shfl_sync(kFull, run_cnt, src), y0 = __shfl_sync(kFull, run_y, src);
+            if (cr == 0 || cr == hb) continue;
+            for (int i = lane; i < hb; i += 32) {
+              const int rt = (r << lg_hb) + i;
+              const bool v = i < cr;
+              const size_t off = size_t(v ? y0 + i : 0) * (D * 2);
 #pragma unroll
-          for (int h = 0; h < SM::kHalves; ++h) {
-            const uint32_t off = h * kHalfBytes + ((lane << lg_hb) << 7);
-            tma_load_2d(st + off, &tm_k, 64 * h, y, &full[s]);
-            tma_load_2d(st + SM::kTileBytes + off, &tm_v, 64 * h, y, &full[s]);
-          }
-        }
-        // a ragged run: 16-byte copies of its valid rows, zeros for the rest
-        for (int r = 0; r < rpt; ++r) {
-          const int cr = __shfl_sync(kFull, rc, r), y0 = __shfl_sync(kFull, ry, r);
-          if (cr == 0 || cr == hb) continue;
-          for (int i = lane; i < hb; i += 32) {
-            const int rt = (r << lg_hb) + i;
-            const bool v = i < cr;
-            const size_t off = size_t(v ? y0 + i : 0) * (D * 2);
-#pragma unroll
-            for (int ch = 0; ch < CH; ++ch) {
-              cp_async16_zfill(st + swz(rt, ch), kbase + off + ch * 16, v);
-              cp_async16_zfill(st + SM::kTileBytes + swz(rt, ch), vbase + off + ch * 16, v);
+              for (int ch = 0; ch < CH; ++ch) {
+                cp_async16_zfill(st + swz(rt, ch), kbase + off + ch * 16, v);
+                cp_async16_zfill(st + SM::kTileBytes + swz(rt, ch), vbase + off + ch * 16, v);
+              }
             }
           }
+          cp_async_mbar_arrive_noinc(&rag[s]);
         }
-        cp_async_mbar_arrive_noinc(&full[s]);
+        if (lane == 0) {
+          meta[4 * s] = lo;
+          meta[4 * s + 1] = hi;
+          meta[4 * s + 2] = uint32_t(row);
+          meta[4 * s + 3] = uint32_t(ci) | (j == 0 ? kMetaFirst : 0u) | (j + 1 == nt ? kMetaLast : 0u) |
+                            rag_bits;
+          mbar_arrive_expect_tx(&full[s], bytes);
+        }
+        __syncwarp();                                      // the byte count is posted first
+        // full and empty runs: one box copy per lane (an empty run reads zeros from outside
+        // the tensor); a chunk's first tile also brings the row's queries
+        {
+          const int src = ((j << (6 - lg_hb)) + box_r) & 31;
+          const int ry = __shfl_sync(kFull, run_y, src), rc = __shfl_sync(kFull, run_cnt, src);
+          if (box_lane && (rc == 0 || rc == hb)) {
+            const uint32_t off = (box_v ? SM::kTileBytes : 0) + box_h * kHalfBytes + ((box_r << lg_hb) << 7);
+            tma_load_2d(st + off, box_v ? static_cast<const void*>(&tm_v) : static_cast<const void*>(&tm_k),
+                        64 * box_h, rc ? ry : -hb, &full[s]);
+          }
+        }
+        if (j == 0 && lane == 0) bulk_g2s(st + 2 * SM::kTileBytes, qrow, q_bytes, &full[s]);
       }
       c_cur = c_n1;
       c_n1 = c_n2;
@@ -302,16 +336,16 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
           meta[4 * s + 2] = 0xffffffffu;
           mbar_arrive_expect_tx(&full[s], 0u);
         }
-        cp_async_mbar_arrive_noinc(&full[s]);
         ++t;
       }
     }
     // every copy issued must land before the CTA exits
+    cp_async_commit();
+    cp_async_wait<0>();
     if (lane == 0) {
       for (int j = t > NS ? t - NS : 0; j < t; ++j)
         if (!mbar_wait(&full[j % NS], (j / NS) & 1)) *s_abort = 1;
     }
-    if (lane == 0 && pend > 0x7fffffffu) *s_abort = 1;     // the last claim has returned
     __syncwarp();
     return;
   }
@@ -331,6 +365,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     const int row = int(meta[4 * s + 2]);
     const uint32_t info = meta[4 * s + 3];
     if (row < 0 || row >= a.rows || int(info & 0xffffu) >= cpr) break;   // end marker
+    if ((info & kMetaRag) && !wait_or_abort(&rag[s], (info & kMetaRagPhase) ? 1u : 0u, s_abort)) break;
     const uint8_t* st = smem + s * SM::kStageBytes;
     if (info & kMetaFirst) {
       // query fragments (B operand of S^T): head = lane/4, dims 2*(lane%4)+{0,1}
@@ -636,7 +671,7 @@ static cudaError_t launch_attn_t(const AttnParams& a, const CUtensorMap& mk, con
 }
 
 cudaError_t launch_attn(const Plan& p, const AttnParams& a_in, cudaStream_t s, bool pdl) {
-  if (p.S < kAttnTmaMinRun) return launch_attn_gather(p, a_in, s, pdl);
+  if (!p.attn_tma) return launch_attn_gather(p, a_in, s, pdl);
   AttnParams a = a_in;
   a.run_h = p.S < kTileT ? p.S : kTileT;
   a.log2_S = 0;

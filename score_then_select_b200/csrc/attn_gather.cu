@@ -1,5 +1,6 @@
-// attn_gather.cu - split-K sparse attention for selections of short runs (block size < 8),
-// e.g. token-level selection, with its LSE combine.
+// attn_gather.cu - split-K sparse attention with its LSE combine, for selections of short
+// runs (block size < 8, e.g. token-level selection) and for shapes with too little work per
+// CTA for the tile pipeline of attn.cu (one CTA per (row, split), no separate merge launch).
 //
 // "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 1 and
 // Abstract: gather-free indexed attention reads the original full-dimensional keys and

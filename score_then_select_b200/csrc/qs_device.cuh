@@ -125,11 +125,6 @@ QS_DEV void cp_async16_zfill(void* dst_smem, const void* src_gmem, bool valid) {
                "l"(src_gmem), "r"(valid ? 16 : 0)
                : "memory");
 }
-QS_DEV void cp_async4(void* dst_smem, const void* src_gmem) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)),
-               "l"(src_gmem)
-               : "memory");
-}
 QS_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 QS_DEV void cp_async_wait() {

@@ -29,6 +29,8 @@ constexpr int kCtrAppend = 16;      // header word: append "last CTA" counter
 constexpr int kAttnCtasPerSm = 2;   // resident attention CTAs per SM (shared-memory bound)
 constexpr int kAttnTmaMinRun = 8;   // shorter selected runs (block size) use the gather kernel
 constexpr int kChunkTilesMax = 8;   // attention work unit: up to 8 tiles (512 slots) of one row
+constexpr int kChunksPerCta = 6;    // chunk size target: about this many chunks per CTA
+constexpr int kTmaMinTilesPerCta = 40;  // auto path: tile pipeline from this much work per CTA
 constexpr int kCtrAttnNext = 17;    // header word: next attention chunk to claim
 
 // Workspace carve-up (byte offsets); computed identically by qs_workspace_size and calls.
@@ -48,13 +50,14 @@ struct WsLayout {
   int tiles_per_row = 0; // 64-token tiles of selected slots per row
   int chunk_tiles = 0;   // tiles per attention chunk: min(8, 32 / runs per tile)
   int chunks_per_row = 0;  // chunks per row (one partial each)
-  int gsplits = 0;      // gather kernel (runs < kAttnTmaMinRun): splits per row
+  int gsplits = 0;      // gather kernel: splits per row
   int g_tokens_per_split = 0;
   int parts_per_head = 0;  // attention partials per query head in the workspace
 };
 
 struct Plan {
   int batch, Hq, Hkv, G, d, S, budget, r, nb_stride;
+  bool attn_tma;        // attention by the tile pipeline (else the gather kernel)
   int proxy_dtype, v_dtype, v_agg_dtype, out_dtype;
   int force_sink, force_last, n_keep;
   float scale;

@@ -8,12 +8,12 @@ import score_then_select_b200 as qs
 from score_then_select_b200.layer import Layer
 
 
-def cfg_kwargs(w: synth.Workload) -> dict:
+def cfg_kwargs(w: synth.Workload, attn_path: int = 0) -> dict:
     return dict(n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
                 block_size=w.block_size, budget=w.budget, proxy_rank=w.proxy_rank,
                 proxy_dtype=w.proxy_dtype, v_dtype=w.v_dtype, v_agg_dtype=w.v_agg_dtype,
                 out_dtype=w.out_dtype, force_sink=w.force_sink, force_last=w.force_last,
-                n_keep_hp=w.n_keep_hp, softmax_scale=w.softmax_scale)
+                n_keep_hp=w.n_keep_hp, softmax_scale=w.softmax_scale, attn_path=attn_path)
 
 
 def u16(a: np.ndarray, dt=torch.bfloat16) -> torch.Tensor:
@@ -23,7 +23,7 @@ def u16(a: np.ndarray, dt=torch.bfloat16) -> torch.Tensor:
 class Filled:
     """A layer holding L_b - 1 tokens per sequence, ready for one decode step."""
 
-    def __init__(self, inp: synth.Inputs, dense=None, device="cuda"):
+    def __init__(self, inp: synth.Inputs, dense=None, device="cuda", attn_path: int = 0):
         w = inp.w
         self.inp, self.w = inp, w
         lens = inp.lens
@@ -31,7 +31,7 @@ class Filled:
         self.K, self.V, self.Q = K, V, Q
         Lmax = int(lens.max())
         vdt = torch.float16 if w.v_dtype == "f16" else torch.bfloat16
-        self.layer = Layer.allocate(cfg_kwargs(w), w.batch, inp.num_pages,
+        self.layer = Layer.allocate(cfg_kwargs(w, attn_path), w.batch, inp.num_pages,
                                     inp.page_table.shape[1], Lmax, device)
         lay = self.layer
         lay.page_table.copy_(torch.from_numpy(inp.page_table))

@@ -15,7 +15,10 @@ from tests.util import oracle_row
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-FULL = [synth.BLOCK128K, synth.NVFP4_128K, synth.TOKEN32K, synth.RAGGED]
+# (workload, attention kernel): the automatic choice everywhere, and the tile pipeline
+# forced on the ragged workload (whose rows end in partial blocks)
+FULL = [(synth.BLOCK128K, 0), (synth.NVFP4_128K, 0), (synth.TOKEN32K, 0), (synth.RAGGED, 0),
+        (synth.RAGGED, 1)]
 
 
 def _check_all_rows(w, inp, sel, nsel, out, berr):
@@ -41,14 +44,15 @@ def _check_all_rows(w, inp, sel, nsel, out, berr):
             assert np.all(np.isfinite(out[b, g * G:(g + 1) * G]))
 
 
-@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
-def test_fullsize_sampled_rows(w):
+@pytest.mark.parametrize("case", FULL, ids=lambda c: f"{c[0].name}-path{c[1]}")
+def test_fullsize_sampled_rows(case):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from tests.gpu_util import Filled, out_to_f64
     from tests.util import query_scale_all
+    w, path = case
     inp = synth.Inputs(w)
-    f = Filled(inp)
+    f = Filled(inp, attn_path=path)
     out, sel, nsel = f.decode()
     st = f.status()
     assert st[0] == 0, f"device status {st}"

@@ -25,6 +25,18 @@ RANKR = [synth.TINY, synth.TINY_NEEDLE] + [synth.small(w) for w in
 NVFP4 = [synth.small(synth.NVFP4_128K)]
 
 
+def _paths(ws):
+    """(workload, attention kernel) cases: both kernels where the block size allows the tile
+    pipeline (attn_path 1 forces it, 2 forces the gather kernel), the automatic choice
+    otherwise."""
+    return [(w, p) for w in ws for p in ((1, 2) if w.block_size >= 8 else (0,))]
+
+
+def _ids(case):
+    w, p = case
+    return f"{w.name}-path{p}"
+
+
 def _gpu():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
@@ -40,11 +52,11 @@ def _check_out(w, got, want, where):
         assert err <= 2e-2, f"{where}: max-abs {err:.3e}"
 
 
-def _run_workload(w):
+def _run_workload(w, attn_path=0):
     from tests.gpu_util import Filled, out_to_f64
     import score_then_select_b200 as qs
     inp = synth.Inputs(w)
-    f = Filled(inp)
+    f = Filled(inp, attn_path=attn_path)
     out, sel, nsel = f.decode()
     st = f.status()
     assert st[0] == 0, f"device status {st}"
@@ -65,10 +77,11 @@ def _run_workload(w):
     return inp, f, out_to_f64(out), sel.cpu().numpy(), nsel.cpu().numpy(), scores.cpu().numpy()
 
 
-@pytest.mark.parametrize("w", RANKR, ids=lambda w: w.name)
-def test_rankr_parity(w):
+@pytest.mark.parametrize("case", _paths(RANKR), ids=_ids)
+def test_rankr_parity(case):
     _gpu()
-    inp, f, out, sel, nsel, scores = _run_workload(w)
+    w, path = case
+    inp, f, out, sel, nsel, scores = _run_workload(w, path)
     G = w.group
     for b in range(w.batch):
         L = int(inp.lens[b])
@@ -96,13 +109,14 @@ def test_rankr_parity(w):
             _check_out(w, out[b, g * G:(g + 1) * G], rr["out"], where)
 
 
-@pytest.mark.parametrize("w", NVFP4, ids=lambda w: w.name)
-def test_nvfp4_parity(w):
+@pytest.mark.parametrize("case", _paths(NVFP4), ids=_ids)
+def test_nvfp4_parity(case):
     """NVFP4 path: codes and scales bit-exact, FP4 tensor-core block scores within 1e-4 of
     the largest score, block errors within 1e-5 relative, kept blocks and selection valid
     up to near-ties, attention within the BF16 bound."""
     _gpu()
-    inp, f, out, sel, nsel, scores = _run_workload(w)
+    w, path = case
+    inp, f, out, sel, nsel, scores = _run_workload(w, path)
     gq = query_scale_all(inp)
     berr = f.layer.block_err.cpu().numpy()
     G = w.group
@@ -163,15 +177,16 @@ def test_dense_rows_reduce_to_dense_attention():
             _check_out(w, out[b, g * w.group:(g + 1) * w.group], dense, f"dense row {b},{g}")
 
 
-def test_bad_page_table_entry_is_reported_not_faulted():
+@pytest.mark.parametrize("path", [1, 2])
+def test_bad_page_table_entry_is_reported_not_faulted(path):
     """A page id outside the cache is skipped by every kernel and reported as a bounds
-    error through the workspace status word."""
+    error through the workspace status word (both attention kernels)."""
     _gpu()
     import score_then_select_b200 as qs
     from tests.gpu_util import Filled
     w = synth.small(synth.BLOCK128K)
     inp = synth.Inputs(w)
-    f = Filled(inp)
+    f = Filled(inp, attn_path=path)
     assert f.status()[0] == 0
     f.layer.page_table[0, 3] = inp.num_pages + 5        # host-side corruption
     f.decode()
