@@ -56,6 +56,9 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (small cases for profiling only)")
+    ap.add_argument("--attn-path", type=int, default=0, choices=[0, 1, 2],
+                    help="attention kernel: 0 chosen per shape, 1 tile pipeline, 2 gather "
+                         "(for profiling small cases)")
     return ap.parse_args(argv)
 
 
@@ -361,7 +364,7 @@ def run_ours(args):
         w0 = w0.replace(batch=args.batch)
     w = rank_workload(w0, rank)
     inp = synth.Inputs(w)
-    f = Filled(inp)
+    f = Filled(inp, attn_path=args.attn_path)
     lay, cfg, cache = f.layer, f.cfg, f.cache
     B = w.batch
     lens = inp.lens

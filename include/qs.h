@@ -208,8 +208,8 @@ qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
    kernels only their inputs and outputs, or a decode loop that may not call cudaMalloc
    because the allocation would synchronise the device. The pages describe no such call;
    it exists for these callers only.
-   Computes exactly what qs_sparse_attn computes, with the same kernel; its split partials
-   and per-row counters live in one static device array of QS_ATTN_STATIC_SCRATCH_BYTES
+   Computes exactly what qs_sparse_attn computes, with the same kernels; its partials and
+   counters live in one static device array of QS_ATTN_STATIC_SCRATCH_BYTES
    inside the library (each GPU that loads the library holds it until the process exits),
    so the call allocates nothing and takes no workspace. The first call on a device looks
    up that array's device address (once per device, with the device current); make that
@@ -218,10 +218,11 @@ qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
    on the GPU (different streams, or different threads without ordering) race and must
    not be issued. Device-side bounds checks still skip invalid accesses, but their status
    word is not reported by this call.
-   Returns QS_ERR_UNSUPPORTED if batch * Hq * splits * (head_dim + 2) * 4 bytes of partials
-   plus batch * Hkv * 4 bytes of counters exceed QS_ATTN_STATIC_SCRATCH_BYTES (the split
-   count is the one qs_sparse_attn plans for the shape), and QS_ERR_CUDA if the address
-   lookup or a launch fails; other arguments as for qs_sparse_attn. */
+   Returns QS_ERR_UNSUPPORTED if batch * Hq * parts * (head_dim + 2) * 4 bytes of partials
+   plus batch * Hkv * 4 bytes of counters exceed QS_ATTN_STATIC_SCRATCH_BYTES (parts per
+   query head is what qs_sparse_attn plans for the shape: chunks of the tile pipeline or
+   splits of the gather kernel), and QS_ERR_CUDA if the address lookup or a launch fails;
+   other arguments as for qs_sparse_attn. */
 #define QS_ATTN_STATIC_SCRATCH_BYTES (4u << 20)
 qs_status qs_sparse_attn_noalloc(const qs_config *cfg, const qs_cache *cache, const void *q,
                                  const int32_t *sel, const int32_t *n_sel, int32_t batch,
