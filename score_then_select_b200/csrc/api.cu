@@ -231,7 +231,8 @@ static qs_status do_append(const Plan& p, const qs_cache* c, const void* k_new, 
   return cuda_status(launch_block_err(p, e, s));
 }
 
-static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws, cudaStream_t s) {
+static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws, cudaStream_t s,
+                         bool pdl) {
   if (p.r > 0) {
     PrepParams a{static_cast<const uint16_t*>(q), P, ws_at<float>(ws, p.ws.qt),
                  p.batch, p.Hkv, p.G, p.d, p.r};
@@ -240,7 +241,7 @@ static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws,
   QPackParams a{static_cast<const uint16_t*>(q), ws_at<uint8_t>(ws, p.ws.qtile),
                 ws_at<float>(ws, p.ws.qgscale), p.batch * p.Hq * p.d, p.batch * p.Hkv, p.Hkv,
                 p.G};
-  return cuda_status(launch_qpack(p, a, s));
+  return cuda_status(launch_qpack(p, a, s, pdl));
 }
 
 static qs_status do_score(const Plan& p, const qs_cache* c, float* scores, void* ws, cudaStream_t s,
@@ -387,7 +388,7 @@ qs_status qs_score(const qs_config* cfg, const qs_cache* cache, const void* q, c
   if (!q || !aligned(q, 4) || !block_scores || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
   if (p.r == 0 && !aligned(q, 16)) return QS_ERR_INVALID_ARG;
-  if ((st = do_prep(p, q, P, ws, stream)) != QS_OK) return st;
+  if ((st = do_prep(p, q, P, ws, stream, false)) != QS_OK) return st;
   return do_score(p, cache, block_scores, ws, stream, true);
 }
 
@@ -430,7 +431,7 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   float* scores = ws_at<float>(ws, p.ws.scores);
   // append (+ fused scoring prep on the rank-r path)
   if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, P, q, ws, stream)) != QS_OK) return st;
-  if (p.r == 0 && (st = do_prep(p, q, P, ws, stream)) != QS_OK) return st;
+  if (p.r == 0 && (st = do_prep(p, q, P, ws, stream, true)) != QS_OK) return st;
   if ((st = do_score(p, cache, scores, ws, stream, true)) != QS_OK) return st;
   if ((st = do_select(p, cache, scores, sel, nsel, ws, stream, true)) != QS_OK) return st;
   return do_attend(p, cache, q, sel, nsel, out, ws, stream, true);

@@ -351,6 +351,7 @@ __global__ void __launch_bounds__(128) append_nvfp4_kernel(const AppendParams a)
   constexpr int TT = 64, D = 128, GR = D / 16;
   __shared__ int s_page[TT], s_slot[TT];
   __shared__ float s_mu[D];
+  pdl_trigger();   // the block-error kernel may launch now; it waits for this grid
   const int row = blockIdx.y;
   const int b = row / a.Hkv, g = row % a.Hkv;
   int n_b = a.n_new ? a.n_new[b] : 1;
@@ -422,6 +423,7 @@ __global__ void __launch_bounds__(256) block_err_kernel(const BlockErrParams a) 
   __shared__ float s_mu[D];
   __shared__ float s_red[8];
   pdl_wait();      // the cache and seq_lens come from the append kernel before
+  pdl_trigger();
   const int row = blockIdx.y;
   const int b = row / a.Hkv, g = row % a.Hkv;
   const int n_b = a.n_new ? a.n_new[b] : 1;
@@ -475,6 +477,7 @@ __global__ void __launch_bounds__(256) block_err_kernel(const BlockErrParams a) 
 // ============================================================ scoring prep
 __global__ void __launch_bounds__(128) prep_rankr_kernel(const PrepParams a) {
   __shared__ float qbar[256];
+  pdl_trigger();   // the scan may launch now; it waits for this grid before reading q~
   const int row = blockIdx.x;
   const int b = row / a.Hkv, g = row % a.Hkv;
   row_prep(a.q, a.P + size_t(g) * a.d * a.r, a.qt + size_t(row) * a.r, qbar, b, g, a.Hkv, a.G,
@@ -489,6 +492,7 @@ __global__ void __launch_bounds__(128) prep_rankr_kernel(const PrepParams a) {
 __global__ void __launch_bounds__(256) qpack_kernel(const QPackParams a) {
   __shared__ float s_red[8];
   __shared__ float s_g;
+  pdl_trigger();   // the scan may launch now; it waits for this grid before reading the tiles
   const int tid = threadIdx.x, row = blockIdx.x;
   float m = 0.0f;
   const uint4* q4 = reinterpret_cast<const uint4*>(a.q);
@@ -534,6 +538,9 @@ __global__ void __launch_bounds__(256) qpack_kernel(const QPackParams a) {
     *reinterpret_cast<uint2*>(tile + qtile_code_off(n, gr)) = make_uint2(packed[0], packed[1]);
     tile[qtile_scale_off(n, gr)] = uint8_t(sc);
   }
+  // Packing reads only q, so it runs alongside the kernel before; waiting for that kernel
+  // before exiting keeps "this grid done" implying "every earlier grid done" for the scan.
+  pdl_wait();
 }
 
 // ============================================================ launchers
@@ -594,9 +601,8 @@ cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s) {
-  qpack_kernel<<<a.rows, 256, 0, s>>>(a);
-  return cudaGetLastError();
+cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s, bool pdl) {
+  return launch_k(qpack_kernel, dim3(a.rows), dim3(256), 0, s, pdl, a);
 }
 
 }  // namespace qs

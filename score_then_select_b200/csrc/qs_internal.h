@@ -207,7 +207,7 @@ inline cudaError_t launch_k(void (*kern)(P...), dim3 grid, dim3 block, size_t sm
 cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s);
 cudaError_t launch_block_err(const Plan& p, const BlockErrParams& a, cudaStream_t s);
 cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s);
-cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s);
+cudaError_t launch_qpack(const Plan& p, const QPackParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_attn_gather(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl);
