@@ -438,7 +438,8 @@ def run_ours(args):
     # ---------------- end to end: host buffers, copies inside the timed region. Through the
     # public API twice: eager qs_decode calls, and the same step captured once into a CUDA
     # graph (score_then_select_b200.graph.CapturedDecode) and replayed; each step copies q,
-    # k_new, v_new from pinned host memory, decodes, copies the output back and syncs.
+    # k_new, v_new from pinned host memory (the graph: one packed copy), decodes, copies the
+    # output back and syncs.
     from score_then_select_b200.graph import CapturedDecode
     q_h = f.q.cpu().pin_memory()
     k_h = f.k_last.cpu().pin_memory()
