@@ -200,7 +200,7 @@ qs_status qs_decode(const qs_config *cfg, const qs_cache *cache, const void *q,
    since the last call (QS_OK if none) and clear it. `detail` (HOST pointer, may be NULL)
    receives {kernel id, index} of that error. Returns QS_ERR_CUDA if the synchronisation
    or the read-back fails. Kernel ids: 1 append, 2 block error, 3 scoring prep, 4 score,
-   5 select, 6 attention (with its log-sum-exp combine). */
+   5 select, 6 attention (with its log-sum-exp combine), 7 the wait self-test. */
 qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
 
 /* Sparse attention without a workspace, for callers that cannot allocate device memory:
@@ -233,6 +233,15 @@ const char *qs_status_string(qs_status s);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int32_t qs_version(void);
+
+/* Diagnostic: launch one kernel whose bounded wait (the same mbarrier wait the library's
+   kernels use) waits for an arrival that never comes; it must give up after a short limit
+   and record QS_ERR_DEVICE_TIMEOUT in the workspace status word (kernel id 7), which
+   qs_device_status then returns. The pages describe no such call: it lets a caller check on
+   a given GPU that a lost arrival ends in a reported error, not a hang, and that the
+   context stays usable. ws: a workspace as for the other calls (only its status word is
+   used). */
+qs_status qs_selftest_wait_timeout(void *ws, qs_stream_t stream);
 
 #ifdef __cplusplus
 }

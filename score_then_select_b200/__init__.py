@@ -7,10 +7,10 @@ no CPU fallback: importing the binding's entry points requires the built library
 from .binding import (QsError, LIB_PATH, EXPORTS, lib, make_config, make_cache, qs_version,
                       qs_workspace_size, qs_workspace_init, qs_append_kv, qs_score,
                       qs_select_topk, qs_sparse_attn, qs_decode, qs_device_status,
-                      qs_sparse_attn_noalloc, qs_attention_launches,
+                      qs_sparse_attn_noalloc, qs_attention_launches, qs_selftest_wait_timeout,
                       status_string)
 
 __all__ = ["QsError", "LIB_PATH", "EXPORTS", "lib", "make_config", "make_cache", "qs_version",
            "qs_workspace_size", "qs_workspace_init", "qs_append_kv", "qs_score",
            "qs_select_topk", "qs_sparse_attn", "qs_decode", "qs_device_status", "status_string",
-           "qs_sparse_attn_noalloc", "qs_attention_launches"]
+           "qs_sparse_attn_noalloc", "qs_attention_launches", "qs_selftest_wait_timeout"]

@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
             "qs_workspace_size": ([cfgp, i32, i32, ctypes.POINTER(sz)], i32),
             "qs_workspace_init": ([vp, sz, vp], i32),
             "qs_attention_launches": ([cfgp, i32, i32, ctypes.POINTER(i32)], i32),
+            "qs_selftest_wait_timeout": ([vp, vp], i32),
             "qs_append_kv": ([cfgp, cachep, vp, vp, vp, i32, vp, i32, vp, vp], i32),
             "qs_score": ([cfgp, cachep, vp, vp, i32, vp, vp, vp], i32),
             "qs_select_topk": ([cfgp, cachep, vp, i32, vp, vp, vp, vp], i32),
@@ -78,7 +79,8 @@ def lib() -> ctypes.CDLL:
 
 EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_init",
            "qs_append_kv", "qs_score", "qs_select_topk", "qs_sparse_attn", "qs_decode",
-           "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches")
+           "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches",
+           "qs_selftest_wait_timeout")
 
 
 def status_string(s: int) -> str:
@@ -155,6 +157,10 @@ def qs_attention_launches(cfg: qs_config, batch: int, max_context: int) -> int:
     _check(lib().qs_attention_launches(ctypes.byref(cfg), batch, max_context, ctypes.byref(n)),
            "qs_attention_launches")
     return n.value
+
+
+def qs_selftest_wait_timeout(ws, stream=None):
+    _check(lib().qs_selftest_wait_timeout(_ptr(ws), _stream(stream)), "qs_selftest_wait_timeout")
 
 
 def qs_workspace_init(ws, nbytes: int, stream=None):

@@ -17,7 +17,8 @@ enum KernelId : uint32_t {
   KID_PREP = 3,
   KID_SCORE = 4,
   KID_SELECT = 5,
-  KID_ATTN = 6
+  KID_ATTN = 6,
+  KID_SELFTEST = 7
 };
 
 constexpr int kPage = 128;          // tokens per page (the only page size built)
