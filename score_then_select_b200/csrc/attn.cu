@@ -29,21 +29,18 @@
 //   * consumer warps (warps 0-3): each owns 16 tokens of every tile and keeps its own
 //     online-softmax state (base 2, scale * log2 e folded into the logits). At the end of
 //     a chunk the four states are merged in a fixed order into the chunk's partial
-//     (max, sum, o); the chunk that completes its row's count merges the row's partials by
-//     log-sum-exp into the output.
+//     (max, sum, o).
+// attn_combine_kernel, launched behind this grid, merges each (row, query head)'s chunk
+// partials by log-sum-exp into the output.
 //
-// Tensor-core mapping (mma.m16n8k16, FP32 accumulate), transposed so that the group's
-// <= 8 query heads fill the N = 8 side:
-//   S^T[16 tok x 8 heads]  = K[16 tok x d] . Q^T[d x 8 heads]      (A = K via ldmatrix)
-//   O^T[d x 8 heads]      += V^T[d x 16 tok] . P^T[16 tok x 8 heads] (A = V via ldmatrix.trans,
-//                                                                    B = P via movmatrix)
+// Tensor-core mapping and online softmax: attn_warp_tile (attn_core.cuh).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <cstring>
 #include <mutex>
 
-#include "qs_device.cuh"
+#include "attn_core.cuh"
 
 namespace qs {
 
@@ -384,71 +381,11 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     }
     const uint32_t kst = smem_u32(st), vst = smem_u32(st + SM::kTileBytes);
 
-    // S^T = K Q^T for this warp's 16 tokens
-    float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(a0, a1, a2, a3, kst + swz(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
-      mma_bf16(c, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-    }
     const int tl = warp * 16 + (lane >> 2);       // tokens tl and tl + 8 (same 32-slot word)
     const uint32_t vm = warp < 2 ? lo : hi;
-    const bool v0 = (vm >> (tl & 31)) & 1u, v1 = (vm >> ((tl + 8) & 31)) & 1u;
-    float x0 = v0 ? c[0] * a.scale_log2 : -INFINITY;
-    float x1 = v0 ? c[1] * a.scale_log2 : -INFINITY;
-    float x2 = v1 ? c[2] * a.scale_log2 : -INFINITY;
-    float x3 = v1 ? c[3] * a.scale_log2 : -INFINITY;
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int o2 = 4; o2 < 32; o2 <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o2));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
-    const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
-    const float al0 = ex2(m0 - base0), al1 = ex2(m1 - base1);
-    m0 = mn0;
-    m1 = mn1;
-    const float p0 = ex2(x0 - base0), p1 = ex2(x1 - base1);
-    const float p2 = ex2(x2 - base0), p3 = ex2(x3 - base1);
-    l0 = l0 * al0 + p0 + p2;
-    l1 = l1 * al1 + p1 + p3;
-#pragma unroll
-    for (int m = 0; m < KS; ++m) {
-      o[m][0] *= al0;
-      o[m][1] *= al1;
-      o[m][2] *= al0;
-      o[m][3] *= al1;
-    }
-    // P^T as the B operand: transpose the two 8x8 (token x head) quadrants
-    uint32_t pb0, pb1;
-    if constexpr (AGG_F16) {
-      pb0 = movmatrix_t(pack_f16x2(p0, p1));
-      pb1 = movmatrix_t(pack_f16x2(p2, p3));
-    } else {
-      pb0 = movmatrix_t(pack_bf16x2(p0, p1));
-      pb1 = movmatrix_t(pack_bf16x2(p2, p3));
-    }
-    // O^T += V^T P^T over the head dimension
-#pragma unroll
-    for (int m = 0; m < KS; ++m) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4_t(a0, a1, a2, a3,
-                vst + swz(warp * 16 + (lane & 7) + ((lane >> 4) << 3), m * 2 + ((lane >> 3) & 1)));
-      if constexpr (AGG_F16) {
-        if constexpr (!V_F16) {
-          a0 = bf16x2_to_f16x2(a0);
-          a1 = bf16x2_to_f16x2(a1);
-          a2 = bf16x2_to_f16x2(a2);
-          a3 = bf16x2_to_f16x2(a3);
-        }
-        mma_f16(o[m], a0, a1, a2, a3, pb0, pb1);
-      } else {
-        mma_bf16(o[m], a0, a1, a2, a3, pb0, pb1);
-      }
-    }
+    attn_warp_tile<D, V_F16, AGG_F16>(kst, vst, qb, (vm >> (tl & 31)) & 1u,
+                                      (vm >> ((tl + 8) & 31)) & 1u, a.scale_log2, m0, m1, l0, l1,
+                                      o, warp, lane, [](int r, int c) { return swz(r, c); });
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);        // this warp is done with the stage
     if (!(info & kMetaLast)) continue;

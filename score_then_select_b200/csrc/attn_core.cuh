@@ -1,0 +1,94 @@
+// attn_core.cuh - one warp's share of one 64-token tile of sparse attention: 16 tokens'
+// tensor-core logits, online softmax and value aggregation. Shared by the two attention
+// kernels (attn.cu, attn_gather.cu), which differ in how tiles reach shared memory.
+//
+// Tensor-core mapping (mma.m16n8k16, FP32 accumulate), transposed so that the group's
+// <= 8 query heads fill the N = 8 side:
+//   S^T[16 tok x 8 heads]  = K[16 tok x d] . Q^T[d x 8 heads]      (A = K via ldmatrix)
+//   O^T[d x 8 heads]      += V^T[d x 16 tok] . P^T[16 tok x 8 heads] (A = V via ldmatrix.trans,
+//                                                                    B = P via movmatrix)
+// Lane layout: this lane's heads are h0 = 2 * (lane % 4) and h0 + 1, its tokens
+// lane / 4 and lane / 4 + 8 of the warp's 16; m (running max, base 2) is replicated over
+// the lanes with equal lane % 4, l is this lane's partial sum over its own tokens, and
+// o[m] holds O^T entries (d0, h0), (d0, h0 + 1), (d0 + 8, h0), (d0 + 8, h0 + 1) with
+// d0 = 16 m + lane / 4.
+#pragma once
+
+#include "qs_device.cuh"
+
+namespace qs {
+
+// `swz(r, c)`: byte offset of 16-byte chunk c of token row r inside a K or V tile.
+// qb: the query fragments (B operand of S^T), valid0 / valid1: whether this lane's two
+// tokens are selected (masked ones get probability 0), scale_log2: softmax scale * log2 e.
+template <int D, bool V_F16, bool AGG_F16, typename Swz>
+QS_DEV void attn_warp_tile(uint32_t kst, uint32_t vst, const uint32_t (&qb)[D / 16][2],
+                           bool valid0, bool valid1, float scale_log2, float& m0, float& m1,
+                           float& l0, float& l1, float (&o)[D / 16][4], int warp, int lane,
+                           Swz swz) {
+  constexpr int KS = D / 16;
+  // S^T = K Q^T for this warp's 16 tokens
+  float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4(a0, a1, a2, a3, kst + swz(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
+    mma_bf16(c, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+  }
+  const float x0 = valid0 ? c[0] * scale_log2 : -INFINITY;
+  const float x1 = valid0 ? c[1] * scale_log2 : -INFINITY;
+  const float x2 = valid1 ? c[2] * scale_log2 : -INFINITY;
+  const float x3 = valid1 ? c[3] * scale_log2 : -INFINITY;
+  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+  for (int o2 = 4; o2 < 32; o2 <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o2));
+  }
+  const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+  const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
+  const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
+  const float al0 = ex2(m0 - base0), al1 = ex2(m1 - base1);
+  m0 = mn0;
+  m1 = mn1;
+  const float p0 = ex2(x0 - base0), p1 = ex2(x1 - base1);
+  const float p2 = ex2(x2 - base0), p3 = ex2(x3 - base1);
+  l0 = l0 * al0 + p0 + p2;
+  l1 = l1 * al1 + p1 + p3;
+#pragma unroll
+  for (int m = 0; m < KS; ++m) {
+    o[m][0] *= al0;
+    o[m][1] *= al1;
+    o[m][2] *= al0;
+    o[m][3] *= al1;
+  }
+  // P^T as the B operand: transpose the two 8x8 (token x head) quadrants
+  uint32_t pb0, pb1;
+  if constexpr (AGG_F16) {
+    pb0 = movmatrix_t(pack_f16x2(p0, p1));
+    pb1 = movmatrix_t(pack_f16x2(p2, p3));
+  } else {
+    pb0 = movmatrix_t(pack_bf16x2(p0, p1));
+    pb1 = movmatrix_t(pack_bf16x2(p2, p3));
+  }
+  // O^T += V^T P^T over the head dimension
+#pragma unroll
+  for (int m = 0; m < KS; ++m) {
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4_t(a0, a1, a2, a3,
+              vst + swz(warp * 16 + (lane & 7) + ((lane >> 4) << 3), m * 2 + ((lane >> 3) & 1)));
+    if constexpr (AGG_F16) {
+      if constexpr (!V_F16) {
+        a0 = bf16x2_to_f16x2(a0);
+        a1 = bf16x2_to_f16x2(a1);
+        a2 = bf16x2_to_f16x2(a2);
+        a3 = bf16x2_to_f16x2(a3);
+      }
+      mma_f16(o[m], a0, a1, a2, a3, pb0, pb1);
+    } else {
+      mma_bf16(o[m], a0, a1, a2, a3, pb0, pb1);
+    }
+  }
+}
+
+}  // namespace qs
