@@ -239,6 +239,46 @@ def lse_combine(ms, ls, os_) -> np.ndarray:
 
 
 # ============================================================================================
+# Full-KV attention and gather-then-attend  [JSSA, Figure 2 (b); Figure 6 (a)]
+# The pages compare the sparse attention stage with attention over the whole cache
+# (full-KV) and with a variant that first copies the selected tokens into a contiguous
+# buffer and then runs dense attention over it (gather-then-attend).
+# ============================================================================================
+
+
+def dense_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, L: int,
+                    scale: float) -> np.ndarray:
+    """Full-KV attention: o_h = sum_{t < L} softmax_t(scale * q_h . k_t) v_t (float64).
+
+    q: [G][d]; K/V: [>= L][d] decoded. L = 0 gives zeros (no token to attend to).
+    """
+    if L == 0:
+        return np.zeros((q.shape[0], V.shape[1]))
+    logits = scale * (q @ K[:L].T)
+    w = np.exp(logits - logits.max(axis=1, keepdims=True))
+    return (w @ V[:L]) / w.sum(axis=1, keepdims=True)
+
+
+def gather_blocks(sel: np.ndarray, S: int, L: int):
+    """Gathered layout of one row: the source token of every gathered slot, and the count.
+
+    Gathered slot i * S + u holds token sel[i] * S + u (u < S), for the selected blocks in
+    their ascending order; a slot whose token is at or past L holds nothing (-1). Only the
+    row's last block can be cut by L and it is the last selected block when selected, so
+    the filled slots form a prefix. Returns (src [len(sel) * S] int64, n_valid).
+    """
+    sel = np.asarray(sel, dtype=np.int64)
+    src = np.full(len(sel) * S, -1, dtype=np.int64)
+    for i, blk in enumerate(sel):
+        for u in range(S):
+            t = blk * S + u
+            if t < L:
+                src[i * S + u] = t
+    n_valid = int((src >= 0).sum())
+    return src, n_valid
+
+
+# ============================================================================================
 # NVFP4 path  [JQS, Full text]
 # ============================================================================================
 

@@ -209,3 +209,88 @@ def test_lse_combine_split_invariance(nsplit):
     st = [M.attention_partial(q, K, V, p, 0.3) for p in parts]
     got = M.lse_combine([s[0] for s in st], [s[1] for s in st], [s[2] for s in st])
     assert np.allclose(got, M.sparse_attention(q, K, V, toks, 0.3), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- full-KV and gather-then-attend
+
+def test_dense_attention_matches_loop_softmax():
+    rng = np.random.default_rng(21)
+    G, d, L = 4, 16, 37
+    q = rng.standard_normal((G, d)) * 2
+    K = rng.standard_normal((L + 5, d))            # rows at or past L are not attended
+    V = rng.standard_normal((L + 5, d))
+    got = M.dense_attention(q, K, V, L, 0.3)
+    assert np.allclose(got, _dense_attention_bruteforce(q, K[:L], V[:L], 0.3),
+                       rtol=1e-12, atol=1e-12)
+
+
+def test_dense_attention_closed_forms():
+    rng = np.random.default_rng(22)
+    V = rng.standard_normal((9, 8))
+    q = rng.standard_normal((3, 8))
+    # equal keys: uniform weights, the mean of the values
+    K = np.tile(rng.standard_normal(8), (9, 1))
+    assert np.allclose(M.dense_attention(q, K, V, 9, 1.0), np.broadcast_to(V.mean(0), (3, 8)),
+                       rtol=1e-13, atol=1e-13)
+    # scale 0: the mean of the values whatever the keys
+    K = rng.standard_normal((9, 8))
+    assert np.allclose(M.dense_attention(q, K, V, 9, 0.0), np.broadcast_to(V.mean(0), (3, 8)),
+                       rtol=1e-13, atol=1e-13)
+    # one token: its value row; no token: zeros
+    assert np.array_equal(M.dense_attention(q, K, V, 1, 1.0), np.broadcast_to(V[0], (3, 8)))
+    assert np.array_equal(M.dense_attention(q, K, V, 0, 1.0), np.zeros((3, 8)))
+    # one logit far above the rest: that token's value (weight of the others < e^-700)
+    K2 = np.zeros((9, 8))
+    K2[4, 0] = 1.0
+    q2 = np.zeros((1, 8))
+    q2[0, 0] = 700.0
+    assert np.allclose(M.dense_attention(q2, K2, V, 9, 1.0)[0], V[4], rtol=0, atol=1e-290)
+
+
+def test_gather_blocks_hand_example():
+    # S = 4, L = 14 (blocks 0..3, block 3 holds tokens 12, 13 only); selected 1, 3
+    src, n = M.gather_blocks(np.array([1, 3]), 4, 14)
+    assert src.tolist() == [4, 5, 6, 7, 12, 13, -1, -1]
+    assert n == 6
+    # the cut block not selected: every slot filled
+    src, n = M.gather_blocks(np.array([0, 2]), 4, 14)
+    assert src.tolist() == [0, 1, 2, 3, 8, 9, 10, 11] and n == 8
+    # token level (S = 1): the selection itself
+    src, n = M.gather_blocks(np.array([3, 9, 10]), 1, 11)
+    assert src.tolist() == [3, 9, 10] and n == 3
+    # nothing selected
+    src, n = M.gather_blocks(np.zeros(0, dtype=np.int64), 8, 5)
+    assert src.size == 0 and n == 0
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_gather_prefix_and_count(seed):
+    rng = np.random.default_rng(100 + seed)
+    S = int(rng.choice([1, 2, 8, 16]))
+    L = int(rng.integers(1, 200))
+    nb = -(-L // S)
+    k = int(rng.integers(1, nb + 1))
+    sel = np.sort(rng.choice(nb, k, replace=False))
+    src, n = M.gather_blocks(sel, S, L)
+    # filled slots are a prefix, their tokens are exactly the selected valid tokens
+    assert np.all(src[:n] >= 0) and np.all(src[n:] == -1)
+    assert src[:n].tolist() == M.block_tokens(sel, S, L).tolist()
+    # count: every selected block is full except a selected last block cut by L
+    assert n == sum(min(S, L - b * S) for b in sel)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_gather_then_dense_equals_sparse_attention(seed):
+    # attending densely over the gathered prefix is the sparse attention over the selection
+    rng = np.random.default_rng(200 + seed)
+    G, d, S, L = 3, 16, int(rng.choice([1, 4, 16])), int(rng.integers(20, 300))
+    nb = -(-L // S)
+    sel = np.sort(rng.choice(nb, min(nb, int(rng.integers(1, 12))), replace=False))
+    q = rng.standard_normal((G, d))
+    K, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    src, n = M.gather_blocks(sel, S, L)
+    Kg = np.where(src[:, None] >= 0, K[np.maximum(src, 0)], np.nan)
+    Vg = np.where(src[:, None] >= 0, V[np.maximum(src, 0)], np.nan)
+    got = M.dense_attention(q, Kg, Vg, n, 0.2)
+    want = _dense_attention_bruteforce(q, K[M.block_tokens(sel, S, L)], V[M.block_tokens(sel, S, L)], 0.2)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
