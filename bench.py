@@ -56,6 +56,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (small cases for profiling only)")
+    ap.add_argument("--no-compare", action="store_true",
+                    help="skip the full-KV and gather-then-attend comparison")
     ap.add_argument("--attn-path", type=int, default=0, choices=[0, 1, 2],
                     help="attention kernel: 0 chosen per shape, 1 tile pipeline, 2 gather "
                          "(for profiling small cases)")
@@ -343,6 +345,63 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ our arm
 
+def run_compare(args, w, f, lens, sel, nsel, out, stream):
+    """Attention-stage comparison: gather-free sparse attention, gather-then-attend and
+    full-KV attention, each timed with CUDA events on `stream` (mean of n launches after 3
+    untimed rounds), with the algorithmic HBM bytes of each."""
+    import torch
+    import score_then_select_b200 as qs
+    from score_then_select_b200.layer import GatheredKV, workspace
+    lay, cfg, cache, B = f.layer, f.cfg, f.cache, w.batch
+    ws_d = workspace(qs.qs_dense_workspace_size(cfg, B, lay.max_context))
+    gk = GatheredKV.allocate(lay)
+    ws_g = workspace(qs.qs_dense_workspace_size(cfg, B, gk.max_context))
+    gcache = gk.cache()
+    out_c = torch.empty_like(out)
+    n = min(args.steps, 20)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n + 3)]
+    for ev in evs:
+        ev[0].record(stream)
+        qs.qs_sparse_attn(cfg, cache, f.q, sel, nsel, B, out_c, lay.ws, stream)
+        ev[1].record(stream)
+        qs.qs_gather_kv(cfg, cache, sel, nsel, B, gk.k, gk.v, gk.row_lens, lay.ws, stream)
+        ev[2].record(stream)
+        qs.qs_dense_attn(cfg, gcache, f.q, gk.row_lens, B, out_c, ws_g, stream)
+        ev[3].record(stream)
+        qs.qs_dense_attn(cfg, cache, f.q, None, B, out_c, ws_d, stream)
+        ev[4].record(stream)
+    torch.cuda.synchronize()
+    for ws in (lay.ws, ws_d, ws_g):
+        st = qs.qs_device_status(ws)
+        if st[0] != 0:
+            raise RuntimeError(f"device status in the comparison {st}")
+    acc = np.zeros(4)
+    for ev in evs[3:]:
+        acc += [ev[j].elapsed_time(ev[j + 1]) for j in range(4)]
+    attend, gather, attend_g, full = (acc / n * 1e3).tolist()
+    by = step_bytes(w, lens, sel.cpu().numpy(), nsel.cpu().numpy())
+    qo = by["q"] + by["out"]
+    full_bytes = int(np.sum(lens.astype(np.int64))) * w.n_kv_heads * w.head_dim * 2 * 2 + qo
+    peak, _ = peaks()
+    gta = gather + attend_g
+
+    def hbm(nbytes, us):
+        return {"bytes": int(nbytes), "GB/s": nbytes / (us * 1e-6) / 1e9,
+                "frac": nbytes / (us * 1e-6) / 1e9 / peak}
+
+    return {"attend_us": attend, "gather_us": gather, "attend_gathered_us": attend_g,
+            "gather_then_attend_us": gta, "full_kv_us": full,
+            "speedup_vs_full_kv": full / attend,
+            "gather_then_attend_speedup_vs_full_kv": full / gta,
+            "gather_free_speedup_vs_gather_then_attend": gta / attend,
+            "hbm": {"attend": hbm(by["kv"] + qo, attend), "gather": hbm(2 * by["kv"], gather),
+                    "attend_gathered": hbm(by["kv"] + qo, attend_g),
+                    "full_kv": hbm(full_bytes, full)},
+            "launches": {"attend": qs.qs_attention_launches(cfg, B, lay.max_context),
+                         "gather_then_attend": 3, "full_kv": 2},
+            "timed_launches": n}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -435,6 +494,15 @@ def run_ours(args):
         acc += [ev[j].elapsed_time(ev[j + 1]) for j in range(4)]
     stage_us = dict(zip(["append", "score", "select", "attend"], (acc / n_stage * 1e3).tolist()))
 
+    # ---------------- comparison ("Joint Subspace Sparse Attention ...", Figure 2 (b) and
+    # Figure 6 (a)): the sparse attention stage (gather-free, reading the selected blocks in
+    # place) against full-KV attention over every cached token and against gather-then-attend
+    # (qs_gather_kv into a compact buffer, then the same dense kernel over it), on the
+    # selection of the steps above; CUDA events on the launching stream, caches > L2.
+    compare = None
+    if not args.no_compare:
+        compare = run_compare(args, w, f, lens, sel, nsel, out, stream)
+
     # ---------------- end to end: host buffers, copies inside the timed region. Through the
     # public API twice: eager qs_decode calls, and the same step captured once into a CUDA
     # graph (score_then_select_b200.graph.CapturedDecode) and replayed; each step copies q,
@@ -512,6 +580,8 @@ def run_ours(args):
                     "ms_per_step": e2e_ms, "path": "CapturedDecode (CUDA graph of the step)",
                     "eager_ms_per_step": eager_ms},
             "gpu_launches": args.steps * launches_per_step}
+    if compare is not None:
+        line["comparison"] = compare
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_rows)
     if rank == 0:

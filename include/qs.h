@@ -196,11 +196,54 @@ qs_status qs_decode(const qs_config *cfg, const qs_cache *cache, const void *q,
                     void *out, int32_t *sel_out, int32_t *n_sel_out, void *ws,
                     qs_stream_t stream);
 
+/* ---- Comparison kernels: full-KV attention and gather-then-attend -----------------------
+   "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 2 (b) and
+   Figure 6 (a), compare the sparse attention stage with attention over the whole cache
+   (full-KV) and with a two-step variant that first copies the selected tokens into a
+   contiguous buffer and then runs ordinary attention over it (gather-then-attend). These
+   calls rebuild those comparisons on the same caches; they are not part of qs_decode. */
+
+/* Workspace bytes that qs_dense_attn needs for caches of up to max_context tokens per
+   sequence (host only). Same statuses as qs_workspace_size; max_context <= 131072. */
+qs_status qs_dense_workspace_size(const qs_config *cfg, int32_t batch, int32_t max_context,
+                                  size_t *bytes /* host */);
+
+/* Full-KV decode attention: for every query head h of row (b, g),
+     o_h = sum_{t < len} softmax_t(scale * q_h.k_t) v_t,
+   len = row_lens[b * Hkv + g] if row_lens is not NULL, else seq_lens[b]; a row of length 0
+   gives zeros. Heads, types, softmax scale and output type come from cfg (its block size,
+   budget, forced blocks and attn_path are not used); the cache's proxy fields are not
+   read. Logits are float32 sums of BF16 products, P.V operands v_agg_dtype, float32
+   accumulation; the row is split over the tile-pipeline attention kernel and merged by
+   the log-sum-exp combine (2 launches). Every len must be <= cache->max_context (a row
+   that needs more than ceil(max_context / 128) pages records QS_ERR_DEVICE_BOUNDS). ws: qs_dense_workspace_size(cfg, batch,
+   cache->max_context) bytes, initialised by qs_workspace_init. q is 16-byte aligned. */
+qs_status qs_dense_attn(const qs_config *cfg, const qs_cache *cache, const void *q,
+                        const int32_t *row_lens, int32_t batch, void *out, void *ws,
+                        qs_stream_t stream);
+
+/* Gather the selected blocks of every row into a compact paged buffer (one launch).
+   With P = ceil(budget * block_size / 128) pages per sequence, k_dst and v_dst are
+   [batch * P][Hkv][128][head_dim] (K BF16, V as v_dtype; 16-byte aligned). Gathered slot
+   i * S + u of row (b, g) receives token sel[i] * S + u of that row, for i < n_sel; it is
+   stored at page b * P + slot / 128, row slot % 128. Only a selected last block can be cut
+   by seq_len, so the valid tokens form a prefix: row_lens[b * Hkv + g] (device int32
+   [batch * Hkv]) receives its length, and slots after it are not written.
+   qs_dense_attn over a qs_cache whose k / v are these buffers, whose page_table maps
+   page i of sequence b to b * P + i and whose max_context is P * 128, with these
+   row_lens, attends over exactly the selected tokens. A selection entry outside
+   [0, ceil(seq_len / S)) or an unmapped page records QS_ERR_DEVICE_BOUNDS (kernel id 8)
+   and skips the copy. */
+qs_status qs_gather_kv(const qs_config *cfg, const qs_cache *cache, const int32_t *sel,
+                       const int32_t *n_sel, int32_t batch, void *k_dst, void *v_dst,
+                       int32_t *row_lens, void *ws, qs_stream_t stream);
+
 /* Synchronise `stream`, return the first device-side error recorded in the workspace
    since the last call (QS_OK if none) and clear it. `detail` (HOST pointer, may be NULL)
    receives {kernel id, index} of that error. Returns QS_ERR_CUDA if the synchronisation
    or the read-back fails. Kernel ids: 1 append, 2 block error, 3 scoring prep, 4 score,
-   5 select, 6 attention (with its log-sum-exp combine), 7 the wait self-test. */
+   5 select, 6 attention (with its log-sum-exp combine), 7 the wait self-test,
+   8 the gather of gather-then-attend. */
 qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
 
 /* Sparse attention without a workspace, for callers that cannot allocate device memory:

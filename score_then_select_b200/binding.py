@@ -68,6 +68,9 @@ def lib() -> ctypes.CDLL:
             "qs_decode": ([cfgp, cachep, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp], i32),
             "qs_device_status": ([vp, vp, ctypes.POINTER(ctypes.c_uint32)], i32),
             "qs_sparse_attn_noalloc": ([cfgp, cachep, vp, vp, vp, i32, vp, vp], i32),
+            "qs_dense_workspace_size": ([cfgp, i32, i32, ctypes.POINTER(sz)], i32),
+            "qs_dense_attn": ([cfgp, cachep, vp, vp, i32, vp, vp, vp], i32),
+            "qs_gather_kv": ([cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -80,7 +83,8 @@ def lib() -> ctypes.CDLL:
 EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_init",
            "qs_append_kv", "qs_score", "qs_select_topk", "qs_sparse_attn", "qs_decode",
            "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches",
-           "qs_selftest_wait_timeout")
+           "qs_selftest_wait_timeout", "qs_dense_workspace_size", "qs_dense_attn",
+           "qs_gather_kv")
 
 
 def status_string(s: int) -> str:
@@ -206,6 +210,24 @@ def qs_sparse_attn_noalloc(cfg, cache, q, sel, n_sel, batch, out, stream=None):
     _check(lib().qs_sparse_attn_noalloc(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q),
                                         _ptr(sel), _ptr(n_sel), batch, _ptr(out),
                                         _stream(stream)), "qs_sparse_attn_noalloc")
+
+
+def qs_dense_workspace_size(cfg: qs_config, batch: int, max_context: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().qs_dense_workspace_size(ctypes.byref(cfg), batch, max_context, ctypes.byref(n)),
+           "qs_dense_workspace_size")
+    return n.value
+
+
+def qs_dense_attn(cfg, cache, q, row_lens, batch, out, ws, stream=None):
+    _check(lib().qs_dense_attn(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(row_lens),
+                               batch, _ptr(out), _ptr(ws), _stream(stream)), "qs_dense_attn")
+
+
+def qs_gather_kv(cfg, cache, sel, n_sel, batch, k_dst, v_dst, row_lens, ws, stream=None):
+    _check(lib().qs_gather_kv(ctypes.byref(cfg), ctypes.byref(cache), _ptr(sel), _ptr(n_sel),
+                              batch, _ptr(k_dst), _ptr(v_dst), _ptr(row_lens), _ptr(ws),
+                              _stream(stream)), "qs_gather_kv")
 
 
 def qs_device_status(ws, stream=None) -> tuple[int, int, int]:

@@ -160,6 +160,21 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   return QS_OK;
 }
 
+// Plan of full-KV attention: the configuration's heads, types and scale, with every
+// 128-token block of a row selected in order (block size = page size, budget = pages of
+// max_context), always on the tile pipeline. The configuration itself must be valid.
+static qs_status make_dense_plan(const qs_config* c, int batch, int max_context, Plan& p) {
+  qs_status st = make_plan(c, batch, max_context, p);
+  if (st != QS_OK) return st;
+  qs_config d = *c;
+  d.block_size = kPage;
+  d.budget = (max_context + kPage - 1) / kPage;
+  d.force_sink = d.force_last = 0;
+  d.n_keep_hp = 0;
+  d.attn_path = 1;
+  return make_plan(&d, batch, max_context, p);
+}
+
 qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy) {
   if (!c || !c->k || !c->v || !c->page_table || !c->seq_lens) return QS_ERR_INVALID_ARG;
   if (c->max_pages_per_seq < 1 || c->num_pages < 1 || c->max_context < 1) return QS_ERR_INVALID_ARG;
@@ -290,8 +305,10 @@ static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores
 }
 
 static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, const int32_t* sel,
-                           const int32_t* n_sel, void* out, void* ws, cudaStream_t s, bool pdl) {
+                           const int32_t* n_sel, void* out, void* ws, cudaStream_t s, bool pdl,
+                           const int32_t* row_lens = nullptr) {
   AttnParams a{};
+  a.row_lens = row_lens;
   a.q = static_cast<const uint16_t*>(q);
   a.k = static_cast<const uint16_t*>(c->k);
   a.v = static_cast<const uint16_t*>(c->v);
@@ -412,6 +429,59 @@ qs_status qs_sparse_attn(const qs_config* cfg, const qs_cache* cache, const void
   if ((st = check_cache(p, cache, false)) != QS_OK) return st;
   if (!q || !aligned(q, 16) || !sel || !n_sel || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   return do_attend(p, cache, q, sel, n_sel, out, ws, stream, false);
+}
+
+qs_status qs_dense_workspace_size(const qs_config* cfg, int32_t batch, int32_t max_context,
+                                  size_t* bytes) {
+  if (!bytes) return QS_ERR_INVALID_ARG;
+  Plan p;
+  const qs_status st = make_dense_plan(cfg, batch, max_context, p);
+  if (st != QS_OK) return st;
+  *bytes = p.ws.total;
+  return QS_OK;
+}
+
+qs_status qs_dense_attn(const qs_config* cfg, const qs_cache* cache, const void* q,
+                        const int32_t* row_lens, int32_t batch, void* out, void* ws,
+                        qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_dense_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if ((st = check_cache(p, cache, false)) != QS_OK) return st;
+  if (!q || !aligned(q, 16) || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  return do_attend(p, cache, q, nullptr, nullptr, out, ws, stream, false, row_lens);
+}
+
+qs_status qs_gather_kv(const qs_config* cfg, const qs_cache* cache, const int32_t* sel,
+                       const int32_t* n_sel, int32_t batch, void* k_dst, void* v_dst,
+                       int32_t* row_lens, void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if ((st = check_cache(p, cache, false)) != QS_OK) return st;
+  if (!sel || !n_sel || !k_dst || !v_dst || !row_lens || !ws || !aligned(ws, 256))
+    return QS_ERR_INVALID_ARG;
+  if (!aligned(k_dst, 16) || !aligned(v_dst, 16)) return QS_ERR_INVALID_ARG;
+  GatherParams a{};
+  a.k = static_cast<const uint16_t*>(cache->k);
+  a.v = static_cast<const uint16_t*>(cache->v);
+  a.sel = sel;
+  a.n_sel = n_sel;
+  a.page_table = cache->page_table;
+  a.seq_lens = cache->seq_lens;
+  a.k_dst = static_cast<uint16_t*>(k_dst);
+  a.v_dst = static_cast<uint16_t*>(v_dst);
+  a.row_lens = row_lens;
+  a.hdr = hdr_of(ws);
+  a.rows = p.batch * p.Hkv;
+  a.Hkv = p.Hkv;
+  a.log2_S = 0;
+  while ((1 << a.log2_S) < p.S) ++a.log2_S;
+  a.budget = p.budget;
+  a.dst_pages_per_seq = (p.budget * p.S + kPage - 1) / kPage;
+  a.max_pages_per_seq = cache->max_pages_per_seq;
+  a.num_pages = cache->num_pages;
+  return cuda_status(launch_gather_kv(p, a, stream));
 }
 
 qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, const void* k_new,

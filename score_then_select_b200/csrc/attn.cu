@@ -9,6 +9,10 @@
 // "Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse Attention", Full
 // text: value aggregation in FP16 with FP32 accumulation over contiguous block tiles.
 //
+// Full-KV attention (the dense baseline the pages compare the sparse stage with) runs the
+// same kernel without a selection: every 128-token block of the row in order, optionally
+// over per-row lengths (the compact buffer of gather-then-attend, gather.cu).
+//
 // Work decomposition (persistent grid, dynamic): a row (sequence, KV head) holds
 // `tiles_per_row` 64-token tiles of selected slots, cut into chunks of `chunk_tiles` tiles;
 // CTA c starts with chunks c and c + C, then claims the rest in order from a workspace
@@ -159,10 +163,15 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
         const int tin0 = (c - r.row * cpr) * ktiles, j = lane >> (6 - lg_hb);
         if (j < min(ktiles, tpr - tin0)) {
           r.sl = (tin0 + j) * kTileT + ((lane & (rpt - 1)) << lg_hb);
-          r.n = a.n_sel[r.row];
-          r.L = a.seq_lens[r.row / a.Hkv];
+          r.L = a.row_lens ? a.row_lens[r.row] : a.seq_lens[r.row / a.Hkv];
           const int e = r.sl >> lgS;
-          if (e < a.budget) r.blk = a.sel[size_t(r.row) * a.budget + e];
+          if (a.sel) {
+            r.n = a.n_sel[r.row];
+            if (e < a.budget) r.blk = a.sel[size_t(r.row) * a.budget + e];
+          } else {                                         // full KV: every block, in order
+            r.n = int((static_cast<long long>(r.L) + (1 << lgS) - 1) >> lgS);
+            r.blk = e;
+          }
         } else {
           r.n = -2;                                        // no such run in this chunk
         }

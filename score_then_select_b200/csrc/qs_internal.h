@@ -18,7 +18,8 @@ enum KernelId : uint32_t {
   KID_SCORE = 4,
   KID_SELECT = 5,
   KID_ATTN = 6,
-  KID_SELFTEST = 7
+  KID_SELFTEST = 7,
+  KID_GATHER = 8
 };
 
 constexpr int kPage = 128;          // tokens per page (the only page size built)
@@ -168,10 +169,11 @@ struct AttnParams {
   const uint16_t* q;
   const uint16_t* k;
   const uint16_t* v;
-  const int32_t* sel;
+  const int32_t* sel;        // nullptr: full KV (every block of the row, in order)
   const int32_t* n_sel;
   const int32_t* page_table;
   const int32_t* seq_lens;
+  const int32_t* row_lens;   // [batch * Hkv] tokens per row, or nullptr (=> seq_lens[b])
   float* part_ml;
   float* part_o;
   uint32_t* row_ctr;         // [batch * Hkv] segments finished (self-resetting)
@@ -184,6 +186,20 @@ struct AttnParams {
   int gsplits, g_tokens_per_split;   // gather kernel split plan
   int out_bf16;
   float scale_log2;          // softmax scale * log2(e)
+};
+
+struct GatherParams {        // gather-then-attend: selected blocks -> compact pages
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* sel;
+  const int32_t* n_sel;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  uint16_t* k_dst;           // [batch * dst_pages_per_seq][Hkv][128][d]
+  uint16_t* v_dst;
+  int32_t* row_lens;         // [batch * Hkv] gathered valid tokens
+  uint32_t* hdr;
+  int rows, Hkv, log2_S, budget, dst_pages_per_seq, max_pages_per_seq, num_pages;
 };
 
 // Launch `kern` on `s`; with `pdl` the launch may overlap the tail of the previous kernel
@@ -213,6 +229,7 @@ cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s, bo
 cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_attn_gather(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl);
+cudaError_t launch_gather_kv(const Plan& p, const GatherParams& a, cudaStream_t s);
 
 int num_sms();
 

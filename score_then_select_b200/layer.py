@@ -70,3 +70,48 @@ class Layer:
     def nb_stride(self) -> int:
         ps = self.cfg.page_size
         return -(-self.max_context // ps) * (ps // self.cfg.block_size)
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zeroed workspace of `nbytes` bytes, initialised for the library's calls."""
+    ws = torch.zeros((nbytes,), dtype=torch.uint8, device=device)
+    B.qs_workspace_init(ws, nbytes)
+    return ws
+
+
+@dataclass
+class GatheredKV:
+    """The compact buffers of gather-then-attend (filled by qs_gather_kv) and the cache view
+    over them that qs_dense_attn reads: ceil(budget * block_size / 128) pages per sequence,
+    page i of sequence b at b * pages_per_seq + i."""
+    k: torch.Tensor
+    v: torch.Tensor
+    page_table: torch.Tensor
+    seq_lens: torch.Tensor
+    row_lens: torch.Tensor
+    pages_per_seq: int
+
+    @staticmethod
+    def allocate(layer: Layer, fill: float | None = None) -> "GatheredKV":
+        cfg = layer.cfg
+        ps = cfg.page_size
+        P = -(-cfg.budget * cfg.block_size // ps)
+        dev = layer.k.device
+        shape = (layer.batch * P, cfg.n_kv_heads, ps, cfg.head_dim)
+        k = torch.empty(shape, dtype=layer.k.dtype, device=dev)
+        v = torch.empty(shape, dtype=layer.v.dtype, device=dev)
+        if fill is not None:
+            k.fill_(fill)
+            v.fill_(fill)
+        pt = torch.arange(layer.batch * P, dtype=torch.int32, device=dev).reshape(layer.batch, P)
+        sl = torch.zeros((layer.batch,), dtype=torch.int32, device=dev)
+        rl = torch.zeros((layer.batch * cfg.n_kv_heads,), dtype=torch.int32, device=dev)
+        return GatheredKV(k, v, pt, sl, rl, P)
+
+    @property
+    def max_context(self) -> int:
+        return self.pages_per_seq * 128
+
+    def cache(self) -> B.qs_cache:
+        return B.make_cache(k=self.k, v=self.v, proxy=None, page_table=self.page_table,
+                            seq_lens=self.seq_lens, max_context=self.max_context)

@@ -79,3 +79,29 @@ def test_null_pointers_rejected_without_launch():
     with pytest.raises(qs.QsError) as e:
         qs.qs_decode(cfg, cache, 0, 0, 0, 0, 16, 0, None, None, 0, stream=0)
     assert e.value.status == B.QS_ERR_INVALID_ARG
+
+
+def test_dense_workspace_covers_every_page_and_limits_context():
+    # full-KV attention plans every 128-token page of the row: more partials than the sparse
+    # plan of the same cache, and contexts past 128K tokens are refused on the host
+    sparse = qs.qs_workspace_size(_cfg(), 16, 131072)
+    dense = qs.qs_dense_workspace_size(_cfg(), 16, 131072)
+    assert dense > sparse
+    assert qs.qs_dense_workspace_size(_cfg(), 16, 2048) < dense
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_dense_workspace_size(_cfg(), 16, 131073)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    with pytest.raises(qs.QsError) as e:                      # an invalid configuration
+        qs.qs_dense_workspace_size(_cfg(n_q_heads=41), 16, 4096)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+
+
+def test_comparison_calls_reject_null_pointers_without_launch():
+    cfg = _cfg()
+    cache = B.qs_cache()
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_dense_attn(cfg, cache, 0, None, 16, 0, 0, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_gather_kv(cfg, cache, 0, 0, 16, 0, 0, 0, 0, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
