@@ -260,8 +260,9 @@ static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws,
 }
 
 static qs_status do_score(const Plan& p, const qs_cache* c, float* scores, void* ws, cudaStream_t s,
-                          bool pdl) {
+                          bool pdl, bool early_stream = false) {
   ScoreParams a{};
+  a.early_stream = early_stream ? 1 : 0;
   a.proxy = c->proxy;
   a.proxy_scale = c->proxy_scale;
   a.qt = ws_at<float>(ws, p.ws.qt);
@@ -405,8 +406,10 @@ qs_status qs_score(const qs_config* cfg, const qs_cache* cache, const void* q, c
   if (!q || !aligned(q, 4) || !block_scores || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
   if (p.r == 0 && !aligned(q, 16)) return QS_ERR_INVALID_ARG;
+  // the prep kernel runs in stream order and writes only the query side, so the scan
+  // overlaps it and starts streaming pages before it waits for the query
   if ((st = do_prep(p, q, P, ws, stream, false)) != QS_OK) return st;
-  return do_score(p, cache, block_scores, ws, stream, true);
+  return do_score(p, cache, block_scores, ws, stream, true, true);
 }
 
 qs_status qs_select_topk(const qs_config* cfg, const qs_cache* cache, const float* block_scores,

@@ -476,12 +476,44 @@ __global__ void __launch_bounds__(256) block_err_kernel(const BlockErrParams a) 
 
 // ============================================================ scoring prep
 __global__ void __launch_bounds__(128) prep_rankr_kernel(const PrepParams a) {
+  extern __shared__ __align__(16) float Ps[];      // P[g]: [d][r]
   __shared__ float qbar[256];
   pdl_trigger();   // the scan may launch now; it waits for this grid before reading q~
-  const int row = blockIdx.x;
+  const int row = blockIdx.x, tid = threadIdx.x;
   const int b = row / a.Hkv, g = row % a.Hkv;
-  row_prep(a.q, a.P + size_t(g) * a.d * a.r, a.qt + size_t(row) * a.r, qbar, b, g, a.Hkv, a.G,
-           a.d, a.r);
+  // every global load is issued before any is consumed: P[g] (at most 32 KiB) as float4
+  // and the group's query elements of dimension tid
+  constexpr int kMaxP4 = 128 * 64 / 4 / 128;       // float4 loads per thread (d = 128, r = 64)
+  const int n4 = a.d * a.r / 4;
+  const float4* Pg4 = reinterpret_cast<const float4*>(a.P + size_t(g) * a.d * a.r);
+  float4 pv[kMaxP4];
+#pragma unroll
+  for (int j = 0; j < kMaxP4; ++j)
+    if (j * 128 + tid < n4) pv[j] = Pg4[j * 128 + tid];
+  const int Hq = a.Hkv * a.G;
+  const bool has_q = tid < a.d;
+  uint16_t qraw[kMaxGroup];
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h)
+    qraw[h] = (has_q && h < a.G) ? a.q[(size_t(b) * Hq + g * a.G + h) * a.d + tid] : uint16_t(0);
+#pragma unroll
+  for (int j = 0; j < kMaxP4; ++j)
+    if (j * 128 + tid < n4) reinterpret_cast<float4*>(Ps)[j * 128 + tid] = pv[j];
+  if (has_q) {
+    float s = 0.0f;
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+      if (h < a.G) s += bf16_to_f32(qraw[h]);
+    qbar[tid] = s / float(a.G);
+  }
+  __syncthreads();
+  // q~_j = sum_i qbar_i P_ij, ascending i (the decode append's fused prep does the same)
+  for (int j = tid; j < a.r; j += 128) {
+    float acc = 0.0f;
+#pragma unroll 8
+    for (int i = 0; i < a.d; ++i) acc = fmaf(qbar[i], Ps[i * a.r + j], acc);
+    a.qt[size_t(row) * a.r + j] = acc;
+  }
 }
 
 // NVFP4 query packing: CTA = one row (sequence, KV head). g_q = max|q| / 2688 over the
@@ -597,7 +629,8 @@ cudaError_t launch_block_err(const Plan& p, const BlockErrParams& a, cudaStream_
 }
 
 cudaError_t launch_prep(const Plan& p, const PrepParams& a, cudaStream_t s) {
-  prep_rankr_kernel<<<a.batch * a.Hkv, 128, 0, s>>>(a);
+  const size_t smem = size_t(a.d) * a.r * sizeof(float);      // <= 32 KiB
+  prep_rankr_kernel<<<a.batch * a.Hkv, 128, smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -153,6 +153,10 @@ struct ScoreParams {
   float* scores;
   uint32_t* hdr;
   int batch, Hkv, G, d, S, nb_stride, max_pages_per_seq, num_pages, max_context;
+  // 1: the kernel before this one (launched in stream order, without overlap) writes only
+  // the query side (q~, or the NVFP4 query tiles and g_q), so the page stream may start
+  // before waiting for it; 0: wait for it first (it may still be writing seq_lens)
+  int early_stream;
 };
 
 struct SelectParams {

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
   int* prefix = reinterpret_cast<int*>(info + NST);               // [batch + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_wait();      // q~ and seq_lens come from the kernel before
+  if (!a.early_stream) pdl_wait();   // q~ and seq_lens come from the kernel before
   pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
   const int rot = (SH::kTokenBytes == 64) ? (lane >> 1) : lane;
   float qr[CPT][EPC];                                 // q~ permuted by this lane's rotation
   int cur_row = -1;
+  if (a.early_stream) pdl_wait();                     // q~ comes from the kernel before
   const int bpp = kPage / a.S;  // blocks per page
   for (int k = c; k < n_units; k += kScoreConsumers) {
     const int s = k % NST;

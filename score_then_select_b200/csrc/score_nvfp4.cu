@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kF4Threads) score_nvfp4_kernel(const ScorePara
   int* prefix = reinterpret_cast<int*>(s_tmem + 4);               // [batch + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_wait();      // the query tiles, g_q and seq_lens come from the kernels before
+  if (!a.early_stream) pdl_wait();   // query tiles, g_q and seq_lens: the kernels before
   pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(kF4Threads) score_nvfp4_kernel(const ScorePara
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (one lane)
+    if (a.early_stream) pdl_wait();   // the query tiles come from the kernel before
     if (lane == 0) {
       int cur_row = -1;
       uint32_t bph0 = 0, bph1 = 0;     // parities of the B-tile and drain barriers
@@ -274,6 +275,7 @@ __global__ void __launch_bounds__(kF4Threads) score_nvfp4_kernel(const ScorePara
     const int eg = (warp - 2) >> 2;
     const int q = warp & 3;
     const bool leader = ((warp - 2) & 3) == 0;       // first warp of its group
+    if (a.early_stream) pdl_wait();                   // g_q comes from the kernel before
     const float gscale = __fmul_rn(*a.qgscale, *a.key_gscale);
     const uint32_t lane_addr = uint32_t(32 * q) << 16;
     for (int k = eg; k < n_units; k += kF4EpiGroups) {
