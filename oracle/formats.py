@@ -8,6 +8,8 @@ TEST INFRASTRUCTURE: only tests, the smoke check and the bench's CPU-baseline le
     inf/NaN; magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}; bit 3 is the sign.
   * UE4M3 (the NVFP4 block-scale type, an E4M3 with the sign bit unused): 4 exponent bits,
     bias 7, 3 mantissa bits; subnormals m * 2^-9; largest finite 448 (0x7E); 0x7F is NaN.
+  * E4M3 (the FP8 element type of the reduced-precision projected-key cache): bit 7 is the
+    sign, bits 6..0 a UE4M3 magnitude; 0x7F and 0xFF are NaN.
 
 "Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse Attention" (Full text)
 names NVFP4 storage; the element/scale layout above is the public NVFP4 format.
@@ -96,3 +98,21 @@ def ue4m3_encode(sf: np.ndarray) -> np.ndarray:
     s64 = np.asarray(sf, dtype=np.float32).astype(np.float64)
     code = _nearest_even(UE4M3_VALUES, s64)
     return np.where(s64 >= 448.0, 126, code).astype(np.uint8)
+
+
+# ---- E4M3 (signed FP8) ------------------------------------------------------------------------
+
+def e4m3_value(code: np.ndarray) -> np.ndarray:
+    """Decode signed E4M3 codes (0..255) to float64 (0x7F / 0xFF decode to NaN)."""
+    c = np.asarray(code).astype(np.int64)
+    mag = ue4m3_value(c & 0x7F)
+    return np.where((c & 0x80) != 0, -mag, mag)
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """float32 -> E4M3 code: magnitude to the nearest UE4M3 value (ties to the even code,
+    saturating at 448), sign bit copied (so -0.0 and negative values that round to zero
+    keep it)."""
+    x64 = np.asarray(x, dtype=np.float32).astype(np.float64)
+    mag = ue4m3_encode(np.abs(x64)).astype(np.int64)
+    return (mag | np.where(np.signbit(x64), 0x80, 0)).astype(np.uint8)

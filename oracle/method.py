@@ -61,18 +61,24 @@ def proxy_keys_f32(k_bits: np.ndarray, P: np.ndarray) -> np.ndarray:
 
 
 def proxy_store(k_bits: np.ndarray, P: np.ndarray, dtype: str):
-    """Stored proxy cache entries: float32 values ('f32') or BF16 bit patterns ('bf16')."""
+    """Stored proxy cache entries: float32 values ('f32'), BF16 bit patterns ('bf16') or
+    FP8 E4M3 codes ('e4m3', the reduced-precision scoring cache of [JSSA, Figure 10]), each
+    a rounding of the float32 projected key."""
     acc = proxy_keys_f32(k_bits, P)
     if dtype == "f32":
         return acc
     if dtype == "bf16":
         return F.f32_to_bf16_rne(acc)
+    if dtype == "e4m3":
+        return F.e4m3_encode(acc)
     raise ValueError(dtype)
 
 
 def proxy_decode(stored, dtype: str) -> np.ndarray:
     if dtype == "f32":
         return np.asarray(stored, dtype=np.float32).astype(np.float64)
+    if dtype == "e4m3":
+        return F.e4m3_value(stored)
     return F.bf16_to_f64(stored)
 
 

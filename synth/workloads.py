@@ -26,7 +26,7 @@ class Workload:
     block_size: int              # S
     budget: int                  # k, in blocks
     proxy_rank: int              # r > 0: projected-key proxy; 0: NVFP4 centred keys
-    proxy_dtype: str             # 'f32' | 'bf16' | 'nvfp4'
+    proxy_dtype: str             # 'f32' | 'bf16' | 'e4m3' | 'nvfp4'
     v_dtype: str                 # stored V: 'bf16' | 'f16'
     v_agg_dtype: str             # PV operand precision: 'bf16' | 'f16'
     out_dtype: str               # 'f32' | 'bf16'
@@ -96,6 +96,16 @@ NVFP4_128K = BLOCK128K.replace(
     name="nvfp4_b16_h40kv8_d128_L131072_S128_k128", budget=128, proxy_rank=0,
     proxy_dtype="nvfp4", v_dtype="f16", v_agg_dtype="f16", n_keep_hp=2, seed=1004)
 
+# The 128K block-level step with the projected-key cache stored as FP8 E4M3 ("Joint Subspace
+# Sparse Attention for Efficient Long-Context Decoding", Figure 10: FP8 or BF16 scoring
+# cache; the full KV cache and the attention stay BF16).
+FP8_128K = BLOCK128K.replace(name="fp8_b16_h40kv8_d128_L131072_S128_k64_r32", proxy_dtype="e4m3",
+                             seed=1006)
+
+# Token-level selection over an FP8 E4M3 projected-key cache of rank 64 (B = 2,048 tokens).
+FP8_TOKEN32K = TOKEN32K.replace(name="fp8_token_b16_h32kv8_d128_L32768_r64_B2048",
+                                proxy_rank=64, proxy_dtype="e4m3", seed=1007)
+
 # Ragged batch: 32 sequences, lengths uniform in [4096, 131072], G = 8, r = 64, S = 64.
 RAGGED = Workload(
     name="ragged_b32_h64kv8_d128_S64_k32_r64", batch=32, n_q_heads=64, n_kv_heads=8,
@@ -106,6 +116,8 @@ RAGGED = Workload(
 
 FULL = {w.name: w for w in (TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED)}
 ORDER = [TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED]
+# variants of the configurations above (the FP8 projected-key cache)
+VARIANTS = [FP8_128K, FP8_TOKEN32K]
 
 
 def small(w: Workload) -> Workload:

@@ -36,7 +36,8 @@ def test_round_trips():
 def test_rounding_cases():
     for kind, x, want in read_golden("rounding_cases.txt"):
         arr = np.array([float(x)], dtype=np.float32)
-        got = F.e2m1_encode(arr)[0] if kind == "e2m1" else F.ue4m3_encode(arr)[0]
+        enc = {"e2m1": F.e2m1_encode, "ue4m3": F.ue4m3_encode, "e4m3": F.e4m3_encode}[kind]
+        got = enc(arr)[0]
         assert int(got) == int(want, 16), (kind, x, hex(int(got)))
 
 
@@ -91,3 +92,34 @@ def test_bf16_rounding_exact_rational():
 def test_bf16_midpoints_hand():
     xs = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 2 ** -130], dtype=np.float32)
     assert F.f32_to_bf16_rne(xs).tolist() == [0x3F80, 0x3F82, 0x0008]
+
+
+def test_e4m3_sign_symmetry_and_nan():
+    mags = np.arange(127)
+    pos = F.e4m3_value(mags)
+    neg = F.e4m3_value(mags | 0x80)
+    assert np.array_equal(neg, -pos)
+    assert np.array_equal(pos, F.ue4m3_value(mags))
+    assert np.isnan(F.e4m3_value(np.array([0x7F, 0xFF]))).all()
+    assert math.copysign(1.0, float(F.e4m3_value(np.array([0x80]))[0])) == -1.0
+
+
+def test_e4m3_round_trip_every_finite_code():
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)
+    vals = F.e4m3_value(codes).astype(np.float32)
+    assert np.array_equal(F.e4m3_encode(vals), codes)
+
+
+def test_e4m3_encode_is_nearest():
+    """Brute force over random float32 inputs: the decoded code is a nearest finite E4M3
+    value (or +-448 beyond it), with the input's sign."""
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(4000) * 10.0, rng.standard_normal(2000) * 0.01,
+                        rng.uniform(-600, 600, 1000)]).astype(np.float32)
+    finite = np.unique(np.abs(F.e4m3_value(np.arange(127))))
+    got = F.e4m3_value(F.e4m3_encode(x))
+    for xi, gi in zip(x.astype(np.float64), got):
+        m = min(abs(xi), 448.0)
+        best = np.min(np.abs(finite - m))
+        assert abs(abs(gi) - m) == best, (xi, gi)
+        assert math.copysign(1.0, gi) == math.copysign(1.0, xi)

@@ -294,3 +294,28 @@ def test_gather_then_dense_equals_sparse_attention(seed):
     got = M.dense_attention(q, Kg, Vg, n, 0.2)
     want = _dense_attention_bruteforce(q, K[M.block_tokens(sel, S, L)], V[M.block_tokens(sel, S, L)], 0.2)
     assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_e4m3_proxy_store_exact_for_representable_keys():
+    # P = I and keys that are E4M3 values: the FP8 cache holds the keys exactly
+    rng = np.random.default_rng(30)
+    vals = F.e4m3_value(np.array([c for c in range(256) if c & 0x7F != 0x7F]))
+    k = rng.choice(vals, size=(40, 16))
+    kb = F.f32_to_bf16_rne(k.astype(np.float32))
+    assert np.array_equal(F.bf16_to_f64(kb), k)            # E4M3 values are BF16 values
+    st = M.proxy_store(kb, np.eye(16, dtype=np.float32), "e4m3")
+    assert st.dtype == np.uint8
+    assert np.array_equal(M.proxy_decode(st, "e4m3"), k)
+
+
+def test_e4m3_proxy_store_rounds_the_float32_projection():
+    # each stored entry is the E4M3 value nearest the float32 projection (relative error at
+    # most 2^-4 in the normal range, saturating at 448)
+    rng = np.random.default_rng(31)
+    kb = _bf16(rng.standard_normal((64, 32)) * 3)
+    P = np.linalg.qr(rng.standard_normal((32, 16)))[0].astype(np.float32)
+    f32 = M.proxy_keys_f32(kb, P).astype(np.float64)
+    dec = M.proxy_decode(M.proxy_store(kb, P, "e4m3"), "e4m3")
+    normal = np.abs(f32) >= 2.0 ** -6
+    assert np.all(np.abs(dec - f32)[normal] <= np.abs(f32)[normal] * 2.0 ** -4)
+    assert np.all(np.abs(dec - f32)[~normal] <= 2.0 ** -10)

@@ -23,7 +23,8 @@ def test_literal_tiny_runs(capsys):
     print("literal tiny workload: needle block 37 selected =", 37 in r["sel"].tolist())
 
 
-@pytest.mark.parametrize("w", [synth.small(w) for w in synth.ORDER[1:]], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [synth.small(w) for w in synth.ORDER[1:] + synth.VARIANTS],
+                         ids=lambda w: w.name)
 def test_small_workload_invariants(w):
     inp = synth.Inputs(w)
     gq = query_scale_all(inp) if w.proxy_dtype == "nvfp4" else None
