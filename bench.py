@@ -41,7 +41,8 @@ import synth  # noqa: E402
 
 METRIC = "sparse decode attn steps/s at 128K ctx, batch 16; achieved HBM GB/s vs peak"
 WORKLOADS = {"block128k": synth.BLOCK128K, "token32k": synth.TOKEN32K, "ragged": synth.RAGGED,
-             "nvfp4": synth.NVFP4_128K, "tiny": synth.TINY}
+             "nvfp4": synth.NVFP4_128K, "tiny": synth.TINY, "fp8": synth.FP8_128K,
+             "fp8token": synth.FP8_TOKEN32K}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -148,7 +149,7 @@ def step_bytes(w, lens, sel, nsel):
     if w.proxy_dtype == "nvfp4":
         per_tok = d // 2 + d // 16
     else:
-        per_tok = w.proxy_rank * (4 if w.proxy_dtype == "f32" else 2)
+        per_tok = w.proxy_rank * {"f32": 4, "bf16": 2, "e4m3": 1}[w.proxy_dtype]
     proxy = int(np.sum(lens.astype(np.int64))) * w.n_kv_heads * per_tok
     tokens = 0
     for b in range(w.batch):
@@ -568,7 +569,8 @@ def run_ours(args):
     value = aggregate_steps_per_s(t_ms, world)
     line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.proxy_dtype == "bf16" else f"{w.proxy_dtype}+bf16",
             "data": "synthetic (seeded; shapes of the pages' 128K batch-16 decode)",
             "config": config_of(w, lens),
             "tokens_per_s": value * B, "us_per_layer_step": t_ms * 1e3,

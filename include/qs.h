@@ -46,7 +46,10 @@
  *
  * Memory layouts (row-major, innermost last):
  *   K, V pages      [num_pages][Hkv][page_size][head_dim]   BF16 (V may be FP16)
- *   proxy (rank r)  [num_pages][Hkv][page_size][r]          F32 or BF16
+ *   proxy (rank r)  [num_pages][Hkv][page_size][r]          F32, BF16 or E4M3 (FP8: sign,
+ *                                                           4 exponent bits with bias 7,
+ *                                                           3 mantissa bits; largest 448;
+ *                                                           one byte per entry)
  *   proxy (NVFP4)   [num_pages][Hkv][page_size][head_dim/2] u8: E2M1 codes, element 2i in
  *                                                           the low nibble of byte i
  *   proxy_scale     [num_pages][Hkv][page_size][head_dim/16] u8: UE4M3 scale per 16 elems
@@ -82,7 +85,7 @@ typedef enum {
   QS_ERR_DEVICE_TIMEOUT = 5
 } qs_status;
 
-typedef enum { QS_F32 = 0, QS_BF16 = 1, QS_F16 = 2, QS_NVFP4 = 3 } qs_dtype;
+typedef enum { QS_F32 = 0, QS_BF16 = 1, QS_F16 = 2, QS_NVFP4 = 3, QS_E4M3 = 4 } qs_dtype;
 
 /* Problem statement of one attention layer's decode step. */
 typedef struct {
@@ -93,7 +96,7 @@ typedef struct {
   int32_t block_size;     /* S: a power of two dividing page_size (1 = token level)       */
   int32_t budget;         /* k: blocks selected per row, >= 1                             */
   int32_t proxy_rank;     /* r > 0: projected-key proxy; 0: NVFP4 centred keys            */
-  int32_t proxy_dtype;    /* qs_dtype: F32 or BF16 (rank r), NVFP4 (r == 0)               */
+  int32_t proxy_dtype;    /* qs_dtype: F32, BF16 or E4M3 (rank r), NVFP4 (r == 0)         */
   int32_t v_dtype;        /* qs_dtype of stored V: BF16 or F16                            */
   int32_t v_agg_dtype;    /* precision of the P.V operands: BF16 or F16 (FP32 accumulate) */
   int32_t out_dtype;      /* F32 or BF16                                                  */
@@ -143,7 +146,9 @@ qs_status qs_workspace_init(void *ws, size_t ws_bytes, qs_stream_t stream);
 /* Append n_new[b] tokens to every KV head of sequence b, then advance seq_lens[b].
    Writes K/V into page slot seq_lens[b] + i and the row's scoring cache:
      rank r: proxy = k.P[g] in float32 (ascending index, one rounding per product and per
-             sum), stored F32 or rounded to nearest-even BF16;
+             sum), stored F32, rounded to nearest-even BF16, or rounded to nearest-even E4M3
+             saturating at +-448 (the FP8 scoring cache of "Joint Subspace Sparse Attention
+             ...", Figure 10);
      NVFP4:  x = float(k) - key_center[b][g] (float32), packed per 16 elements to UE4M3
              scale + E2M1 codes with the tensor scale g_k; each block of S tokens that this
              call completes gets block_err = sum of squared (x - dequant(x)).

@@ -91,7 +91,8 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   if (r < 0) return QS_ERR_INVALID_ARG;
   if (r > 0) {
     const bool ok = (c->proxy_dtype == QS_F32 && (r == 16 || (r == 32 && c->head_dim == 128))) ||
-                    (c->proxy_dtype == QS_BF16 && (r == 32 || (r == 64 && c->head_dim == 128)));
+                    ((c->proxy_dtype == QS_BF16 || c->proxy_dtype == QS_E4M3) &&
+                     (r == 32 || (r == 64 && c->head_dim == 128)));
     if (!ok) return QS_ERR_UNSUPPORTED;
     if (c->n_keep_hp != 0) return QS_ERR_INVALID_ARG;
   } else {

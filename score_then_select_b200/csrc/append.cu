@@ -48,6 +48,11 @@ QS_DEV uint32_t ue4m3_encode(float sf) {
   if (rem > 0x80000u || (rem == 0x80000u && (code & 1u))) code += 1u;
   return code > 0x7Eu ? 0x7Eu : code;
 }
+// Signed E4M3 (the FP8 projected-key cache): the magnitude as UE4M3 above, bit 7 the sign
+// (kept for negative values that round to zero, and for -0).
+QS_DEV uint32_t e4m3_encode(float x) {
+  return ue4m3_encode(fabsf(x)) | (signbit(x) ? 0x80u : 0u);
+}
 QS_DEV float ue4m3_decode(uint32_t c) {
   const uint32_t e = c >> 3, m = c & 7u;
   if (e == 0u) return float(m) * 0.001953125f;
@@ -231,6 +236,10 @@ append_rankr_kernel(const AppendParams a) {
       if constexpr (sizeof(PT) == 4) {
         *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.proxy) + base) =
             make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+      } else if constexpr (sizeof(PT) == 1) {
+        *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.proxy) + base) =
+            e4m3_encode(acc[x][0]) | (e4m3_encode(acc[x][1]) << 8) |
+            (e4m3_encode(acc[x][2]) << 16) | (e4m3_encode(acc[x][3]) << 24);
       } else {
         const uint32_t lo = uint32_t(f32_to_bf16_rn(acc[x][0])) |
                             (uint32_t(f32_to_bf16_rn(acc[x][1])) << 16);
@@ -331,6 +340,8 @@ __global__ void __launch_bounds__(128) append_one_rankr_kernel(const AppendParam
       const size_t pdst = ((size_t(page) * a.Hkv + g) * kPage + s_slot) * R + tid;
       if constexpr (sizeof(PT) == 4)
         reinterpret_cast<float*>(a.proxy)[pdst] = acc;
+      else if constexpr (sizeof(PT) == 1)
+        reinterpret_cast<uint8_t*>(a.proxy)[pdst] = uint8_t(e4m3_encode(acc));
       else
         reinterpret_cast<uint16_t*>(a.proxy)[pdst] = f32_to_bf16_rn(acc);
     }
@@ -596,9 +607,16 @@ cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) 
     return cudaGetLastError();
   }
   const bool f32 = p.proxy_dtype == QS_F32;
+  const bool fp8 = p.proxy_dtype == QS_E4M3;
   if (a.max_new == 1) {
 #define QS_ONE(PT, R, D) \
   { append_one_rankr_kernel<PT, R, D><<<a.batch * a.Hkv, 128, 0, s>>>(a); return cudaGetLastError(); }
+    if (fp8) {
+      if (p.d == 64 && p.r == 32) QS_ONE(uint8_t, 32, 64)
+      if (p.d == 128 && p.r == 32) QS_ONE(uint8_t, 32, 128)
+      if (p.d == 128 && p.r == 64) QS_ONE(uint8_t, 64, 128)
+      return cudaErrorInvalidValue;
+    }
     if (p.d == 64) {
       if (f32 && p.r == 16) QS_ONE(float, 16, 64)
       if (!f32 && p.r == 32) QS_ONE(uint16_t, 32, 64)
@@ -609,6 +627,12 @@ cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) 
       if (!f32 && p.r == 64) QS_ONE(uint16_t, 64, 128)
     }
 #undef QS_ONE
+    return cudaErrorInvalidValue;
+  }
+  if (fp8) {
+    if (p.d == 64 && p.r == 32) return launch_rankr<uint8_t, 32, 64>(p, a, s);
+    if (p.d == 128 && p.r == 32) return launch_rankr<uint8_t, 32, 128>(p, a, s);
+    if (p.d == 128 && p.r == 64) return launch_rankr<uint8_t, 64, 128>(p, a, s);
     return cudaErrorInvalidValue;
   }
   if (p.d == 64) {

@@ -178,6 +178,15 @@ QS_DEV uint32_t pack_f16x2(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Two FP8 E4M3 codes (byte 0 -> low half, byte 1 -> high half) -> f16x2; exact (every
+// E4M3 value is an FP16 value). Used to decode the FP8 projected-key cache.
+QS_DEV uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(uint16_t(two_codes)));
+  return r;
+}
+QS_DEV float f16_lo(uint32_t x) { return __half2float(__ushort_as_half(uint16_t(x))); }
+QS_DEV float f16_hi(uint32_t x) { return __half2float(__ushort_as_half(uint16_t(x >> 16))); }
 // bf16x2 -> f16x2 (for FP16 value aggregation of BF16-stored values)
 QS_DEV uint32_t bf16x2_to_f16x2(uint32_t x) { return pack_f16x2(bf16_lo(x), bf16_hi(x)); }
 

@@ -7,7 +7,9 @@
 // its valid tokens' scores (the reading taken for block selection, "Jet-QSparse",
 // Full text, which selects 128-token blocks from a dense scan).
 //
-// The scan is bound by HBM bandwidth (2r bytes and 2r flops per token). Design:
+// The scan is bound by HBM bandwidth (r, 2r or 4r bytes and 2r flops per token for an FP8,
+// BF16 or FP32 cache; "Joint Subspace Sparse Attention ...", Figure 10, keeps the
+// projected-key cache at FP8 or BF16). Design:
 //   - persistent grid; the (sequence, KV head, page) units of all rows are split evenly
 //     over the CTAs, counting only pages that hold tokens (ragged batches balance);
 //   - one elected producer lane per CTA streams each unit's contiguous page chunk
@@ -169,7 +171,8 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
   constexpr int CPT = SH::kTokenBytes / 16;           // 16-byte chunks per token: 4 or 8
   constexpr int EPC = SH::kEPL;                       // elements per chunk: 8 (bf16) / 4 (f32)
   const int c = warp - 1;
-  const int rot = (SH::kTokenBytes == 64) ? (lane >> 1) : lane;
+  // lanes that share a 128-byte bank window in a quarter-warp start at different chunks
+  const int rot = lane / (128 / SH::kTokenBytes);
   float qr[CPT][EPC];                                 // q~ permuted by this lane's rotation
   int cur_row = -1;
   if (a.early_stream) pdl_wait();                     // q~ comes from the kernel before
@@ -207,7 +210,16 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
           const uint4 v = *reinterpret_cast<const uint4*>(tp + (((kk + rot) & (CPT - 1)) << 4));
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
           float t = 0.0f;
-          if constexpr (sizeof(PT) == 2) {
+          if constexpr (sizeof(PT) == 1) {            // FP8 E4M3, decoded exactly via FP16
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t h01 = e4m3x2_to_f16x2(w[e]), h23 = e4m3x2_to_f16x2(w[e] >> 16);
+              t = fmaf(f16_lo(h01), qr[kk][4 * e], t);
+              t = fmaf(f16_hi(h01), qr[kk][4 * e + 1], t);
+              t = fmaf(f16_lo(h23), qr[kk][4 * e + 2], t);
+              t = fmaf(f16_hi(h23), qr[kk][4 * e + 3], t);
+            }
+          } else if constexpr (sizeof(PT) == 2) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               t = fmaf(bf16_lo(w[e]), qr[kk][2 * e], t);
@@ -278,6 +290,11 @@ cudaError_t launch_score_nvfp4(const Plan& p, const ScoreParams& a, cudaStream_t
 
 cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl) {
   if (p.r == 0) return launch_score_nvfp4(p, a, s, pdl);
+  if (p.proxy_dtype == QS_E4M3) {
+    if (p.r == 32) return launch_rankr_score<uint8_t, 32>(a, s, pdl);
+    if (p.r == 64) return launch_rankr_score<uint8_t, 64>(a, s, pdl);
+    return cudaErrorInvalidValue;
+  }
   const bool f32 = p.proxy_dtype == QS_F32;
   if (f32 && p.r == 16) return launch_rankr_score<float, 16>(a, s, pdl);
   if (f32 && p.r == 32) return launch_rankr_score<float, 32>(a, s, pdl);

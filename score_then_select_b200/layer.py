@@ -41,7 +41,8 @@ class Layer:
         v = torch.zeros((num_pages, Hkv, ps, d), dtype=vdt, device=device)
         extra = {}
         if r > 0:
-            pdt = torch.float32 if cfg.proxy_dtype == B.QS_F32 else torch.bfloat16
+            pdt = {B.QS_F32: torch.float32, B.QS_E4M3: torch.uint8}.get(cfg.proxy_dtype,
+                                                                        torch.bfloat16)
             proxy = torch.zeros((num_pages, Hkv, ps, r), dtype=pdt, device=device)
         else:
             proxy = torch.zeros((num_pages, Hkv, ps, d // 2), dtype=torch.uint8, device=device)

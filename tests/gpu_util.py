@@ -87,7 +87,7 @@ class Filled:
             codes[:, 1::2] = c >> 4
             return codes, s
         p = self.layer.proxy[pages, g].reshape(npg * 128, -1)[:L]
-        if self.w.proxy_dtype == "f32":
+        if self.w.proxy_dtype in ("f32", "e4m3"):
             return p.cpu().numpy()
         return p.view(torch.int16).cpu().numpy().view(np.uint16)
 

@@ -57,6 +57,9 @@ def test_workspace_size_is_positive_and_monotone():
     (dict(proxy_rank=0), B.QS_ERR_INVALID_ARG),          # rank 0 needs the NVFP4 proxy
     (dict(v_dtype="f16", v_agg_dtype="bf16"), B.QS_ERR_UNSUPPORTED),
     (dict(block_size=1, budget=2048), None),
+    (dict(proxy_dtype="e4m3"), None),                     # FP8 projected keys, r = 32
+    (dict(proxy_dtype="e4m3", proxy_rank=64), None),
+    (dict(proxy_dtype="e4m3", proxy_rank=16), B.QS_ERR_UNSUPPORTED),
 ])
 def test_host_validation(kw, status):
     if status is None:

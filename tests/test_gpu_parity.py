@@ -21,7 +21,8 @@ from tests.util import oracle_row, query_scale_all, row_params
 pytestmark = pytest.mark.gpu
 
 RANKR = [synth.TINY, synth.TINY_NEEDLE] + [synth.small(w) for w in
-                                          (synth.TOKEN32K, synth.BLOCK128K, synth.RAGGED)]
+                                          (synth.TOKEN32K, synth.BLOCK128K, synth.RAGGED,
+                                           synth.FP8_128K, synth.FP8_TOKEN32K)]
 NVFP4 = [synth.small(synth.NVFP4_128K)]
 
 
