@@ -178,7 +178,8 @@ qs_status qs_score(const qs_config *cfg, const qs_cache *cache, const void *q,
    set F (block 0 if force_sink, block nb-1 if force_last, and on the NVFP4 path the
    n_keep_hp complete blocks with the largest block_err, ties to the lower index) is taken
    first; the remaining budget - |F| blocks are the best-scoring others, ties to the lower
-   index. NaN scores rank as the lowest finite value. Output ascending, padded with -1. */
+   index. A NaN or -inf score ranks as -FLT_MAX and +inf as FLT_MAX (ties between them and
+   those values go to the lower index). Output ascending, padded with -1. */
 qs_status qs_select_topk(const qs_config *cfg, const qs_cache *cache,
                          const float *block_scores, int32_t batch, int32_t *sel,
                          int32_t *n_sel, void *ws, qs_stream_t stream);

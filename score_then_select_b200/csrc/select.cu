@@ -9,20 +9,22 @@
 // kept) plus the k - |F| best other blocks by score, equal scores ordered by lower index;
 // ascending.
 //
-// Algorithm, one CTA per row; thread t owns blocks t, t + NT, t + 2 NT, ... in registers
-// (coalesced loads); shared-memory bitmaps restore index order at the end:
-//   1. forced blocks are marked (the kept blocks are the n_keep complete blocks with the
-//      largest block error, found by two block-wide arg-max reductions);
+// Algorithm, one CTA per row. Warp w owns the contiguous blocks w * 32 * ITEMS ..
+// (w + 1) * 32 * ITEMS - 1; lane l holds its blocks l, l + 32, ... in registers, so loads
+// coalesce and index order is (warp, item, lane):
+//   1. the score loads are issued first; forced blocks are marked by their owners (the
+//      kept blocks are the n_keep complete blocks with the largest block error, found by
+//      two block-wide arg-max reductions);
 //   2. one pass of a 2048-bin histogram that is linear in the score between the active
 //      minimum and maximum (a monotone map, so every block in a higher bin scores higher)
 //      selects every bin above the threshold bin and leaves only the threshold bin active;
+//      the bins stay packed in registers for the classification;
 //   3. the few blocks left in the threshold bin are ranked pairwise (score descending,
-//      index ascending) and the first ones taken; only if many are left (many equal or
-//      nearly equal scores) does an exact MSB-first radix select (4 x 8-bit digits) over
-//      order-preserving uint32 keys narrow them to one key value;
-//   4. the remaining slots go to the lowest-indexed blocks holding that key (a scan over
-//      the bitmap of remaining candidates);
-//   5. a scan over the bitmap of chosen blocks writes the ascending indices.
+//      index ascending) and kept by their owners if ranked within the need; only if many
+//      are left (many equal or nearly equal scores) does an exact MSB-first radix select
+//      (4 x 8-bit digits) over order-preserving uint32 keys narrow them to one key value;
+//   4. the remaining slots go to the lowest-indexed blocks holding that key;
+//   5. the ascending indices are written with one ballot per item and a prefix over warps.
 // The count left in the threshold bin is read from the histogram, so no extra block-wide
 // reduction is needed between passes.
 #include <cfloat>
@@ -46,7 +48,7 @@ template <int NT>
 struct BlockOps {
   static constexpr int NW = NT / 32;
   int* s_i;      // [NW + 1]
-  float* s_f;    // [2 * NW]
+  float* s_f;    // [2 * NW + 2]
 
   // exclusive prefix sum over threads; total via *total
   QS_DEV int exclusive_sum(int v, int* total) {
@@ -86,10 +88,15 @@ struct BlockOps {
     hi = warp_max(hi);
     if (lane == 0) { s_f[w] = lo; s_f[NW + w] = hi; }
     __syncthreads();
-    lo = s_f[0];
-    hi = s_f[NW];
-    for (int i = 1; i < NW; ++i) { lo = fminf(lo, s_f[i]); hi = fmaxf(hi, s_f[NW + i]); }
+    if (w == 0) {                                  // warp 0 combines the warps' results
+      float a = lane < NW ? s_f[lane] : FLT_MAX, b = lane < NW ? s_f[NW + lane] : -FLT_MAX;
+      a = warp_min(a);
+      b = warp_max(b);
+      if (lane == 0) { s_f[2 * NW] = a; s_f[2 * NW + 1] = b; }
+    }
     __syncthreads();
+    lo = s_f[2 * NW];
+    hi = s_f[2 * NW + 1];
   }
   // arg-max of (value, -index) over the CTA; returns the index (or -1 if none valid)
   QS_DEV int argmax(float v, int idx) {
@@ -142,29 +149,74 @@ QS_DEV void find_threshold_bin(const int* hist, int nbins, int need, int* s_bin,
   __syncthreads();
 }
 
+// NaN ranks lowest (fmaxf returns the other operand); +-inf are clamped to +-FLT_MAX
+QS_DEV float sanitize(float x) { return fminf(fmaxf(x, -FLT_MAX), FLT_MAX); }
+
+// Exclusive prefix of one value per warp (lane 0's `v`) over the CTA's warps, and the total;
+// every lane of warp w receives the sum over warps 0 .. w-1.
+template <int NW>
+QS_DEV int warp_exclusive(int v, int* s_w, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) s_w[w] = v;
+  __syncthreads();
+  int x = lane < NW ? s_w[lane] : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  const int before = __shfl_sync(kFull, x, w) - __shfl_sync(kFull, lane < NW ? s_w[lane] : 0, w);
+  *total = __shfl_sync(kFull, x, NW - 1);
+  __syncthreads();
+  return before;
+}
+
+// Transpose of a 32 x 32 bit matrix held one row per lane (bit c of lane r = M[r][c]): lane
+// c receives column c (bit r = M[r][c]). Five rounds swap the off-diagonal j x j blocks.
+QS_DEV uint32_t transpose32(uint32_t x, int lane) {
+  const uint32_t hi[5] = {0xFFFF0000u, 0xFF00FF00u, 0xF0F0F0F0u, 0xCCCCCCCCu, 0xAAAAAAAAu};
+#pragma unroll
+  for (int t = 0; t < 5; ++t) {
+    const int j = 16 >> t;
+    const uint32_t y = __shfl_xor_sync(kFull, x, j);
+    // the row with bit j set keeps its right half and takes its partner's right half into
+    // its left half; the other keeps its left half and takes the partner's left half
+    x = (lane & j) ? ((x & hi[t]) | ((y & hi[t]) >> j)) : ((x & ~hi[t]) | ((y & ~hi[t]) << j));
+  }
+  return x;
+}
+
 template <int NT, int ITEMS>
 __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   constexpr int NW = NT / 32;
   constexpr int CAP = NT * ITEMS;                 // blocks one CTA can hold
-  constexpr int NWORDS = CAP / 32;                // bitmap words
-  constexpr int WPT = (NWORDS + NT - 1) / NT;     // bitmap words per thread (contiguous)
+  constexpr int SPAN = 32 * ITEMS;                // blocks of one warp (contiguous)
   __shared__ int s_i[NW + 1];
-  __shared__ float s_f[2 * NW];
+  __shared__ float s_f[2 * NW + 2];
   __shared__ int hist[kLinBins];
-  __shared__ uint32_t chosen_bits[NWORDS], active_bits[NWORDS];
   __shared__ float list_v[kRankCap];
   __shared__ int list_j[kRankCap];
   __shared__ int s_bin, s_above, s_cnt, s_forced[4], s_nforced;
+  __shared__ uint32_t s_out[NW * 64];
   BlockOps<NT> ops{s_i, s_f};
 
   pdl_wait();      // the scores come from the kernel before
   pdl_trigger();
   const int row = blockIdx.x;
   const int b = row / a.Hkv;
-  const int tid = threadIdx.x;
-  int L = a.seq_lens[b];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // item i of this thread is block j = warp * SPAN + i * 32 + lane: each warp owns a
+  // contiguous range (index order = warp, then item, then lane) and its loads coalesce
+  const int jw = warp * SPAN + lane;
+  const float* sc = a.scores + size_t(row) * a.nb_stride;
   const int nb_cap = a.nb_stride < CAP ? a.nb_stride : CAP;
-  int nb = (L + a.S - 1) / a.S;
+  // the loads are issued before the row length arrives: every entry of the row's stride is
+  // readable, and blocks at or past nb are masked out below
+  float v[ITEMS];
+#pragma unroll
+  for (int i = 0; i < ITEMS; ++i) v[i] = (jw + i * 32 < nb_cap) ? sc[jw + i * 32] : -FLT_MAX;
+  int L = a.seq_lens[b];
+  int nb = int((static_cast<long long>(L) + a.S - 1) / a.S);
   if (L < 0 || nb > nb_cap) {
     if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
     nb = L < 0 ? 0 : nb_cap;
@@ -179,16 +231,6 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     for (int i = tid; i < k; i += NT) sel[i] = i < nb ? i : -1;
     return;
   }
-
-  // item i of this thread is block j = i * NT + tid (coalesced loads)
-  const float* sc = a.scores + size_t(row) * a.nb_stride;
-  float v[ITEMS];
-#pragma unroll
-  for (int i = 0; i < ITEMS; ++i) {
-    const int j = i * NT + tid;
-    v[i] = j < nb ? sc[j] : -FLT_MAX;
-  }
-  for (int w = tid; w < NWORDS; w += NT) chosen_bits[w] = active_bits[w] = 0u;
 
   // ---------------- forced blocks: sink, last, and the kept (largest-error) blocks
   if (a.n_keep > 0 && a.block_err != nullptr) {
@@ -225,22 +267,24 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     }
     s_nforced = n;
   }
-  __syncthreads();
-  int need = k - s_nforced;
   uint32_t active = 0u, chosen = 0u;
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) {
-    const int j = i * NT + tid;
-    if (j < nb) {
-      bool f = false;
+    if (jw + i * 32 < nb) active |= 1u << i;
+    v[i] = sanitize(v[i]);
+  }
+  __syncthreads();
+  // each forced block moves from active to chosen in the thread that owns it
 #pragma unroll
-      for (int q = 0; q < 4; ++q) f |= (s_forced[q] == j);
-      if (f) chosen |= 1u << i; else active |= 1u << i;
-      float x = v[i];
-      if (x != x) x = -FLT_MAX;                      // NaN ranks lowest
-      v[i] = fminf(fmaxf(x, -FLT_MAX), FLT_MAX);
+  for (int q = 0; q < 4; ++q) {
+    const int f = s_forced[q];
+    if (f >= 0 && f / SPAN == warp && (f & 31) == lane) {
+      const int i = (f % SPAN) >> 5;
+      chosen |= 1u << i;
+      active &= ~(1u << i);
     }
   }
+  int need = k - s_nforced;
   int n_active = nb - s_nforced;                     // known exactly: no reduction needed
 
   // ---------------- linear-bin pass: everything above the threshold bin is chosen
@@ -253,27 +297,29 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     if (hi > lo) {
       for (int i = tid; i < kLinBins; i += NT) hist[i] = 0;
       __syncthreads();
-      // bin = trunc((x - lo) * scale): a rounded subtraction, a rounded product by a
-      // positive constant and a truncation are each monotone, so a higher bin always holds
-      // higher scores (recomputed below rather than kept, to stay within the 64 registers
-      // of a 1024-thread CTA); an overflowing range saturates and only coarsens the bins
-      const float scale = float(kLinBins) / (hi - lo);
-      auto bin_of = [&](float x) {
-        const int bn = __float2int_rz((x - lo) * scale);
-        return bn < 0 ? 0 : (bn >= kLinBins ? kLinBins - 1 : bn);
-      };
+      // bin = nearest integer to fma(x, scale, -lo * scale), clamped to the last bin: a
+      // correctly rounded FMA with a positive scale, rounding to an integer (adding
+      // 1.5 * 2^23) and a clamp are each monotone, so a higher bin always holds higher
+      // scores. An overflowing range saturates and only coarsens the bins.
+      const float scale = float(kLinBins - 1) / (hi - lo);
+      const float off = -lo * scale;
+      uint32_t bins[(ITEMS + 1) / 2];                // two 16-bit bins per word
 #pragma unroll
-      for (int i = 0; i < ITEMS; ++i)
-        if (active >> i & 1u) atomicAdd(&hist[bin_of(v[i])], 1);
+      for (int i = 0; i < ITEMS; ++i) {
+        int bn = __float_as_int(__fadd_rn(__fmaf_rn(v[i], scale, off), 12582912.0f)) - 0x4B400000;
+        bn = bn < 0 ? 0 : (bn >= kLinBins ? kLinBins - 1 : bn);
+        if (i % 2 == 0) bins[i / 2] = uint32_t(bn); else bins[i / 2] |= uint32_t(bn) << 16;
+        if (active >> i & 1u) atomicAdd(&hist[bn], 1);
+      }
       __syncthreads();
       find_threshold_bin<NT>(hist, kLinBins, need, &s_bin, &s_above, ops);
-      const int bstar = s_bin;
+      const uint32_t bstar = uint32_t(s_bin);
       const int above = s_above;
       const int cnt = hist[bstar];
 #pragma unroll
       for (int i = 0; i < ITEMS; ++i) {
+        const uint32_t bn = (bins[i / 2] >> (16 * (i % 2))) & 0xFFFFu;
         if (!(active >> i & 1u)) continue;
-        const int bn = bin_of(v[i]);
         if (bn > bstar) { chosen |= 1u << i; active &= ~(1u << i); }
         else if (bn < bstar) active &= ~(1u << i);
       }
@@ -284,29 +330,42 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   }
 
   // ---------------- few candidates left (the usual case): rank them all pairwise under the
-  // order (higher score, then lower index) and keep the first `need`
+  // order (higher score, then lower index); each candidate's owner keeps it if its rank is
+  // below `need`
   if (need > 0 && n_active > need && n_active <= kRankCap) {
     if (tid == 0) s_cnt = 0;
     __syncthreads();
+    // one shared-memory atomic per warp reserves the warp's slots
+    const int my = __popc(active);
+    int incl = my;
 #pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      if (active >> i & 1u) {
-        const int slot = atomicAdd(&s_cnt, 1);
-        list_v[slot] = v[i];
-        list_j[slot] = i * NT + tid;
-      }
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int base = 0;
+    if (lane == 31 && incl > 0) base = atomicAdd(&s_cnt, incl);
+    int slot = __shfl_sync(kFull, base, 31) + incl - my;
+    // (scores are re-read from the row's buffer: the registers now hold the packed bins;
+    // loops over this thread's few candidates, not over all items, keep the code small)
+    for (uint32_t bits = active; bits != 0u; bits &= bits - 1u) {
+      const int jc = jw + (__ffs(bits) - 1) * 32;
+      list_v[slot] = sanitize(sc[jc]);
+      list_j[slot] = jc;
+      ++slot;
     }
     __syncthreads();
     const int n = s_cnt;
-    for (int c = tid; c < n; c += NT) {
-      const float vc = list_v[c];
-      const int jc = list_j[c];
+    for (uint32_t bits = active; bits != 0u; bits &= bits - 1u) {
+      const int i = __ffs(bits) - 1;
+      const int jc = jw + i * 32;
+      const float vc = sanitize(sc[jc]);
       int rank = 0;
       for (int o = 0; o < n; ++o) {
         const float vo = list_v[o];
         rank += (vo > vc) || (vo == vc && list_j[o] < jc);
       }
-      if (rank < need) atomicOr(&chosen_bits[jc >> 5], 1u << (jc & 31));
+      if (rank < need) chosen |= 1u << i;
     }
     need = 0;
     active = 0u;
@@ -319,7 +378,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < ITEMS; ++i)
-      if (active >> i & 1u) atomicAdd(&hist[(order_key(v[i]) >> shift) & 255u], 1);
+      if (active >> i & 1u) atomicAdd(&hist[(order_key(sanitize(sc[jw + i * 32])) >> shift) & 255u], 1);
     __syncthreads();
     find_threshold_bin<NT>(hist, 256, need, &s_bin, &s_above, ops);
     const uint32_t dstar = uint32_t(s_bin);
@@ -328,7 +387,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
 #pragma unroll
     for (int i = 0; i < ITEMS; ++i) {
       if (!(active >> i & 1u)) continue;
-      const uint32_t dg = (order_key(v[i]) >> shift) & 255u;
+      const uint32_t dg = (order_key(sanitize(sc[jw + i * 32])) >> shift) & 255u;
       if (dg > dstar) { chosen |= 1u << i; active &= ~(1u << i); }
       else if (dg < dstar) active &= ~(1u << i);
     }
@@ -337,52 +396,41 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
     __syncthreads();
   }
 
-  // ---------------- index order: chosen blocks, plus the `need` lowest-indexed actives
-#pragma unroll
-  for (int i = 0; i < ITEMS; ++i) {
-    const int j = i * NT + tid;
-    if (chosen >> i & 1u) atomicOr(&chosen_bits[j >> 5], 1u << (j & 31));
-    if (need > 0 && (active >> i & 1u)) atomicOr(&active_bits[j >> 5], 1u << (j & 31));
-  }
-  __syncthreads();
-  const int w0 = tid * WPT;
+  // ---------------- remaining slots: the lowest-indexed actives (they share one key)
   if (need > 0) {
-    // remaining actives share one key (or exactly fill the need): lowest indices first
-    int cnt = 0;
-#pragma unroll
-    for (int w = 0; w < WPT; ++w)
-      if (w0 + w < NWORDS) cnt += __popc(active_bits[w0 + w]);
+    int wcnt = 0;
+#pragma unroll 1
+    for (int i = 0; i < ITEMS; ++i) wcnt += __popc(__ballot_sync(kFull, active >> i & 1u));
     int tot;
-    int before = ops.exclusive_sum(cnt, &tot);
-#pragma unroll
-    for (int w = 0; w < WPT; ++w) {
-      if (w0 + w >= NWORDS) break;
-      uint32_t bits = active_bits[w0 + w];
-      while (bits != 0u && before < need) {
-        const uint32_t low = bits & (~bits + 1u);
-        chosen_bits[w0 + w] |= low;
-        bits ^= low;
-        ++before;
-      }
+    int before = warp_exclusive<NW>(wcnt, s_i, &tot);
+#pragma unroll 1
+    for (int i = 0; i < ITEMS; ++i) {
+      const uint32_t m = __ballot_sync(kFull, active >> i & 1u);
+      if ((active >> i & 1u) && before + __popc(m & ((1u << lane) - 1u)) < need) chosen |= 1u << i;
+      before += __popc(m);
     }
-    __syncthreads();
   }
-  int cnt = 0;
+
+  // ---------------- ascending output: warp ranges in order, items in order, lanes in order.
+  // Transposing the warp's 32 x 32 bit matrix (lane = row, item = column) gives lane i the
+  // mask of lanes that chose item i; a scan of their counts over the lanes places every item.
+  uint32_t tr = transpose32(chosen, lane);
+  const int cnt_i = __popc(tr);
+  int incl = cnt_i;
 #pragma unroll
-  for (int w = 0; w < WPT; ++w)
-    if (w0 + w < NWORDS) cnt += __popc(chosen_bits[w0 + w]);
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t* s_tr = s_out + warp * 64;                  // [lane masks of item i, items before i]
+  s_tr[lane] = tr;
+  s_tr[32 + lane] = uint32_t(incl - cnt_i);
   int tot;
-  int pos = ops.exclusive_sum(cnt, &tot);
-#pragma unroll
-  for (int w = 0; w < WPT; ++w) {
-    if (w0 + w >= NWORDS) break;
-    uint32_t bits = chosen_bits[w0 + w];
-    while (bits != 0u) {
-      const int bit = __ffs(bits) - 1;
-      if (pos < k) sel[pos] = (w0 + w) * 32 + bit;
-      ++pos;
-      bits &= bits - 1u;
-    }
+  const int pos = warp_exclusive<NW>(__shfl_sync(kFull, incl, 31), s_i, &tot);  // syncs the CTA
+  for (uint32_t bits = chosen; bits != 0u; bits &= bits - 1u) {
+    const int i = __ffs(bits) - 1;
+    const int p = pos + int(s_tr[32 + i]) + __popc(s_tr[i] & ((1u << lane) - 1u));
+    if (p < k) sel[p] = jw + i * 32;
   }
   if (tot != n_out && tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
   for (int i = tot + tid; i < k; i += NT) sel[i] = -1;
