@@ -245,6 +245,50 @@ def lse_combine(ms, ls, os_) -> np.ndarray:
 
 
 # ============================================================================================
+# JSSA-style basis from calibration moments  [JSSA, Abstract; Table 9]
+# The pages learn the shared subspace by minimising a tractable (marginal) bound on the
+# token-score preservation error, with a closed-form spectral solution, and compare raw
+# with unit-trace-normalised group-mean moments (Table 9). The bound itself is not on the
+# pages. Reading: P = the top-r eigenvectors of M = C_q / tr(C_q) + C_k / tr(C_k), with
+# C_q the second moment of the calibration group-mean queries and C_k that of the keys
+# (each normalised to unit trace, so neither side dominates by scale). PARITY UNPINNED as
+# a reading of the pages; the spectral solution of this definition is pinned.
+# ============================================================================================
+
+
+def calibration_moment(q_bits: np.ndarray, k_bits: np.ndarray) -> np.ndarray:
+    """M = C_q / tr(C_q) + C_k / tr(C_k) for one KV head (float64).
+
+    q_bits: BF16 calibration queries [n][G][d] (the group's heads), k_bits: BF16 keys [m][d].
+    C_q = mean over positions of qbar qbar^T, qbar = mean of the group's heads; C_k likewise.
+    """
+    qbar = F.bf16_to_f64(q_bits).mean(axis=1)
+    k = F.bf16_to_f64(k_bits)
+    cq = qbar.T @ qbar / qbar.shape[0]
+    ck = k.T @ k / k.shape[0]
+    return cq / np.trace(cq) + ck / np.trace(ck)
+
+
+def spectral_basis(Mx: np.ndarray, r: int):
+    """Top-r eigenvectors of the symmetric Mx as columns of P [d][r] (eigenvalue descending),
+    each signed so that its largest-magnitude entry (lowest index on ties) is positive;
+    returns (P, eigenvalues[:r])."""
+    w, V = np.linalg.eigh(Mx)
+    order = np.argsort(-w, kind="stable")[:r]
+    P = V[:, order].copy()
+    for c in range(r):
+        i = int(np.argmax(np.abs(P[:, c])))
+        if P[i, c] < 0:
+            P[:, c] = -P[:, c]
+    return P, w[order]
+
+
+def jssa_basis(q_bits: np.ndarray, k_bits: np.ndarray, r: int):
+    """The basis of one KV head: spectral_basis(calibration_moment(q, k), r)."""
+    return spectral_basis(calibration_moment(q_bits, k_bits), r)
+
+
+# ============================================================================================
 # Full-KV attention and gather-then-attend  [JSSA, Figure 2 (b); Figure 6 (a)]
 # The pages compare the sparse attention stage with attention over the whole cache
 # (full-KV) and with a variant that first copies the selected tokens into a contiguous

@@ -319,3 +319,85 @@ def test_e4m3_proxy_store_rounds_the_float32_projection():
     normal = np.abs(f32) >= 2.0 ** -6
     assert np.all(np.abs(dec - f32)[normal] <= np.abs(f32)[normal] * 2.0 ** -4)
     assert np.all(np.abs(dec - f32)[~normal] <= 2.0 ** -10)
+
+
+# ---------------------------------------------------------------- JSSA-style basis (spectral)
+
+def _bf(x):
+    return F.f32_to_bf16_rne(np.asarray(x, dtype=np.float32))
+
+
+def test_basis_diagonal_moments_pick_coordinate_axes():
+    # independent coordinates with distinct variances: the basis is the axes of the r
+    # largest normalised variances, in that order, each with entry +1
+    rng = np.random.default_rng(40)
+    d, r, n = 16, 4, 4096
+    sq = np.linspace(1.0, 4.0, d)[rng.permutation(d)]
+    sk = np.linspace(0.5, 2.0, d)[rng.permutation(d)]
+    # sign-randomised columns with exact per-coordinate energy (a Hadamard-like design)
+    signs = rng.choice([-1.0, 1.0], size=(n, d))
+    q = _bf((signs * sq)[:, None, :] * np.ones((1, 2, 1)))
+    k = _bf(rng.choice([-1.0, 1.0], size=(n, d)) * sk)
+    Mx = M.calibration_moment(q, k)
+    # the diagonal is exactly the normalised energies of the coordinates
+    eq, ek = np.array(sq, dtype=np.float64) ** 2, np.array(sk, dtype=np.float64) ** 2
+    assert np.allclose(np.diag(Mx), eq / eq.sum() + ek / ek.sum(), rtol=1e-2)
+    P, w = M.spectral_basis(np.diag(np.diag(Mx)), r)
+    want_axes = np.argsort(-np.diag(Mx), kind="stable")[:r]
+    assert np.array_equal(np.argmax(np.abs(P), axis=0), want_axes)
+    assert np.allclose(np.abs(P).max(axis=0), 1.0) and np.all(P.max(axis=0) > 0)
+
+
+def test_basis_recovers_a_shared_subspace():
+    # queries and keys confined to span(U): the basis spans U exactly
+    rng = np.random.default_rng(41)
+    d, r, n = 32, 6, 2000
+    U = np.linalg.qr(rng.standard_normal((d, r)))[0]
+    q = _bf((rng.standard_normal((n, 3, r)) * np.array([5, 4, 3, 2, 1.5, 1.0])) @ U.T)
+    k = _bf((rng.standard_normal((n, r)) * np.array([1, 2, 3, 4, 5, 6])) @ U.T)
+    P, w = M.jssa_basis(q, k, r)
+    # BF16 rounding adds a small component outside span(U)
+    assert np.linalg.norm(P - U @ (U.T @ P)) < 0.02
+    assert np.allclose(P.T @ P, np.eye(r), atol=1e-12)
+
+
+def test_basis_unit_trace_normalisation():
+    # scaling all queries (or all keys) by a power of two changes neither M nor P
+    rng = np.random.default_rng(42)
+    d, r, n = 24, 5, 1500
+    A = rng.standard_normal((d, d))
+    q = _bf(rng.standard_normal((n, 2, d)) @ A.T)
+    k = _bf(rng.standard_normal((n, d)) @ np.diag(np.linspace(0.2, 3, d)))
+    P0, w0 = M.jssa_basis(q, k, r)
+    qs = _bf(F.bf16_to_f64(q) * 64.0)
+    ks = _bf(F.bf16_to_f64(k) * 2.0 ** -5)
+    P1, w1 = M.jssa_basis(qs, ks, r)
+    assert np.allclose(M.calibration_moment(q, k), M.calibration_moment(qs, ks), atol=1e-13)
+    assert np.allclose(P0, P1, atol=1e-10) and np.allclose(w0, w1, atol=1e-13)
+
+
+def test_basis_normalisation_balances_queries_and_keys():
+    # keys 1000x larger than queries: raw moments would follow the keys alone; the
+    # normalised moment weighs both, so the query direction stays in the basis
+    rng = np.random.default_rng(43)
+    d, n = 8, 4000
+    e = np.eye(d)
+    q = _bf((rng.standard_normal((n, 1, 1)) * 3.0) * e[0][None, None, :])     # queries along e0
+    k = _bf(rng.standard_normal((n, 2)) * 1000.0 @ e[[1, 2]])                  # keys along e1, e2
+    P, w = M.jssa_basis(q, k, 1)
+    assert np.argmax(np.abs(P[:, 0])) == 0 and abs(P[0, 0] - 1.0) < 1e-12
+    assert abs(w[0] - 1.0) < 1e-12                                             # tr-normalised
+
+
+def test_basis_is_rotation_equivariant():
+    rng = np.random.default_rng(44)
+    d, r, n = 16, 4, 3000
+    Q = rng.standard_normal((n, 2, d)) * np.linspace(3, 0.5, d)
+    K = rng.standard_normal((n, d)) * np.linspace(0.5, 2, d)[::-1]
+    R = np.linalg.qr(rng.standard_normal((d, d)))[0]
+    P0, w0 = M.spectral_basis(M.calibration_moment(_bf(Q), _bf(K)), r)
+    # rotating the exact moment (not the rounded inputs) rotates the eigenvectors
+    Mx = M.calibration_moment(_bf(Q), _bf(K))
+    P1, w1 = M.spectral_basis(R @ Mx @ R.T, r)
+    assert np.allclose(w0, w1, atol=1e-12)
+    assert np.allclose(np.abs((R @ P0).T @ P1), np.eye(r), atol=1e-8)
