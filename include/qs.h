@@ -244,6 +244,30 @@ qs_status qs_gather_kv(const qs_config *cfg, const qs_cache *cache, const int32_
                        const int32_t *n_sel, int32_t batch, void *k_dst, void *v_dst,
                        int32_t *row_lens, void *ws, qs_stream_t stream);
 
+/* ---- Calibration of the scoring basis (once, before decoding) ----------------------------
+   "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Abstract and
+   Table 9: the shared subspace minimises a tractable bound on the token-score preservation
+   error with a spectral solution, and unit-trace-normalised group-mean moments are
+   compared with raw ones. The bound is not on the pages; the reading built here is
+     M = C_q / tr(C_q) + C_k / tr(C_k)   (per KV head),
+     C_q = mean over positions of qbar qbar^T, qbar = mean of the group's query heads,
+     C_k = mean over positions of k k^T,
+     P = the r eigenvectors of M with the largest eigenvalues, descending, each column
+         signed so that its largest-magnitude entry (lowest index on ties) is positive.
+   Moments are summed in FP64; the eigenvectors come from a cyclic Jacobi iteration on M in
+   FP64 with the rotations accumulated in FP32 (one CTA per KV head). */
+
+/* Workspace bytes for qs_calibrate_basis (host only): 256 + 2 * Hkv * d * d * 8. */
+qs_status qs_calib_workspace_size(const qs_config *cfg, size_t *bytes /* host */);
+
+/* Compute P [Hkv][d][r] (FP32, the layout qs_append_kv and qs_score take) from n calibration
+   positions: q [n][Hq][d] BF16 queries and k [n][Hkv][d] BF16 keys. eigvals [Hkv][r] (FP32,
+   may be NULL) receives the eigenvalues of M in the same order. r = cfg->proxy_rank (> 0,
+   else QS_ERR_UNSUPPORTED). ws: qs_calib_workspace_size bytes, 256-byte aligned (no
+   initialisation needed). Two launches; asynchronous on stream. */
+qs_status qs_calibrate_basis(const qs_config *cfg, const void *q, const void *k, int32_t n,
+                             float *P, float *eigvals, void *ws, qs_stream_t stream);
+
 /* Synchronise `stream`, return the first device-side error recorded in the workspace
    since the last call (QS_OK if none) and clear it. `detail` (HOST pointer, may be NULL)
    receives {kernel id, index} of that error. Returns QS_ERR_CUDA if the synchronisation

@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
             "qs_dense_workspace_size": ([cfgp, i32, i32, ctypes.POINTER(sz)], i32),
             "qs_dense_attn": ([cfgp, cachep, vp, vp, i32, vp, vp, vp], i32),
             "qs_gather_kv": ([cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp], i32),
+            "qs_calib_workspace_size": ([cfgp, ctypes.POINTER(sz)], i32),
+            "qs_calibrate_basis": ([cfgp, vp, vp, i32, vp, vp, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -85,7 +87,7 @@ EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_
            "qs_append_kv", "qs_score", "qs_select_topk", "qs_sparse_attn", "qs_decode",
            "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches",
            "qs_selftest_wait_timeout", "qs_dense_workspace_size", "qs_dense_attn",
-           "qs_gather_kv")
+           "qs_gather_kv", "qs_calib_workspace_size", "qs_calibrate_basis")
 
 
 def status_string(s: int) -> str:
@@ -229,6 +231,19 @@ def qs_gather_kv(cfg, cache, sel, n_sel, batch, k_dst, v_dst, row_lens, ws, stre
     _check(lib().qs_gather_kv(ctypes.byref(cfg), ctypes.byref(cache), _ptr(sel), _ptr(n_sel),
                               batch, _ptr(k_dst), _ptr(v_dst), _ptr(row_lens), _ptr(ws),
                               _stream(stream)), "qs_gather_kv")
+
+
+def qs_calib_workspace_size(cfg: qs_config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().qs_calib_workspace_size(ctypes.byref(cfg), ctypes.byref(n)),
+           "qs_calib_workspace_size")
+    return n.value
+
+
+def qs_calibrate_basis(cfg, q, k, n, P, eigvals, ws, stream=None):
+    _check(lib().qs_calibrate_basis(ctypes.byref(cfg), _ptr(q), _ptr(k), n, _ptr(P),
+                                    _ptr(eigvals), _ptr(ws), _stream(stream)),
+           "qs_calibrate_basis")
 
 
 def qs_device_status(ws, stream=None) -> tuple[int, int, int]:

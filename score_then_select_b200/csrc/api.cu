@@ -488,6 +488,38 @@ qs_status qs_gather_kv(const qs_config* cfg, const qs_cache* cache, const int32_
   return cuda_status(launch_gather_kv(p, a, stream));
 }
 
+qs_status qs_calib_workspace_size(const qs_config* cfg, size_t* bytes) {
+  Plan p;
+  const qs_status st = make_plan(cfg, 1, 1, p);
+  if (st != QS_OK) return st;
+  if (!bytes) return QS_ERR_INVALID_ARG;
+  if (p.r <= 0) return QS_ERR_UNSUPPORTED;
+  *bytes = calib_ws_bytes(p.Hkv, p.d);
+  return QS_OK;
+}
+
+qs_status qs_calibrate_basis(const qs_config* cfg, const void* q, const void* k, int32_t n,
+                             float* P, float* eigvals, void* ws, qs_stream_t stream) {
+  Plan p;
+  const qs_status st = make_plan(cfg, 1, 1, p);
+  if (st != QS_OK) return st;
+  if (p.r <= 0) return QS_ERR_UNSUPPORTED;
+  if (!q || !k || n < 1 || !P || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  CalibParams a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.mq = ws_at<double>(ws, size_t(kHdrWords) * 4);
+  a.mk = a.mq + size_t(p.Hkv) * p.d * p.d;
+  a.P = P;
+  a.eig = eigvals;
+  a.n = n;
+  a.Hkv = p.Hkv;
+  a.G = p.G;
+  a.d = p.d;
+  a.r = p.r;
+  return cuda_status(launch_calibrate(a, stream));
+}
+
 qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, const void* k_new,
                     const void* v_new, const float* P, int32_t batch, void* out, int32_t* sel_out,
                     int32_t* n_sel_out, void* ws, qs_stream_t stream) {

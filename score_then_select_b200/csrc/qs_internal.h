@@ -206,6 +206,16 @@ struct GatherParams {        // gather-then-attend: selected blocks -> compact p
   int rows, Hkv, log2_S, budget, dst_pages_per_seq, max_pages_per_seq, num_pages;
 };
 
+struct CalibParams {        // calibration of the scoring basis (calib.cu)
+  const uint16_t* q;         // [n][Hq][d] BF16
+  const uint16_t* k;         // [n][Hkv][d] BF16
+  double* mq;                // [Hkv][d][d] sum of qbar qbar^T
+  double* mk;                // [Hkv][d][d] sum of k k^T
+  float* P;                  // [Hkv][d][r]
+  float* eig;                // [Hkv][r] or nullptr
+  int n, Hkv, G, d, r;
+};
+
 // Launch `kern` on `s`; with `pdl` the launch may overlap the tail of the previous kernel
 // in the stream (the kernel must call pdl_wait() before reading that kernel's results).
 template <typename... P, typename... A>
@@ -234,6 +244,8 @@ cudaError_t launch_select(const Plan& p, const SelectParams& a, cudaStream_t s, 
 cudaError_t launch_attn_gather(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_attn(const Plan& p, const AttnParams& a, cudaStream_t s, bool pdl);
 cudaError_t launch_gather_kv(const Plan& p, const GatherParams& a, cudaStream_t s);
+cudaError_t launch_calibrate(const CalibParams& a, cudaStream_t s);
+size_t calib_ws_bytes(int Hkv, int d);
 
 int num_sms();
 
