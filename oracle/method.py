@@ -245,6 +245,36 @@ def lse_combine(ms, ls, os_) -> np.ndarray:
 
 
 # ============================================================================================
+# Centroid scoring of contiguous blocks  ["Coarse Semantic Blocks ...", Abstract]
+# The page scores each block by its centroid against the query. Reading: the centroid of a
+# block is the mean of its valid stored keys, kept as a float32 running sum in token order
+# (the cache entry) and divided by the block's valid count when scoring; the block score is
+# the group-mean query dotted with it, which equals the mean of the block's exact
+# group-mean scores. Blocks stay contiguous (the semantic, non-contiguous clustering of
+# the page is not built).
+# ============================================================================================
+
+
+def centroid_sums(k_bits: np.ndarray, S: int, L: int) -> np.ndarray:
+    """float32 sums of the valid keys of each block, added in token order -> [nb][d]."""
+    k32 = F.bf16_to_f64(k_bits[:L]).astype(np.float32)
+    nb = -(-L // S)
+    out = np.zeros((nb, k32.shape[1]), dtype=np.float32)
+    for t in range(L):
+        j = t // S
+        out[j] = k32[t] if t % S == 0 else (out[j] + k32[t])   # one float32 rounding per add
+    return out
+
+
+def centroid_block_scores(q_bits: np.ndarray, sums: np.ndarray, S: int, L: int) -> np.ndarray:
+    """beta_j = qbar . (sum_j / count_j) in float64, count_j = valid tokens of block j."""
+    qbar = F.bf16_to_f64(q_bits).mean(axis=0)
+    nb = sums.shape[0]
+    cnt = np.minimum(S, L - np.arange(nb) * S).astype(np.float64)
+    return (sums.astype(np.float64) @ qbar) / cnt
+
+
+# ============================================================================================
 # JSSA-style basis from calibration moments  [JSSA, Abstract; Table 9]
 # The pages learn the shared subspace by minimising a tractable (marginal) bound on the
 # token-score preservation error, with a closed-form spectral solution, and compare raw

@@ -26,7 +26,7 @@ class RowParams:
     S: int                     # block size
     budget: int                # k, blocks
     scale: float               # softmax scale
-    proxy: str                 # 'f32' | 'bf16' | 'nvfp4'
+    proxy: str                 # 'f32' | 'bf16' | 'e4m3' | 'nvfp4' | 'centroid'
     v_dtype: str               # 'bf16' | 'f16'
     force_sink: bool = False
     force_last: bool = False
@@ -38,7 +38,10 @@ def decode_v(v_bits: np.ndarray, v_dtype: str) -> np.ndarray:
 
 
 def row_scoring_cache(p: RowParams, k_bits, P=None, mu=None, g_k=None):
-    """The row's stored scoring cache: proxy entries, or (codes, scales, x32) for NVFP4."""
+    """The row's stored scoring cache: proxy entries, (codes, scales, x32) for NVFP4, or the
+    per-block key sums for centroid scoring."""
+    if p.proxy == "centroid":
+        return M.centroid_sums(k_bits, p.S, len(k_bits))
     if p.proxy == "nvfp4":
         x32 = M.centre(k_bits, mu)
         codes, scales = M.nvfp4_pack(x32, g_k)
@@ -49,6 +52,8 @@ def row_scoring_cache(p: RowParams, k_bits, P=None, mu=None, g_k=None):
 def row_block_scores(p: RowParams, cache, q_bits, L: int, P=None, g_q=None, g_k=None,
                      q_all_bits=None):
     """beta [nb] for one row from its scoring cache."""
+    if p.proxy == "centroid":
+        return M.centroid_block_scores(q_bits, cache[:-(-L // p.S)], p.S, L)
     if p.proxy == "nvfp4":
         codes, scales, _ = cache
         qx = F.bf16_to_f64(q_bits).astype(np.float32)

@@ -26,7 +26,7 @@ class Workload:
     block_size: int              # S
     budget: int                  # k, in blocks
     proxy_rank: int              # r > 0: projected-key proxy; 0: NVFP4 centred keys
-    proxy_dtype: str             # 'f32' | 'bf16' | 'e4m3' | 'nvfp4'
+    proxy_dtype: str             # 'f32' | 'bf16' | 'e4m3' | 'nvfp4' | 'centroid'
     v_dtype: str                 # stored V: 'bf16' | 'f16'
     v_agg_dtype: str             # PV operand precision: 'bf16' | 'f16'
     out_dtype: str               # 'f32' | 'bf16'
@@ -106,6 +106,14 @@ FP8_128K = BLOCK128K.replace(name="fp8_b16_h40kv8_d128_L131072_S128_k64_r32", pr
 FP8_TOKEN32K = TOKEN32K.replace(name="fp8_token_b16_h32kv8_d128_L32768_r64_B2048",
                                 proxy_rank=64, proxy_dtype="e4m3", seed=1007)
 
+# Centroid scoring ("Coarse Semantic Blocks ...", Abstract): each block scored by the mean
+# of its keys against the group-mean query, from per-block FP32 key sums (no projection).
+CENTROID_128K = BLOCK128K.replace(name="centroid_b16_h40kv8_d128_L131072_S128_k64",
+                                  proxy_rank=0, proxy_dtype="centroid", seed=1008)
+# The same with 32-token blocks (four centroids per page), k = 256 blocks.
+CENTROID_S32 = BLOCK128K.replace(name="centroid_b16_h40kv8_d128_L131072_S32_k256", block_size=32,
+                                 budget=256, proxy_rank=0, proxy_dtype="centroid", seed=1009)
+
 # Ragged batch: 32 sequences, lengths uniform in [4096, 131072], G = 8, r = 64, S = 64.
 RAGGED = Workload(
     name="ragged_b32_h64kv8_d128_S64_k32_r64", batch=32, n_q_heads=64, n_kv_heads=8,
@@ -116,8 +124,8 @@ RAGGED = Workload(
 
 FULL = {w.name: w for w in (TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED)}
 ORDER = [TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED]
-# variants of the configurations above (the FP8 projected-key cache)
-VARIANTS = [FP8_128K, FP8_TOKEN32K]
+# variants of the configurations above (FP8 projected keys, centroid scoring)
+VARIANTS = [FP8_128K, FP8_TOKEN32K, CENTROID_128K, CENTROID_S32]
 
 
 def small(w: Workload) -> Workload:

@@ -401,3 +401,37 @@ def test_basis_is_rotation_equivariant():
     P1, w1 = M.spectral_basis(R @ Mx @ R.T, r)
     assert np.allclose(w0, w1, atol=1e-12)
     assert np.allclose(np.abs((R @ P0).T @ P1), np.eye(r), atol=1e-8)
+
+
+# ---------------------------------------------------------------- centroid scoring
+
+def test_centroid_score_is_the_mean_token_score():
+    # linearity: qbar . mean(k) = mean(qbar . k) over the block's valid tokens
+    rng = np.random.default_rng(50)
+    G, d, S, L = 3, 16, 8, 45                    # 6 blocks, the last holds 5 tokens
+    kb = _bf(rng.standard_normal((L, d)))
+    qb = _bf(rng.standard_normal((G, d)))
+    sums = M.centroid_sums(kb, S, L)
+    beta = M.centroid_block_scores(qb, sums, S, L)
+    qbar = F.bf16_to_f64(qb).mean(axis=0)
+    tok = F.bf16_to_f64(kb) @ qbar
+    want = np.array([tok[j * S:min(L, (j + 1) * S)].mean() for j in range(6)])
+    assert np.allclose(beta, want, rtol=1e-6, atol=1e-6)
+
+
+def test_centroid_sums_in_token_order():
+    # hand case in float32: a block's sum restarts at its first token; exact for small ints
+    k = _bf(np.array([[1.0, -2.0], [3.0, 0.5], [4.0, 4.0], [-1.0, 1.0], [2.0, 2.0]]))
+    sums = M.centroid_sums(k, 2, 5)
+    assert sums.tolist() == [[4.0, -1.5], [3.0, 5.0], [2.0, 2.0]]
+    beta = M.centroid_block_scores(_bf(np.array([[1.0, 1.0]])), sums, 2, 5)
+    assert beta.tolist() == [2.5 / 2, 8.0 / 2, 4.0 / 1]
+
+
+def test_centroid_sums_round_in_float32_sequence():
+    # 1 + 2^-24 + 2^-24: sequential float32 adds lose both small terms
+    k = _bf(np.array([[1.0], [2.0 ** -24], [2.0 ** -24]]))
+    assert M.centroid_sums(k, 4, 3)[0, 0] == np.float32(1.0)
+    # token-level blocks (S = 1): each sum is the key itself
+    kk = _bf(np.random.default_rng(51).standard_normal((7, 4)))
+    assert np.array_equal(M.centroid_sums(kk, 1, 7), F.bf16_to_f64(kk).astype(np.float32))
