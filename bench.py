@@ -42,7 +42,8 @@ import synth  # noqa: E402
 METRIC = "sparse decode attn steps/s at 128K ctx, batch 16; achieved HBM GB/s vs peak"
 WORKLOADS = {"block128k": synth.BLOCK128K, "token32k": synth.TOKEN32K, "ragged": synth.RAGGED,
              "nvfp4": synth.NVFP4_128K, "tiny": synth.TINY, "fp8": synth.FP8_128K,
-             "fp8token": synth.FP8_TOKEN32K}
+             "fp8token": synth.FP8_TOKEN32K, "centroid": synth.CENTROID_128K,
+             "centroid32": synth.CENTROID_S32}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -146,11 +147,15 @@ def step_bytes(w, lens, sel, nsel):
     """Algorithmic bytes of one decode step: proxy-cache bytes streamed + selected K/V bytes
     (valid tokens only) + q + out."""
     d, S = w.head_dim, w.block_size
-    if w.proxy_dtype == "nvfp4":
-        per_tok = d // 2 + d // 16
+    if w.proxy_dtype == "centroid":                 # one FP32 key sum per block
+        nbs = (lens.astype(np.int64) + S - 1) // S
+        proxy = int(nbs.sum()) * w.n_kv_heads * d * 4
     else:
-        per_tok = w.proxy_rank * {"f32": 4, "bf16": 2, "e4m3": 1}[w.proxy_dtype]
-    proxy = int(np.sum(lens.astype(np.int64))) * w.n_kv_heads * per_tok
+        if w.proxy_dtype == "nvfp4":
+            per_tok = d // 2 + d // 16
+        else:
+            per_tok = w.proxy_rank * {"f32": 4, "bf16": 2, "e4m3": 1}[w.proxy_dtype]
+        proxy = int(np.sum(lens.astype(np.int64))) * w.n_kv_heads * per_tok
     tokens = 0
     for b in range(w.batch):
         L = int(lens[b])
@@ -447,7 +452,7 @@ def run_ours(args):
     nsel_h = nsel.cpu().numpy()
     sel_h = sel.cpu().numpy()
     # append [+ block errors + query tiles] + score + select + attention (1 or 2 launches)
-    launches_per_step = (3 if w.proxy_rank > 0 else 5) + qs.qs_attention_launches(
+    launches_per_step = (5 if w.proxy_dtype == "nvfp4" else 3) + qs.qs_attention_launches(
         lay.cfg, w.batch, lay.max_context)
 
     def barrier():
@@ -558,7 +563,8 @@ def run_ours(args):
     peak, peak_src = peaks()
     by = step_bytes(w, lens, sel_h, nsel_h)
     score_us = stage_us["score"]
-    score_kernel_file = "score.cu" if w.proxy_rank > 0 else "score_nvfp4.cu"
+    score_kernel_file = {"nvfp4": "score_nvfp4.cu", "centroid": "score_centroid.cu"}.get(
+        w.proxy_dtype, "score.cu")
     traffic = profiled_traffic(score_kernel_file.replace(".cu", ""), w.name)
     roof = {"bound": "hbm", "kernel": "score (scoring prep + proxy scan, one qs_score call)",
             "achieved": by["proxy"] / (score_us * 1e-6) / 1e9, "peak": peak, "unit": "GB/s",
@@ -570,7 +576,8 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if w.proxy_dtype == "bf16" else f"{w.proxy_dtype}+bf16",
+            "dtype": {"bf16": "bf16", "f32": "f32+bf16", "centroid": "f32+bf16"}.get(
+                w.proxy_dtype, f"{w.proxy_dtype}+bf16"),
             "data": "synthetic (seeded; shapes of the pages' 128K batch-16 decode)",
             "config": config_of(w, lens),
             "tokens_per_s": value * B, "us_per_layer_step": t_ms * 1e3,

@@ -53,6 +53,8 @@
  *   proxy (NVFP4)   [num_pages][Hkv][page_size][head_dim/2] u8: E2M1 codes, element 2i in
  *                                                           the low nibble of byte i
  *   proxy_scale     [num_pages][Hkv][page_size][head_dim/16] u8: UE4M3 scale per 16 elems
+ *   proxy (centroid)[num_pages][Hkv][page_size/S][head_dim] F32: the sum of the keys of each
+ *                                                           S-token block of the page
  *   page_table      [batch][max_pages_per_seq]              int32 physical page ids
  *   seq_lens        [batch]                                 int32 tokens in the cache
  *   P               [Hkv][head_dim][r]                      F32
@@ -85,7 +87,10 @@ typedef enum {
   QS_ERR_DEVICE_TIMEOUT = 5
 } qs_status;
 
-typedef enum { QS_F32 = 0, QS_BF16 = 1, QS_F16 = 2, QS_NVFP4 = 3, QS_E4M3 = 4 } qs_dtype;
+typedef enum {
+  QS_F32 = 0, QS_BF16 = 1, QS_F16 = 2, QS_NVFP4 = 3, QS_E4M3 = 4,
+  QS_CENTROID = 5   /* proxy_dtype only: per-block FP32 key sums (centroid scoring), r = 0 */
+} qs_dtype;
 
 /* Problem statement of one attention layer's decode step. */
 typedef struct {
@@ -96,7 +101,7 @@ typedef struct {
   int32_t block_size;     /* S: a power of two dividing page_size (1 = token level)       */
   int32_t budget;         /* k: blocks selected per row, >= 1                             */
   int32_t proxy_rank;     /* r > 0: projected-key proxy; 0: NVFP4 centred keys            */
-  int32_t proxy_dtype;    /* qs_dtype: F32, BF16 or E4M3 (rank r), NVFP4 (r == 0)         */
+  int32_t proxy_dtype;    /* qs_dtype: F32, BF16 or E4M3 (rank r); NVFP4 or CENTROID (r 0) */
   int32_t v_dtype;        /* qs_dtype of stored V: BF16 or F16                            */
   int32_t v_agg_dtype;    /* precision of the P.V operands: BF16 or F16 (FP32 accumulate) */
   int32_t out_dtype;      /* F32 or BF16                                                  */
@@ -149,6 +154,9 @@ qs_status qs_workspace_init(void *ws, size_t ws_bytes, qs_stream_t stream);
              sum), stored F32, rounded to nearest-even BF16, or rounded to nearest-even E4M3
              saturating at +-448 (the FP8 scoring cache of "Joint Subspace Sparse Attention
              ...", Figure 10);
+     centroid: the block's FP32 key sum, continued in token order (one rounding per add;
+             restarted at the block's first token): "Coarse Semantic Blocks ...", Abstract,
+             scores blocks by their centroids;
      NVFP4:  x = float(k) - key_center[b][g] (float32), packed per 16 elements to UE4M3
              scale + E2M1 codes with the tensor scale g_k; each block of S tokens that this
              call completes gets block_err = sum of squared (x - dequant(x)).
@@ -162,6 +170,9 @@ qs_status qs_append_kv(const qs_config *cfg, const qs_cache *cache, const void *
    rank r: qbar = mean of the group's query heads (float32), q~ = qbar.P[g] (float32),
            s_t = q~ . proxy_t (float32 accumulation), beta_j = max of s over the block's
            valid tokens (t < seq_len).
+   centroid: qbar = mean of the group's query heads (float32); beta_j = qbar . sum_j /
+           count_j (float32), count_j = valid tokens of block j (the mean of the block's
+           exact group-mean scores);
    NVFP4:  the whole q tensor is packed with g_q = max|q| / 2688; per head h,
            s_{h,t} = g_q g_k sum_c sq_{h,c} sk_{t,c} sum_i eq_{h,16c+i} ek_{t,16c+i} on the
            block-scaled FP4 tensor cores; beta_j = max over the group's heads and the

@@ -14,9 +14,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqs.so")
 
 QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA, QS_ERR_DEVICE_BOUNDS, \
     QS_ERR_DEVICE_TIMEOUT = range(6)
-QS_F32, QS_BF16, QS_F16, QS_NVFP4, QS_E4M3 = range(5)
+QS_F32, QS_BF16, QS_F16, QS_NVFP4, QS_E4M3, QS_CENTROID = range(6)
 DTYPE_CODES = {"f32": QS_F32, "bf16": QS_BF16, "f16": QS_F16, "nvfp4": QS_NVFP4,
-               "e4m3": QS_E4M3}
+               "e4m3": QS_E4M3, "centroid": QS_CENTROID}
 
 
 class QsError(RuntimeError):

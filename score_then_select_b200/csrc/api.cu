@@ -89,7 +89,10 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   if (c->head_dim != 64 && c->head_dim != 128) return QS_ERR_UNSUPPORTED;
   const int r = c->proxy_rank;
   if (r < 0) return QS_ERR_INVALID_ARG;
-  if (r > 0) {
+  p.kind = r > 0 ? PK_RANKR : (c->proxy_dtype == QS_CENTROID ? PK_CENTROID : PK_NVFP4);
+  if (p.kind == PK_CENTROID) {
+    if (c->n_keep_hp != 0) return QS_ERR_INVALID_ARG;
+  } else if (r > 0) {
     const bool ok = (c->proxy_dtype == QS_F32 && (r == 16 || (r == 32 && c->head_dim == 128))) ||
                     ((c->proxy_dtype == QS_BF16 || c->proxy_dtype == QS_E4M3) &&
                      (r == 32 || (r == 64 && c->head_dim == 128)));
@@ -149,7 +152,7 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   size_t off = size_t(kHdrWords) * 4;
   const size_t rows = size_t(batch) * p.Hkv, rows_q = size_t(batch) * p.Hq;
   w.qt = off;      off = align_up(off + rows * (r > 0 ? r : 1) * 4, 256);
-  w.qtile = off;   off = align_up(off + (r == 0 ? rows * kQTileBytes : 0), 256);
+  w.qtile = off;   off = align_up(off + (p.kind == PK_NVFP4 ? rows * kQTileBytes : 0), 256);
   w.qgscale = off; off = align_up(off + 16, 256);
   w.scores = off;  off = align_up(off + rows * p.nb_stride * 4, 256);
   w.sel = off;     off = align_up(off + rows * p.budget * 4, 256);
@@ -183,7 +186,8 @@ qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy) {
   if (!aligned(c->k, 16) || !aligned(c->v, 16)) return QS_ERR_INVALID_ARG;
   if (need_proxy) {
     if (!c->proxy || !aligned(c->proxy, 16)) return QS_ERR_INVALID_ARG;
-    if (p.r == 0 && (!c->proxy_scale || !c->key_center || !c->key_gscale)) return QS_ERR_INVALID_ARG;
+    if (p.kind == PK_NVFP4 && (!c->proxy_scale || !c->key_center || !c->key_gscale))
+      return QS_ERR_INVALID_ARG;
   }
   return QS_OK;
 }
@@ -225,8 +229,9 @@ static qs_status do_append(const Plan& p, const qs_cache* c, const void* k_new, 
   a.max_pages_per_seq = c->max_pages_per_seq;
   a.num_pages = c->num_pages;
   a.max_context = c->max_context;
+  a.S = p.S;
   qs_status st = cuda_status(launch_append(p, a, s));
-  if (st != QS_OK || p.r != 0) return st;
+  if (st != QS_OK || p.kind != PK_NVFP4) return st;
   BlockErrParams e{};
   e.k = a.k;
   e.key_center = c->key_center;
@@ -249,6 +254,7 @@ static qs_status do_append(const Plan& p, const qs_cache* c, const void* k_new, 
 
 static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws, cudaStream_t s,
                          bool pdl) {
+  if (p.kind == PK_CENTROID) return QS_OK;          // the scan averages the queries itself
   if (p.r > 0) {
     PrepParams a{static_cast<const uint16_t*>(q), P, ws_at<float>(ws, p.ws.qt),
                  p.batch, p.Hkv, p.G, p.d, p.r};
@@ -260,10 +266,11 @@ static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws,
   return cuda_status(launch_qpack(p, a, s, pdl));
 }
 
-static qs_status do_score(const Plan& p, const qs_cache* c, float* scores, void* ws, cudaStream_t s,
-                          bool pdl, bool early_stream = false) {
+static qs_status do_score(const Plan& p, const qs_cache* c, const void* q, float* scores, void* ws,
+                          cudaStream_t s, bool pdl, bool early_stream = false) {
   ScoreParams a{};
   a.early_stream = early_stream ? 1 : 0;
+  a.q = static_cast<const uint16_t*>(q);
   a.proxy = c->proxy;
   a.proxy_scale = c->proxy_scale;
   a.qt = ws_at<float>(ws, p.ws.qt);
@@ -290,7 +297,7 @@ static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores
                            int32_t* n_sel, void* ws, cudaStream_t s, bool pdl) {
   SelectParams a{};
   a.scores = scores;
-  a.block_err = (p.r == 0 && p.n_keep > 0) ? c->block_err : nullptr;
+  a.block_err = (p.kind == PK_NVFP4 && p.n_keep > 0) ? c->block_err : nullptr;
   a.seq_lens = c->seq_lens;
   a.sel = sel;
   a.n_sel = n_sel;
@@ -394,7 +401,7 @@ qs_status qs_append_kv(const qs_config* cfg, const qs_cache* cache, const void* 
   if (!k_new || !v_new || !n_new || max_new < 1 || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
-  if (p.r == 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
+  if (p.kind == PK_NVFP4 && !cache->block_err) return QS_ERR_INVALID_ARG;
   return do_append(p, cache, k_new, v_new, n_new, max_new, P, nullptr, ws, stream);
 }
 
@@ -407,10 +414,11 @@ qs_status qs_score(const qs_config* cfg, const qs_cache* cache, const void* q, c
   if (!q || !aligned(q, 4) || !block_scores || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
   if (p.r == 0 && !aligned(q, 16)) return QS_ERR_INVALID_ARG;
+  if (p.kind == PK_CENTROID) return do_score(p, cache, q, block_scores, ws, stream, false);
   // the prep kernel runs in stream order and writes only the query side, so the scan
   // overlaps it and starts streaming pages before it waits for the query
   if ((st = do_prep(p, q, P, ws, stream, false)) != QS_OK) return st;
-  return do_score(p, cache, block_scores, ws, stream, true, true);
+  return do_score(p, cache, q, block_scores, ws, stream, true, true);
 }
 
 qs_status qs_select_topk(const qs_config* cfg, const qs_cache* cache, const float* block_scores,
@@ -420,7 +428,7 @@ qs_status qs_select_topk(const qs_config* cfg, const qs_cache* cache, const floa
   if (st != QS_OK) return st;
   if (!cache || !cache->seq_lens) return QS_ERR_INVALID_ARG;
   if (!block_scores || !sel || !n_sel || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
-  if (p.r == 0 && p.n_keep > 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
+  if (p.kind == PK_NVFP4 && p.n_keep > 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
   return do_select(p, cache, block_scores, sel, n_sel, ws, stream, false);
 }
 
@@ -530,15 +538,15 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   if (!q || !aligned(q, 16) || !k_new || !v_new || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
-  if (p.r == 0 && (!cache->block_err || !aligned(q, 16))) return QS_ERR_INVALID_ARG;
+  if (p.kind == PK_NVFP4 && !cache->block_err) return QS_ERR_INVALID_ARG;
   if ((sel_out == nullptr) != (n_sel_out == nullptr)) return QS_ERR_INVALID_ARG;
   int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, p.ws.sel);
   int32_t* nsel = n_sel_out ? n_sel_out : ws_at<int32_t>(ws, p.ws.nsel);
   float* scores = ws_at<float>(ws, p.ws.scores);
   // append (+ fused scoring prep on the rank-r path)
   if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, P, q, ws, stream)) != QS_OK) return st;
-  if (p.r == 0 && (st = do_prep(p, q, P, ws, stream, true)) != QS_OK) return st;
-  if ((st = do_score(p, cache, scores, ws, stream, true)) != QS_OK) return st;
+  if (p.kind == PK_NVFP4 && (st = do_prep(p, q, P, ws, stream, true)) != QS_OK) return st;
+  if ((st = do_score(p, cache, q, scores, ws, stream, true)) != QS_OK) return st;
   if ((st = do_select(p, cache, scores, sel, nsel, ws, stream, true)) != QS_OK) return st;
   return do_attend(p, cache, q, sel, nsel, out, ws, stream, true);
 }

@@ -356,6 +356,60 @@ __global__ void __launch_bounds__(128) append_one_rankr_kernel(const AppendParam
   finish_append(a);
 }
 
+// ============================================================ centroid writer
+// "Coarse Semantic Blocks ...", Abstract: blocks are scored by their centroids. The cache
+// holds each block's FP32 key sum; the scan divides by the block's valid count.
+// CTA = (row, one block touched by this call): thread i < d carries dimension i of the
+// block's sum through the call's tokens in order (restarting at the block's first token,
+// continuing a sum left by an earlier call otherwise); all threads copy the tokens' K and V
+// rows into their page slots.
+template <int D>
+__global__ void __launch_bounds__(128) append_centroid_kernel(const AppendParams a) {
+  pdl_trigger();   // the scan may launch now; it waits for this grid before reading
+  const int row = blockIdx.y;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  const int tid = threadIdx.x;
+  int n_b = a.n_new ? a.n_new[b] : 1;
+  if (n_b < 0 || n_b > a.max_new) {
+    if (tid == 0 && blockIdx.x == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_APPEND, uint32_t(b));
+    n_b = 0;
+  }
+  const int old = a.seq_lens[b], S = a.S;
+  const int j = (old >= 0 ? old / S : 0) + int(blockIdx.x);     // this CTA's block
+  const int t_lo = max(old, j * S), t_hi = min(old + n_b, (j + 1) * S);
+  if (old >= 0 && t_lo < t_hi) {
+    const int pi = (j * S) >> 7;                                  // kPage = 128
+    int page = -1;
+    if (pi < a.max_pages_per_seq) page = a.page_table[size_t(b) * a.max_pages_per_seq + pi];
+    if (page < 0 || page >= a.num_pages || t_hi > a.max_context) {
+      if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_APPEND, uint32_t(row));
+    } else {
+      const size_t src0 = size_t(row) * a.max_new * D;           // token 0 of this row's k_new
+      // K and V rows of the block's new tokens -> their page slots (16 bytes per step)
+      constexpr int CH = D / 8;
+      for (int e = tid; e < (t_hi - t_lo) * CH; e += blockDim.x) {
+        const int t = t_lo + e / CH, c = e % CH;
+        const size_t src = src0 + size_t(t - old) * D + c * 8;
+        const size_t dst = ((size_t(page) * a.Hkv + g) * kPage + (t & (kPage - 1))) * D + c * 8;
+        *reinterpret_cast<uint4*>(a.k + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+        *reinterpret_cast<uint4*>(a.v + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+      }
+      // the block's key sum, dimension tid, in token order
+      float* sum = reinterpret_cast<float*>(a.proxy) +
+                   ((size_t(page) * a.Hkv + g) * (kPage / S) + ((j * S) & (kPage - 1)) / S) * D;
+      if (tid < D) {
+        float acc = t_lo == j * S ? 0.0f : sum[tid];
+        for (int t = t_lo; t < t_hi; ++t) {
+          const float x = bf16_to_f32(a.k_new[src0 + size_t(t - old) * D + tid]);
+          acc = t == j * S ? x : __fadd_rn(acc, x);
+        }
+        sum[tid] = acc;
+      }
+    }
+  }
+  finish_append(a);
+}
+
 // ============================================================ NVFP4 writer
 // CTA = one row x 64 tokens; thread = (token, 16-element group).
 __global__ void __launch_bounds__(128) append_nvfp4_kernel(const AppendParams a) {
@@ -601,7 +655,14 @@ static cudaError_t launch_rankr(const Plan& p, const AppendParams& a, cudaStream
 }
 
 cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) {
-  if (p.r == 0) {
+  if (p.kind == PK_CENTROID) {
+    // blocks a call can touch: ceil(max_new / S) + 1 (the first may be partly filled)
+    const dim3 grid((a.max_new + p.S - 1) / p.S + 1, a.batch * a.Hkv);
+    if (p.d == 128) append_centroid_kernel<128><<<grid, 128, 0, s>>>(a);
+    else append_centroid_kernel<64><<<grid, 128, 0, s>>>(a);
+    return cudaGetLastError();
+  }
+  if (p.kind == PK_NVFP4) {
     dim3 grid((a.max_new + 63) / 64, a.batch * a.Hkv);
     append_nvfp4_kernel<<<grid, 128, 0, s>>>(a);
     return cudaGetLastError();

@@ -57,8 +57,12 @@ struct WsLayout {
   int parts_per_head = 0;  // attention partials per query head in the workspace
 };
 
+// Scoring proxy of a configuration
+enum ProxyKind : int { PK_RANKR = 0, PK_NVFP4 = 1, PK_CENTROID = 2 };
+
 struct Plan {
   int batch, Hq, Hkv, G, d, S, budget, r, nb_stride;
+  int kind;             // ProxyKind
   bool attn_tma;        // attention by the tile pipeline (else the gather kernel)
   int proxy_dtype, v_dtype, v_agg_dtype, out_dtype;
   int force_sink, force_last, n_keep;
@@ -85,6 +89,7 @@ struct AppendParams {
   const uint16_t* q;
   float* qt;
   int batch, Hkv, G, d, r, max_new, max_pages_per_seq, num_pages, max_context;
+  int S;                     // block size (centroid sums)
 };
 
 struct BlockErrParams {
@@ -142,6 +147,7 @@ __host__ __device__ inline int qtile_scale_off(int head, int group) {
 }
 
 struct ScoreParams {
+  const uint16_t* q;         // centroid scoring: the queries [batch][Hq][d]
   const void* proxy;
   const uint8_t* proxy_scale;
   const float* qt;           // rank r: [batch][Hkv][r]

@@ -287,9 +287,11 @@ static cudaError_t launch_rankr_score(const ScoreParams& a, cudaStream_t st, boo
 }
 
 cudaError_t launch_score_nvfp4(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl);
+cudaError_t launch_score_centroid(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl);
 
 cudaError_t launch_score(const Plan& p, const ScoreParams& a, cudaStream_t s, bool pdl) {
-  if (p.r == 0) return launch_score_nvfp4(p, a, s, pdl);
+  if (p.kind == PK_CENTROID) return launch_score_centroid(p, a, s, pdl);
+  if (p.kind == PK_NVFP4) return launch_score_nvfp4(p, a, s, pdl);
   if (p.proxy_dtype == QS_E4M3) {
     if (p.r == 32) return launch_rankr_score<uint8_t, 32>(a, s, pdl);
     if (p.r == 64) return launch_rankr_score<uint8_t, 64>(a, s, pdl);

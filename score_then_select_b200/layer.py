@@ -40,7 +40,11 @@ class Layer:
         k = torch.zeros((num_pages, Hkv, ps, d), dtype=torch.bfloat16, device=device)
         v = torch.zeros((num_pages, Hkv, ps, d), dtype=vdt, device=device)
         extra = {}
-        if r > 0:
+        if cfg.proxy_dtype == B.QS_CENTROID:
+            # per-block FP32 key sums: [num_pages][Hkv][page_size / S][d]
+            proxy = torch.zeros((num_pages, Hkv, ps // cfg.block_size, d), dtype=torch.float32,
+                                device=device)
+        elif r > 0:
             pdt = {B.QS_F32: torch.float32, B.QS_E4M3: torch.uint8}.get(cfg.proxy_dtype,
                                                                         torch.bfloat16)
             proxy = torch.zeros((num_pages, Hkv, ps, r), dtype=pdt, device=device)

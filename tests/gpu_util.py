@@ -86,6 +86,9 @@ class Filled:
             codes[:, 0::2] = c & 15
             codes[:, 1::2] = c >> 4
             return codes, s
+        if self.w.proxy_dtype == "centroid":
+            nb = -(-L // self.w.block_size)
+            return self.layer.proxy[pages, g].reshape(-1, self.w.head_dim)[:nb].cpu().numpy()
         p = self.layer.proxy[pages, g].reshape(npg * 128, -1)[:L]
         if self.w.proxy_dtype in ("f32", "e4m3"):
             return p.cpu().numpy()

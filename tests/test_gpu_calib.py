@@ -115,3 +115,30 @@ def test_calibrated_basis_raises_selection_recall():
     cal, rnd = np.mean(recalls["calibrated"]), np.mean(recalls["random"])
     print(f"top-{B} recall: calibrated basis {cal:.3f}, random basis {rnd:.3f}")
     assert cal >= 0.8 and cal >= rnd + 0.3, (cal, rnd)
+
+
+def test_calibration_time():
+    """One calibration of 8 KV heads (d 128, r 32, 4,096 positions, G 5): CUDA-event time,
+    printed; it runs once before decoding, so only a loose bound is asserted."""
+    _gpu()
+    import score_then_select_b200 as qs
+    Hkv, G, d, r, n = 8, 5, 128, 32, 4096
+    cfg = qs.make_config(n_q_heads=Hkv * G, n_kv_heads=Hkv, head_dim=d, block_size=128,
+                         budget=64, proxy_rank=r, proxy_dtype="bf16")
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    q = (torch.randn((n, Hkv * G, d), device="cuda", generator=gen)).to(torch.bfloat16)
+    k = (torch.randn((n, Hkv, d), device="cuda", generator=gen)).to(torch.bfloat16)
+    ws = torch.zeros((qs.qs_calib_workspace_size(cfg),), dtype=torch.uint8, device="cuda")
+    P = torch.empty((Hkv, d, r), dtype=torch.float32, device="cuda")
+    qs.qs_calibrate_basis(cfg, q, k, n, P, None, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(5):
+        qs.qs_calibrate_basis(cfg, q, k, n, P, None, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 5
+    print(f"calibration of {Hkv} heads from {n} positions: {ms:.2f} ms")
+    assert ms < 200.0
+    assert torch.isfinite(P).all()

@@ -22,7 +22,8 @@ pytestmark = pytest.mark.gpu
 
 RANKR = [synth.TINY, synth.TINY_NEEDLE] + [synth.small(w) for w in
                                           (synth.TOKEN32K, synth.BLOCK128K, synth.RAGGED,
-                                           synth.FP8_128K, synth.FP8_TOKEN32K)]
+                                           synth.FP8_128K, synth.FP8_TOKEN32K,
+                                           synth.CENTROID_128K, synth.CENTROID_S32)]
 NVFP4 = [synth.small(synth.NVFP4_128K)]
 
 
