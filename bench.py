@@ -43,7 +43,7 @@ METRIC = "sparse decode attn steps/s at 128K ctx, batch 16; achieved HBM GB/s vs
 WORKLOADS = {"block128k": synth.BLOCK128K, "token32k": synth.TOKEN32K, "ragged": synth.RAGGED,
              "nvfp4": synth.NVFP4_128K, "tiny": synth.TINY, "fp8": synth.FP8_128K,
              "fp8token": synth.FP8_TOKEN32K, "centroid": synth.CENTROID_128K,
-             "centroid32": synth.CENTROID_S32}
+             "centroid32": synth.CENTROID_S32, "token128k": synth.TOKEN128K}
 FALLBACK_HBM_GBS = 6650.0
 
 

@@ -127,6 +127,7 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   const long long pages = (max_context + kPage - 1) / kPage;
   const long long nbs = pages * (kPage / p.S);
   if (nbs > kMaxSelectBlocks) return QS_ERR_UNSUPPORTED;
+  if (nbs > 32768 && c->n_keep_hp > 0) return QS_ERR_UNSUPPORTED;  // kept blocks: one CTA per row
   p.nb_stride = int(nbs);
   const long long slots = (long long)p.budget * p.S;
   if (slots > 64LL * 2048) return QS_ERR_UNSUPPORTED;

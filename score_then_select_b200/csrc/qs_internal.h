@@ -25,7 +25,7 @@ enum KernelId : uint32_t {
 constexpr int kPage = 128;          // tokens per page (the only page size built)
 constexpr int kMaxBatch = 1024;     // sequences per call
 constexpr int kMaxGroup = 8;        // query heads per KV head
-constexpr int kMaxSelectBlocks = 32768;
+constexpr int kMaxSelectBlocks = 131072;  // 32768 per CTA, clusters of 4 CTAs beyond
 constexpr int kHdrWords = 64;       // workspace header (256 bytes)
 constexpr int kCtrAppend = 16;      // header word: append "last CTA" counter
 constexpr int kAttnCtasPerSm = 2;   // resident attention CTAs per SM (shared-memory bound)

@@ -106,6 +106,12 @@ FP8_128K = BLOCK128K.replace(name="fp8_b16_h40kv8_d128_L131072_S128_k64_r32", pr
 FP8_TOKEN32K = TOKEN32K.replace(name="fp8_token_b16_h32kv8_d128_L32768_r64_B2048",
                                 proxy_rank=64, proxy_dtype="e4m3", seed=1007)
 
+# Token-level selection at 128K context, B = 2,048 tokens per KV head: the setting of the
+# component-level latency ("Joint Subspace Sparse Attention ...", Figure 9) and of the
+# gather-free comparison (Figure 6); selection over 131,072 candidates per row.
+TOKEN128K = TOKEN32K.replace(name="token_b16_h32kv8_d128_L131072_r32_B2048", context=131072,
+                             seed=1010)
+
 # Centroid scoring ("Coarse Semantic Blocks ...", Abstract): each block scored by the mean
 # of its keys against the group-mean query, from per-block FP32 key sums (no projection).
 CENTROID_128K = BLOCK128K.replace(name="centroid_b16_h40kv8_d128_L131072_S128_k64",
@@ -124,8 +130,8 @@ RAGGED = Workload(
 
 FULL = {w.name: w for w in (TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED)}
 ORDER = [TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED]
-# variants of the configurations above (FP8 projected keys, centroid scoring)
-VARIANTS = [FP8_128K, FP8_TOKEN32K, CENTROID_128K, CENTROID_S32]
+# variants of the configurations above (FP8 projected keys, centroid scoring, 128K token level)
+VARIANTS = [FP8_128K, FP8_TOKEN32K, CENTROID_128K, CENTROID_S32, TOKEN128K]
 
 
 def small(w: Workload) -> Workload:

@@ -71,8 +71,10 @@ def test_host_validation(kw, status):
 
 
 def test_token_level_context_limit():
+    # token-level selection runs up to 131,072 candidates per row (a cluster of 4 CTAs)
+    assert qs.qs_workspace_size(_cfg(block_size=1, budget=2048), 16, 131072) > 0
     with pytest.raises(qs.QsError) as e:
-        qs.qs_workspace_size(_cfg(block_size=1, budget=2048), 16, 65536)
+        qs.qs_workspace_size(_cfg(block_size=1, budget=2048), 16, 131073)
     assert e.value.status == B.QS_ERR_UNSUPPORTED
 
 

@@ -19,7 +19,7 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 # (workload, attention kernel): the automatic choice everywhere, and the tile pipeline
 # forced on the ragged workload (whose rows end in partial blocks)
 FULL = [(synth.BLOCK128K, 0), (synth.NVFP4_128K, 0), (synth.TOKEN32K, 0), (synth.RAGGED, 0),
-        (synth.RAGGED, 1), (synth.FP8_128K, 0), (synth.CENTROID_128K, 0)]
+        (synth.RAGGED, 1), (synth.FP8_128K, 0), (synth.CENTROID_128K, 0), (synth.TOKEN128K, 0)]
 
 
 def _check_all_rows(w, inp, sel, nsel, out, berr):

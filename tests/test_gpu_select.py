@@ -2,7 +2,8 @@
 selection must equal the oracle's (forced blocks, then the best others with ties to the
 lower index, ascending) exactly.
 
-Rows cover the three kernel shapes (up to 1,024, 4,096 and 32,768 blocks per row) and the
+Rows cover the kernel shapes (up to 1,024, 4,096 and 32,768 blocks per row in one CTA, and
+131,072 in a cluster of 4 CTAs) and the
 cases the workloads rarely reach:
 - heavy ties (few distinct values, which takes the radix passes);
 - all scores equal;
@@ -68,9 +69,9 @@ def _scores(kind, rng, n):
 
 
 KINDS = ["normal", "ties", "equal", "signed_zero", "nonfinite", "extreme", "clustered"]
-# (block size, budget, max_context, forced sink / last): 1,024 / 4,096 / 32,768 blocks
+# (block size, budget, max_context, forced sink / last): 1,024 / 4,096 / 32,768 / 131,072 blocks
 SHAPES = [(128, 64, 131072, True), (32, 100, 131072, False), (1, 2048, 32768, False),
-          (1, 500, 32768, True)]
+          (1, 500, 32768, True), (1, 2048, 131072, False), (1, 3000, 131072, True)]
 
 
 def _run(shape, kind, seed):
