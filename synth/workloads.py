@@ -128,6 +128,12 @@ RAGGED = Workload(
     n_keep_hp=0, softmax_scale=0.0, key_recipe="mixture", query_recipe="normal", seed=1005,
     ragged=True, ragged_overrides=((29, 100), (30, 1000), (31, 2047)))
 
+# d = 64 variants of the tiny step: FP8 projected keys (rank 32) and centroid scoring
+TINY_FP8 = TINY.replace(name="tiny_fp8_b1_h4_d64_L2048_r32", proxy_rank=32, proxy_dtype="e4m3",
+                        seed=1011)
+TINY_CENTROID = TINY.replace(name="tiny_centroid_b1_h4_d64_L2048", proxy_rank=0,
+                             proxy_dtype="centroid", seed=1012)
+
 FULL = {w.name: w for w in (TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED)}
 ORDER = [TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED]
 # variants of the configurations above (FP8 projected keys, centroid scoring, 128K token level)

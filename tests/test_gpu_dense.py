@@ -20,8 +20,8 @@ from tests.util import oracle_row, query_scale_all
 
 pytestmark = pytest.mark.gpu
 
-WORKLOADS = [synth.TINY] + [synth.small(w) for w in (synth.TOKEN32K, synth.BLOCK128K,
-                                                      synth.NVFP4_128K, synth.RAGGED)]
+WORKLOADS = [synth.TINY, synth.TINY_CENTROID] + [synth.small(w) for w in (
+    synth.TOKEN32K, synth.BLOCK128K, synth.NVFP4_128K, synth.RAGGED)]
 
 
 def _gpu():

@@ -20,7 +20,7 @@ from tests.util import oracle_row, query_scale_all, row_params
 
 pytestmark = pytest.mark.gpu
 
-RANKR = [synth.TINY, synth.TINY_NEEDLE] + [synth.small(w) for w in
+RANKR = [synth.TINY, synth.TINY_NEEDLE, synth.TINY_FP8, synth.TINY_CENTROID] + [synth.small(w) for w in
                                           (synth.TOKEN32K, synth.BLOCK128K, synth.RAGGED,
                                            synth.FP8_128K, synth.FP8_TOKEN32K,
                                            synth.CENTROID_128K, synth.CENTROID_S32)]
