@@ -110,3 +110,38 @@ def test_comparison_calls_reject_null_pointers_without_launch():
     with pytest.raises(qs.QsError) as e:
         qs.qs_gather_kv(cfg, cache, 0, 0, 16, 0, 0, 0, 0, stream=0)
     assert e.value.status == B.QS_ERR_INVALID_ARG
+
+
+def test_centroid_and_fp8_configurations():
+    # centroid scoring: rank 0 with the centroid proxy; kept blocks are NVFP4-only
+    assert qs.qs_workspace_size(_cfg(proxy_rank=0, proxy_dtype="centroid"), 16, 131072) > 0
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_workspace_size(_cfg(proxy_rank=0, proxy_dtype="centroid", n_keep_hp=2), 16, 4096)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    # a rank-r proxy cannot be a centroid cache
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_workspace_size(_cfg(proxy_dtype="centroid"), 16, 4096)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+
+
+def test_calibration_entry_points_validate_on_the_host():
+    cfg = _cfg(n_q_heads=32, n_kv_heads=8, proxy_rank=32)
+    assert qs.qs_calib_workspace_size(cfg) == 256 + 2 * 8 * 128 * 128 * 8
+    with pytest.raises(qs.QsError) as e:                      # no rank, no basis
+        qs.qs_calib_workspace_size(_cfg(proxy_rank=0, proxy_dtype="nvfp4", block_size=128))
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    with pytest.raises(qs.QsError) as e:                      # null pointers, no launch
+        qs.qs_calibrate_basis(cfg, 0, 0, 16, 0, None, 0, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    with pytest.raises(qs.QsError) as e:                      # no positions
+        qs.qs_calibrate_basis(cfg, 16, 16, 0, 16, None, 256, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+
+
+def test_kept_blocks_limited_to_one_cta_rows():
+    # NVFP4 kept blocks with more than 32,768 blocks per row are refused on the host
+    cfg = _cfg(proxy_rank=0, proxy_dtype="nvfp4", block_size=128, n_keep_hp=2)
+    assert qs.qs_workspace_size(cfg, 1, 128 * 32768) > 0
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_workspace_size(cfg, 1, 128 * 32768 + 1)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
