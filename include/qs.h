@@ -41,8 +41,12 @@
  *     reads. Waits inside kernels are bounded; running out records QS_ERR_DEVICE_TIMEOUT.
  *   - A launch error is returned as QS_ERR_CUDA (the CUDA error is left for
  *     cudaGetLastError by the caller).
- *   - Entry points are re-entrant and keep no global state; two calls that share a
- *     workspace must not overlap on the GPU.
+ *   - Entry points are re-entrant; two calls that share a workspace must not overlap on
+ *     the GPU. The library keeps only process-wide caches, each guarded by a mutex or
+ *     atomic: encoded TMA tensor maps (keyed by tensor address and shape, 16 entries),
+ *     the kernels' shared-memory limits (set once per kernel and device) and the SM
+ *     count of each device. One process may drive several GPUs (the current device at
+ *     the call is used).
  *
  * Memory layouts (row-major, innermost last):
  *   K, V pages      [num_pages][Hkv][page_size][head_dim]   BF16 (V may be FP16)

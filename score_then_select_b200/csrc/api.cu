@@ -1,25 +1,46 @@
 // api.cu - the C ABI of libqs: argument validation, launch plans, workspace layout and
 // the entry points declared in include/qs.h. No device memory is allocated here.
+#include <atomic>
 #include <cmath>
 #include <algorithm>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "qs_internal.h"
 
 namespace qs {
 
 int num_sms() {
-  static thread_local int cached = 0;
-  if (cached > 0) return cached;
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cached[kMaxDevices] = {};
   int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess &&
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-    cached = n;
-  else {
+  if (cudaGetDevice(&dev) != cudaSuccess) {
     cudaGetLastError();
-    cached = 148;
+    return 148;
   }
-  return cached;
+  if (dev >= 0 && dev < kMaxDevices && cached[dev].load() > 0) return cached[dev].load();
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 148;
+  }
+  if (dev >= 0 && dev < kMaxDevices) cached[dev].store(n);
+  return n;
+}
+
+cudaError_t set_smem_limit(const void* kern, int bytes) {
+  struct Done { const void* kern; int dev, bytes; };
+  static std::mutex mu;
+  static std::vector<Done> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Done& d : done)
+    if (d.kern == kern && d.dev == dev && d.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back(Done{kern, dev, bytes});
+  return e;
 }
 
 static bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }

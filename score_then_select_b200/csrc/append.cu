@@ -646,8 +646,7 @@ static cudaError_t launch_rankr(const Plan& p, const AppendParams& a, cudaStream
   constexpr int NT = 64 * R / 16;
   const size_t smem = size_t(D) * R * 4 + size_t(D) * 64 * 4;
   auto k = append_rankr_kernel<PT, R, D>;
-  static const cudaError_t attr =
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  const cudaError_t attr = set_smem_limit(k, int(smem));
   if (attr != cudaSuccess) return attr;
   dim3 grid((a.max_new + 63) / 64, a.batch * a.Hkv);
   k<<<grid, NT, smem, s>>>(a);

@@ -606,8 +606,7 @@ static cudaError_t launch_attn_t(const AttnParams& a, const CUtensorMap& mk, con
                                  int grid, cudaStream_t s, bool pdl) {
   auto k = attn_kernel<D, VF, AF>;
   const int smem = AttnSmem<D>::kTotal;
-  static const cudaError_t attr =
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const cudaError_t attr = set_smem_limit(k, smem);
   if (attr != cudaSuccess) return attr;
   cudaError_t e = launch_k(k, dim3(grid), dim3(kAttnThreads), smem, s, pdl, a, mk, mv);
   if (e != cudaSuccess) return e;

@@ -308,8 +308,7 @@ template <int D, bool VF, bool AF>
 static cudaError_t launch_gather_t(const AttnParams& a, cudaStream_t s, bool pdl) {
   auto k = attn_gather_kernel<D, VF, AF>;
   const int smem = GatherSmem<D>::kTotal;
-  static const cudaError_t attr =
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const cudaError_t attr = set_smem_limit(k, smem);
   if (attr != cudaSuccess) return attr;
   return launch_k(k, dim3(a.gsplits, a.rows), dim3(128), smem, s, pdl, a);
 }

@@ -218,8 +218,7 @@ cudaError_t launch_calibrate(const CalibParams& a, cudaStream_t s) {
            size_t(dd / 2) * 2 * 4 + 64 * 8 + size_t(dd) * 4;
   };
   const size_t smem = bytes(d);                     // 194.5 KiB at d = 128
-  static const cudaError_t attr = cudaFuncSetAttribute(
-      basis_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes(128)));
+  const cudaError_t attr = set_smem_limit(basis_kernel, int(bytes(128)));
   if (attr != cudaSuccess) return attr;
   basis_kernel<<<a.Hkv, kBasisThreads, smem, s>>>(a);
   return cudaGetLastError();

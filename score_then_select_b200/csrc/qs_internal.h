@@ -253,7 +253,16 @@ cudaError_t launch_gather_kv(const Plan& p, const GatherParams& a, cudaStream_t 
 cudaError_t launch_calibrate(const CalibParams& a, cudaStream_t s);
 size_t calib_ws_bytes(int Hkv, int d);
 
-int num_sms();
+int num_sms();   // SM count of the current device (cached per device)
+
+// Raise `kern`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device): function attributes are per device, and one process may drive several
+// GPUs. Thread-safe.
+cudaError_t set_smem_limit(const void* kern, int bytes);
+template <typename... P>
+inline cudaError_t set_smem_limit(void (*kern)(P...), int bytes) {
+  return set_smem_limit(reinterpret_cast<const void*>(kern), bytes);
+}
 
 // host-side validation and launch planning (api.cu)
 qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p);

@@ -268,12 +268,13 @@ static cudaError_t launch_rankr_score(const ScoreParams& a, cudaStream_t st, boo
                           size_t(kMaxBatch + 1) * sizeof(int);
   const size_t smem = smem_max - size_t(kMaxBatch - a.batch) * sizeof(int);
   auto k = score_rankr_kernel<PT, R>;
-  // one-time per-process kernel attributes (sized for the largest batch)
-  static int per_sm = [&] {
+  // the shared-memory limit is set once per device (sized for the largest batch); the
+  // resident CTAs per SM follow from it and are the same on every B200
+  const cudaError_t attr = set_smem_limit(k, int(smem_max));
+  if (attr != cudaSuccess) return attr;
+  static const int per_sm = [&] {
     int n = 0;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max)) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kScoreThreads, smem_max) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kScoreThreads, smem_max) != cudaSuccess)
       n = 0;
     return n;
   }();

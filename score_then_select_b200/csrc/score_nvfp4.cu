@@ -333,8 +333,7 @@ cudaError_t launch_score_nvfp4(const Plan& p, const ScoreParams& a, cudaStream_t
                           size_t(kMaxBatch + 1) * sizeof(int);
   const size_t smem = smem_max - size_t(kMaxBatch - a.batch) * sizeof(int);
   auto k = score_nvfp4_kernel;
-  static const cudaError_t attr =
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
+  const cudaError_t attr = set_smem_limit(k, int(smem_max));
   if (attr != cudaSuccess) return attr;
   // kF4CtasPerSm CTAs per SM, each with its share of the SM's tensor memory
   const long long units = (long long)a.batch * a.Hkv * ((a.max_context + kPage - 1) / kPage);
