@@ -108,17 +108,9 @@ QS_DEV void cp_async_mbar_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
-// Barrier among `nthreads` threads (whole warps) of the CTA on hardware barrier `id`.
-QS_DEV void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // ---------------------------------------------------------------- cp.async (16 bytes)
-QS_DEV void cp_async16(void* dst_smem, const void* src_gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)),
-               "l"(src_gmem)
-               : "memory");
-}
+// 16-byte copy into shared memory; `valid` false writes zeros (source size 0)
 QS_DEV void cp_async16_zfill(void* dst_smem, const void* src_gmem, bool valid) {
   // src-size 0 writes 16 zero bytes without reading global memory
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)),
@@ -271,19 +263,6 @@ QS_DEV float warp_min(float v) {
   for (int m = 16; m > 0; m >>= 1) v = fminf(v, __shfl_xor_sync(kFull, v, m));
   return v;
 }
-QS_DEV int warp_sum(int v) {
-#pragma unroll
-  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
-  return v;
-}
 
-// 16-byte vector load through the non-coherent path
-QS_DEV uint4 ldg_nc_v4(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
 
 }  // namespace qs
