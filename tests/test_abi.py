@@ -145,3 +145,27 @@ def test_kept_blocks_limited_to_one_cta_rows():
     with pytest.raises(qs.QsError) as e:
         qs.qs_workspace_size(cfg, 1, 128 * 32768 + 1)
     assert e.value.status == B.QS_ERR_UNSUPPORTED
+
+
+def _prototypes():
+    """{name: number of parameters} of every entry point declared in include/qs.h."""
+    out = {}
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        txt = open(os.path.join(ROOT, "include", fn)).read()
+        txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+        for m in re.finditer(r"\b(qs_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", txt):
+            params = m.group(2).strip()
+            out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    L = qs.lib()
+    protos = _prototypes()
+    assert set(protos) == set(_declared())
+    for name, n in protos.items():
+        f = getattr(L, name)
+        assert f.argtypes is not None, f"{name}: no argtypes in the binding"
+        assert len(f.argtypes) == n, f"{name}: header has {n} parameters, binding {len(f.argtypes)}"
