@@ -71,7 +71,9 @@ def _scores(kind, rng, n):
 KINDS = ["normal", "ties", "equal", "signed_zero", "nonfinite", "extreme", "clustered"]
 # (block size, budget, max_context, forced sink / last): 1,024 / 4,096 / 32,768 / 131,072 blocks
 SHAPES = [(128, 64, 131072, True), (32, 100, 131072, False), (1, 2048, 32768, False),
-          (1, 500, 32768, True), (1, 2048, 131072, False), (1, 3000, 131072, True)]
+          (1, 500, 32768, True), (1, 2048, 131072, False), (1, 3000, 131072, True),
+          # forced blocks fill the budget: only the sink and the last block are selected
+          (128, 2, 131072, True), (1, 2, 131072, True)]
 
 
 def _run(shape, kind, seed):
