@@ -216,6 +216,7 @@ def qs_sparse_attn_noalloc(cfg, cache, q, sel, n_sel, batch, out, stream=None):
 
 
 def qs_dense_workspace_size(cfg: qs_config, batch: int, max_context: int) -> int:
+    """Workspace bytes qs_dense_attn needs for caches of up to max_context tokens."""
     n = ctypes.c_size_t(0)
     _check(lib().qs_dense_workspace_size(ctypes.byref(cfg), batch, max_context, ctypes.byref(n)),
            "qs_dense_workspace_size")
@@ -223,17 +224,23 @@ def qs_dense_workspace_size(cfg: qs_config, batch: int, max_context: int) -> int
 
 
 def qs_dense_attn(cfg, cache, q, row_lens, batch, out, ws, stream=None):
+    """Full-KV attention over every valid token of each row: q [batch][Hq][d] BF16, row_lens
+    [batch * Hkv] int32 or None (then seq_lens[b]), out [batch][Hq][d]."""
     _check(lib().qs_dense_attn(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(row_lens),
                                batch, _ptr(out), _ptr(ws), _stream(stream)), "qs_dense_attn")
 
 
 def qs_gather_kv(cfg, cache, sel, n_sel, batch, k_dst, v_dst, row_lens, ws, stream=None):
+    """Copy each row's selected blocks into compact pages k_dst / v_dst [batch * P][Hkv][128][d]
+    (P = ceil(budget * block_size / 128)) and write the valid lengths to row_lens
+    [batch * Hkv] (the first half of gather-then-attend)."""
     _check(lib().qs_gather_kv(ctypes.byref(cfg), ctypes.byref(cache), _ptr(sel), _ptr(n_sel),
                               batch, _ptr(k_dst), _ptr(v_dst), _ptr(row_lens), _ptr(ws),
                               _stream(stream)), "qs_gather_kv")
 
 
 def qs_calib_workspace_size(cfg: qs_config) -> int:
+    """Workspace bytes qs_calibrate_basis needs (2 * Hkv * d * d FP64 moments + 256)."""
     n = ctypes.c_size_t(0)
     _check(lib().qs_calib_workspace_size(ctypes.byref(cfg), ctypes.byref(n)),
            "qs_calib_workspace_size")
@@ -241,6 +248,8 @@ def qs_calib_workspace_size(cfg: qs_config) -> int:
 
 
 def qs_calibrate_basis(cfg, q, k, n, P, eigvals, ws, stream=None):
+    """The scoring basis P [Hkv][d][r] FP32 from n calibration positions: q [n][Hq][d] and
+    k [n][Hkv][d] BF16; eigvals [Hkv][r] FP32 or None. r = cfg.proxy_rank."""
     _check(lib().qs_calibrate_basis(ctypes.byref(cfg), _ptr(q), _ptr(k), n, _ptr(P),
                                     _ptr(eigvals), _ptr(ws), _stream(stream)),
            "qs_calibrate_basis")
