@@ -245,6 +245,28 @@ def lse_combine(ms, ls, os_) -> np.ndarray:
 
 
 # ============================================================================================
+# Attending over the NVFP4 keys  [JQS, Full text]
+# The storage variant of the page keeps the attended keys in NVFP4 too, with at most two
+# blocks per sequence kept in BF16 to bound the quantisation error. Reading: the key of a
+# token in a kept block is its stored BF16 key; every other key is its NVFP4 scoring copy
+# decoded and un-centred (dequantised value + the row's calibrated mean). Not yet built on
+# the GPU; defined here so that a kernel can be checked against it.
+# ============================================================================================
+
+
+def nvfp4_attended_keys(k_bits: np.ndarray, codes: np.ndarray, scales: np.ndarray, g_k,
+                        mu: np.ndarray, keep, S: int, L: int) -> np.ndarray:
+    """Keys [L][d] (float64) the storage variant attends over: BF16 keys in kept blocks,
+    dequant(codes, scales, g_k) + mu elsewhere."""
+    K = nvfp4_dequant(codes[:L], scales[:L], g_k) + np.asarray(mu, dtype=np.float32).astype(np.float64)
+    bf = F.bf16_to_f64(k_bits[:L])
+    for j in keep:
+        t0, t1 = int(j) * S, min(L, (int(j) + 1) * S)
+        K[t0:t1] = bf[t0:t1]
+    return K
+
+
+# ============================================================================================
 # Centroid scoring of contiguous blocks  ["Coarse Semantic Blocks ...", Abstract]
 # The page scores each block by its centroid against the query. Reading: the centroid of a
 # block is the mean of its valid stored keys, kept as a float32 running sum in token order

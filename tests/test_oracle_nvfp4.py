@@ -120,3 +120,49 @@ def test_kept_blocks_exhaustive(seed):
 def test_query_scale():
     q = F.f32_to_bf16_rne(np.array([[0.5, -3.0], [2.0, 1.0]], dtype=np.float32))
     assert M.query_scale(q) == np.float32(np.float32(3.0) / np.float32(2688.0))
+
+
+# ---------------------------------------------------------------- attending over NVFP4 keys
+
+def _nvfp4_row(rng, L, d=128):
+    kb = F.f32_to_bf16_rne(rng.standard_normal((L, d)).astype(np.float32) * 2)
+    mu = rng.standard_normal(d).astype(np.float32) * 0.1
+    x32 = M.centre(kb, mu)
+    g_k = np.float32(np.abs(x32).max() / (6.0 * 448.0))
+    codes, scales = M.nvfp4_pack(x32, g_k)
+    return kb, mu, x32, g_k, codes, scales
+
+
+def test_attended_keys_use_bf16_in_kept_blocks_only():
+    rng = np.random.default_rng(60)
+    S, L = 16, 70
+    kb, mu, x32, g_k, codes, scales = _nvfp4_row(rng, L)
+    K = M.nvfp4_attended_keys(kb, codes, scales, g_k, mu, [1, 4], S, L)
+    bf = F.bf16_to_f64(kb)
+    deq = M.nvfp4_dequant(codes, scales, g_k) + mu.astype(np.float64)
+    for t in range(L):
+        want = bf[t] if t // S in (1, 4) else deq[t]
+        assert np.array_equal(K[t], want), t
+    # the cut last block (4: tokens 64..69) is kept whole up to L
+    assert np.array_equal(K[64:70], bf[64:70])
+
+
+def test_attended_keys_all_kept_is_bf16_attention():
+    rng = np.random.default_rng(61)
+    S, L = 8, 40
+    kb, mu, x32, g_k, codes, scales = _nvfp4_row(rng, L)
+    K = M.nvfp4_attended_keys(kb, codes, scales, g_k, mu, range(5), S, L)
+    assert np.array_equal(K, F.bf16_to_f64(kb))
+
+
+def test_attended_keys_error_within_the_nvfp4_bound():
+    # away from kept blocks each key differs from the float32 key by at most the per-element
+    # NVFP4 bound: half the largest E2M1 step (2 at magnitude 4..6) times sigma * g_k, plus
+    # the float32 rounding of the centring
+    rng = np.random.default_rng(62)
+    S, L, d = 16, 64, 128
+    kb, mu, x32, g_k, codes, scales = _nvfp4_row(rng, L, d)
+    K = M.nvfp4_attended_keys(kb, codes, scales, g_k, mu, [], S, L)
+    sig = F.ue4m3_value(scales).repeat(16, axis=1) * np.float64(g_k)
+    err = np.abs(K - F.bf16_to_f64(kb))
+    assert np.all(err <= 1.0 * sig + 1e-6 * np.abs(F.bf16_to_f64(kb)) + 1e-7)
