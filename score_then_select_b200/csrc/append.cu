@@ -3,8 +3,11 @@
 // Rank-r writer ("Joint Subspace Sparse Attention for Efficient Long-Context Decoding",
 // Figure 1): the projected-key cache entry of a new token is k . P[g], evaluated in float32
 // in ascending index order with one rounding per product and per sum (no fused
-// multiply-add), then stored as float32 or rounded to nearest-even BF16 (Figure 10 allows
-// a reduced-precision scoring cache).
+// multiply-add), then stored as float32, or rounded to nearest-even BF16 or FP8 E4M3
+// (saturating at +-448; Figure 10 keeps the scoring cache at FP8 or BF16).
+//
+// Centroid writer ("Coarse Semantic Blocks ...", Abstract): each block's FP32 key sum,
+// continued in token order.
 //
 // NVFP4 writer ("Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse
 // Attention", Full text): the persistent scoring cache is packed straight from the BF16
