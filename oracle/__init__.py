@@ -16,7 +16,12 @@ Pins (what each part is checked against, in tests/test_oracle_*.py):
               every block; one-hot selection; split-count invariance of the LSE combine;
   NVFP4     - factored block-scaled dot product against dequantise-then-dot; exactly
               representable round trips; the per-element error bound; kept blocks by
-              exhaustive search; planted needle selected.
+              exhaustive search; planted needle selected;
+  binary    - an exactly representable rotated case whose estimate is the exact score; the
+              mean over random rotations and query roundings against the exact score
+              (unbiasedness); identity and signed-permutation rotations; bit packing;
+  top-p     - exhaustive subset search on tiny inputs; closed forms for uniform and
+              geometric masses; the budget cap; forced blocks.
 Parity unpinned: the aggregation of per-head NVFP4 scores into one block score (max over
 the group's heads) is a reading the pages leave open; only its implementation is pinned.
 """

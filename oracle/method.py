@@ -22,12 +22,21 @@ Sources (page title, then the part of the page):
           - Full text: NVFP4 cache; a dense FP4 scan scores the whole key history; 128-token
             blocks are selected; FP16 value aggregation with FP32 accumulation; calibrated
             key centring; at most two BF16 pages kept; cache packed from BF16 activations.
+  [RQC]   "RaBitQCache" (the abstract page)
+          - Abstract: keys scored through randomised rotated binary quantisation with
+            binary-INT4 arithmetic, an unbiased estimator with an error bound, and a top-p
+            budget that follows the estimated attention mass.
+  [RBQ]   The estimator's published form: J. Gao and C. Long, "RaBitQ: Quantizing
+          High-Dimensional Vectors with a Theoretical Error Bound for Approximate Nearest
+          Neighbor Search", SIGMOD 2024 (section 3: the codebook, the estimator and its
+          unbiasedness; the randomised uniform scalar quantisation of the query).
 
 Readings where the pages are silent (each listed in the design notes):
   * block score = max over the block's valid tokens (and, on the NVFP4 path, over the
     group's query heads); the proxy scores are unscaled (scaling does not change order);
   * forced blocks (sink, last, kept) count against the budget; ties go to the lower index;
-  * attention is exact softmax over the selected tokens only.
+  * attention is exact softmax over the selected tokens only;
+  * the binary proxy's readings are listed above its section.
 
 Parity pins live in tests/test_oracle_*.py. The aggregation of per-head NVFP4 scores into
 one score per block (max over heads) is a reading the pages do not fix: its *definition*
@@ -464,3 +473,195 @@ def kept_blocks(err: np.ndarray, n_keep: int) -> np.ndarray:
     valid = np.nonzero(np.isfinite(err))[0]
     order = np.lexsort((valid, -err[valid]))
     return np.sort(valid[order[:n_keep]])
+
+
+# ============================================================================================
+# Binary proxy with an adaptive top-p budget  [RQC, Abstract; RBQ]
+# The page scores every cached key with a 1-bit code of its randomly rotated direction and
+# an INT4 code of the rotated query, and lets the attended set grow until the estimated
+# attention mass reaches p. The estimator is the published RaBitQ one [RBQ]:
+#   o = k - c (the row's centre c), y = o R (R a random d x d rotation, its columns the
+#   rotated axes), code bits b_i = [y_i > 0], x_i = (2 b_i - 1) / sqrt(d);
+#   <o, q> ~= |o| <x, q R> / <x, y / |o|> = (|o|^2 / |y|_1) sum_i (2 b_i - 1) (q R)_i.
+# Over a uniformly random rotation the ratio is an unbiased estimate of <o, q>, and
+# rounding each rotated query entry to the 4-bit grid at random (floor(t + u), u uniform)
+# keeps it unbiased. Readings (the pages give no more than the abstract):
+#   * the query is the mean of the group's query heads, the centre one vector per row;
+#   * the estimated score of token t is g_t sum_i (2 b_i - 1)(Delta n_i + v_l) + <c, qbar>;
+#   * the estimated attention weights are softmax(scale * score) over the row's valid
+#     tokens; a block's mass is the sum of its tokens' weights (S = 1: token level);
+#   * forced blocks are taken first and count toward the mass; the rest follow in order of
+#     decreasing mass (ties: lower index) until the taken mass reaches p, or the budget
+#     (the largest number of blocks a row may attend) is full.
+# The stored code bits, g_t and the query's codes are decided in float32 in a fixed order
+# (as the CUDA writer and scan compute them), so they compare bit for bit; scores, weights
+# and masses are float64.
+# ============================================================================================
+
+RQ_QUERY_BITS = 4
+RQ_QUERY_LEVELS = (1 << RQ_QUERY_BITS) - 1           # codes 0 .. 15
+
+
+def _rotate_f32(x32: np.ndarray, R: np.ndarray) -> np.ndarray:
+    """y = x R in float32: y_i = sum over j ascending of fp32(x_j * R_ji), each product and
+    each partial sum rounded (no fused multiply-add). x32: [n][d]; R: float32 [d][d]."""
+    x32 = np.asarray(x32, dtype=np.float32)
+    R32 = np.asarray(R, dtype=np.float32)
+    acc = np.zeros((x32.shape[0], R32.shape[1]), dtype=np.float32)
+    for j in range(x32.shape[1]):
+        acc = acc + x32[:, j:j + 1] * R32[j:j + 1, :]
+    return acc
+
+
+def _f32_sum_seq(x32: np.ndarray) -> np.ndarray:
+    """Row sums of a float32 [n][m] array, added left to right with a rounding per step."""
+    acc = np.zeros(x32.shape[0], dtype=np.float32)
+    for j in range(x32.shape[1]):
+        acc = acc + x32[:, j]
+    return acc
+
+
+def rabitq_encode(k_bits: np.ndarray, R: np.ndarray, c: np.ndarray):
+    """Binary codes of keys [n][d] (BF16): bits [n][d] (0/1, uint8) and g [n] (float32).
+
+    o = fp32(k) - c (rounded float32); y = o R (_rotate_f32); b_i = [y_i > 0];
+    g = fp32(fp32 sum_j o_j^2 / fp32 sum_i |y_i|) with both sums taken left to right in
+    float32, and g = 0 where sum |y_i| = 0 (a key equal to the centre).
+    """
+    o = centre(k_bits, c)
+    y = _rotate_f32(o, R)
+    bits = (y > 0).astype(np.uint8)
+    n2 = _f32_sum_seq((o * o).astype(np.float32))
+    l1 = _f32_sum_seq(np.abs(y))
+    safe = np.where(l1 > 0, l1, np.float32(1.0))
+    g = np.where(l1 > 0, (n2 / safe).astype(np.float32), np.float32(0.0)).astype(np.float32)
+    return bits, g
+
+
+def rabitq_pack_bits(bits: np.ndarray) -> np.ndarray:
+    """Stored code: bit i of a key in byte i // 8, at bit position i % 8 -> [n][d / 8] uint8."""
+    return np.packbits(np.asarray(bits, dtype=np.uint8), axis=-1, bitorder="little")
+
+
+def rabitq_unpack_bits(packed: np.ndarray, d: int) -> np.ndarray:
+    return np.unpackbits(np.asarray(packed, dtype=np.uint8), axis=-1, count=d,
+                         bitorder="little")
+
+
+def rabitq_query(q_bits: np.ndarray, R: np.ndarray, u: np.ndarray):
+    """The rotated group-mean query and its 4-bit code, all in float32.
+
+    qbar_j = fp32(sum over heads in order of fp32(q_h,j)) / G (a rounded division);
+    q' = qbar R (_rotate_f32); v_l = min q', v_r = max q';
+    Delta = fp32(fp32(v_r - v_l) / 15); n_i = min(15, floor(fp32(fp32(fp32(q'_i - v_l) /
+    Delta) + u_i))), with n = 0 everywhere when Delta = 0. u [d]: uniform draws in [0, 1).
+    Returns (n [d] int64, Delta, v_l, qbar [d] float32).
+    """
+    q32 = F.bf16_to_f64(q_bits).astype(np.float32)
+    acc = np.zeros(q32.shape[1], dtype=np.float32)
+    for h in range(q32.shape[0]):
+        acc = acc + q32[h]
+    qbar = (acc / np.float32(q32.shape[0])).astype(np.float32)
+    qr = _rotate_f32(qbar[None, :], R)[0]
+    vl, vr = np.float32(qr.min()), np.float32(qr.max())
+    delta = np.float32(np.float32(vr - vl) / np.float32(RQ_QUERY_LEVELS))
+    if delta == 0:
+        return np.zeros(qr.shape[0], dtype=np.int64), delta, vl, qbar
+    t = ((qr - vl).astype(np.float32) / delta).astype(np.float32)
+    n = np.floor((t + np.asarray(u, dtype=np.float32)).astype(np.float32)).astype(np.int64)
+    return np.minimum(n, RQ_QUERY_LEVELS), delta, vl, qbar
+
+
+def rabitq_scores(bits: np.ndarray, g: np.ndarray, n: np.ndarray, delta, vl, c: np.ndarray,
+                  qbar: np.ndarray) -> np.ndarray:
+    """Estimated scores [n_keys] (float64): g_t sum_i (2 b_ti - 1)(Delta n_i + v_l) + <c, qbar>."""
+    qhat = np.float64(delta) * np.asarray(n, dtype=np.float64) + np.float64(vl)
+    sgn = 2.0 * np.asarray(bits, dtype=np.float64) - 1.0
+    shift = float(np.asarray(c, dtype=np.float64) @ np.asarray(qbar, dtype=np.float64))
+    return np.asarray(g, dtype=np.float64) * (sgn @ qhat) + shift
+
+
+def estimated_weights(s: np.ndarray, scale: float) -> np.ndarray:
+    """softmax(scale * s) over the given (valid) tokens, float64."""
+    x = scale * np.asarray(s, dtype=np.float64)
+    e = np.exp(x - x.max())
+    return e / e.sum()
+
+
+def block_mass(w: np.ndarray, S: int) -> np.ndarray:
+    """Sum of the weights of each block's valid tokens -> [ceil(L / S)]."""
+    L = w.shape[0]
+    nb = (L + S - 1) // S
+    pad = np.zeros(nb * S - L)
+    return np.concatenate([w, pad]).reshape(nb, S).sum(axis=1)
+
+
+def select_top_p(mass: np.ndarray, p: float, budget: int, forced: np.ndarray) -> np.ndarray:
+    """Indices (ascending) of the forced blocks plus the fewest highest-mass others whose
+    total mass, with the forced blocks', reaches p of the row's mass; at most ``budget``.
+
+    Requires 0 < p <= 1 and |forced| <= budget. Blocks are added in order of decreasing
+    mass, ties to the lower index; the running mass is summed in the order taken (forced
+    blocks first, ascending) and compared with p * (sum of all masses).
+    """
+    if not (0.0 < p <= 1.0):
+        raise ValueError("p must be in (0, 1]")
+    forced = np.unique(np.asarray(forced, dtype=np.int64))
+    if len(forced) > budget:
+        raise ValueError("more forced blocks than the budget")
+    nb = mass.shape[0]
+    goal = p * float(mass.sum())
+    taken = [int(j) for j in forced]
+    acc = 0.0
+    for j in taken:
+        acc += float(mass[j])
+    is_forced = np.zeros(nb, dtype=bool)
+    is_forced[forced] = True
+    rest = np.nonzero(~is_forced)[0]
+    for j in rest[np.lexsort((rest, -mass[rest]))]:
+        if len(taken) >= budget or acc >= goal:
+            break
+        taken.append(int(j))
+        acc += float(mass[j])
+    return np.sort(np.array(taken, dtype=np.int64))
+
+
+def top_p_valid(mass: np.ndarray, p: float, budget: int, forced: np.ndarray, got: np.ndarray,
+                rel_tol: float = 1e-4) -> tuple[bool, str]:
+    """Is ``got`` a valid top-p selection, up to rounding of the masses and the goal?
+
+    Valid iff it is strictly ascending, in range, holds every forced block and at most
+    ``budget`` blocks; its non-forced blocks are the highest-mass ones up to near-ties
+    (relative band rel_tol at the last one taken); and its size is right: either the goal
+    p * total is reached (within rel_tol of the total) and dropping the lightest non-forced
+    block would miss it, or the budget is full without reaching it.
+    """
+    got = np.asarray(got, dtype=np.int64)
+    nb = mass.shape[0]
+    forced = np.unique(np.asarray(forced, dtype=np.int64))
+    if np.any(np.diff(got) <= 0):
+        return False, "not strictly ascending"
+    if got.size and (got[0] < 0 or got[-1] >= nb):
+        return False, "index out of range"
+    if not set(forced.tolist()) <= set(got.tolist()):
+        return False, "forced block missing"
+    if len(got) > budget:
+        return False, f"{len(got)} blocks over the budget {budget}"
+    total = float(mass.sum())
+    tol = rel_tol * total
+    goal = p * total
+    extra = np.setdiff1d(got, forced)
+    others = np.setdiff1d(np.arange(nb), got)
+    if extra.size and others.size:
+        lightest = float(mass[extra].min())
+        band = rel_tol * max(abs(lightest), 1e-300)
+        if float(mass[others].max()) > lightest + band:
+            return False, "an unchosen block outweighs a chosen one"
+    have = float(mass[got].sum())
+    if have >= goal - tol:
+        if extra.size and have - float(mass[extra].min()) >= goal + tol:
+            return False, "not minimal: the goal is met without the lightest block"
+        return True, "goal reached"
+    if len(got) == budget or others.size == 0:
+        return True, "budget full"
+    return False, f"mass {have} short of the goal {goal}"

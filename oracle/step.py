@@ -94,3 +94,37 @@ def decode_row(p: RowParams, k_bits, v_bits, q_bits, L: int, P=None, mu=None, g_
     out = M.sparse_attention(q, K, V, tokens, p.scale)
     return dict(cache=cache, beta=beta, forced=forced, keep=keep, sel=sel, tokens=tokens,
                 out=out)
+
+
+# ---- the binary proxy with a top-p budget ("RaBitQCache", Abstract) ------------------------
+
+@dataclass
+class TopPParams:
+    S: int                     # block size (1: token level)
+    p: float                   # fraction of the estimated attention mass to cover
+    budget: int                # most blocks a row may attend
+    scale: float               # softmax scale (estimated weights and attention)
+    v_dtype: str               # 'bf16' | 'f16'
+    force_sink: bool = False
+    force_last: bool = False
+
+
+def decode_row_top_p(p: TopPParams, k_bits, v_bits, q_bits, L: int, R, c, u,
+                     sel_override=None):
+    """One row's step with the binary proxy: codes of the keys, the query's 4-bit code,
+    estimated scores and weights, block masses, the top-p selection, then exact attention
+    over the selected tokens. R: rotation [d][d]; c: the row's centre [d]; u: the query's
+    rounding draws [d]."""
+    bits, g = M.rabitq_encode(k_bits[:L], R, c)
+    n, delta, vl, qbar = M.rabitq_query(q_bits, R, u)
+    s = M.rabitq_scores(bits, g, n, delta, vl, c, qbar)
+    w = M.estimated_weights(s, p.scale)
+    mass = M.block_mass(w, p.S)
+    forced = M.forced_blocks(mass.shape[0], p.force_sink, p.force_last)
+    sel = M.select_top_p(mass, p.p, p.budget, forced)
+    use = sel if sel_override is None else np.asarray(sel_override, dtype=np.int64)
+    tokens = M.block_tokens(use, p.S, L)
+    out = M.sparse_attention(F.bf16_to_f64(q_bits), F.bf16_to_f64(k_bits[:L]),
+                             decode_v(v_bits[:L], p.v_dtype), tokens, p.scale)
+    return dict(bits=bits, g=g, codes=n, delta=delta, vl=vl, qbar=qbar, scores=s, weights=w,
+                mass=mass, forced=forced, sel=sel, tokens=tokens, out=out)
