@@ -23,6 +23,12 @@
  *     Full text: NVFP4 scoring keys scanned densely on FP4 tensor cores; 128-token blocks;
  *     FP16 value aggregation with FP32 accumulation; calibrated key centring; at most two
  *     blocks kept at BF16 per sequence; the cache is packed directly from BF16 activations.
+ *   "RaBitQCache" (Abstract): keys scored through randomly rotated binary codes with
+ *     binary-INT4 arithmetic (an unbiased estimate of q . k) and a top-p budget that grows
+ *     the attended set until the estimated attention mass reaches p. The estimator is the
+ *     published RaBitQ one: J. Gao and C. Long, "RaBitQ: Quantizing High-Dimensional
+ *     Vectors with a Theoretical Error Bound for Approximate Nearest Neighbor Search",
+ *     SIGMOD 2024, section 3.
  *
  * Conventions (all entry points):
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise; the caller owns
@@ -59,15 +65,21 @@
  *   proxy_scale     [num_pages][Hkv][page_size][head_dim/16] u8: UE4M3 scale per 16 elems
  *   proxy (centroid)[num_pages][Hkv][page_size/S][head_dim] F32: the sum of the keys of each
  *                                                           S-token block of the page
+ *   proxy (binary)  [num_pages][Hkv] x (page_size * head_dim/8 bytes of code bits, then
+ *                                       page_size F32 factors g): token slot s has bits
+ *                                       at byte s * head_dim/8 (bit i of the key in byte
+ *                                       i / 8, position i % 8) and g at index s
  *   page_table      [batch][max_pages_per_seq]              int32 physical page ids
  *   seq_lens        [batch]                                 int32 tokens in the cache
  *   P               [Hkv][head_dim][r]                      F32
+ *   R (binary)      [Hkv][head_dim][head_dim]               F32 rotation, y = x . R
  *   q, out          [batch][Hq][head_dim]                   q BF16; out F32 or BF16
  *   k_new, v_new    [batch][Hkv][max_new][head_dim]         K BF16, V as v_dtype
  *   block scores    [batch][Hkv][nb_stride]  F32, nb_stride = ceil(max_context / page_size)
  *                                                                 * (page_size / block_size)
  *   sel             [batch][Hkv][budget]     int32 ascending block ids, padded with -1
  *   n_sel           [batch][Hkv]             int32 = min(budget, ceil(seq_len / block_size))
+ *                                            (top-p: the number of blocks taken)
  * Query head h belongs to KV head h / (Hq / Hkv).
  */
 #ifndef QS_H
@@ -93,7 +105,8 @@ typedef enum {
 
 typedef enum {
   QS_F32 = 0, QS_BF16 = 1, QS_F16 = 2, QS_NVFP4 = 3, QS_E4M3 = 4,
-  QS_CENTROID = 5   /* proxy_dtype only: per-block FP32 key sums (centroid scoring), r = 0 */
+  QS_CENTROID = 5,  /* proxy_dtype only: per-block FP32 key sums (centroid scoring), r = 0 */
+  QS_RABITQ = 6     /* proxy_dtype only: binary codes of rotated centred keys, r = 0      */
 } qs_dtype;
 
 /* Problem statement of one attention layer's decode step. */
@@ -104,8 +117,9 @@ typedef struct {
   int32_t page_size;      /* tokens per cache page: 128                                   */
   int32_t block_size;     /* S: a power of two dividing page_size (1 = token level)       */
   int32_t budget;         /* k: blocks selected per row, >= 1                             */
-  int32_t proxy_rank;     /* r > 0: projected-key proxy; 0: NVFP4 centred keys            */
-  int32_t proxy_dtype;    /* qs_dtype: F32, BF16 or E4M3 (rank r); NVFP4 or CENTROID (r 0) */
+  int32_t proxy_rank;     /* r > 0: projected-key proxy; 0: NVFP4, centroid or binary     */
+  int32_t proxy_dtype;    /* qs_dtype: F32, BF16 or E4M3 (rank r); NVFP4, CENTROID or
+                             RABITQ (r 0)                                                 */
   int32_t v_dtype;        /* qs_dtype of stored V: BF16 or F16                            */
   int32_t v_agg_dtype;    /* precision of the P.V operands: BF16 or F16 (FP32 accumulate) */
   int32_t out_dtype;      /* F32 or BF16                                                  */
@@ -129,7 +143,7 @@ typedef struct {
   uint8_t *proxy_scale;       /* NVFP4 only: UE4M3 scales; NULL otherwise                 */
   float *block_err;           /* NVFP4 only: [batch][Hkv][nb_stride] squared quantisation
                                  error of each complete block (written by qs_append_kv)   */
-  const float *key_center;    /* NVFP4 only: [batch][Hkv][d] calibrated centring mean     */
+  const float *key_center;    /* NVFP4 and binary proxy: [batch][Hkv][d] centring mean    */
   const float *key_gscale;    /* NVFP4 only: 1 float, the key tensor scale g_k            */
   const int32_t *page_table;  /* [batch][max_pages_per_seq]                               */
   int32_t *seq_lens;          /* [batch]; advanced by qs_append_kv / qs_decode            */
@@ -164,8 +178,13 @@ qs_status qs_workspace_init(void *ws, size_t ws_bytes, qs_stream_t stream);
      NVFP4:  x = float(k) - key_center[b][g] (float32), packed per 16 elements to UE4M3
              scale + E2M1 codes with the tensor scale g_k; each block of S tokens that this
              call completes gets block_err = sum of squared (x - dequant(x)).
+     binary: o = float(k) - key_center[b][g] (float32), y = o . R[g] (R passed as P; y_i
+             summed over j ascending, one rounding per product and per sum), code bits
+             b_i = [y_i > 0] and g = fp32(sum_j o_j^2) / fp32(sum_i |y_i|) (both sums left to
+             right; 0 when the second is 0): the RaBitQ code ("RaBitQCache", Abstract).
    k_new/v_new: [batch][Hkv][max_new][d]; n_new: device int32 [batch], each <= max_new;
-   P: [Hkv][d][r] (NULL for NVFP4). Pages for the new tokens must be in page_table. */
+   P: [Hkv][d][r] (NULL for NVFP4 and centroid; R [Hkv][d][d] for the binary proxy).
+   Pages for the new tokens must be in page_table. */
 qs_status qs_append_kv(const qs_config *cfg, const qs_cache *cache, const void *k_new,
                        const void *v_new, const int32_t *n_new, int32_t max_new,
                        const float *P, int32_t batch, void *ws, qs_stream_t stream);
@@ -183,7 +202,8 @@ qs_status qs_append_kv(const qs_config *cfg, const qs_cache *cache, const void *
            block's valid tokens.
    Blocks past ceil(seq_len / S) that share a page with valid tokens are written -inf;
    entries past the last page of a row are not written.
-   q: [batch][Hq][d] BF16; P as in qs_append_kv; block_scores: [batch][Hkv][nb_stride]. */
+   q: [batch][Hq][d] BF16; P as in qs_append_kv; block_scores: [batch][Hkv][nb_stride].
+   The binary proxy needs its rounding draws: qs_rabitq_score (QS_ERR_UNSUPPORTED here). */
 qs_status qs_score(const qs_config *cfg, const qs_cache *cache, const void *q,
                    const float *P, int32_t batch, float *block_scores, void *ws,
                    qs_stream_t stream);
@@ -211,11 +231,48 @@ qs_status qs_sparse_attn(const qs_config *cfg, const qs_cache *cache, const void
 
 /* One decode step: append one token per sequence (k_new/v_new: [batch][Hkv][d]), then
    score, select and attend over seq_len + 1 tokens. sel_out / n_sel_out may be NULL; the
-   selection then stays in the workspace. */
+   selection then stays in the workspace. The binary proxy with its top-p budget runs as
+   separate calls (qs_append_kv, qs_rabitq_score, qs_select_top_p, qs_sparse_attn); this
+   call returns QS_ERR_UNSUPPORTED for it. */
 qs_status qs_decode(const qs_config *cfg, const qs_cache *cache, const void *q,
                     const void *k_new, const void *v_new, const float *P, int32_t batch,
                     void *out, int32_t *sel_out, int32_t *n_sel_out, void *ws,
                     qs_stream_t stream);
+
+/* ---- Binary proxy with a top-p budget ("RaBitQCache", Abstract) -------------------------
+   Per row (b, g), with the rotation R[g] and the draws u[b][g] (uniform in [0, 1)):
+     qbar_i = fp32(sum over the group's heads, in order) / G;  q' = qbar . R[g] (j
+       ascending, one rounding per product and per sum); v_l = min q', Delta =
+       fp32(max q' - v_l) / 15; code n_i = min(15, floor(fp32(fp32((q'_i - v_l) / Delta) +
+       u_i))), all 0 when Delta = 0 (every step a rounded float32 operation);
+     s_t = g_t sum_i (2 b_ti - 1)(Delta n_i + v_l) + key_center[b][g] . qbar, computed as
+       g_t (Delta (2A - Q) + v_l (2B - d)) + c . qbar with A = sum_p 2^p popc(b & plane_p),
+       B = popc(b), Q = sum n_i (the RaBitQ estimate of qbar . k_t);
+     block_scores[b][g][j] = log sum_{t in block j, t < seq_len} e^(scale * s_t), the
+       natural log of the block's estimated attention mass up to the row's normaliser
+       (-inf for blocks with no valid token that share a page with valid ones; entries past
+       the last page of a row are not written).
+   q: [batch][Hq][d] BF16 (4-byte aligned); R: [Hkv][d][d] (16-byte aligned); u: [batch]
+   [Hkv][d] F32. Two launches (query codes into the workspace, then the scan). cfg must
+   have proxy_dtype QS_RABITQ (else QS_ERR_UNSUPPORTED) and cache->key_center set. */
+qs_status qs_rabitq_score(const qs_config *cfg, const qs_cache *cache, const void *q,
+                          const float *R, const float *u, int32_t batch, float *block_scores,
+                          void *ws, qs_stream_t stream);
+
+/* Top-p block selection of every row (one launch). block_scores hold natural-log block
+   masses (as qs_rabitq_score writes them); with M = the row's largest, block j weighs
+   w_j = e^(score_j - M), held in fixed point (units of 2^-40, so sums are exact). Over the
+   nb = ceil(seq_len / S) blocks, Z = sum w, goal = min(Z, ceil(p Z)). The forced blocks
+   (block 0 if force_sink, block nb-1 if force_last) are taken first and their mass
+   counts; the others follow in order of decreasing score, ties to the lower index, until
+   the taken mass reaches the goal or budget blocks are taken. A NaN score counts as -inf
+   (mass 0) and +inf as FLT_MAX. sel: ascending block ids padded with -1; n_sel: the count.
+   0 < p <= 1 and budget >= force_sink + force_last, else QS_ERR_INVALID_ARG. Any proxy
+   kind's configuration is accepted; only its block size, budget and forced blocks are
+   used. */
+qs_status qs_select_top_p(const qs_config *cfg, const qs_cache *cache,
+                          const float *block_scores, float p, int32_t batch, int32_t *sel,
+                          int32_t *n_sel, void *ws, qs_stream_t stream);
 
 /* ---- Comparison kernels: full-KV attention and gather-then-attend -----------------------
    "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 2 (b) and
@@ -288,7 +345,8 @@ qs_status qs_calibrate_basis(const qs_config *cfg, const void *q, const void *k,
    receives {kernel id, index} of that error. Returns QS_ERR_CUDA if the synchronisation
    or the read-back fails. Kernel ids: 1 append, 2 block error, 3 scoring prep, 4 score,
    5 select, 6 attention (with its log-sum-exp combine), 7 the wait self-test,
-   8 the gather of gather-then-attend. */
+   8 the gather of gather-then-attend. The binary proxy's writer, scan and top-p selection
+   report as 1, 4 and 5. */
 qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
 
 /* Sparse attention without a workspace, for callers that cannot allocate device memory:

@@ -9,11 +9,13 @@ from .binding import (QsError, LIB_PATH, EXPORTS, lib, make_config, make_cache, 
                       qs_select_topk, qs_sparse_attn, qs_decode, qs_device_status,
                       qs_sparse_attn_noalloc, qs_attention_launches, qs_selftest_wait_timeout,
                       qs_dense_workspace_size, qs_dense_attn, qs_gather_kv,
-                      qs_calib_workspace_size, qs_calibrate_basis, status_string)
+                      qs_calib_workspace_size, qs_calibrate_basis, qs_rabitq_score,
+                      qs_select_top_p, status_string)
 
 __all__ = ["QsError", "LIB_PATH", "EXPORTS", "lib", "make_config", "make_cache", "qs_version",
            "qs_workspace_size", "qs_workspace_init", "qs_append_kv", "qs_score",
            "qs_select_topk", "qs_sparse_attn", "qs_decode", "qs_device_status", "status_string",
            "qs_sparse_attn_noalloc", "qs_attention_launches", "qs_selftest_wait_timeout",
            "qs_dense_workspace_size", "qs_dense_attn", "qs_gather_kv",
-           "qs_calib_workspace_size", "qs_calibrate_basis"]
+           "qs_calib_workspace_size", "qs_calibrate_basis", "qs_rabitq_score",
+           "qs_select_top_p"]

@@ -14,9 +14,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqs.so")
 
 QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA, QS_ERR_DEVICE_BOUNDS, \
     QS_ERR_DEVICE_TIMEOUT = range(6)
-QS_F32, QS_BF16, QS_F16, QS_NVFP4, QS_E4M3, QS_CENTROID = range(6)
+QS_F32, QS_BF16, QS_F16, QS_NVFP4, QS_E4M3, QS_CENTROID, QS_RABITQ = range(7)
 DTYPE_CODES = {"f32": QS_F32, "bf16": QS_BF16, "f16": QS_F16, "nvfp4": QS_NVFP4,
-               "e4m3": QS_E4M3, "centroid": QS_CENTROID}
+               "e4m3": QS_E4M3, "centroid": QS_CENTROID, "rabitq": QS_RABITQ}
 
 
 class QsError(RuntimeError):
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "qs_gather_kv": ([cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp], i32),
             "qs_calib_workspace_size": ([cfgp, ctypes.POINTER(sz)], i32),
             "qs_calibrate_basis": ([cfgp, vp, vp, i32, vp, vp, vp, vp], i32),
+            "qs_rabitq_score": ([cfgp, cachep, vp, vp, vp, i32, vp, vp, vp], i32),
+            "qs_select_top_p": ([cfgp, cachep, vp, ctypes.c_float, i32, vp, vp, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -87,7 +89,8 @@ EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_
            "qs_append_kv", "qs_score", "qs_select_topk", "qs_sparse_attn", "qs_decode",
            "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches",
            "qs_selftest_wait_timeout", "qs_dense_workspace_size", "qs_dense_attn",
-           "qs_gather_kv", "qs_calib_workspace_size", "qs_calibrate_basis")
+           "qs_gather_kv", "qs_calib_workspace_size", "qs_calibrate_basis", "qs_rabitq_score",
+           "qs_select_top_p")
 
 
 def status_string(s: int) -> str:
@@ -253,6 +256,23 @@ def qs_calibrate_basis(cfg, q, k, n, P, eigvals, ws, stream=None):
     _check(lib().qs_calibrate_basis(ctypes.byref(cfg), _ptr(q), _ptr(k), n, _ptr(P),
                                     _ptr(eigvals), _ptr(ws), _stream(stream)),
            "qs_calibrate_basis")
+
+
+def qs_rabitq_score(cfg, cache, q, R, u, batch, block_scores, ws, stream=None):
+    """Binary-proxy block scores: q [batch][Hq][d] BF16, R [Hkv][d][d] FP32 rotations,
+    u [batch][Hkv][d] FP32 rounding draws in [0, 1); block_scores [batch][Hkv][nb_stride]
+    receive the natural log of each block's estimated attention mass."""
+    _check(lib().qs_rabitq_score(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(R),
+                                 _ptr(u), batch, _ptr(block_scores), _ptr(ws),
+                                 _stream(stream)), "qs_rabitq_score")
+
+
+def qs_select_top_p(cfg, cache, block_scores, p, batch, sel, n_sel, ws, stream=None):
+    """Forced blocks, then the highest-mass blocks until their mass reaches p of the row's
+    (block_scores are log masses), at most cfg.budget; sel ascending, padded with -1."""
+    _check(lib().qs_select_top_p(ctypes.byref(cfg), ctypes.byref(cache), _ptr(block_scores),
+                                 float(p), batch, _ptr(sel), _ptr(n_sel), _ptr(ws),
+                                 _stream(stream)), "qs_select_top_p")
 
 
 def qs_device_status(ws, stream=None) -> tuple[int, int, int]:

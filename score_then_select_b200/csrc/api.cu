@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "qs_internal.h"
+#include "rabitq.h"
 
 namespace qs {
 
@@ -110,8 +111,10 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   if (c->head_dim != 64 && c->head_dim != 128) return QS_ERR_UNSUPPORTED;
   const int r = c->proxy_rank;
   if (r < 0) return QS_ERR_INVALID_ARG;
-  p.kind = r > 0 ? PK_RANKR : (c->proxy_dtype == QS_CENTROID ? PK_CENTROID : PK_NVFP4);
-  if (p.kind == PK_CENTROID) {
+  p.kind = r > 0 ? PK_RANKR
+                 : (c->proxy_dtype == QS_CENTROID ? PK_CENTROID
+                                                  : (c->proxy_dtype == QS_RABITQ ? PK_RABITQ : PK_NVFP4));
+  if (p.kind == PK_CENTROID || p.kind == PK_RABITQ) {
     if (c->n_keep_hp != 0) return QS_ERR_INVALID_ARG;
   } else if (r > 0) {
     const bool ok = (c->proxy_dtype == QS_F32 && (r == 16 || (r == 32 && c->head_dim == 128))) ||
@@ -173,7 +176,7 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   }
   size_t off = size_t(kHdrWords) * 4;
   const size_t rows = size_t(batch) * p.Hkv, rows_q = size_t(batch) * p.Hq;
-  w.qt = off;      off = align_up(off + rows * (r > 0 ? r : 1) * 4, 256);
+  w.qt = off;      off = align_up(off + rows * (r > 0 ? r : (p.kind == PK_RABITQ ? kRqRowWords : 1)) * 4, 256);
   w.qtile = off;   off = align_up(off + (p.kind == PK_NVFP4 ? rows * kQTileBytes : 0), 256);
   w.qgscale = off; off = align_up(off + 16, 256);
   w.scores = off;  off = align_up(off + rows * p.nb_stride * 4, 256);
@@ -210,6 +213,7 @@ qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy) {
     if (!c->proxy || !aligned(c->proxy, 16)) return QS_ERR_INVALID_ARG;
     if (p.kind == PK_NVFP4 && (!c->proxy_scale || !c->key_center || !c->key_gscale))
       return QS_ERR_INVALID_ARG;
+    if (p.kind == PK_RABITQ && !c->key_center) return QS_ERR_INVALID_ARG;
   }
   return QS_OK;
 }
@@ -422,7 +426,7 @@ qs_status qs_append_kv(const qs_config* cfg, const qs_cache* cache, const void* 
   if ((st = check_cache(p, cache, true)) != QS_OK) return st;
   if (!k_new || !v_new || !n_new || max_new < 1 || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
-  if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
+  if ((p.r > 0 || p.kind == PK_RABITQ) && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
   if (p.kind == PK_NVFP4 && !cache->block_err) return QS_ERR_INVALID_ARG;
   return do_append(p, cache, k_new, v_new, n_new, max_new, P, nullptr, ws, stream);
 }
@@ -436,6 +440,7 @@ qs_status qs_score(const qs_config* cfg, const qs_cache* cache, const void* q, c
   if (!q || !aligned(q, 4) || !block_scores || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
   if (p.r == 0 && !aligned(q, 16)) return QS_ERR_INVALID_ARG;
+  if (p.kind == PK_RABITQ) return QS_ERR_UNSUPPORTED;     // qs_rabitq_score takes its draws
   if (p.kind == PK_CENTROID) return do_score(p, cache, q, block_scores, ws, stream, false);
   // the prep kernel runs in stream order and writes only the query side, so the scan
   // overlaps it and starts streaming pages before it waits for the query
@@ -557,6 +562,7 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
   if (st != QS_OK) return st;
   if ((st = check_cache(p, cache, true)) != QS_OK) return st;
+  if (p.kind == PK_RABITQ) return QS_ERR_UNSUPPORTED;     // its stages are separate calls
   if (!q || !aligned(q, 16) || !k_new || !v_new || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
@@ -571,6 +577,67 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   if ((st = do_score(p, cache, q, scores, ws, stream, true)) != QS_OK) return st;
   if ((st = do_select(p, cache, scores, sel, nsel, ws, stream, true)) != QS_OK) return st;
   return do_attend(p, cache, q, sel, nsel, out, ws, stream, true);
+}
+
+qs_status qs_rabitq_score(const qs_config* cfg, const qs_cache* cache, const void* q,
+                          const float* R, const float* u, int32_t batch, float* block_scores,
+                          void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (p.kind != PK_RABITQ) return QS_ERR_UNSUPPORTED;
+  if ((st = check_cache(p, cache, true)) != QS_OK) return st;
+  if (!q || !aligned(q, 4) || !R || !aligned(R, 16) || !u || !block_scores || !ws ||
+      !aligned(ws, 256))
+    return QS_ERR_INVALID_ARG;
+  uint32_t* qcode = ws_at<uint32_t>(ws, p.ws.qt);
+  RqPrepParams a{static_cast<const uint16_t*>(q), R, u, cache->key_center, qcode,
+                 p.batch, p.Hkv, p.G, p.d};
+  if ((st = cuda_status(launch_rq_prep(a, stream))) != QS_OK) return st;
+  RqScoreParams b{};
+  b.proxy = static_cast<const uint8_t*>(cache->proxy);
+  b.qcode = qcode;
+  b.page_table = cache->page_table;
+  b.seq_lens = cache->seq_lens;
+  b.scores = block_scores;
+  b.hdr = hdr_of(ws);
+  b.batch = p.batch;
+  b.Hkv = p.Hkv;
+  b.d = p.d;
+  b.S = p.S;
+  b.nb_stride = p.nb_stride;
+  b.max_pages_per_seq = cache->max_pages_per_seq;
+  b.num_pages = cache->num_pages;
+  b.max_context = cache->max_context;
+  b.scale = p.scale;
+  return cuda_status(launch_rq_score(b, stream));
+}
+
+qs_status qs_select_top_p(const qs_config* cfg, const qs_cache* cache, const float* block_scores,
+                          float p_mass, int32_t batch, int32_t* sel, int32_t* n_sel, void* ws,
+                          qs_stream_t stream) {
+  Plan p;
+  const qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (!cache || !cache->seq_lens) return QS_ERR_INVALID_ARG;
+  if (!block_scores || !sel || !n_sel || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (!(p_mass > 0.0f && p_mass <= 1.0f)) return QS_ERR_INVALID_ARG;
+  if (p.budget < p.force_sink + p.force_last) return QS_ERR_INVALID_ARG;
+  TopPParams a{};
+  a.scores = block_scores;
+  a.seq_lens = cache->seq_lens;
+  a.sel = sel;
+  a.n_sel = n_sel;
+  a.hdr = hdr_of(ws);
+  a.rows = p.batch * p.Hkv;
+  a.Hkv = p.Hkv;
+  a.S = p.S;
+  a.nb_stride = p.nb_stride;
+  a.budget = p.budget;
+  a.force_sink = p.force_sink;
+  a.force_last = p.force_last;
+  a.p = p_mass;
+  return cuda_status(launch_top_p(a, stream));
 }
 
 qs_status qs_device_status(void* ws, qs_stream_t stream, uint32_t* detail) {

@@ -9,6 +9,9 @@
 // Centroid writer ("Coarse Semantic Blocks ...", Abstract): each block's FP32 key sum,
 // continued in token order.
 //
+// Binary-code writer ("RaBitQCache", Abstract): the sign bits of the rotated centred key
+// and its factor |o|^2 / |y|_1 (the RaBitQ code).
+//
 // NVFP4 writer ("Jet-QSparse: Accelerating Agentic LLM Inference with 4-Bit Sparse
 // Attention", Full text): the persistent scoring cache is packed straight from the BF16
 // keys after calibrated centring: x = float(k) - mu (float32), then per 16 elements
@@ -17,6 +20,7 @@
 // saturating. Blocks completed by the append get their squared quantisation error, which
 // decides the blocks kept at full precision.
 #include "qs_device.cuh"
+#include "rabitq.h"
 
 namespace qs {
 
@@ -481,6 +485,92 @@ __global__ void __launch_bounds__(128) append_nvfp4_kernel(const AppendParams a)
   finish_append(a);
 }
 
+// ============================================================ binary-code writer
+// "RaBitQCache", Abstract, with the RaBitQ code (Gao and Long, SIGMOD 2024, section 3):
+// o = float(k) - c (float32), y = o R[g] with each y_i summed over j ascending (one
+// rounding per product and per sum), bits b_i = [y_i > 0] packed 32 to a word by a warp
+// ballot (little-endian words, so bit i lands in byte i / 8 at position i % 8), and
+// g = fp32(sum_j o_j^2) / fp32(sum_i |y_i|) with both sums taken left to right (g = 0 when
+// the second is 0). CTA = one row x 16 tokens, thread i = dimension i (blockDim = D):
+// each R[g][j][i] is loaded once per CTA and applied to the 16 tokens.
+template <int D>
+__global__ void __launch_bounds__(D) append_rabitq_kernel(const AppendParams a) {
+  constexpr int TT = 16;
+  constexpr int PB = kPage * (D / 8) + kPage * 4;      // bytes per (page, KV head)
+  __shared__ float s_o[TT][D];
+  __shared__ float s_ay[TT][D];
+  __shared__ int s_page[TT], s_slot[TT];
+  const int row = blockIdx.y;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int n_b = a.n_new ? a.n_new[b] : 1;
+  if (n_b < 0 || n_b > a.max_new) {
+    if (tid == 0 && blockIdx.x == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_APPEND, uint32_t(b));
+    n_b = 0;
+  }
+  const int old = a.seq_lens[b];
+  const int t0 = blockIdx.x * TT;
+  const int cnt = min(TT, n_b - t0);
+  if (cnt > 0) {
+    if (tid < TT) {
+      int page = -1, slot = 0;
+      if (tid < cnt)
+        cache_slot(a.page_table, b, old + t0 + tid, a.max_pages_per_seq, a.num_pages,
+                   a.max_context, a.hdr, KID_APPEND, page, slot);
+      s_page[tid] = page;
+      s_slot[tid] = slot;
+    }
+    const float c_i = a.key_center[size_t(row) * D + tid];
+    const size_t src0 = (size_t(row) * a.max_new + t0) * D;
+    for (int n = 0; n < TT; ++n)
+      s_o[n][tid] = n < cnt ? __fsub_rn(bf16_to_f32(a.k_new[src0 + size_t(n) * D + tid]), c_i)
+                            : 0.0f;
+    __syncthreads();
+    // K and V rows of the chunk's tokens -> their page slots (16 bytes per step)
+    constexpr int CH = D / 8;
+    for (int it = tid; it < cnt * CH; it += D) {
+      const int n = it / CH, c = it % CH;
+      const int page = s_page[n];
+      if (page < 0) continue;
+      const size_t src = src0 + size_t(n) * D + c * 8;
+      const size_t dst = ((size_t(page) * a.Hkv + g) * kPage + s_slot[n]) * D + c * 8;
+      *reinterpret_cast<uint4*>(a.k + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+      *reinterpret_cast<uint4*>(a.v + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+    }
+    // y_i of every token of the chunk, j ascending
+    const float* Rg = a.P + size_t(g) * D * D;
+    float acc[TT];
+#pragma unroll
+    for (int n = 0; n < TT; ++n) acc[n] = 0.0f;
+    for (int j = 0; j < D; ++j) {
+      const float r = Rg[size_t(j) * D + tid];
+#pragma unroll
+      for (int n = 0; n < TT; ++n) acc[n] = __fadd_rn(acc[n], __fmul_rn(s_o[n][j], r));
+    }
+    uint8_t* base = static_cast<uint8_t*>(a.proxy);
+#pragma unroll
+    for (int n = 0; n < TT; ++n) {
+      const unsigned word = __ballot_sync(kFull, acc[n] > 0.0f);
+      s_ay[n][tid] = fabsf(acc[n]);
+      if (n < cnt && lane == 0 && s_page[n] >= 0) {
+        uint8_t* pg = base + (size_t(s_page[n]) * a.Hkv + g) * PB;
+        reinterpret_cast<uint32_t*>(pg + s_slot[n] * (D / 8))[warp] = word;
+      }
+    }
+    __syncthreads();
+    // the factor g of each token: one thread per token, both sums in index order
+    if (tid < cnt && s_page[tid] >= 0) {
+      float n2 = 0.0f, l1 = 0.0f;
+      for (int j = 0; j < D; ++j) n2 = __fadd_rn(n2, __fmul_rn(s_o[tid][j], s_o[tid][j]));
+      for (int i = 0; i < D; ++i) l1 = __fadd_rn(l1, s_ay[tid][i]);
+      uint8_t* pg = base + (size_t(s_page[tid]) * a.Hkv + g) * PB;
+      reinterpret_cast<float*>(pg + kPage * (D / 8))[s_slot[tid]] =
+          l1 > 0.0f ? __fdiv_rn(n2, l1) : 0.0f;
+    }
+  }
+  finish_append(a);
+}
+
 // ============================================================ NVFP4 block error
 // CTA = one (row, block) pair that this append may have completed; 256 threads, each
 // owning (token, 16-element group) items i = tid + 256 m. An item's error is summed over
@@ -657,6 +747,12 @@ static cudaError_t launch_rankr(const Plan& p, const AppendParams& a, cudaStream
 }
 
 cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) {
+  if (p.kind == PK_RABITQ) {
+    const dim3 grid((a.max_new + 15) / 16, a.batch * a.Hkv);
+    if (p.d == 128) append_rabitq_kernel<128><<<grid, 128, 0, s>>>(a);
+    else append_rabitq_kernel<64><<<grid, 64, 0, s>>>(a);
+    return cudaGetLastError();
+  }
   if (p.kind == PK_CENTROID) {
     // blocks a call can touch: ceil(max_new / S) + 1 (the first may be partly filled)
     const dim3 grid((a.max_new + p.S - 1) / p.S + 1, a.batch * a.Hkv);

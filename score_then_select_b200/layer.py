@@ -40,7 +40,14 @@ class Layer:
         k = torch.zeros((num_pages, Hkv, ps, d), dtype=torch.bfloat16, device=device)
         v = torch.zeros((num_pages, Hkv, ps, d), dtype=vdt, device=device)
         extra = {}
-        if cfg.proxy_dtype == B.QS_CENTROID:
+        if cfg.proxy_dtype == B.QS_RABITQ:
+            # per (page, KV head): page_size x d/8 bytes of code bits, then page_size FP32
+            # factors; the row centres c
+            proxy = torch.zeros((num_pages, Hkv, ps * (d // 8) + ps * 4), dtype=torch.uint8,
+                                device=device)
+            extra = dict(key_center=torch.zeros((batch, Hkv, d), dtype=torch.float32,
+                                                device=device))
+        elif cfg.proxy_dtype == B.QS_CENTROID:
             # per-block FP32 key sums: [num_pages][Hkv][page_size / S][d]
             proxy = torch.zeros((num_pages, Hkv, ps // cfg.block_size, d), dtype=torch.float32,
                                 device=device)

@@ -169,3 +169,55 @@ def test_binding_argument_counts_match_the_header():
         f = getattr(L, name)
         assert f.argtypes is not None, f"{name}: no argtypes in the binding"
         assert len(f.argtypes) == n, f"{name}: header has {n} parameters, binding {len(f.argtypes)}"
+
+
+def _fake_cache(with_center=True):
+    """A cache whose pointers are aligned placeholders: valid for the host checks, never
+    dereferenced (every call below returns before any launch)."""
+    c = B.qs_cache()
+    c.k = c.v = c.proxy = c.page_table = c.seq_lens = 1 << 20
+    c.key_center = (1 << 20) if with_center else None
+    c.max_pages_per_seq, c.num_pages, c.max_context = 8, 64, 1024
+    return c
+
+
+def test_binary_proxy_configuration_and_calls_validate_on_the_host():
+    rq = dict(proxy_rank=0, proxy_dtype="rabitq", block_size=1, budget=256)
+    assert qs.qs_workspace_size(_cfg(**rq), 16, 131072) > 0
+    assert qs.qs_workspace_size(_cfg(head_dim=64, **rq), 2, 1000) > 0
+    with pytest.raises(qs.QsError) as e:                      # kept blocks are NVFP4-only
+        qs.qs_workspace_size(_cfg(n_keep_hp=1, **rq), 16, 4096)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_workspace_size(_cfg(head_dim=96, **rq), 16, 4096)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    cfg, cache, a = _cfg(**rq), _fake_cache(), 1 << 20
+    # its stages are separate calls: the fused step and the draw-less score refuse it
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_score(cfg, cache, a, a, 4, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_decode(cfg, cache, a, a, a, a, 4, a, None, None, a, stream=0)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    # the binary scan needs the binary proxy, its centres and its rotation
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_rabitq_score(_cfg(), cache, a, a, a, 4, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_rabitq_score(cfg, _fake_cache(with_center=False), a, a, a, 4, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_rabitq_score(cfg, cache, a, None, a, 4, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    with pytest.raises(qs.QsError) as e:                      # the writer needs R
+        qs.qs_append_kv(cfg, cache, a, a, a, 1, None, 4, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    # top-p: 0 < p <= 1, and room for the forced blocks
+    for p in (0.0, -0.5, 1.5, float("nan")):
+        with pytest.raises(qs.QsError) as e:
+            qs.qs_select_top_p(cfg, cache, a, p, 4, a, a, a, stream=0)
+        assert e.value.status == B.QS_ERR_INVALID_ARG, p
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_select_top_p(_cfg(budget=1, **{k: v for k, v in rq.items() if k != "budget"}),
+                           cache, a, 0.5, 4, a, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
