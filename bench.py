@@ -43,7 +43,8 @@ METRIC = "sparse decode attn steps/s at 128K ctx, batch 16; achieved HBM GB/s vs
 WORKLOADS = {"block128k": synth.BLOCK128K, "token32k": synth.TOKEN32K, "ragged": synth.RAGGED,
              "nvfp4": synth.NVFP4_128K, "tiny": synth.TINY, "fp8": synth.FP8_128K,
              "fp8token": synth.FP8_TOKEN32K, "centroid": synth.CENTROID_128K,
-             "centroid32": synth.CENTROID_S32, "token128k": synth.TOKEN128K}
+             "centroid32": synth.CENTROID_S32, "token128k": synth.TOKEN128K,
+             "rabitq128k": synth.RABITQ_TOKEN128K}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -153,6 +154,8 @@ def step_bytes(w, lens, sel, nsel):
     else:
         if w.proxy_dtype == "nvfp4":
             per_tok = d // 2 + d // 16
+        elif w.proxy_dtype == "rabitq":                # d code bits + one FP32 factor
+            per_tok = d // 8 + 4
         else:
             per_tok = w.proxy_rank * {"f32": 4, "bf16": 2, "e4m3": 1}[w.proxy_dtype]
         proxy = int(np.sum(lens.astype(np.int64))) * w.n_kv_heads * per_tok
@@ -200,9 +203,9 @@ def oracle_prepare(w, inp, rows, threads):
     from threadpoolctl import threadpool_limits
     from oracle import method as M
     from oracle import step as OS
-    from tests.util import row_params
+    from tests.util import row_params, top_p_params
 
-    p = row_params(w)
+    p = top_p_params(w) if w.proxy_dtype == "rabitq" else row_params(w)
 
     def prep(bg):
         b, g = bg
@@ -210,7 +213,10 @@ def oracle_prepare(w, inp, rows, threads):
         L = int(inp.lens[b])
         P = inp.P[g] if inp.P is not None else None
         mu = inp.mu[b, g] if inp.mu is not None else None
-        cache = OS.row_scoring_cache(p, k[:L], P, mu, inp.g_k)
+        if w.proxy_dtype == "rabitq":                 # the binary codes (P holds R)
+            cache = M.rabitq_encode(k[:L], P, mu)
+        else:
+            cache = OS.row_scoring_cache(p, k[:L], P, mu, inp.g_k)
         return (b, g, k, v, q, L, P, cache)
 
     with threadpool_limits(limits=1):
@@ -234,9 +240,17 @@ def oracle_time(w, inp, prep, threads):
 
     def one(x):
         b, g, k, v, q, L, P, cache = x
-        beta = OS.row_block_scores(p, cache, q, L, P=P, g_q=g_q, g_k=inp.g_k)
-        forced, _ = OS.row_forced(p, beta.shape[0], cache, L, inp.g_k)
-        sel = M.select_blocks(beta, p.budget, forced)
+        if w.proxy_dtype == "rabitq":
+            bits, gk = cache
+            n, delta, vl, qbar = M.rabitq_query(q, P, inp.u[b, g])
+            s = M.rabitq_scores(bits, gk, n, delta, vl, inp.mu[b, g], qbar)
+            mass = M.block_mass(M.estimated_weights(s, p.scale), p.S)
+            forced = M.forced_blocks(mass.shape[0], p.force_sink, p.force_last)
+            sel = M.select_top_p(mass, p.p, p.budget, forced)
+        else:
+            beta = OS.row_block_scores(p, cache, q, L, P=P, g_q=g_q, g_k=inp.g_k)
+            forced, _ = OS.row_forced(p, beta.shape[0], cache, L, inp.g_k)
+            sel = M.select_blocks(beta, p.budget, forced)
         tok = M.block_tokens(sel, p.S, L)
         return M.sparse_attention(F.bf16_to_f64(q), F.bf16_to_f64(k[tok]),
                                   OS.decode_v(v[tok], p.v_dtype), np.arange(len(tok)), p.scale)
@@ -430,6 +444,8 @@ def run_ours(args):
     w = rank_workload(w0, rank)
     inp = synth.Inputs(w)
     f = Filled(inp, attn_path=args.attn_path)
+    if w.proxy_dtype == "rabitq":
+        return run_ours_top_p(args, w, inp, f, world, rank, local)
     lay, cfg, cache = f.layer, f.cfg, f.cache
     B = w.batch
     lens = inp.lens
@@ -591,6 +607,154 @@ def run_ours(args):
             "gpu_launches": args.steps * launches_per_step}
     if compare is not None:
         line["comparison"] = compare
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_ours_top_p(args, w, inp, f, world, rank, local):
+    """The binary proxy's step ("RaBitQCache", Abstract) through its entry points: append
+    (binary writer), qs_rabitq_score (query code + scan), qs_select_top_p, qs_sparse_attn;
+    timed, broken into stages and run end to end like the fused step of the other proxies
+    (the end-to-end leg issues the four calls eagerly, without a captured graph)."""
+    import torch
+    import torch.distributed as dist
+    import score_then_select_b200 as qs
+
+    lay, cfg, cache = f.layer, f.cfg, f.cache
+    B, lens, Hkv = w.batch, inp.lens, w.n_kv_heads
+    start_lens = torch.from_numpy((lens - 1).astype(np.int32)).cuda()
+    ones = torch.ones((B,), dtype=torch.int32, device="cuda")
+    u = torch.from_numpy(inp.u).cuda()
+    out = torch.zeros((B, w.n_q_heads, w.head_dim),
+                      dtype=torch.float32 if w.out_dtype == "f32" else torch.bfloat16, device="cuda")
+    sel = torch.zeros((B, Hkv, w.budget), dtype=torch.int32, device="cuda")
+    nsel = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+    scores = torch.empty((B, Hkv, lay.nb_stride), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    p = float(w.top_p)
+
+    def step(q, k, v, ev=None):
+        lay.seq_lens.copy_(start_lens, non_blocking=True)
+        if ev:
+            ev[0].record(stream)
+        qs.qs_append_kv(cfg, cache, k, v, ones, 1, f.P, B, lay.ws, stream)
+        if ev:
+            ev[1].record(stream)
+        qs.qs_rabitq_score(cfg, cache, q, f.P, u, B, scores, lay.ws, stream)
+        if ev:
+            ev[2].record(stream)
+        qs.qs_select_top_p(cfg, cache, scores, p, B, sel, nsel, lay.ws, stream)
+        if ev:
+            ev[3].record(stream)
+        qs.qs_sparse_attn(cfg, cache, q, sel, nsel, B, out, lay.ws, stream)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step(f.q, f.k_last, f.v_last)
+    st = qs.qs_device_status(lay.ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device status {st}")
+    sel_h, nsel_h = sel.cpu().numpy(), nsel.cpu().numpy()
+    # append + query code + scan + top-p select + attention (1 or 2 launches)
+    launches_per_step = 4 + qs.qs_attention_launches(cfg, B, lay.max_context)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---------------- timed region: K steps
+    clocks = Clocks(local)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(f.q, f.k_last, f.v_last)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    t_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, "cuda")
+    st = qs.qs_device_status(lay.ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device status after timing {st}")
+
+    # ---------------- per-stage breakdown (events between the four calls)
+    n_stage = min(args.steps, 50)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_stage + 3)]
+    for ev in evs:
+        step(f.q, f.k_last, f.v_last, ev)
+    torch.cuda.synchronize()
+    acc = np.zeros(4)
+    for ev in evs[3:]:
+        acc += [ev[j].elapsed_time(ev[j + 1]) for j in range(4)]
+    stage_us = dict(zip(["append", "score", "select", "attend"], (acc / n_stage * 1e3).tolist()))
+
+    # ---------------- end to end: q, k_new, v_new from pinned host memory, the four calls,
+    # the output back to the host, then a sync
+    q_h = f.q.cpu().pin_memory()
+    k_h = f.k_last.cpu().pin_memory()
+    v_h = f.v_last.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_d, k_d, v_d = torch.empty_like(f.q), torch.empty_like(f.k_last), torch.empty_like(f.v_last)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        step(q_d, k_d, v_d)
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    n_e2e = max(args.steps, 10)
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(n_e2e):
+        e2e_step()
+    e2e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3 / n_e2e, world, "cuda")
+    st = qs.qs_device_status(lay.ws)
+    if st[0] != 0:
+        raise RuntimeError(f"device status after the end-to-end runs {st}")
+    h2d = q_h.numel() * q_h.element_size() + 2 * k_h.numel() * k_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    # ---------------- roofline: the scan (query code + binary scan, one qs_rabitq_score)
+    peak, peak_src = peaks()
+    by = step_bytes(w, lens, sel_h, nsel_h)
+    score_us = stage_us["score"]
+    roof = {"bound": "hbm", "kernel": "score (query code + binary scan, one qs_rabitq_score call)",
+            "achieved": by["proxy"] / (score_us * 1e-6) / 1e9, "peak": peak, "unit": "GB/s",
+            "frac": by["proxy"] / (score_us * 1e-6) / 1e9 / peak, "peak_source": peak_src,
+            "algorithmic_bytes_per_launch": by["proxy"], "launch_us": score_us,
+            "traffic": profiled_traffic("rabitq", w.name)}
+    step_gbs = by["total"] / (t_ms * 1e-3) / 1e9
+    value = aggregate_steps_per_s(t_ms, world)
+    cfg_line = config_of(w, lens)
+    cfg_line["top_p"] = w.top_p
+    cfg_line["mean_selected_blocks"] = float(nsel_h.mean())
+    line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "b1xi4+f32+bf16",
+            "data": "synthetic (seeded; shapes of the pages' 128K batch-16 decode)",
+            "config": cfg_line, "tokens_per_s": value * B, "us_per_layer_step": t_ms * 1e3,
+            "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": step_gbs / peak, "bytes_per_step": by},
+            "stage_us": stage_us, "roofline": roof, "clocks": clk,
+            "e2e": {"value": aggregate_steps_per_s(e2e_ms, world), "unit": "steps/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "path": "eager calls of the four entry points"},
+            "gpu_launches": args.steps * launches_per_step}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_rows)
     if rank == 0:

@@ -24,6 +24,9 @@ Recipe (Gaussians are written N(mean, variance)):
         q_h = z_h + 3 * sum_j unit(mean key of block j - mean key of the row), z_h ~ N(0, I);
   * P: QR of a Gaussian d x r matrix, columns sign-fixed so diag(R) > 0; one P per layer,
     repeated for every KV head;
+  * binary proxy: one rotation per KV head (QR of a Gaussian d x d matrix, sign-fixed),
+    the row centres as the NVFP4 centring mean below, and rounding draws uniform in
+    [0, 1) per (sequence, KV head, dimension);
   * ragged lengths: integers uniform in [min, max], redrawn while a multiple of the block
     size, then fixed overrides for the last few sequences;
   * paging: 128-token pages; each sequence's physical pages are a slice of one seeded
@@ -41,6 +44,7 @@ from .workloads import Workload
 
 TAG_K, TAG_V, TAG_Q, TAG_P, TAG_LENS, TAG_PAGES, TAG_OUTL, TAG_PLANT, TAG_ROWPAR, TAG_MIX = (
     1, 2, 3, 4, 5, 6, 7, 8, 9, 10)
+TAG_ROT, TAG_U = 11, 12
 
 
 def _rng(w: Workload, tag: int, *ids: int) -> np.random.Generator:
@@ -97,6 +101,23 @@ def proj_matrix(w: Workload) -> np.ndarray:
     q = q * np.sign(np.diag(r))[None, :]
     p = q.astype(np.float32)
     return np.ascontiguousarray(np.broadcast_to(p, (w.n_kv_heads,) + p.shape))
+
+
+def rotations(w: Workload) -> np.ndarray:
+    """R as float32 [Hkv][d][d]: one uniformly random rotation per KV head (QR of a Gaussian
+    matrix, columns sign-fixed so diag(R) > 0), the binary proxy's random rotation."""
+    out = np.empty((w.n_kv_heads, w.head_dim, w.head_dim), dtype=np.float32)
+    for g in range(w.n_kv_heads):
+        a = _rng(w, TAG_ROT, g).standard_normal((w.head_dim, w.head_dim))
+        q, r = np.linalg.qr(a)
+        out[g] = (q * np.sign(np.diag(r))[None, :]).astype(np.float32)
+    return out
+
+
+def rounding_draws(w: Workload) -> np.ndarray:
+    """u as float32 [batch][Hkv][d], uniform in [0, 1): the binary proxy's random rounding
+    of the rotated query to its 4-bit grid (one draw per dimension per step)."""
+    return _rng(w, TAG_U).random((w.batch, w.n_kv_heads, w.head_dim), dtype=np.float32)
 
 
 def outlier_channels(w: Workload, g: int) -> np.ndarray:
@@ -232,8 +253,15 @@ class Inputs:
         self.page_table, self.num_pages = page_table(w, self.lens, extra_tokens)
         self.P = proj_matrix(w) if w.proxy_rank > 0 else None
         self.threads = threads or os.cpu_count()
+        self.u = None
         if w.proxy_dtype == "nvfp4":
             self.mu, self.g_k = calibration(w, self.lens, self.threads)
+        elif w.proxy_dtype == "rabitq":
+            # the rotation R takes P's place; the row centres are the calibration means
+            self.P = rotations(w)
+            self.mu, _ = calibration(w, self.lens, self.threads)
+            self.g_k = None
+            self.u = rounding_draws(w)
         else:
             self.mu, self.g_k = None, None
 

@@ -25,8 +25,8 @@ class Workload:
     context: int                 # L for fixed-length workloads (tokens incl. the current one)
     block_size: int              # S
     budget: int                  # k, in blocks
-    proxy_rank: int              # r > 0: projected-key proxy; 0: NVFP4 centred keys
-    proxy_dtype: str             # 'f32' | 'bf16' | 'e4m3' | 'nvfp4' | 'centroid'
+    proxy_rank: int              # r > 0: projected-key proxy; 0: NVFP4, centroid or binary
+    proxy_dtype: str             # 'f32' | 'bf16' | 'e4m3' | 'nvfp4' | 'centroid' | 'rabitq'
     v_dtype: str                 # stored V: 'bf16' | 'f16'
     v_agg_dtype: str             # PV operand precision: 'bf16' | 'f16'
     out_dtype: str               # 'f32' | 'bf16'
@@ -48,6 +48,8 @@ class Workload:
     ragged_overrides: tuple = ()  # ((seq, L), ...) applied after the uniform draw
     ragged_min: int = 4096
     ragged_max: int = 131072
+    top_p: float = 0.0           # > 0: top-p selection of this share of the estimated mass,
+                                 # at most `budget` blocks (binary proxy)
 
     @property
     def group(self) -> int:
@@ -120,6 +122,13 @@ CENTROID_128K = BLOCK128K.replace(name="centroid_b16_h40kv8_d128_L131072_S128_k6
 CENTROID_S32 = BLOCK128K.replace(name="centroid_b16_h40kv8_d128_L131072_S32_k256", block_size=32,
                                  budget=256, proxy_rank=0, proxy_dtype="centroid", seed=1009)
 
+# Binary (RaBitQ) proxy with a top-p budget ("RaBitQCache", Abstract): 1-bit codes of the
+# rotated centred keys against a 4-bit query code; the fewest tokens whose estimated
+# attention mass reaches p = 0.9, at most 2,048 per KV head. The 128K token-level shape,
+# so it compares with the rank-32 top-k step on the same keys and queries' recipe.
+RABITQ_TOKEN128K = TOKEN128K.replace(name="rabitq_b16_h32kv8_d128_L131072_p0.9_B2048",
+                                     proxy_rank=0, proxy_dtype="rabitq", top_p=0.9, seed=1013)
+
 # Ragged batch: 32 sequences, lengths uniform in [4096, 131072], G = 8, r = 64, S = 64.
 RAGGED = Workload(
     name="ragged_b32_h64kv8_d128_S64_k32_r64", batch=32, n_q_heads=64, n_kv_heads=8,
@@ -136,8 +145,9 @@ TINY_CENTROID = TINY.replace(name="tiny_centroid_b1_h4_d64_L2048", proxy_rank=0,
 
 FULL = {w.name: w for w in (TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED)}
 ORDER = [TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED]
-# variants of the configurations above (FP8 projected keys, centroid scoring, 128K token level)
-VARIANTS = [FP8_128K, FP8_TOKEN32K, CENTROID_128K, CENTROID_S32, TOKEN128K]
+# variants of the configurations above (FP8 projected keys, centroid scoring, 128K token
+# level, the binary proxy with a top-p budget)
+VARIANTS = [FP8_128K, FP8_TOKEN32K, CENTROID_128K, CENTROID_S32, TOKEN128K, RABITQ_TOKEN128K]
 
 
 def small(w: Workload) -> Workload:

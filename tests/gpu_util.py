@@ -35,8 +35,9 @@ class Filled:
                                     inp.page_table.shape[1], Lmax, device)
         lay = self.layer
         lay.page_table.copy_(torch.from_numpy(inp.page_table))
-        if w.proxy_dtype == "nvfp4":
+        if w.proxy_dtype in ("nvfp4", "rabitq"):
             lay.key_center.copy_(torch.from_numpy(inp.mu))
+        if w.proxy_dtype == "nvfp4":
             lay.key_gscale.fill_(float(inp.g_k))
         self.P = torch.from_numpy(np.array(inp.P)).to(device) if inp.P is not None else None
         self.q = u16(Q).to(device)

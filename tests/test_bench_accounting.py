@@ -25,7 +25,7 @@ def test_rank_r_bf16_bytes_at_128k():
     assert by["selected_tokens"] == 16 * 8 * 64 * 128
 
 
-def test_fp8_nvfp4_and_centroid_proxy_bytes():
+def test_fp8_nvfp4_centroid_and_binary_proxy_bytes():
     lens = np.full(16, 131072, dtype=np.int64)
     fp8 = synth.FP8_128K
     sel, nsel = _full_selection(fp8, lens)
@@ -38,6 +38,10 @@ def test_fp8_nvfp4_and_centroid_proxy_bytes():
     sel, nsel = _full_selection(ce, lens)
     # one FP32 key sum of d = 128 per 128-token block
     assert bench.step_bytes(ce, lens, sel, nsel)["proxy"] == 16 * 8 * 1024 * 128 * 4
+    rq = synth.RABITQ_TOKEN128K
+    sel, nsel = _full_selection(rq, lens)
+    # 128 code bits (16 bytes) + one FP32 factor per token
+    assert bench.step_bytes(rq, lens, sel, nsel)["proxy"] == 16 * 8 * 131072 * (16 + 4)
 
 
 def test_ragged_lengths_count_valid_tokens_only():

@@ -34,7 +34,12 @@ def test_small_workload_invariants(w):
             L = int(inp.lens[b])
             nb = (L + w.block_size - 1) // w.block_size
             sel = r["sel"]
-            assert len(sel) == min(w.budget, nb)
+            if w.top_p > 0:
+                assert 1 <= len(sel) <= w.budget
+                assert M.top_p_valid(r["mass"], float(np.float32(w.top_p)), w.budget,
+                                     r["forced"], sel)[0]
+            else:
+                assert len(sel) == min(w.budget, nb)
             assert set(r["forced"].tolist()) <= set(sel.tolist())
             if w.force_sink:
                 assert sel[0] == 0
@@ -42,7 +47,7 @@ def test_small_workload_invariants(w):
                 assert sel[-1] == nb - 1
             if w.n_keep_hp:
                 assert len(r["keep"]) == min(w.n_keep_hp, L // w.block_size)
-            if nb <= w.budget:
+            if nb <= w.budget and w.top_p == 0:
                 # budget covers every block: exactly dense attention
                 assert r["tokens"].tolist() == list(range(L))
             assert np.all(np.isfinite(r["out"]))
