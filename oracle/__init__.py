@@ -21,8 +21,12 @@ Pins (what each part is checked against, in tests/test_oracle_*.py):
               mean over random rotations and query roundings against the exact score
               (unbiasedness); identity and signed-permutation rotations; bit packing;
   top-p     - exhaustive subset search on tiny inputs; closed forms for uniform and
-              geometric masses; the budget cap; forced blocks.
+              geometric masses; the budget cap; forced blocks;
+  semantic  - Lloyd's objective never increases; converged partitions are fixed points;
+              exactly placed keys recovered; one token per cluster = token level; cluster
+              score = mean member score; full budget = dense attention; planted cluster.
 Parity unpinned: the aggregation of per-head NVFP4 scores into one block score (max over
-the group's heads) is a reading the pages leave open; only its implementation is pinned.
+the group's heads), and the semantic blocks' clustering (Lloyd's k-means, evenly spaced
+seeds), are readings the pages leave open; only their implementations are pinned.
 """
 from . import formats, method, step  # noqa: F401

@@ -26,6 +26,10 @@ Sources (page title, then the part of the page):
           - Abstract: keys scored through randomised rotated binary quantisation with
             binary-INT4 arithmetic, an unbiased estimator with an error bound, and a top-p
             budget that follows the estimated attention mass.
+  [CSB]   "Coarse Semantic Blocks for Efficient Training-Free Sparse Attention"
+          - Abstract: a prompt-specific key index clusters the keys into large blocks of
+            non-contiguous tokens; a query scores blocks by their centroids and attends to
+            the original keys and values of the blocks it selects.
   [RBQ]   The estimator's published form: J. Gao and C. Long, "RaBitQ: Quantizing
           High-Dimensional Vectors with a Theoretical Error Bound for Approximate Nearest
           Neighbor Search", SIGMOD 2024 (section 3: the codebook, the estimator and its
@@ -665,3 +669,64 @@ def top_p_valid(mass: np.ndarray, p: float, budget: int, forced: np.ndarray, got
     if len(got) == budget or others.size == 0:
         return True, "budget full"
     return False, f"mass {have} short of the goal {goal}"
+
+
+# ============================================================================================
+# Semantic blocks: clustered, non-contiguous key blocks  [CSB, Abstract]
+# The page builds a key index for the prompt: its keys are clustered into large blocks of
+# tokens from anywhere in the prompt; a query scores each block by its centroid and attends
+# to the original keys and values of the blocks it selects. The abstract gives no
+# clustering algorithm. Readings:
+#   * clustering = Lloyd's k-means in Euclidean distance on the stored keys (float64), with
+#     C = ceil(L0 / S) clusters for a prompt of L0 tokens and a target block size S, seeded
+#     with the keys at the evenly spaced positions floor(i * L0 / C), for a fixed number of
+#     iterations; a token joins its nearest centroid (ties: the lower cluster index); an
+#     empty cluster keeps its centroid;
+#   * block score = qbar . centroid, the centroid being the mean of the member keys (so the
+#     score is the mean of the members' exact group-mean scores);
+#   * the budget counts clusters; ties go to the lower cluster index;
+#   * tokens after the prompt (decoded after the index was built) are always attended.
+# The clustering definition is parity unpinned (a reading); its implementation is pinned by
+# the properties of Lloyd's algorithm.
+# ============================================================================================
+
+
+def kmeans_keys(k_bits: np.ndarray, C: int, iters: int):
+    """Cluster keys [L0][d] (BF16) into C groups: (assign [L0] int64, centroids [C][d]).
+
+    Centroids start at the keys at positions floor(i * L0 / C); each iteration assigns every
+    key to its nearest centroid (squared Euclidean distance, ties to the lower index), then
+    moves every non-empty cluster's centroid to the mean of its members.
+    """
+    x = F.bf16_to_f64(k_bits)
+    L0 = x.shape[0]
+    if not (1 <= C <= L0):
+        raise ValueError("need 1 <= C <= L0")
+    cent = x[(np.arange(C) * L0) // C].copy()
+    assign = np.zeros(L0, dtype=np.int64)
+    for _ in range(max(iters, 1)):
+        d2 = ((x[:, None, :] - cent[None, :, :]) ** 2).sum(axis=2)          # [L0][C]
+        assign = np.argmin(d2, axis=1)                                       # first minimum
+        for j in range(C):
+            members = x[assign == j]
+            if len(members):
+                cent[j] = members.mean(axis=0)
+    return assign, cent
+
+
+def kmeans_objective(k_bits: np.ndarray, assign: np.ndarray, cent: np.ndarray) -> float:
+    """Sum over keys of the squared distance to the assigned centroid."""
+    x = F.bf16_to_f64(k_bits)
+    return float(((x - cent[assign]) ** 2).sum())
+
+
+def semantic_block_scores(q_bits: np.ndarray, cent: np.ndarray) -> np.ndarray:
+    """beta_j = qbar . centroid_j (float64); q_bits: the group's BF16 queries [G][d]."""
+    return cent @ F.bf16_to_f64(q_bits).mean(axis=0)
+
+
+def semantic_tokens(assign: np.ndarray, sel: np.ndarray, L0: int, L: int) -> np.ndarray:
+    """The attended positions, ascending: the members of the selected clusters, then every
+    token after the prompt (L0 <= t < L)."""
+    members = np.nonzero(np.isin(assign, np.asarray(sel, dtype=np.int64)))[0]
+    return np.concatenate([members, np.arange(L0, L)]).astype(np.int64)

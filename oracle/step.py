@@ -128,3 +128,30 @@ def decode_row_top_p(p: TopPParams, k_bits, v_bits, q_bits, L: int, R, c, u,
                              decode_v(v_bits[:L], p.v_dtype), tokens, p.scale)
     return dict(bits=bits, g=g, codes=n, delta=delta, vl=vl, qbar=qbar, scores=s, weights=w,
                 mass=mass, forced=forced, sel=sel, tokens=tokens, out=out)
+
+
+# ---- semantic blocks ("Coarse Semantic Blocks ...", Abstract) -------------------------------
+
+@dataclass
+class SemanticParams:
+    S: int                     # target tokens per cluster: C = ceil(L0 / S)
+    budget: int                # clusters selected
+    iters: int                 # Lloyd iterations of the index
+    scale: float               # softmax scale
+    v_dtype: str               # 'bf16' | 'f16'
+
+
+def decode_row_semantic(p: SemanticParams, k_bits, v_bits, q_bits, L0: int, L: int,
+                        sel_override=None):
+    """One row's step with a semantic-block index over its first L0 tokens: cluster the
+    prompt's keys, score the clusters by their centroids, select the top clusters, then
+    exact attention over their members and every token after the prompt."""
+    C = -(-L0 // p.S)
+    assign, cent = M.kmeans_keys(k_bits[:L0], C, p.iters)
+    beta = M.semantic_block_scores(q_bits, cent)
+    sel = M.select_blocks(beta, p.budget, np.zeros(0, dtype=np.int64))
+    use = sel if sel_override is None else np.asarray(sel_override, dtype=np.int64)
+    tokens = M.semantic_tokens(assign, use, L0, L)
+    out = M.sparse_attention(F.bf16_to_f64(q_bits), F.bf16_to_f64(k_bits[:L]),
+                             decode_v(v_bits[:L], p.v_dtype), tokens, p.scale)
+    return dict(assign=assign, centroids=cent, beta=beta, sel=sel, tokens=tokens, out=out)
