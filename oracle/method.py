@@ -44,7 +44,8 @@ Readings where the pages are silent (each listed in the design notes):
 
 Parity pins live in tests/test_oracle_*.py. The aggregation of per-head NVFP4 scores into
 one score per block (max over heads) is a reading the pages do not fix: its *definition*
-is parity unpinned; its implementation is checked by brute force on tiny inputs.
+is parity unpinned; its implementation is checked by brute force on tiny inputs. The same
+holds for the semantic blocks' clustering algorithm.
 """
 from __future__ import annotations
 
