@@ -141,6 +141,8 @@ CASES = [  # (d, S, G, Hkv, budget, lens)
     (128, 16, 4, 2, 24, [1000, 2048, 77]),
     (64, 128, 2, 3, 4, [900, 1280, 300]),
     (128, 64, 5, 1, 6, [1, 640, 385]),
+    (128, 32, 2, 2, 16, [1100, 257, 640]),
+    (64, 4, 8, 1, 64, [513, 1024]),
 ]
 
 
