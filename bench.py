@@ -5,7 +5,8 @@
 
 A step is one qs_decode call over one batch: append the new token of every sequence,
 score the whole key history through the proxy cache, select the top-k blocks per
-(sequence, KV head), and attend over the selected keys and values. The default workload
+(sequence, KV head), and attend over the selected keys and values. For the binary proxy
+(--workload rabitq128k) it is one qs_decode_top_p call, which selects a top-p set. The default workload
 is the 128K-context, batch-16 block-level step (40 query / 8 KV heads, d = 128, rank-32
 BF16 proxy, 128-token blocks, budget 64 with the sink and last blocks forced); its
 seeded synthetic caches (about 9 GiB) exceed the L2, so no flush is needed.
@@ -618,10 +619,11 @@ def run_ours(args):
 
 
 def run_ours_top_p(args, w, inp, f, world, rank, local):
-    """The binary proxy's step ("RaBitQCache", Abstract) through its entry points: append
-    (binary writer), qs_rabitq_score (query code + scan), qs_select_top_p, qs_sparse_attn;
-    timed, broken into stages and run end to end like the fused step of the other proxies
-    (the end-to-end leg issues the four calls eagerly, without a captured graph)."""
+    """The binary proxy's step ("RaBitQCache", Abstract): qs_decode_top_p (append with the
+    binary writer, query code + scan, top-p select, sparse attention) timed like the fused
+    step of the other proxies; the stage breakdown issues the four stage calls with events
+    between them; end to end, the step is captured once into a CUDA graph with its host
+    copies (CapturedDecode) and replayed."""
     import torch
     import torch.distributed as dist
     import score_then_select_b200 as qs
@@ -639,22 +641,21 @@ def run_ours_top_p(args, w, inp, f, world, rank, local):
     stream = torch.cuda.current_stream()
     p = float(w.top_p)
 
-    def step(q, k, v, ev=None):
+    def step(q, k, v):
         lay.seq_lens.copy_(start_lens, non_blocking=True)
-        if ev:
-            ev[0].record(stream)
+        qs.qs_decode_top_p(cfg, cache, q, k, v, f.P, u, p, B, out, sel, nsel, lay.ws, stream)
+
+    def stages(q, k, v, ev):
+        lay.seq_lens.copy_(start_lens, non_blocking=True)
+        ev[0].record(stream)
         qs.qs_append_kv(cfg, cache, k, v, ones, 1, f.P, B, lay.ws, stream)
-        if ev:
-            ev[1].record(stream)
+        ev[1].record(stream)
         qs.qs_rabitq_score(cfg, cache, q, f.P, u, B, scores, lay.ws, stream)
-        if ev:
-            ev[2].record(stream)
+        ev[2].record(stream)
         qs.qs_select_top_p(cfg, cache, scores, p, B, sel, nsel, lay.ws, stream)
-        if ev:
-            ev[3].record(stream)
+        ev[3].record(stream)
         qs.qs_sparse_attn(cfg, cache, q, sel, nsel, B, out, lay.ws, stream)
-        if ev:
-            ev[4].record(stream)
+        ev[4].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step(f.q, f.k_last, f.v_last)
@@ -691,42 +692,37 @@ def run_ours_top_p(args, w, inp, f, world, rank, local):
     n_stage = min(args.steps, 50)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_stage + 3)]
     for ev in evs:
-        step(f.q, f.k_last, f.v_last, ev)
+        stages(f.q, f.k_last, f.v_last, ev)
     torch.cuda.synchronize()
     acc = np.zeros(4)
     for ev in evs[3:]:
         acc += [ev[j].elapsed_time(ev[j + 1]) for j in range(4)]
     stage_us = dict(zip(["append", "score", "select", "attend"], (acc / n_stage * 1e3).tolist()))
 
-    # ---------------- end to end: q, k_new, v_new from pinned host memory, the four calls,
-    # the output back to the host, then a sync
-    q_h = f.q.cpu().pin_memory()
-    k_h = f.k_last.cpu().pin_memory()
-    v_h = f.v_last.cpu().pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    q_d, k_d, v_d = torch.empty_like(f.q), torch.empty_like(f.k_last), torch.empty_like(f.v_last)
-
-    def e2e_step():
-        q_d.copy_(q_h, non_blocking=True)
-        k_d.copy_(k_h, non_blocking=True)
-        v_d.copy_(v_h, non_blocking=True)
-        step(q_d, k_d, v_d)
-        out_h.copy_(out, non_blocking=True)
-        stream.synchronize()
-
+    # ---------------- end to end: the step captured once with its host copies (q, k_new,
+    # v_new from pinned host memory in one packed copy; the output back to pinned memory)
+    # and replayed; each replay is followed by a sync
+    from score_then_select_b200.graph import CapturedDecode
+    cap = CapturedDecode(
+        cfg, cache, f.P, B, out, sel, nsel, lay.ws, f.q, f.k_last, f.v_last,
+        before=lambda: lay.seq_lens.copy_(start_lens, non_blocking=True),
+        call=lambda q, k, v, s_: qs.qs_decode_top_p(cfg, cache, q, k, v, f.P, u, p, B, out,
+                                                    sel, nsel, lay.ws, s_))
+    cap.q_host.copy_(f.q.cpu())
+    cap.k_host.copy_(f.k_last.cpu())
+    cap.v_host.copy_(f.v_last.cpu())
     for _ in range(3):
-        e2e_step()
+        cap.step()
     n_e2e = max(args.steps, 10)
     barrier()
     t0 = time.perf_counter()
     for _ in range(n_e2e):
-        e2e_step()
+        cap.step()
     e2e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3 / n_e2e, world, "cuda")
     st = qs.qs_device_status(lay.ws)
     if st[0] != 0:
         raise RuntimeError(f"device status after the end-to-end runs {st}")
-    h2d = q_h.numel() * q_h.element_size() + 2 * k_h.numel() * k_h.element_size()
-    d2h = out_h.numel() * out_h.element_size()
+    h2d, d2h = cap.h2d_bytes, cap.d2h_bytes
 
     # ---------------- roofline: the scan (query code + binary scan, one qs_rabitq_score)
     peak, peak_src = peaks()
@@ -753,7 +749,8 @@ def run_ours_top_p(args, w, inp, f, world, rank, local):
             "stage_us": stage_us, "roofline": roof, "clocks": clk,
             "e2e": {"value": aggregate_steps_per_s(e2e_ms, world), "unit": "steps/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms, "path": "eager calls of the four entry points"},
+                    "ms_per_step": e2e_ms,
+                    "path": "CapturedDecode (CUDA graph of qs_decode_top_p)"},
             "gpu_launches": args.steps * launches_per_step}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_rows)

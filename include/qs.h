@@ -231,9 +231,8 @@ qs_status qs_sparse_attn(const qs_config *cfg, const qs_cache *cache, const void
 
 /* One decode step: append one token per sequence (k_new/v_new: [batch][Hkv][d]), then
    score, select and attend over seq_len + 1 tokens. sel_out / n_sel_out may be NULL; the
-   selection then stays in the workspace. The binary proxy with its top-p budget runs as
-   separate calls (qs_append_kv, qs_rabitq_score, qs_select_top_p, qs_sparse_attn); this
-   call returns QS_ERR_UNSUPPORTED for it. */
+   selection then stays in the workspace. The binary proxy with its top-p budget has its
+   own step call, qs_decode_top_p; this call returns QS_ERR_UNSUPPORTED for it. */
 qs_status qs_decode(const qs_config *cfg, const qs_cache *cache, const void *q,
                     const void *k_new, const void *v_new, const float *P, int32_t batch,
                     void *out, int32_t *sel_out, int32_t *n_sel_out, void *ws,
@@ -273,6 +272,18 @@ qs_status qs_rabitq_score(const qs_config *cfg, const qs_cache *cache, const voi
 qs_status qs_select_top_p(const qs_config *cfg, const qs_cache *cache,
                           const float *block_scores, float p, int32_t batch, int32_t *sel,
                           int32_t *n_sel, void *ws, qs_stream_t stream);
+
+/* One decode step with the binary proxy, as qs_decode is for the others: append one token
+   per sequence (k_new / v_new: [batch][Hkv][d]; the binary writer with R), then
+   qs_rabitq_score, qs_select_top_p with p, and qs_sparse_attn over seq_len + 1 tokens, in
+   stream order (5 launches, plus the row merge when the tile pipeline runs). The block
+   scores live in the workspace; sel_out / n_sel_out may both be NULL, the selection then
+   stays in the workspace too. Arguments and statuses as in the four calls. */
+qs_status qs_decode_top_p(const qs_config *cfg, const qs_cache *cache, const void *q,
+                          const void *k_new, const void *v_new, const float *R,
+                          const float *u, float p, int32_t batch, void *out,
+                          int32_t *sel_out, int32_t *n_sel_out, void *ws,
+                          qs_stream_t stream);
 
 /* ---- Comparison kernels: full-KV attention and gather-then-attend -----------------------
    "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 2 (b) and

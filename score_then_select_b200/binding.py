@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "qs_calibrate_basis": ([cfgp, vp, vp, i32, vp, vp, vp, vp], i32),
             "qs_rabitq_score": ([cfgp, cachep, vp, vp, vp, i32, vp, vp, vp], i32),
             "qs_select_top_p": ([cfgp, cachep, vp, ctypes.c_float, i32, vp, vp, vp, vp], i32),
+            "qs_decode_top_p": ([cfgp, cachep, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp,
+                                 vp, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -90,7 +92,7 @@ EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_
            "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches",
            "qs_selftest_wait_timeout", "qs_dense_workspace_size", "qs_dense_attn",
            "qs_gather_kv", "qs_calib_workspace_size", "qs_calibrate_basis", "qs_rabitq_score",
-           "qs_select_top_p")
+           "qs_select_top_p", "qs_decode_top_p")
 
 
 def status_string(s: int) -> str:
@@ -273,6 +275,16 @@ def qs_select_top_p(cfg, cache, block_scores, p, batch, sel, n_sel, ws, stream=N
     _check(lib().qs_select_top_p(ctypes.byref(cfg), ctypes.byref(cache), _ptr(block_scores),
                                  float(p), batch, _ptr(sel), _ptr(n_sel), _ptr(ws),
                                  _stream(stream)), "qs_select_top_p")
+
+
+def qs_decode_top_p(cfg, cache, q, k_new, v_new, R, u, p, batch, out, sel_out, n_sel_out, ws,
+                    stream=None):
+    """One decode step with the binary proxy: append, qs_rabitq_score, qs_select_top_p and
+    qs_sparse_attn in stream order (sel_out / n_sel_out may both be None)."""
+    _check(lib().qs_decode_top_p(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(k_new),
+                                 _ptr(v_new), _ptr(R), _ptr(u), float(p), batch, _ptr(out),
+                                 _ptr(sel_out), _ptr(n_sel_out), _ptr(ws), _stream(stream)),
+           "qs_decode_top_p")
 
 
 def qs_device_status(ws, stream=None) -> tuple[int, int, int]:

@@ -579,53 +579,42 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   return do_attend(p, cache, q, sel, nsel, out, ws, stream, true);
 }
 
-qs_status qs_rabitq_score(const qs_config* cfg, const qs_cache* cache, const void* q,
-                          const float* R, const float* u, int32_t batch, float* block_scores,
-                          void* ws, qs_stream_t stream) {
-  Plan p;
-  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
-  if (st != QS_OK) return st;
-  if (p.kind != PK_RABITQ) return QS_ERR_UNSUPPORTED;
-  if ((st = check_cache(p, cache, true)) != QS_OK) return st;
-  if (!q || !aligned(q, 4) || !R || !aligned(R, 16) || !u || !block_scores || !ws ||
-      !aligned(ws, 256))
-    return QS_ERR_INVALID_ARG;
+}  // extern "C"
+
+// ------------------------------------------------------------ binary proxy (validated input)
+namespace qs {
+
+static qs_status do_rq_score(const Plan& p, const qs_cache* c, const void* q, const float* R,
+                             const float* u, float* scores, void* ws, cudaStream_t s) {
   uint32_t* qcode = ws_at<uint32_t>(ws, p.ws.qt);
-  RqPrepParams a{static_cast<const uint16_t*>(q), R, u, cache->key_center, qcode,
+  RqPrepParams a{static_cast<const uint16_t*>(q), R, u, c->key_center, qcode,
                  p.batch, p.Hkv, p.G, p.d};
-  if ((st = cuda_status(launch_rq_prep(a, stream))) != QS_OK) return st;
+  const qs_status st = cuda_status(launch_rq_prep(a, s));
+  if (st != QS_OK) return st;
   RqScoreParams b{};
-  b.proxy = static_cast<const uint8_t*>(cache->proxy);
+  b.proxy = static_cast<const uint8_t*>(c->proxy);
   b.qcode = qcode;
-  b.page_table = cache->page_table;
-  b.seq_lens = cache->seq_lens;
-  b.scores = block_scores;
+  b.page_table = c->page_table;
+  b.seq_lens = c->seq_lens;
+  b.scores = scores;
   b.hdr = hdr_of(ws);
   b.batch = p.batch;
   b.Hkv = p.Hkv;
   b.d = p.d;
   b.S = p.S;
   b.nb_stride = p.nb_stride;
-  b.max_pages_per_seq = cache->max_pages_per_seq;
-  b.num_pages = cache->num_pages;
-  b.max_context = cache->max_context;
+  b.max_pages_per_seq = c->max_pages_per_seq;
+  b.num_pages = c->num_pages;
+  b.max_context = c->max_context;
   b.scale = p.scale;
-  return cuda_status(launch_rq_score(b, stream));
+  return cuda_status(launch_rq_score(b, s));
 }
 
-qs_status qs_select_top_p(const qs_config* cfg, const qs_cache* cache, const float* block_scores,
-                          float p_mass, int32_t batch, int32_t* sel, int32_t* n_sel, void* ws,
-                          qs_stream_t stream) {
-  Plan p;
-  const qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
-  if (st != QS_OK) return st;
-  if (!cache || !cache->seq_lens) return QS_ERR_INVALID_ARG;
-  if (!block_scores || !sel || !n_sel || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
-  if (!(p_mass > 0.0f && p_mass <= 1.0f)) return QS_ERR_INVALID_ARG;
-  if (p.budget < p.force_sink + p.force_last) return QS_ERR_INVALID_ARG;
+static qs_status do_top_p(const Plan& p, const qs_cache* c, const float* scores, float p_mass,
+                          int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t s) {
   TopPParams a{};
-  a.scores = block_scores;
-  a.seq_lens = cache->seq_lens;
+  a.scores = scores;
+  a.seq_lens = c->seq_lens;
   a.sel = sel;
   a.n_sel = n_sel;
   a.hdr = hdr_of(ws);
@@ -637,7 +626,66 @@ qs_status qs_select_top_p(const qs_config* cfg, const qs_cache* cache, const flo
   a.force_sink = p.force_sink;
   a.force_last = p.force_last;
   a.p = p_mass;
-  return cuda_status(launch_top_p(a, stream));
+  return cuda_status(launch_top_p(a, s));
+}
+
+static bool top_p_args_ok(const Plan& p, float p_mass) {
+  return p_mass > 0.0f && p_mass <= 1.0f && p.budget >= p.force_sink + p.force_last;
+}
+
+}  // namespace qs
+
+extern "C" {
+
+qs_status qs_rabitq_score(const qs_config* cfg, const qs_cache* cache, const void* q,
+                          const float* R, const float* u, int32_t batch, float* block_scores,
+                          void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (p.kind != PK_RABITQ) return QS_ERR_UNSUPPORTED;
+  if ((st = check_cache(p, cache, true)) != QS_OK) return st;
+  if (!q || !aligned(q, 4) || !R || !aligned(R, 16) || !u || !block_scores || !ws ||
+      !aligned(ws, 256))
+    return QS_ERR_INVALID_ARG;
+  return do_rq_score(p, cache, q, R, u, block_scores, ws, stream);
+}
+
+qs_status qs_select_top_p(const qs_config* cfg, const qs_cache* cache, const float* block_scores,
+                          float p_mass, int32_t batch, int32_t* sel, int32_t* n_sel, void* ws,
+                          qs_stream_t stream) {
+  Plan p;
+  const qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (!cache || !cache->seq_lens) return QS_ERR_INVALID_ARG;
+  if (!block_scores || !sel || !n_sel || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (!top_p_args_ok(p, p_mass)) return QS_ERR_INVALID_ARG;
+  return do_top_p(p, cache, block_scores, p_mass, sel, n_sel, ws, stream);
+}
+
+qs_status qs_decode_top_p(const qs_config* cfg, const qs_cache* cache, const void* q,
+                          const void* k_new, const void* v_new, const float* R, const float* u,
+                          float p_mass, int32_t batch, void* out, int32_t* sel_out,
+                          int32_t* n_sel_out, void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (p.kind != PK_RABITQ) return QS_ERR_UNSUPPORTED;
+  if ((st = check_cache(p, cache, true)) != QS_OK) return st;
+  if (!q || !aligned(q, 16) || !k_new || !v_new || !out || !ws || !aligned(ws, 256))
+    return QS_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
+  if (!R || !aligned(R, 16) || !u) return QS_ERR_INVALID_ARG;
+  if (!top_p_args_ok(p, p_mass)) return QS_ERR_INVALID_ARG;
+  if ((sel_out == nullptr) != (n_sel_out == nullptr)) return QS_ERR_INVALID_ARG;
+  int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, p.ws.sel);
+  int32_t* nsel = n_sel_out ? n_sel_out : ws_at<int32_t>(ws, p.ws.nsel);
+  float* scores = ws_at<float>(ws, p.ws.scores);
+  if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, R, nullptr, ws, stream)) != QS_OK)
+    return st;
+  if ((st = do_rq_score(p, cache, q, R, u, scores, ws, stream)) != QS_OK) return st;
+  if ((st = do_top_p(p, cache, scores, p_mass, sel, nsel, ws, stream)) != QS_OK) return st;
+  return do_attend(p, cache, q, sel, nsel, out, ws, stream, false);
 }
 
 qs_status qs_device_status(void* ws, qs_stream_t stream, uint32_t* detail) {

@@ -19,10 +19,12 @@ _ALIGN = 256
 
 class CapturedDecode:
     def __init__(self, cfg, cache, P, batch, out, sel, nsel, ws, q_like, k_like, v_like,
-                 before=None, warmup: int = 2):
+                 before=None, warmup: int = 2, call=None):
         """`q_like`, `k_like`, `v_like`: tensors giving the shapes and dtypes of the step's
         inputs. `before`: an optional callable recorded ahead of the copy (e.g. a
-        device-side reset the caller wants replayed every step)."""
+        device-side reset the caller wants replayed every step). `call`: an optional
+        callable (q, k_new, v_new, stream) that issues the step instead of qs_decode, e.g.
+        qs_decode_top_p with its extra arguments bound."""
         offs, total = [], 0
         for t in (q_like, k_like, v_like):
             offs.append(total)
@@ -48,7 +50,10 @@ class CapturedDecode:
             if before is not None:
                 before()
             self.dev_buf.copy_(self.host_buf, non_blocking=True)
-            B.qs_decode(*args, stream=self.stream)
+            if call is None:
+                B.qs_decode(*args, stream=self.stream)
+            else:
+                call(q_dev, k_dev, v_dev, self.stream)
             self.out_host.copy_(out, non_blocking=True)
 
         self.stream.wait_stream(torch.cuda.current_stream())

@@ -221,3 +221,14 @@ def test_binary_proxy_configuration_and_calls_validate_on_the_host():
         qs.qs_select_top_p(_cfg(budget=1, **{k: v for k, v in rq.items() if k != "budget"}),
                            cache, a, 0.5, 4, a, a, a, stream=0)
     assert e.value.status == B.QS_ERR_INVALID_ARG
+    # the binary step: its own proxy only, its rotation and draws, 0 < p <= 1
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_decode_top_p(_cfg(), cache, a, a, a, a, a, 0.9, 4, a, None, None, a, stream=0)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    for R, u, p in ((None, a, 0.9), (a, None, 0.9), (a, a, 0.0), (a, a, 1.01)):
+        with pytest.raises(qs.QsError) as e:
+            qs.qs_decode_top_p(cfg, cache, a, a, a, R, u, p, 4, a, None, None, a, stream=0)
+        assert e.value.status == B.QS_ERR_INVALID_ARG, (R, u, p)
+    with pytest.raises(qs.QsError) as e:                      # sel_out without n_sel_out
+        qs.qs_decode_top_p(cfg, cache, a, a, a, a, a, 0.9, 4, a, a, None, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
