@@ -283,6 +283,16 @@ def test_top_p_geometric_masses_closed_form():
         assert got.tolist() == sorted(pos[:k].tolist()), p
 
 
+def test_top_p_goal_reached_exactly_stops():
+    """Dyadic masses sum exactly: a set whose mass equals p * total reaches the goal, so
+    nothing more is taken ("reaches" is >=, the fewest blocks)."""
+    mass = np.array([0.125, 0.5, 0.125, 0.25])
+    assert M.select_top_p(mass, 0.75, 4, np.zeros(0)).tolist() == [1, 3]
+    assert M.select_top_p(mass, 0.5, 4, np.zeros(0)).tolist() == [1]
+    assert M.select_top_p(np.full(4, 0.25), 0.5, 4, np.zeros(0)).tolist() == [0, 1]
+    assert M.select_top_p(mass, 1.0, 4, np.zeros(0)).tolist() == [0, 1, 2, 3]
+
+
 def test_top_p_budget_caps_and_forced_blocks_count():
     mass = np.array([0.01, 0.3, 0.05, 0.2, 0.25, 0.04, 0.15])
     assert M.select_top_p(mass, 0.99, 3, np.zeros(0)).tolist() == [1, 3, 4]
