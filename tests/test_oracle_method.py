@@ -46,6 +46,17 @@ def test_proxy_summation_order_is_ascending():
     assert M.proxy_keys_f32(k, P)[0, 0] == 0.0
 
 
+def test_proxy_rounds_each_product_before_adding():
+    # The first term is -(1 + 2^-7 + 2^-23), exact. The second is (1 + 2^-7)(1 + 2^-23) =
+    # 1 + 2^-7 + 2^-23 + 2^-30: rounded to float32 first, it cancels the first exactly; a
+    # fused multiply-add onto the first would leave 2^-30.
+    k = _bf16(np.array([[-1.0, 1.0 + 2.0 ** -7]]))
+    assert F.bf16_to_f64(k)[0, 1] == 1.0 + 2.0 ** -7
+    P = np.array([[1.0 + 2.0 ** -7 + 2.0 ** -23], [1.0 + 2.0 ** -23]], dtype=np.float32)
+    assert float(P[0, 0]) == 1.0 + 2.0 ** -7 + 2.0 ** -23
+    assert M.proxy_keys_f32(k, P)[0, 0] == 0.0
+
+
 def test_proxy_float32_error_bound():
     rng = np.random.default_rng(2)
     d, r = 128, 32

@@ -157,6 +157,19 @@ def test_signed_permutation_moves_and_flips_the_bits():
     assert np.allclose(g, g0, rtol=2e-6, atol=0)
 
 
+def test_rotation_rounds_each_product_before_adding():
+    """y_0 = -(1 + 2^-7 + 2^-23) + fp32((1 + 2^-7)(1 + 2^-23)) = 0 exactly, so its code bit
+    is 0; a fused multiply-add would leave +2^-30 and set the bit."""
+    k_bits = _bf(np.array([[-1.0, 1.0 + 2.0 ** -7]]))
+    R = np.zeros((2, 2), dtype=np.float32)
+    R[0, 0], R[1, 0] = 1.0 + 2.0 ** -7 + 2.0 ** -23, 1.0 + 2.0 ** -23
+    R[0, 1] = 1.0
+    bits, g = M.rabitq_encode(k_bits, R, np.zeros(2, dtype=np.float32))
+    assert bits[0].tolist() == [0, 0]
+    # |y|_1 = |y_1| = 1 and |o|^2 = 1 + (1 + 2^-7)^2 in float32
+    assert g[0] == np.float32(np.float32(1.0) + np.float32((1.0 + 2.0 ** -7) ** 2))
+
+
 def test_key_equal_to_the_centre_has_zero_factor():
     c = np.linspace(-1, 1, 16).astype(np.float32)
     k_bits = _bf(c[None, :])
