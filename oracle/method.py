@@ -731,3 +731,38 @@ def semantic_tokens(assign: np.ndarray, sel: np.ndarray, L0: int, L: int) -> np.
     token after the prompt (L0 <= t < L)."""
     members = np.nonzero(np.isin(assign, np.asarray(sel, dtype=np.int64)))[0]
     return np.concatenate([members, np.arange(L0, L)]).astype(np.int64)
+
+
+def kmeans_keys_f32(k_bits: np.ndarray, C: int, iters: int):
+    """kmeans_keys with every decision taken in float32 in a fixed order, as a kernel takes
+    it: (assign [L0] int64, centroids [C][d] float32).
+
+    x = fp32(k). Seeds: the keys at floor(i * L0 / C). Per iteration:
+      * distance d_tj = sum over i ascending of fp32((x_ti - c_ji)^2), each difference,
+        square and partial sum rounded to float32; a key joins the smallest d_tj (ties:
+        the lower cluster index);
+      * a non-empty cluster's centroid becomes fp32(fp32 sum of its members in token order,
+        dimension by dimension, one rounding per add) / fp32(count); an empty one keeps
+        its centroid.
+    """
+    x = F.bf16_to_f64(k_bits).astype(np.float32)
+    L0, d = x.shape
+    if not (1 <= C <= L0):
+        raise ValueError("need 1 <= C <= L0")
+    cent = x[(np.arange(C) * L0) // C].copy()
+    assign = np.zeros(L0, dtype=np.int64)
+    for _ in range(max(iters, 1)):
+        acc = np.zeros((L0, C), dtype=np.float32)
+        for i in range(d):
+            diff = (x[:, i:i + 1] - cent[None, :, i]).astype(np.float32)
+            acc = (acc + (diff * diff).astype(np.float32)).astype(np.float32)
+        assign = np.argmin(acc, axis=1)                                      # first minimum
+        for j in range(C):
+            members = np.nonzero(assign == j)[0]
+            if len(members) == 0:
+                continue
+            s = np.zeros(d, dtype=np.float32)
+            for t in members:                                                # token order
+                s = (s + x[t]).astype(np.float32)
+            cent[j] = (s / np.float32(len(members))).astype(np.float32)
+    return assign, cent

@@ -107,13 +107,33 @@ MUTATIONS = [
     # semantic blocks
     ("method", "k-means: farthest centroid", "assign = np.argmin(d2, axis=1)",
      "assign = np.argmax(d2, axis=1)"),
-    ("method", "k-means: seeds at the first C keys", "cent = x[(np.arange(C) * L0) // C].copy()",
-     "cent = x[np.arange(C)].copy()"),
+    ("method", "k-means: seeds at the first C keys",
+     "cent = x[(np.arange(C) * L0) // C].copy()\n    assign = np.zeros(L0, dtype=np.int64)\n"
+     "    for _ in range(max(iters, 1)):\n        d2",
+     "cent = x[np.arange(C)].copy()\n    assign = np.zeros(L0, dtype=np.int64)\n"
+     "    for _ in range(max(iters, 1)):\n        d2"),
+    ("method", "k-means float32: seeds at the first C keys",
+     "cent = x[(np.arange(C) * L0) // C].copy()\n    assign = np.zeros(L0, dtype=np.int64)\n"
+     "    for _ in range(max(iters, 1)):\n        acc",
+     "cent = x[np.arange(C)].copy()\n    assign = np.zeros(L0, dtype=np.int64)\n"
+     "    for _ in range(max(iters, 1)):\n        acc"),
     ("method", "semantic: head sum, not mean", "return cent @ F.bf16_to_f64(q_bits).mean(axis=0)",
      "return cent @ F.bf16_to_f64(q_bits).sum(axis=0)"),
     ("method", "semantic: tokens after the prompt dropped",
      "return np.concatenate([members, np.arange(L0, L)]).astype(np.int64)",
      "return members.astype(np.int64)"),
+    ("method", "k-means float32: distances in float64",
+     "        acc = np.zeros((L0, C), dtype=np.float32)\n        for i in range(d):\n"
+     "            diff = (x[:, i:i + 1] - cent[None, :, i]).astype(np.float32)\n"
+     "            acc = (acc + (diff * diff).astype(np.float32)).astype(np.float32)",
+     "        acc = ((x[:, None, :].astype(np.float64) - cent[None, :, :]) ** 2).sum(axis=2)"),
+    ("method", "k-means float32: dimensions summed in reverse",
+     "        for i in range(d):\n            diff = (x[:, i:i + 1] - cent[None, :, i]).astype(np.float32)",
+     "        for i in reversed(range(d)):\n            diff = (x[:, i:i + 1] - cent[None, :, i]).astype(np.float32)"),
+    ("method", "k-means float32: members summed pairwise",
+     "            s = np.zeros(d, dtype=np.float32)\n            for t in members:                                                # token order\n"
+     "                s = (s + x[t]).astype(np.float32)",
+     "            s = x[members].sum(axis=0, dtype=np.float64).astype(np.float32)"),
     # number formats
     ("formats", "BF16: ties away from zero", "y = np.round(x64 / step) * step            # np.round is half-to-even",
      "y = np.floor(x64 / step + 0.5) * step"),

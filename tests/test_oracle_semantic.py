@@ -138,3 +138,45 @@ def test_planted_non_contiguous_cluster_is_selected():
     assert set(planted.tolist()) <= set(members.tolist())
     assert set(range(L0, L)) <= set(r["tokens"].tolist())
     assert np.all(np.diff(r["tokens"]) > 0)
+
+
+# ---- the float32 definition a kernel matches bit for bit --------------------------------------
+
+def test_f32_distance_is_summed_in_float32_in_dimension_order():
+    """Key (4096, 1, 1) against seeds (0, 0, 0) and (0, 1, 0): squared terms 2^24, 1, 1.
+    In float32, in dimension order, both distances are 2^24, a tie won by cluster 0. In
+    float64 (2^24 + 2 against 2^24 + 1), or in float32 in reversed order (2^24 + 2 against
+    2^24), cluster 1 wins."""
+    k = _bf(np.array([[0.0, 0.0, 0.0], [0.0, 1.0, 0.0], [4096.0, 1.0, 1.0]]))
+    a32, _ = M.kmeans_keys_f32(k, 2, 1)
+    a64, _ = M.kmeans_keys(k, 2, 1)
+    assert a32.tolist() == [0, 1, 0]
+    assert a64.tolist() == [0, 1, 1]
+
+
+def test_f32_centroid_sums_members_in_token_order():
+    """One cluster of 2^24, 1, -2^24: in float32 in token order the 1 is lost (mean 0);
+    the exact mean is 1/3."""
+    k = _bf(np.array([[2.0 ** 24], [1.0], [-(2.0 ** 24)]]))
+    _, c32 = M.kmeans_keys_f32(k, 1, 1)
+    _, c64 = M.kmeans_keys(k, 1, 1)
+    assert c32.dtype == np.float32 and c32[0, 0] == 0.0
+    assert abs(c64[0, 0] - 1.0 / 3.0) < 1e-15
+
+
+def test_f32_definition_agrees_with_the_reading_away_from_ties():
+    rng = np.random.default_rng(9)
+    k = _mixture(rng, 1500, 32, 8, spread=5.0, noise=0.4)
+    a32, c32 = M.kmeans_keys_f32(k, 12, 6)
+    a64, c64 = M.kmeans_keys(k, 12, 6)
+    assert np.array_equal(a32, a64)
+    assert np.abs(c32 - c64).max() < 1e-5
+    # exactly placed keys: identical, centroids exact
+    C, L0 = 4, 64
+    points = np.zeros((C, 8))
+    points[np.arange(C), np.arange(C)] = 4.0
+    lab = rng.integers(0, C, size=L0)
+    lab[(np.arange(C) * L0) // C] = np.arange(C)
+    kk = _bf(points[lab])
+    a, c = M.kmeans_keys_f32(kk, C, 2)
+    assert np.array_equal(a, lab) and np.array_equal(c.astype(np.float64), points)
