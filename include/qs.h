@@ -23,6 +23,10 @@
  *     Full text: NVFP4 scoring keys scanned densely on FP4 tensor cores; 128-token blocks;
  *     FP16 value aggregation with FP32 accumulation; calibrated key centring; at most two
  *     blocks kept at BF16 per sequence; the cache is packed directly from BF16 activations.
+ *   "Coarse Semantic Blocks for Efficient Training-Free Sparse Attention" (Abstract): a
+ *     prompt-specific key index: the prompt's keys clustered into large blocks of
+ *     non-contiguous tokens, scored by their centroids; the selected blocks' original keys
+ *     and values are attended.
  *   "RaBitQCache" (Abstract): keys scored through randomly rotated binary codes with
  *     binary-INT4 arithmetic (an unbiased estimate of q . k) and a top-p budget that grows
  *     the attended set until the estimated attention mass reaches p. The estimator is the
@@ -106,7 +110,8 @@ typedef enum {
 typedef enum {
   QS_F32 = 0, QS_BF16 = 1, QS_F16 = 2, QS_NVFP4 = 3, QS_E4M3 = 4,
   QS_CENTROID = 5,  /* proxy_dtype only: per-block FP32 key sums (centroid scoring), r = 0 */
-  QS_RABITQ = 6     /* proxy_dtype only: binary codes of rotated centred keys, r = 0      */
+  QS_RABITQ = 6,    /* proxy_dtype only: binary codes of rotated centred keys, r = 0      */
+  QS_SEMANTIC = 7   /* proxy_dtype only: semantic-block index outside the cache, r = 0   */
 } qs_dtype;
 
 /* Problem statement of one attention layer's decode step. */
@@ -118,8 +123,8 @@ typedef struct {
   int32_t block_size;     /* S: a power of two dividing page_size (1 = token level)       */
   int32_t budget;         /* k: blocks selected per row, >= 1                             */
   int32_t proxy_rank;     /* r > 0: projected-key proxy; 0: NVFP4, centroid or binary     */
-  int32_t proxy_dtype;    /* qs_dtype: F32, BF16 or E4M3 (rank r); NVFP4, CENTROID or
-                             RABITQ (r 0)                                                 */
+  int32_t proxy_dtype;    /* qs_dtype: F32, BF16 or E4M3 (rank r); NVFP4, CENTROID, RABITQ
+                             or SEMANTIC (r 0)                                            */
   int32_t v_dtype;        /* qs_dtype of stored V: BF16 or F16                            */
   int32_t v_agg_dtype;    /* precision of the P.V operands: BF16 or F16 (FP32 accumulate) */
   int32_t out_dtype;      /* F32 or BF16                                                  */
@@ -285,6 +290,62 @@ qs_status qs_decode_top_p(const qs_config *cfg, const qs_cache *cache, const voi
                           int32_t *sel_out, int32_t *n_sel_out, void *ws,
                           qs_stream_t stream);
 
+/* ---- Semantic blocks ("Coarse Semantic Blocks ...", Abstract) ---------------------------
+   The index covers each sequence's prompt (L0 = prompt_lens[b] tokens already in the
+   cache); it is built once, and every decode step scores it. With cfg->proxy_dtype =
+   QS_SEMANTIC (rank 0), cfg->block_size S is the target cluster size and cfg->budget the
+   number of clusters selected. C_b = ceil(L0_b / S) clusters; C_max = ceil(max_context / S).
+   Index of row (b, g) = b * Hkv + g:
+     centroids [rows][C_max][head_dim] F32;
+     offsets   [rows][C_max + 1] int32: cluster j's members are members[offsets[j] ..
+               offsets[j + 1]) of the row;
+     members   [rows][max_context] int32 token positions, grouped by cluster, ascending
+               within a cluster.
+   The clustering is Lloyd's k-means with every decision in float32 in a fixed order:
+     seeds c_j = fp32(key at floor(j * L0 / C)); then, `iters` times,
+     assign: d_tj = sum over i ascending of fp32((x_ti - c_ji)^2) (one rounding per
+             difference, square and add); key t joins the smallest d_tj, ties to the lower j;
+     update: c_j = fp32(sum of the members' keys in token order) / fp32(count); an empty
+             cluster keeps its centroid.
+   Tokens appended after the index was built are not in it: qs_append_kv with this
+   proxy_dtype writes their K/V only, and qs_semantic_select always adds them. */
+
+/* Workspace bytes for qs_semantic_index (host only): 256 + 4 * rows * (max_context +
+   C_max). QS_ERR_UNSUPPORTED unless proxy_dtype is QS_SEMANTIC. */
+qs_status qs_semantic_index_workspace_size(const qs_config *cfg, int32_t batch,
+                                           int32_t max_context, size_t *bytes /* host */);
+
+/* Build the index of every row from the cached keys (K pages only; the cache's proxy
+   fields are not read). prompt_lens: device int32 [batch], each <= cache->max_context
+   (larger values are clamped). iters >= 1. Outputs as laid out above; entries past a row's
+   C_b clusters or L0 members are not written. ws: qs_semantic_index_workspace_size bytes,
+   256-byte aligned, its first 256 bytes zeroed once (qs_workspace_init). 1 + 3 * iters
+   launches. A page-table entry that is not mapped records QS_ERR_DEVICE_BOUNDS (kernel
+   id 9). */
+qs_status qs_semantic_index(const qs_config *cfg, const qs_cache *cache,
+                            const int32_t *prompt_lens, int32_t iters, float *centroids,
+                            int32_t *offsets, int32_t *members, int32_t batch, void *ws,
+                            qs_stream_t stream);
+
+/* One decode step's selection over the index (3 launches):
+     beta_j = qbar . c_j (float32; qbar = the mean of the group's query heads), for
+       j < C_b;
+     the cfg->budget best clusters, ties to the lower index (all of them if C_b <= budget;
+       no forced clusters);
+     tokens[row] = the members of the selected clusters (clusters in ascending order, each
+       cluster's members ascending), then every token L0 <= t < seq_len; n_tokens[row] =
+       their count; the rest of the row is padded with -1.
+   Attend with qs_sparse_attn on a configuration equal to cfg except block_size = 1 and
+   budget = max_tokens (and a workspace sized for it), passing tokens / n_tokens as the
+   selection. tokens: [rows][max_tokens] int32; a row needing more than max_tokens entries
+   is cut and records QS_ERR_DEVICE_BOUNDS (kernel id 9). ws: qs_workspace_size(cfg, ...)
+   bytes. q: [batch][Hq][head_dim] BF16, 4-byte aligned. */
+qs_status qs_semantic_select(const qs_config *cfg, const qs_cache *cache, const void *q,
+                             const int32_t *prompt_lens, const float *centroids,
+                             const int32_t *offsets, const int32_t *members, int32_t batch,
+                             int32_t *tokens, int32_t *n_tokens, int32_t max_tokens, void *ws,
+                             qs_stream_t stream);
+
 /* ---- Comparison kernels: full-KV attention and gather-then-attend -----------------------
    "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Figure 2 (b) and
    Figure 6 (a), compare the sparse attention stage with attention over the whole cache
@@ -356,8 +417,8 @@ qs_status qs_calibrate_basis(const qs_config *cfg, const void *q, const void *k,
    receives {kernel id, index} of that error. Returns QS_ERR_CUDA if the synchronisation
    or the read-back fails. Kernel ids: 1 append, 2 block error, 3 scoring prep, 4 score,
    5 select, 6 attention (with its log-sum-exp combine), 7 the wait self-test,
-   8 the gather of gather-then-attend. The binary proxy's writer, scan and top-p selection
-   report as 1, 4 and 5. */
+   8 the gather of gather-then-attend, 9 the semantic-block index and expansion. The binary
+   proxy's writer, scan and top-p selection report as 1, 4 and 5. */
 qs_status qs_device_status(void *ws, qs_stream_t stream, uint32_t *detail);
 
 /* Sparse attention without a workspace, for callers that cannot allocate device memory:

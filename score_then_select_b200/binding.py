@@ -14,9 +14,10 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqs.so")
 
 QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA, QS_ERR_DEVICE_BOUNDS, \
     QS_ERR_DEVICE_TIMEOUT = range(6)
-QS_F32, QS_BF16, QS_F16, QS_NVFP4, QS_E4M3, QS_CENTROID, QS_RABITQ = range(7)
+QS_F32, QS_BF16, QS_F16, QS_NVFP4, QS_E4M3, QS_CENTROID, QS_RABITQ, QS_SEMANTIC = range(8)
 DTYPE_CODES = {"f32": QS_F32, "bf16": QS_BF16, "f16": QS_F16, "nvfp4": QS_NVFP4,
-               "e4m3": QS_E4M3, "centroid": QS_CENTROID, "rabitq": QS_RABITQ}
+               "e4m3": QS_E4M3, "centroid": QS_CENTROID, "rabitq": QS_RABITQ,
+               "semantic": QS_SEMANTIC}
 
 
 class QsError(RuntimeError):
@@ -78,6 +79,10 @@ def lib() -> ctypes.CDLL:
             "qs_select_top_p": ([cfgp, cachep, vp, ctypes.c_float, i32, vp, vp, vp, vp], i32),
             "qs_decode_top_p": ([cfgp, cachep, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp,
                                  vp, vp, vp], i32),
+            "qs_semantic_index_workspace_size": ([cfgp, i32, i32, ctypes.POINTER(sz)], i32),
+            "qs_semantic_index": ([cfgp, cachep, vp, i32, vp, vp, vp, i32, vp, vp], i32),
+            "qs_semantic_select": ([cfgp, cachep, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp],
+                                   i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -92,7 +97,8 @@ EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_
            "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches",
            "qs_selftest_wait_timeout", "qs_dense_workspace_size", "qs_dense_attn",
            "qs_gather_kv", "qs_calib_workspace_size", "qs_calibrate_basis", "qs_rabitq_score",
-           "qs_select_top_p", "qs_decode_top_p")
+           "qs_select_top_p", "qs_decode_top_p", "qs_semantic_index_workspace_size",
+           "qs_semantic_index", "qs_semantic_select")
 
 
 def status_string(s: int) -> str:
@@ -285,6 +291,35 @@ def qs_decode_top_p(cfg, cache, q, k_new, v_new, R, u, p, batch, out, sel_out, n
                                  _ptr(v_new), _ptr(R), _ptr(u), float(p), batch, _ptr(out),
                                  _ptr(sel_out), _ptr(n_sel_out), _ptr(ws), _stream(stream)),
            "qs_decode_top_p")
+
+
+def qs_semantic_index_workspace_size(cfg: qs_config, batch: int, max_context: int) -> int:
+    """Workspace bytes qs_semantic_index needs."""
+    n = ctypes.c_size_t(0)
+    _check(lib().qs_semantic_index_workspace_size(ctypes.byref(cfg), batch, max_context,
+                                                  ctypes.byref(n)),
+           "qs_semantic_index_workspace_size")
+    return n.value
+
+
+def qs_semantic_index(cfg, cache, prompt_lens, iters, centroids, offsets, members, batch, ws,
+                      stream=None):
+    """Build the semantic-block index over each sequence's first prompt_lens[b] keys:
+    centroids [rows][C_max][d] FP32, offsets [rows][C_max + 1], members [rows][max_context]."""
+    _check(lib().qs_semantic_index(ctypes.byref(cfg), ctypes.byref(cache), _ptr(prompt_lens),
+                                   iters, _ptr(centroids), _ptr(offsets), _ptr(members), batch,
+                                   _ptr(ws), _stream(stream)), "qs_semantic_index")
+
+
+def qs_semantic_select(cfg, cache, q, prompt_lens, centroids, offsets, members, batch, tokens,
+                       n_tokens, max_tokens, ws, stream=None):
+    """Score the clusters, select cfg.budget of them and expand them (plus the tokens after
+    the prompt) into tokens [rows][max_tokens] / n_tokens [rows] for the token-level
+    attention."""
+    _check(lib().qs_semantic_select(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q),
+                                    _ptr(prompt_lens), _ptr(centroids), _ptr(offsets),
+                                    _ptr(members), batch, _ptr(tokens), _ptr(n_tokens),
+                                    max_tokens, _ptr(ws), _stream(stream)), "qs_semantic_select")
 
 
 def qs_device_status(ws, stream=None) -> tuple[int, int, int]:

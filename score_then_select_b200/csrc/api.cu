@@ -9,6 +9,7 @@
 
 #include "qs_internal.h"
 #include "rabitq.h"
+#include "semantic.h"
 
 namespace qs {
 
@@ -112,9 +113,11 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   const int r = c->proxy_rank;
   if (r < 0) return QS_ERR_INVALID_ARG;
   p.kind = r > 0 ? PK_RANKR
-                 : (c->proxy_dtype == QS_CENTROID ? PK_CENTROID
-                                                  : (c->proxy_dtype == QS_RABITQ ? PK_RABITQ : PK_NVFP4));
-  if (p.kind == PK_CENTROID || p.kind == PK_RABITQ) {
+         : c->proxy_dtype == QS_CENTROID ? PK_CENTROID
+         : c->proxy_dtype == QS_RABITQ   ? PK_RABITQ
+         : c->proxy_dtype == QS_SEMANTIC ? PK_SEMANTIC
+                                         : PK_NVFP4;
+  if (p.kind == PK_CENTROID || p.kind == PK_RABITQ || p.kind == PK_SEMANTIC) {
     if (c->n_keep_hp != 0) return QS_ERR_INVALID_ARG;
   } else if (r > 0) {
     const bool ok = (c->proxy_dtype == QS_F32 && (r == 16 || (r == 32 && c->head_dim == 128))) ||
@@ -209,7 +212,7 @@ qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy) {
   if (c->max_pages_per_seq < 1 || c->num_pages < 1 || c->max_context < 1) return QS_ERR_INVALID_ARG;
   if ((long long)c->num_pages * p.Hkv * kPage >= (1LL << 31)) return QS_ERR_UNSUPPORTED;
   if (!aligned(c->k, 16) || !aligned(c->v, 16)) return QS_ERR_INVALID_ARG;
-  if (need_proxy) {
+  if (need_proxy && p.kind != PK_SEMANTIC) {      // the semantic index lives outside the cache
     if (!c->proxy || !aligned(c->proxy, 16)) return QS_ERR_INVALID_ARG;
     if (p.kind == PK_NVFP4 && (!c->proxy_scale || !c->key_center || !c->key_gscale))
       return QS_ERR_INVALID_ARG;
@@ -441,6 +444,7 @@ qs_status qs_score(const qs_config* cfg, const qs_cache* cache, const void* q, c
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
   if (p.r == 0 && !aligned(q, 16)) return QS_ERR_INVALID_ARG;
   if (p.kind == PK_RABITQ) return QS_ERR_UNSUPPORTED;     // qs_rabitq_score takes its draws
+  if (p.kind == PK_SEMANTIC) return QS_ERR_UNSUPPORTED;   // qs_semantic_select scores clusters
   if (p.kind == PK_CENTROID) return do_score(p, cache, q, block_scores, ws, stream, false);
   // the prep kernel runs in stream order and writes only the query side, so the scan
   // overlaps it and starts streaming pages before it waits for the query
@@ -562,7 +566,7 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
   if (st != QS_OK) return st;
   if ((st = check_cache(p, cache, true)) != QS_OK) return st;
-  if (p.kind == PK_RABITQ) return QS_ERR_UNSUPPORTED;     // its stages are separate calls
+  if (p.kind == PK_RABITQ || p.kind == PK_SEMANTIC) return QS_ERR_UNSUPPORTED;  // own calls
   if (!q || !aligned(q, 16) || !k_new || !v_new || !out || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return QS_ERR_INVALID_ARG;
   if (p.r > 0 && (!P || !aligned(P, 16))) return QS_ERR_INVALID_ARG;
@@ -686,6 +690,119 @@ qs_status qs_decode_top_p(const qs_config* cfg, const qs_cache* cache, const voi
   if ((st = do_rq_score(p, cache, q, R, u, scores, ws, stream)) != QS_OK) return st;
   if ((st = do_top_p(p, cache, scores, p_mass, sel, nsel, ws, stream)) != QS_OK) return st;
   return do_attend(p, cache, q, sel, nsel, out, ws, stream, false);
+}
+
+// ---- semantic blocks ("Coarse Semantic Blocks ...", Abstract)
+static int sem_c_max(const Plan& p, int max_context) { return (max_context + p.S - 1) / p.S; }
+
+static size_t sem_index_ws_bytes(const Plan& p, int max_context) {
+  const size_t rows = size_t(p.batch) * p.Hkv;
+  return size_t(kHdrWords) * 4 + rows * size_t(max_context) * 4 +
+         rows * size_t(sem_c_max(p, max_context)) * 4;
+}
+
+qs_status qs_semantic_index_workspace_size(const qs_config* cfg, int32_t batch,
+                                           int32_t max_context, size_t* bytes) {
+  if (!bytes) return QS_ERR_INVALID_ARG;
+  Plan p;
+  const qs_status st = make_plan(cfg, batch, max_context, p);
+  if (st != QS_OK) return st;
+  if (p.kind != PK_SEMANTIC) return QS_ERR_UNSUPPORTED;
+  *bytes = sem_index_ws_bytes(p, max_context);
+  return QS_OK;
+}
+
+qs_status qs_semantic_index(const qs_config* cfg, const qs_cache* cache,
+                            const int32_t* prompt_lens, int32_t iters, float* centroids,
+                            int32_t* offsets, int32_t* members, int32_t batch, void* ws,
+                            qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (p.kind != PK_SEMANTIC) return QS_ERR_UNSUPPORTED;
+  if ((st = check_cache(p, cache, false)) != QS_OK) return st;
+  if (!prompt_lens || !centroids || !offsets || !members || !ws || !aligned(ws, 256) ||
+      iters < 1)
+    return QS_ERR_INVALID_ARG;
+  const int l_max = cache->max_context, c_max = sem_c_max(p, l_max);
+  const size_t rows = size_t(p.batch) * p.Hkv;
+  SemIndexParams a{};
+  a.k = static_cast<const uint16_t*>(cache->k);
+  a.page_table = cache->page_table;
+  a.prompt_lens = prompt_lens;
+  a.cent = centroids;
+  a.offsets = offsets;
+  a.members = members;
+  a.assign = ws_at<int32_t>(ws, size_t(kHdrWords) * 4);
+  a.cursor = a.assign + rows * l_max;
+  a.hdr = hdr_of(ws);
+  a.batch = p.batch;
+  a.Hkv = p.Hkv;
+  a.d = p.d;
+  a.S = p.S;
+  a.c_max = c_max;
+  a.l_max = l_max;
+  a.max_pages_per_seq = cache->max_pages_per_seq;
+  a.num_pages = cache->num_pages;
+  return cuda_status(launch_sem_index(a, iters, stream));
+}
+
+qs_status qs_semantic_select(const qs_config* cfg, const qs_cache* cache, const void* q,
+                             const int32_t* prompt_lens, const float* centroids,
+                             const int32_t* offsets, const int32_t* members, int32_t batch,
+                             int32_t* tokens, int32_t* n_tokens, int32_t max_tokens, void* ws,
+                             qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (p.kind != PK_SEMANTIC) return QS_ERR_UNSUPPORTED;
+  if (!cache || !cache->seq_lens) return QS_ERR_INVALID_ARG;
+  if (!q || !aligned(q, 4) || !prompt_lens || !centroids || !offsets || !members || !tokens ||
+      !n_tokens || max_tokens < 1 || !ws || !aligned(ws, 256))
+    return QS_ERR_INVALID_ARG;
+  const int l_max = cache->max_context, c_max = sem_c_max(p, l_max);
+  SemSelectParams a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.prompt_lens = prompt_lens;
+  a.seq_lens = cache->seq_lens;
+  a.cent = centroids;
+  a.offsets = offsets;
+  a.members = members;
+  a.scores = ws_at<float>(ws, p.ws.scores);          // rows x nb_stride >= rows x c_max
+  a.n_clusters = ws_at<int32_t>(ws, p.ws.qt);        // batch <= rows entries
+  a.csel = ws_at<int32_t>(ws, p.ws.sel);
+  a.n_csel = ws_at<int32_t>(ws, p.ws.nsel);
+  a.tokens = tokens;
+  a.n_tokens = n_tokens;
+  a.hdr = hdr_of(ws);
+  a.batch = p.batch;
+  a.Hkv = p.Hkv;
+  a.G = p.G;
+  a.d = p.d;
+  a.S = p.S;
+  a.c_max = c_max;
+  a.l_max = l_max;
+  a.budget = p.budget;
+  a.max_tokens = max_tokens;
+  if ((st = cuda_status(launch_sem_score(a, stream))) != QS_OK) return st;
+  // the top clusters: the select kernel over C_b candidates per row (block size 1)
+  SelectParams sp{};
+  sp.scores = a.scores;
+  sp.block_err = nullptr;
+  sp.seq_lens = a.n_clusters;
+  sp.sel = ws_at<int32_t>(ws, p.ws.sel);
+  sp.n_sel = ws_at<int32_t>(ws, p.ws.nsel);
+  sp.hdr = a.hdr;
+  sp.rows = p.batch * p.Hkv;
+  sp.Hkv = p.Hkv;
+  sp.S = 1;
+  sp.nb_stride = c_max;
+  sp.budget = p.budget;
+  sp.force_sink = 0;
+  sp.force_last = 0;
+  sp.n_keep = 0;
+  if ((st = cuda_status(launch_select(p, sp, stream, false))) != QS_OK) return st;
+  return cuda_status(launch_sem_expand(a, stream));
 }
 
 qs_status qs_device_status(void* ws, qs_stream_t stream, uint32_t* detail) {

@@ -21,6 +21,7 @@
 // decides the blocks kept at full precision.
 #include "qs_device.cuh"
 #include "rabitq.h"
+#include "semantic.h"
 
 namespace qs {
 
@@ -571,6 +572,48 @@ __global__ void __launch_bounds__(D) append_rabitq_kernel(const AppendParams a) 
   finish_append(a);
 }
 
+// ============================================================ K/V only
+// The semantic-block index covers the prompt; tokens decoded after it have no scoring
+// entry (they are always attended), so their append copies K and V only.
+// CTA = one row x 64 tokens.
+__global__ void __launch_bounds__(128) append_kv_kernel(const AppendParams a) {
+  constexpr int TT = 64;
+  __shared__ int s_page[TT], s_slot[TT];
+  const int row = blockIdx.y;
+  const int b = row / a.Hkv, g = row % a.Hkv;
+  int n_b = a.n_new ? a.n_new[b] : 1;
+  if (n_b < 0 || n_b > a.max_new) {
+    if (threadIdx.x == 0 && blockIdx.x == 0)
+      flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_APPEND, uint32_t(b));
+    n_b = 0;
+  }
+  const int old = a.seq_lens[b];
+  const int t0 = blockIdx.x * TT;
+  const int cnt = min(TT, n_b - t0);
+  if (cnt > 0) {
+    if (threadIdx.x < TT) {
+      int page = -1, slot = 0;
+      if (int(threadIdx.x) < cnt)
+        cache_slot(a.page_table, b, old + t0 + threadIdx.x, a.max_pages_per_seq, a.num_pages,
+                   a.max_context, a.hdr, KID_APPEND, page, slot);
+      s_page[threadIdx.x] = page;
+      s_slot[threadIdx.x] = slot;
+    }
+    __syncthreads();
+    const int CH = a.d / 8;
+    for (int it = threadIdx.x; it < cnt * CH; it += blockDim.x) {
+      const int n = it / CH, c = it % CH;
+      const int page = s_page[n];
+      if (page < 0) continue;
+      const size_t src = ((size_t(row) * a.max_new) + t0 + n) * a.d + c * 8;
+      const size_t dst = ((size_t(page) * a.Hkv + g) * kPage + s_slot[n]) * a.d + c * 8;
+      *reinterpret_cast<uint4*>(a.k + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+      *reinterpret_cast<uint4*>(a.v + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+    }
+  }
+  finish_append(a);
+}
+
 // ============================================================ NVFP4 block error
 // CTA = one (row, block) pair that this append may have completed; 256 threads, each
 // owning (token, 16-element group) items i = tid + 256 m. An item's error is summed over
@@ -747,6 +790,10 @@ static cudaError_t launch_rankr(const Plan& p, const AppendParams& a, cudaStream
 }
 
 cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) {
+  if (p.kind == PK_SEMANTIC) {
+    append_kv_kernel<<<dim3((a.max_new + 63) / 64, a.batch * a.Hkv), 128, 0, s>>>(a);
+    return cudaGetLastError();
+  }
   if (p.kind == PK_RABITQ) {
     const dim3 grid((a.max_new + 15) / 16, a.batch * a.Hkv);
     if (p.d == 128) append_rabitq_kernel<128><<<grid, 128, 0, s>>>(a);

@@ -1,0 +1,325 @@
+// semantic.cu - the semantic-block index (float32 k-means over the prompt's keys) and its
+// decode side ("Coarse Semantic Blocks for Efficient Training-Free Sparse Attention",
+// Abstract; the readings are in semantic.h).
+//
+// Index build, per row (sequence b, KV head g), L0 = the prompt length, C = ceil(L0 / S):
+//   sem_seed_kernel:   c_j = key at floor(j * L0 / C).
+//   then `iters` times:
+//   sem_assign_kernel: CTA = (row, page of 128 keys), thread = key; the page's keys sit
+//                      transposed in shared memory (conflict-free per-thread columns), the
+//                      centroids stream through in chunks of 32; distances summed over the
+//                      dimensions in order with one rounding per operation.
+//   sem_csr_kernel:    CTA = row: member counts, offsets (exclusive scan), then a stable
+//                      fill: 1,024 keys at a time, warps in order, each warp's equal-cluster
+//                      lanes found with match.any, so members stay in token order.
+//   sem_update_kernel: thread = (cluster, dimension): the members' sum in token order, then
+//                      one division by the count (an empty cluster keeps its centroid).
+// Decode:
+//   sem_score_kernel:  warp = (row, cluster): beta_j = qbar . c_j (float32).
+//   (the existing select kernel picks the top clusters over C_b candidates)
+//   sem_expand_kernel: CTA = row: the selected clusters' members, then the tokens after the
+//                      prompt, as the row's token list for the token-level attention.
+#include <cfloat>
+
+#include "qs_device.cuh"
+#include "semantic.h"
+
+namespace qs {
+
+constexpr int kSemTile = 128;        // keys per assignment CTA (one page)
+constexpr int kSemChunk = 32;        // centroids per shared-memory chunk
+constexpr int kSemThreads = 1024;    // CSR and expansion CTAs
+
+QS_DEV int sem_clusters(int L0, int S) { return L0 > 0 ? (L0 + S - 1) / S : 0; }
+
+// The prompt length of sequence b, clamped to the index's capacity.
+QS_DEV int sem_prompt(const int32_t* prompt_lens, int b, int l_max) {
+  const int L0 = prompt_lens[b];
+  return L0 < 0 ? 0 : (L0 > l_max ? l_max : L0);
+}
+
+// Pointer to key t of row (b, g) in the paged cache, or nullptr (and an error flag).
+QS_DEV const uint16_t* sem_key(const SemIndexParams& a, int b, int g, int t) {
+  const int pi = t / kPage;
+  int page = -1;
+  if (pi < a.max_pages_per_seq) page = a.page_table[size_t(b) * a.max_pages_per_seq + pi];
+  if (page < 0 || page >= a.num_pages) {
+    flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SEMANTIC, uint32_t(b));
+    return nullptr;
+  }
+  return a.k + ((size_t(page) * a.Hkv + g) * kPage + (t % kPage)) * a.d;
+}
+
+// Exclusive prefix of v over the CTA's threads in order (blockDim = kSemThreads); total
+// receives the sum of all v.
+QS_DEV int sem_scan(int v, int* s, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = s[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, t, o);
+      if (lane >= o) t += y;
+    }
+    s[lane] = t;
+  }
+  __syncthreads();
+  const int before = warp ? s[warp - 1] : 0;
+  total = s[kSemThreads / 32 - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// ============================================================ index build
+__global__ void __launch_bounds__(256) sem_seed_kernel(const SemIndexParams a) {
+  const int row = blockIdx.x, b = row / a.Hkv, g = row % a.Hkv;
+  const int L0 = sem_prompt(a.prompt_lens, b, a.l_max);
+  const int C = min(sem_clusters(L0, a.S), a.c_max);
+  float* cent = a.cent + size_t(row) * a.c_max * a.d;
+  for (int e = threadIdx.x; e < C * a.d; e += blockDim.x) {
+    const int j = e / a.d, i = e % a.d;
+    const int t = int((long long)j * L0 / C);
+    const uint16_t* kp = sem_key(a, b, g, t);
+    cent[size_t(j) * a.d + i] = kp ? bf16_to_f32(kp[i]) : 0.0f;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSemTile) sem_assign_kernel(const SemIndexParams a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float* xs = reinterpret_cast<float*>(smem_raw);                  // [D][kSemTile]
+  float* cs = xs + D * kSemTile;                                    // [kSemChunk][D]
+  const int row = blockIdx.y, b = row / a.Hkv, g = row % a.Hkv, tid = threadIdx.x;
+  const int L0 = sem_prompt(a.prompt_lens, b, a.l_max);
+  const int C = min(sem_clusters(L0, a.S), a.c_max);
+  const int t0 = blockIdx.x * kSemTile;
+  if (t0 >= L0) return;
+  const uint16_t* kp = sem_key(a, b, g, t0);                        // the page's first key
+  if (!kp) return;
+  // the page's keys, transposed: xs[i][t]
+  for (int e = tid; e < kSemTile * D; e += kSemTile) {
+    const int t = e / D, i = e % D;
+    xs[i * kSemTile + t] = t0 + t < L0 ? bf16_to_f32(kp[size_t(t) * D + i]) : 0.0f;
+  }
+  const float* cent = a.cent + size_t(row) * a.c_max * D;
+  float best = INFINITY;
+  int arg = 0;
+  for (int c0 = 0; c0 < C; c0 += kSemChunk) {
+    const int n = min(kSemChunk, C - c0);
+    __syncthreads();
+    for (int e = tid; e < n * D; e += kSemTile) cs[e] = cent[size_t(c0) * D + e];
+    __syncthreads();
+    for (int jj = 0; jj < n; ++jj) {
+      float dist = 0.0f;
+#pragma unroll 8
+      for (int i = 0; i < D; ++i) {
+        const float diff = __fsub_rn(xs[i * kSemTile + tid], cs[jj * D + i]);
+        dist = __fadd_rn(dist, __fmul_rn(diff, diff));
+      }
+      if (dist < best) {
+        best = dist;
+        arg = c0 + jj;
+      }
+    }
+  }
+  if (t0 + tid < L0) a.assign[size_t(row) * a.l_max + t0 + tid] = arg;
+}
+
+__global__ void __launch_bounds__(kSemThreads) sem_csr_kernel(const SemIndexParams a) {
+  __shared__ int s_scan[kSemThreads / 32];
+  const int row = blockIdx.x, b = row / a.Hkv, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int L0 = sem_prompt(a.prompt_lens, b, a.l_max);
+  const int C = min(sem_clusters(L0, a.S), a.c_max);
+  const int32_t* asg = a.assign + size_t(row) * a.l_max;
+  int32_t* cur = a.cursor + size_t(row) * a.c_max;
+  int32_t* off = a.offsets + size_t(row) * (a.c_max + 1);
+  int32_t* mem = a.members + size_t(row) * a.l_max;
+  // member counts
+  for (int j = tid; j < C; j += kSemThreads) cur[j] = 0;
+  __syncthreads();
+  for (int t = tid; t < L0; t += kSemThreads) {
+    const int j = asg[t];
+    if (j >= 0 && j < C) atomicAdd(&cur[j], 1);
+    else flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SEMANTIC, uint32_t(row));
+  }
+  __syncthreads();
+  // offsets: exclusive prefix of the counts
+  int running = 0;
+  for (int base = 0; base < C; base += kSemThreads) {
+    const int j = base + tid;
+    const int v = j < C ? cur[j] : 0;
+    int total;
+    const int ex = sem_scan(v, s_scan, total);
+    if (j < C) off[j] = running + ex;
+    running += total;
+  }
+  if (tid == 0) off[C] = running;
+  __syncthreads();
+  for (int j = tid; j < C; j += kSemThreads) cur[j] = 0;
+  // stable fill: keys in order, 1,024 at a time; warps take turns
+  for (int base = 0; base < L0; base += kSemThreads) {
+    const int t = base + tid;
+    int j = t < L0 ? asg[t] : -1;
+    if (j >= C) j = -1;
+    const unsigned grp = __match_any_sync(kFull, j);
+    const int rank = __popc(grp & ((1u << lane) - 1u));
+    const int leader = __ffs(grp) - 1;
+    for (int w = 0; w < kSemThreads / 32; ++w) {
+      __syncthreads();
+      if (warp == w) {                     // the whole warp: each lane reads its group leader
+        int pos = 0;
+        if (j >= 0 && lane == leader) {
+          pos = cur[j];
+          cur[j] = pos + __popc(grp);
+        }
+        pos = __shfl_sync(kFull, pos, leader);
+        if (j >= 0) mem[off[j] + pos + rank] = t;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(256) sem_update_kernel(const SemIndexParams a) {
+  const int row = blockIdx.y, b = row / a.Hkv, g = row % a.Hkv;
+  const int L0 = sem_prompt(a.prompt_lens, b, a.l_max);
+  const int C = min(sem_clusters(L0, a.S), a.c_max);
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j = e / a.d, i = e % a.d;
+  if (j >= C) return;
+  const int32_t* off = a.offsets + size_t(row) * (a.c_max + 1);
+  const int32_t* mem = a.members + size_t(row) * a.l_max;
+  const int lo = off[j], hi = off[j + 1];
+  if (hi <= lo) return;                                  // empty: the centroid stays
+  float s = 0.0f;
+  for (int m = lo; m < hi; ++m) {
+    const uint16_t* kp = sem_key(a, b, g, mem[m]);
+    s = __fadd_rn(s, kp ? bf16_to_f32(kp[i]) : 0.0f);
+  }
+  a.cent[(size_t(row) * a.c_max + j) * a.d + i] = __fdiv_rn(s, float(hi - lo));
+}
+
+cudaError_t launch_sem_index(const SemIndexParams& a, int iters, cudaStream_t s) {
+  const int rows = a.batch * a.Hkv;
+  sem_seed_kernel<<<rows, 256, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t(a.d) * kSemTile + size_t(kSemChunk) * a.d) * sizeof(float);
+  auto assign = a.d == 128 ? sem_assign_kernel<128> : sem_assign_kernel<64>;
+  if ((e = set_smem_limit(assign, int(smem))) != cudaSuccess) return e;
+  const dim3 agrid((a.l_max + kSemTile - 1) / kSemTile, rows);
+  const dim3 ugrid((a.c_max * a.d + 255) / 256, rows);
+  for (int it = 0; it < (iters < 1 ? 1 : iters); ++it) {
+    assign<<<agrid, kSemTile, smem, s>>>(a);
+    sem_csr_kernel<<<rows, kSemThreads, 0, s>>>(a);
+    sem_update_kernel<<<ugrid, 256, 0, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// ============================================================ decode
+constexpr int kSemScoreWarps = 8;
+
+// warp = (row, cluster j): beta_j = qbar . c_j (float32); -inf past the row's clusters.
+// Also writes each sequence's cluster count, which the select kernel takes as its number
+// of candidates.
+template <int D>
+__global__ void __launch_bounds__(kSemScoreWarps * 32) sem_score_kernel(const SemSelectParams a) {
+  constexpr int PER = D / 32;
+  const int row = blockIdx.y, b = row / a.Hkv, g = row % a.Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int L0 = sem_prompt(a.prompt_lens, b, a.l_max);
+  const int C = min(sem_clusters(L0, a.S), a.c_max);
+  if (blockIdx.x == 0 && g == 0 && threadIdx.x == 0) a.n_clusters[b] = C;
+  const int j = blockIdx.x * kSemScoreWarps + warp;
+  if (j >= a.c_max) return;
+  float* out = a.scores + size_t(row) * a.c_max;
+  if (j >= C) {
+    if (lane == 0) out[j] = -INFINITY;
+    return;
+  }
+  const int Hq = a.Hkv * a.G;
+  const float* c = a.cent + (size_t(row) * a.c_max + j) * D;
+  float dot = 0.0f;
+#pragma unroll
+  for (int m = 0; m < PER; ++m) {
+    const int i = lane + 32 * m;
+    float s = 0.0f;
+    for (int h = 0; h < a.G; ++h)
+      s += bf16_to_f32(a.q[(size_t(b) * Hq + size_t(g) * a.G + h) * D + i]);
+    dot = fmaf(c[i], s / float(a.G), dot);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(kFull, dot, o);
+  if (lane == 0) out[j] = dot;
+}
+
+// CTA = row: the members of the selected clusters (each cluster's in token order, the
+// clusters in the order selected), then the tokens after the prompt, L0 <= t < seq_len.
+__global__ void __launch_bounds__(kSemThreads) sem_expand_kernel(const SemSelectParams a) {
+  __shared__ int s_scan[kSemThreads / 32];
+  const int row = blockIdx.x, b = row / a.Hkv, tid = threadIdx.x;
+  const int L0 = sem_prompt(a.prompt_lens, b, a.l_max);
+  const int C = min(sem_clusters(L0, a.S), a.c_max);
+  int L = a.seq_lens[b];
+  if (L < L0) L = L0;
+  const int32_t* off = a.offsets + size_t(row) * (a.c_max + 1);
+  const int32_t* mem = a.members + size_t(row) * a.l_max;
+  const int32_t* cs = a.csel + size_t(row) * a.budget;
+  int32_t* out = a.tokens + size_t(row) * a.max_tokens;
+  int ncs = a.n_csel[row];
+  if (ncs < 0 || ncs > a.budget) {
+    if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SEMANTIC, uint32_t(row));
+    ncs = 0;
+  }
+  int running = 0;
+  bool over = false;
+  for (int base = 0; base < ncs; base += kSemThreads) {
+    const int i = base + tid;
+    const int c = i < ncs ? cs[i] : -1;
+    const bool ok = c >= 0 && c < C;
+    if (i < ncs && !ok) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SEMANTIC, uint32_t(row));
+    const int lo = ok ? off[c] : 0, sz = ok ? off[c + 1] - lo : 0;
+    int total;
+    const int dst = running + sem_scan(sz, s_scan, total);
+    for (int m = 0; m < sz; ++m) {
+      if (dst + m < a.max_tokens) out[dst + m] = mem[lo + m];
+      else over = true;
+    }
+    running += total;
+  }
+  for (int t = L0 + tid; t < L; t += kSemThreads) {
+    const int pos = running + (t - L0);
+    if (pos < a.max_tokens) out[pos] = t;
+    else over = true;
+  }
+  if (over) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SEMANTIC, uint32_t(row));
+  int n = running + (L - L0);
+  if (n > a.max_tokens) n = a.max_tokens;
+  if (tid == 0) a.n_tokens[row] = n;
+  for (int i = n + tid; i < a.max_tokens; i += kSemThreads) out[i] = -1;
+}
+
+cudaError_t launch_sem_score(const SemSelectParams& a, cudaStream_t s) {
+  const dim3 grid((a.c_max + kSemScoreWarps - 1) / kSemScoreWarps, a.batch * a.Hkv);
+  if (a.d == 128) sem_score_kernel<128><<<grid, kSemScoreWarps * 32, 0, s>>>(a);
+  else sem_score_kernel<64><<<grid, kSemScoreWarps * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sem_expand(const SemSelectParams& a, cudaStream_t s) {
+  sem_expand_kernel<<<a.batch * a.Hkv, kSemThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace qs

@@ -40,7 +40,10 @@ class Layer:
         k = torch.zeros((num_pages, Hkv, ps, d), dtype=torch.bfloat16, device=device)
         v = torch.zeros((num_pages, Hkv, ps, d), dtype=vdt, device=device)
         extra = {}
-        if cfg.proxy_dtype == B.QS_RABITQ:
+        if cfg.proxy_dtype == B.QS_SEMANTIC:
+            # the semantic-block index lives outside the cache (qs_semantic_index)
+            proxy = torch.zeros((16,), dtype=torch.uint8, device=device)
+        elif cfg.proxy_dtype == B.QS_RABITQ:
             # per (page, KV head): page_size x d/8 bytes of code bits, then page_size FP32
             # factors; the row centres c
             proxy = torch.zeros((num_pages, Hkv, ps * (d // 8) + ps * 4), dtype=torch.uint8,

@@ -232,3 +232,37 @@ def test_binary_proxy_configuration_and_calls_validate_on_the_host():
     with pytest.raises(qs.QsError) as e:                      # sel_out without n_sel_out
         qs.qs_decode_top_p(cfg, cache, a, a, a, a, a, 0.9, 4, a, a, None, a, stream=0)
     assert e.value.status == B.QS_ERR_INVALID_ARG
+
+
+def test_semantic_configuration_and_calls_validate_on_the_host():
+    sem = dict(proxy_rank=0, proxy_dtype="semantic", block_size=64, budget=16,
+               force_sink=False, force_last=False)
+    cfg = _cfg(**sem)
+    assert qs.qs_workspace_size(cfg, 4, 8192) > 0
+    rows, c_max = 4 * 8, 8192 // 64
+    assert qs.qs_semantic_index_workspace_size(cfg, 4, 8192) == 256 + 4 * rows * (8192 + c_max)
+    with pytest.raises(qs.QsError) as e:                      # only the semantic kind
+        qs.qs_semantic_index_workspace_size(_cfg(), 4, 8192)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    with pytest.raises(qs.QsError) as e:                      # kept blocks are NVFP4-only
+        qs.qs_workspace_size(_cfg(n_keep_hp=1, **sem), 4, 8192)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    cache, a = _fake_cache(with_center=False), 1 << 20
+    cache.proxy = None                                        # the index is outside the cache
+    for call in (lambda: qs.qs_score(cfg, cache, a, a, 4, a, a, stream=0),
+                 lambda: qs.qs_decode(cfg, cache, a, a, a, a, 4, a, None, None, a, stream=0),
+                 lambda: qs.qs_semantic_index(_cfg(), cache, a, 2, a, a, a, 4, a, stream=0),
+                 lambda: qs.qs_semantic_select(_cfg(), cache, a, a, a, a, a, 4, a, a, 64, a,
+                                               stream=0)):
+        with pytest.raises(qs.QsError) as e:
+            call()
+        assert e.value.status == B.QS_ERR_UNSUPPORTED
+    for call in (lambda: qs.qs_semantic_index(cfg, cache, a, 0, a, a, a, 4, a, stream=0),
+                 lambda: qs.qs_semantic_index(cfg, cache, None, 2, a, a, a, 4, a, stream=0),
+                 lambda: qs.qs_semantic_select(cfg, cache, a, a, a, a, a, 4, a, a, 0, a,
+                                               stream=0),
+                 lambda: qs.qs_semantic_select(cfg, cache, a, a, None, a, a, 4, a, a, 64, a,
+                                               stream=0)):
+        with pytest.raises(qs.QsError) as e:
+            call()
+        assert e.value.status == B.QS_ERR_INVALID_ARG
