@@ -388,6 +388,20 @@ qs_status qs_gather_kv(const qs_config *cfg, const qs_cache *cache, const int32_
                        const int32_t *n_sel, int32_t batch, void *k_dst, void *v_dst,
                        int32_t *row_lens, void *ws, qs_stream_t stream);
 
+/* The gather of the NVFP4 storage variant ("Jet-QSparse ...", Full text: the persistent
+   cache keeps the keys in NVFP4 and at most two blocks per sequence at BF16). As
+   qs_gather_kv (same arguments, layout and row_lens; one launch), except for the keys of
+   blocks that are not kept: a kept block is one of the n_keep_hp complete blocks with the
+   largest block_err, ties to the lower index; its keys are copied from the BF16 K pages.
+   Every other selected token's key is read from the NVFP4 scoring cache and written as
+     bf16_rne(fp32(fp32(e * sigma * g_k) + key_center[b][g][i]))   per element i
+   (e * sigma is exact in float32). qs_dense_attn over the compact buffer then attends the
+   way the storage variant does. cfg must be the NVFP4 configuration (else
+   QS_ERR_UNSUPPORTED); block_err is needed when n_keep_hp > 0. */
+qs_status qs_gather_kv_nvfp4k(const qs_config *cfg, const qs_cache *cache, const int32_t *sel,
+                              const int32_t *n_sel, int32_t batch, void *k_dst, void *v_dst,
+                              int32_t *row_lens, void *ws, qs_stream_t stream);
+
 /* ---- Calibration of the scoring basis (once, before decoding) ----------------------------
    "Joint Subspace Sparse Attention for Efficient Long-Context Decoding", Abstract and
    Table 9: the shared subspace minimises a tractable bound on the token-score preservation

@@ -280,6 +280,26 @@ def nvfp4_attended_keys(k_bits: np.ndarray, codes: np.ndarray, scales: np.ndarra
     return K
 
 
+def nvfp4_attended_keys_bf16(k_bits: np.ndarray, codes: np.ndarray, scales: np.ndarray, g_k,
+                             mu: np.ndarray, keep, S: int, L: int) -> np.ndarray:
+    """The same keys as BF16 bit patterns [L][d], as an attention with BF16 operands takes
+    them: kept blocks keep their stored BF16 keys; elsewhere, per element,
+    bf16_rne(fp32(fp32(fp32(e * sigma) * g_k) + mu)) (e * sigma is exact in float32; the
+    product with g_k and the sum with mu are each rounded to float32)."""
+    n, d = codes[:L].shape
+    e = F.e2m1_value(codes[:L]).astype(np.float32)
+    sig = F.ue4m3_value(scales[:L]).astype(np.float32).repeat(16, axis=1)
+    v = (e * sig).astype(np.float32)                                        # exact
+    v = (v * np.float32(g_k)).astype(np.float32)
+    v = (v + np.asarray(mu, dtype=np.float32)[None, :]).astype(np.float32)
+    out = F.f32_to_bf16_rne(v)
+    bits = np.asarray(k_bits[:L], dtype=np.uint16)
+    for j in keep:
+        t0, t1 = int(j) * S, min(L, (int(j) + 1) * S)
+        out[t0:t1] = bits[t0:t1]
+    return out
+
+
 # ============================================================================================
 # Centroid scoring of contiguous blocks  ["Coarse Semantic Blocks ...", Abstract]
 # The page scores each block by its centroid against the query. Reading: the centroid of a

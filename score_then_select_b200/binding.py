@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "qs_select_top_p": ([cfgp, cachep, vp, ctypes.c_float, i32, vp, vp, vp, vp], i32),
             "qs_decode_top_p": ([cfgp, cachep, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp,
                                  vp, vp, vp], i32),
+            "qs_gather_kv_nvfp4k": ([cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp], i32),
             "qs_semantic_index_workspace_size": ([cfgp, i32, i32, ctypes.POINTER(sz)], i32),
             "qs_semantic_index": ([cfgp, cachep, vp, i32, vp, vp, vp, i32, vp, vp], i32),
             "qs_semantic_select": ([cfgp, cachep, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp],
@@ -97,7 +98,8 @@ EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_
            "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches",
            "qs_selftest_wait_timeout", "qs_dense_workspace_size", "qs_dense_attn",
            "qs_gather_kv", "qs_calib_workspace_size", "qs_calibrate_basis", "qs_rabitq_score",
-           "qs_select_top_p", "qs_decode_top_p", "qs_semantic_index_workspace_size",
+           "qs_select_top_p", "qs_decode_top_p", "qs_gather_kv_nvfp4k",
+           "qs_semantic_index_workspace_size",
            "qs_semantic_index", "qs_semantic_select")
 
 
@@ -248,6 +250,15 @@ def qs_gather_kv(cfg, cache, sel, n_sel, batch, k_dst, v_dst, row_lens, ws, stre
     _check(lib().qs_gather_kv(ctypes.byref(cfg), ctypes.byref(cache), _ptr(sel), _ptr(n_sel),
                               batch, _ptr(k_dst), _ptr(v_dst), _ptr(row_lens), _ptr(ws),
                               _stream(stream)), "qs_gather_kv")
+
+
+def qs_gather_kv_nvfp4k(cfg, cache, sel, n_sel, batch, k_dst, v_dst, row_lens, ws, stream=None):
+    """qs_gather_kv for the NVFP4 storage variant: kept blocks' keys from BF16, every
+    other selected key dequantised from NVFP4, un-centred and rounded to BF16."""
+    _check(lib().qs_gather_kv_nvfp4k(ctypes.byref(cfg), ctypes.byref(cache), _ptr(sel),
+                                     _ptr(n_sel), batch, _ptr(k_dst), _ptr(v_dst),
+                                     _ptr(row_lens), _ptr(ws), _stream(stream)),
+           "qs_gather_kv_nvfp4k")
 
 
 def qs_calib_workspace_size(cfg: qs_config) -> int:

@@ -10,6 +10,7 @@
 #include "qs_internal.h"
 #include "rabitq.h"
 #include "semantic.h"
+#include "nvfp4k.h"
 
 namespace qs {
 
@@ -690,6 +691,47 @@ qs_status qs_decode_top_p(const qs_config* cfg, const qs_cache* cache, const voi
   if ((st = do_rq_score(p, cache, q, R, u, scores, ws, stream)) != QS_OK) return st;
   if ((st = do_top_p(p, cache, scores, p_mass, sel, nsel, ws, stream)) != QS_OK) return st;
   return do_attend(p, cache, q, sel, nsel, out, ws, stream, false);
+}
+
+// ---- the NVFP4 storage variant's attended keys ("Jet-QSparse ...", Full text)
+qs_status qs_gather_kv_nvfp4k(const qs_config* cfg, const qs_cache* cache, const int32_t* sel,
+                              const int32_t* n_sel, int32_t batch, void* k_dst, void* v_dst,
+                              int32_t* row_lens, void* ws, qs_stream_t stream) {
+  Plan p;
+  qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (p.kind != PK_NVFP4) return QS_ERR_UNSUPPORTED;
+  if ((st = check_cache(p, cache, true)) != QS_OK) return st;
+  if (!sel || !n_sel || !k_dst || !v_dst || !row_lens || !ws || !aligned(ws, 256))
+    return QS_ERR_INVALID_ARG;
+  if (!aligned(k_dst, 16) || !aligned(v_dst, 16)) return QS_ERR_INVALID_ARG;
+  if (p.n_keep > 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
+  GatherNvParams a{};
+  a.base.k = static_cast<const uint16_t*>(cache->k);
+  a.base.v = static_cast<const uint16_t*>(cache->v);
+  a.base.sel = sel;
+  a.base.n_sel = n_sel;
+  a.base.page_table = cache->page_table;
+  a.base.seq_lens = cache->seq_lens;
+  a.base.k_dst = static_cast<uint16_t*>(k_dst);
+  a.base.v_dst = static_cast<uint16_t*>(v_dst);
+  a.base.row_lens = row_lens;
+  a.base.hdr = hdr_of(ws);
+  a.base.rows = p.batch * p.Hkv;
+  a.base.Hkv = p.Hkv;
+  a.base.log2_S = 7;                                  // the NVFP4 path has S = 128
+  a.base.budget = p.budget;
+  a.base.dst_pages_per_seq = p.budget;                // one 128-token page per block
+  a.base.max_pages_per_seq = cache->max_pages_per_seq;
+  a.base.num_pages = cache->num_pages;
+  a.codes = static_cast<const uint8_t*>(cache->proxy);
+  a.scales = cache->proxy_scale;
+  a.key_center = cache->key_center;
+  a.key_gscale = cache->key_gscale;
+  a.block_err = p.n_keep > 0 ? cache->block_err : nullptr;
+  a.nb_stride = p.nb_stride;
+  a.n_keep = p.n_keep;
+  return cuda_status(launch_gather_kv_nvfp4k(p, a, stream));
 }
 
 // ---- semantic blocks ("Coarse Semantic Blocks ...", Abstract)

@@ -266,3 +266,23 @@ def test_semantic_configuration_and_calls_validate_on_the_host():
         with pytest.raises(qs.QsError) as e:
             call()
         assert e.value.status == B.QS_ERR_INVALID_ARG
+
+
+def test_nvfp4_storage_gather_validates_on_the_host():
+    cache, a = _fake_cache(), 1 << 20
+    with pytest.raises(qs.QsError) as e:                      # only the NVFP4 configuration
+        qs.qs_gather_kv_nvfp4k(_cfg(), cache, a, a, 4, a, a, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    nv = _cfg(proxy_rank=0, proxy_dtype="nvfp4", block_size=128, n_keep_hp=2)
+    with pytest.raises(qs.QsError) as e:                      # no scales / tensor scale
+        qs.qs_gather_kv_nvfp4k(nv, cache, a, a, 4, a, a, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    cache.proxy_scale = a
+    cache.key_gscale = a
+    with pytest.raises(qs.QsError) as e:                      # kept blocks need block_err
+        qs.qs_gather_kv_nvfp4k(nv, cache, a, a, 4, a, a, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    cache.block_err = a
+    with pytest.raises(qs.QsError) as e:                      # no destination
+        qs.qs_gather_kv_nvfp4k(nv, cache, a, a, 4, None, a, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG

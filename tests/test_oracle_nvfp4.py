@@ -166,3 +166,45 @@ def test_attended_keys_error_within_the_nvfp4_bound():
     sig = F.ue4m3_value(scales).repeat(16, axis=1) * np.float64(g_k)
     err = np.abs(K - F.bf16_to_f64(kb))
     assert np.all(err <= 1.0 * sig + 1e-6 * np.abs(F.bf16_to_f64(kb)) + 1e-7)
+
+
+def test_attended_keys_bf16_round_the_float64_keys():
+    """The BF16 form is the float64 keys rounded to BF16, up to the float32 steps before the
+    rounding: within half a BF16 step (plus the float32 error) everywhere, and the stored
+    bits in kept blocks."""
+    rng = np.random.default_rng(63)
+    S, L = 16, 70
+    kb, mu, x32, g_k, codes, scales = _nvfp4_row(rng, L)
+    K64 = M.nvfp4_attended_keys(kb, codes, scales, g_k, mu, [2], S, L)
+    Kb = M.nvfp4_attended_keys_bf16(kb, codes, scales, g_k, mu, [2], S, L)
+    assert Kb.dtype == np.uint16
+    assert np.array_equal(Kb[32:48], kb[32:48])
+    got = F.bf16_to_f64(Kb)
+    half_ulp = np.abs(K64) * 2.0 ** -8
+    assert np.all(np.abs(got - K64) <= half_ulp + np.abs(K64) * 2.0 ** -22 + 1e-30)
+
+
+def test_attended_keys_bf16_exact_for_representable_values():
+    """Codes of E2M1 values, unit scales, g_k a power of two and a zero centre: every step
+    is exact, so the BF16 keys are the dequantised values themselves."""
+    rng = np.random.default_rng(64)
+    L, d = 20, 128
+    codes = rng.integers(0, 16, size=(L, d)).astype(np.uint8)
+    scales = np.full((L, d // 16), 0x38, dtype=np.uint8)            # UE4M3 1.0
+    g_k = np.float32(0.25)
+    kb = np.zeros((L, d), dtype=np.uint16)
+    Kb = M.nvfp4_attended_keys_bf16(kb, codes, scales, g_k, np.zeros(d, np.float32), [], 16, L)
+    assert np.array_equal(F.bf16_to_f64(Kb), F.e2m1_value(codes) * 0.25)
+
+
+def test_attended_keys_bf16_round_half_to_even():
+    """A dequantised value halfway between two BF16 neighbours rounds to the even one:
+    e * sigma * g = 1 * 1 * (1 + 2^-8) is exactly between 1 and 1 + 2^-7."""
+    L, d = 1, 128
+    codes = np.zeros((L, d), dtype=np.uint8)
+    codes[0, 0] = 2                                                  # E2M1 1.0
+    scales = np.full((L, d // 16), 0x38, dtype=np.uint8)
+    g_k = np.float32(1.0 + 2.0 ** -8)
+    Kb = M.nvfp4_attended_keys_bf16(np.zeros((L, d), np.uint16), codes, scales, g_k,
+                                    np.zeros(d, np.float32), [], 16, L)
+    assert F.bf16_to_f64(Kb)[0, 0] == 1.0
