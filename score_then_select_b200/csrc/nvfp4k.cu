@@ -10,10 +10,12 @@
 // This kernel writes those keys (and the values) of every row's selected blocks into the
 // compact buffer of gather-then-attend (gather.cu), which dense attention then reads. The
 // kept blocks are recomputed per CTA from the per-block errors: the n_keep complete blocks
-// with the largest error, ties to the lower index, as the select kernel takes them.
+// with the largest error (a NaN error ranking as -FLT_MAX), ties to the lower index, as the
+// select kernel takes them.
 //
 // One CTA per (row, 128 slots = one selected block, since the NVFP4 path has S = 128):
 // thread = one 16-byte chunk (8 elements) of a token row.
+#include <cfloat>
 #include <cuda_bf16.h>
 
 #include "qs_device.cuh"
@@ -48,8 +50,9 @@ QS_DEV int nk_argmax(const float* err, int n_complete, int skip, float* s_v, int
   float bv = -INFINITY;
   int bj = -1;
   for (int j = threadIdx.x; j < n_complete; j += blockDim.x) {
-    const float v = err[j];
-    if (j != skip && v >= 0.0f && (bj < 0 || nk_better(v, j, bv, bj))) {
+    const float e = err[j];
+    const float v = e != e ? -FLT_MAX : e;              // NaN ranks as -FLT_MAX
+    if (j != skip && (bj < 0 || nk_better(v, j, bv, bj))) {
       bv = v;
       bj = j;
     }
