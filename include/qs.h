@@ -224,6 +224,15 @@ qs_status qs_select_topk(const qs_config *cfg, const qs_cache *cache,
                          const float *block_scores, int32_t batch, int32_t *sel,
                          int32_t *n_sel, void *ws, qs_stream_t stream);
 
+/* The same selection as qs_select_topk (same arguments, rules and output), computed by
+   three counting passes over the order-preserving keys of the scores (their top 11, next
+   11 and last 10 bits) instead of pairwise ranking: one CTA of 1,024 threads per row, a
+   few streaming passes over the row's scores. For rows of many candidates (token-level
+   selection at long context). One launch. */
+qs_status qs_select_topk_radix(const qs_config *cfg, const qs_cache *cache,
+                               const float *block_scores, int32_t batch, int32_t *sel,
+                               int32_t *n_sel, void *ws, qs_stream_t stream);
+
 /* Exact softmax attention over the selected blocks' valid tokens (stage 3).
    For every query head h of row (b, g): o_h = sum_t softmax_t(scale * q_h.k_t) v_t over
    t in the selected blocks (t < seq_len), normalised over those tokens only. Logits are

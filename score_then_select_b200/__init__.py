@@ -10,7 +10,7 @@ from .binding import (QsError, LIB_PATH, EXPORTS, lib, make_config, make_cache, 
                       qs_sparse_attn_noalloc, qs_attention_launches, qs_selftest_wait_timeout,
                       qs_dense_workspace_size, qs_dense_attn, qs_gather_kv,
                       qs_calib_workspace_size, qs_calibrate_basis, qs_rabitq_score,
-                      qs_select_top_p, qs_decode_top_p, qs_gather_kv_nvfp4k,
+                      qs_select_top_p, qs_decode_top_p, qs_gather_kv_nvfp4k, qs_select_topk_radix,
                       qs_semantic_index_workspace_size,
                       qs_semantic_index, qs_semantic_select, status_string)
 
@@ -20,6 +20,6 @@ __all__ = ["QsError", "LIB_PATH", "EXPORTS", "lib", "make_config", "make_cache",
            "qs_sparse_attn_noalloc", "qs_attention_launches", "qs_selftest_wait_timeout",
            "qs_dense_workspace_size", "qs_dense_attn", "qs_gather_kv",
            "qs_calib_workspace_size", "qs_calibrate_basis", "qs_rabitq_score",
-           "qs_select_top_p", "qs_decode_top_p", "qs_gather_kv_nvfp4k",
+           "qs_select_top_p", "qs_decode_top_p", "qs_gather_kv_nvfp4k", "qs_select_topk_radix",
            "qs_semantic_index_workspace_size",
            "qs_semantic_index", "qs_semantic_select"]

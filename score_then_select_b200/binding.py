@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "qs_decode_top_p": ([cfgp, cachep, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp,
                                  vp, vp, vp], i32),
             "qs_gather_kv_nvfp4k": ([cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp], i32),
+            "qs_select_topk_radix": ([cfgp, cachep, vp, i32, vp, vp, vp, vp], i32),
             "qs_semantic_index_workspace_size": ([cfgp, i32, i32, ctypes.POINTER(sz)], i32),
             "qs_semantic_index": ([cfgp, cachep, vp, i32, vp, vp, vp, i32, vp, vp], i32),
             "qs_semantic_select": ([cfgp, cachep, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp],
@@ -98,7 +99,7 @@ EXPORTS = ("qs_version", "qs_status_string", "qs_workspace_size", "qs_workspace_
            "qs_device_status", "qs_sparse_attn_noalloc", "qs_attention_launches",
            "qs_selftest_wait_timeout", "qs_dense_workspace_size", "qs_dense_attn",
            "qs_gather_kv", "qs_calib_workspace_size", "qs_calibrate_basis", "qs_rabitq_score",
-           "qs_select_top_p", "qs_decode_top_p", "qs_gather_kv_nvfp4k",
+           "qs_select_top_p", "qs_decode_top_p", "qs_gather_kv_nvfp4k", "qs_select_topk_radix",
            "qs_semantic_index_workspace_size",
            "qs_semantic_index", "qs_semantic_select")
 
@@ -202,6 +203,13 @@ def qs_select_topk(cfg, cache, block_scores, batch, sel, n_sel, ws, stream=None)
     _check(lib().qs_select_topk(ctypes.byref(cfg), ctypes.byref(cache), _ptr(block_scores),
                                 batch, _ptr(sel), _ptr(n_sel), _ptr(ws), _stream(stream)),
            "qs_select_topk")
+
+
+def qs_select_topk_radix(cfg, cache, block_scores, batch, sel, n_sel, ws, stream=None):
+    """qs_select_topk's selection by histogram passes instead of pairwise ranking."""
+    _check(lib().qs_select_topk_radix(ctypes.byref(cfg), ctypes.byref(cache), _ptr(block_scores),
+                                      batch, _ptr(sel), _ptr(n_sel), _ptr(ws), _stream(stream)),
+           "qs_select_topk_radix")
 
 
 def qs_sparse_attn(cfg, cache, q, sel, n_sel, batch, out, ws, stream=None):

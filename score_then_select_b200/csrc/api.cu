@@ -13,6 +13,10 @@
 #include "nvfp4k.h"
 
 namespace qs {
+cudaError_t launch_select_radix(const SelectParams& a, cudaStream_t s);
+}
+
+namespace qs {
 
 int num_sms() {
   constexpr int kMaxDevices = 64;
@@ -691,6 +695,34 @@ qs_status qs_decode_top_p(const qs_config* cfg, const qs_cache* cache, const voi
   if ((st = do_rq_score(p, cache, q, R, u, scores, ws, stream)) != QS_OK) return st;
   if ((st = do_top_p(p, cache, scores, p_mass, sel, nsel, ws, stream)) != QS_OK) return st;
   return do_attend(p, cache, q, sel, nsel, out, ws, stream, false);
+}
+
+// ---- top-k by histogram passes (the same result as qs_select_topk)
+qs_status qs_select_topk_radix(const qs_config* cfg, const qs_cache* cache,
+                               const float* block_scores, int32_t batch, int32_t* sel,
+                               int32_t* n_sel, void* ws, qs_stream_t stream) {
+  Plan p;
+  const qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
+  if (st != QS_OK) return st;
+  if (!cache || !cache->seq_lens) return QS_ERR_INVALID_ARG;
+  if (!block_scores || !sel || !n_sel || !ws || !aligned(ws, 256)) return QS_ERR_INVALID_ARG;
+  if (p.kind == PK_NVFP4 && p.n_keep > 0 && !cache->block_err) return QS_ERR_INVALID_ARG;
+  SelectParams a{};
+  a.scores = block_scores;
+  a.block_err = (p.kind == PK_NVFP4 && p.n_keep > 0) ? cache->block_err : nullptr;
+  a.seq_lens = cache->seq_lens;
+  a.sel = sel;
+  a.n_sel = n_sel;
+  a.hdr = hdr_of(ws);
+  a.rows = p.batch * p.Hkv;
+  a.Hkv = p.Hkv;
+  a.S = p.S;
+  a.nb_stride = p.nb_stride;
+  a.budget = p.budget;
+  a.force_sink = p.force_sink;
+  a.force_last = p.force_last;
+  a.n_keep = a.block_err ? p.n_keep : 0;
+  return cuda_status(launch_select_radix(a, stream));
 }
 
 // ---- the NVFP4 storage variant's attended keys ("Jet-QSparse ...", Full text)

@@ -286,3 +286,15 @@ def test_nvfp4_storage_gather_validates_on_the_host():
     with pytest.raises(qs.QsError) as e:                      # no destination
         qs.qs_gather_kv_nvfp4k(nv, cache, a, a, 4, None, a, a, a, stream=0)
     assert e.value.status == B.QS_ERR_INVALID_ARG
+
+
+def test_radix_select_validates_on_the_host():
+    cache, a = B.qs_cache(), 1 << 20
+    with pytest.raises(qs.QsError) as e:                      # no seq_lens
+        qs.qs_select_topk_radix(_cfg(), cache, a, 4, a, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    cache.seq_lens = a
+    with pytest.raises(qs.QsError) as e:                      # kept blocks need block_err
+        qs.qs_select_topk_radix(_cfg(proxy_rank=0, proxy_dtype="nvfp4", block_size=128,
+                                     n_keep_hp=2), cache, a, 4, a, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
