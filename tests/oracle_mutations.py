@@ -73,6 +73,14 @@ MUTATIONS = [
      "return block_max(head_scores.mean(axis=0), S)"),
     ("method", "NVFP4: kept blocks with the smallest error",
      "order = np.lexsort((valid, -err[valid]))", "order = np.lexsort((valid, err[valid]))"),
+    ("method", "NVFP4 attended keys: centre not added before rounding",
+     "    v = (v + np.asarray(mu, dtype=np.float32)[None, :]).astype(np.float32)\n    out = F.f32_to_bf16_rne(v)",
+     "    out = F.f32_to_bf16_rne(v)"),
+    ("method", "NVFP4 attended keys: BF16 by truncation",
+     "    out = F.f32_to_bf16_rne(v)\n    bits = np.asarray(k_bits[:L], dtype=np.uint16)",
+     "    out = (v.view(np.uint32) >> 16).astype(np.uint16)\n    bits = np.asarray(k_bits[:L], dtype=np.uint16)"),
+    ("method", "NVFP4 attended keys: kept blocks not restored",
+     "        out[t0:t1] = bits[t0:t1]\n    return out", "        pass\n    return out"),
     # binary proxy and top-p
     ("method", "binary: bit set at y = 0", "bits = (y > 0).astype(np.uint8)",
      "bits = (y >= 0).astype(np.uint8)"),
