@@ -45,7 +45,7 @@ WORKLOADS = {"block128k": synth.BLOCK128K, "token32k": synth.TOKEN32K, "ragged":
              "nvfp4": synth.NVFP4_128K, "tiny": synth.TINY, "fp8": synth.FP8_128K,
              "fp8token": synth.FP8_TOKEN32K, "centroid": synth.CENTROID_128K,
              "centroid32": synth.CENTROID_S32, "token128k": synth.TOKEN128K,
-             "rabitq128k": synth.RABITQ_TOKEN128K}
+             "rabitq128k": synth.RABITQ_TOKEN128K, "semantic128k": synth.SEMANTIC_128K}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -447,6 +447,8 @@ def run_ours(args):
     f = Filled(inp, attn_path=args.attn_path)
     if w.proxy_dtype == "rabitq":
         return run_ours_top_p(args, w, inp, f, world, rank, local)
+    if w.proxy_dtype == "semantic":
+        return run_ours_semantic(args, w, inp, f, world, rank, local)
     lay, cfg, cache = f.layer, f.cfg, f.cache
     B = w.batch
     lens = inp.lens
@@ -754,6 +756,161 @@ def run_ours_top_p(args, w, inp, f, world, rank, local):
             "gpu_launches": args.steps * launches_per_step}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_ours_semantic(args, w, inp, f, world, rank, local):
+    """The semantic-block step ("Coarse Semantic Blocks ...", Abstract). Before timing, the
+    k-means index over each sequence's prompt (all but the newest token) is built once.
+    Each timed step appends the newest token (K/V only), runs qs_semantic_select (cluster
+    scores, top clusters, expansion into a token list) and attends over that list with the
+    token-level attention. No CPU baseline: the oracle's float32 k-means is far too slow at
+    this size."""
+    import torch
+    import torch.distributed as dist
+    import score_then_select_b200 as qs
+    from score_then_select_b200.graph import CapturedDecode
+    from score_then_select_b200.layer import workspace
+    from tests.gpu_util import cfg_kwargs
+
+    lay, cfg, cache = f.layer, f.cfg, f.cache
+    B, Hkv, d = w.batch, w.n_kv_heads, w.head_dim
+    lens = inp.lens
+    start_lens = torch.from_numpy((lens - 1).astype(np.int32)).cuda()
+    prompt = start_lens.clone()
+    Lmax = lay.max_context
+    rows, c_max = B * Hkv, -(-Lmax // w.block_size)
+    cent = torch.empty((rows, c_max, d), dtype=torch.float32, device="cuda")
+    offsets = torch.empty((rows, c_max + 1), dtype=torch.int32, device="cuda")
+    members = torch.empty((rows, Lmax), dtype=torch.int32, device="cuda")
+    ws_idx = workspace(qs.qs_semantic_index_workspace_size(cfg, B, Lmax))
+    lay.seq_lens.copy_(start_lens)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    qs.qs_semantic_index(cfg, cache, prompt, 4, cent, offsets, members, B, ws_idx)
+    torch.cuda.synchronize()
+    index_ms = (time.perf_counter() - t0) * 1e3
+    st = qs.qs_device_status(ws_idx)
+    if st[0] != 0:
+        raise RuntimeError(f"device status after the index build {st}")
+    max_tokens = Lmax
+    cfg_tok = qs.make_config(**dict(cfg_kwargs(w), block_size=1, budget=max_tokens))
+    ws_tok = workspace(qs.qs_workspace_size(cfg_tok, B, Lmax))
+    tokens = torch.empty((B, Hkv, max_tokens), dtype=torch.int32, device="cuda")
+    ntok = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
+    ones = torch.ones((B,), dtype=torch.int32, device="cuda")
+    out = torch.zeros((B, w.n_q_heads, d), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def calls(q, k, v, s_, ev=None):
+        if ev:
+            ev[0].record(s_)
+        qs.qs_append_kv(cfg, cache, k, v, ones, 1, None, B, lay.ws, s_)
+        if ev:
+            ev[1].record(s_)
+        qs.qs_semantic_select(cfg, cache, q, prompt, cent, offsets, members, B, tokens, ntok,
+                              max_tokens, lay.ws, s_)
+        if ev:
+            ev[2].record(s_)
+        qs.qs_sparse_attn(cfg_tok, cache, q, tokens, ntok, B, out, ws_tok, s_)
+        if ev:
+            ev[3].record(s_)
+
+    def step(ev=None):
+        lay.seq_lens.copy_(start_lens, non_blocking=True)
+        calls(f.q, f.k_last, f.v_last, stream, ev)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    for ws in (lay.ws, ws_tok):
+        st = qs.qs_device_status(ws)
+        if st[0] != 0:
+            raise RuntimeError(f"device status {st}")
+    ntok_h = ntok.cpu().numpy()
+    launches_per_step = 1 + 3 + qs.qs_attention_launches(cfg_tok, B, Lmax)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    clocks = Clocks(local)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    t_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, "cuda")
+
+    n_stage = min(args.steps, 50)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_stage + 3)]
+    for ev in evs:
+        step(ev)
+    torch.cuda.synchronize()
+    acc = np.zeros(3)
+    for ev in evs[3:]:
+        acc += [ev[j].elapsed_time(ev[j + 1]) for j in range(3)]
+    stage_us = dict(zip(["append", "score+select", "attend"], (acc / n_stage * 1e3).tolist()))
+
+    cap = CapturedDecode(cfg, cache, None, B, out, None, None, lay.ws, f.q, f.k_last, f.v_last,
+                         before=lambda: lay.seq_lens.copy_(start_lens, non_blocking=True),
+                         call=lambda q, k, v, s_: calls(q, k, v, s_))
+    cap.q_host.copy_(f.q.cpu())
+    cap.k_host.copy_(f.k_last.cpu())
+    cap.v_host.copy_(f.v_last.cpu())
+    for _ in range(3):
+        cap.step()
+    n_e2e = max(args.steps, 10)
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(n_e2e):
+        cap.step()
+    e2e_ms = max_over_ranks((time.perf_counter() - t0) * 1e3 / n_e2e, world, "cuda")
+    for ws in (lay.ws, ws_tok):
+        st = qs.qs_device_status(ws)
+        if st[0] != 0:
+            raise RuntimeError(f"device status after the end-to-end runs {st}")
+
+    # bytes: centroids scanned, the attended tokens' K and V, q and out
+    peak, peak_src = peaks()
+    clusters = -(-(lens.astype(np.int64) - 1) // w.block_size)
+    by_cent = int(clusters.sum()) * Hkv * d * 4
+    by_kv = int(ntok_h.astype(np.int64).sum()) * d * 2 * 2
+    by_qo = 2 * B * w.n_q_heads * d * 2
+    by = {"centroids": by_cent, "kv": by_kv, "q+out": by_qo, "total": by_cent + by_kv + by_qo,
+          "attended_tokens": int(ntok_h.sum())}
+    att_us = stage_us["attend"]
+    roof = {"bound": "hbm", "kernel": "attend (token-level attention over the expanded list)",
+            "achieved": by_kv / (att_us * 1e-6) / 1e9, "peak": peak, "unit": "GB/s",
+            "frac": by_kv / (att_us * 1e-6) / 1e9 / peak, "peak_source": peak_src,
+            "algorithmic_bytes_per_launch": by_kv, "launch_us": att_us, "traffic": None}
+    value = aggregate_steps_per_s(t_ms, world)
+    cfg_line = config_of(w, lens)
+    cfg_line.update({"index_build_ms": index_ms, "kmeans_iters": 4,
+                     "mean_attended_tokens": float(ntok_h.mean())})
+    step_gbs = by["total"] / (t_ms * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32+bf16", "data": "synthetic (seeded; shapes of the pages' 128K batch-16 decode)",
+            "config": cfg_line, "tokens_per_s": value * B, "us_per_layer_step": t_ms * 1e3,
+            "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": step_gbs / peak, "bytes_per_step": by},
+            "stage_us": stage_us, "roofline": roof, "clocks": clk,
+            "e2e": {"value": aggregate_steps_per_s(e2e_ms, world), "unit": "steps/s",
+                    "h2d_bytes_per_step": cap.h2d_bytes, "d2h_bytes_per_step": cap.d2h_bytes,
+                    "ms_per_step": e2e_ms, "path": "CapturedDecode (CUDA graph of the three calls)"},
+            "gpu_launches": args.steps * launches_per_step}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -129,6 +129,15 @@ CENTROID_S32 = BLOCK128K.replace(name="centroid_b16_h40kv8_d128_L131072_S32_k256
 RABITQ_TOKEN128K = TOKEN128K.replace(name="rabitq_b16_h32kv8_d128_L131072_p0.9_B2048",
                                      proxy_rank=0, proxy_dtype="rabitq", top_p=0.9, seed=1013)
 
+# Semantic blocks ("Coarse Semantic Blocks ...", Abstract): a k-means index over each
+# sequence's prompt (all but the newest token), clusters of about 128 tokens, the 64
+# best-scoring clusters attended, together with every token after the prompt. Keys from
+# the mixture recipe, so that clusters of non-contiguous tokens exist.
+SEMANTIC_128K = BLOCK128K.replace(name="semantic_b16_h40kv8_d128_L131072_S128_k64",
+                                  proxy_rank=0, proxy_dtype="semantic", key_recipe="mixture",
+                                  query_recipe="normal", force_sink=False, force_last=False,
+                                  seed=1014)
+
 # Ragged batch: 32 sequences, lengths uniform in [4096, 131072], G = 8, r = 64, S = 64.
 RAGGED = Workload(
     name="ragged_b32_h64kv8_d128_S64_k32_r64", batch=32, n_q_heads=64, n_kv_heads=8,
@@ -148,6 +157,7 @@ ORDER = [TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED]
 # variants of the configurations above (FP8 projected keys, centroid scoring, 128K token
 # level, the binary proxy with a top-p budget)
 VARIANTS = [FP8_128K, FP8_TOKEN32K, CENTROID_128K, CENTROID_S32, TOKEN128K, RABITQ_TOKEN128K]
+# SEMANTIC_128K is not among them: its oracle step also needs the prompt length.
 
 
 def small(w: Workload) -> Workload:
