@@ -2,8 +2,9 @@
 
     python tests/oracle_mutations.py
 
-Each entry below is a plausible mistake in the oracle: a dropped term, a wrong rounding,
-a transposed operand, a tie broken the wrong way. For each one, a child process alters the
+Each entry below is a plausible mistake in the oracle (its methods, number formats and
+per-row step compositions): a dropped term, a wrong rounding, a transposed operand, a tie
+broken the wrong way. For each one, a child process alters the
 oracle module's source in memory (nothing is written to disk), installs the altered module
 in place of the real one, and runs the oracle pin tests (`-m "not gpu"`). A mistake that no
 pin catches is reported as MISSED. Two entries are rewrites that compute the same thing for
@@ -142,6 +143,22 @@ MUTATIONS = [
      "            s = np.zeros(d, dtype=np.float32)\n            for t in members:                                                # token order\n"
      "                s = (s + x[t]).astype(np.float32)",
      "            s = x[members].sum(axis=0, dtype=np.float64).astype(np.float32)"),
+    # the per-row step compositions
+    ("step", "step: V decoded as BF16 when stored FP16",
+     "return F.f16_to_f64(v_bits) if v_dtype == \"f16\" else F.bf16_to_f64(v_bits)",
+     "return F.bf16_to_f64(v_bits)"),
+    ("step", "step: attention over the oracle's selection, ignoring an accepted one",
+     "    use = sel if sel_override is None else np.asarray(sel_override, dtype=np.int64)\n"
+     "    tokens = M.block_tokens(use, p.S, L)\n    q = F.bf16_to_f64(q_bits)",
+     "    use = sel\n    tokens = M.block_tokens(use, p.S, L)\n    q = F.bf16_to_f64(q_bits)"),
+    ("step", "top-p step: weights without the softmax scale",
+     "    w = M.estimated_weights(s, p.scale)", "    w = M.estimated_weights(s, 1.0)"),
+    ("step", "top-p step: forced blocks dropped",
+     "    forced = M.forced_blocks(mass.shape[0], p.force_sink, p.force_last)",
+     "    forced = np.zeros(0, dtype=np.int64)"),
+    ("step", "semantic step: tokens after the prompt dropped",
+     "    tokens = M.semantic_tokens(assign, use, L0, L)",
+     "    tokens = M.semantic_tokens(assign, use, L0, L0)"),
     # number formats
     ("formats", "BF16: ties away from zero", "y = np.round(x64 / step) * step            # np.round is half-to-even",
      "y = np.floor(x64 / step + 0.5) * step"),

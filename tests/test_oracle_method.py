@@ -446,3 +446,38 @@ def test_centroid_sums_round_in_float32_sequence():
     # token-level blocks (S = 1): each sum is the key itself
     kk = _bf(np.random.default_rng(51).standard_normal((7, 4)))
     assert np.array_equal(M.centroid_sums(kk, 1, 7), F.bf16_to_f64(kk).astype(np.float32))
+
+
+# ---------------------------------------------------------------- the per-row step
+
+def test_step_decodes_fp16_values_as_fp16():
+    # 0x3E00 is 1.5 as FP16 but 0.125 as the top half of a float32 (BF16)
+    from oracle import step as OS
+    bits = np.array([[0x3E00, 0xBC00]], dtype=np.uint16)            # 1.5, -1.0 in FP16
+    assert OS.decode_v(bits, "f16").tolist() == [[1.5, -1.0]]
+    assert OS.decode_v(bits, "bf16").tolist() == [[0.125, -0.0078125]]
+
+
+def test_step_attends_over_an_accepted_override():
+    """With sel_override, the output is attention over the override's tokens (checked by a
+    brute-force softmax), not over the oracle's own selection."""
+    from oracle import step as OS
+    rng = np.random.default_rng(31)
+    S, L, d, G = 8, 64, 16, 2
+    k = _bf16(rng.standard_normal((L, d)))
+    v = _bf16(rng.standard_normal((L, d)))
+    q = _bf16(rng.standard_normal((G, d)))
+    P = np.linalg.qr(rng.standard_normal((d, 8)))[0].astype(np.float32)
+    p = OS.RowParams(S=S, budget=3, scale=0.25, proxy="f32", v_dtype="bf16")
+    own = OS.decode_row(p, k, v, q, L, P=P)
+    other = np.setdiff1d(np.arange(L // S), own["sel"])[:3]
+    r = OS.decode_row(p, k, v, q, L, P=P, sel_override=other)
+    toks = [t for j in other for t in range(j * S, j * S + S)]
+    K, V, Q = F.bf16_to_f64(k), F.bf16_to_f64(v), F.bf16_to_f64(q)
+    for h in range(G):
+        x = [0.25 * math.fsum(Q[h] * K[t]) for t in toks]
+        m = max(x)
+        w = [math.exp(z - m) for z in x]
+        want = [math.fsum(w[i] * V[t, c] for i, t in enumerate(toks)) / math.fsum(w)
+                for c in range(d)]
+        assert np.allclose(r["out"][h], want, rtol=1e-12, atol=1e-12)

@@ -374,3 +374,24 @@ def test_step_selects_a_planted_block_and_attends_exactly():
     e = np.exp(x - x.max(axis=1, keepdims=True))
     assert np.allclose(r["out"], (e @ V[toks]) / e.sum(axis=1, keepdims=True), rtol=1e-12,
                        atol=1e-12)
+
+
+def test_step_weights_use_the_softmax_scale():
+    """The top-p step's estimated weights are softmax(scale * score), recomputed here with
+    math.fsum from the step's own scores; at another scale they differ."""
+    rng = np.random.default_rng(23)
+    d, G, S, L = 32, 2, 4, 90
+    k_bits = _bf(rng.standard_normal((L, d)) * 2)
+    v_bits = _bf(rng.standard_normal((L, d)))
+    q_bits = _bf(rng.standard_normal((G, d)) * 2)
+    R = _haar(rng, d)
+    c = np.zeros(d, dtype=np.float32)
+    u = rng.random(d).astype(np.float32)
+    p = ST.TopPParams(S=S, p=0.7, budget=10, scale=0.3, v_dtype="bf16")
+    r = ST.decode_row_top_p(p, k_bits, v_bits, q_bits, L, R, c, u)
+    x = [0.3 * s for s in r["scores"]]
+    m = max(x)
+    e = [math.exp(z - m) for z in x]
+    z = math.fsum(e)
+    assert np.allclose(r["weights"], np.array(e) / z, rtol=1e-12, atol=0)
+    assert not np.allclose(M.estimated_weights(r["scores"], 1.0), r["weights"], rtol=1e-3)
