@@ -159,6 +159,18 @@ MUTATIONS = [
     ("step", "semantic step: tokens after the prompt dropped",
      "    tokens = M.semantic_tokens(assign, use, L0, L)",
      "    tokens = M.semantic_tokens(assign, use, L0, L0)"),
+    ("step", "NVFP4 step: query packed with the key scale",
+     "        q_codes, q_scales = M.nvfp4_pack(qx, g_q)",
+     "        q_codes, q_scales = M.nvfp4_pack(qx, g_k)"),
+    ("step", "step: kept blocks not forced",
+     "    return M.forced_blocks(nb, p.force_sink, p.force_last, keep), keep",
+     "    return M.forced_blocks(nb, p.force_sink, p.force_last), keep"),
+    ("step", "step: projected query over the whole group, not its mean",
+     "    qt = M.proxy_query(q_bits, P)\n    s = M.token_scores",
+     "    qt = M.proxy_query(q_bits, P) * q_bits.shape[0]\n    s = M.token_scores"),
+    ("step", "centroid step: sums of the blocks past the row read",
+     "        return M.centroid_block_scores(q_bits, cache[:-(-L // p.S)], p.S, L)",
+     "        return M.centroid_block_scores(q_bits, cache[:-(-L // p.S) - 1], p.S, L)"),
     # number formats
     ("formats", "BF16: ties away from zero", "y = np.round(x64 / step) * step            # np.round is half-to-even",
      "y = np.floor(x64 / step + 0.5) * step"),

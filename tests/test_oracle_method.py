@@ -481,3 +481,20 @@ def test_step_attends_over_an_accepted_override():
         want = [math.fsum(w[i] * V[t, c] for i, t in enumerate(toks)) / math.fsum(w)
                 for c in range(d)]
         assert np.allclose(r["out"][h], want, rtol=1e-12, atol=1e-12)
+
+
+def test_step_rank_r_scores_are_the_group_mean_scores():
+    """Rank d with P = I and an FP32 proxy: the step's block scores are the block maxima of
+    the exact group-mean scores (the mean of the heads, not their sum)."""
+    from oracle import step as OS
+    rng = np.random.default_rng(32)
+    S, L, d, G = 4, 30, 16, 3
+    k = _bf16(rng.standard_normal((L, d)))
+    q = _bf16(rng.standard_normal((G, d)))
+    p = OS.RowParams(S=S, budget=2, scale=0.25, proxy="f32", v_dtype="bf16")
+    r = OS.decode_row(p, k, k, q, L, P=np.eye(d, dtype=np.float32))
+    K, Q = F.bf16_to_f64(k), F.bf16_to_f64(q)
+    qbar = [math.fsum(Q[:, i]) / G for i in range(d)]
+    s = [math.fsum(qbar[i] * K[t, i] for i in range(d)) for t in range(L)]
+    want = [max(s[j * S:min(L, (j + 1) * S)]) for j in range(-(-L // S))]
+    assert np.allclose(r["beta"], want, rtol=0, atol=1e-5 * max(map(abs, want)))

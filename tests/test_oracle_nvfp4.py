@@ -208,3 +208,39 @@ def test_attended_keys_bf16_round_half_to_even():
     Kb = M.nvfp4_attended_keys_bf16(np.zeros((L, d), np.uint16), codes, scales, g_k,
                                     np.zeros(d, np.float32), [], 16, L)
     assert F.bf16_to_f64(Kb)[0, 0] == 1.0
+
+
+def _nvfp4_step_row(rng, L=512, G=4, n_keep=2, budget=3):
+    from oracle import step as OS
+    d, S = 128, 128
+    k = F.f32_to_bf16_rne((rng.standard_normal((L, d)) * 1.5 + 0.5).astype(np.float32))
+    v = F.f32_to_bf16_rne(rng.standard_normal((L, d)).astype(np.float32))
+    # queries 40x larger than the keys: their tensor scale differs from the keys' by as much
+    q = F.f32_to_bf16_rne((rng.standard_normal((G, d)) * 80).astype(np.float32))
+    mu = F.bf16_to_f64(k).mean(axis=0).astype(np.float32)
+    g_k = np.float32(np.abs(M.centre(k, mu)).max() / np.float32(2688.0))
+    g_q = M.query_scale(q)
+    p = OS.RowParams(S=S, budget=budget, scale=1 / np.sqrt(d), proxy="nvfp4", v_dtype="bf16",
+                     force_sink=False, force_last=False, n_keep=n_keep)
+    r = OS.decode_row(p, k, v, q, L, mu=mu, g_k=g_k, g_q=g_q)
+    return r, k, q, mu
+
+
+def test_step_nvfp4_scores_approximate_the_exact_centred_scores():
+    """The NVFP4 step's block scores (max over heads and tokens of the FP4 dot of the packed
+    query and centred keys) are within a quarter of the largest exact score of
+    max_h,t q_h . (k_t - mu): the query packed with its own tensor scale."""
+    rng = np.random.default_rng(70)
+    r, k, q, mu = _nvfp4_step_row(rng)
+    x = F.bf16_to_f64(k) - mu.astype(np.float64)
+    s = F.bf16_to_f64(q) @ x.T
+    exact = s.max(axis=0).reshape(-1, 128).max(axis=1)
+    assert np.abs(r["beta"] - exact).max() <= 0.25 * np.abs(exact).max()
+
+
+def test_step_nvfp4_kept_blocks_are_forced_and_selected():
+    rng = np.random.default_rng(71)
+    r, *_ = _nvfp4_step_row(rng, L=1024, n_keep=2, budget=3)
+    assert len(r["keep"]) == 2
+    assert set(r["keep"].tolist()) <= set(r["forced"].tolist())
+    assert set(r["keep"].tolist()) <= set(r["sel"].tolist())
