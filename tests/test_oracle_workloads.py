@@ -77,3 +77,23 @@ def test_projection_is_orthonormal():
     assert P.shape == (8, 128, 32)
     assert np.allclose(P[0].T.astype(np.float64) @ P[0], np.eye(32), atol=1e-6)
     assert np.array_equal(P[0], P[7])
+
+
+def test_semantic_workload_rows():
+    """The semantic workload's small copy through the oracle's semantic step: C = ceil(L0/S)
+    clusters, min(budget, C) selected, every token after the prompt attended, finite
+    outputs."""
+    from oracle import step as OS
+    w = synth.small(synth.SEMANTIC_128K)
+    inp = synth.Inputs(w)
+    p = OS.SemanticParams(S=w.block_size, budget=w.budget, iters=2, scale=w.scale,
+                          v_dtype=w.v_dtype)
+    for b in range(w.batch):
+        L = int(inp.lens[b])
+        L0 = L - 1
+        k, v, q = inp.row(b, 0)
+        r = OS.decode_row_semantic(p, k, v, q, L0, L)
+        C = -(-L0 // w.block_size)
+        assert r["centroids"].shape[0] == C and len(r["sel"]) == min(w.budget, C)
+        assert L0 in r["tokens"].tolist() and np.all(np.diff(r["tokens"]) > 0)
+        assert np.all(np.isfinite(r["out"]))
