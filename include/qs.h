@@ -3,8 +3,11 @@
  *
  * The decode step, per row = (sequence b, KV head g):
  *   1. score  - a cheap proxy score of the current query against the row's whole key
- *               history, reduced to one score per block of S tokens (max over the block);
+ *               history, reduced to one score per block of S tokens (max over the block;
+ *               with the binary proxy, the log of the block's estimated attention mass;
+ *               with semantic blocks, one score per cluster of the prompt's keys);
  *   2. select - the top-k blocks per row (forced blocks first), ties to the lower index;
+ *               with the binary proxy, the fewest blocks whose estimated mass reaches p;
  *   3. attend - exact softmax attention of each of the group's query heads over the
  *               selected original keys and values only, FP32 accumulation, split over the
  *               selection and finished by a log-sum-exp combine.
