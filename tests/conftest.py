@@ -11,8 +11,6 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size workloads")
-    config.addinivalue_line("markers", "gpu_pending: needs a CUDA device; written, not yet "
-                                       "run on one (selected with -m gpu_pending)")
 
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")

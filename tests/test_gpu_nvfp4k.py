@@ -1,6 +1,5 @@
 """The NVFP4 storage variant's attended keys ("Jet-QSparse ...", Full text): qs_gather_kv_nvfp4k
-against the oracle, then dense attention over the gathered buffer. Marked gpu_pending:
-written, not yet run on a GPU (`pytest -m gpu_pending` selects it).
+against the oracle, then dense attention over the gathered buffer.
 
 Inputs: the small copy of the NVFP4 128K workload (two kept blocks per row), filled and
 decoded one step through the validated path.
@@ -22,7 +21,7 @@ from oracle import method as M
 from oracle import step as OS
 from tests.util import oracle_row, query_scale_all
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 
 def _gpu():

@@ -1,6 +1,5 @@
 """More parity cases of the binary proxy with a top-p budget ("RaBitQCache", Abstract),
-written after the first GPU run of tests/test_gpu_rabitq.py and marked gpu_pending until
-they have run on a GPU (`pytest -m gpu_pending` selects them):
+beyond those of tests/test_gpu_rabitq.py:
 - two more configurations, through the same checks: S = 32 (one 32-lane reduction per
   block), and S = 4 with d = 64 and a group of 8 query heads;
 - the step call qs_decode_top_p against the four stage calls, bit for bit.
@@ -14,7 +13,7 @@ from tests.test_gpu_rabitq import test_block_log_masses as _log_masses
 from tests.test_gpu_rabitq import test_chain_selects_valid_sets_and_attends_exactly as _chain
 from tests.test_gpu_rabitq import test_writer_codes_bit_exact as _writer
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 MORE = [  # (d, S, G, Hkv, budget, lens)
     (128, 32, 2, 2, 16, [1100, 257, 640]),

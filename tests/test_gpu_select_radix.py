@@ -1,6 +1,5 @@
 """qs_select_topk_radix (top-k by histogram passes) against qs_select_topk and the oracle,
-on the crafted block scores of the select tests. Marked gpu_pending: written, not yet run
-on a GPU (`pytest -m gpu_pending` selects it).
+on the crafted block scores of the select tests.
 
 The bar: the radix selection equals qs_select_topk's exactly, and both equal the oracle's
 (forced blocks, then the best others with ties to the lower index, ascending; NaN and
@@ -14,7 +13,7 @@ import torch
 from oracle import method as M
 from tests.test_gpu_select import KINDS, SHAPES, _mapped, _scores
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 
 def _gpu():

@@ -1,6 +1,5 @@
 """Parity of the semantic-block path ("Coarse Semantic Blocks ...", Abstract) with the
-oracle, through the C ABI. Marked gpu_pending: written, not yet run on a GPU
-(`pytest -m gpu_pending` selects it).
+oracle, through the C ABI.
 
 Inputs: per row, keys drawn around 6 centres N(0, 9 I) with N(0, 0.25 I) noise, so the
 clusters are non-contiguous; V and q N(0, 1); ragged lengths; the index covers a prefix
@@ -24,7 +23,7 @@ import torch
 from oracle import method as M
 from synth.gen import to_bf16_bits
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 
 def _gpu():
