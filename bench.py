@@ -204,9 +204,8 @@ def oracle_prepare(w, inp, rows, threads):
     from threadpoolctl import threadpool_limits
     from oracle import method as M
     from oracle import step as OS
-    from tests.util import row_params, top_p_params
 
-    p = top_p_params(w) if w.proxy_dtype == "rabitq" else row_params(w)
+    p = OS.top_p_params_of(w) if w.proxy_dtype == "rabitq" else OS.row_params_of(w)
 
     def prep(bg):
         b, g = bg
@@ -442,7 +441,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     import score_then_select_b200 as qs
-    from tests.gpu_util import Filled
+    from score_then_select_b200.filled import Filled
 
     w0 = WORKLOADS[args.workload]
     if args.batch:
@@ -781,7 +780,7 @@ def run_ours_semantic(args, w, inp, f, world, rank, local):
     import score_then_select_b200 as qs
     from score_then_select_b200.graph import CapturedDecode
     from score_then_select_b200.layer import workspace
-    from tests.gpu_util import cfg_kwargs
+    from score_then_select_b200.filled import cfg_kwargs
 
     lay, cfg, cache = f.layer, f.cfg, f.cache
     B, Hkv, d = w.batch, w.n_kv_heads, w.head_dim

@@ -33,6 +33,14 @@ class RowParams:
     n_keep: int = 0            # NVFP4: blocks kept at full precision
 
 
+def row_params_of(w) -> RowParams:
+    """The row parameters of a workload description (its block size, budget, softmax scale,
+    proxy kind, value format and forced blocks)."""
+    return RowParams(S=w.block_size, budget=w.budget, scale=w.scale, proxy=w.proxy_dtype,
+                     v_dtype=w.v_dtype, force_sink=w.force_sink, force_last=w.force_last,
+                     n_keep=w.n_keep_hp)
+
+
 def decode_v(v_bits: np.ndarray, v_dtype: str) -> np.ndarray:
     return F.f16_to_f64(v_bits) if v_dtype == "f16" else F.bf16_to_f64(v_bits)
 
@@ -107,6 +115,14 @@ class TopPParams:
     v_dtype: str               # 'bf16' | 'f16'
     force_sink: bool = False
     force_last: bool = False
+
+
+def top_p_params_of(w) -> TopPParams:
+    """The binary proxy's row parameters of a workload description; p as the float32 that
+    the library takes."""
+    return TopPParams(S=w.block_size, p=float(np.float32(w.top_p)), budget=w.budget,
+                      scale=w.scale, v_dtype=w.v_dtype, force_sink=w.force_sink,
+                      force_last=w.force_last)
 
 
 def decode_row_top_p(p: TopPParams, k_bits, v_bits, q_bits, L: int, R, c, u,
