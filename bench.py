@@ -42,7 +42,8 @@ import synth  # noqa: E402
 
 METRIC = "sparse decode attn steps/s at 128K ctx, batch 16; achieved HBM GB/s vs peak"
 WORKLOADS = {"block128k": synth.BLOCK128K, "token32k": synth.TOKEN32K, "ragged": synth.RAGGED,
-             "nvfp4": synth.NVFP4_128K, "tiny": synth.TINY, "fp8": synth.FP8_128K,
+             "nvfp4": synth.NVFP4_128K, "nvfp4store": synth.NVFP4_STORE_128K,
+             "tiny": synth.TINY, "fp8": synth.FP8_128K,
              "fp8token": synth.FP8_TOKEN32K, "centroid": synth.CENTROID_128K,
              "centroid32": synth.CENTROID_S32, "token128k": synth.TOKEN128K,
              "rabitq128k": synth.RABITQ_TOKEN128K, "semantic128k": synth.SEMANTIC_128K}
@@ -161,12 +162,18 @@ def step_bytes(w, lens, sel, nsel):
             per_tok = w.proxy_rank * {"f32": 4, "bf16": 2, "e4m3": 1}[w.proxy_dtype]
         proxy = int(np.sum(lens.astype(np.int64))) * w.n_kv_heads * per_tok
     tokens = 0
+    kept_tokens = 0                      # NVFP4 key storage: tokens of the kept BF16 blocks
     for b in range(w.batch):
         L = int(lens[b])
         for g in range(w.n_kv_heads):
             blk = sel[b, g, :int(nsel[b, g])].astype(np.int64)
             tokens += int(np.minimum(S, L - blk * S).sum())
-    kv = tokens * d * 2 * 2
+            kept_tokens += min(w.n_keep_hp, L // S) * S     # complete, always selected
+    if getattr(w, "key_storage", "bf16") == "nvfp4":
+        # K: 72 bytes per token (d/2 of codes, d/16 of scales) except the kept blocks' BF16
+        kv = tokens * d * 2 + (tokens - kept_tokens) * (d // 2 + d // 16) + kept_tokens * d * 2
+    else:
+        kv = tokens * d * 2 * 2
     q = w.batch * w.n_q_heads * d * 2
     out = w.batch * w.n_q_heads * d * (4 if w.out_dtype == "f32" else 2)
     return {"proxy": proxy, "kv": kv, "q": q, "out": out, "total": proxy + kv + q + out,
@@ -341,27 +348,30 @@ def run_reference(args):
             "longer than a bounded timing run")}), flush=True)
         return 0
     inp = synth.Inputs(w)
-    cores = host_cores()
     rows_all = [(b, g) for b in range(w.batch) for g in range(w.n_kv_heads)]
-    per_step = min(cores, len(rows_all), 8)
-    total_rows = len(rows_all)
-    prep = oracle_prepare(w, inp, rows_all[:per_step], per_step)
+    threads = min(host_cores(), len(rows_all))
+    # untimed: the rows' stored inputs and scoring caches (the writer's output)
+    prep = oracle_prepare(w, inp, rows_all, threads)
     times = []
+    t_run = time.perf_counter()
     for i in range(args.warmup + args.steps):
-        t = oracle_time(w, inp, prep, per_step)
+        t = oracle_time(w, inp, prep, threads)            # one whole step: every row
         if i >= args.warmup:
             times.append(t)
+    run_s = time.perf_counter() - t_run
     t_step = sum(times) / len(times)
-    value = (per_step / total_rows) / t_step
+    value = 1.0 / t_step
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": 1e3 * t_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, inp.lens),
-            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": per_step,
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": threads,
                              "kind": "oracle",
-                             "sample": f"{per_step} of {total_rows} rows per step, "
-                                       "score+select+attend from prepared scoring caches"},
+                             "sample": f"whole steps: all {len(rows_all)} (sequence, KV head) "
+                                       f"rows, score+select+attend from prepared scoring "
+                                       f"caches, float64 numpy, one row per host thread; "
+                                       f"{args.warmup}+{args.steps} steps in {run_s:.1f} s"},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -612,6 +622,23 @@ def run_ours(args):
                     "ms_per_step": e2e_ms, "path": "CapturedDecode (CUDA graph of the step)",
                     "eager_ms_per_step": eager_ms},
             "gpu_launches": args.steps * launches_per_step}
+    # the attention stage's own roofline: selected K/V bytes + q + out over its stage time
+    att_b = by["kv"] + by["q"] + by["out"]
+    line["attend_hbm"] = {"achieved": att_b / (stage_us["attend"] * 1e-6) / 1e9, "peak": peak,
+                          "unit": "GB/s",
+                          "frac": att_b / (stage_us["attend"] * 1e-6) / 1e9 / peak,
+                          "bytes": att_b, "us": stage_us["attend"]}
+    if getattr(w, "key_storage", "bf16") == "nvfp4":
+        # capacity of the storage variant ("Jet-QSparse ...", Full text): bytes held per
+        # cached token by the key and value pages the attention needs, against a BF16 K/V
+        # cache (the two kept BF16 blocks of each row are spread over its tokens)
+        d = w.head_dim
+        kept = w.n_keep_hp * w.block_size * d * 2 / float(lens.mean())
+        per_tok = (d // 2 + d // 16) + d * 2 + kept
+        line["capacity"] = {"bytes_per_token": per_tok, "bf16_kv_bytes_per_token": 4 * d,
+                            "tokens_vs_bf16_kv": 4 * d / per_tok,
+                            "note": "NVFP4 keys (codes + scales), FP16 values, 2 BF16 blocks "
+                                    "per (sequence, KV head)"}
     if compare is not None:
         line["comparison"] = compare
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -67,9 +67,18 @@
  *                                                           4 exponent bits with bias 7,
  *                                                           3 mantissa bits; largest 448;
  *                                                           one byte per entry)
- *   proxy (NVFP4)   [num_pages][Hkv][page_size][head_dim/2] u8: E2M1 codes, element 2i in
- *                                                           the low nibble of byte i
- *   proxy_scale     [num_pages][Hkv][page_size][head_dim/16] u8: UE4M3 scale per 16 elems
+ *   proxy (NVFP4)   [num_pages][Hkv] x 8192 bytes (head_dim 128, page_size 128) of E2M1
+ *                   codes, chunk-major: element e (0..127) of token slot m (0..127) is in
+ *                   byte (e / 32) * 2048 + m * 16 + (e % 32) / 2, in the low nibble when e
+ *                   is even and the high nibble when it is odd. Each 32-element chunk of a
+ *                   token is one 16-byte row, so a contiguous copy of the page lands as the
+ *                   K-major operand of the FP4 tensor-core MMA (8-token x 16-byte core
+ *                   matrices, chunks 2048 bytes apart).
+ *   proxy_scale     [num_pages][Hkv] x 1024 bytes of UE4M3 scales: the scale of elements
+ *                   16j .. 16j+15 (j = 0..7) of token slot m is byte
+ *                   (j / 4) * 512 + 16 * (m % 32) + 4 * (m / 32) + j % 4, the order in
+ *                   which the tensor cores' scale-factor copy (tcgen05.cp 32x128b.warpx4)
+ *                   expects a 128-token tile's scales.
  *   proxy (centroid)[num_pages][Hkv][page_size/S][head_dim] F32: the sum of the keys of each
  *                                                           S-token block of the page
  *   proxy (binary)  [num_pages][Hkv] x (page_size * head_dim/8 bytes of code bits, then
@@ -141,6 +150,21 @@ typedef struct {
                              per resident CTA, else the gather kernel); 1 tile pipeline
                              (needs block_size >= 8); 2 gather kernel. Same results up to
                              float32 summation order.                                    */
+  int32_t key_storage;    /* the keys the attention reads ("Jet-QSparse ...", Full text: the
+                             persistent cache keeps the attended keys in NVFP4, at most two
+                             blocks per sequence at BF16). 0 (or QS_BF16): the BF16 key
+                             pages. QS_NVFP4 (needs proxy_dtype QS_NVFP4, the tile pipeline,
+                             head_dim 128): a token of one of the row's n_keep_hp kept blocks
+                             is read from the BF16 key pages; every other token's key is its
+                             NVFP4 scoring copy, decoded, un-centred and rounded to BF16 in
+                             the kernel, bf16_rne(fp32(fp32(e * sigma) * g_k) + mu). The K
+                             bytes read per token fall from 2 * head_dim to 72 (codes and
+                             scales); a plain copy of the BF16 key pages is then needed only
+                             for the kept blocks. Every call that attends then needs the
+                             cache's proxy, proxy_scale, key_center (16-byte aligned),
+                             key_gscale and, with n_keep_hp > 0, block_err
+                             (QS_ERR_INVALID_ARG otherwise); qs_dense_attn always reads the
+                             BF16 keys; qs_sparse_attn_noalloc returns QS_ERR_UNSUPPORTED. */
 } qs_config;
 
 /* The paged caches of one layer. All pointers are device pointers owned by the caller. */
@@ -165,8 +189,9 @@ typedef struct {
 qs_status qs_workspace_size(const qs_config *cfg, int32_t batch, int32_t max_context,
                             size_t *bytes /* host */);
 
-/* Number of kernel launches qs_sparse_attn makes for this shape (1: gather kernel with an
-   in-kernel merge; 2: tile pipeline, then the row merge). Host only. */
+/* Number of kernel launches qs_sparse_attn makes for this shape: 1 (both attention
+   kernels, the gather kernel and the tile pipeline, merge each row's partials in the same
+   launch), 2 with key_storage QS_NVFP4 (the rows' kept blocks first). Host only. */
 qs_status qs_attention_launches(const qs_config *cfg, int32_t batch, int32_t max_context,
                                 int32_t *launches /* host */);
 
@@ -377,7 +402,7 @@ qs_status qs_dense_workspace_size(const qs_config *cfg, int32_t batch, int32_t m
    budget, forced blocks and attn_path are not used); the cache's proxy fields are not
    read. Logits are float32 sums of BF16 products, P.V operands v_agg_dtype, float32
    accumulation; the row is split over the tile-pipeline attention kernel and merged by
-   the log-sum-exp combine (2 launches). Every len must be <= cache->max_context (a row
+   the log-sum-exp combine inside the same launch (1 launch). Every len must be <= cache->max_context (a row
    that needs more than ceil(max_context / 128) pages records QS_ERR_DEVICE_BOUNDS). ws: qs_dense_workspace_size(cfg, batch,
    cache->max_context) bytes, initialised by qs_workspace_init. q is 16-byte aligned. */
 qs_status qs_dense_attn(const qs_config *cfg, const qs_cache *cache, const void *q,

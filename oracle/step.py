@@ -31,6 +31,7 @@ class RowParams:
     force_sink: bool = False
     force_last: bool = False
     n_keep: int = 0            # NVFP4: blocks kept at full precision
+    key_storage: str = "bf16"  # 'nvfp4': attention over the NVFP4 storage variant's keys
 
 
 def row_params_of(w) -> RowParams:
@@ -38,7 +39,7 @@ def row_params_of(w) -> RowParams:
     proxy kind, value format and forced blocks)."""
     return RowParams(S=w.block_size, budget=w.budget, scale=w.scale, proxy=w.proxy_dtype,
                      v_dtype=w.v_dtype, force_sink=w.force_sink, force_last=w.force_last,
-                     n_keep=w.n_keep_hp)
+                     n_keep=w.n_keep_hp, key_storage=getattr(w, "key_storage", "bf16"))
 
 
 def decode_v(v_bits: np.ndarray, v_dtype: str) -> np.ndarray:
@@ -83,11 +84,18 @@ def row_forced(p: RowParams, nb: int, cache=None, L: int = 0, g_k=None):
 
 
 def decode_row(p: RowParams, k_bits, v_bits, q_bits, L: int, P=None, mu=None, g_k=None,
-               g_q=None, sel_override=None):
+               g_q=None, sel_override=None, keep_override=None):
     """Full oracle step for one row. Returns a dict of every intermediate.
 
     ``sel_override``: attend over this selection instead of the oracle's own (used once a
     GPU selection has been accepted as a valid top-k under the near-tie rule).
+    ``keep_override``: with NVFP4 key storage, the kept (BF16) blocks whose stored keys are
+    attended (used once the GPU's kept pair has been accepted under the near-tie rule).
+
+    With ``p.key_storage == 'nvfp4'`` ("Jet-QSparse ...", Full text: the persistent cache
+    keeps the attended keys in NVFP4, at most two blocks per sequence at BF16), the keys
+    attended are nvfp4_attended_keys_bf16: the kept blocks' stored BF16 keys, elsewhere the
+    NVFP4 code dequantised and un-centred, rounded to BF16 (returned as ``K_att``).
     """
     cache = row_scoring_cache(p, k_bits[:L], P, mu, g_k)
     beta = row_block_scores(p, cache, q_bits, L, P=P, g_q=g_q, g_k=g_k)
@@ -97,11 +105,17 @@ def decode_row(p: RowParams, k_bits, v_bits, q_bits, L: int, P=None, mu=None, g_
     use = sel if sel_override is None else np.asarray(sel_override, dtype=np.int64)
     tokens = M.block_tokens(use, p.S, L)
     q = F.bf16_to_f64(q_bits)
-    K = F.bf16_to_f64(k_bits[:L])
+    if p.key_storage == "nvfp4":
+        codes, scales, _ = cache
+        kept = keep if keep_override is None else np.asarray(keep_override, dtype=np.int64)
+        K = F.bf16_to_f64(M.nvfp4_attended_keys_bf16(k_bits[:L], codes, scales, g_k, mu, kept,
+                                                     p.S, L))
+    else:
+        K = F.bf16_to_f64(k_bits[:L])
     V = decode_v(v_bits[:L], p.v_dtype)
     out = M.sparse_attention(q, K, V, tokens, p.scale)
     return dict(cache=cache, beta=beta, forced=forced, keep=keep, sel=sel, tokens=tokens,
-                out=out)
+                out=out, K_att=K)
 
 
 # ---- the binary proxy with a top-p budget ("RaBitQCache", Abstract) ------------------------

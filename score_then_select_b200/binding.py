@@ -31,7 +31,8 @@ class qs_config(ctypes.Structure):
         "n_q_heads", "n_kv_heads", "head_dim", "page_size", "block_size", "budget",
         "proxy_rank", "proxy_dtype", "v_dtype", "v_agg_dtype", "out_dtype", "force_sink",
         "force_last", "n_keep_hp")] + [("softmax_scale", ctypes.c_float),
-                                         ("attn_path", ctypes.c_int32)]
+                                         ("attn_path", ctypes.c_int32),
+                                         ("key_storage", ctypes.c_int32)]
 
 
 class qs_cache(ctypes.Structure):
@@ -133,7 +134,7 @@ def _check(st: int, where: str):
 def make_config(*, n_q_heads, n_kv_heads, head_dim, block_size, budget, proxy_rank,
                 proxy_dtype, v_dtype="bf16", v_agg_dtype="bf16", out_dtype="bf16",
                 force_sink=False, force_last=False, n_keep_hp=0, softmax_scale=0.0,
-                page_size=128, attn_path=0) -> qs_config:
+                page_size=128, attn_path=0, key_storage="bf16") -> qs_config:
     c = qs_config()
     c.n_q_heads, c.n_kv_heads, c.head_dim = n_q_heads, n_kv_heads, head_dim
     c.page_size, c.block_size, c.budget = page_size, block_size, budget
@@ -144,6 +145,7 @@ def make_config(*, n_q_heads, n_kv_heads, head_dim, block_size, budget, proxy_ra
     c.force_sink, c.force_last, c.n_keep_hp = int(force_sink), int(force_last), n_keep_hp
     c.softmax_scale = softmax_scale
     c.attn_path = attn_path
+    c.key_storage = 0 if key_storage == "bf16" else DTYPE_CODES[key_storage]
     return c
 
 

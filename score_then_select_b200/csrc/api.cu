@@ -139,6 +139,15 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   if (c->v_agg_dtype != QS_BF16 && c->v_agg_dtype != QS_F16) return QS_ERR_INVALID_ARG;
   if (c->v_dtype == QS_F16 && c->v_agg_dtype != QS_F16) return QS_ERR_UNSUPPORTED;
   if (c->out_dtype != QS_F32 && c->out_dtype != QS_BF16) return QS_ERR_INVALID_ARG;
+  if (c->key_storage != 0 && c->key_storage != QS_BF16 && c->key_storage != QS_NVFP4)
+    return QS_ERR_INVALID_ARG;
+  p.key_nvfp4 = c->key_storage == QS_NVFP4;
+  if (p.key_nvfp4) {
+    // the scoring copy must be NVFP4 (d = 128, 128-token blocks, checked above); the
+    // decode happens in the tile pipeline
+    if (p.kind != PK_NVFP4) return QS_ERR_INVALID_ARG;
+    if (c->attn_path == 2) return QS_ERR_UNSUPPORTED;
+  }
 
   p.batch = batch;
   p.Hq = c->n_q_heads;
@@ -172,7 +181,7 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   {
     const long long tiles = (long long)batch * p.Hkv * ((slots + 63) / 64);
     const long long ctas = (long long)kAttnCtasPerSm * num_sms();
-    p.attn_tma = c->attn_path == 1 ||
+    p.attn_tma = c->attn_path == 1 || p.key_nvfp4 ||
                  (c->attn_path == 0 && p.S >= kAttnTmaMinRun && tiles >= kTmaMinTilesPerCta * ctas);
   }
   if (p.attn_tma) {
@@ -184,6 +193,9 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   }
   size_t off = size_t(kHdrWords) * 4;
   const size_t rows = size_t(batch) * p.Hkv, rows_q = size_t(batch) * p.Hq;
+  // the self-resetting row counters first: at the same place for every batch, so a
+  // workspace initialised for `batch` sequences serves calls of fewer sequences too
+  w.row_ctr = off; off = align_up(off + rows * 4, 256);
   w.qt = off;      off = align_up(off + rows * (r > 0 ? r : (p.kind == PK_RABITQ ? kRqRowWords : 1)) * 4, 256);
   w.qtile = off;   off = align_up(off + (p.kind == PK_NVFP4 ? rows * kQTileBytes : 0), 256);
   w.qgscale = off; off = align_up(off + 16, 256);
@@ -192,7 +204,7 @@ qs_status make_plan(const qs_config* c, int batch, int max_context, Plan& p) {
   w.nsel = off;    off = align_up(off + rows * 4, 256);
   w.part_ml = off; off = align_up(off + rows_q * w.parts_per_head * 2 * 4, 256);
   w.part_o = off;  off = align_up(off + rows_q * w.parts_per_head * p.d * 4, 256);
-  w.row_ctr = off; off = align_up(off + rows * 4, 256);
+  w.kept = off;    off = align_up(off + (p.key_nvfp4 ? rows * 2 * 4 : 0), 256);
   w.total = off;
   return QS_OK;
 }
@@ -209,6 +221,7 @@ static qs_status make_dense_plan(const qs_config* c, int batch, int max_context,
   d.force_sink = d.force_last = 0;
   d.n_keep_hp = 0;
   d.attn_path = 1;
+  d.key_storage = 0;            // the full-KV comparison reads the BF16 key pages
   return make_plan(&d, batch, max_context, p);
 }
 
@@ -222,6 +235,14 @@ qs_status check_cache(const Plan& p, const qs_cache* c, bool need_proxy) {
     if (p.kind == PK_NVFP4 && (!c->proxy_scale || !c->key_center || !c->key_gscale))
       return QS_ERR_INVALID_ARG;
     if (p.kind == PK_RABITQ && !c->key_center) return QS_ERR_INVALID_ARG;
+  }
+  // attention over the NVFP4 keys reads the codes, scales and centres by bulk copies and
+  // the block errors for the kept blocks, whatever the call
+  if (p.key_nvfp4) {
+    if (!c->proxy || !c->proxy_scale || !c->key_center || !c->key_gscale) return QS_ERR_INVALID_ARG;
+    if (p.n_keep > 0 && !c->block_err) return QS_ERR_INVALID_ARG;
+    if (!aligned(c->proxy, 16) || !aligned(c->proxy_scale, 16) || !aligned(c->key_center, 16))
+      return QS_ERR_INVALID_ARG;
   }
   return QS_OK;
 }
@@ -237,8 +258,9 @@ static qs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QS_OK : 
 // ------------------------------------------------------------ stage bodies (validated input)
 static qs_status do_append(const Plan& p, const qs_cache* c, const void* k_new, const void* v_new,
                            const int32_t* n_new, int max_new, const float* P, const void* q,
-                           void* ws, cudaStream_t s) {
+                           void* ws, cudaStream_t s, bool keep_lens = false) {
   AppendParams a{};
+  a.keep_lens = keep_lens ? 1 : 0;
   a.k_new = static_cast<const uint16_t*>(k_new);
   a.v_new = static_cast<const uint16_t*>(v_new);
   a.n_new = n_new;
@@ -300,10 +322,26 @@ static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws,
   return cuda_status(launch_qpack(p, a, s, pdl));
 }
 
+// Step modes of the rank-r decode (qs_decode): the writer leaves seq_lens alone and every
+// later kernel reads seq_lens + 1; the scan starts streaming at once and computes q~ itself
+// (rank <= 32; rank 64 takes it from the writer); the attention advances seq_lens at its end.
+struct StepMode {
+  bool decode = false;      // the one-token decode step of a rank-r configuration
+  const float* P = nullptr;
+};
+
 static qs_status do_score(const Plan& p, const qs_cache* c, const void* q, float* scores, void* ws,
-                          cudaStream_t s, bool pdl, bool early_stream = false) {
+                          cudaStream_t s, bool pdl, bool early_stream = false,
+                          const StepMode& m = StepMode()) {
   ScoreParams a{};
   a.early_stream = early_stream ? 1 : 0;
+  if (m.decode) {
+    a.early_stream = 1;
+    a.len_add = 1;
+    a.wait_last = 1;
+    a.inline_qt = p.r <= 32 ? 1 : 0;
+    a.P = m.P;
+  }
   a.q = static_cast<const uint16_t*>(q);
   a.proxy = c->proxy;
   a.proxy_scale = c->proxy_scale;
@@ -328,8 +366,10 @@ static qs_status do_score(const Plan& p, const qs_cache* c, const void* q, float
 }
 
 static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores, int32_t* sel,
-                           int32_t* n_sel, void* ws, cudaStream_t s, bool pdl) {
+                           int32_t* n_sel, void* ws, cudaStream_t s, bool pdl,
+                           const StepMode& m = StepMode()) {
   SelectParams a{};
+  a.len_add = m.decode ? 1 : 0;
   a.scores = scores;
   a.block_err = (p.kind == PK_NVFP4 && p.n_keep > 0) ? c->block_err : nullptr;
   a.seq_lens = c->seq_lens;
@@ -349,8 +389,12 @@ static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores
 
 static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, const int32_t* sel,
                            const int32_t* n_sel, void* out, void* ws, cudaStream_t s, bool pdl,
-                           const int32_t* row_lens = nullptr) {
+                           const int32_t* row_lens = nullptr, const StepMode& m = StepMode()) {
   AttnParams a{};
+  if (m.decode) {
+    a.len_add = 1;
+    a.lens_out = c->seq_lens;
+  }
   a.row_lens = row_lens;
   a.q = static_cast<const uint16_t*>(q);
   a.k = static_cast<const uint16_t*>(c->k);
@@ -378,6 +422,20 @@ static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, cons
   a.max_pages_per_seq = c->max_pages_per_seq;
   a.num_pages = c->num_pages;
   a.scale_log2 = p.scale * 1.4426950408889634f;
+  if (p.key_nvfp4) {
+    // NVFP4 keys: the row's kept blocks first (one CTA per row), then the attention
+    a.k_codes = static_cast<const uint8_t*>(c->proxy);
+    a.k_scales = c->proxy_scale;
+    a.key_center = c->key_center;
+    a.key_gscale = c->key_gscale;
+    int32_t* kept = ws_at<int32_t>(ws, p.ws.kept);
+    a.kept = kept;
+    KeptParams kp{c->block_err, c->seq_lens, kept, p.batch * p.Hkv, p.Hkv, p.nb_stride,
+                  p.n_keep, a.len_add};
+    const qs_status st = cuda_status(launch_kept_blocks(kp, s, pdl));
+    if (st != QS_OK) return st;
+    pdl = true;
+  }
   return cuda_status(launch_attn(p, a, s, pdl));
 }
 
@@ -416,7 +474,8 @@ qs_status qs_attention_launches(const qs_config* cfg, int32_t batch, int32_t max
   const qs_status st = make_plan(cfg, batch, max_context, p);
   if (st != QS_OK) return st;
   if (!launches) return QS_ERR_INVALID_ARG;
-  *launches = p.attn_tma ? 2 : 1;
+  // both kernels merge their partials in-kernel; NVFP4 keys add the kept-block kernel
+  *launches = p.key_nvfp4 ? 2 : 1;
   return QS_OK;
 }
 
@@ -580,7 +639,22 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, p.ws.sel);
   int32_t* nsel = n_sel_out ? n_sel_out : ws_at<int32_t>(ws, p.ws.nsel);
   float* scores = ws_at<float>(ws, p.ws.scores);
-  // append (+ fused scoring prep on the rank-r path)
+  if (p.kind == PK_RANKR) {
+    // the writer runs under the scan: it leaves seq_lens alone (the step reads seq_lens + 1),
+    // the scan computes q~ itself (rank <= 32; else the writer's fused prep gives it) and
+    // waits for the writer only before a row's last page, and the attention advances
+    // seq_lens once every kernel of the step has read them
+    StepMode m;
+    m.decode = true;
+    m.P = P;
+    const void* prep_q = p.r <= 32 ? nullptr : q;
+    if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, P, prep_q, ws, stream, true)) != QS_OK)
+      return st;
+    if ((st = do_score(p, cache, q, scores, ws, stream, true, true, m)) != QS_OK) return st;
+    if ((st = do_select(p, cache, scores, sel, nsel, ws, stream, true, m)) != QS_OK) return st;
+    return do_attend(p, cache, q, sel, nsel, out, ws, stream, true, nullptr, m);
+  }
+  // append (+ query packing on the NVFP4 path), then the stages in stream order
   if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, P, q, ws, stream)) != QS_OK) return st;
   if (p.kind == PK_NVFP4 && (st = do_prep(p, q, P, ws, stream, true)) != QS_OK) return st;
   if ((st = do_score(p, cache, q, scores, ws, stream, true)) != QS_OK) return st;

@@ -126,6 +126,7 @@ QS_DEV void row_prep(const uint16_t* q, const float* Pg, float* qt_row, float* q
 // Advance seq_lens once every CTA of the append grid has read them ("last CTA" pattern).
 QS_DEV void finish_append(const AppendParams& a) {
   __shared__ int s_last;
+  if (a.keep_lens) return;      // the decode step advances the lengths at its end
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -492,11 +493,11 @@ __global__ void __launch_bounds__(128) append_nvfp4_kernel(const AppendParams a)
 // rounding per product and per sum), bits b_i = [y_i > 0] packed 32 to a word by a warp
 // ballot (little-endian words, so bit i lands in byte i / 8 at position i % 8), and
 // g = fp32(sum_j o_j^2) / fp32(sum_i |y_i|) with both sums taken left to right (g = 0 when
-// the second is 0). CTA = one row x 16 tokens, thread i = dimension i (blockDim = D):
-// each R[g][j][i] is loaded once per CTA and applied to the 16 tokens.
-template <int D>
+// the second is 0). CTA = one row x TT tokens (16 for bulk appends, 1 for a decode step's
+// single token), thread i = dimension i (blockDim = D): each R[g][j][i] is loaded once per
+// CTA (16 loads in flight) and applied to the TT tokens.
+template <int D, int TT>
 __global__ void __launch_bounds__(D) append_rabitq_kernel(const AppendParams a) {
-  constexpr int TT = 16;
   constexpr int PB = kPage * (D / 8) + kPage * 4;      // bytes per (page, KV head)
   __shared__ float s_o[TT][D];
   __shared__ float s_ay[TT][D];
@@ -543,10 +544,14 @@ __global__ void __launch_bounds__(D) append_rabitq_kernel(const AppendParams a) 
     float acc[TT];
 #pragma unroll
     for (int n = 0; n < TT; ++n) acc[n] = 0.0f;
-    for (int j = 0; j < D; ++j) {
-      const float r = Rg[size_t(j) * D + tid];
+    for (int j0 = 0; j0 < D; j0 += 16) {             // 16 loads of R in flight at a time
+      float r[16];
 #pragma unroll
-      for (int n = 0; n < TT; ++n) acc[n] = __fadd_rn(acc[n], __fmul_rn(s_o[n][j], r));
+      for (int u = 0; u < 16; ++u) r[u] = __ldg(Rg + size_t(j0 + u) * D + tid);
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+#pragma unroll
+        for (int n = 0; n < TT; ++n) acc[n] = __fadd_rn(acc[n], __fmul_rn(s_o[n][j0 + u], r[u]));
     }
     uint8_t* base = static_cast<uint8_t*>(a.proxy);
 #pragma unroll
@@ -795,9 +800,15 @@ cudaError_t launch_append(const Plan& p, const AppendParams& a, cudaStream_t s) 
     return cudaGetLastError();
   }
   if (p.kind == PK_RABITQ) {
-    const dim3 grid((a.max_new + 15) / 16, a.batch * a.Hkv);
-    if (p.d == 128) append_rabitq_kernel<128><<<grid, 128, 0, s>>>(a);
-    else append_rabitq_kernel<64><<<grid, 64, 0, s>>>(a);
+    if (a.max_new == 1) {
+      const dim3 grid(1, a.batch * a.Hkv);
+      if (p.d == 128) append_rabitq_kernel<128, 1><<<grid, 128, 0, s>>>(a);
+      else append_rabitq_kernel<64, 1><<<grid, 64, 0, s>>>(a);
+    } else {
+      const dim3 grid((a.max_new + 15) / 16, a.batch * a.Hkv);
+      if (p.d == 128) append_rabitq_kernel<128, 16><<<grid, 128, 0, s>>>(a);
+      else append_rabitq_kernel<64, 16><<<grid, 64, 0, s>>>(a);
+    }
     return cudaGetLastError();
   }
   if (p.kind == PK_CENTROID) {

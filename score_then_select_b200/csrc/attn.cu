@@ -34,8 +34,10 @@
 //     online-softmax state (base 2, scale * log2 e folded into the logits). At the end of
 //     a chunk the four states are merged in a fixed order into the chunk's partial
 //     (max, sum, o).
-// attn_combine_kernel, launched behind this grid, merges each (row, query head)'s chunk
-// partials by log-sum-exp into the output.
+// Row merge, in the same kernel: the CTA that finishes a row's last chunk (counted on the
+// row's counter in the workspace) merges the row's chunk partials by log-sum-exp into the
+// output with its four consumer warps, while the other CTAs keep streaming. The last CTA
+// of the grid to finish resets the chunk-claim counter for the next launch.
 //
 // Tensor-core mapping and online softmax: attn_warp_tile (attn_core.cuh).
 #include <cuda.h>
@@ -55,6 +57,8 @@ constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kAttnThreads = kConsumerThreads + 32;
 constexpr int kHalfBytes = kTileT * 128;         // 64 rows x 64 elements (one swizzled box column)
 
+constexpr int kRecCap = 32;       // rows whose chunk counts a CTA holds before adding them
+
 template <int D>
 struct AttnSmem {
   static constexpr int kHalves = D / 64;
@@ -64,10 +68,11 @@ struct AttnSmem {
   static constexpr int kMetaOff = kAttnStages * kStageBytes;        // u32 [stages][4]
   static constexpr int kBarOff = kMetaOff + kAttnStages * 16;       // u64 full[], empty[], rag[]
   static constexpr int kMlOff = kBarOff + 3 * kAttnStages * 8;      // f32 [2][m [4][8], l [4][8]]
-  static constexpr int kMiscOff = kMlOff + 2 * 64 * 4;              // i32 abort, u64 barrier
+  static constexpr int kMiscOff = kMlOff + 2 * 64 * 4;              // i32 abort, i32 records, u64 barrier
   static constexpr int kScrOff = kMiscOff + 16;                     // merge buffer
   static constexpr int kBufStride = D + 4;                          // floats per head (merge)
-  static constexpr int kUsed = kScrOff + 2 * 8 * kBufStride * 4;
+  static constexpr int kRecOff = kScrOff + 2 * 8 * kBufStride * 4;   // i32 [kRecCap][row, chunks]
+  static constexpr int kUsed = kRecOff + kRecCap * 8;
   static constexpr int kTotal = kUsed + 1024;                       // + alignment slack
 };
 static_assert(AttnSmem<128>::kTotal + 1024 <= 228 * 1024 / kAttnCtasPerSm,
@@ -94,6 +99,12 @@ QS_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort) {
 // flag | phase parity of the stage's ragged-copy barrier.
 constexpr uint32_t kMetaFirst = 1u << 16, kMetaLast = 1u << 17;
 constexpr uint32_t kMetaRag = 1u << 18, kMetaRagPhase = 1u << 19;
+// NVFP4 key storage: the tile's K region holds NVFP4 codes, scales and the row's centre
+// (else BF16 keys); the tile covers page slots 64..127 (else 0..63)
+constexpr uint32_t kMetaRawK = 1u << 20, kMetaHalf = 1u << 21;
+// NVFP4 key storage: layout of the K region of a stage for a tile of NVFP4 keys
+constexpr int kRawCodes = 0, kRawScales = 4096, kRawMu = 5120;
+constexpr uint32_t kRawBytes = 4096 + 1024 + 512;
 
 // Barrier of the four consumer warps on an mbarrier (count 4), bounded like every wait
 // here: a warp that gives up cannot leave the others waiting on a hardware barrier.
@@ -105,258 +116,145 @@ QS_DEV void consumer_sync(uint64_t* bar, uint32_t& phase, int lane, volatile int
   __syncwarp();
 }
 
-template <int D, bool V_F16, bool AGG_F16>
-__global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
-    attn_kernel(const __grid_constant__ AttnParams a, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v) {
-  using SM = AttnSmem<D>;
-  constexpr int KS = D / 16;       // k-steps over the head dimension
-  constexpr int CH = D / 8;        // 16-byte chunks per row
-  constexpr int NS = kAttnStages;
-  extern __shared__ uint8_t smem_raw[];
-  // the swizzled boxes need 1024-byte aligned stages
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint32_t* meta = reinterpret_cast<uint32_t*>(smem + SM::kMetaOff);   // [stage][mask lo, hi, row, info]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
-  uint64_t* empty = full + NS;
-  uint64_t* rag = empty + NS;       // ragged-run copies of a stage (one cp.async arrival per lane)
-  float* s_ml = reinterpret_cast<float*>(smem + SM::kMlOff);         // [2][m [4][8], l [4][8]]
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::kMiscOff);
-  uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + SM::kMiscOff + 8);
-  float* s_buf = reinterpret_cast<float*>(smem + SM::kScrOff);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);                 // producer lane 0 (with the stage's byte count)
-      mbar_init(&empty[s], kConsumerWarps);
-      mbar_init(&rag[s], 32);
-      meta[4 * s + 2] = 0xffffffffu;          // an unfilled stage reads as the end marker
-    }
-    mbar_init(cbar, kConsumerWarps);
-    *s_abort = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  pdl_wait();      // the selection comes from the kernel before
-  pdl_trigger();   // the row merge may be scheduled now; it waits for this grid to finish
-
-  const int Hq = a.Hkv * a.G;
-  const int tpr = a.tiles_per_row, cpr = a.chunks_per_row, ktiles = a.chunk_tiles;
-  const int nchunks = a.rows * cpr;
-
-  if (warp == kConsumerWarps) {
-    // ======================= producer: chunk claims, run table, copies ================
-    // A run is hb = min(S, 64) consecutive slots of a tile: one selected block, or one half
-    // of a 128-slot block; lane u of a chunk's table holds run u (tile u / rpt, run u % rpt).
-    // Three stages a chunk apart: A loads the selection entry and the row's n_sel / length;
-    // B validates and loads the page-table entry; C yields the cache row of the run's first
-    // slot and its valid count (0: empty; hb: full; else a ragged last block).
-    const int hb = a.run_h, lg_hb = a.log2_run, rpt = kTileT >> lg_hb, lgS = a.log2_S;
-    uint32_t* next_ctr = a.hdr + kCtrAttnNext;
-    struct RunA { int row, sl, blk, n, L; };
-    struct RunB { int pg, t0, g, cnt, row; };
-    auto stage_a = [&](int c) {
-      RunA r{0, 0, -1, 0, 0};
-      if (c < nchunks) {
-        r.row = c / cpr;
-        const int tin0 = (c - r.row * cpr) * ktiles, j = lane >> (6 - lg_hb);
-        if (j < min(ktiles, tpr - tin0)) {
-          r.sl = (tin0 + j) * kTileT + ((lane & (rpt - 1)) << lg_hb);
-          r.L = a.row_lens ? a.row_lens[r.row] : a.seq_lens[r.row / a.Hkv];
-          const int e = r.sl >> lgS;
-          if (a.sel) {
-            r.n = a.n_sel[r.row];
-            if (e < a.budget) r.blk = a.sel[size_t(r.row) * a.budget + e];
-          } else {                                         // full KV: every block, in order
-            r.n = int((static_cast<long long>(r.L) + (1 << lgS) - 1) >> lgS);
-            r.blk = e;
-          }
-        } else {
-          r.n = -2;                                        // no such run in this chunk
-        }
+// Merge row `row`'s chunk partials into the output (the four consumer warps, thread ct):
+//   out[h][d] = sum_p 2^(m_p - M) o_p[d] / sum_p 2^(m_p - M) l_p, M = max_p m_p over
+//   partials with l_p > 0 (a row with no tokens -> 0); p in order, so the result is fixed.
+// Warp w first turns head w's (and w + 4's) chunk maxima and sums into weights and 1/den in
+// shared memory (w_buf, G x cpr + G floats); then each thread forms its outputs with all of
+// a head's partial loads in flight at once. Rows with more partials than w_buf holds take
+// the same sums in batches of 8 partials with a running maximum.
+template <int D>
+QS_DEV void attn_merge_row(const AttnParams& a, int row, int ct, float* w_buf, int w_cap,
+                           uint32_t& cphase, uint64_t* cbar, volatile int* s_abort) {
+  const int cpr = a.chunks_per_row, lane = ct & 31, warp = ct >> 5;
+  const size_t rq0 = size_t(row / a.Hkv) * (a.Hkv * a.G) + (row % a.Hkv) * a.G;
+  auto store = [&](size_t rq, int d, float r) {
+    if (a.out_bf16)
+      reinterpret_cast<uint16_t*>(a.out)[rq * D + d] = f32_to_bf16_rn(r);
+    else
+      reinterpret_cast<float*>(a.out)[rq * D + d] = r;
+  };
+  if (a.G * cpr + a.G <= w_cap) {
+    float* inv = w_buf + a.G * cpr;
+    for (int h = warp; h < a.G; h += kConsumerWarps) {
+      const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + (rq0 + h) * cpr;
+      float M = -INFINITY;
+      for (int p = lane; p < cpr; p += 32) {
+        const float2 v = __ldcg(ml + p);
+        if (v.y > 0.0f) M = fmaxf(M, v.x);
       }
-      return r;
-    };
-    auto stage_b = [&](int c, const RunA& x) {
-      RunB r{-1, 0, 0, 0, x.row};
-      if (c >= nchunks || x.n == -2) return r;
-      const int b = x.row / a.Hkv;
-      r.g = x.row - b * a.Hkv;
-      if (x.n < 0 || x.n > a.budget || x.L < 0) {
-        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
-        return r;
-      }
-      if (x.sl >= (x.n << lgS)) return r;                  // beyond the row's selection
-      const int nbr = (x.L + (1 << lgS) - 1) >> lgS;
-      if (x.blk < 0 || x.blk >= nbr) {
-        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
-        return r;
-      }
-      r.t0 = (x.blk << lgS) + (x.sl & ((1 << lgS) - 1));
-      if (r.t0 >= x.L) return r;                           // ragged tail of the last block
-      r.cnt = min(hb, x.L - r.t0);
-      const int pi = r.t0 >> 7;                            // kPage = 128
-      r.pg = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
-      return r;                                            // pg is checked once it has landed
-    };
-    auto stage_c = [&](const RunB& x, int& y, int& cnt) {
-      cnt = x.cnt;
-      y = -1;
-      if (cnt == 0) return;
-      if (x.pg < 0 || x.pg >= a.num_pages) {
-        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
-        cnt = 0;
-        return;
-      }
-      y = (x.pg * a.Hkv + x.g) * kPage + (x.t0 & (kPage - 1));
-    };
-
-    // chunks: the first two of each CTA are fixed (blockIdx, blockIdx + C), the rest are
-    // claimed from the counter (value + 2C), two claims in flight, each used two chunks
-    // after it is issued (an atomic on the shared counter is slow under full HBM load)
-    const unsigned C2 = 2u * gridDim.x;
-    unsigned pend_a = 0, pend_b = 0;
-    if (lane == 0) {
-      pend_a = atomicAdd(next_ctr, 1u) + C2;
-      pend_b = atomicAdd(next_ctr, 1u) + C2;
-    }
-    int c_cur = int(min(blockIdx.x, unsigned(nchunks)));
-    int c_n1 = int(min(blockIdx.x + gridDim.x, unsigned(nchunks)));
-    RunA pa = stage_a(c_n1);
-    RunB pb = stage_b(c_cur, stage_a(c_cur));
-
-    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k);
-    const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v);
-    int t = 0;                                             // stages filled so far
-    int kseq = 0;                                          // chunks started by this CTA
-    uint32_t rag_uses = 0;                                 // bit s: parity of stage s's ragged uses
-    bool ok = true;
-    while (ok && c_cur < nchunks) {
-      int run_y, run_cnt;
-      stage_c(pb, run_y, run_cnt);
-      pb = stage_b(c_n1, pa);
-      // the two pending claims alternate by chunk parity: neither register is touched
-      // until two chunks after its atomic was issued
-      int c_n2;
-      if ((kseq & 1) == 0) {
-        c_n2 = int(min(__shfl_sync(kFull, pend_a, 0), unsigned(nchunks)));
-        if (lane == 0) pend_a = c_n2 < nchunks ? atomicAdd(next_ctr, 1u) + C2 : unsigned(nchunks);
-      } else {
-        c_n2 = int(min(__shfl_sync(kFull, pend_b, 0), unsigned(nchunks)));
-        if (lane == 0) pend_b = c_n2 < nchunks ? atomicAdd(next_ctr, 1u) + C2 : unsigned(nchunks);
-      }
-      ++kseq;
-      pa = stage_a(c_n2);
-
-      const int row = c_cur / cpr, ci = c_cur - row * cpr;
-      const int nt = min(ktiles, tpr - ci * ktiles);
-      const int b = row / a.Hkv, g = row - b * a.Hkv;
-      // per-tile summary, lane j for tile j of the chunk: valid-slot mask, box bytes,
-      // whether a ragged run needs the 16-byte copy path
-      uint32_t t_lo = 0, t_hi = 0, t_bytes = 0, t_rag = 0;
-      for (int r = 0; r < rpt; ++r) {
-        const int cr = __shfl_sync(kFull, run_cnt, ((lane << (6 - lg_hb)) + r) & 31);
-        if (cr > 0) {
-          const unsigned long long m = (cr >= 64 ? ~0ull : ((1ull << cr) - 1)) << (r << lg_hb);
-          t_lo |= uint32_t(m);
-          t_hi |= uint32_t(m >> 32);
-        }
-        if (cr == 0 || cr == hb) t_bytes += uint32_t(2 * SM::kHalves * hb * 128);
-        else t_rag = 1;
-      }
-      const uint32_t q_bytes = uint32_t(a.G * D * 2);
-      const uint16_t* qrow = a.q + (size_t(b) * Hq + g * a.G) * D;
-      // box copy owned by this lane: run lane / (2 halves), column half, K or V
-      const int box_r = lane / (2 * SM::kHalves), box_h = (lane >> 1) % SM::kHalves, box_v = lane & 1;
-      const bool box_lane = lane < rpt * SM::kHalves * 2;
-      for (int j = 0; j < nt; ++j, ++t) {
-        const int s = t % NS;
-        bool got = true;
-        if (lane == 0 && t >= NS) got = wait_or_abort(&empty[s], ((t / NS) - 1) & 1, s_abort);
-        ok = __shfl_sync(kFull, got, 0);
-        __syncwarp();
-        if (!ok) break;
-
-        uint8_t* st = smem + s * SM::kStageBytes;
-        const uint32_t lo = __shfl_sync(kFull, t_lo, j), hi = __shfl_sync(kFull, t_hi, j);
-        const uint32_t bytes = __shfl_sync(kFull, t_bytes, j) + (j == 0 ? q_bytes : 0u);
-        const bool ragged = __shfl_sync(kFull, t_rag, j) != 0;
-        uint32_t rag_bits = 0;
-        if (ragged) {
-          // a ragged run: 16-byte copies of its valid rows, zeros for the rest, counted on
-          // the stage's ragged-copy barrier (its phase parity travels in the metadata)
-          rag_bits = kMetaRag | ((rag_uses >> s) & 1u ? kMetaRagPhase : 0u);
-          rag_uses ^= 1u << s;
-          for (int r = 0; r < rpt; ++r) {
-            const int src = (j << (6 - lg_hb)) + r;
-            const int cr = __shfl_sync(kFull, run_cnt, src), y0 = __shfl_sync(kFull, run_y, src);
-            if (cr == 0 || cr == hb) continue;
-            for (int i = lane; i < hb; i += 32) {
-              const int rt = (r << lg_hb) + i;
-              const bool v = i < cr;
-              const size_t off = size_t(v ? y0 + i : 0) * (D * 2);
 #pragma unroll
-              for (int ch = 0; ch < CH; ++ch) {
-                cp_async16_zfill(st + swz(rt, ch), kbase + off + ch * 16, v);
-                cp_async16_zfill(st + SM::kTileBytes + swz(rt, ch), vbase + off + ch * 16, v);
-              }
-            }
-          }
-          cp_async_mbar_arrive_noinc(&rag[s]);
-        }
-        if (lane == 0) {
-          meta[4 * s] = lo;
-          meta[4 * s + 1] = hi;
-          meta[4 * s + 2] = uint32_t(row);
-          meta[4 * s + 3] = uint32_t(ci) | (j == 0 ? kMetaFirst : 0u) | (j + 1 == nt ? kMetaLast : 0u) |
-                            rag_bits;
-          mbar_arrive_expect_tx(&full[s], bytes);
-        }
-        __syncwarp();                                      // the byte count is posted first
-        // full and empty runs: one box copy per lane (an empty run reads zeros from outside
-        // the tensor); a chunk's first tile also brings the row's queries
-        {
-          const int src = ((j << (6 - lg_hb)) + box_r) & 31;
-          const int ry = __shfl_sync(kFull, run_y, src), rc = __shfl_sync(kFull, run_cnt, src);
-          if (box_lane && (rc == 0 || rc == hb)) {
-            const uint32_t off = (box_v ? SM::kTileBytes : 0) + box_h * kHalfBytes + ((box_r << lg_hb) << 7);
-            tma_load_2d(st + off, box_v ? static_cast<const void*>(&tm_v) : static_cast<const void*>(&tm_k),
-                        64 * box_h, rc ? ry : -hb, &full[s]);
-          }
-        }
-        if (j == 0 && lane == 0) bulk_g2s(st + 2 * SM::kTileBytes, qrow, q_bytes, &full[s]);
+      for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
+      float den = 0.0f;
+      for (int p = lane; p < cpr; p += 32) {
+        const float2 v = __ldcg(ml + p);
+        const float w = v.y > 0.0f ? ex2(v.x - M) : 0.0f;
+        w_buf[h * cpr + p] = w;
+        den += w * v.y;
       }
-      c_cur = c_n1;
-      c_n1 = c_n2;
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(kFull, den, o2);
+      if (lane == 0) inv[h] = den > 0.0f ? 1.0f / den : 0.0f;
     }
-    // end marker: one more stage whose row is -1
-    if (ok) {
-      const int s = t % NS;
-      bool got = true;
-      if (lane == 0 && t >= NS) got = wait_or_abort(&empty[s], ((t / NS) - 1) & 1, s_abort);
-      ok = __shfl_sync(kFull, got, 0);
-      __syncwarp();
-      if (ok) {
-        if (lane == 0) {
-          meta[4 * s + 2] = 0xffffffffu;
-          mbar_arrive_expect_tx(&full[s], 0u);
-        }
-        ++t;
+    consumer_sync(cbar, cphase, lane, s_abort);
+    for (int idx = ct; idx < a.G * D; idx += kConsumerThreads) {
+      const int h = idx / D, d = idx - h * D;
+      const size_t rq = rq0 + h;
+      const float* po = a.part_o + rq * cpr * D + d;
+      const float* wh = w_buf + h * cpr;
+      float num = 0.0f;
+      int p = 0;
+      for (; p + 16 <= cpr; p += 16) {
+        float x[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) x[u] = __ldcg(po + size_t(p + u) * D);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) num += wh[p + u] * x[u];
       }
+      for (; p < cpr; ++p) num += wh[p] * __ldcg(po + size_t(p) * D);
+      store(rq, d, num * inv[h]);
     }
-    // every copy issued must land before the CTA exits
-    cp_async_commit();
-    cp_async_wait<0>();
-    if (lane == 0) {
-      for (int j = t > NS ? t - NS : 0; j < t; ++j)
-        if (!mbar_wait(&full[j % NS], (j / NS) & 1)) *s_abort = 1;
-    }
-    __syncwarp();
+    consumer_sync(cbar, cphase, lane, s_abort);          // w_buf is free again
     return;
   }
+  for (int idx = ct; idx < a.G * D; idx += kConsumerThreads) {
+    const int h = idx / D, d = idx - h * D;
+    const size_t rq = rq0 + h;
+    const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + rq * cpr;
+    const float* po = a.part_o + rq * cpr * D + d;
+    float M = -INFINITY, den = 0.0f, num = 0.0f;
+    for (int p0 = 0; p0 < cpr; p0 += 8) {
+      float2 v[8];
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool in = p0 + u < cpr;
+        v[u] = in ? __ldcg(ml + p0 + u) : make_float2(-INFINITY, 0.0f);
+        x[u] = in ? __ldcg(po + size_t(p0 + u) * D) : 0.0f;
+      }
+      float Mb = M;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v[u].y > 0.0f) Mb = fmaxf(Mb, v[u].x);
+      if (Mb > M) {
+        const float f = M == -INFINITY ? 0.0f : ex2(M - Mb);
+        den *= f;
+        num *= f;
+        M = Mb;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = v[u].y > 0.0f ? ex2(v[u].x - M) : 0.0f;
+        den += w * v[u].y;
+        num += w * x[u];
+      }
+    }
+    store(rq, d, den > 0.0f ? num * (1.0f / den) : 0.0f);
+  }
+}
 
-  // ======================= consumers: online softmax, chunk partials, row merge ==========
+// Add this CTA's recorded chunk counts to the rows' counters (the four consumer warps; one
+// fence first, so the chunk partials are visible before any count); a row whose count
+// reaches chunks_per_row is complete and this CTA merges it, then clears its counter.
+template <int D>
+QS_DEV void attn_count_rows(const AttnParams& a, int ct, volatile int* s_nrec, int* s_rec,
+                            float* s_buf, uint32_t& cphase, uint64_t* cbar, volatile int* s_abort) {
+  using SM = AttnSmem<D>;
+  const int lane = ct & 31;
+  __threadfence();
+  consumer_sync(cbar, cphase, lane, s_abort);
+  const int n = *s_nrec;
+  if (ct == 0) {
+    for (int i = 0; i < n; ++i) {
+      const unsigned c = unsigned(s_rec[2 * i + 1]);
+      const unsigned prev = atomicAdd(a.row_ctr + s_rec[2 * i], c);
+      s_rec[2 * i + 1] = prev + c == unsigned(a.chunks_per_row) ? 1 : 0;
+    }
+  }
+  consumer_sync(cbar, cphase, lane, s_abort);
+  for (int i = 0; i < n; ++i) {
+    if (!s_rec[2 * i + 1] || *s_abort) continue;
+    const int row = s_rec[2 * i];
+    __threadfence();
+    attn_merge_row<D>(a, row, ct, s_buf, 2 * 8 * SM::kBufStride, cphase, cbar, s_abort);
+    if (ct == 0) a.row_ctr[row] = 0u;                      // ready for the next launch
+  }
+  consumer_sync(cbar, cphase, lane, s_abort);
+  if (ct == 0) *s_nrec = 0;
+}
+
+// ======================= consumers: online softmax, chunk partials, row merge ==========
+template <int D, bool V_F16, bool AGG_F16, bool KQ4>
+QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uint64_t* full,
+                         uint64_t* empty, uint64_t* rag, float* s_ml, volatile int* s_abort,
+                         volatile int* s_nrec, int* s_rec, uint64_t* cbar, float* s_buf) {
+  using SM = AttnSmem<D>;
+  constexpr int KS = D / 16;
+  constexpr int NS = kAttnStages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Hq = a.Hkv * a.G;
+  const int cpr = a.chunks_per_row;
+  const float gk = KQ4 ? *a.key_gscale : 0.0f;            // NVFP4 key tensor scale
   uint32_t cphase = 0, mpar = 0;
   const int h0 = 2 * (lane & 3);                           // this lane's heads h0, h0 + 1
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
@@ -392,9 +290,18 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
 
     const int tl = warp * 16 + (lane >> 2);       // tokens tl and tl + 8 (same 32-slot word)
     const uint32_t vm = warp < 2 ? lo : hi;
-    attn_warp_tile<D, V_F16, AGG_F16>(kst, vst, qb, (vm >> (tl & 31)) & 1u,
-                                      (vm >> ((tl + 8) & 31)) & 1u, a.scale_log2, m0, m1, l0, l1,
-                                      o, warp, lane, [](int r, int c) { return swz(r, c); });
+    const bool v0 = (vm >> (tl & 31)) & 1u, v1 = (vm >> ((tl + 8) & 31)) & 1u;
+    const auto sw = [](int r, int c) { return swz(r, c); };
+    if (KQ4 && (info & kMetaRawK)) {
+      const KFragNvfp4 kf(st + kRawCodes, st + kRawScales,
+                          reinterpret_cast<const float*>(st + kRawMu), gk,
+                          (info & kMetaHalf) ? 64 : 0, warp, lane);
+      attn_warp_tile<D, V_F16, AGG_F16>(kf, vst, qb, v0, v1, a.scale_log2, m0, m1, l0, l1, o,
+                                        warp, lane, sw);
+    } else {
+      attn_warp_tile<D, V_F16, AGG_F16>(KFragLdsm<decltype(sw)>{kst, warp, lane, sw}, vst, qb, v0,
+                                        v1, a.scale_log2, m0, m1, l0, l1, o, warp, lane, sw);
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);        // this warp is done with the stage
     if (!(info & kMetaLast)) continue;
@@ -494,64 +401,334 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
           }
         }
       }
+      // the chunk's partial is out: record its row (the count is added to the row's counter
+      // once this CTA's work is done, behind one fence, off the streaming path)
+      if (lane == 0) {
+        const int n = *s_nrec;
+        if (n > 0 && s_rec[2 * (n - 1)] == row) {
+          s_rec[2 * (n - 1) + 1] += 1;
+        } else {
+          s_rec[2 * n] = row;
+          s_rec[2 * n + 1] = 1;
+          *s_nrec = n + 1;
+        }
+      }
     }
+    consumer_sync(cbar, cphase, lane, s_abort);
+    if (*s_nrec == kRecCap && !*s_abort)                   // the record is full: add it now
+      attn_count_rows<D>(a, tid, s_nrec, s_rec, s_buf, cphase, cbar, s_abort);
   }
-  if (tid == 0 && *s_abort) flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_ATTN, blockIdx.x);
+  if (*s_nrec > 0 && !*s_abort)
+    attn_count_rows<D>(a, tid, s_nrec, s_rec, s_buf, cphase, cbar, s_abort);
 }
 
-// ---------------------------------------------------------------- combine
-// One CTA per (row, query head): the head's chunk partials -> output by log-sum-exp,
-//   out[d] = sum_p 2^(m_p - M) o_p[d] / sum_p 2^(m_p - M) l_p  (a row with no tokens -> 0).
-// Thread d owns output element d; all of its partial loads are in flight together.
-// Waits for the attention grid (programmatic dependent launch), then resets the chunk
-// claim counter for the next attention launch.
-template <int D>
-__global__ void __launch_bounds__(D) attn_combine_kernel(const AttnParams a) {
-  extern __shared__ float s_w[];                           // [cpr] weights, then 1/den
-  pdl_wait();
-  const int row = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
-  const int cpr = a.chunks_per_row;
-  if (row == 0 && h == 0 && tid == 0) a.hdr[kCtrAttnNext] = 0u;
-  const size_t rq = size_t(row / a.Hkv) * (a.Hkv * a.G) + (row % a.Hkv) * a.G + h;
-  const float* ml = a.part_ml + rq * cpr * 2;
-  if (tid < 32) {
-    float M = -INFINITY;
-    for (int p = lane; p < cpr; p += 32) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(ml) + p);
-      if (v.y > 0.0f) M = fmaxf(M, v.x);
+template <int D, bool V_F16, bool AGG_F16, bool KQ4>
+__global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
+    attn_kernel(const __grid_constant__ AttnParams a, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v) {
+  using SM = AttnSmem<D>;
+  constexpr int CH = D / 8;        // 16-byte chunks per row
+  constexpr int NS = kAttnStages;
+  extern __shared__ uint8_t smem_raw[];
+  // the swizzled boxes need 1024-byte aligned stages
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint32_t* meta = reinterpret_cast<uint32_t*>(smem + SM::kMetaOff);   // [stage][mask lo, hi, row, info]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
+  uint64_t* empty = full + NS;
+  uint64_t* rag = empty + NS;       // ragged-run copies of a stage (one cp.async arrival per lane)
+  float* s_ml = reinterpret_cast<float*>(smem + SM::kMlOff);         // [2][m [4][8], l [4][8]]
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::kMiscOff);
+  volatile int* s_nrec = reinterpret_cast<volatile int*>(smem + SM::kMiscOff + 4);
+  int* s_rec = reinterpret_cast<int*>(smem + SM::kRecOff);
+  uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + SM::kMiscOff + 8);
+  float* s_buf = reinterpret_cast<float*>(smem + SM::kScrOff);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);                 // producer lane 0 (with the stage's byte count)
+      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&rag[s], 32);
+      meta[4 * s + 2] = 0xffffffffu;          // an unfilled stage reads as the end marker
     }
-#pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
-    float den = 0.0f;
-    for (int p = lane; p < cpr; p += 32) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(ml) + p);
-      const float w = v.y > 0.0f ? ex2(v.x - M) : 0.0f;
-      s_w[p] = w;
-      den += w * v.y;
-    }
-#pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(kFull, den, o2);
-    if (lane == 0) s_w[cpr] = den > 0.0f ? 1.0f / den : 0.0f;
+    mbar_init(cbar, kConsumerWarps);
+    *s_abort = 0;
+    *s_nrec = 0;
+    fence_mbar_init();
   }
   __syncthreads();
-  const float* po = a.part_o + rq * cpr * D + tid;
-  float acc = 0.0f;
-  int p = 0;
-  for (; p + 8 <= cpr; p += 8) {
-    float v[8];
+  pdl_wait();      // the selection comes from the kernel before
+  pdl_trigger();   // the next kernel may be scheduled now; it waits for this grid to finish
+
+  const int Hq = a.Hkv * a.G;
+  const int tpr = a.tiles_per_row, cpr = a.chunks_per_row, ktiles = a.chunk_tiles;
+  const int nchunks = a.rows * cpr;
+
+  if (warp == kConsumerWarps) {
+    // ======================= producer: chunk claims, run table, copies ================
+    // A run is hb = min(S, 64) consecutive slots of a tile: one selected block, or one half
+    // of a 128-slot block; lane u of a chunk's table holds run u (tile u / rpt, run u % rpt).
+    // Three stages a chunk apart: A loads the selection entry and the row's n_sel / length;
+    // B validates and loads the page-table entry; C yields the cache row of the run's first
+    // slot and its valid count (0: empty; hb: full; else a ragged last block).
+    const int hb = a.run_h, lg_hb = a.log2_run, rpt = kTileT >> lg_hb, lgS = a.log2_S;
+    uint32_t* next_ctr = a.hdr + kCtrAttnNext;
+    struct RunA { int row, sl, blk, n, L, k0, k1; };
+    struct RunB { int pg, t0, g, cnt, row, raw; };
+    auto stage_a = [&](int c) {
+      RunA r{0, 0, -1, 0, 0, -1, -1};
+      if (c < nchunks) {
+        r.row = c / cpr;
+        const int tin0 = (c - r.row * cpr) * ktiles, j = lane >> (6 - lg_hb);
+        if (j < min(ktiles, tpr - tin0)) {
+          r.sl = (tin0 + j) * kTileT + ((lane & (rpt - 1)) << lg_hb);
+          r.L = a.row_lens ? a.row_lens[r.row] : a.seq_lens[r.row / a.Hkv] + a.len_add;
+          const int e = r.sl >> lgS;
+          if constexpr (KQ4) {                             // the row's kept (BF16) blocks
+            r.k0 = a.kept[2 * r.row];
+            r.k1 = a.kept[2 * r.row + 1];
+          }
+          if (a.sel) {
+            r.n = a.n_sel[r.row];
+            if (e < a.budget) r.blk = a.sel[size_t(r.row) * a.budget + e];
+          } else {                                         // full KV: every block, in order
+            r.n = int((static_cast<long long>(r.L) + (1 << lgS) - 1) >> lgS);
+            r.blk = e;
+          }
+        } else {
+          r.n = -2;                                        // no such run in this chunk
+        }
+      }
+      return r;
+    };
+    auto stage_b = [&](int c, const RunA& x) {
+      RunB r{-1, 0, 0, 0, x.row, 0};
+      if (c >= nchunks || x.n == -2) return r;
+      const int b = x.row / a.Hkv;
+      r.g = x.row - b * a.Hkv;
+      if (x.n < 0 || x.n > a.budget || x.L < 0) {
+        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
+        return r;
+      }
+      if (x.sl >= (x.n << lgS)) return r;                  // beyond the row's selection
+      const int nbr = (x.L + (1 << lgS) - 1) >> lgS;
+      if (x.blk < 0 || x.blk >= nbr) {
+        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
+        return r;
+      }
+      r.t0 = (x.blk << lgS) + (x.sl & ((1 << lgS) - 1));
+      if (r.t0 >= x.L) return r;                           // ragged tail of the last block
+      r.cnt = min(hb, x.L - r.t0);
+      r.raw = KQ4 && x.blk != x.k0 && x.blk != x.k1;       // keys from the NVFP4 cache
+      const int pi = r.t0 >> 7;                            // kPage = 128
+      r.pg = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
+      return r;                                            // pg is checked once it has landed
+    };
+    auto stage_c = [&](const RunB& x, int& y, int& cnt, int& raw) {
+      cnt = x.cnt;
+      y = -1;
+      raw = 0;
+      if (cnt == 0) return;
+      if (x.pg < 0 || x.pg >= a.num_pages) {
+        flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(x.row));
+        cnt = 0;
+        return;
+      }
+      y = (x.pg * a.Hkv + x.g) * kPage + (x.t0 & (kPage - 1));
+      raw = x.raw;
+    };
+
+    // chunks: the first two of each CTA are fixed (blockIdx, blockIdx + C), the rest are
+    // claimed from the counter (value + 2C), two claims in flight, each used two chunks
+    // after it is issued (an atomic on the shared counter is slow under full HBM load)
+    const unsigned C2 = 2u * gridDim.x;
+    unsigned pend_a = 0, pend_b = 0;
+    if (lane == 0) {
+      pend_a = atomicAdd(next_ctr, 1u) + C2;
+      pend_b = atomicAdd(next_ctr, 1u) + C2;
+    }
+    int c_cur = int(min(blockIdx.x, unsigned(nchunks)));
+    int c_n1 = int(min(blockIdx.x + gridDim.x, unsigned(nchunks)));
+    RunA pa = stage_a(c_n1);
+    RunB pb = stage_b(c_cur, stage_a(c_cur));
+
+    const uint8_t* kbase = reinterpret_cast<const uint8_t*>(a.k);
+    const uint8_t* vbase = reinterpret_cast<const uint8_t*>(a.v);
+    int t = 0;                                             // stages filled so far
+    int kseq = 0;                                          // chunks started by this CTA
+    uint32_t rag_uses = 0;                                 // bit s: parity of stage s's ragged uses
+    bool ok = true;
+    while (ok && c_cur < nchunks) {
+      int run_y, run_cnt, run_raw;
+      stage_c(pb, run_y, run_cnt, run_raw);
+      pb = stage_b(c_n1, pa);
+      // the two pending claims alternate by chunk parity: neither register is touched
+      // until two chunks after its atomic was issued
+      int c_n2;
+      if ((kseq & 1) == 0) {
+        c_n2 = int(min(__shfl_sync(kFull, pend_a, 0), unsigned(nchunks)));
+        if (lane == 0) pend_a = c_n2 < nchunks ? atomicAdd(next_ctr, 1u) + C2 : unsigned(nchunks);
+      } else {
+        c_n2 = int(min(__shfl_sync(kFull, pend_b, 0), unsigned(nchunks)));
+        if (lane == 0) pend_b = c_n2 < nchunks ? atomicAdd(next_ctr, 1u) + C2 : unsigned(nchunks);
+      }
+      ++kseq;
+      pa = stage_a(c_n2);
+
+      const int row = c_cur / cpr, ci = c_cur - row * cpr;
+      const int nt = min(ktiles, tpr - ci * ktiles);
+      const int b = row / a.Hkv, g = row - b * a.Hkv;
+      // per-tile summary, lane j for tile j of the chunk: valid-slot mask, box bytes,
+      // whether a ragged run needs the 16-byte copy path
+      uint32_t t_lo = 0, t_hi = 0, t_bytes = 0, t_rag = 0;
+      for (int r = 0; r < rpt; ++r) {
+        const int cr = __shfl_sync(kFull, run_cnt, ((lane << (6 - lg_hb)) + r) & 31);
+        if (cr > 0) {
+          const unsigned long long m = (cr >= 64 ? ~0ull : ((1ull << cr) - 1)) << (r << lg_hb);
+          t_lo |= uint32_t(m);
+          t_hi |= uint32_t(m >> 32);
+        }
+        const int rr = __shfl_sync(kFull, run_raw, ((lane << (6 - lg_hb)) + r) & 31);
+        // NVFP4 keys (rr): the K box is replaced by the tile's codes, scales and centre
+        if (cr == 0 || cr == hb)
+          t_bytes += rr ? uint32_t(SM::kHalves * hb * 128) + kRawBytes
+                        : uint32_t(2 * SM::kHalves * hb * 128);
+        else {
+          t_rag = 1;
+          if (rr) t_bytes += kRawBytes;
+        }
+      }
+      const uint32_t q_bytes = uint32_t(a.G * D * 2);
+      const uint16_t* qrow = a.q + (size_t(b) * Hq + g * a.G) * D;
+      // box copy owned by this lane: run lane / (2 halves), column half, K or V
+      const int box_r = lane / (2 * SM::kHalves), box_h = (lane >> 1) % SM::kHalves, box_v = lane & 1;
+      const bool box_lane = lane < rpt * SM::kHalves * 2;
+      for (int j = 0; j < nt; ++j, ++t) {
+        const int s = t % NS;
+        bool got = true;
+        if (lane == 0 && t >= NS) got = wait_or_abort(&empty[s], ((t / NS) - 1) & 1, s_abort);
+        ok = __shfl_sync(kFull, got, 0);
+        __syncwarp();
+        if (!ok) break;
+
+        uint8_t* st = smem + s * SM::kStageBytes;
+        const uint32_t lo = __shfl_sync(kFull, t_lo, j), hi = __shfl_sync(kFull, t_hi, j);
+        const uint32_t bytes = __shfl_sync(kFull, t_bytes, j) + (j == 0 ? q_bytes : 0u);
+        const bool ragged = __shfl_sync(kFull, t_rag, j) != 0;
+        uint32_t rag_bits = 0;
+        if (ragged) {
+          // a ragged run: 16-byte copies of its valid rows, zeros for the rest, counted on
+          // the stage's ragged-copy barrier (its phase parity travels in the metadata)
+          rag_bits = kMetaRag | ((rag_uses >> s) & 1u ? kMetaRagPhase : 0u);
+          rag_uses ^= 1u << s;
+          for (int r = 0; r < rpt; ++r) {
+            const int src = (j << (6 - lg_hb)) + r;
+            const int cr = __shfl_sync(kFull, run_cnt, src), y0 = __shfl_sync(kFull, run_y, src);
+            const int rr = __shfl_sync(kFull, run_raw, src);
+            if (cr == 0 || cr == hb) continue;
+            for (int i = lane; i < hb; i += 32) {
+              const int rt = (r << lg_hb) + i;
+              const bool v = i < cr;
+              const size_t off = size_t(v ? y0 + i : 0) * (D * 2);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = __ldcg(po + size_t(p + u) * D);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) acc += s_w[p + u] * v[u];
+              for (int ch = 0; ch < CH; ++ch) {
+                if (!rr) cp_async16_zfill(st + swz(rt, ch), kbase + off + ch * 16, v);
+                cp_async16_zfill(st + SM::kTileBytes + swz(rt, ch), vbase + off + ch * 16, v);
+              }
+            }
+          }
+          cp_async_mbar_arrive_noinc(&rag[s]);
+        }
+        uint32_t kq4_bits = 0;
+        if constexpr (KQ4) {                               // one run per tile (S = 128)
+          const int src = (j << (6 - lg_hb)) & 31;
+          const int yr = __shfl_sync(kFull, run_y, src), rr = __shfl_sync(kFull, run_raw, src);
+          if (rr) kq4_bits = kMetaRawK | ((yr & 64) ? kMetaHalf : 0u);
+        }
+        if (lane == 0) {
+          meta[4 * s] = lo;
+          meta[4 * s + 1] = hi;
+          meta[4 * s + 2] = uint32_t(row);
+          meta[4 * s + 3] = uint32_t(ci) | (j == 0 ? kMetaFirst : 0u) | (j + 1 == nt ? kMetaLast : 0u) |
+                            rag_bits | kq4_bits;
+          mbar_arrive_expect_tx(&full[s], bytes);
+        }
+        __syncwarp();                                      // the byte count is posted first
+        // full and empty runs: one box copy per lane (an empty run reads zeros from outside
+        // the tensor); a chunk's first tile also brings the row's queries
+        {
+          const int src = ((j << (6 - lg_hb)) + box_r) & 31;
+          const int ry = __shfl_sync(kFull, run_y, src), rc = __shfl_sync(kFull, run_cnt, src);
+          const int rr = __shfl_sync(kFull, run_raw, src);
+          if (box_lane && (rc == 0 || rc == hb) && !(rr && box_v == 0)) {
+            const uint32_t off = (box_v ? SM::kTileBytes : 0) + box_h * kHalfBytes + ((box_r << lg_hb) << 7);
+            tma_load_2d(st + off, box_v ? static_cast<const void*>(&tm_v) : static_cast<const void*>(&tm_k),
+                        64 * box_h, rc ? ry : -hb, &full[s]);
+          }
+          if constexpr (KQ4) {
+            // NVFP4 keys, by the two K lanes: the tile's 64 token rows of each of the 4 code
+            // chunks (1 KB each), the page's 1 KB of scales and the row's centre
+            if (rr && box_lane && box_v == 0) {
+              const size_t ph = size_t(ry >> 7);             // page * Hkv + head
+              const uint8_t* cb = a.k_codes + ph * kNvfp4PageCodeBytes + (ry & 127) * 16;
+              const int c0 = 2 * box_h;
+              bulk_g2s(st + kRawCodes + c0 * 1024, cb + c0 * 2048, 1024u, &full[s]);
+              bulk_g2s(st + kRawCodes + (c0 + 1) * 1024, cb + (c0 + 1) * 2048, 1024u, &full[s]);
+              if (box_h == 0)
+                bulk_g2s(st + kRawScales, a.k_scales + ph * kNvfp4PageScaleBytes, 1024u, &full[s]);
+              else
+                bulk_g2s(st + kRawMu, a.key_center + size_t(row) * D, uint32_t(D * 4), &full[s]);
+            }
+          }
+        }
+        if (j == 0 && lane == 0) bulk_g2s(st + 2 * SM::kTileBytes, qrow, q_bytes, &full[s]);
+      }
+      c_cur = c_n1;
+      c_n1 = c_n2;
+    }
+    // end marker: one more stage whose row is -1
+    if (ok) {
+      const int s = t % NS;
+      bool got = true;
+      if (lane == 0 && t >= NS) got = wait_or_abort(&empty[s], ((t / NS) - 1) & 1, s_abort);
+      ok = __shfl_sync(kFull, got, 0);
+      __syncwarp();
+      if (ok) {
+        if (lane == 0) {
+          meta[4 * s + 2] = 0xffffffffu;
+          mbar_arrive_expect_tx(&full[s], 0u);
+        }
+        ++t;
+      }
+    }
+    // every copy issued must land before the CTA exits
+    cp_async_commit();
+    cp_async_wait<0>();
+    if (lane == 0) {
+      for (int j = t > NS ? t - NS : 0; j < t; ++j)
+        if (!mbar_wait(&full[j % NS], (j / NS) & 1)) *s_abort = 1;
+    }
+    __syncwarp();
+  } else {
+    attn_consume<D, V_F16, AGG_F16, KQ4>(a, smem, meta, full, empty, rag, s_ml, s_abort, s_nrec,
+                                         s_rec, cbar, s_buf);
   }
-  for (; p < cpr; ++p) acc += s_w[p] * __ldcg(po + size_t(p) * D);
-  const float r = acc * s_w[cpr];
-  const size_t oi = rq * D + tid;
-  if (a.out_bf16)
-    reinterpret_cast<uint16_t*>(a.out)[oi] = f32_to_bf16_rn(r);
-  else
-    reinterpret_cast<float*>(a.out)[oi] = r;
+  // the grid's last CTA to finish resets the chunk-claim counter for the next launch (every
+  // CTA has issued its last claim by now)
+  __syncthreads();
+  if (tid == 0) {
+    if (*s_abort) flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_ATTN, blockIdx.x);
+    __threadfence();
+    if (atomicAdd(a.hdr + kCtrAttnDone, 1u) == gridDim.x - 1) {
+      a.hdr[kCtrAttnNext] = 0u;
+      a.hdr[kCtrAttnDone] = 0u;
+      // the decode step's lengths advance once every CTA has read them
+      if (a.lens_out)
+        for (int b = 0; b < a.rows / a.Hkv; ++b) a.lens_out[b] += a.len_add;
+    }
+  }
 }
+
 
 // ------------------------------------------------------------------ tensor maps (host)
 // A 2-D map over one cache tensor viewed as [num_pages * Hkv * 128 rows][d] 16-bit
@@ -601,18 +778,14 @@ static bool cache_map(const void* base, uint64_t rows, int d, int box_rows, CUte
   return true;
 }
 
-template <int D, bool VF, bool AF>
+template <int D, bool VF, bool AF, bool KQ4 = false>
 static cudaError_t launch_attn_t(const AttnParams& a, const CUtensorMap& mk, const CUtensorMap& mv,
                                  int grid, cudaStream_t s, bool pdl) {
-  auto k = attn_kernel<D, VF, AF>;
+  auto k = attn_kernel<D, VF, AF, KQ4>;
   const int smem = AttnSmem<D>::kTotal;
   const cudaError_t attr = set_smem_limit(k, smem);
   if (attr != cudaSuccess) return attr;
-  cudaError_t e = launch_k(k, dim3(grid), dim3(kAttnThreads), smem, s, pdl, a, mk, mv);
-  if (e != cudaSuccess) return e;
-  // the row merge, launched behind the attention grid (it waits for it before reading)
-  const size_t csmem = size_t(a.chunks_per_row + 1) * sizeof(float);
-  return launch_k(attn_combine_kernel<D>, dim3(a.rows, a.G), dim3(D), csmem, s, true, a);
+  return launch_k(k, dim3(grid), dim3(kAttnThreads), smem, s, pdl, a, mk, mv);
 }
 
 cudaError_t launch_attn(const Plan& p, const AttnParams& a_in, cudaStream_t s, bool pdl) {
@@ -630,6 +803,10 @@ cudaError_t launch_attn(const Plan& p, const AttnParams& a_in, cudaStream_t s, b
     return cudaErrorNotSupported;
   const bool vf = p.v_dtype == QS_F16, af = p.v_agg_dtype == QS_F16;
   const int grid = p.ws.attn_ctas;
+  if (p.key_nvfp4) {                  // NVFP4 keys: d = 128, V and P.V in FP16
+    if (p.d != 128 || !vf) return cudaErrorInvalidValue;
+    return launch_attn_t<128, true, true, true>(a, mk, mv, grid, s, pdl);
+  }
   if (p.d == 128) {
     if (vf) return launch_attn_t<128, true, true>(a, mk, mv, grid, s, pdl);
     if (af) return launch_attn_t<128, false, true>(a, mk, mv, grid, s, pdl);

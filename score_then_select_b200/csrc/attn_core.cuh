@@ -18,11 +18,75 @@
 
 namespace qs {
 
-// `swz(r, c)`: byte offset of 16-byte chunk c of token row r inside a K or V tile.
-// qb: the query fragments (B operand of S^T), valid0 / valid1: whether this lane's two
-// tokens are selected (masked ones get probability 0), scale_log2: softmax scale * log2 e.
-template <int D, bool V_F16, bool AGG_F16, typename Swz>
-QS_DEV void attn_warp_tile(uint32_t kst, uint32_t vst, const uint32_t (&qb)[D / 16][2],
+// K fragments (A operand of S^T) of k-step ks for this warp's 16 tokens, read from a BF16
+// tile in shared memory by ldmatrix: `swz(r, c)` is the byte offset of 16-byte chunk c of
+// token row r inside the tile.
+template <typename Swz>
+struct KFragLdsm {
+  uint32_t kst;
+  int warp, lane;
+  Swz swz;
+  QS_DEV void operator()(int ks, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) const {
+    ldsm_x4(a0, a1, a2, a3, kst + swz(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
+  }
+};
+
+// K fragments decoded from one 64-token tile of NVFP4 keys in shared memory (the storage
+// variant of "Jet-QSparse ...", Full text): each element becomes
+// bf16_rne(fp32(fp32(e * sigma) * g_k) + mu), e * sigma exact in float32.
+//   codes:  [4 chunks][64 tokens][16 bytes]; chunk c holds elements 32c..32c+31 of a
+//           token, element 2i + u in nibble u of byte i;
+//   scales: the page's 1,024 bytes; token slot m's scale of elements 16j..16j+15 at
+//           (j / 4) * 512 + 16 * (m % 32) + 4 * (m / 32) + j % 4; m0 = the page slot of
+//           the tile's first token;
+//   mu:     the row's centre, d floats.
+// This lane's rows are tokens r0 = 16 warp + lane / 4 and r0 + 8 of the tile, its elements
+// 2t, 2t + 1, 2t + 8, 2t + 9 of each k-step (t = lane % 4), as the mma A fragment holds them.
+struct KFragNvfp4 {
+  const uint8_t* codes;
+  const float* mu;
+  float gk;
+  int r0, t;
+  uint32_t sc[2][2];       // scale words: [row r0, r0 + 8][elements 0-63, 64-127]
+
+  QS_DEV KFragNvfp4(const uint8_t* codes_, const uint8_t* scales, const float* mu_, float gk_,
+                    int m0, int warp, int lane)
+      : codes(codes_), mu(mu_), gk(gk_), r0(warp * 16 + (lane >> 2)), t(lane & 3) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int m = m0 + r0 + 8 * r;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        sc[r][h] = *reinterpret_cast<const uint32_t*>(scales + h * 512 + 16 * (m & 31) + 4 * (m >> 5));
+    }
+  }
+  // byte t of w (two elements) -> bf16x2
+  QS_DEV uint32_t dec(uint32_t w, float sig, float2 m) const {
+    const uint32_t e = e2m1x2_to_f16x2(w >> (8 * t));
+    const float lo = __fadd_rn(__fmul_rn(__fmul_rn(f16_lo(e), sig), gk), m.x);
+    const float hi = __fadd_rn(__fmul_rn(__fmul_rn(f16_hi(e), sig), gk), m.y);
+    return pack_bf16x2(lo, hi);
+  }
+  QS_DEV void operator()(int ks, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) const {
+    const int c = ks >> 1, h = ks & 1;
+    const uint2 w0 = *reinterpret_cast<const uint2*>(codes + c * 1024 + r0 * 16 + 8 * h);
+    const uint2 w1 = *reinterpret_cast<const uint2*>(codes + c * 1024 + (r0 + 8) * 16 + 8 * h);
+    const float s0 = f16_lo(e4m3x2_to_f16x2(sc[0][ks >> 2] >> (8 * (ks & 3))));
+    const float s1 = f16_lo(e4m3x2_to_f16x2(sc[1][ks >> 2] >> (8 * (ks & 3))));
+    const float2 m01 = *reinterpret_cast<const float2*>(mu + 16 * ks + 2 * t);
+    const float2 m89 = *reinterpret_cast<const float2*>(mu + 16 * ks + 2 * t + 8);
+    a0 = dec(w0.x, s0, m01);
+    a1 = dec(w1.x, s1, m01);
+    a2 = dec(w0.y, s0, m89);
+    a3 = dec(w1.y, s1, m89);
+  }
+};
+
+// kf(ks, a0..a3): the K fragments of k-step ks (see KFragLdsm). qb: the query fragments (B
+// operand of S^T), valid0 / valid1: whether this lane's two tokens are selected (masked
+// ones get probability 0), scale_log2: softmax scale * log2 e; `swz` addresses the V tile.
+template <int D, bool V_F16, bool AGG_F16, typename KF, typename Swz>
+QS_DEV void attn_warp_tile(const KF& kf, uint32_t vst, const uint32_t (&qb)[D / 16][2],
                            bool valid0, bool valid1, float scale_log2, float& m0, float& m1,
                            float& l0, float& l1, float (&o)[D / 16][4], int warp, int lane,
                            Swz swz) {
@@ -32,7 +96,7 @@ QS_DEV void attn_warp_tile(uint32_t kst, uint32_t vst, const uint32_t (&qb)[D / 
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
     uint32_t a0, a1, a2, a3;
-    ldsm_x4(a0, a1, a2, a3, kst + swz(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
+    kf(ks, a0, a1, a2, a3);
     mma_bf16(c, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
   }
   const float x0 = valid0 ? c[0] * scale_log2 : -INFINITY;

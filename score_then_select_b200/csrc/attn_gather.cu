@@ -41,6 +41,9 @@ QS_DEV uint32_t gswz(int r, int c) {
   return uint32_t(r * (D * 2) + ((c ^ (r & 7)) << 4));
 }
 
+template <int D>
+QS_DEV void gather_merge_row(const AttnParams& a, int row, uint8_t* smem);
+
 template <int D, bool V_F16, bool AGG_F16>
 __global__ void __launch_bounds__(128, 2) attn_gather_kernel(const AttnParams a) {
   using SM = GatherSmem<D>;
@@ -56,7 +59,7 @@ __global__ void __launch_bounds__(128, 2) attn_gather_kernel(const AttnParams a)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   int n = a.n_sel[row];
-  int L = a.seq_lens[b];
+  int L = a.seq_lens[b] + a.len_add;
   if (n < 0 || n > a.budget || L < 0) {
     if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
     n = 0;
@@ -194,9 +197,10 @@ __global__ void __launch_bounds__(128, 2) attn_gather_kernel(const AttnParams a)
     const uint32_t kst = smem_u32(st), vst = smem_u32(st + SM::kTileBytes);
 
     const int tl = tile * kGTileT + warp * 16 + (lane >> 2);
-    attn_warp_tile<D, V_F16, AGG_F16>(kst, vst, qb, s_rows[tl] >= 0, s_rows[tl + 8] >= 0,
-                                      a.scale_log2, m0, m1, l0, l1, o, warp, lane,
-                                      [](int r, int c) { return gswz<D>(r, c); });
+    const auto sw = [](int r, int c) { return gswz<D>(r, c); };
+    attn_warp_tile<D, V_F16, AGG_F16>(KFragLdsm<decltype(sw)>{kst, warp, lane, sw}, vst, qb,
+                                      s_rows[tl] >= 0, s_rows[tl + 8] >= 0, a.scale_log2, m0,
+                                      m1, l0, l1, o, warp, lane, sw);
   }
   cp_async_wait<0>();
   __syncthreads();
@@ -261,7 +265,24 @@ __global__ void __launch_bounds__(128, 2) attn_gather_kernel(const AttnParams a)
     s_last = prev == unsigned(a.gsplits - 1);
   }
   __syncthreads();
-  if (!s_last) return;
+  if (s_last) gather_merge_row<D>(a, row, smem);
+  // the grid's last CTA advances the decode step's lengths (every CTA has read them)
+  if (a.lens_out) {
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      if (atomicAdd(a.hdr + kCtrAttnDone, 1u) == gridDim.x * gridDim.y - 1) {
+        a.hdr[kCtrAttnDone] = 0u;
+        for (int bb = 0; bb < a.rows / a.Hkv; ++bb) a.lens_out[bb] += a.len_add;
+      }
+    }
+  }
+}
+
+// The last split of row `row` to finish merges all of the row's splits (LSE combine).
+template <int D>
+QS_DEV void gather_merge_row(const AttnParams& a, int row, uint8_t* smem) {
+  const int b = row / a.Hkv, g = row % a.Hkv, Hq = a.Hkv * a.G, tid = threadIdx.x;
   __threadfence();
   float* s_w = reinterpret_cast<float*>(smem);          // [G][splits] weights, then [G] 1/den
   const int ns = a.gsplits;

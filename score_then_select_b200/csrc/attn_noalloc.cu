@@ -51,6 +51,7 @@ extern "C" qs_status qs_sparse_attn_noalloc(const qs_config* cfg, const qs_cache
   qs_status st = make_plan(cfg, batch, cache ? cache->max_context : 0, p);
   if (st != QS_OK) return st;
   if ((st = check_cache(p, cache, false)) != QS_OK) return st;
+  if (p.key_nvfp4) return QS_ERR_UNSUPPORTED;      // its kept blocks live in a workspace
   if (!q || (reinterpret_cast<uintptr_t>(q) & 15) || !sel || !n_sel || !out) return QS_ERR_INVALID_ARG;
   // carve the static array: status header | row counters | partial (m, l) | partial o
   const size_t rows = size_t(batch) * p.Hkv, rows_q = size_t(batch) * p.Hq;

@@ -178,6 +178,30 @@ __global__ void __launch_bounds__(kNkThreads) gather_kv_nvfp4k_kernel(const Gath
   }
 }
 
+// CTA = one row: its n_keep kept blocks (the complete blocks with the largest error, ranked
+// as the select kernel ranks them), written for the attention over the NVFP4 keys.
+__global__ void __launch_bounds__(128) kept_blocks_kernel(const KeptParams p) {
+  __shared__ float s_v[4];
+  __shared__ int s_j[4];
+  pdl_wait();                  // the errors (and the step before) come from earlier kernels
+  pdl_trigger();
+  const int row = blockIdx.x, b = row / p.Hkv;
+  const int L = max(0, p.seq_lens[b] + p.len_add);
+  const float* err = p.block_err + size_t(row) * p.nb_stride;
+  const int complete = min(L / kPage, p.nb_stride);
+  int k1 = -1, k2 = -1;
+  if (p.n_keep > 0) k1 = nk_argmax(err, complete, -1, s_v, s_j);
+  if (p.n_keep > 1 && k1 >= 0) k2 = nk_argmax(err, complete, k1, s_v, s_j);
+  if (threadIdx.x == 0) {
+    p.kept[2 * row] = k1;
+    p.kept[2 * row + 1] = k2;
+  }
+}
+
+cudaError_t launch_kept_blocks(const KeptParams& p, cudaStream_t s, bool pdl) {
+  return launch_k(kept_blocks_kernel, dim3(p.rows), dim3(128), 0, s, pdl, p);
+}
+
 cudaError_t launch_gather_kv_nvfp4k(const Plan& pl, const GatherNvParams& p, cudaStream_t s) {
   const int per_cta = (kNkThreads / 16) * kNkUnroll;            // 128 slots
   const int slices = (pl.budget * kPage + per_cta - 1) / per_cta;

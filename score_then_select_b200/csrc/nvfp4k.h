@@ -17,4 +17,13 @@ struct GatherNvParams {
 
 cudaError_t launch_gather_kv_nvfp4k(const Plan& pl, const GatherNvParams& p, cudaStream_t s);
 
+// The kept (BF16) blocks of every row, for attention over the NVFP4 keys.
+struct KeptParams {
+  const float* block_err;     // [rows][nb_stride]
+  const int32_t* seq_lens;
+  int32_t* kept;              // [rows][2], -1: none
+  int rows, Hkv, nb_stride, n_keep, len_add;
+};
+cudaError_t launch_kept_blocks(const KeptParams& p, cudaStream_t s, bool pdl);
+
 }  // namespace qs

@@ -177,6 +177,14 @@ QS_DEV uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(uint16_t(two_codes)));
   return r;
 }
+// two E2M1 codes (low byte of v: the low nibble is the first element) -> f16x2, exact
+QS_DEV uint32_t e2m1x2_to_f16x2(uint32_t v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+      : "=r"(r) : "r"(v));
+  return r;
+}
 QS_DEV float f16_lo(uint32_t x) { return __half2float(__ushort_as_half(uint16_t(x))); }
 QS_DEV float f16_hi(uint32_t x) { return __half2float(__ushort_as_half(uint16_t(x >> 16))); }
 // bf16x2 -> f16x2 (for FP16 value aggregation of BF16-stored values)

@@ -34,6 +34,7 @@ constexpr int kChunkTilesMax = 8;   // attention work unit: up to 8 tiles (512 s
 constexpr int kChunksPerCta = 6;    // chunk size target: about this many chunks per CTA
 constexpr int kTmaMinTilesPerCta = 40;  // auto path: tile pipeline from this much work per CTA
 constexpr int kCtrAttnNext = 17;    // header word: next attention chunk to claim
+constexpr int kCtrAttnDone = 18;    // header word: attention CTAs finished (last one resets)
 
 // Workspace carve-up (byte offsets); computed identically by qs_workspace_size and calls.
 struct WsLayout {
@@ -46,6 +47,7 @@ struct WsLayout {
   size_t part_ml = 0;   // [batch][Hq][parts_per_head][2] f32 attention partials (m, l)
   size_t part_o = 0;    // [batch][Hq][parts_per_head][d] f32 attention partials o
   size_t row_ctr = 0;   // [batch][Hkv] u32 attention segments finished per row
+  size_t kept = 0;      // NVFP4 key storage: [batch][Hkv][2] i32 kept blocks (-1: none)
   size_t total = 0;
   int nb_stride = 0;
   int attn_ctas = 0;     // attention grid (persistent; chunks claimed dynamically)
@@ -66,6 +68,7 @@ struct Plan {
   bool attn_tma;        // attention by the tile pipeline (else the gather kernel)
   int proxy_dtype, v_dtype, v_agg_dtype, out_dtype;
   int force_sink, force_last, n_keep;
+  bool key_nvfp4 = false;   // attention reads the NVFP4 keys (kept blocks BF16)
   float scale;
   WsLayout ws;
 };
@@ -90,6 +93,9 @@ struct AppendParams {
   float* qt;
   int batch, Hkv, G, d, r, max_new, max_pages_per_seq, num_pages, max_context;
   int S;                     // block size (centroid sums)
+  // 1: leave seq_lens as they are (the decode step reads them as seq_lens + 1 and its
+  // attention kernel advances them at the end); 0: advance them by n_new
+  int keep_lens;
 };
 
 struct BlockErrParams {
@@ -163,6 +169,12 @@ struct ScoreParams {
   // the query side (q~, or the NVFP4 query tiles and g_q), so the page stream may start
   // before waiting for it; 0: wait for it first (it may still be writing seq_lens)
   int early_stream;
+  // rank r, decode step: the kernel before is the one-token writer, which leaves seq_lens
+  // unchanged (the step's length is seq_lens + len_add) and writes only the newest token's
+  // slot. The scan computes q~ itself from q and P (inline_qt), streams every page at once,
+  // and waits for the writer only before copying a row's last page (wait_last).
+  const float* P;
+  int len_add, inline_qt, wait_last;
 };
 
 struct SelectParams {
@@ -173,6 +185,7 @@ struct SelectParams {
   int32_t* n_sel;
   uint32_t* hdr;
   int rows, Hkv, S, nb_stride, budget, force_sink, force_last, n_keep;
+  int len_add;               // the step's length is seq_lens + len_add
 };
 
 struct AttnParams {
@@ -196,6 +209,15 @@ struct AttnParams {
   int gsplits, g_tokens_per_split;   // gather kernel split plan
   int out_bf16;
   float scale_log2;          // softmax scale * log2(e)
+  int len_add;               // the step's length is seq_lens + len_add
+  int32_t* lens_out;         // non-null: the grid's last CTA adds len_add to lens_out[b]
+  // NVFP4 key storage: keys from the scoring cache (codes, scales, g_k, the row's centre),
+  // except the row's kept blocks (kept[row][0..1], -1: none), which come from k
+  const uint8_t* k_codes;
+  const uint8_t* k_scales;
+  const float* key_center;
+  const float* key_gscale;
+  const int32_t* kept;
 };
 
 struct GatherParams {        // gather-then-attend: selected blocks -> compact pages

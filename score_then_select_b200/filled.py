@@ -19,7 +19,8 @@ def cfg_kwargs(w, attn_path: int = 0) -> dict:
                 block_size=w.block_size, budget=w.budget, proxy_rank=w.proxy_rank,
                 proxy_dtype=w.proxy_dtype, v_dtype=w.v_dtype, v_agg_dtype=w.v_agg_dtype,
                 out_dtype=w.out_dtype, force_sink=w.force_sink, force_last=w.force_last,
-                n_keep_hp=w.n_keep_hp, softmax_scale=w.softmax_scale, attn_path=attn_path)
+                n_keep_hp=w.n_keep_hp, softmax_scale=w.softmax_scale, attn_path=attn_path,
+                key_storage=getattr(w, "key_storage", "bf16"))
 
 
 def u16(a: np.ndarray, dt=torch.bfloat16) -> torch.Tensor:

@@ -50,6 +50,7 @@ class Workload:
     ragged_max: int = 131072
     top_p: float = 0.0           # > 0: top-p selection of this share of the estimated mass,
                                  # at most `budget` blocks (binary proxy)
+    key_storage: str = "bf16"    # 'nvfp4': the attention reads the NVFP4 keys (kept blocks BF16)
 
     @property
     def group(self) -> int:
@@ -97,6 +98,12 @@ BLOCK128K = Workload(
 NVFP4_128K = BLOCK128K.replace(
     name="nvfp4_b16_h40kv8_d128_L131072_S128_k128", budget=128, proxy_rank=0,
     proxy_dtype="nvfp4", v_dtype="f16", v_agg_dtype="f16", n_keep_hp=2, seed=1004)
+
+# The NVFP4 storage variant ("Jet-QSparse ...", Full text): the same step, with the
+# attention reading every key from the NVFP4 cache (dequantised, un-centred, rounded to
+# BF16) except the two kept blocks, whose BF16 keys are read.
+NVFP4_STORE_128K = NVFP4_128K.replace(name="nvfp4store_b16_h40kv8_d128_L131072_S128_k128",
+                                      key_storage="nvfp4", seed=1015)
 
 # The 128K block-level step with the projected-key cache stored as FP8 E4M3 ("Joint Subspace
 # Sparse Attention for Efficient Long-Context Decoding", Figure 10: FP8 or BF16 scoring
@@ -156,7 +163,8 @@ FULL = {w.name: w for w in (TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED)}
 ORDER = [TINY, TOKEN32K, BLOCK128K, NVFP4_128K, RAGGED]
 # variants of the configurations above (FP8 projected keys, centroid scoring, 128K token
 # level, the binary proxy with a top-p budget)
-VARIANTS = [FP8_128K, FP8_TOKEN32K, CENTROID_128K, CENTROID_S32, TOKEN128K, RABITQ_TOKEN128K]
+VARIANTS = [FP8_128K, FP8_TOKEN32K, CENTROID_128K, CENTROID_S32, TOKEN128K, RABITQ_TOKEN128K,
+            NVFP4_STORE_128K]
 # SEMANTIC_128K is not among them: its oracle step also needs the prompt length.
 
 

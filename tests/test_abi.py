@@ -298,3 +298,43 @@ def test_radix_select_validates_on_the_host():
         qs.qs_select_topk_radix(_cfg(proxy_rank=0, proxy_dtype="nvfp4", block_size=128,
                                      n_keep_hp=2), cache, a, 4, a, a, a, stream=0)
     assert e.value.status == B.QS_ERR_INVALID_ARG
+
+
+def test_nvfp4_key_storage_validates_on_the_host():
+    """Attention over the NVFP4 keys: only on the NVFP4 configuration and the tile pipeline;
+    every attending call needs the NVFP4 pointers (16-byte aligned codes, scales, centres)
+    and the block errors for kept blocks; full-KV attention plans the BF16 keys regardless;
+    the no-allocation entry point refuses it. All rejected before any launch."""
+    nv = dict(proxy_rank=0, proxy_dtype="nvfp4", block_size=128, n_keep_hp=2, budget=128,
+              v_dtype="f16", v_agg_dtype="f16")
+    st = _cfg(key_storage="nvfp4", **nv)
+    assert qs.qs_workspace_size(st, 16, 131072) > qs.qs_workspace_size(_cfg(**nv), 16, 131072)
+    assert qs.qs_attention_launches(st, 16, 131072) == 2
+    assert qs.qs_attention_launches(_cfg(**nv), 16, 131072) == 1
+    assert qs.qs_dense_workspace_size(st, 16, 131072) == qs.qs_dense_workspace_size(
+        _cfg(**nv), 16, 131072)
+    with pytest.raises(qs.QsError) as e:                      # rank-r scoring copy
+        qs.qs_workspace_size(_cfg(key_storage="nvfp4"), 16, 131072)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    with pytest.raises(qs.QsError) as e:                      # the gather kernel cannot decode
+        qs.qs_workspace_size(_cfg(key_storage="nvfp4", attn_path=2, **nv), 16, 131072)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED
+    a = 1 << 20
+    cache = _fake_cache()
+    with pytest.raises(qs.QsError) as e:                      # no scales / tensor scale
+        qs.qs_sparse_attn(st, cache, a, a, a, 4, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    cache.proxy_scale = a
+    cache.key_gscale = a
+    with pytest.raises(qs.QsError) as e:                      # kept blocks need block_err
+        qs.qs_sparse_attn(st, cache, a, a, a, 4, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    cache.block_err = a
+    cache.key_center = a + 8                                  # centres copied in 16-byte units
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_sparse_attn(st, cache, a, a, a, 4, a, a, stream=0)
+    assert e.value.status == B.QS_ERR_INVALID_ARG
+    cache.key_center = a
+    with pytest.raises(qs.QsError) as e:
+        qs.qs_sparse_attn_noalloc(st, cache, a, a, a, 4, a, stream=0)
+    assert e.value.status == B.QS_ERR_UNSUPPORTED

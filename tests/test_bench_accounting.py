@@ -70,3 +70,17 @@ def test_ragged_lengths_count_valid_tokens_only():
 def test_steps_per_s_aggregates_over_ranks():
     assert bench.aggregate_steps_per_s(0.5, 1) == 2000.0
     assert bench.aggregate_steps_per_s(0.5, 4) == 8000.0
+
+
+def test_nvfp4_key_storage_bytes():
+    """The NVFP4 storage variant reads 72 bytes of key per selected token (64 of codes, 8 of
+    scales), 256 for the two kept blocks' BF16 keys, and the FP16 values in full."""
+    w = synth.NVFP4_STORE_128K
+    lens = np.full(16, 131072, dtype=np.int64)
+    sel, nsel = _full_selection(w, lens)
+    by = bench.step_bytes(w, lens, sel, nsel)
+    rows, tok_row = 16 * 8, 128 * 128
+    v = rows * tok_row * 256
+    k = rows * ((tok_row - 2 * 128) * 72 + 2 * 128 * 256)
+    assert by["kv"] == v + k
+    assert by["proxy"] == rows * 131072 * 72

@@ -61,8 +61,11 @@ def _dense(f, cache, row_lens, max_context):
     return out
 
 
-@pytest.mark.parametrize("w", WORKLOADS, ids=lambda w: w.name)
+@pytest.mark.parametrize("w", WORKLOADS + [synth.small(synth.NVFP4_STORE_128K)],
+                         ids=lambda w: w.name)
 def test_dense_full_kv(w):
+    """Full-KV attention; under the NVFP4 storage configuration it still reads the BF16
+    key pages (the comparison the pages make is with BF16 attention)."""
     _gpu()
     from tests.gpu_util import Filled, out_to_f64
     inp = synth.Inputs(w)

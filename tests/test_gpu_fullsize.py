@@ -24,7 +24,8 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 # (workload, attention kernel): the automatic choice everywhere, and the tile pipeline
 # forced on the ragged workload (whose rows end in partial blocks)
 FULL = [(synth.BLOCK128K, 0), (synth.NVFP4_128K, 0), (synth.TOKEN32K, 0), (synth.RAGGED, 0),
-        (synth.RAGGED, 1), (synth.FP8_128K, 0), (synth.CENTROID_128K, 0), (synth.TOKEN128K, 0)]
+        (synth.RAGGED, 1), (synth.FP8_128K, 0), (synth.CENTROID_128K, 0), (synth.TOKEN128K, 0),
+        (synth.NVFP4_STORE_128K, 0)]
 
 
 def _gpu():
@@ -83,6 +84,7 @@ def test_fullsize_every_row(case):
         if n and not (np.all(np.diff(got) > 0) and got[0] >= 0 and got[-1] < nb):
             return "selection not ascending and in range"
         forced = r["forced"]
+        kept = None
         if w.n_keep_hp:
             nfull = L // w.block_size
             codes, scl, x32 = r["cache"]
@@ -98,6 +100,9 @@ def test_fullsize_every_row(case):
         if not ok:
             return f"selection {why}"
         q, K, V = decoded_row(w, row)
+        if w.key_storage == "nvfp4":               # the storage variant's attended keys
+            r = oracle_row(inp, b, g, row=row, g_q=gq, sel_override=got, keep_override=kept)
+            K = r["K_att"]
         tokens = r["tokens"] if np.array_equal(got, r["sel"]) else \
             M.block_tokens(got, w.block_size, L)
         want = r["out"] if np.array_equal(got, r["sel"]) else \

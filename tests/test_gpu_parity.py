@@ -25,14 +25,15 @@ RANKR = [synth.TINY, synth.TINY_NEEDLE, synth.TINY_FP8, synth.TINY_CENTROID] + [
                                           (synth.TOKEN32K, synth.BLOCK128K, synth.RAGGED,
                                            synth.FP8_128K, synth.FP8_TOKEN32K,
                                            synth.CENTROID_128K, synth.CENTROID_S32)]
-NVFP4 = [synth.small(synth.NVFP4_128K)]
+NVFP4 = [synth.small(synth.NVFP4_128K), synth.small(synth.NVFP4_STORE_128K)]
 
 
 def _paths(ws):
     """(workload, attention kernel) cases: both kernels where the block size allows the tile
     pipeline (attn_path 1 forces it, 2 forces the gather kernel), the automatic choice
-    otherwise."""
-    return [(w, p) for w in ws for p in ((1, 2) if w.block_size >= 8 else (0,))]
+    otherwise; NVFP4 key storage is decoded by the tile pipeline only."""
+    return [(w, p) for w in ws
+            for p in ((1,) if w.key_storage == "nvfp4" else (1, 2) if w.block_size >= 8 else (0,))]
 
 
 def _ids(case):
@@ -143,8 +144,10 @@ def test_nvfp4_parity(case):
             got = sel[b, g, :n]
             ok, why = M.selection_valid(r["beta"], w.budget, forced, got)
             assert ok, f"{where}: selection {why}"
-            rr = oracle_row(inp, b, g, row=row, g_q=gq, sel_override=got)
-            check_attention(w, out[b, g * G:(g + 1) * G], rr["out"], row, rr["tokens"], where)
+            rr = oracle_row(inp, b, g, row=row, g_q=gq, sel_override=got, keep_override=kept)
+            # with NVFP4 key storage the attended keys are the storage variant's (K_att)
+            check_attention(w, out[b, g * G:(g + 1) * G], rr["out"], row, rr["tokens"], where,
+                            K=rr["K_att"])
 
 
 def test_needle_selected_on_gpu():

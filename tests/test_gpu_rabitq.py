@@ -277,6 +277,11 @@ def _crafted():
                 (True, True)))
     out.append(("blocks-S16", (rng.standard_normal(200) * 2).astype(np.float32), 16, 40, 0.7,
                 (True, True)))
+    # budgets above 4,096 blocks take the histogram kernel instead of the sorted candidates
+    out.append(("large-budget", (rng.standard_normal(20000) * 2).astype(np.float32), 1, 6000,
+                0.9, (True, True)))
+    out.append(("integer-ties-large-budget", np.round(rng.standard_normal(9000)).astype(np.float32),
+                1, 5000, 0.6, (True, False)))
     return out
 
 
@@ -292,7 +297,8 @@ def test_top_p_on_crafted_scores(case):
     mass, want = _oracle_top_p(scores, p32, budget, forced)
     ok, why = M.top_p_valid(mass, p32, budget, forced, got, rel_tol=1e-5)
     assert ok, f"{name}: {why} (got {len(got)}, oracle {len(want)})"
-    if name in ("all-equal", "one-block", "all-neg-inf", "inf-nan", "integer-ties"):
+    if name in ("all-equal", "one-block", "all-neg-inf", "inf-nan", "integer-ties",
+                "integer-ties-large-budget"):
         assert np.array_equal(got, want), name
     if name == "all-equal":
         assert len(got) == math.ceil(0.375 * 300)     # equal masses: the lowest indices

@@ -244,3 +244,36 @@ def test_step_nvfp4_kept_blocks_are_forced_and_selected():
     assert len(r["keep"]) == 2
     assert set(r["keep"].tolist()) <= set(r["forced"].tolist())
     assert set(r["keep"].tolist()) <= set(r["sel"].tolist())
+
+
+def test_step_key_storage_attends_the_storage_keys():
+    """With NVFP4 key storage the row step attends over nvfp4_attended_keys_bf16 (the kept
+    blocks' BF16 keys, elsewhere the decoded, un-centred keys rounded to BF16), with the
+    same selection; keeping every selected block gives exactly the BF16-key output."""
+    import dataclasses
+    from oracle import step as OS
+    rng = np.random.default_rng(72)
+    L, G, d, S = 1000, 4, 128, 128
+    k = F.f32_to_bf16_rne((rng.standard_normal((L, d)) * 1.5 + 0.5).astype(np.float32))
+    v = F.f32_to_bf16_rne(rng.standard_normal((L, d)).astype(np.float32))
+    q = F.f32_to_bf16_rne((rng.standard_normal((G, d)) * 3).astype(np.float32))
+    mu = F.bf16_to_f64(k).mean(axis=0).astype(np.float32)
+    g_k = np.float32(np.abs(M.centre(k, mu)).max() / np.float32(2688.0))
+    g_q = M.query_scale(q)
+    p = OS.RowParams(S=S, budget=5, scale=1 / np.sqrt(d), proxy="nvfp4", v_dtype="bf16",
+                     force_sink=True, force_last=True, n_keep=2)
+    ps = dataclasses.replace(p, key_storage="nvfp4")
+    r_bf = OS.decode_row(p, k, v, q, L, mu=mu, g_k=g_k, g_q=g_q)
+    r_st = OS.decode_row(ps, k, v, q, L, mu=mu, g_k=g_k, g_q=g_q)
+    assert np.array_equal(r_st["sel"], r_bf["sel"]) and len(r_st["keep"]) == 2
+    codes, scales, _ = r_st["cache"]
+    want_k = F.bf16_to_f64(M.nvfp4_attended_keys_bf16(k, codes, scales, g_k, mu, r_st["keep"],
+                                                      S, L))
+    assert np.array_equal(r_st["K_att"], want_k)
+    Vd = OS.decode_v(v, p.v_dtype)
+    assert np.array_equal(r_st["out"], M.sparse_attention(F.bf16_to_f64(q), want_k, Vd,
+                                                          r_st["tokens"], p.scale))
+    # the non-kept selected blocks are attended with their NVFP4 keys: the output moves
+    assert not np.allclose(r_st["out"], r_bf["out"], rtol=1e-6, atol=0)
+    r_all = OS.decode_row(ps, k, v, q, L, mu=mu, g_k=g_k, g_q=g_q, keep_override=r_st["sel"])
+    assert np.array_equal(r_all["out"], r_bf["out"])

@@ -10,7 +10,8 @@ row_params = OS.row_params_of
 top_p_params = OS.top_p_params_of
 
 
-def oracle_row(inp: synth.Inputs, b: int, g: int, row=None, g_q=None, sel_override=None):
+def oracle_row(inp: synth.Inputs, b: int, g: int, row=None, g_q=None, sel_override=None,
+               keep_override=None):
     w = inp.w
     k, v, q = row if row is not None else inp.row(b, g)
     L = int(inp.lens[b])
@@ -20,7 +21,7 @@ def oracle_row(inp: synth.Inputs, b: int, g: int, row=None, g_q=None, sel_overri
     P = inp.P[g] if inp.P is not None else None
     mu = inp.mu[b, g] if inp.mu is not None else None
     return OS.decode_row(row_params(w), k, v, q, L, P=P, mu=mu, g_k=inp.g_k, g_q=g_q,
-                         sel_override=sel_override)
+                         sel_override=sel_override, keep_override=keep_override)
 
 
 def query_scale_all(inp: synth.Inputs, Q=None):
