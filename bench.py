@@ -61,6 +61,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (small cases for profiling only)")
+    ap.add_argument("--context", type=int, default=0,
+                    help="override the workload's context (small cases for profiling only)")
     ap.add_argument("--no-compare", action="store_true",
                     help="skip the full-KV and gather-then-attend comparison")
     ap.add_argument("--attn-path", type=int, default=0, choices=[0, 1, 2],
@@ -456,6 +458,8 @@ def run_ours(args):
     w0 = WORKLOADS[args.workload]
     if args.batch:
         w0 = w0.replace(batch=args.batch)
+    if args.context:
+        w0 = w0.replace(context=args.context, calib_tokens=min(w0.calib_tokens, args.context))
     w = rank_workload(w0, rank)
     inp = synth.Inputs(w)
     f = Filled(inp, attn_path=args.attn_path)

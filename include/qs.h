@@ -189,9 +189,9 @@ typedef struct {
 qs_status qs_workspace_size(const qs_config *cfg, int32_t batch, int32_t max_context,
                             size_t *bytes /* host */);
 
-/* Number of kernel launches qs_sparse_attn makes for this shape: 1 (both attention
-   kernels, the gather kernel and the tile pipeline, merge each row's partials in the same
-   launch), 2 with key_storage QS_NVFP4 (the rows' kept blocks first). Host only. */
+/* Number of kernel launches qs_sparse_attn makes for this shape: 1 for the gather kernel
+   (its log-sum-exp merge is in-kernel), 2 for the tile pipeline (then the row merge), 3 with
+   key_storage QS_NVFP4 (the rows' kept blocks first). Host only. */
 qs_status qs_attention_launches(const qs_config *cfg, int32_t batch, int32_t max_context,
                                 int32_t *launches /* host */);
 
@@ -402,7 +402,7 @@ qs_status qs_dense_workspace_size(const qs_config *cfg, int32_t batch, int32_t m
    budget, forced blocks and attn_path are not used); the cache's proxy fields are not
    read. Logits are float32 sums of BF16 products, P.V operands v_agg_dtype, float32
    accumulation; the row is split over the tile-pipeline attention kernel and merged by
-   the log-sum-exp combine inside the same launch (1 launch). Every len must be <= cache->max_context (a row
+   the log-sum-exp combine (2 launches). Every len must be <= cache->max_context (a row
    that needs more than ceil(max_context / 128) pages records QS_ERR_DEVICE_BOUNDS). ws: qs_dense_workspace_size(cfg, batch,
    cache->max_context) bytes, initialised by qs_workspace_init. q is 16-byte aligned. */
 qs_status qs_dense_attn(const qs_config *cfg, const qs_cache *cache, const void *q,

@@ -261,10 +261,12 @@ def lse_combine(ms, ls, os_) -> np.ndarray:
 # ============================================================================================
 # Attending over the NVFP4 keys  [JQS, Full text]
 # The storage variant of the page keeps the attended keys in NVFP4 too, with at most two
-# blocks per sequence kept in BF16 to bound the quantisation error. Reading: the key of a
-# token in a kept block is its stored BF16 key; every other key is its NVFP4 scoring copy
-# decoded and un-centred (dequantised value + the row's calibrated mean). Not yet built on
-# the GPU; defined here so that a kernel can be checked against it.
+# blocks per sequence kept in BF16 to bound the quantisation error, and computes attention
+# on them. Reading: the key of a token in a kept block is its stored BF16 key; every other
+# key is its NVFP4 scoring copy decoded and un-centred (dequantised value + the row's
+# calibrated mean), exactly (nvfp4_attended_keys: what the fused attention computes with).
+# nvfp4_attended_keys_bf16 is the same key rounded to BF16: what a gather into a BF16
+# buffer for dense attention holds.
 # ============================================================================================
 
 

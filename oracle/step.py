@@ -93,9 +93,10 @@ def decode_row(p: RowParams, k_bits, v_bits, q_bits, L: int, P=None, mu=None, g_
     attended (used once the GPU's kept pair has been accepted under the near-tie rule).
 
     With ``p.key_storage == 'nvfp4'`` ("Jet-QSparse ...", Full text: the persistent cache
-    keeps the attended keys in NVFP4, at most two blocks per sequence at BF16), the keys
-    attended are nvfp4_attended_keys_bf16: the kept blocks' stored BF16 keys, elsewhere the
-    NVFP4 code dequantised and un-centred, rounded to BF16 (returned as ``K_att``).
+    keeps the attended keys in NVFP4, at most two blocks per sequence at BF16, and attention
+    is computed on them), the keys attended are nvfp4_attended_keys: the kept blocks'
+    stored BF16 keys, elsewhere the NVFP4 value dequantised and un-centred, exactly
+    (returned as ``K_att``).
     """
     cache = row_scoring_cache(p, k_bits[:L], P, mu, g_k)
     beta = row_block_scores(p, cache, q_bits, L, P=P, g_q=g_q, g_k=g_k)
@@ -108,8 +109,7 @@ def decode_row(p: RowParams, k_bits, v_bits, q_bits, L: int, P=None, mu=None, g_
     if p.key_storage == "nvfp4":
         codes, scales, _ = cache
         kept = keep if keep_override is None else np.asarray(keep_override, dtype=np.int64)
-        K = F.bf16_to_f64(M.nvfp4_attended_keys_bf16(k_bits[:L], codes, scales, g_k, mu, kept,
-                                                     p.S, L))
+        K = M.nvfp4_attended_keys(k_bits[:L], codes, scales, g_k, mu, kept, p.S, L)
     else:
         K = F.bf16_to_f64(k_bits[:L])
     V = decode_v(v_bits[:L], p.v_dtype)

@@ -258,9 +258,8 @@ static qs_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QS_OK : 
 // ------------------------------------------------------------ stage bodies (validated input)
 static qs_status do_append(const Plan& p, const qs_cache* c, const void* k_new, const void* v_new,
                            const int32_t* n_new, int max_new, const float* P, const void* q,
-                           void* ws, cudaStream_t s, bool keep_lens = false) {
+                           void* ws, cudaStream_t s) {
   AppendParams a{};
-  a.keep_lens = keep_lens ? 1 : 0;
   a.k_new = static_cast<const uint16_t*>(k_new);
   a.v_new = static_cast<const uint16_t*>(v_new);
   a.n_new = n_new;
@@ -322,26 +321,10 @@ static qs_status do_prep(const Plan& p, const void* q, const float* P, void* ws,
   return cuda_status(launch_qpack(p, a, s, pdl));
 }
 
-// Step modes of the rank-r decode (qs_decode): the writer leaves seq_lens alone and every
-// later kernel reads seq_lens + 1; the scan starts streaming at once and computes q~ itself
-// (rank <= 32; rank 64 takes it from the writer); the attention advances seq_lens at its end.
-struct StepMode {
-  bool decode = false;      // the one-token decode step of a rank-r configuration
-  const float* P = nullptr;
-};
-
 static qs_status do_score(const Plan& p, const qs_cache* c, const void* q, float* scores, void* ws,
-                          cudaStream_t s, bool pdl, bool early_stream = false,
-                          const StepMode& m = StepMode()) {
+                          cudaStream_t s, bool pdl, bool early_stream = false) {
   ScoreParams a{};
   a.early_stream = early_stream ? 1 : 0;
-  if (m.decode) {
-    a.early_stream = 1;
-    a.len_add = 1;
-    a.wait_last = 1;
-    a.inline_qt = p.r <= 32 ? 1 : 0;
-    a.P = m.P;
-  }
   a.q = static_cast<const uint16_t*>(q);
   a.proxy = c->proxy;
   a.proxy_scale = c->proxy_scale;
@@ -366,10 +349,8 @@ static qs_status do_score(const Plan& p, const qs_cache* c, const void* q, float
 }
 
 static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores, int32_t* sel,
-                           int32_t* n_sel, void* ws, cudaStream_t s, bool pdl,
-                           const StepMode& m = StepMode()) {
+                           int32_t* n_sel, void* ws, cudaStream_t s, bool pdl) {
   SelectParams a{};
-  a.len_add = m.decode ? 1 : 0;
   a.scores = scores;
   a.block_err = (p.kind == PK_NVFP4 && p.n_keep > 0) ? c->block_err : nullptr;
   a.seq_lens = c->seq_lens;
@@ -389,12 +370,8 @@ static qs_status do_select(const Plan& p, const qs_cache* c, const float* scores
 
 static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, const int32_t* sel,
                            const int32_t* n_sel, void* out, void* ws, cudaStream_t s, bool pdl,
-                           const int32_t* row_lens = nullptr, const StepMode& m = StepMode()) {
+                           const int32_t* row_lens = nullptr) {
   AttnParams a{};
-  if (m.decode) {
-    a.len_add = 1;
-    a.lens_out = c->seq_lens;
-  }
   a.row_lens = row_lens;
   a.q = static_cast<const uint16_t*>(q);
   a.k = static_cast<const uint16_t*>(c->k);
@@ -431,7 +408,7 @@ static qs_status do_attend(const Plan& p, const qs_cache* c, const void* q, cons
     int32_t* kept = ws_at<int32_t>(ws, p.ws.kept);
     a.kept = kept;
     KeptParams kp{c->block_err, c->seq_lens, kept, p.batch * p.Hkv, p.Hkv, p.nb_stride,
-                  p.n_keep, a.len_add};
+                  p.n_keep};
     const qs_status st = cuda_status(launch_kept_blocks(kp, s, pdl));
     if (st != QS_OK) return st;
     pdl = true;
@@ -474,8 +451,9 @@ qs_status qs_attention_launches(const qs_config* cfg, int32_t batch, int32_t max
   const qs_status st = make_plan(cfg, batch, max_context, p);
   if (st != QS_OK) return st;
   if (!launches) return QS_ERR_INVALID_ARG;
-  // both kernels merge their partials in-kernel; NVFP4 keys add the kept-block kernel
-  *launches = p.key_nvfp4 ? 2 : 1;
+  // gather kernel: 1 (its merge is in-kernel); tile pipeline: 2 (the row merge follows),
+  // 3 with NVFP4 keys (the rows' kept blocks first)
+  *launches = p.attn_tma ? (p.key_nvfp4 ? 3 : 2) : 1;
   return QS_OK;
 }
 
@@ -639,22 +617,8 @@ qs_status qs_decode(const qs_config* cfg, const qs_cache* cache, const void* q, 
   int32_t* sel = sel_out ? sel_out : ws_at<int32_t>(ws, p.ws.sel);
   int32_t* nsel = n_sel_out ? n_sel_out : ws_at<int32_t>(ws, p.ws.nsel);
   float* scores = ws_at<float>(ws, p.ws.scores);
-  if (p.kind == PK_RANKR) {
-    // the writer runs under the scan: it leaves seq_lens alone (the step reads seq_lens + 1),
-    // the scan computes q~ itself (rank <= 32; else the writer's fused prep gives it) and
-    // waits for the writer only before a row's last page, and the attention advances
-    // seq_lens once every kernel of the step has read them
-    StepMode m;
-    m.decode = true;
-    m.P = P;
-    const void* prep_q = p.r <= 32 ? nullptr : q;
-    if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, P, prep_q, ws, stream, true)) != QS_OK)
-      return st;
-    if ((st = do_score(p, cache, q, scores, ws, stream, true, true, m)) != QS_OK) return st;
-    if ((st = do_select(p, cache, scores, sel, nsel, ws, stream, true, m)) != QS_OK) return st;
-    return do_attend(p, cache, q, sel, nsel, out, ws, stream, true, nullptr, m);
-  }
-  // append (+ query packing on the NVFP4 path), then the stages in stream order
+  // append (+ fused scoring prep on the rank-r path, query packing on the NVFP4 path), then
+  // the stages in stream order, each launched behind the one before
   if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, P, q, ws, stream)) != QS_OK) return st;
   if (p.kind == PK_NVFP4 && (st = do_prep(p, q, P, ws, stream, true)) != QS_OK) return st;
   if ((st = do_score(p, cache, q, scores, ws, stream, true)) != QS_OK) return st;

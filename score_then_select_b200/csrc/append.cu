@@ -42,25 +42,6 @@ QS_DEV float e2m1_decode(uint32_t c) {
   float v = (m < 4u) ? 0.5f * float(m) : (m == 7u ? 6.0f : float(m - 2u));
   return (c & 8u) ? -v : v;
 }
-// UE4M3 (bias 7, 3 mantissa bits, subnormal step 2^-9, largest finite 448 = 0x7E):
-// nearest even, saturating; non-positive and NaN inputs give code 0.
-QS_DEV uint32_t ue4m3_encode(float sf) {
-  if (!(sf > 0.0f)) return 0u;
-  if (sf >= 448.0f) return 0x7Eu;
-  const uint32_t u = __float_as_uint(sf);
-  const int e = int(u >> 23) - 127;
-  if (e < -6) return __float2uint_rn(sf * 512.0f);  // subnormal range: m * 2^-9, m <= 8
-  const uint32_t mant = u & 0x7FFFFFu;
-  uint32_t code = (uint32_t(e + 7) << 3) | (mant >> 20);
-  const uint32_t rem = mant & 0xFFFFFu;
-  if (rem > 0x80000u || (rem == 0x80000u && (code & 1u))) code += 1u;
-  return code > 0x7Eu ? 0x7Eu : code;
-}
-// Signed E4M3 (the FP8 projected-key cache): the magnitude as UE4M3 above, bit 7 the sign
-// (kept for negative values that round to zero, and for -0).
-QS_DEV uint32_t e4m3_encode(float x) {
-  return ue4m3_encode(fabsf(x)) | (signbit(x) ? 0x80u : 0u);
-}
 QS_DEV float ue4m3_decode(uint32_t c) {
   const uint32_t e = c >> 3, m = c & 7u;
   if (e == 0u) return float(m) * 0.001953125f;
@@ -126,7 +107,6 @@ QS_DEV void row_prep(const uint16_t* q, const float* Pg, float* qt_row, float* q
 // Advance seq_lens once every CTA of the append grid has read them ("last CTA" pattern).
 QS_DEV void finish_append(const AppendParams& a) {
   __shared__ int s_last;
-  if (a.keep_lens) return;      // the decode step advances the lengths at its end
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();

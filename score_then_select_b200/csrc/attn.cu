@@ -34,10 +34,9 @@
 //     online-softmax state (base 2, scale * log2 e folded into the logits). At the end of
 //     a chunk the four states are merged in a fixed order into the chunk's partial
 //     (max, sum, o).
-// Row merge, in the same kernel: the CTA that finishes a row's last chunk (counted on the
-// row's counter in the workspace) merges the row's chunk partials by log-sum-exp into the
-// output with its four consumer warps, while the other CTAs keep streaming. The last CTA
-// of the grid to finish resets the chunk-claim counter for the next launch.
+// attn_combine_kernel, launched behind this grid, merges each (row, query head)'s chunk
+// partials by log-sum-exp into the output (one CTA per row and head: the merge's L2 reads
+// are spread over the whole GPU instead of adding a serial tail to one CTA's work).
 //
 // Tensor-core mapping and online softmax: attn_warp_tile (attn_core.cuh).
 #include <cuda.h>
@@ -57,8 +56,6 @@ constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kAttnThreads = kConsumerThreads + 32;
 constexpr int kHalfBytes = kTileT * 128;         // 64 rows x 64 elements (one swizzled box column)
 
-constexpr int kRecCap = 32;       // rows whose chunk counts a CTA holds before adding them
-
 template <int D>
 struct AttnSmem {
   static constexpr int kHalves = D / 64;
@@ -68,11 +65,10 @@ struct AttnSmem {
   static constexpr int kMetaOff = kAttnStages * kStageBytes;        // u32 [stages][4]
   static constexpr int kBarOff = kMetaOff + kAttnStages * 16;       // u64 full[], empty[], rag[]
   static constexpr int kMlOff = kBarOff + 3 * kAttnStages * 8;      // f32 [2][m [4][8], l [4][8]]
-  static constexpr int kMiscOff = kMlOff + 2 * 64 * 4;              // i32 abort, i32 records, u64 barrier
+  static constexpr int kMiscOff = kMlOff + 2 * 64 * 4;              // i32 abort, u64 barrier
   static constexpr int kScrOff = kMiscOff + 16;                     // merge buffer
   static constexpr int kBufStride = D + 4;                          // floats per head (merge)
-  static constexpr int kRecOff = kScrOff + 2 * 8 * kBufStride * 4;   // i32 [kRecCap][row, chunks]
-  static constexpr int kUsed = kRecOff + kRecCap * 8;
+  static constexpr int kUsed = kScrOff + 2 * 8 * kBufStride * 4;
   static constexpr int kTotal = kUsed + 1024;                       // + alignment slack
 };
 static_assert(AttnSmem<128>::kTotal + 1024 <= 228 * 1024 / kAttnCtasPerSm,
@@ -103,8 +99,8 @@ constexpr uint32_t kMetaRag = 1u << 18, kMetaRagPhase = 1u << 19;
 // (else BF16 keys); the tile covers page slots 64..127 (else 0..63)
 constexpr uint32_t kMetaRawK = 1u << 20, kMetaHalf = 1u << 21;
 // NVFP4 key storage: layout of the K region of a stage for a tile of NVFP4 keys
-constexpr int kRawCodes = 0, kRawScales = 4096, kRawMu = 5120;
-constexpr uint32_t kRawBytes = 4096 + 1024 + 512;
+constexpr int kRawCodes = 0, kRawScales = 4096;
+constexpr uint32_t kRawBytes = 4096 + 1024;
 
 // Barrier of the four consumer warps on an mbarrier (count 4), bounded like every wait
 // here: a warp that gives up cannot leave the others waiting on a hardware barrier.
@@ -116,138 +112,11 @@ QS_DEV void consumer_sync(uint64_t* bar, uint32_t& phase, int lane, volatile int
   __syncwarp();
 }
 
-// Merge row `row`'s chunk partials into the output (the four consumer warps, thread ct):
-//   out[h][d] = sum_p 2^(m_p - M) o_p[d] / sum_p 2^(m_p - M) l_p, M = max_p m_p over
-//   partials with l_p > 0 (a row with no tokens -> 0); p in order, so the result is fixed.
-// Warp w first turns head w's (and w + 4's) chunk maxima and sums into weights and 1/den in
-// shared memory (w_buf, G x cpr + G floats); then each thread forms its outputs with all of
-// a head's partial loads in flight at once. Rows with more partials than w_buf holds take
-// the same sums in batches of 8 partials with a running maximum.
-template <int D>
-QS_DEV void attn_merge_row(const AttnParams& a, int row, int ct, float* w_buf, int w_cap,
-                           uint32_t& cphase, uint64_t* cbar, volatile int* s_abort) {
-  const int cpr = a.chunks_per_row, lane = ct & 31, warp = ct >> 5;
-  const size_t rq0 = size_t(row / a.Hkv) * (a.Hkv * a.G) + (row % a.Hkv) * a.G;
-  auto store = [&](size_t rq, int d, float r) {
-    if (a.out_bf16)
-      reinterpret_cast<uint16_t*>(a.out)[rq * D + d] = f32_to_bf16_rn(r);
-    else
-      reinterpret_cast<float*>(a.out)[rq * D + d] = r;
-  };
-  if (a.G * cpr + a.G <= w_cap) {
-    float* inv = w_buf + a.G * cpr;
-    for (int h = warp; h < a.G; h += kConsumerWarps) {
-      const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + (rq0 + h) * cpr;
-      float M = -INFINITY;
-      for (int p = lane; p < cpr; p += 32) {
-        const float2 v = __ldcg(ml + p);
-        if (v.y > 0.0f) M = fmaxf(M, v.x);
-      }
-#pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
-      float den = 0.0f;
-      for (int p = lane; p < cpr; p += 32) {
-        const float2 v = __ldcg(ml + p);
-        const float w = v.y > 0.0f ? ex2(v.x - M) : 0.0f;
-        w_buf[h * cpr + p] = w;
-        den += w * v.y;
-      }
-#pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(kFull, den, o2);
-      if (lane == 0) inv[h] = den > 0.0f ? 1.0f / den : 0.0f;
-    }
-    consumer_sync(cbar, cphase, lane, s_abort);
-    for (int idx = ct; idx < a.G * D; idx += kConsumerThreads) {
-      const int h = idx / D, d = idx - h * D;
-      const size_t rq = rq0 + h;
-      const float* po = a.part_o + rq * cpr * D + d;
-      const float* wh = w_buf + h * cpr;
-      float num = 0.0f;
-      int p = 0;
-      for (; p + 16 <= cpr; p += 16) {
-        float x[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) x[u] = __ldcg(po + size_t(p + u) * D);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) num += wh[p + u] * x[u];
-      }
-      for (; p < cpr; ++p) num += wh[p] * __ldcg(po + size_t(p) * D);
-      store(rq, d, num * inv[h]);
-    }
-    consumer_sync(cbar, cphase, lane, s_abort);          // w_buf is free again
-    return;
-  }
-  for (int idx = ct; idx < a.G * D; idx += kConsumerThreads) {
-    const int h = idx / D, d = idx - h * D;
-    const size_t rq = rq0 + h;
-    const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + rq * cpr;
-    const float* po = a.part_o + rq * cpr * D + d;
-    float M = -INFINITY, den = 0.0f, num = 0.0f;
-    for (int p0 = 0; p0 < cpr; p0 += 8) {
-      float2 v[8];
-      float x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const bool in = p0 + u < cpr;
-        v[u] = in ? __ldcg(ml + p0 + u) : make_float2(-INFINITY, 0.0f);
-        x[u] = in ? __ldcg(po + size_t(p0 + u) * D) : 0.0f;
-      }
-      float Mb = M;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (v[u].y > 0.0f) Mb = fmaxf(Mb, v[u].x);
-      if (Mb > M) {
-        const float f = M == -INFINITY ? 0.0f : ex2(M - Mb);
-        den *= f;
-        num *= f;
-        M = Mb;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float w = v[u].y > 0.0f ? ex2(v[u].x - M) : 0.0f;
-        den += w * v[u].y;
-        num += w * x[u];
-      }
-    }
-    store(rq, d, den > 0.0f ? num * (1.0f / den) : 0.0f);
-  }
-}
-
-// Add this CTA's recorded chunk counts to the rows' counters (the four consumer warps; one
-// fence first, so the chunk partials are visible before any count); a row whose count
-// reaches chunks_per_row is complete and this CTA merges it, then clears its counter.
-template <int D>
-QS_DEV void attn_count_rows(const AttnParams& a, int ct, volatile int* s_nrec, int* s_rec,
-                            float* s_buf, uint32_t& cphase, uint64_t* cbar, volatile int* s_abort) {
-  using SM = AttnSmem<D>;
-  const int lane = ct & 31;
-  __threadfence();
-  consumer_sync(cbar, cphase, lane, s_abort);
-  const int n = *s_nrec;
-  if (ct == 0) {
-    for (int i = 0; i < n; ++i) {
-      const unsigned c = unsigned(s_rec[2 * i + 1]);
-      const unsigned prev = atomicAdd(a.row_ctr + s_rec[2 * i], c);
-      s_rec[2 * i + 1] = prev + c == unsigned(a.chunks_per_row) ? 1 : 0;
-    }
-  }
-  consumer_sync(cbar, cphase, lane, s_abort);
-  for (int i = 0; i < n; ++i) {
-    if (!s_rec[2 * i + 1] || *s_abort) continue;
-    const int row = s_rec[2 * i];
-    __threadfence();
-    attn_merge_row<D>(a, row, ct, s_buf, 2 * 8 * SM::kBufStride, cphase, cbar, s_abort);
-    if (ct == 0) a.row_ctr[row] = 0u;                      // ready for the next launch
-  }
-  consumer_sync(cbar, cphase, lane, s_abort);
-  if (ct == 0) *s_nrec = 0;
-}
-
 // ======================= consumers: online softmax, chunk partials, row merge ==========
 template <int D, bool V_F16, bool AGG_F16, bool KQ4>
 QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uint64_t* full,
                          uint64_t* empty, uint64_t* rag, float* s_ml, volatile int* s_abort,
-                         volatile int* s_nrec, int* s_rec, uint64_t* cbar, float* s_buf) {
+                         uint64_t* cbar, float* s_buf) {
   using SM = AttnSmem<D>;
   constexpr int KS = D / 16;
   constexpr int NS = kAttnStages;
@@ -262,6 +131,7 @@ QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uin
 #pragma unroll
   for (int m = 0; m < KS; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.0f;
   uint32_t qb[KS][2];
+  float qmu0 = 0.0f, qmu1 = 0.0f;                          // NVFP4 keys: q . mu, heads h0, h0 + 1
   for (int t = 0;; ++t) {
     const int s = t % NS;
     if (!wait_or_abort(&full[s], (t / NS) & 1, s_abort)) break;
@@ -285,6 +155,32 @@ QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uin
       l0 = l1 = 0.0f;
 #pragma unroll
       for (int m = 0; m < KS; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.0f;
+      if constexpr (KQ4) {
+        // q . mu of heads h0 and h0 + 1: lane slice j = lane / 4 covers dims 16j .. 16j + 15,
+        // the eight slices summed by shuffles (every lane of a t = lane % 4 class agrees)
+        const int j = lane >> 2;
+        const float4* mu4 = reinterpret_cast<const float4*>(a.key_center + size_t(row) * D + 16 * j);
+        const uint16_t* qsb = reinterpret_cast<const uint16_t*>(st + 2 * SM::kTileBytes);
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          const float4 mv = __ldg(mu4 + i4);
+          const float mu[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int d = 16 * j + 4 * i4 + e;
+            if (h0 < a.G) s0 = fmaf(bf16_to_f32(qsb[h0 * D + d]), mu[e], s0);
+            if (h0 + 1 < a.G) s1 = fmaf(bf16_to_f32(qsb[(h0 + 1) * D + d]), mu[e], s1);
+          }
+        }
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+          s0 += __shfl_xor_sync(kFull, s0, o2);
+          s1 += __shfl_xor_sync(kFull, s1, o2);
+        }
+        qmu0 = s0;
+        qmu1 = s1;
+      }
     }
     const uint32_t kst = smem_u32(st), vst = smem_u32(st + SM::kTileBytes);
 
@@ -293,8 +189,7 @@ QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uin
     const bool v0 = (vm >> (tl & 31)) & 1u, v1 = (vm >> ((tl + 8) & 31)) & 1u;
     const auto sw = [](int r, int c) { return swz(r, c); };
     if (KQ4 && (info & kMetaRawK)) {
-      const KFragNvfp4 kf(st + kRawCodes, st + kRawScales,
-                          reinterpret_cast<const float*>(st + kRawMu), gk,
+      const KFragNvfp4 kf(st + kRawCodes, st + kRawScales, gk, qmu0, qmu1,
                           (info & kMetaHalf) ? 64 : 0, warp, lane);
       attn_warp_tile<D, V_F16, AGG_F16>(kf, vst, qb, v0, v1, a.scale_log2, m0, m1, l0, l1, o,
                                         warp, lane, sw);
@@ -401,25 +296,8 @@ QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uin
           }
         }
       }
-      // the chunk's partial is out: record its row (the count is added to the row's counter
-      // once this CTA's work is done, behind one fence, off the streaming path)
-      if (lane == 0) {
-        const int n = *s_nrec;
-        if (n > 0 && s_rec[2 * (n - 1)] == row) {
-          s_rec[2 * (n - 1) + 1] += 1;
-        } else {
-          s_rec[2 * n] = row;
-          s_rec[2 * n + 1] = 1;
-          *s_nrec = n + 1;
-        }
-      }
     }
-    consumer_sync(cbar, cphase, lane, s_abort);
-    if (*s_nrec == kRecCap && !*s_abort)                   // the record is full: add it now
-      attn_count_rows<D>(a, tid, s_nrec, s_rec, s_buf, cphase, cbar, s_abort);
   }
-  if (*s_nrec > 0 && !*s_abort)
-    attn_count_rows<D>(a, tid, s_nrec, s_rec, s_buf, cphase, cbar, s_abort);
 }
 
 template <int D, bool V_F16, bool AGG_F16, bool KQ4>
@@ -438,8 +316,6 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
   uint64_t* rag = empty + NS;       // ragged-run copies of a stage (one cp.async arrival per lane)
   float* s_ml = reinterpret_cast<float*>(smem + SM::kMlOff);         // [2][m [4][8], l [4][8]]
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SM::kMiscOff);
-  volatile int* s_nrec = reinterpret_cast<volatile int*>(smem + SM::kMiscOff + 4);
-  int* s_rec = reinterpret_cast<int*>(smem + SM::kRecOff);
   uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + SM::kMiscOff + 8);
   float* s_buf = reinterpret_cast<float*>(smem + SM::kScrOff);
 
@@ -453,7 +329,6 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     }
     mbar_init(cbar, kConsumerWarps);
     *s_abort = 0;
-    *s_nrec = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -482,7 +357,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
         const int tin0 = (c - r.row * cpr) * ktiles, j = lane >> (6 - lg_hb);
         if (j < min(ktiles, tpr - tin0)) {
           r.sl = (tin0 + j) * kTileT + ((lane & (rpt - 1)) << lg_hb);
-          r.L = a.row_lens ? a.row_lens[r.row] : a.seq_lens[r.row / a.Hkv] + a.len_add;
+          r.L = a.row_lens ? a.row_lens[r.row] : a.seq_lens[r.row / a.Hkv];
           const int e = r.sl >> lgS;
           if constexpr (KQ4) {                             // the row's kept (BF16) blocks
             r.k0 = a.kept[2 * r.row];
@@ -667,7 +542,7 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
           }
           if constexpr (KQ4) {
             // NVFP4 keys, by the two K lanes: the tile's 64 token rows of each of the 4 code
-            // chunks (1 KB each), the page's 1 KB of scales and the row's centre
+            // chunks (1 KB each) and the page's 1 KB of scales
             if (rr && box_lane && box_v == 0) {
               const size_t ph = size_t(ry >> 7);             // page * Hkv + head
               const uint8_t* cb = a.k_codes + ph * kNvfp4PageCodeBytes + (ry & 127) * 16;
@@ -676,8 +551,6 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
               bulk_g2s(st + kRawCodes + (c0 + 1) * 1024, cb + (c0 + 1) * 2048, 1024u, &full[s]);
               if (box_h == 0)
                 bulk_g2s(st + kRawScales, a.k_scales + ph * kNvfp4PageScaleBytes, 1024u, &full[s]);
-              else
-                bulk_g2s(st + kRawMu, a.key_center + size_t(row) * D, uint32_t(D * 4), &full[s]);
             }
           }
         }
@@ -710,25 +583,67 @@ __global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     }
     __syncwarp();
   } else {
-    attn_consume<D, V_F16, AGG_F16, KQ4>(a, smem, meta, full, empty, rag, s_ml, s_abort, s_nrec,
-                                         s_rec, cbar, s_buf);
+    attn_consume<D, V_F16, AGG_F16, KQ4>(a, smem, meta, full, empty, rag, s_ml, s_abort, cbar,
+                                         s_buf);
   }
-  // the grid's last CTA to finish resets the chunk-claim counter for the next launch (every
-  // CTA has issued its last claim by now)
   __syncthreads();
-  if (tid == 0) {
-    if (*s_abort) flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_ATTN, blockIdx.x);
-    __threadfence();
-    if (atomicAdd(a.hdr + kCtrAttnDone, 1u) == gridDim.x - 1) {
-      a.hdr[kCtrAttnNext] = 0u;
-      a.hdr[kCtrAttnDone] = 0u;
-      // the decode step's lengths advance once every CTA has read them
-      if (a.lens_out)
-        for (int b = 0; b < a.rows / a.Hkv; ++b) a.lens_out[b] += a.len_add;
-    }
-  }
+  if (tid == 0 && *s_abort) flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_ATTN, blockIdx.x);
 }
 
+
+// ---------------------------------------------------------------- combine
+// One CTA per (row, query head): the head's chunk partials -> output by log-sum-exp,
+//   out[d] = sum_p 2^(m_p - M) o_p[d] / sum_p 2^(m_p - M) l_p  (a row with no tokens -> 0).
+// Thread d owns output element d; all of its partial loads are in flight together.
+// Waits for the attention grid (programmatic dependent launch), then resets the chunk
+// claim counter for the next attention launch.
+template <int D>
+__global__ void __launch_bounds__(D) attn_combine_kernel(const AttnParams a) {
+  extern __shared__ float s_w[];                           // [cpr] weights, then 1/den
+  pdl_wait();
+  const int row = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int cpr = a.chunks_per_row;
+  if (row == 0 && h == 0 && tid == 0) a.hdr[kCtrAttnNext] = 0u;
+  const size_t rq = size_t(row / a.Hkv) * (a.Hkv * a.G) + (row % a.Hkv) * a.G + h;
+  const float* ml = a.part_ml + rq * cpr * 2;
+  if (tid < 32) {
+    float M = -INFINITY;
+    for (int p = lane; p < cpr; p += 32) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(ml) + p);
+      if (v.y > 0.0f) M = fmaxf(M, v.x);
+    }
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o2));
+    float den = 0.0f;
+    for (int p = lane; p < cpr; p += 32) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(ml) + p);
+      const float w = v.y > 0.0f ? ex2(v.x - M) : 0.0f;
+      s_w[p] = w;
+      den += w * v.y;
+    }
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(kFull, den, o2);
+    if (lane == 0) s_w[cpr] = den > 0.0f ? 1.0f / den : 0.0f;
+  }
+  __syncthreads();
+  const float* po = a.part_o + rq * cpr * D + tid;
+  float acc = 0.0f;
+  int p = 0;
+  for (; p + 8 <= cpr; p += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldcg(po + size_t(p + u) * D);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += s_w[p + u] * v[u];
+  }
+  for (; p < cpr; ++p) acc += s_w[p] * __ldcg(po + size_t(p) * D);
+  const float r = acc * s_w[cpr];
+  const size_t oi = rq * D + tid;
+  if (a.out_bf16)
+    reinterpret_cast<uint16_t*>(a.out)[oi] = f32_to_bf16_rn(r);
+  else
+    reinterpret_cast<float*>(a.out)[oi] = r;
+}
 
 // ------------------------------------------------------------------ tensor maps (host)
 // A 2-D map over one cache tensor viewed as [num_pages * Hkv * 128 rows][d] 16-bit
@@ -785,7 +700,11 @@ static cudaError_t launch_attn_t(const AttnParams& a, const CUtensorMap& mk, con
   const int smem = AttnSmem<D>::kTotal;
   const cudaError_t attr = set_smem_limit(k, smem);
   if (attr != cudaSuccess) return attr;
-  return launch_k(k, dim3(grid), dim3(kAttnThreads), smem, s, pdl, a, mk, mv);
+  cudaError_t e = launch_k(k, dim3(grid), dim3(kAttnThreads), smem, s, pdl, a, mk, mv);
+  if (e != cudaSuccess) return e;
+  // the row merge, launched behind the attention grid (it waits for it before reading)
+  const size_t csmem = size_t(a.chunks_per_row + 1) * sizeof(float);
+  return launch_k(attn_combine_kernel<D>, dim3(a.rows, a.G), dim3(D), csmem, s, true, a);
 }
 
 cudaError_t launch_attn(const Plan& p, const AttnParams& a_in, cudaStream_t s, bool pdl) {

@@ -29,29 +29,31 @@ struct KFragLdsm {
   QS_DEV void operator()(int ks, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) const {
     ldsm_x4(a0, a1, a2, a3, kst + swz(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
   }
+  QS_DEV void fix(float (&)[4]) const {}     // the accumulator is the logit
 };
 
-// K fragments decoded from one 64-token tile of NVFP4 keys in shared memory (the storage
-// variant of "Jet-QSparse ...", Full text): each element becomes
-// bf16_rne(fp32(fp32(e * sigma) * g_k) + mu), e * sigma exact in float32.
+// K fragments of one 64-token tile of NVFP4 keys in shared memory (the storage variant of
+// "Jet-QSparse ...", Full text). The attended key is the dequantised, un-centred value
+// k = g_k (e sigma) + mu. The A operand is e * sigma, which is exact in BF16 (an E2M1 value
+// has at most 2 significant bits and a UE4M3 scale 4); the products with the BF16 query
+// are then exact and the MMA sums them in float32, so the logit q . k is
+// g_k (q . (e sigma)) + q . mu, formed in `fix` from the accumulator and the head's q . mu.
 //   codes:  [4 chunks][64 tokens][16 bytes]; chunk c holds elements 32c..32c+31 of a
 //           token, element 2i + u in nibble u of byte i;
 //   scales: the page's 1,024 bytes; token slot m's scale of elements 16j..16j+15 at
 //           (j / 4) * 512 + 16 * (m % 32) + 4 * (m / 32) + j % 4; m0 = the page slot of
-//           the tile's first token;
-//   mu:     the row's centre, d floats.
+//           the tile's first token.
 // This lane's rows are tokens r0 = 16 warp + lane / 4 and r0 + 8 of the tile, its elements
 // 2t, 2t + 1, 2t + 8, 2t + 9 of each k-step (t = lane % 4), as the mma A fragment holds them.
 struct KFragNvfp4 {
   const uint8_t* codes;
-  const float* mu;
-  float gk;
+  float gk, qmu0, qmu1;    // g_k; q . mu of this lane's heads 2t and 2t + 1
   int r0, t;
   uint32_t sc[2][2];       // scale words: [row r0, r0 + 8][elements 0-63, 64-127]
 
-  QS_DEV KFragNvfp4(const uint8_t* codes_, const uint8_t* scales, const float* mu_, float gk_,
-                    int m0, int warp, int lane)
-      : codes(codes_), mu(mu_), gk(gk_), r0(warp * 16 + (lane >> 2)), t(lane & 3) {
+  QS_DEV KFragNvfp4(const uint8_t* codes_, const uint8_t* scales, float gk_, float qmu0_,
+                    float qmu1_, int m0, int warp, int lane)
+      : codes(codes_), gk(gk_), qmu0(qmu0_), qmu1(qmu1_), r0(warp * 16 + (lane >> 2)), t(lane & 3) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int m = m0 + r0 + 8 * r;
@@ -60,25 +62,34 @@ struct KFragNvfp4 {
         sc[r][h] = *reinterpret_cast<const uint32_t*>(scales + h * 512 + 16 * (m & 31) + 4 * (m >> 5));
     }
   }
-  // byte t of w (two elements) -> bf16x2
-  QS_DEV uint32_t dec(uint32_t w, float sig, float2 m) const {
+  // sigma of k-step ks of row r as an f16 pair (both halves)
+  QS_DEV uint32_t sig2(int r, int ks) const {
+    const uint32_t f = e4m3x2_to_f16x2(sc[r][ks >> 2] >> (8 * (ks & 3))) & 0xffffu;
+    return f | (f << 16);
+  }
+  // byte t of w (two codes) times sigma -> bf16x2, exact
+  QS_DEV uint32_t dec(uint32_t w, uint32_t s2) const {
     const uint32_t e = e2m1x2_to_f16x2(w >> (8 * t));
-    const float lo = __fadd_rn(__fmul_rn(__fmul_rn(f16_lo(e), sig), gk), m.x);
-    const float hi = __fadd_rn(__fmul_rn(__fmul_rn(f16_hi(e), sig), gk), m.y);
-    return pack_bf16x2(lo, hi);
+    uint32_t p;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p) : "r"(e), "r"(s2));
+    return __byte_perm(__float_as_uint(f16_lo(p)), __float_as_uint(f16_hi(p)), 0x7632);
   }
   QS_DEV void operator()(int ks, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) const {
     const int c = ks >> 1, h = ks & 1;
     const uint2 w0 = *reinterpret_cast<const uint2*>(codes + c * 1024 + r0 * 16 + 8 * h);
     const uint2 w1 = *reinterpret_cast<const uint2*>(codes + c * 1024 + (r0 + 8) * 16 + 8 * h);
-    const float s0 = f16_lo(e4m3x2_to_f16x2(sc[0][ks >> 2] >> (8 * (ks & 3))));
-    const float s1 = f16_lo(e4m3x2_to_f16x2(sc[1][ks >> 2] >> (8 * (ks & 3))));
-    const float2 m01 = *reinterpret_cast<const float2*>(mu + 16 * ks + 2 * t);
-    const float2 m89 = *reinterpret_cast<const float2*>(mu + 16 * ks + 2 * t + 8);
-    a0 = dec(w0.x, s0, m01);
-    a1 = dec(w1.x, s1, m01);
-    a2 = dec(w0.y, s0, m89);
-    a3 = dec(w1.y, s1, m89);
+    const uint32_t s0 = sig2(0, ks), s1 = sig2(1, ks);
+    a0 = dec(w0.x, s0);
+    a1 = dec(w1.x, s1);
+    a2 = dec(w0.y, s0);
+    a3 = dec(w1.y, s1);
+  }
+  // accumulator (tokens r0 / r0 + 8 x heads 2t, 2t + 1) -> logits q . k
+  QS_DEV void fix(float (&c)[4]) const {
+    c[0] = fmaf(c[0], gk, qmu0);
+    c[1] = fmaf(c[1], gk, qmu1);
+    c[2] = fmaf(c[2], gk, qmu0);
+    c[3] = fmaf(c[3], gk, qmu1);
   }
 };
 
@@ -99,6 +110,7 @@ QS_DEV void attn_warp_tile(const KF& kf, uint32_t vst, const uint32_t (&qb)[D / 
     kf(ks, a0, a1, a2, a3);
     mma_bf16(c, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
   }
+  kf.fix(c);
   const float x0 = valid0 ? c[0] * scale_log2 : -INFINITY;
   const float x1 = valid0 ? c[1] * scale_log2 : -INFINITY;
   const float x2 = valid1 ? c[2] * scale_log2 : -INFINITY;

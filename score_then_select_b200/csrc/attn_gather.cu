@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(128, 2) attn_gather_kernel(const AttnParams a)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   int n = a.n_sel[row];
-  int L = a.seq_lens[b] + a.len_add;
+  int L = a.seq_lens[b];
   if (n < 0 || n > a.budget || L < 0) {
     if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_ATTN, uint32_t(row));
     n = 0;
@@ -266,17 +266,6 @@ __global__ void __launch_bounds__(128, 2) attn_gather_kernel(const AttnParams a)
   }
   __syncthreads();
   if (s_last) gather_merge_row<D>(a, row, smem);
-  // the grid's last CTA advances the decode step's lengths (every CTA has read them)
-  if (a.lens_out) {
-    __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      if (atomicAdd(a.hdr + kCtrAttnDone, 1u) == gridDim.x * gridDim.y - 1) {
-        a.hdr[kCtrAttnDone] = 0u;
-        for (int bb = 0; bb < a.rows / a.Hkv; ++bb) a.lens_out[bb] += a.len_add;
-      }
-    }
-  }
 }
 
 // The last split of row `row` to finish merges all of the row's splits (LSE combine).

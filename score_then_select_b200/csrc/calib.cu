@@ -212,7 +212,7 @@ cudaError_t launch_calibrate(const CalibParams& a, cudaStream_t s) {
   moments_kernel<<<grid, kCalThreads, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int d = a.d, half = d / 2;
+  const int d = a.d;
   auto bytes = [](int dd) {
     return size_t(dd) * dd * 8 + size_t(dd) * dd * 4 + size_t(dd / 2) * 2 * 8 +
            size_t(dd / 2) * 2 * 4 + 64 * 8 + size_t(dd) * 4;

@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(128) kept_blocks_kernel(const KeptParams p) {
   pdl_wait();                  // the errors (and the step before) come from earlier kernels
   pdl_trigger();
   const int row = blockIdx.x, b = row / p.Hkv;
-  const int L = max(0, p.seq_lens[b] + p.len_add);
+  const int L = max(0, p.seq_lens[b]);
   const float* err = p.block_err + size_t(row) * p.nb_stride;
   const int complete = min(L / kPage, p.nb_stride);
   int k1 = -1, k2 = -1;

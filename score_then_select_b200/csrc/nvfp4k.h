@@ -22,7 +22,7 @@ struct KeptParams {
   const float* block_err;     // [rows][nb_stride]
   const int32_t* seq_lens;
   int32_t* kept;              // [rows][2], -1: none
-  int rows, Hkv, nb_stride, n_keep, len_add;
+  int rows, Hkv, nb_stride, n_keep;
 };
 cudaError_t launch_kept_blocks(const KeptParams& p, cudaStream_t s, bool pdl);
 

@@ -177,6 +177,25 @@ QS_DEV uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(uint16_t(two_codes)));
   return r;
 }
+// UE4M3 (bias 7, 3 mantissa bits, subnormal step 2^-9, largest finite 448 = 0x7E):
+// nearest even, saturating; non-positive and NaN inputs give code 0.
+QS_DEV uint32_t ue4m3_encode(float sf) {
+  if (!(sf > 0.0f)) return 0u;
+  if (sf >= 448.0f) return 0x7Eu;
+  const uint32_t u = __float_as_uint(sf);
+  const int e = int(u >> 23) - 127;
+  if (e < -6) return __float2uint_rn(sf * 512.0f);  // subnormal range: m * 2^-9, m <= 8
+  const uint32_t mant = u & 0x7FFFFFu;
+  uint32_t code = (uint32_t(e + 7) << 3) | (mant >> 20);
+  const uint32_t rem = mant & 0xFFFFFu;
+  if (rem > 0x80000u || (rem == 0x80000u && (code & 1u))) code += 1u;
+  return code > 0x7Eu ? 0x7Eu : code;
+}
+// Signed E4M3 (the FP8 projected-key cache): the magnitude as UE4M3 above, bit 7 the sign
+// (kept for negative values that round to zero, and for -0).
+QS_DEV uint32_t e4m3_encode(float x) {
+  return ue4m3_encode(fabsf(x)) | (signbit(x) ? 0x80u : 0u);
+}
 // two E2M1 codes (low byte of v: the low nibble is the first element) -> f16x2, exact
 QS_DEV uint32_t e2m1x2_to_f16x2(uint32_t v) {
   uint32_t r;

@@ -34,7 +34,6 @@ constexpr int kChunkTilesMax = 8;   // attention work unit: up to 8 tiles (512 s
 constexpr int kChunksPerCta = 6;    // chunk size target: about this many chunks per CTA
 constexpr int kTmaMinTilesPerCta = 40;  // auto path: tile pipeline from this much work per CTA
 constexpr int kCtrAttnNext = 17;    // header word: next attention chunk to claim
-constexpr int kCtrAttnDone = 18;    // header word: attention CTAs finished (last one resets)
 
 // Workspace carve-up (byte offsets); computed identically by qs_workspace_size and calls.
 struct WsLayout {
@@ -93,9 +92,6 @@ struct AppendParams {
   float* qt;
   int batch, Hkv, G, d, r, max_new, max_pages_per_seq, num_pages, max_context;
   int S;                     // block size (centroid sums)
-  // 1: leave seq_lens as they are (the decode step reads them as seq_lens + 1 and its
-  // attention kernel advances them at the end); 0: advance them by n_new
-  int keep_lens;
 };
 
 struct BlockErrParams {
@@ -169,12 +165,6 @@ struct ScoreParams {
   // the query side (q~, or the NVFP4 query tiles and g_q), so the page stream may start
   // before waiting for it; 0: wait for it first (it may still be writing seq_lens)
   int early_stream;
-  // rank r, decode step: the kernel before is the one-token writer, which leaves seq_lens
-  // unchanged (the step's length is seq_lens + len_add) and writes only the newest token's
-  // slot. The scan computes q~ itself from q and P (inline_qt), streams every page at once,
-  // and waits for the writer only before copying a row's last page (wait_last).
-  const float* P;
-  int len_add, inline_qt, wait_last;
 };
 
 struct SelectParams {
@@ -185,7 +175,6 @@ struct SelectParams {
   int32_t* n_sel;
   uint32_t* hdr;
   int rows, Hkv, S, nb_stride, budget, force_sink, force_last, n_keep;
-  int len_add;               // the step's length is seq_lens + len_add
 };
 
 struct AttnParams {
@@ -209,8 +198,6 @@ struct AttnParams {
   int gsplits, g_tokens_per_split;   // gather kernel split plan
   int out_bf16;
   float scale_log2;          // softmax scale * log2(e)
-  int len_add;               // the step's length is seq_lens + len_add
-  int32_t* lens_out;         // non-null: the grid's last CTA adds len_add to lens_out[b]
   // NVFP4 key storage: keys from the scoring cache (codes, scales, g_k, the row's centre),
   // except the row's kept blocks (kept[row][0..1], -1: none), which come from k
   const uint8_t* k_codes;

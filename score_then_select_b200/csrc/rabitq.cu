@@ -105,7 +105,6 @@ cudaError_t launch_rq_prep(const RqPrepParams& a, cudaStream_t s) {
 }
 
 // ============================================================ scan
-constexpr int kRqScanWarps = 8;
 
 // Merge of log-sum-exp states: (m, l) stands for l * e^m.
 QS_DEV void lse_merge(float& m, float& l, float m2, float l2) {
@@ -119,187 +118,219 @@ QS_DEV void lse_merge(float& m, float& l, float m2, float l2) {
   m = mm;
 }
 
-// Persistent grid; a unit is one (sequence b, page p, KV head g), g fastest so that a
-// page's heads (contiguous in the cache) go to neighbouring warps. Warp w of the grid takes
-// units w, w + W, ... and loads the next unit's codes, factors and query code before it
-// scores the current one, so every warp keeps a unit's loads in flight.
-struct RqUnit {
-  int row, pi, L;
-  bool ok;
-  const uint8_t* pg;
+// Persistent grid, one producer warp and four consumer warps per CTA. A unit is one
+// (sequence b, page p, KV head g), g fastest (a page's heads are contiguous in the cache);
+// the units are split evenly over the CTAs. The producer's lanes resolve 32 units' pages at
+// a time and lane 0 streams each unit's whole (page, head) record (code bits and factors,
+// 2,560 bytes at d = 128) with one bulk copy into a 16-stage shared-memory ring, completion
+// counted on the stage's mbarrier; units past a row's length are skipped. Consumer warp c
+// scores units c, c + 4, ...: lane l the token slots l + 32 k from shared memory.
+constexpr int kRqConsumers = 4;
+constexpr int kRqThreads = 32 * (1 + kRqConsumers);
+constexpr int kRqStages = 16;
+
+template <int D>
+struct RqShape {
+  static constexpr int kPageBytes = kPage * (D / 8) + kPage * 4;
+  static constexpr int kSmem = kRqStages * kPageBytes + 2 * kRqStages * 8 + kRqStages * 16;
 };
 
-template <int D>
-QS_DEV RqUnit rq_unit(const RqScoreParams& a, long long u, int max_pages) {
-  RqUnit x{0, 0, 0, false, nullptr};
-  const long long per_b = (long long)max_pages * a.Hkv;
-  const int b = int(u / per_b);
-  const int rem = int(u - (long long)b * per_b);
-  x.pi = rem / a.Hkv;
-  const int g = rem - x.pi * a.Hkv;
-  x.row = b * a.Hkv + g;
-  int L = a.seq_lens[b];
-  if (L > a.max_context) {
-    if (x.pi == 0 && g == 0 && (threadIdx.x & 31) == 0)
-      flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SCORE, uint32_t(b));
-    L = a.max_context;
-  }
-  x.L = L;
-  const int pages = L > 0 ? (L + kPage - 1) / kPage : 0;
-  if (x.pi >= pages) return x;                         // past the row's tokens: nothing
-  int page = -1;
-  if (x.pi < a.max_pages_per_seq) page = a.page_table[size_t(b) * a.max_pages_per_seq + x.pi];
-  if (page < 0 || page >= a.num_pages) {
-    if ((threadIdx.x & 31) == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SCORE, uint32_t(x.row));
-    return x;
-  }
-  constexpr int PB = kPage * (D / 8) + kPage * 4;
-  x.pg = a.proxy + (size_t(page) * a.Hkv + g) * PB;
-  x.ok = true;
-  return x;
-}
-
-template <int D>
-struct RqLoad {                                        // one lane's share of a unit's codes
-  uint32_t code[4][D / 32];
-  float gk[4];
-};
-
-template <int D>
-QS_DEV void rq_load(const RqScoreParams& a, const RqUnit& x, int lane, RqLoad<D>& r) {
-  constexpr int W = D / 32;
-  if (!x.ok) return;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int slot = lane + 32 * k;
-    if constexpr (W == 4) {
-      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(x.pg + slot * 16));
-      r.code[k][0] = v.x;
-      r.code[k][1] = v.y;
-      r.code[k][2] = v.z;
-      r.code[k][3] = v.w;
-    } else {
-      const uint2 v = __ldcs(reinterpret_cast<const uint2*>(x.pg + slot * 8));
-      r.code[k][0] = v.x;
-      r.code[k][1] = v.y;
-    }
-    r.gk[k] = __ldcs(reinterpret_cast<const float*>(x.pg + kPage * (D / 8)) + slot);
-  }
-}
-
 template <int D, int S>
-QS_DEV void rq_score_unit(const RqScoreParams& a, const RqUnit& x, const RqLoad<D>& r, int lane) {
-  constexpr int W = D / 32;
-  // the row's query code (a few hundred bytes per row, cached close to the SM)
-  const uint32_t* qc = a.qcode + size_t(x.row) * kRqRowWords;
-  uint32_t plane[kRqBits][W];
-#pragma unroll
-  for (int p = 0; p < kRqBits; ++p)
-#pragma unroll
-    for (int w = 0; w < W; ++w) plane[p][w] = __ldg(qc + p * W + w);
-  const float delta = __uint_as_float(__ldg(qc + kRqDelta)), vl = __uint_as_float(__ldg(qc + kRqVl));
-  const float shift = __uint_as_float(__ldg(qc + kRqShift));
-  const int Q = int(__ldg(qc + kRqQsum));
-  float m[4], l[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    int A = 0, B = 0;
-#pragma unroll
-    for (int w = 0; w < W; ++w) {
-      B += __popc(r.code[k][w]);
-#pragma unroll
-      for (int p = 0; p < kRqBits; ++p) A += __popc(r.code[k][w] & plane[p][w]) << p;
+__global__ void __launch_bounds__(kRqThreads, 4) rq_score_kernel(const RqScoreParams a) {
+  using SH = RqShape<D>;
+  constexpr int W = D / 32, PB = SH::kPageBytes;
+  extern __shared__ __align__(128) uint8_t rq_smem[];
+  uint8_t* slots = rq_smem;                                        // [stages][PB]
+  uint64_t* full = reinterpret_cast<uint64_t*>(rq_smem + kRqStages * PB);
+  uint64_t* empty = full + kRqStages;
+  int4* info = reinterpret_cast<int4*>(empty + kRqStages);         // {row, page idx, L, page}
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRqStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    const float est = r.gk[k] * (delta * float(2 * A - Q) + vl * float(2 * B - D)) + shift;
-    const bool valid = x.pi * kPage + lane + 32 * k < x.L;
-    m[k] = valid ? a.scale * est : -INFINITY;
-    l[k] = valid ? 1.0f : 0.0f;
+    fence_mbar_init();
   }
-  float* out = a.scores + size_t(x.row) * a.nb_stride + size_t(x.pi) * (kPage / S);
-  if constexpr (S < 32) {
-    // a block = S neighbouring lanes of one k
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float mk = m[k], lk = l[k];
-#pragma unroll
-      for (int o = 1; o < S; o <<= 1) {
-        const float m2 = __shfl_xor_sync(kFull, mk, o), l2 = __shfl_xor_sync(kFull, lk, o);
-        lse_merge(mk, lk, m2, l2);
-      }
-      if ((lane & (S - 1)) == 0) out[(lane + 32 * k) / S] = lk > 0.0f ? mk + logf(lk) : -INFINITY;
-    }
-  } else {
-    // a block = S / 32 consecutive k of every lane
-    constexpr int KB = S / 32;
-#pragma unroll
-    for (int k0 = 0; k0 < 4; k0 += KB) {
-      float mk = m[k0], lk = l[k0];
-#pragma unroll
-      for (int k = k0 + 1; k < k0 + KB; ++k) lse_merge(mk, lk, m[k], l[k]);
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float m2 = __shfl_xor_sync(kFull, mk, o), l2 = __shfl_xor_sync(kFull, lk, o);
-        lse_merge(mk, lk, m2, l2);
-      }
-      if (lane == 0) out[(32 * k0) / S] = lk > 0.0f ? mk + logf(lk) : -INFINITY;
-    }
-  }
-}
-
-template <int D, int S>
-__global__ void __launch_bounds__(kRqScanWarps * 32) rq_score_kernel(const RqScoreParams a) {
-  const int lane = threadIdx.x & 31;
+  __syncthreads();
   const int max_pages = a.nb_stride / (kPage / S);
-  const long long units = (long long)a.batch * max_pages * a.Hkv;
-  const long long stride = (long long)gridDim.x * kRqScanWarps;
-  long long u = (long long)blockIdx.x * kRqScanWarps + (threadIdx.x >> 5);
-  if (u >= units) return;
-  RqUnit x = rq_unit<D>(a, u, max_pages);
-  RqLoad<D> cur;
-  rq_load<D>(a, x, lane, cur);
-  while (true) {
-    const long long un = u + stride;
-    RqUnit xn{0, 0, 0, false, nullptr};
-    RqLoad<D> nxt;
-    if (un < units) {
-      xn = rq_unit<D>(a, un, max_pages);
-      rq_load<D>(a, xn, lane, nxt);                    // in flight while this unit is scored
+  const long long U = (long long)a.batch * max_pages * a.Hkv;
+  const long long u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
+  const int n_units = int(u1 - u0);
+
+  if (warp == 0) {
+    // ---------------- producer
+    bool dead = false;
+    for (int k0 = 0; k0 < n_units && !dead; k0 += 32) {
+      int row = 0, pi = 0, L = 0, page = -1;
+      if (k0 + lane < n_units) {
+        const long long u = u0 + k0 + lane;
+        const long long per_b = (long long)max_pages * a.Hkv;
+        const int b = int(u / per_b);
+        const int rem = int(u - (long long)b * per_b);
+        pi = rem / a.Hkv;
+        const int g = rem - pi * a.Hkv;
+        row = b * a.Hkv + g;
+        L = a.seq_lens[b];
+        if (L > a.max_context || L < 0) {
+          if (pi == 0 && g == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SCORE, uint32_t(b));
+          L = L < 0 ? 0 : a.max_context;
+        }
+        const int pages = (L + kPage - 1) / kPage;
+        if (pi < pages) {
+          page = pi < a.max_pages_per_seq ? a.page_table[size_t(b) * a.max_pages_per_seq + pi] : -1;
+          if (page < 0 || page >= a.num_pages) {
+            flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SCORE, uint32_t(row));
+            page = -1;
+          }
+        } else {
+          page = -2;                                   // past the row's tokens: nothing
+        }
+      }
+      const int m = min(32, n_units - k0);
+      for (int j = 0; j < m; ++j) {
+        const int jrow = __shfl_sync(kFull, row, j), jp = __shfl_sync(kFull, pi, j);
+        const int jL = __shfl_sync(kFull, L, j), jpage = __shfl_sync(kFull, page, j);
+        if (lane == 0) {
+          const int k = k0 + j;
+          const int s = k % kRqStages;
+          if (!mbar_wait(&empty[s], (uint32_t(k / kRqStages) & 1u) ^ 1u)) {
+            flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_SCORE, uint32_t(k));
+            dead = true;
+          } else {
+            info[s] = make_int4(jrow, jp, jL, jpage);
+            if (jpage >= 0) {
+              const int g = jrow % a.Hkv;
+              mbar_arrive_expect_tx(&full[s], uint32_t(PB));
+              bulk_g2s(slots + s * PB, a.proxy + (size_t(jpage) * a.Hkv + g) * PB, uint32_t(PB),
+                       &full[s]);
+            } else {
+              mbar_arrive(&full[s]);
+            }
+          }
+        }
+        dead = __shfl_sync(kFull, int(dead), 0) != 0;
+        if (dead) break;
+      }
     }
-    if (x.ok) rq_score_unit<D, S>(a, x, cur, lane);
-    if (un >= units) break;
-    u = un;
-    x = xn;
-    cur = nxt;
+    return;
+  }
+
+  // ---------------- consumers
+  const int c = warp - 1;
+  for (int k = c; k < n_units; k += kRqConsumers) {
+    const int s = k % kRqStages;
+    if (!mbar_wait(&full[s], uint32_t(k / kRqStages) & 1u)) {
+      if (lane == 0) flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_SCORE, uint32_t(k));
+      break;
+    }
+    const int4 x = info[s];
+    if (x.w >= 0) {
+      const int row = x.x, pi = x.y, L = x.z;
+      const uint8_t* pg = slots + s * PB;
+      const uint32_t* qc = a.qcode + size_t(row) * kRqRowWords;
+      uint32_t plane[kRqBits][W];
+#pragma unroll
+      for (int p = 0; p < kRqBits; ++p)
+#pragma unroll
+        for (int w = 0; w < W; ++w) plane[p][w] = __ldg(qc + p * W + w);
+      const float delta = __uint_as_float(__ldg(qc + kRqDelta));
+      const float vl = __uint_as_float(__ldg(qc + kRqVl));
+      const float shift = __uint_as_float(__ldg(qc + kRqShift));
+      const int Q = int(__ldg(qc + kRqQsum));
+      float m[4], l[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int slot = lane + 32 * kk;
+        uint32_t code[W];
+        if constexpr (W == 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(pg + slot * 16);
+          code[0] = v.x;
+          code[1] = v.y;
+          code[2] = v.z;
+          code[3] = v.w;
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2*>(pg + slot * 8);
+          code[0] = v.x;
+          code[1] = v.y;
+        }
+        const float gk = reinterpret_cast<const float*>(pg + kPage * (D / 8))[slot];
+        int A = 0, B = 0;
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          B += __popc(code[w]);
+#pragma unroll
+          for (int p = 0; p < kRqBits; ++p) A += __popc(code[w] & plane[p][w]) << p;
+        }
+        const float est = gk * (delta * float(2 * A - Q) + vl * float(2 * B - D)) + shift;
+        const bool valid = pi * kPage + slot < L;
+        m[kk] = valid ? a.scale * est : -INFINITY;
+        l[kk] = valid ? 1.0f : 0.0f;
+      }
+      float* out = a.scores + size_t(row) * a.nb_stride + size_t(pi) * (kPage / S);
+      if constexpr (S < 32) {
+        // a block = S neighbouring lanes of one k
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          float mk = m[kk], lk = l[kk];
+#pragma unroll
+          for (int o = 1; o < S; o <<= 1) {
+            const float m2 = __shfl_xor_sync(kFull, mk, o), l2 = __shfl_xor_sync(kFull, lk, o);
+            lse_merge(mk, lk, m2, l2);
+          }
+          if ((lane & (S - 1)) == 0) out[(lane + 32 * kk) / S] = lk > 0.0f ? mk + logf(lk) : -INFINITY;
+        }
+      } else {
+        // a block = S / 32 consecutive k of every lane
+        constexpr int KB = S / 32;
+#pragma unroll
+        for (int k0 = 0; k0 < 4; k0 += KB) {
+          float mk = m[k0], lk = l[k0];
+#pragma unroll
+          for (int kk = k0 + 1; kk < k0 + KB; ++kk) lse_merge(mk, lk, m[kk], l[kk]);
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float m2 = __shfl_xor_sync(kFull, mk, o), l2 = __shfl_xor_sync(kFull, lk, o);
+            lse_merge(mk, lk, m2, l2);
+          }
+          if (lane == 0) out[(32 * k0) / S] = lk > 0.0f ? mk + logf(lk) : -INFINITY;
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
 }
 
 template <int D>
 static cudaError_t launch_rq_score_d(const RqScoreParams& a, cudaStream_t s) {
+  using SH = RqShape<D>;
   const int max_pages = a.nb_stride / (kPage / a.S);
-  const long long warps = (long long)a.batch * max_pages * a.Hkv;
-  static const int per_sm = [] {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rq_score_kernel<D, 1>,
-                                                      kRqScanWarps * 32, 0) != cudaSuccess)
-      n = 0;
-    return n > 0 ? n : 1;
-  }();
-  long long grid = (long long)num_sms() * per_sm;
-  const long long need = (warps + kRqScanWarps - 1) / kRqScanWarps;
-  if (grid > need) grid = need;
+  const long long units = (long long)a.batch * max_pages * a.Hkv;
+  long long grid = (long long)num_sms() * 4;
+  if (grid > units) grid = units;
   if (grid < 1) grid = 1;
-  const dim3 block(kRqScanWarps * 32);
+  const dim3 block(kRqThreads);
+  const int smem = SH::kSmem;
+#define QS_RQ(SV)                                                                          \
+  {                                                                                        \
+    const cudaError_t e = set_smem_limit(rq_score_kernel<D, SV>, smem);                    \
+    if (e != cudaSuccess) return e;                                                        \
+    rq_score_kernel<D, SV><<<unsigned(grid), block, smem, s>>>(a);                         \
+    break;                                                                                 \
+  }
   switch (a.S) {
-    case 1: rq_score_kernel<D, 1><<<unsigned(grid), block, 0, s>>>(a); break;
-    case 2: rq_score_kernel<D, 2><<<unsigned(grid), block, 0, s>>>(a); break;
-    case 4: rq_score_kernel<D, 4><<<unsigned(grid), block, 0, s>>>(a); break;
-    case 8: rq_score_kernel<D, 8><<<unsigned(grid), block, 0, s>>>(a); break;
-    case 16: rq_score_kernel<D, 16><<<unsigned(grid), block, 0, s>>>(a); break;
-    case 32: rq_score_kernel<D, 32><<<unsigned(grid), block, 0, s>>>(a); break;
-    case 64: rq_score_kernel<D, 64><<<unsigned(grid), block, 0, s>>>(a); break;
-    case 128: rq_score_kernel<D, 128><<<unsigned(grid), block, 0, s>>>(a); break;
+    case 1: QS_RQ(1)
+    case 2: QS_RQ(2)
+    case 4: QS_RQ(4)
+    case 8: QS_RQ(8)
+    case 16: QS_RQ(16)
+    case 32: QS_RQ(32)
+    case 64: QS_RQ(64)
+    case 128: QS_RQ(128)
     default: return cudaErrorInvalidValue;
   }
+#undef QS_RQ
   return cudaGetLastError();
 }
 
@@ -626,19 +657,23 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_kernel(const TopPParams a
 
 // ------------------------------------------------------------ top-p by sorted candidates
 // The same selection without 64-bit shared-memory atomics, for budgets of at most
-// kTpCandMax blocks (the token-level budgets of the pages: B = 2,048):
-//   1. M, Z and the forced mass as above (per-thread 64-bit sums, then a block scan);
-//   2. the key of the cap-th best non-forced block (cap = budget minus the forced blocks)
-//      by three count-only histogram passes (11, 11 and 10 bits; 32-bit counts, lanes of a
-//      warp that share a bin combined first);
-//   3. the candidates: the non-forced blocks above that key and the first blocks (in index
-//      order) holding it, cap at most, compacted into shared memory as 64-bit sort keys
-//      (key << 32 | ~index) and bitonic-sorted, largest first: decreasing beta, ties to the
-//      lower index, exactly the order in which blocks are taken;
-//   4. their masses in that order, an exact prefix sum, and the number taken: the fewest
-//      whose mass with the forced blocks' reaches the goal, else all of them;
-//   5. the taken blocks and the forced ones marked in a bitmap of the row, written out in
-//      ascending order.
+// kTpCandMax blocks (the token-level budgets of the pages: B = 2,048), in three passes
+// over the row's scores:
+//   1. M, the largest score, and the smallest finite score of a non-forced block;
+//   2. Z and the forced mass (per-thread 64-bit integer sums, then a block scan), and a
+//      2,048-bin histogram of the finite non-forced scores linear between that minimum
+//      and M (32-bit counts);
+//   3. the candidates: every block in the bins from the one where the count from the top
+//      reaches cap (= budget minus the forced blocks) upwards, compacted into shared
+//      memory as 64-bit sort keys (key << 32 | ~index). If that bin is crowded (many equal
+//      or nearly equal scores) three count-only passes over the key bits find the cap-th
+//      key instead, and the candidates are the blocks above it and the first blocks (in
+//      index order) holding it;
+// then the candidates are bitonic-sorted, largest first (decreasing beta, ties to the
+// lower index: the order in which blocks are taken), their masses summed in that order
+// over the first cap of them, and the fewest whose mass with the forced blocks' reaches
+// the goal are taken (all cap if none); the taken and forced blocks are marked in a bitmap
+// of the row and written out in ascending order.
 constexpr int kTpCandMax = 4096;
 
 QS_DEV void tp_count_add(uint32_t* h, bool active, uint32_t bin) {
@@ -702,86 +737,146 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
   const int nF = (f0 >= 0) + (f1 >= 0);
   const int nb_up = (nb + kTpThreads - 1) / kTpThreads * kTpThreads;
 
-  // 1. the row's largest score; Z and the forced mass
-  float mx = -INFINITY;
-  for (int j = tid; j < nb; j += kTpThreads) mx = fmaxf(mx, tp_clean(sc[j]));
-  const float M = tp_block_max(mx, s_f);
-  unsigned long long z = 0, mf = 0;
+  // 1. the row's largest score, and the smallest finite score of a non-forced block
+  float mx = -INFINITY, mn = INFINITY;
   for (int j = tid; j < nb; j += kTpThreads) {
-    const unsigned long long w = tp_mass(tp_clean(sc[j]), M);
-    z += w;
-    if (j == f0 || j == f1) mf += w;
+    const float x = tp_clean(sc[j]);
+    mx = fmaxf(mx, x);
+    if (x > -INFINITY && j != f0 && j != f1) mn = fminf(mn, x);
   }
-  unsigned long long Z, MF;
-  tp_scan(z, s_u, Z);
+  const float M = tp_block_max(mx, s_f);
+  const float lo = -tp_block_max(-mn, s_f);
+  const uint32_t cap = uint32_t(max(0, min(a.budget - nF, nb - nF)));
+  // 2. Z, the forced mass, the count of finite non-forced blocks and (when the finite span
+  // is finite) a 2,048-bin histogram of them linear in the score between lo and M
+  const float span = M - lo;
+  const bool lin = cap > 0 && lo < INFINITY && span < INFINITY;
+  const float inv = span > 0.0f ? float(kTpBins) / span : 0.0f;
+  if (lin) {
+    for (int i = tid; i < kTpBins; i += kTpThreads) hist[i] = 0u;
+    __syncthreads();
+  }
+  unsigned long long z = 0, mf = 0, nfin = 0;
+  for (int j = tid; j < nb; j += kTpThreads) {
+    const float x = tp_clean(sc[j]);
+    const unsigned long long w = tp_mass(x, M);
+    z += w;
+    if (j == f0 || j == f1) {
+      mf += w;
+    } else if (x > -INFINITY) {
+      ++nfin;
+      if (lin) atomicAdd(&hist[min(kTpBins - 1, int((x - lo) * inv))], 1u);
+    }
+  }
+  unsigned long long Z, MF, NFIN;
+  tp_scan(z, s_u, Z);             // the barriers inside also complete the histogram
   tp_scan(mf, s_u, MF);
+  tp_scan(nfin, s_u, NFIN);
   unsigned long long goal = (unsigned long long)ceil(double(a.p) * double(Z));
   if (goal > Z) goal = Z;
-  const uint32_t cap = uint32_t(max(0, min(a.budget - nF, nb - nF)));
 
-  // 2. the key of the cap-th best non-forced block (all of them if cap covers them, none
-  // if cap is 0: no key lies above 0xffffffff)
-  uint32_t kc = cap == 0 ? 0xffffffffu : 0u, ties_take = 0u;
-  if (cap > 0 && cap < uint32_t(nb - nF)) {
-    uint32_t prefix = 0u, need = cap;
-    int known = 32;
-    for (int pass = 0; pass < 3; ++pass) {
-      const int width = pass < 2 ? 11 : 10, nbins = 1 << width, shift = known - width;
-      for (int i = tid; i < kTpBins; i += kTpThreads) hist[i] = 0u;
+  // 3. the candidates: at least the cap best non-forced blocks, compacted as 64-bit sort
+  // keys (key << 32 | ~index). First by a 2,048-bin histogram linear in the score between
+  // the row's finite minimum and maximum (a monotone map: a higher bin never holds a lower
+  // score): the bins above the one where the count reaches cap, and that bin, in one pass.
+  // Blocks at -inf carry no mass and are never needed. If that bin is too crowded (many
+  // equal or nearly equal scores), three count-only passes over the key bits find the
+  // cap-th key and the candidates are the blocks above it plus the first blocks holding it.
+  __shared__ unsigned s_nc;
+  unsigned c_tot = 0u;
+  bool linear_ok = false;
+  if (lin) {
+    // the bin where the count of finite blocks from the top reaches cap (all bins when
+    // there are no more than cap finite blocks)
+    uint32_t above = 0u;
+    int cut = 0;
+    uint32_t n_cand = uint32_t(NFIN);
+    if (NFIN > cap) {
+      cut = tp_find_count(hist, kTpBins, cap, s_u, &s_found, above);
+      n_cand = above + hist[cut];
+    }
+    if (n_cand <= uint32_t(kTpCandMax)) {
+      linear_ok = true;
+      if (tid == 0) s_nc = 0u;
       __syncthreads();
       for (int j = tid; j < nb_up; j += kTpThreads) {
-        const bool in = j < nb && j != f0 && j != f1;
-        const uint32_t key = in ? tp_key(tp_clean(sc[j])) : 0u;
-        const bool hit = in && (known == 32 || (key >> known) == prefix);
-        tp_count_add(hist, hit, (key >> shift) & uint32_t(nbins - 1));
+        const float x = j < nb ? tp_clean(sc[j]) : -INFINITY;
+        const bool take = j < nb && x > -INFINITY && j != f0 && j != f1 &&
+                          min(kTpBins - 1, int((x - lo) * inv)) >= cut;
+        const unsigned tm = __ballot_sync(kFull, take);
+        unsigned base = 0u;
+        if (lane == 0 && tm) base = atomicAdd(&s_nc, unsigned(__popc(tm)));
+        base = __shfl_sync(kFull, base, 0);
+        if (take)
+          cand[base + __popc(tm & ((1u << lane) - 1u))] =
+              ((unsigned long long)tp_key(x) << 32) | (0xffffffffu - uint32_t(j));
       }
       __syncthreads();
-      uint32_t above;
-      const int bin = tp_find_count(hist, nbins < kTpThreads ? kTpThreads : nbins, need, s_u,
-                                    &s_found, above);
-      if (bin < 0) {                                   // cannot happen: cap < non-forced count
-        if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
-        break;
+      c_tot = s_nc;
+    }
+  }
+  if (cap > 0 && lo < INFINITY && !linear_ok) {      // the key-bit passes
+    uint32_t kc = 0u, ties_take = 0u;
+    if (cap < uint32_t(nb - nF)) {
+      uint32_t prefix = 0u, need = cap;
+      int known = 32;
+      for (int pass = 0; pass < 3; ++pass) {
+        const int width = pass < 2 ? 11 : 10, nbins = 1 << width, shift = known - width;
+        for (int i = tid; i < kTpBins; i += kTpThreads) hist[i] = 0u;
+        __syncthreads();
+        for (int j = tid; j < nb_up; j += kTpThreads) {
+          const bool in = j < nb && j != f0 && j != f1;
+          const uint32_t key = in ? tp_key(tp_clean(sc[j])) : 0u;
+          const bool hit = in && (known == 32 || (key >> known) == prefix);
+          tp_count_add(hist, hit, (key >> shift) & uint32_t(nbins - 1));
+        }
+        __syncthreads();
+        uint32_t above;
+        const int bin = tp_find_count(hist, nbins < kTpThreads ? kTpThreads : nbins, need, s_u,
+                                      &s_found, above);
+        if (bin < 0) {                                 // cannot happen: cap < non-forced count
+          if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
+          break;
+        }
+        prefix = (prefix << width) | uint32_t(bin);
+        known = shift;
+        need -= above;
       }
-      prefix = (prefix << width) | uint32_t(bin);
-      known = shift;
-      need -= above;
+      kc = prefix;
+      ties_take = need;                                // blocks holding kc still to take
     }
-    kc = prefix;
-    ties_take = need;                                  // blocks holding kc still to take
-  }
-
-  // 3. the candidates, compacted in index order: warp w owns [w E, w E + E)
-  const int E = (nb + kTpThreads - 1) / kTpThreads * 32;
-  const int j0 = warp * E, j1 = min(nb, j0 + E);
-  unsigned n_gt = 0, n_eq = 0;
-  for (int jb = j0; jb < j1; jb += 32) {
-    const int j = jb + lane;
-    const bool in = j < j1 && j != f0 && j != f1;
-    const uint32_t key = in ? tp_key(tp_clean(sc[j])) : 0u;
-    n_gt += __popc(__ballot_sync(kFull, in && key > kc));
-    n_eq += __popc(__ballot_sync(kFull, in && key == kc));
-  }
-  unsigned eq_tot, c_tot;
-  const unsigned eq_before = tp_warp_scan(n_eq, s_w, eq_tot);
-  const unsigned eq_take = eq_before >= ties_take ? 0u : min(n_eq, ties_take - eq_before);
-  unsigned pos = tp_warp_scan(n_gt + eq_take, s_w, c_tot);
-  unsigned eq_rank = eq_before;
-  for (int jb = j0; jb < j1; jb += 32) {
-    const int j = jb + lane;
-    const bool in = j < j1 && j != f0 && j != f1;
-    const uint32_t key = in ? tp_key(tp_clean(sc[j])) : 0u;
-    const bool eq = in && key == kc;
-    const unsigned em = __ballot_sync(kFull, eq), below = (1u << lane) - 1u;
-    const bool take = (in && key > kc) || (eq && eq_rank + __popc(em & below) < ties_take);
-    const unsigned tm = __ballot_sync(kFull, take);
-    if (take) {
-      const unsigned at = pos + __popc(tm & below);
-      if (at < unsigned(kTpCandMax))
-        cand[at] = ((unsigned long long)key << 32) | (0xffffffffu - uint32_t(j));
+    // the candidates compacted in index order: warp w owns [w E, w E + E)
+    const int E = (nb + kTpThreads - 1) / kTpThreads * 32;
+    const int j0 = warp * E, j1 = min(nb, j0 + E);
+    unsigned n_gt = 0, n_eq = 0;
+    for (int jb = j0; jb < j1; jb += 32) {
+      const int j = jb + lane;
+      const bool in = j < j1 && j != f0 && j != f1;
+      const uint32_t key = in ? tp_key(tp_clean(sc[j])) : 0u;
+      n_gt += __popc(__ballot_sync(kFull, in && key > kc));
+      n_eq += __popc(__ballot_sync(kFull, in && key == kc));
     }
-    pos += __popc(tm);
-    eq_rank += __popc(em);
+    unsigned eq_tot;
+    const unsigned eq_before = tp_warp_scan(n_eq, s_w, eq_tot);
+    const unsigned eq_take = eq_before >= ties_take ? 0u : min(n_eq, ties_take - eq_before);
+    unsigned pos = tp_warp_scan(n_gt + eq_take, s_w, c_tot);
+    unsigned eq_rank = eq_before;
+    for (int jb = j0; jb < j1; jb += 32) {
+      const int j = jb + lane;
+      const bool in = j < j1 && j != f0 && j != f1;
+      const uint32_t key = in ? tp_key(tp_clean(sc[j])) : 0u;
+      const bool eq = in && key == kc;
+      const unsigned em = __ballot_sync(kFull, eq), below = (1u << lane) - 1u;
+      const bool take = (in && key > kc) || (eq && eq_rank + __popc(em & below) < ties_take);
+      const unsigned tm = __ballot_sync(kFull, take);
+      if (take) {
+        const unsigned at = pos + __popc(tm & below);
+        if (at < unsigned(kTpCandMax))
+          cand[at] = ((unsigned long long)key << 32) | (0xffffffffu - uint32_t(j));
+      }
+      pos += __popc(tm);
+      eq_rank += __popc(em);
+    }
   }
   const int n_c = int(min(c_tot, unsigned(kTpCandMax)));
   int n_pow = 1;
@@ -807,19 +902,21 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
     }
   }
 
-  // 4. masses in that order; the fewest whose mass with the forced blocks reaches the goal
+  // 4. masses in that order (the first cap candidates: the cap best blocks); the fewest
+  // whose mass with the forced blocks' reaches the goal
+  const int n_top = min(n_c, int(cap));
   const int per = (n_pow + kTpThreads - 1) / kTpThreads;     // consecutive entries per thread
   const int e0 = tid * per;
   unsigned long long loc = 0;
-  for (int i = e0; i < min(n_c, e0 + per); ++i)
+  for (int i = e0; i < min(n_top, e0 + per); ++i)
     loc += tp_mass(tp_clean(sc[0xffffffffu - uint32_t(cand[i])]), M);
-  if (tid == 0) s_take = n_c;
+  if (tid == 0) s_take = n_top;
   unsigned long long tot_c;
   unsigned long long cum = MF + tp_scan(loc, s_u, tot_c);
   if (MF >= goal) {
     if (tid == 0) s_take = 0;
   } else {
-    for (int i = e0; i < min(n_c, e0 + per); ++i) {
+    for (int i = e0; i < min(n_top, e0 + per); ++i) {
       cum += tp_mass(tp_clean(sc[0xffffffffu - uint32_t(cand[i])]), M);
       if (cum >= goal) {
         atomicMin(&s_take, i + 1);

@@ -47,7 +47,7 @@ QS_DEV void unit_prefix(const ScoreParams& a, int* prefix) {
       const int b = base + lane;
       int u = 0;
       if (b < a.batch) {
-        int L = a.seq_lens[b] + a.len_add;
+        int L = a.seq_lens[b];
         if (L < 0 || L > a.max_context) {
           flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SCORE, uint32_t(b));
           L = L < 0 ? 0 : a.max_context;
@@ -79,7 +79,7 @@ QS_DEV Unit decode_unit(const ScoreParams& a, const int* prefix, int u, int& b) 
   const int off = u - prefix[b];
   x.g = off / np;
   x.p = off % np;
-  int L = a.seq_lens[b] + a.len_add;
+  int L = a.seq_lens[b];
   L = L < 0 ? 0 : (L > a.max_context ? a.max_context : L);
   x.L = L;
   x.nv = min(kPage, L - x.p * kPage);
@@ -87,44 +87,6 @@ QS_DEV Unit decode_unit(const ScoreParams& a, const int* prefix, int u, int& b) 
   x.page = x.ok ? a.page_table[size_t(b) * a.max_pages_per_seq + x.p] : -1;
   x.ok = x.ok && x.page >= 0 && x.page < a.num_pages;
   return x;
-}
-
-// q~ of one row computed by one warp, the same float32 evaluation as the scoring prep
-// (qbar_i = (sum over the group's heads, in order) / G; q~_j = fma chain over i ascending),
-// so both give the same bits. Writes q~[0, R) to qt (this warp's shared-memory slot).
-template <int R, int D>
-QS_DEV void warp_qtilde(const ScoreParams& a, int row, int lane, float* qt) {
-  constexpr int T = (R + 31) / 32, DW = D / 32;
-  const int b = row / a.Hkv, g = row - b * a.Hkv;
-  const int Hq = a.Hkv * a.G;
-  const uint16_t* qrow = a.q + (size_t(b) * Hq + size_t(g) * a.G) * D;
-  float qb[DW];                                   // qbar_i for i = lane + 32 k
-#pragma unroll
-  for (int k = 0; k < DW; ++k) {
-    float s = 0.0f;
-    for (int h = 0; h < a.G; ++h) s += bf16_to_f32(qrow[size_t(h) * D + lane + 32 * k]);
-    qb[k] = s / float(a.G);
-  }
-  const float* Pg = a.P + size_t(g) * D * R;
-#pragma unroll
-  for (int t = 0; t < T; ++t) {
-    const int j = lane + 32 * t;
-    const bool on = j < R;
-    float acc = 0.0f;
-#pragma unroll
-    for (int i0 = 0; i0 < D; i0 += 8) {
-      float pv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) pv[u] = on ? __ldg(Pg + size_t(i0 + u) * R + j) : 0.0f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u;
-        acc = fmaf(__shfl_sync(kFull, qb[i / 32], i % 32), pv[u], acc);
-      }
-    }
-    if (on) qt[j] = acc;
-  }
-  __syncwarp();
 }
 
 template <typename PT, int R>
@@ -136,8 +98,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + NST * SH::kPageBytes);
   uint64_t* empty = full + NST;
   int4* info = reinterpret_cast<int4*>(empty + NST);              // [NST] {row, page idx, nv, ok}
-  float* s_qt = reinterpret_cast<float*>(info + NST);             // [consumers][R] inline q~
-  int* prefix = reinterpret_cast<int*>(s_qt + kScoreConsumers * R);  // [batch + 1]
+  int* prefix = reinterpret_cast<int*>(info + NST);               // [batch + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (!a.early_stream) pdl_wait();   // q~ and seq_lens come from the kernel before
@@ -176,13 +137,10 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
         const int jok = __shfl_sync(kFull, int(x.ok), j);
         const int jpage = __shfl_sync(kFull, x.page, j);
         const int jg = __shfl_sync(kFull, x.g, j);
-        const int jlast = __shfl_sync(kFull, int(x.p == (x.L + kPage - 1) / kPage - 1), j);
         if (lane == 0) {
           const int k = k0 + j;
           const int s = k % NST;
           const uint32_t ph = uint32_t(k / NST) & 1u;
-          // the writer fills the newest token's slot of the row's last page
-          if (a.wait_last && jlast) pdl_wait();
           if (!mbar_wait(&empty[s], ph ^ 1u)) {
             flag_error(a.hdr, QS_ERR_DEVICE_TIMEOUT, KID_SCORE, uint32_t(k));
             dead = true;
@@ -204,8 +162,6 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
         if (dead) break;
       }
     }
-    // this grid completes only after the writer has (the kernels after it rely on that)
-    if (a.wait_last && lane == 0) pdl_wait();
     return;
   }
 
@@ -219,7 +175,7 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
   const int rot = lane / (128 / SH::kTokenBytes);
   float qr[CPT][EPC];                                 // q~ permuted by this lane's rotation
   int cur_row = -1;
-  if (a.early_stream && !a.inline_qt) pdl_wait();     // q~ comes from the kernel before
+  if (a.early_stream) pdl_wait();                     // q~ comes from the kernel before
   const int bpp = kPage / a.S;  // blocks per page
   for (int k = c; k < n_units; k += kScoreConsumers) {
     const int s = k % NST;
@@ -233,21 +189,11 @@ __global__ void __launch_bounds__(kScoreThreads, 3) score_rankr_kernel(const Sco
     if (x.w) {
       if (row != cur_row) {
         cur_row = row;
-        const float* qsrc = a.qt + size_t(row) * R;
-        if constexpr (R <= 32) {                       // rank 64 takes q~ from the writer
-          if (a.inline_qt) {
-            float* mine = s_qt + c * R;
-            __syncwarp();                              // the previous row's reads are done
-            if (a.d == 128) warp_qtilde<R, 128>(a, row, lane, mine);
-            else warp_qtilde<R, 64>(a, row, lane, mine);
-            qsrc = mine;
-          }
-        }
 #pragma unroll
         for (int kk = 0; kk < CPT; ++kk) {
           const int ch = (kk + rot) & (CPT - 1);
 #pragma unroll
-          for (int e = 0; e < EPC; ++e) qr[kk][e] = qsrc[ch * EPC + e];
+          for (int e = 0; e < EPC; ++e) qr[kk][e] = a.qt[size_t(row) * R + ch * EPC + e];
         }
       }
       const uint8_t* slot = slots + s * SH::kPageBytes;
@@ -319,7 +265,6 @@ static cudaError_t launch_rankr_score(const ScoreParams& a, cudaStream_t st, boo
   using SH = ProxyShape<PT, R>;
   const size_t smem_max = size_t(SH::kStages) * SH::kPageBytes +
                           2 * SH::kStages * sizeof(uint64_t) + SH::kStages * sizeof(int4) +
-                          size_t(kScoreConsumers) * R * sizeof(float) +
                           size_t(kMaxBatch + 1) * sizeof(int);
   const size_t smem = smem_max - size_t(kMaxBatch - a.batch) * sizeof(int);
   auto k = score_rankr_kernel<PT, R>;

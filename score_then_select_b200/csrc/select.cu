@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams a) {
   float v[ITEMS];
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) v[i] = (jw + i * 32 < nb_cap) ? sc[jw + i * 32] : -FLT_MAX;
-  int L = a.seq_lens[b] + a.len_add;
+  int L = a.seq_lens[b];
   int nb = int((static_cast<long long>(L) + a.S - 1) / a.S);
   if (L < 0 || nb > nb_cap) {
     if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));

@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kRxThreads, 1) select_radix_kernel(const Selec
   const float* sc = a.scores + size_t(row) * a.nb_stride;
   int32_t* sel = a.sel + size_t(row) * a.budget;
   const int k = a.budget;
-  int L = a.seq_lens[b] + a.len_add;
+  int L = a.seq_lens[b];
   int nb = int((static_cast<long long>(L) + a.S - 1) / a.S);
   if (L < 0 || nb > a.nb_stride) {
     if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));

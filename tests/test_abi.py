@@ -309,8 +309,8 @@ def test_nvfp4_key_storage_validates_on_the_host():
               v_dtype="f16", v_agg_dtype="f16")
     st = _cfg(key_storage="nvfp4", **nv)
     assert qs.qs_workspace_size(st, 16, 131072) > qs.qs_workspace_size(_cfg(**nv), 16, 131072)
-    assert qs.qs_attention_launches(st, 16, 131072) == 2
-    assert qs.qs_attention_launches(_cfg(**nv), 16, 131072) == 1
+    assert qs.qs_attention_launches(st, 16, 131072) == 3
+    assert qs.qs_attention_launches(_cfg(**nv), 16, 131072) == 2
     assert qs.qs_dense_workspace_size(st, 16, 131072) == qs.qs_dense_workspace_size(
         _cfg(**nv), 16, 131072)
     with pytest.raises(qs.QsError) as e:                      # rank-r scoring copy

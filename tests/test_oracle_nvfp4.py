@@ -247,9 +247,9 @@ def test_step_nvfp4_kept_blocks_are_forced_and_selected():
 
 
 def test_step_key_storage_attends_the_storage_keys():
-    """With NVFP4 key storage the row step attends over nvfp4_attended_keys_bf16 (the kept
-    blocks' BF16 keys, elsewhere the decoded, un-centred keys rounded to BF16), with the
-    same selection; keeping every selected block gives exactly the BF16-key output."""
+    """With NVFP4 key storage the row step attends over nvfp4_attended_keys (the kept
+    blocks' BF16 keys, elsewhere the exactly dequantised, un-centred keys), with the same
+    selection; keeping every selected block gives exactly the BF16-key output."""
     import dataclasses
     from oracle import step as OS
     rng = np.random.default_rng(72)
@@ -267,8 +267,7 @@ def test_step_key_storage_attends_the_storage_keys():
     r_st = OS.decode_row(ps, k, v, q, L, mu=mu, g_k=g_k, g_q=g_q)
     assert np.array_equal(r_st["sel"], r_bf["sel"]) and len(r_st["keep"]) == 2
     codes, scales, _ = r_st["cache"]
-    want_k = F.bf16_to_f64(M.nvfp4_attended_keys_bf16(k, codes, scales, g_k, mu, r_st["keep"],
-                                                      S, L))
+    want_k = M.nvfp4_attended_keys(k, codes, scales, g_k, mu, r_st["keep"], S, L)
     assert np.array_equal(r_st["K_att"], want_k)
     Vd = OS.decode_v(v, p.v_dtype)
     assert np.array_equal(r_st["out"], M.sparse_attention(F.bf16_to_f64(q), want_k, Vd,
