@@ -131,7 +131,9 @@ QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uin
 #pragma unroll
   for (int m = 0; m < KS; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.0f;
   uint32_t qb[KS][2];
-  float qmu0 = 0.0f, qmu1 = 0.0f;                          // NVFP4 keys: q . mu, heads h0, h0 + 1
+  // NVFP4 keys: q 2^-qexp as FP16 fragments, 2^qexp g_k, and q . mu of heads h0, h0 + 1
+  uint32_t qh[KS][2];
+  float gks = 0.0f, qmu0 = 0.0f, qmu1 = 0.0f;
   for (int t = 0;; ++t) {
     const int s = t % NS;
     if (!wait_or_abort(&full[s], (t / NS) & 1, s_abort)) break;
@@ -180,6 +182,24 @@ QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uin
         }
         qmu0 = s0;
         qmu1 = s1;
+        // qexp puts the group's largest |q| in [2^14, 2^15): every BF16 query element then
+        // converts to FP16 exactly unless it is below 2^-28 of that maximum (FP16 subnormals)
+        uint32_t mx = 0u;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks)
+          mx = max(mx, max(max(qb[ks][0] & 0x7fff7fffu, qb[ks][1] & 0x7fff7fffu) >> 16,
+                           max(qb[ks][0] & 0x7fffu, qb[ks][1] & 0x7fffu)));
+#pragma unroll
+        for (int o2 = 1; o2 < 32; o2 <<= 1) mx = max(mx, __shfl_xor_sync(kFull, mx, o2));
+        const int e = int(mx >> 7);                        // biased exponent of max |q|
+        const int qexp = mx == 0u ? 0 : max(-60, min(100, e - 127 - 14));
+        const float down = __uint_as_float(uint32_t(127 - qexp) << 23);
+        gks = gk * __uint_as_float(uint32_t(127 + qexp) << 23);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+            qh[ks][i] = pack_f16x2(bf16_lo(qb[ks][i]) * down, bf16_hi(qb[ks][i]) * down);
       }
     }
     const uint32_t kst = smem_u32(st), vst = smem_u32(st + SM::kTileBytes);
@@ -189,8 +209,8 @@ QS_DEV void attn_consume(const AttnParams& a, uint8_t* smem, uint32_t* meta, uin
     const bool v0 = (vm >> (tl & 31)) & 1u, v1 = (vm >> ((tl + 8) & 31)) & 1u;
     const auto sw = [](int r, int c) { return swz(r, c); };
     if (KQ4 && (info & kMetaRawK)) {
-      const KFragNvfp4 kf(st + kRawCodes, st + kRawScales, gk, qmu0, qmu1,
-                          (info & kMetaHalf) ? 64 : 0, warp, lane);
+      const KFragNvfp4<KS> kf(st + kRawCodes, st + kRawScales, qh, gks, qmu0, qmu1,
+                              (info & kMetaHalf) ? 64 : 0, warp, lane);
       attn_warp_tile<D, V_F16, AGG_F16>(kf, vst, qb, v0, v1, a.scale_log2, m0, m1, l0, l1, o,
                                         warp, lane, sw);
     } else {

@@ -26,18 +26,23 @@ struct KFragLdsm {
   uint32_t kst;
   int warp, lane;
   Swz swz;
-  QS_DEV void operator()(int ks, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) const {
+  // c += K Q^T over k-step ks (BF16 keys and queries)
+  QS_DEV void qk(float (&c)[4], int ks, const uint32_t (&qb)[2]) const {
+    uint32_t a0, a1, a2, a3;
     ldsm_x4(a0, a1, a2, a3, kst + swz(warp * 16 + (lane & 15), ks * 2 + (lane >> 4)));
+    mma_bf16(c, a0, a1, a2, a3, qb[0], qb[1]);
   }
   QS_DEV void fix(float (&)[4]) const {}     // the accumulator is the logit
 };
 
 // K fragments of one 64-token tile of NVFP4 keys in shared memory (the storage variant of
 // "Jet-QSparse ...", Full text). The attended key is the dequantised, un-centred value
-// k = g_k (e sigma) + mu. The A operand is e * sigma, which is exact in BF16 (an E2M1 value
-// has at most 2 significant bits and a UE4M3 scale 4); the products with the BF16 query
-// are then exact and the MMA sums them in float32, so the logit q . k is
-// g_k (q . (e sigma)) + q . mu, formed in `fix` from the accumulator and the head's q . mu.
+// k = g_k (e sigma) + mu. The A operand is e * sigma, exact in FP16 (an E2M1 value has at
+// most 2 significant bits and a UE4M3 scale 4; the product lies in [2^-10, 2688]), made by
+// one conversion of two codes and one f16x2 multiply; the B operand is the query in FP16,
+// scaled by 2^-qexp (qexp > 0 only for queries beyond FP16's range), so the products are
+// exact and the MMA sums them in float32. The logit is then
+// q . k = 2^qexp g_k (q' . (e sigma)) + q . mu, formed in `fix`.
 //   codes:  [4 chunks][64 tokens][16 bytes]; chunk c holds elements 32c..32c+31 of a
 //           token, element 2i + u in nibble u of byte i;
 //   scales: the page's 1,024 bytes; token slot m's scale of elements 16j..16j+15 at
@@ -45,55 +50,58 @@ struct KFragLdsm {
 //           the tile's first token.
 // This lane's rows are tokens r0 = 16 warp + lane / 4 and r0 + 8 of the tile, its elements
 // 2t, 2t + 1, 2t + 8, 2t + 9 of each k-step (t = lane % 4), as the mma A fragment holds them.
+template <int KS>
 struct KFragNvfp4 {
   const uint8_t* codes;
-  float gk, qmu0, qmu1;    // g_k; q . mu of this lane's heads 2t and 2t + 1
+  const uint32_t (&qh)[KS][2];  // FP16 query fragments (B operand), scaled by 2^-qexp
+  float gks, qmu0, qmu1;        // 2^qexp g_k; q . mu of this lane's heads 2t and 2t + 1
   int r0, t;
-  uint32_t sc[2][2];       // scale words: [row r0, r0 + 8][elements 0-63, 64-127]
+  uint32_t sg[2][KS];           // sigma of each k-step of rows r0, r0 + 8, as f16 pairs
 
-  QS_DEV KFragNvfp4(const uint8_t* codes_, const uint8_t* scales, float gk_, float qmu0_,
-                    float qmu1_, int m0, int warp, int lane)
-      : codes(codes_), gk(gk_), qmu0(qmu0_), qmu1(qmu1_), r0(warp * 16 + (lane >> 2)), t(lane & 3) {
+  QS_DEV KFragNvfp4(const uint8_t* codes_, const uint8_t* scales, const uint32_t (&qh_)[KS][2],
+                    float gks_, float qmu0_, float qmu1_, int m0, int warp, int lane)
+      : codes(codes_), qh(qh_), gks(gks_), qmu0(qmu0_), qmu1(qmu1_), r0(warp * 16 + (lane >> 2)),
+        t(lane & 3) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int m = m0 + r0 + 8 * r;
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        sc[r][h] = *reinterpret_cast<const uint32_t*>(scales + h * 512 + 16 * (m & 31) + 4 * (m >> 5));
+      for (int h = 0; h < KS / 4; ++h) {
+        const uint32_t w =
+            *reinterpret_cast<const uint32_t*>(scales + h * 512 + 16 * (m & 31) + 4 * (m >> 5));
+        const uint32_t lo = e4m3x2_to_f16x2(w), hi = e4m3x2_to_f16x2(w >> 16);
+        sg[r][4 * h + 0] = __byte_perm(lo, 0u, 0x1010);      // low half in both halves
+        sg[r][4 * h + 1] = __byte_perm(lo, 0u, 0x3232);      // high half in both halves
+        sg[r][4 * h + 2] = __byte_perm(hi, 0u, 0x1010);
+        sg[r][4 * h + 3] = __byte_perm(hi, 0u, 0x3232);
+      }
     }
   }
-  // sigma of k-step ks of row r as an f16 pair (both halves)
-  QS_DEV uint32_t sig2(int r, int ks) const {
-    const uint32_t f = e4m3x2_to_f16x2(sc[r][ks >> 2] >> (8 * (ks & 3))) & 0xffffu;
-    return f | (f << 16);
-  }
-  // byte t of w (two codes) times sigma -> bf16x2, exact
+  // byte t of w (two codes) times sigma: f16x2, exact
   QS_DEV uint32_t dec(uint32_t w, uint32_t s2) const {
     const uint32_t e = e2m1x2_to_f16x2(w >> (8 * t));
     uint32_t p;
     asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p) : "r"(e), "r"(s2));
-    return __byte_perm(__float_as_uint(f16_lo(p)), __float_as_uint(f16_hi(p)), 0x7632);
+    return p;
   }
-  QS_DEV void operator()(int ks, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) const {
-    const int c = ks >> 1, h = ks & 1;
-    const uint2 w0 = *reinterpret_cast<const uint2*>(codes + c * 1024 + r0 * 16 + 8 * h);
-    const uint2 w1 = *reinterpret_cast<const uint2*>(codes + c * 1024 + (r0 + 8) * 16 + 8 * h);
-    const uint32_t s0 = sig2(0, ks), s1 = sig2(1, ks);
-    a0 = dec(w0.x, s0);
-    a1 = dec(w1.x, s1);
-    a2 = dec(w0.y, s0);
-    a3 = dec(w1.y, s1);
+  // c += K Q^T over k-step ks (FP16 e * sigma and queries)
+  QS_DEV void qk(float (&c)[4], int ks, const uint32_t (&)[2]) const {
+    const int cc = ks >> 1, h = ks & 1;
+    const uint2 w0 = *reinterpret_cast<const uint2*>(codes + cc * 1024 + r0 * 16 + 8 * h);
+    const uint2 w1 = *reinterpret_cast<const uint2*>(codes + cc * 1024 + (r0 + 8) * 16 + 8 * h);
+    mma_f16(c, dec(w0.x, sg[0][ks]), dec(w1.x, sg[1][ks]), dec(w0.y, sg[0][ks]),
+            dec(w1.y, sg[1][ks]), qh[ks][0], qh[ks][1]);
   }
   // accumulator (tokens r0 / r0 + 8 x heads 2t, 2t + 1) -> logits q . k
   QS_DEV void fix(float (&c)[4]) const {
-    c[0] = fmaf(c[0], gk, qmu0);
-    c[1] = fmaf(c[1], gk, qmu1);
-    c[2] = fmaf(c[2], gk, qmu0);
-    c[3] = fmaf(c[3], gk, qmu1);
+    c[0] = fmaf(c[0], gks, qmu0);
+    c[1] = fmaf(c[1], gks, qmu1);
+    c[2] = fmaf(c[2], gks, qmu0);
+    c[3] = fmaf(c[3], gks, qmu1);
   }
 };
 
-// kf(ks, a0..a3): the K fragments of k-step ks (see KFragLdsm). qb: the query fragments (B
+// kf.qk(c, ks, qb): c += K Q^T over k-step ks; kf.fix(c): accumulator -> logits. qb: the query fragments (B
 // operand of S^T), valid0 / valid1: whether this lane's two tokens are selected (masked
 // ones get probability 0), scale_log2: softmax scale * log2 e; `swz` addresses the V tile.
 template <int D, bool V_F16, bool AGG_F16, typename KF, typename Swz>
@@ -105,11 +113,7 @@ QS_DEV void attn_warp_tile(const KF& kf, uint32_t vst, const uint32_t (&qb)[D / 
   // S^T = K Q^T for this warp's 16 tokens
   float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    uint32_t a0, a1, a2, a3;
-    kf(ks, a0, a1, a2, a3);
-    mma_bf16(c, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-  }
+  for (int ks = 0; ks < KS; ++ks) kf.qk(c, ks, qb[ks]);
   kf.fix(c);
   const float x0 = valid0 ? c[0] * scale_log2 : -INFINITY;
   const float x1 = valid0 ? c[1] * scale_log2 : -INFINITY;
