@@ -67,7 +67,9 @@ __global__ void __launch_bounds__(128, 2) attn_gather_kernel(const AttnParams a)
   const int slots = n * a.S;
   const int s0 = split * a.g_tokens_per_split;
   const int s1 = min(s0 + a.g_tokens_per_split, slots);
-  const int cnt = s1 - s0;
+  // slots of this split; none when the row selected fewer slots than the splits before it
+  // cover (s0 >= slots), so that every index below stays inside the split's table
+  const int cnt = max(0, s1 - s0);
 
   // ---------------- token table of this split: cache row index of each slot, or -1.
   // Slots [lo, hi) are resolved on demand: for blocks of >= 16 tokens each selection entry

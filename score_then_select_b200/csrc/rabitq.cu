@@ -106,6 +106,11 @@ cudaError_t launch_rq_prep(const RqPrepParams& a, cudaStream_t s) {
 
 // ============================================================ scan
 
+// float(n) for |n| < 2^22 without a conversion instruction (those share the quarter-rate
+// pipe with the population counts): 1.5 * 2^23 + n is exact in float32 (its ulp is 1), so
+// adding n to that value's bit pattern and subtracting it again gives n exactly.
+QS_DEV float rq_int_to_float(int n) { return __int_as_float(0x4B400000 + n) - 12582912.0f; }
+
 // Merge of log-sum-exp states: (m, l) stands for l * e^m.
 QS_DEV void lse_merge(float& m, float& l, float m2, float l2) {
   const float mm = fmaxf(m, m2);
@@ -119,15 +124,18 @@ QS_DEV void lse_merge(float& m, float& l, float m2, float l2) {
 }
 
 // Persistent grid, one producer warp and four consumer warps per CTA. A unit is one
-// (sequence b, page p, KV head g), g fastest (a page's heads are contiguous in the cache);
-// the units are split evenly over the CTAs. The producer's lanes resolve 32 units' pages at
-// a time and lane 0 streams each unit's whole (page, head) record (code bits and factors,
-// 2,560 bytes at d = 128) with one bulk copy into a 16-stage shared-memory ring, completion
-// counted on the stage's mbarrier; units past a row's length are skipped. Consumer warp c
-// scores units c, c + 4, ...: lane l the token slots l + 32 k from shared memory.
+// (row = (sequence b, KV head g), page p), p fastest, so that a CTA's contiguous share of
+// the units covers one or two rows: a consumer keeps the row's query code in registers
+// and reloads it only when the row changes. The producer's lanes resolve 32 units' pages
+// at a time and lane 0 streams each unit's (page, head) record (code bits and factors,
+// 2,560 bytes at d = 128) with one bulk copy into a 12-stage shared-memory ring,
+// completion counted on the stage's mbarrier; units past a row's length are skipped.
+// Consumer warp c scores units c, c + 4, ...: lane l the token slots l + 32 k. The scoring
+// is bound by instruction latency (20 AND/POPC pairs per token), so the CTA is kept to 64
+// registers and 31 KB of shared memory: six CTAs (24 consumer warps) per SM.
 constexpr int kRqConsumers = 4;
 constexpr int kRqThreads = 32 * (1 + kRqConsumers);
-constexpr int kRqStages = 16;
+constexpr int kRqStages = 12;
 
 template <int D>
 struct RqShape {
@@ -136,7 +144,7 @@ struct RqShape {
 };
 
 template <int D, int S>
-__global__ void __launch_bounds__(kRqThreads, 4) rq_score_kernel(const RqScoreParams a) {
+__global__ void __launch_bounds__(kRqThreads, 6) rq_score_kernel(const RqScoreParams a) {
   using SH = RqShape<D>;
   constexpr int W = D / 32, PB = SH::kPageBytes;
   extern __shared__ __align__(128) uint8_t rq_smem[];
@@ -154,7 +162,7 @@ __global__ void __launch_bounds__(kRqThreads, 4) rq_score_kernel(const RqScorePa
   }
   __syncthreads();
   const int max_pages = a.nb_stride / (kPage / S);
-  const long long U = (long long)a.batch * max_pages * a.Hkv;
+  const long long U = (long long)a.batch * a.Hkv * max_pages;
   const long long u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
   const int n_units = int(u1 - u0);
 
@@ -165,12 +173,9 @@ __global__ void __launch_bounds__(kRqThreads, 4) rq_score_kernel(const RqScorePa
       int row = 0, pi = 0, L = 0, page = -1;
       if (k0 + lane < n_units) {
         const long long u = u0 + k0 + lane;
-        const long long per_b = (long long)max_pages * a.Hkv;
-        const int b = int(u / per_b);
-        const int rem = int(u - (long long)b * per_b);
-        pi = rem / a.Hkv;
-        const int g = rem - pi * a.Hkv;
-        row = b * a.Hkv + g;
+        row = int(u / max_pages);
+        pi = int(u - (long long)row * max_pages);
+        const int b = row / a.Hkv, g = row - b * a.Hkv;
         L = a.seq_lens[b];
         if (L > a.max_context || L < 0) {
           if (pi == 0 && g == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SCORE, uint32_t(b));
@@ -218,6 +223,10 @@ __global__ void __launch_bounds__(kRqThreads, 4) rq_score_kernel(const RqScorePa
 
   // ---------------- consumers
   const int c = warp - 1;
+  int cur = -1;                                    // the row whose query code is loaded
+  uint32_t plane[kRqBits][W];
+  float delta = 0.0f, vl = 0.0f, shift = 0.0f;
+  int Q = 0;
   for (int k = c; k < n_units; k += kRqConsumers) {
     const int s = k % kRqStages;
     if (!mbar_wait(&full[s], uint32_t(k / kRqStages) & 1u)) {
@@ -228,16 +237,18 @@ __global__ void __launch_bounds__(kRqThreads, 4) rq_score_kernel(const RqScorePa
     if (x.w >= 0) {
       const int row = x.x, pi = x.y, L = x.z;
       const uint8_t* pg = slots + s * PB;
-      const uint32_t* qc = a.qcode + size_t(row) * kRqRowWords;
-      uint32_t plane[kRqBits][W];
+      if (row != cur) {                            // warp-uniform
+        const uint32_t* qc = a.qcode + size_t(row) * kRqRowWords;
 #pragma unroll
-      for (int p = 0; p < kRqBits; ++p)
+        for (int p = 0; p < kRqBits; ++p)
 #pragma unroll
-        for (int w = 0; w < W; ++w) plane[p][w] = __ldg(qc + p * W + w);
-      const float delta = __uint_as_float(__ldg(qc + kRqDelta));
-      const float vl = __uint_as_float(__ldg(qc + kRqVl));
-      const float shift = __uint_as_float(__ldg(qc + kRqShift));
-      const int Q = int(__ldg(qc + kRqQsum));
+          for (int w = 0; w < W; ++w) plane[p][w] = __ldg(qc + p * W + w);
+        delta = __uint_as_float(__ldg(qc + kRqDelta));
+        vl = __uint_as_float(__ldg(qc + kRqVl));
+        shift = __uint_as_float(__ldg(qc + kRqShift));
+        Q = int(__ldg(qc + kRqQsum));
+        cur = row;
+      }
       float m[4], l[4];
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
@@ -262,13 +273,18 @@ __global__ void __launch_bounds__(kRqThreads, 4) rq_score_kernel(const RqScorePa
 #pragma unroll
           for (int p = 0; p < kRqBits; ++p) A += __popc(code[w] & plane[p][w]) << p;
         }
-        const float est = gk * (delta * float(2 * A - Q) + vl * float(2 * B - D)) + shift;
+        const float est = gk * (delta * rq_int_to_float(2 * A - Q) +
+                                vl * rq_int_to_float(2 * B - D)) + shift;
         const bool valid = pi * kPage + slot < L;
         m[kk] = valid ? a.scale * est : -INFINITY;
         l[kk] = valid ? 1.0f : 0.0f;
       }
       float* out = a.scores + size_t(row) * a.nb_stride + size_t(pi) * (kPage / S);
-      if constexpr (S < 32) {
+      if constexpr (S == 1) {
+        // a block = one token: its log-sum-exp is its own scaled estimate
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) out[lane + 32 * kk] = m[kk];
+      } else if constexpr (S < 32) {
         // a block = S neighbouring lanes of one k
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -307,7 +323,7 @@ static cudaError_t launch_rq_score_d(const RqScoreParams& a, cudaStream_t s) {
   using SH = RqShape<D>;
   const int max_pages = a.nb_stride / (kPage / a.S);
   const long long units = (long long)a.batch * max_pages * a.Hkv;
-  long long grid = (long long)num_sms() * 4;
+  long long grid = (long long)num_sms() * 6;
   if (grid > units) grid = units;
   if (grid < 1) grid = 1;
   const dim3 block(kRqThreads);
@@ -361,6 +377,30 @@ QS_DEV uint32_t tp_key(float x) {
 QS_DEV unsigned long long tp_mass(float x, float M) {
   if (!(M > -INFINITY)) return 0ull;
   return __float2ull_rn(expf(x - M) * kTpUnit);
+}
+
+// One streaming pass over a row's nb scores. Sweep `it` gives thread t the blocks
+// j = it + t + u kTpThreads, u < kTpUnroll: all kTpUnroll loads are issued before the first
+// is used, so every thread keeps that many in flight (a pass over a token-level row is
+// otherwise one dependent load after another). Every thread runs the same number of sweeps
+// and calls f(j, x, in) for each of its blocks, in = j < nb, x = the cleaned score (-inf
+// when !in), so whole warps stay together for warp-collective steps inside f.
+constexpr int kTpUnroll = 8;
+template <typename F>
+QS_DEV void tp_sweep(const float* sc, int nb, F&& f) {
+  for (int it = 0; it < nb; it += kTpUnroll * kTpThreads) {
+    float x[kTpUnroll];
+#pragma unroll
+    for (int u = 0; u < kTpUnroll; ++u) {
+      const int j = it + int(threadIdx.x) + u * kTpThreads;
+      x[u] = j < nb ? sc[j] : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < kTpUnroll; ++u) {
+      const int j = it + int(threadIdx.x) + u * kTpThreads;
+      f(j, tp_clean(x[u]), j < nb);
+    }
+  }
 }
 
 QS_DEV float tp_block_max(float v, float* s) {
@@ -515,11 +555,10 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_kernel(const TopPParams a
   const int f0 = (a.force_sink && nb > 0) ? 0 : -1;
   const int f1 = (a.force_last && nb > 0 && nb - 1 != f0) ? nb - 1 : -1;
   const int nF = (f0 >= 0) + (f1 >= 0);
-  const int nb_up = (nb + kTpThreads - 1) / kTpThreads * kTpThreads;   // whole warps per step
 
   // the row's largest score
   float mx = -INFINITY;
-  for (int j = tid; j < nb; j += kTpThreads) mx = fmaxf(mx, tp_clean(sc[j]));
+  tp_sweep(sc, nb, [&](int, float x, bool) { mx = fmaxf(mx, x); });
   const float M = tp_block_max(mx, s_f);
 
   // Z, the forced blocks' mass, and the histogram of the others' top 11 key bits
@@ -529,15 +568,13 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_kernel(const TopPParams a
   }
   __syncthreads();
   unsigned long long z = 0, mf = 0;
-  for (int j = tid; j < nb_up; j += kTpThreads) {
-    const bool in = j < nb;
-    const float x = in ? tp_clean(sc[j]) : -INFINITY;
+  tp_sweep(sc, nb, [&](int j, float x, bool in) {
     const unsigned long long w = in ? tp_mass(x, M) : 0ull;
     const bool forced = j == f0 || j == f1;
     z += w;
     if (forced) mf += w;
     tp_hist_add(h_cnt, h_mass, in && !forced, tp_key(x) >> 21, w);
-  }
+  });
   unsigned long long Z, MF;
   tp_scan(z, s_u, Z);            // totals; the barriers inside also complete the histogram
   tp_scan(mf, s_u, MF);
@@ -568,14 +605,13 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_kernel(const TopPParams a
           h_mass[i] = 0ull;
         }
         __syncthreads();
-        for (int j = tid; j < nb_up; j += kTpThreads) {
-          const bool in = j < nb && j != f0 && j != f1;
-          const float x = in ? tp_clean(sc[j]) : -INFINITY;
+        tp_sweep(sc, nb, [&](int j, float x, bool in) {
+          in = in && j != f0 && j != f1;
           const uint32_t key = tp_key(x);
           const bool hit = in && (key >> known) == prefix;
           tp_hist_add(h_cnt, h_mass, hit, (key >> shift) & uint32_t(nbins - 1),
                       hit ? tp_mass(x, M) : 0ull);
-        }
+        });
         __syncthreads();
         f = tp_find(h_cnt, h_mass, nbins, cap, need, s_u, &s_found);
         if (f.bin < 0) {
@@ -675,6 +711,7 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_kernel(const TopPParams a
 // the goal are taken (all cap if none); the taken and forced blocks are marked in a bitmap
 // of the row and written out in ascending order.
 constexpr int kTpCandMax = 4096;
+static_assert(kTpCandMax <= 4 * kTpThreads, "tp_sort holds at most 4 keys per thread");
 
 QS_DEV void tp_count_add(uint32_t* h, bool active, uint32_t bin) {
   const unsigned act = __ballot_sync(kFull, active);
@@ -712,6 +749,59 @@ QS_DEV int tp_find_count(const uint32_t* cnt, int nbins, uint32_t cap, unsigned 
   return bin;
 }
 
+// Bitonic sort of cand[0, 1024 E), largest first (the same compare-exchange network as
+// sorting in shared memory). Element i = 1024 s + t is held by thread t in v[s]: a stage
+// whose partner i ^ jj is in the same warp (jj < 32) exchanges by shuffles, one in the same
+// thread (jj >= 1024) in registers, and only the others (32 <= jj < 1024) through cand.
+// Every thread of the CTA calls it.
+QS_DEV unsigned long long tp_keep(unsigned long long x, unsigned long long y, bool keep_max) {
+  return (x > y) == keep_max ? x : y;
+}
+template <int E>
+QS_DEV void tp_sort(unsigned long long* cand) {
+  const int t = int(threadIdx.x);
+  unsigned long long v[E];
+#pragma unroll
+  for (int s = 0; s < E; ++s) v[s] = cand[s * kTpThreads + t];
+  for (int k = 2; k <= kTpThreads * E; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      if (jj < 32) {
+#pragma unroll
+        for (int s = 0; s < E; ++s) {
+          const int i = s * kTpThreads + t;
+          const unsigned long long o = __shfl_xor_sync(kFull, v[s], jj);
+          v[s] = tp_keep(v[s], o, ((i & jj) == 0) == ((i & k) == 0));
+        }
+      } else if (jj < kTpThreads) {
+#pragma unroll
+        for (int s = 0; s < E; ++s) cand[s * kTpThreads + t] = v[s];
+        __syncthreads();
+#pragma unroll
+        for (int s = 0; s < E; ++s) {
+          const int i = s * kTpThreads + t;
+          v[s] = tp_keep(v[s], cand[i ^ jj], ((i & jj) == 0) == ((i & k) == 0));
+        }
+        __syncthreads();
+      } else {
+        const int js = jj / kTpThreads;
+#pragma unroll
+        for (int s = 0; s < E; ++s)
+#pragma unroll
+          for (int s2 = s + 1; s2 < E; ++s2)
+            if ((s ^ s2) == js) {                     // pair (s, s2), s the lower index
+              const bool desc = ((s * kTpThreads + t) & k) == 0;
+              const unsigned long long x = v[s], y = v[s2];
+              v[s] = tp_keep(x, y, desc);
+              v[s2] = tp_keep(x, y, !desc);
+            }
+      }
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < E; ++s) cand[s * kTpThreads + t] = v[s];
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPParams a) {
   extern __shared__ __align__(16) uint8_t tp_smem[];
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(tp_smem);   // [kTpCandMax]
@@ -735,15 +825,13 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
   const int f0 = (a.force_sink && nb > 0) ? 0 : -1;
   const int f1 = (a.force_last && nb > 0 && nb - 1 != f0) ? nb - 1 : -1;
   const int nF = (f0 >= 0) + (f1 >= 0);
-  const int nb_up = (nb + kTpThreads - 1) / kTpThreads * kTpThreads;
 
   // 1. the row's largest score, and the smallest finite score of a non-forced block
   float mx = -INFINITY, mn = INFINITY;
-  for (int j = tid; j < nb; j += kTpThreads) {
-    const float x = tp_clean(sc[j]);
+  tp_sweep(sc, nb, [&](int j, float x, bool) {
     mx = fmaxf(mx, x);
     if (x > -INFINITY && j != f0 && j != f1) mn = fminf(mn, x);
-  }
+  });
   const float M = tp_block_max(mx, s_f);
   const float lo = -tp_block_max(-mn, s_f);
   const uint32_t cap = uint32_t(max(0, min(a.budget - nF, nb - nF)));
@@ -756,9 +844,10 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
     for (int i = tid; i < kTpBins; i += kTpThreads) hist[i] = 0u;
     __syncthreads();
   }
-  unsigned long long z = 0, mf = 0, nfin = 0;
-  for (int j = tid; j < nb; j += kTpThreads) {
-    const float x = tp_clean(sc[j]);
+  unsigned long long z = 0, mf = 0;
+  unsigned nfin = 0u;
+  tp_sweep(sc, nb, [&](int j, float x, bool in) {
+    if (!in) return;
     const unsigned long long w = tp_mass(x, M);
     z += w;
     if (j == f0 || j == f1) {
@@ -767,7 +856,7 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
       ++nfin;
       if (lin) atomicAdd(&hist[min(kTpBins - 1, int((x - lo) * inv))], 1u);
     }
-  }
+  });
   unsigned long long Z, MF, NFIN;
   tp_scan(z, s_u, Z);             // the barriers inside also complete the histogram
   tp_scan(mf, s_u, MF);
@@ -799,18 +888,18 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
       linear_ok = true;
       if (tid == 0) s_nc = 0u;
       __syncthreads();
-      for (int j = tid; j < nb_up; j += kTpThreads) {
-        const float x = j < nb ? tp_clean(sc[j]) : -INFINITY;
-        const bool take = j < nb && x > -INFINITY && j != f0 && j != f1 &&
+      tp_sweep(sc, nb, [&](int j, float x, bool in) {
+        const bool take = in && x > -INFINITY && j != f0 && j != f1 &&
                           min(kTpBins - 1, int((x - lo) * inv)) >= cut;
         const unsigned tm = __ballot_sync(kFull, take);
+        if (tm == 0u) return;                          // warp-uniform
         unsigned base = 0u;
-        if (lane == 0 && tm) base = atomicAdd(&s_nc, unsigned(__popc(tm)));
+        if (lane == 0) base = atomicAdd(&s_nc, unsigned(__popc(tm)));
         base = __shfl_sync(kFull, base, 0);
         if (take)
           cand[base + __popc(tm & ((1u << lane) - 1u))] =
               ((unsigned long long)tp_key(x) << 32) | (0xffffffffu - uint32_t(j));
-      }
+      });
       __syncthreads();
       c_tot = s_nc;
     }
@@ -824,12 +913,12 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
         const int width = pass < 2 ? 11 : 10, nbins = 1 << width, shift = known - width;
         for (int i = tid; i < kTpBins; i += kTpThreads) hist[i] = 0u;
         __syncthreads();
-        for (int j = tid; j < nb_up; j += kTpThreads) {
-          const bool in = j < nb && j != f0 && j != f1;
-          const uint32_t key = in ? tp_key(tp_clean(sc[j])) : 0u;
+        tp_sweep(sc, nb, [&](int j, float x, bool in) {
+          in = in && j != f0 && j != f1;
+          const uint32_t key = in ? tp_key(x) : 0u;
           const bool hit = in && (known == 32 || (key >> known) == prefix);
           tp_count_add(hist, hit, (key >> shift) & uint32_t(nbins - 1));
-        }
+        });
         __syncthreads();
         uint32_t above;
         const int bin = tp_find_count(hist, nbins < kTpThreads ? kTpThreads : nbins, need, s_u,
@@ -879,27 +968,16 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
     }
   }
   const int n_c = int(min(c_tot, unsigned(kTpCandMax)));
-  int n_pow = 1;
+  int n_pow = kTpThreads;                              // sorted length: 1,024, 2,048 or 4,096
   while (n_pow < n_c) n_pow <<= 1;
-  for (int i = n_c + tid; i < n_pow; i += kTpThreads) cand[i] = 0ull;   // below every block
-  __syncthreads();
-  // bitonic sort, largest first
+  __syncthreads();                                     // every candidate written
+  // bitonic sort, largest first; the padding (0) lies below every block's key
   if (n_c > 1) {
-    for (int k = 2; k <= n_pow; k <<= 1) {
-      for (int jj = k >> 1; jj > 0; jj >>= 1) {
-        for (int i = tid; i < n_pow; i += kTpThreads) {
-          const int ixj = i ^ jj;
-          if (ixj > i) {
-            const unsigned long long x = cand[i], y = cand[ixj];
-            if (((i & k) == 0) ? (x < y) : (x > y)) {
-              cand[i] = y;
-              cand[ixj] = x;
-            }
-          }
-        }
-        __syncthreads();
-      }
-    }
+    for (int i = n_c + tid; i < n_pow; i += kTpThreads) cand[i] = 0ull;
+    __syncthreads();
+    if (n_pow == kTpThreads) tp_sort<1>(cand);
+    else if (n_pow == 2 * kTpThreads) tp_sort<2>(cand);
+    else tp_sort<4>(cand);
   }
 
   // 4. masses in that order (the first cap candidates: the cap best blocks); the fewest

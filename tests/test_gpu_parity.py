@@ -17,7 +17,7 @@ import torch
 
 import synth
 from oracle import method as M
-from tests.util import check_attention, oracle_row, query_scale_all, row_params
+from tests.util import check_attention, decoded_row, oracle_row, query_scale_all, row_params
 
 pytestmark = pytest.mark.gpu
 
@@ -173,6 +173,59 @@ def test_dense_rows_reduce_to_dense_attention():
             assert sel[b, g, :nsel[b, g]].tolist() == list(range(-(-L // w.block_size)))
             check_attention(w, out[b, g * w.group:(g + 1) * w.group], dense, (k, v, q),
                             np.arange(L), f"dense row {b},{g}")
+
+
+def test_gather_short_selections_under_a_large_budget():
+    """Token-level selections far shorter than the budget. The gather kernel's split plan
+    covers the whole budget (every slot a sequence could select: here 16 K), so most splits
+    of a row hold none of its tokens and must contribute nothing (their slot range starts
+    past the row's selection). Rows select 0, 1, 37, 2,049, 5,000 and all of their tokens;
+    each output matches the oracle's attention over the row's tokens, an empty row is 0."""
+    _gpu()
+    import score_then_select_b200 as qs
+    from score_then_select_b200.filled import cfg_kwargs
+    from score_then_select_b200.layer import workspace
+    from tests.gpu_util import Filled, out_to_f64
+    w = synth.small(synth.TOKEN32K).replace(context=16384 + 77)
+    inp = synth.Inputs(w)
+    f = Filled(inp)
+    held = inp.lens - 1                                  # tokens in the cache
+    budget = int(inp.lens.max())
+    cfg = qs.make_config(**dict(cfg_kwargs(w), budget=budget))
+    ws = workspace(qs.qs_workspace_size(cfg, w.batch, f.layer.max_context))
+    rng = np.random.default_rng(77)
+    counts = [0, 1, 37, 2049, 5000, -1]                  # -1: every token
+    sel = np.full((w.batch, w.n_kv_heads, budget), -1, dtype=np.int32)
+    nsel = np.zeros((w.batch, w.n_kv_heads), dtype=np.int32)
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            L = int(held[b])
+            n = counts[(b * w.n_kv_heads + g) % len(counts)]
+            n = L if n < 0 else min(n, L)
+            t = np.sort(rng.choice(L, size=n, replace=False)).astype(np.int32)
+            sel[b, g, :n] = t
+            nsel[b, g] = n
+    out = torch.full((w.batch, w.n_q_heads, w.head_dim), float("nan"), dtype=torch.bfloat16,
+                     device="cuda")
+    qs.qs_sparse_attn(cfg, f.cache, f.q, torch.from_numpy(sel).cuda(),
+                      torch.from_numpy(nsel).cuda(), w.batch, out, ws)
+    st = qs.qs_device_status(ws)
+    assert st[0] == 0, f"device status {st}"
+    out = out_to_f64(out)
+    G = w.group
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            n = int(nsel[b, g])
+            got = out[b, g * G:(g + 1) * G]
+            if n == 0:
+                assert np.all(got == 0.0), f"row {b},{g}: an empty selection gives 0"
+                continue
+            L = int(held[b])
+            row = (f.K[b, g, :L], f.V[b, g, :L], f.Q[b, g * G:(g + 1) * G])
+            q, K, V = decoded_row(w, row)
+            tokens = sel[b, g, :n].astype(np.int64)
+            check_attention(w, got, M.sparse_attention(q, K, V, tokens, w.scale), row, tokens,
+                            f"row {b},{g} ({n} tokens)")
 
 
 @pytest.mark.parametrize("path", [1, 2])
