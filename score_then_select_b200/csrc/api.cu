@@ -657,10 +657,15 @@ static qs_status do_rq_score(const Plan& p, const qs_cache* c, const void* q, co
   return cuda_status(launch_rq_score(b, s));
 }
 
+// row_max: the rows' largest scores as recorded by the scan that wrote `scores` (the step
+// call), or null (scores from the caller: the select finds them)
 static qs_status do_top_p(const Plan& p, const qs_cache* c, const float* scores, float p_mass,
-                          int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t s) {
+                          int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t s,
+                          const uint32_t* row_max = nullptr) {
   TopPParams a{};
   a.scores = scores;
+  a.row_max = row_max;
+  a.row_max_stride = kRqRowWords;
   a.seq_lens = c->seq_lens;
   a.sel = sel;
   a.n_sel = n_sel;
@@ -731,7 +736,9 @@ qs_status qs_decode_top_p(const qs_config* cfg, const qs_cache* cache, const voi
   if ((st = do_append(p, cache, k_new, v_new, nullptr, 1, R, nullptr, ws, stream)) != QS_OK)
     return st;
   if ((st = do_rq_score(p, cache, q, R, u, scores, ws, stream)) != QS_OK) return st;
-  if ((st = do_top_p(p, cache, scores, p_mass, sel, nsel, ws, stream)) != QS_OK) return st;
+  const uint32_t* row_max = ws_at<uint32_t>(ws, p.ws.qt) + kRqRowMax;
+  if ((st = do_top_p(p, cache, scores, p_mass, sel, nsel, ws, stream, row_max)) != QS_OK)
+    return st;
   return do_attend(p, cache, q, sel, nsel, out, ws, stream, false);
 }
 

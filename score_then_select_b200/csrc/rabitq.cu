@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(D) rq_prep_kernel(const RqPrepParams a) {
     out[kRqVl] = __float_as_uint(mn);
     out[kRqQsum] = uint32_t(q);
     out[kRqShift] = __float_as_uint(dot);
+    out[kRqRowMax] = 0u;                         // raised by the scan
   }
 }
 
@@ -105,6 +106,17 @@ cudaError_t launch_rq_prep(const RqPrepParams& a, cudaStream_t s) {
 }
 
 // ============================================================ scan
+
+// A score as the select kernels read it: NaN counts as -inf, +inf as FLT_MAX; and its
+// order-preserving unsigned key (a larger score, a larger key; -inf > 0).
+QS_DEV float tp_clean(float x) { return x != x ? -INFINITY : fminf(x, FLT_MAX); }
+QS_DEV uint32_t tp_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+QS_DEV float tp_unkey(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 // float(n) for |n| < 2^22 without a conversion instruction (those share the quarter-rate
 // pipe with the population counts): 1.5 * 2^23 + n is exact in float32 (its ulp is 1), so
@@ -238,15 +250,16 @@ __global__ void __launch_bounds__(kRqThreads, 6) rq_score_kernel(const RqScorePa
       const int row = x.x, pi = x.y, L = x.z;
       const uint8_t* pg = slots + s * PB;
       if (row != cur) {                            // warp-uniform
+        // plain loads: word kRqRowMax of the same record is raised during this kernel
         const uint32_t* qc = a.qcode + size_t(row) * kRqRowWords;
 #pragma unroll
         for (int p = 0; p < kRqBits; ++p)
 #pragma unroll
-          for (int w = 0; w < W; ++w) plane[p][w] = __ldg(qc + p * W + w);
-        delta = __uint_as_float(__ldg(qc + kRqDelta));
-        vl = __uint_as_float(__ldg(qc + kRqVl));
-        shift = __uint_as_float(__ldg(qc + kRqShift));
-        Q = int(__ldg(qc + kRqQsum));
+          for (int w = 0; w < W; ++w) plane[p][w] = qc[p * W + w];
+        delta = __uint_as_float(qc[kRqDelta]);
+        vl = __uint_as_float(qc[kRqVl]);
+        shift = __uint_as_float(qc[kRqShift]);
+        Q = int(qc[kRqQsum]);
         cur = row;
       }
       float m[4], l[4];
@@ -280,10 +293,14 @@ __global__ void __launch_bounds__(kRqThreads, 6) rq_score_kernel(const RqScorePa
         l[kk] = valid ? 1.0f : 0.0f;
       }
       float* out = a.scores + size_t(row) * a.nb_stride + size_t(pi) * (kPage / S);
+      float vmax = -INFINITY;                      // the largest score this warp writes
       if constexpr (S == 1) {
         // a block = one token: its log-sum-exp is its own scaled estimate
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) out[lane + 32 * kk] = m[kk];
+        for (int kk = 0; kk < 4; ++kk) {
+          out[lane + 32 * kk] = m[kk];
+          vmax = fmaxf(vmax, tp_clean(m[kk]));
+        }
       } else if constexpr (S < 32) {
         // a block = S neighbouring lanes of one k
 #pragma unroll
@@ -294,7 +311,11 @@ __global__ void __launch_bounds__(kRqThreads, 6) rq_score_kernel(const RqScorePa
             const float m2 = __shfl_xor_sync(kFull, mk, o), l2 = __shfl_xor_sync(kFull, lk, o);
             lse_merge(mk, lk, m2, l2);
           }
-          if ((lane & (S - 1)) == 0) out[(lane + 32 * kk) / S] = lk > 0.0f ? mk + logf(lk) : -INFINITY;
+          if ((lane & (S - 1)) == 0) {
+            const float v = lk > 0.0f ? mk + logf(lk) : -INFINITY;
+            out[(lane + 32 * kk) / S] = v;
+            vmax = fmaxf(vmax, tp_clean(v));
+          }
         }
       } else {
         // a block = S / 32 consecutive k of every lane
@@ -309,9 +330,17 @@ __global__ void __launch_bounds__(kRqThreads, 6) rq_score_kernel(const RqScorePa
             const float m2 = __shfl_xor_sync(kFull, mk, o), l2 = __shfl_xor_sync(kFull, lk, o);
             lse_merge(mk, lk, m2, l2);
           }
-          if (lane == 0) out[(32 * k0) / S] = lk > 0.0f ? mk + logf(lk) : -INFINITY;
+          if (lane == 0) {
+            const float v = lk > 0.0f ? mk + logf(lk) : -INFINITY;
+            out[(32 * k0) / S] = v;
+            vmax = fmaxf(vmax, tp_clean(v));
+          }
         }
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, o));
+      if (lane == 0 && vmax > -INFINITY)
+        atomicMax(a.qcode + size_t(row) * kRqRowWords + kRqRowMax, tp_key(vmax));
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -369,11 +398,6 @@ constexpr int kTpThreads = 1024;
 constexpr int kTpBins = 2048;
 constexpr float kTpUnit = 1099511627776.0f;   // 2^40
 
-QS_DEV float tp_clean(float x) { return x != x ? -INFINITY : fminf(x, FLT_MAX); }
-QS_DEV uint32_t tp_key(float x) {
-  const uint32_t u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 QS_DEV unsigned long long tp_mass(float x, float M) {
   if (!(M > -INFINITY)) return 0ull;
   return __float2ull_rn(expf(x - M) * kTpUnit);
@@ -711,6 +735,12 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_kernel(const TopPParams a
 // the goal are taken (all cap if none); the taken and forced blocks are marked in a bitmap
 // of the row and written out in ascending order.
 constexpr int kTpCandMax = 4096;
+
+// Bin of a finite score x in the histogram linear between lo and lo + kTpBins / inv,
+// clamped to [0, kTpBins - 1]: monotone in x.
+QS_DEV int tp_lin_bin(float x, float lo, float inv) {
+  return min(kTpBins - 1, int(fmaxf(0.0f, (x - lo) * inv)));
+}
 static_assert(kTpCandMax <= 4 * kTpThreads, "tp_sort holds at most 4 keys per thread");
 
 QS_DEV void tp_count_add(uint32_t* h, bool active, uint32_t bin) {
@@ -826,14 +856,26 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
   const int f1 = (a.force_last && nb > 0 && nb - 1 != f0) ? nb - 1 : -1;
   const int nF = (f0 >= 0) + (f1 >= 0);
 
-  // 1. the row's largest score, and the smallest finite score of a non-forced block
-  float mx = -INFINITY, mn = INFINITY;
-  tp_sweep(sc, nb, [&](int j, float x, bool) {
-    mx = fmaxf(mx, x);
-    if (x > -INFINITY && j != f0 && j != f1) mn = fminf(mn, x);
-  });
-  const float M = tp_block_max(mx, s_f);
-  const float lo = -tp_block_max(-mn, s_f);
+  // 1. the row's largest score, and the smallest finite score of a non-forced block. When
+  // the scan that wrote the scores recorded each row's largest (its order-preserving key),
+  // this pass is skipped: M is that score, and the histogram below starts at M - 28
+  // instead of the smallest score (a block 28 below M has mass e^-28 < 2^-40, which rounds
+  // to 0; bins only need to be monotone in the score, lower scores fall into bin 0, and a
+  // cut in bin 0 with too many candidates takes the key-bit passes).
+  float M, lo;
+  if (a.row_max) {
+    const uint32_t k = a.row_max[size_t(row) * a.row_max_stride];
+    M = k ? tp_unkey(k) : -INFINITY;
+    lo = M > -INFINITY ? M - 28.0f : INFINITY;
+  } else {
+    float mx = -INFINITY, mn = INFINITY;
+    tp_sweep(sc, nb, [&](int j, float x, bool) {
+      mx = fmaxf(mx, x);
+      if (x > -INFINITY && j != f0 && j != f1) mn = fminf(mn, x);
+    });
+    M = tp_block_max(mx, s_f);
+    lo = -tp_block_max(-mn, s_f);
+  }
   const uint32_t cap = uint32_t(max(0, min(a.budget - nF, nb - nF)));
   // 2. Z, the forced mass, the count of finite non-forced blocks and (when the finite span
   // is finite) a 2,048-bin histogram of them linear in the score between lo and M
@@ -854,7 +896,7 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
       mf += w;
     } else if (x > -INFINITY) {
       ++nfin;
-      if (lin) atomicAdd(&hist[min(kTpBins - 1, int((x - lo) * inv))], 1u);
+      if (lin) atomicAdd(&hist[tp_lin_bin(x, lo, inv)], 1u);
     }
   });
   unsigned long long Z, MF, NFIN;
@@ -890,7 +932,7 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
       __syncthreads();
       tp_sweep(sc, nb, [&](int j, float x, bool in) {
         const bool take = in && x > -INFINITY && j != f0 && j != f1 &&
-                          min(kTpBins - 1, int((x - lo) * inv)) >= cut;
+                          tp_lin_bin(x, lo, inv) >= cut;
         const unsigned tm = __ballot_sync(kFull, take);
         if (tm == 0u) return;                          // warp-uniform
         unsigned base = 0u;

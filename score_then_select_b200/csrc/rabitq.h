@@ -29,7 +29,9 @@ inline int rq_page_bytes(int d) { return kPage * (d / 8) + kPage * 4; }
 //   [0, 4 * d/32)   bit planes: plane p, word w holds bit p of the codes of dims 32w..32w+31
 //   [24]            Delta (float bits)       [25] v_l (float bits)
 //   [26]            Q = sum of the codes     [27] c . qbar (float bits)
-constexpr int kRqDelta = 24, kRqVl = 25, kRqQsum = 26, kRqShift = 27;
+//   [28]            the row's largest block score, as its order-preserving key (0: none),
+//                   reset by the query-code kernel and raised by the scan
+constexpr int kRqDelta = 24, kRqVl = 25, kRqQsum = 26, kRqShift = 27, kRqRowMax = 28;
 
 struct RqPrepParams {
   const uint16_t* q;          // [batch][Hq][d] BF16
@@ -42,7 +44,7 @@ struct RqPrepParams {
 
 struct RqScoreParams {
   const uint8_t* proxy;       // scoring cache pages
-  const uint32_t* qcode;
+  uint32_t* qcode;            // read; word kRqRowMax of each row raised
   const int32_t* page_table;
   const int32_t* seq_lens;
   float* scores;              // [batch][Hkv][nb_stride]: log of each block's mass
@@ -57,6 +59,10 @@ struct TopPParams {
   int32_t* sel;               // [rows][budget]
   int32_t* n_sel;             // [rows]
   uint32_t* hdr;
+  // the rows' largest scores as order-preserving keys, written by the scan that produced
+  // `scores` (row r's at row_max[r * row_max_stride]); null: the select finds them itself
+  const uint32_t* row_max;
+  int row_max_stride;
   int rows, Hkv, S, nb_stride, budget, force_sink, force_last;
   float p;
 };

@@ -229,46 +229,63 @@ cudaError_t launch_sem_index(const SemIndexParams& a, int iters, cudaStream_t s)
 
 // ============================================================ decode
 constexpr int kSemScoreWarps = 8;
+constexpr int kSemScorePerWarp = 4;                        // clusters per warp
 
-// warp = (row, cluster j): beta_j = qbar . c_j (float32); -inf past the row's clusters.
-// Also writes each sequence's cluster count, which the select kernel takes as its number
-// of candidates.
+// CTA = (row, 32 clusters): beta_j = qbar . c_j (float32); -inf past the row's clusters.
+// qbar (the group's head sum in order, divided by G) is formed once per CTA in shared
+// memory; warp w scores clusters 4w .. 4w + 3 of the CTA's 32, lane l summing dimensions
+// l + 32 m in order and the lanes combined by shuffles. Also writes each sequence's
+// cluster count, which the select kernel takes as its number of candidates.
 template <int D>
 __global__ void __launch_bounds__(kSemScoreWarps * 32) sem_score_kernel(const SemSelectParams a) {
   constexpr int PER = D / 32;
+  constexpr int CPB = kSemScoreWarps * kSemScorePerWarp;
+  __shared__ float s_qbar[D];
   const int row = blockIdx.y, b = row / a.Hkv, g = row % a.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int L0 = sem_prompt(a.prompt_lens, b, a.l_max);
   const int C = min(sem_clusters(L0, a.S), a.c_max);
   if (blockIdx.x == 0 && g == 0 && threadIdx.x == 0) a.n_clusters[b] = C;
-  const int j = blockIdx.x * kSemScoreWarps + warp;
-  if (j >= a.c_max) return;
-  float* out = a.scores + size_t(row) * a.c_max;
-  if (j >= C) {
-    if (lane == 0) out[j] = -INFINITY;
-    return;
-  }
   const int Hq = a.Hkv * a.G;
-  const float* c = a.cent + (size_t(row) * a.c_max + j) * D;
-  float dot = 0.0f;
-#pragma unroll
-  for (int m = 0; m < PER; ++m) {
-    const int i = lane + 32 * m;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
     float s = 0.0f;
     for (int h = 0; h < a.G; ++h)
       s += bf16_to_f32(a.q[(size_t(b) * Hq + size_t(g) * a.G + h) * D + i]);
-    dot = fmaf(c[i], s / float(a.G), dot);
+    s_qbar[i] = s / float(a.G);
+  }
+  __syncthreads();
+  float* out = a.scores + size_t(row) * a.c_max;
+  const int j0 = blockIdx.x * CPB + warp * kSemScorePerWarp;
+  float cv[kSemScorePerWarp][PER];
+#pragma unroll
+  for (int u = 0; u < kSemScorePerWarp; ++u) {
+    const int j = j0 + u;
+    const float* c = a.cent + (size_t(row) * a.c_max + (j < C ? j : 0)) * D;
+#pragma unroll
+    for (int m = 0; m < PER; ++m) cv[u][m] = j < C ? __ldg(c + lane + 32 * m) : 0.0f;
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(kFull, dot, o);
-  if (lane == 0) out[j] = dot;
+  for (int u = 0; u < kSemScorePerWarp; ++u) {
+    const int j = j0 + u;
+    if (j >= a.c_max) break;                       // warp-uniform
+    float dot = 0.0f;
+#pragma unroll
+    for (int m = 0; m < PER; ++m) dot = fmaf(cv[u][m], s_qbar[lane + 32 * m], dot);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(kFull, dot, o);
+    if (lane == 0) out[j] = j < C ? dot : -INFINITY;
+  }
 }
 
 // CTA = row: the members of the selected clusters (each cluster's in token order, the
 // clusters in the order selected), then the tokens after the prompt, L0 <= t < seq_len.
+// A scan over the selected clusters' sizes gives each cluster's place in the list; warp w
+// then copies clusters w, w + 32, ..., its lanes striding over the cluster's members.
 __global__ void __launch_bounds__(kSemThreads) sem_expand_kernel(const SemSelectParams a) {
   __shared__ int s_scan[kSemThreads / 32];
+  __shared__ int s_lo[kSemThreads], s_sz[kSemThreads], s_dst[kSemThreads];
   const int row = blockIdx.x, b = row / a.Hkv, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int L0 = sem_prompt(a.prompt_lens, b, a.l_max);
   const int C = min(sem_clusters(L0, a.S), a.c_max);
   int L = a.seq_lens[b];
@@ -292,10 +309,19 @@ __global__ void __launch_bounds__(kSemThreads) sem_expand_kernel(const SemSelect
     const int lo = ok ? off[c] : 0, sz = ok ? off[c + 1] - lo : 0;
     int total;
     const int dst = running + sem_scan(sz, s_scan, total);
-    for (int m = 0; m < sz; ++m) {
-      if (dst + m < a.max_tokens) out[dst + m] = mem[lo + m];
-      else over = true;
+    s_lo[tid] = lo;
+    s_sz[tid] = sz;
+    s_dst[tid] = dst;
+    __syncthreads();
+    const int nc = min(kSemThreads, ncs - base);
+    for (int k = warp; k < nc; k += kSemThreads / 32) {
+      const int klo = s_lo[k], ksz = s_sz[k], kdst = s_dst[k];
+      for (int m = lane; m < ksz; m += 32) {
+        if (kdst + m < a.max_tokens) out[kdst + m] = mem[klo + m];
+        else over = true;
+      }
     }
+    __syncthreads();                               // before the next batch's table
     running += total;
   }
   for (int t = L0 + tid; t < L; t += kSemThreads) {
@@ -311,7 +337,8 @@ __global__ void __launch_bounds__(kSemThreads) sem_expand_kernel(const SemSelect
 }
 
 cudaError_t launch_sem_score(const SemSelectParams& a, cudaStream_t s) {
-  const dim3 grid((a.c_max + kSemScoreWarps - 1) / kSemScoreWarps, a.batch * a.Hkv);
+  constexpr int CPB = kSemScoreWarps * kSemScorePerWarp;
+  const dim3 grid((a.c_max + CPB - 1) / CPB, a.batch * a.Hkv);
   if (a.d == 128) sem_score_kernel<128><<<grid, kSemScoreWarps * 32, 0, s>>>(a);
   else sem_score_kernel<64><<<grid, kSemScoreWarps * 32, 0, s>>>(a);
   return cudaGetLastError();
