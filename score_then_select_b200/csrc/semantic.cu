@@ -333,7 +333,14 @@ __global__ void __launch_bounds__(kSemThreads) sem_expand_kernel(const SemSelect
   int n = running + (L - L0);
   if (n > a.max_tokens) n = a.max_tokens;
   if (tid == 0) a.n_tokens[row] = n;
-  for (int i = n + tid; i < a.max_tokens; i += kSemThreads) out[i] = -1;
+  // the padding: 4-byte stores up to a 16-byte boundary, then 16-byte stores, then the tail
+  int i0 = n;
+  while (i0 < a.max_tokens && (reinterpret_cast<uintptr_t>(out + i0) & 15u) != 0u) ++i0;
+  if (tid < i0 - n) out[n + tid] = -1;
+  const int nv = (a.max_tokens - i0) / 4;
+  int4* out4 = reinterpret_cast<int4*>(out + i0);
+  for (int i = tid; i < nv; i += kSemThreads) out4[i] = make_int4(-1, -1, -1, -1);
+  for (int i = i0 + 4 * nv + tid; i < a.max_tokens; i += kSemThreads) out[i] = -1;
 }
 
 cudaError_t launch_sem_score(const SemSelectParams& a, cudaStream_t s) {

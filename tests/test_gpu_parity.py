@@ -175,18 +175,21 @@ def test_dense_rows_reduce_to_dense_attention():
                             np.arange(L), f"dense row {b},{g}")
 
 
-def test_gather_short_selections_under_a_large_budget():
+@pytest.mark.parametrize("context", [16384 + 77, 40000 + 77])
+def test_gather_short_selections_under_a_large_budget(context):
     """Token-level selections far shorter than the budget. The gather kernel's split plan
-    covers the whole budget (every slot a sequence could select: here 16 K), so most splits
-    of a row hold none of its tokens and must contribute nothing (their slot range starts
-    past the row's selection). Rows select 0, 1, 37, 2,049, 5,000 and all of their tokens;
-    each output matches the oracle's attention over the row's tokens, an empty row is 0."""
+    covers the whole budget (every slot a sequence could select), so most splits of a row
+    hold none of its tokens and must contribute nothing. At 16 K the plan's grid fits one
+    wave of resident CTAs; at 40 K it does not (30 splits of 1,344 slots for 16 rows), so
+    each row gets fewer CTAs than splits and a CTA takes several of its row's splits in
+    turn. Rows select 0, 1, 37, 2,049, 5,000 and all of their tokens; each output matches
+    the oracle's attention over the row's tokens, an empty row is 0."""
     _gpu()
     import score_then_select_b200 as qs
     from score_then_select_b200.filled import cfg_kwargs
     from score_then_select_b200.layer import workspace
     from tests.gpu_util import Filled, out_to_f64
-    w = synth.small(synth.TOKEN32K).replace(context=16384 + 77)
+    w = synth.small(synth.TOKEN32K).replace(context=context)
     inp = synth.Inputs(w)
     f = Filled(inp)
     held = inp.lens - 1                                  # tokens in the cache
