@@ -78,7 +78,7 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (measured copy bandwidth)"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback 6650 GB/s (earlier measurement on this pool)"
+        return FALLBACK_HBM_GBS, "fallback 6650 GB/s (an earlier copy-bandwidth measurement on B200)"
 
 
 # ------------------------------------------------------------------ clocks (NVML sampling)

@@ -44,7 +44,7 @@
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and never
  *     synchronise, except qs_device_status.
  *   - Arguments are validated on the host before any launch. On failure the call returns
- *     QS_ERR_INVALID_ARG (bad pointer/size) or QS_ERR_UNSUPPORTED (a shape this build does
+ *     QS_ERR_INVALID_ARG (bad pointer/size) or QS_ERR_UNSUPPORTED (a shape the library does
  *     not implement) and launches nothing. There is no fallback path.
  *   - Cache tensors (K, V, proxy) and q must be 16-byte aligned (q may be 4-byte aligned
  *     for qs_score on the rank-r path).
