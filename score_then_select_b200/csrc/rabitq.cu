@@ -835,13 +835,14 @@ QS_DEV void tp_sort(unsigned long long* cand) {
 __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPParams a) {
   extern __shared__ __align__(16) uint8_t tp_smem[];
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(tp_smem);   // [kTpCandMax]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(cand + kTpCandMax);             // [kTpBins]
+  unsigned long long* tmp = cand + kTpCandMax;                                 // [kTpCandMax]
+  unsigned long long* hmass = tmp + kTpCandMax;                                // [kTpBins]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(hmass + kTpBins);               // [kTpBins]
   uint32_t* bits = hist + kTpBins;                                              // [row words]
   __shared__ unsigned long long s_u[kTpThreads / 32];
   __shared__ unsigned s_w[kTpThreads / 32];
   __shared__ float s_f[kTpThreads / 32];
   __shared__ TpFound s_found;
-  __shared__ int s_take;
   const int row = blockIdx.x, b = row / a.Hkv, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const float* sc = a.scores + size_t(row) * a.nb_stride;
@@ -1010,42 +1011,104 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
     }
   }
   const int n_c = int(min(c_tot, unsigned(kTpCandMax)));
-  int n_pow = kTpThreads;                              // sorted length: 1,024, 2,048 or 4,096
-  while (n_pow < n_c) n_pow <<= 1;
+  const int n_top = min(n_c, int(cap));                // the cap best blocks at most
   __syncthreads();                                     // every candidate written
-  // bitonic sort, largest first; the padding (0) lies below every block's key
-  if (n_c > 1) {
-    for (int i = n_c + tid; i < n_pow; i += kTpThreads) cand[i] = 0ull;
-    __syncthreads();
-    if (n_pow == kTpThreads) tp_sort<1>(cand);
-    else if (n_pow == 2 * kTpThreads) tp_sort<2>(cand);
-    else tp_sort<4>(cand);
-  }
 
-  // 4. masses in that order (the first cap candidates: the cap best blocks); the fewest
-  // whose mass with the forced blocks' reaches the goal
-  const int n_top = min(n_c, int(cap));
-  const int per = (n_pow + kTpThreads - 1) / kTpThreads;     // consecutive entries per thread
-  const int e0 = tid * per;
-  unsigned long long loc = 0;
-  for (int i = e0; i < min(n_top, e0 + per); ++i)
-    loc += tp_mass(tp_clean(sc[0xffffffffu - uint32_t(cand[i])]), M);
-  if (tid == 0) s_take = n_top;
-  unsigned long long tot_c;
-  unsigned long long cum = MF + tp_scan(loc, s_u, tot_c);
-  if (MF >= goal) {
-    if (tid == 0) s_take = 0;
-  } else {
-    for (int i = e0; i < min(n_top, e0 + per); ++i) {
-      cum += tp_mass(tp_clean(sc[0xffffffffu - uint32_t(cand[i])]), M);
-      if (cum >= goal) {
-        atomicMin(&s_take, i + 1);
+  // 4. The taken candidates, in the order decreasing beta, ties to the lower index: the
+  // fewest whose mass with the forced blocks' reaches the goal, at most n_top. Instead of
+  // sorting every candidate, a 2,048-bin histogram linear in the score over the candidates
+  // (count and exact fixed-point mass per bin) finds, walking from the highest bin, the bin
+  // gb where the count reaches n_top or the mass the remaining goal. Bins are monotone in
+  // the score, so every candidate above gb is taken, and only gb's candidates are sorted
+  // (key descending, index ascending) to take the first t_in of them.
+  __shared__ unsigned s_nt;
+  __shared__ int s_tin;
+  int gb = kTpBins, t_in = 0;                          // no candidate taken
+  uint32_t cnt_above = 0u;
+  unsigned long long mass_above = 0ull;
+  float cmin = 0.0f, cinv = 0.0f;
+  if (n_top > 0 && MF < goal) {
+    const unsigned long long need = goal - MF;
+    float mx2 = -INFINITY, mn2 = INFINITY;
+    for (int i = tid; i < n_c; i += kTpThreads) {
+      const float x = tp_unkey(uint32_t(cand[i] >> 32));
+      mx2 = fmaxf(mx2, x);
+      mn2 = fminf(mn2, x);
+    }
+    const float cmax = tp_block_max(mx2, s_f);
+    cmin = -tp_block_max(-mn2, s_f);
+    cinv = cmax > cmin ? float(kTpBins) / (cmax - cmin) : 0.0f;
+    for (int i = tid; i < kTpBins; i += kTpThreads) {
+      hist[i] = 0u;
+      hmass[i] = 0ull;
+    }
+    if (tid == 0) s_nt = 0u;
+    __syncthreads();
+    for (int i = tid; i < n_c; i += kTpThreads) {
+      const float x = tp_unkey(uint32_t(cand[i] >> 32));
+      const int bin = tp_lin_bin(x, cmin, cinv);
+      atomicAdd(&hist[bin], 1u);
+      atomicAdd(&hmass[bin], tp_mass(x, M));
+    }
+    __syncthreads();
+    const TpFound f = tp_find(hist, hmass, kTpBins, uint32_t(n_top), need, s_u, &s_found);
+    gb = f.bin;                                        // >= 0: the counts reach n_top
+    cnt_above = f.cnt_above;
+    mass_above = f.mass_above;
+    if (gb < 0) {                                      // cannot happen; take no candidate
+      if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SELECT, uint32_t(row));
+      gb = kTpBins;
+    }
+  }
+  if (gb < kTpBins) {
+    const unsigned long long need = goal - MF;
+    // gb's candidates, then sorted
+    for (int i = tid; i < n_c; i += kTpThreads) {
+      const float x = tp_unkey(uint32_t(cand[i] >> 32));
+      if (tp_lin_bin(x, cmin, cinv) == gb) tmp[atomicAdd(&s_nt, 1u)] = cand[i];
+    }
+    __syncthreads();
+    const int n_t = int(s_nt);
+    if (n_t <= 32) {
+      if (warp == 0) {                                 // one warp: bitonic by shuffles
+        unsigned long long v = lane < n_t ? tmp[lane] : 0ull;
+#pragma unroll
+        for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+          for (int jj = k >> 1; jj > 0; jj >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(kFull, v, jj);
+            v = tp_keep(v, o, ((lane & jj) == 0) == ((lane & k) == 0));
+          }
+        tmp[lane] = v;
+      }
+      __syncthreads();
+    } else {
+      int n_pow = kTpThreads;                          // 1,024, 2,048 or 4,096 entries
+      while (n_pow < n_t) n_pow <<= 1;
+      for (int i = n_t + tid; i < n_pow; i += kTpThreads) tmp[i] = 0ull;   // below every key
+      __syncthreads();
+      if (n_pow == kTpThreads) tp_sort<1>(tmp);
+      else if (n_pow == 2 * kTpThreads) tp_sort<2>(tmp);
+      else tp_sort<4>(tmp);
+    }
+    // the first t_in of them: where the count reaches n_top or the mass the goal
+    const int per = (n_t + kTpThreads - 1) / kTpThreads;     // consecutive entries per thread
+    const int e0 = tid * per, e1 = min(n_t, e0 + per);
+    unsigned long long loc = 0;
+    for (int i = e0; i < e1; ++i) loc += tp_mass(tp_unkey(uint32_t(tmp[i] >> 32)), M);
+    if (tid == 0) s_tin = n_t;
+    unsigned long long tot_t;
+    unsigned long long cum = mass_above + tp_scan(loc, s_u, tot_t);
+    for (int i = e0; i < e1; ++i) {
+      cum += tp_mass(tp_unkey(uint32_t(tmp[i] >> 32)), M);
+      if (cnt_above + uint32_t(i) + 1u >= uint32_t(n_top) || cum >= need) {
+        atomicMin(&s_tin, i + 1);
         break;
       }
     }
+    __syncthreads();
+    t_in = s_tin;
   }
-  __syncthreads();
-  const int n_take = s_take;
 
   // 5. bitmap of the taken blocks, written out ascending
   const int words = (nb + 31) / 32;
@@ -1055,8 +1118,14 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
     if (f0 >= 0) atomicOr(&bits[f0 >> 5], 1u << (f0 & 31));
     if (f1 >= 0) atomicOr(&bits[f1 >> 5], 1u << (f1 & 31));
   }
-  for (int i = tid; i < n_take; i += kTpThreads) {
-    const uint32_t j = 0xffffffffu - uint32_t(cand[i]);
+  for (int i = tid; i < n_c && gb < kTpBins; i += kTpThreads) {   // the bins above gb
+    if (tp_lin_bin(tp_unkey(uint32_t(cand[i] >> 32)), cmin, cinv) > gb) {
+      const uint32_t j = 0xffffffffu - uint32_t(cand[i]);
+      atomicOr(&bits[j >> 5], 1u << (j & 31));
+    }
+  }
+  for (int i = tid; i < t_in; i += kTpThreads) {                  // the first t_in of gb
+    const uint32_t j = 0xffffffffu - uint32_t(tmp[i]);
     atomicOr(&bits[j >> 5], 1u << (j & 31));
   }
   __syncthreads();
@@ -1084,7 +1153,7 @@ __global__ void __launch_bounds__(kTpThreads, 1) top_p_sorted_kernel(const TopPP
 cudaError_t launch_top_p(const TopPParams& a, cudaStream_t s) {
   if (a.budget <= kTpCandMax) {
     // candidates, histogram and the row's bitmap in dynamic shared memory
-    const size_t smem = size_t(kTpCandMax) * 8 + size_t(kTpBins) * 4 +
+    const size_t smem = size_t(kTpCandMax) * 8 * 2 + size_t(kTpBins) * (8 + 4) +
                         size_t((a.nb_stride + 31) / 32) * 4;
     if (smem <= size_t(200) * 1024) {
       const cudaError_t e = set_smem_limit(top_p_sorted_kernel, int(200 * 1024));
