@@ -7,14 +7,16 @@
 //                    Delta + u_i)) (all 0 when Delta = 0), stored as 4 bit planes, with
 //                    Delta, v_l, sum n_i and c . qbar. Every step is a rounded float32
 //                    operation, so the codes are those of the float32 definition.
-//   rq_score_kernel: one warp per (page, KV head): lane l scores token slots l + 32k,
-//                    k < 4. With A = sum_p 2^p popc(b & plane_p) and B = popc(b),
+//   rq_score_kernel: a warp scores one (row, page) unit at a time: lane l the token slots
+//                    l + 32k, k < 4. With A = sum_p 2^p popc(b & plane_p) and B = popc(b),
 //                      s = g (Delta (2A - Q) + v_l (2B - d)) + c . qbar
 //                    = g sum_i (2 b_i - 1)(Delta n_i + v_l) + c . qbar (the RaBitQ estimate
 //                    of q . k, Gao and Long, SIGMOD 2024, section 3), then each block's
 //                    log-sum-exp of scale * s over its valid tokens (the log of its
-//                    estimated attention mass up to the row's normaliser).
-//   top_p_kernel:    CTA = one row; see its comment.
+//                    estimated attention mass up to the row's normaliser); the row's
+//                    largest block score is recorded in its query-code record.
+//   top_p_sorted_kernel, top_p_kernel: CTA = one row (budgets up to 4,096 blocks, and
+//                    larger ones); see their comments.
 #include <cfloat>
 
 #include "qs_device.cuh"

@@ -15,7 +15,8 @@
 //   sem_update_kernel: thread = (cluster, dimension): the members' sum in token order, then
 //                      one division by the count (an empty cluster keeps its centroid).
 // Decode:
-//   sem_score_kernel:  warp = (row, cluster): beta_j = qbar . c_j (float32).
+//   sem_score_kernel:  CTA = (row, 32 clusters), qbar formed once in shared memory, a warp
+//                      per 4 clusters: beta_j = qbar . c_j (float32).
 //   (the existing select kernel picks the top clusters over C_b candidates)
 //   sem_expand_kernel: CTA = row: the selected clusters' members, then the tokens after the
 //                      prompt, as the row's token list for the token-level attention.
