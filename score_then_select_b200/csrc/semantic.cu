@@ -278,10 +278,14 @@ __global__ void __launch_bounds__(kSemScoreWarps * 32) sem_score_kernel(const Se
   }
 }
 
-// CTA = row: the members of the selected clusters (each cluster's in token order, the
+// CTA (row, 0): the members of the selected clusters (each cluster's in token order, the
 // clusters in the order selected), then the tokens after the prompt, L0 <= t < seq_len.
 // A scan over the selected clusters' sizes gives each cluster's place in the list; warp w
 // then copies clusters w, w + 32, ..., its lanes striding over the cluster's members.
+// CTAs (row, 1 .. kSemPadParts): the rest of the row's list, up to max_tokens, padded with
+// -1 in kSemPadParts slices by 16-byte stores; each finds the list's length n itself from
+// the selected clusters' sizes.
+constexpr int kSemPadParts = 7;
 __global__ void __launch_bounds__(kSemThreads) sem_expand_kernel(const SemSelectParams a) {
   __shared__ int s_scan[kSemThreads / 32];
   __shared__ int s_lo[kSemThreads], s_sz[kSemThreads], s_dst[kSemThreads];
@@ -297,8 +301,34 @@ __global__ void __launch_bounds__(kSemThreads) sem_expand_kernel(const SemSelect
   int32_t* out = a.tokens + size_t(row) * a.max_tokens;
   int ncs = a.n_csel[row];
   if (ncs < 0 || ncs > a.budget) {
-    if (tid == 0) flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SEMANTIC, uint32_t(row));
+    if (tid == 0 && blockIdx.y == 0)
+      flag_error(a.hdr, QS_ERR_DEVICE_BOUNDS, KID_SEMANTIC, uint32_t(row));
     ncs = 0;
+  }
+  if (blockIdx.y > 0) {
+    // the list's length, as CTA (row, 0) forms it
+    int sz = 0;
+    for (int i = tid; i < ncs; i += kSemThreads) {
+      const int c = cs[i];
+      if (c >= 0 && c < C) sz += off[c + 1] - off[c];
+    }
+    int total;
+    sem_scan(sz, s_scan, total);
+    const int n = min(a.max_tokens, total + (L - L0));
+    // 4-byte stores up to a 16-byte boundary and after the last whole vector (slice 0),
+    // 16-byte stores in between, split into kSemPadParts slices
+    int i0 = n;
+    while (i0 < a.max_tokens && (reinterpret_cast<uintptr_t>(out + i0) & 15u) != 0u) ++i0;
+    const int nv = (a.max_tokens - i0) / 4;
+    const int p = int(blockIdx.y) - 1, P = int(gridDim.y) - 1;
+    const int v0 = int((long long)nv * p / P), v1 = int((long long)nv * (p + 1) / P);
+    int4* out4 = reinterpret_cast<int4*>(out + i0);
+    for (int i = v0 + tid; i < v1; i += kSemThreads) out4[i] = make_int4(-1, -1, -1, -1);
+    if (p == 0) {
+      if (tid < i0 - n) out[n + tid] = -1;
+      for (int i = i0 + 4 * nv + tid; i < a.max_tokens; i += kSemThreads) out[i] = -1;
+    }
+    return;
   }
   int running = 0;
   bool over = false;
@@ -334,14 +364,6 @@ __global__ void __launch_bounds__(kSemThreads) sem_expand_kernel(const SemSelect
   int n = running + (L - L0);
   if (n > a.max_tokens) n = a.max_tokens;
   if (tid == 0) a.n_tokens[row] = n;
-  // the padding: 4-byte stores up to a 16-byte boundary, then 16-byte stores, then the tail
-  int i0 = n;
-  while (i0 < a.max_tokens && (reinterpret_cast<uintptr_t>(out + i0) & 15u) != 0u) ++i0;
-  if (tid < i0 - n) out[n + tid] = -1;
-  const int nv = (a.max_tokens - i0) / 4;
-  int4* out4 = reinterpret_cast<int4*>(out + i0);
-  for (int i = tid; i < nv; i += kSemThreads) out4[i] = make_int4(-1, -1, -1, -1);
-  for (int i = i0 + 4 * nv + tid; i < a.max_tokens; i += kSemThreads) out[i] = -1;
 }
 
 cudaError_t launch_sem_score(const SemSelectParams& a, cudaStream_t s) {
@@ -353,7 +375,7 @@ cudaError_t launch_sem_score(const SemSelectParams& a, cudaStream_t s) {
 }
 
 cudaError_t launch_sem_expand(const SemSelectParams& a, cudaStream_t s) {
-  sem_expand_kernel<<<a.batch * a.Hkv, kSemThreads, 0, s>>>(a);
+  sem_expand_kernel<<<dim3(a.batch * a.Hkv, 1 + kSemPadParts), kSemThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
